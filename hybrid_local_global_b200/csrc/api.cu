@@ -1,0 +1,485 @@
+// api.cu -- the extern "C" entry points of libgemma_attn.so: argument
+// validation, workspace planning, launches, the device status word and the
+// host-only KV-share binding. Declarations and contracts: gemma_attn.h.
+#include <algorithm>
+#include <atomic>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "common.cuh"
+#include "kernels.h"
+
+using namespace hlg;
+
+namespace {
+
+thread_local std::string t_err;
+
+int fail(int code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  t_err = buf;
+  return code;
+}
+
+int succeed() {
+  t_err.clear();
+  return GEMMA_OK;
+}
+
+__device__ int g_status;  // first device-side failure since the last sync_status
+
+std::mutex g_mu;
+int* g_status_ptr[128] = {nullptr};
+int g_sm_count[128] = {0};
+std::atomic<long long> g_wait_ns{1000000000LL};
+std::atomic<int> g_drop_next{0};
+
+int current_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+  return dev;
+}
+
+// Device address of g_status for the current device (looked up once).
+int* status_ptr() {
+  int dev = current_device();
+  if (dev < 0 || dev >= 128) return nullptr;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_status_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_status) != cudaSuccess) return nullptr;
+    g_status_ptr[dev] = static_cast<int*>(p);
+  }
+  return g_status_ptr[dev];
+}
+
+int sm_count() {
+  int dev = current_device();
+  if (dev < 0 || dev >= 128) return 148;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_sm_count[dev]) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      n = 148;
+    g_sm_count[dev] = n;
+  }
+  return g_sm_count[dev];
+}
+
+// Measurement hook state (gemma_attn_profile): event pairs around launches.
+struct ProfRec {
+  int kind;
+  cudaEvent_t a, b;
+};
+std::mutex g_prof_mu;
+std::vector<ProfRec> g_prof;
+std::atomic<bool> g_prof_on{false};
+
+struct ProfScope {
+  ProfRec rec{-1, nullptr, nullptr};
+  cudaStream_t st;
+  ProfScope(int kind, cudaStream_t s) : st(s) {
+    if (!g_prof_on.load()) return;
+    if (cudaEventCreate(&rec.a) != cudaSuccess || cudaEventCreate(&rec.b) != cudaSuccess) return;
+    rec.kind = kind;
+    cudaEventRecord(rec.a, st);
+  }
+  void done() {
+    if (rec.kind < 0) return;
+    cudaEventRecord(rec.b, st);
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    g_prof.push_back(rec);
+    rec.kind = -1;
+  }
+};
+
+void prof_clear() {
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  for (auto& r : g_prof) {
+    cudaEventDestroy(r.a);
+    cudaEventDestroy(r.b);
+  }
+  g_prof.clear();
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+int check_heads(int Hq, int Hkv, int D, int window, float rope_frac, float rope_theta, float scale) {
+  if (Hq <= 0 || Hkv <= 0 || Hq % Hkv)
+    return fail(GEMMA_ERR_INVALID_ARG, "n_q_heads (%d) must be a positive multiple of n_kv_heads (%d)", Hq, Hkv);
+  if (Hq / Hkv > 8)
+    return fail(GEMMA_ERR_UNSUPPORTED, "query heads per KV head %d > 8", Hq / Hkv);
+  if (D != 256 && D != 512) return fail(GEMMA_ERR_UNSUPPORTED, "head_dim %d (supported: 256, 512)", D);
+  if (window < 0 || window % 16)
+    return fail(GEMMA_ERR_INVALID_ARG, "window %d must be 0 or a positive multiple of 16", window);
+  if (!(rope_frac >= 0.f && rope_frac <= 1.f))
+    return fail(GEMMA_ERR_INVALID_ARG, "rope_frac %g outside [0, 1]", (double)rope_frac);
+  if (!(rope_theta > 0.f) || !std::isfinite(rope_theta))
+    return fail(GEMMA_ERR_INVALID_ARG, "rope_theta %g must be positive and finite", (double)rope_theta);
+  if (!std::isfinite(scale)) return fail(GEMMA_ERR_INVALID_ARG, "scale must be finite");
+  return GEMMA_OK;
+}
+
+int cuda_fail(cudaError_t e, const char* what) {
+  return fail(GEMMA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+// Split-K plan of a decode call: keys per split (multiple of 16) and splits
+// per (sequence, KV head). About 2048 keys per unit, the unit count rounded
+// up to whole waves of two CTAs per SM, so equal-length batches fill every
+// wave.
+void decode_plan(int B, int Hkv, int window, int max_len, int* chunk, int* n_splits) {
+  const int64_t keys_max = window > 0 ? std::min<int64_t>(max_len, window) : max_len;
+  const int64_t pairs = (int64_t)B * Hkv;
+  const int64_t wave = (int64_t)sm_count() * 2;
+  int64_t units = (keys_max * pairs + 2047) / 2048;
+  units = ((units + wave - 1) / wave) * wave;
+  int64_t c = (keys_max * pairs + units - 1) / units;
+  c = ((c + 15) / 16) * 16;
+  c = std::max<int64_t>(c, 256);
+  c = std::min<int64_t>(c, ((keys_max + 15) / 16) * 16);
+  *chunk = (int)c;
+  *n_splits = (int)((keys_max + c - 1) / c);
+}
+
+size_t decode_ws_parts(int B, int Hq, int D, int n_splits, size_t* off_lse, size_t* off_o) {
+  size_t q = align256((size_t)B * Hq * D * 2);
+  size_t lse = align256((size_t)B * Hq * n_splits * 4);
+  size_t o = align256((size_t)B * Hq * n_splits * D * 4);
+  *off_lse = q;
+  *off_o = q + lse;
+  return q + lse + o;
+}
+
+size_t prefill_ws_parts(int B, int S, int Hq, int Hkv, int D, int window, size_t* off_k) {
+  size_t q = align256((size_t)B * S * Hq * D * 2);
+  size_t k = window > 0 ? align256((size_t)B * S * Hkv * D * 2) : 0;
+  *off_k = q;
+  return q + k;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* gemma_last_error(void) { return t_err.c_str(); }
+
+int gemma_attn_set_wait_limit(long long max_ns) {
+  if (max_ns < 0) return fail(GEMMA_ERR_INVALID_ARG, "wait limit must be >= 0");
+  g_wait_ns.store(max_ns == 0 ? 1000000000LL : max_ns);
+  return succeed();
+}
+
+int gemma_attn_debug_drop_next_copy(int enable) {
+  g_drop_next.store(enable ? 1 : 0);
+  return succeed();
+}
+
+int gemma_layer_schedule(int n_layers, int ratio, int n_shared, int* is_global, int* share_src) {
+  if (n_layers <= 0 || ratio < 0 || n_shared < 0 || n_shared > n_layers || !is_global)
+    return fail(GEMMA_ERR_INVALID_ARG, "bad schedule arguments (n_layers %d, ratio %d, n_shared %d)",
+                n_layers, ratio, n_shared);
+  for (int l = 0; l < n_layers; ++l)
+    is_global[l] = (l == n_layers - 1) || ((l + 1) % (ratio + 1) == 0);
+  if (share_src) {
+    const int first = n_layers - n_shared;
+    for (int l = 0; l < n_layers; ++l) {
+      if (l < first) {
+        share_src[l] = l;
+        continue;
+      }
+      int src = -1;
+      for (int s = first - 1; s >= 0; --s)
+        if (is_global[s] == is_global[l]) {
+          src = s;
+          break;
+        }
+      share_src[l] = src;
+    }
+  }
+  return succeed();
+}
+
+int gemma_kv_share_bind(gemma_kv_desc* dst, const gemma_kv_desc* src) {
+  if (!dst || !src) return fail(GEMMA_ERR_INVALID_ARG, "null descriptor");
+  if (!src->k_cache || !src->v_cache) return fail(GEMMA_ERR_INVALID_ARG, "source layer has no cache");
+  if (src->layer >= dst->layer)
+    return fail(GEMMA_ERR_SHARE_MISMATCH, "source layer %d must precede layer %d", src->layer, dst->layer);
+  if ((src->window == 0) != (dst->window == 0))
+    return fail(GEMMA_ERR_SHARE_MISMATCH, "layers %d and %d have different attention types", src->layer,
+                dst->layer);
+  if (src->window != dst->window || src->cache_cap != dst->cache_cap ||
+      src->n_kv_heads != dst->n_kv_heads || src->head_dim != dst->head_dim ||
+      src->rope_frac != dst->rope_frac || src->rope_theta != dst->rope_theta)
+    return fail(GEMMA_ERR_SHARE_MISMATCH,
+                "layers %d and %d differ in window, capacity, KV heads, head_dim or RoPE", src->layer,
+                dst->layer);
+  dst->k_cache = src->k_cache;
+  dst->v_cache = src->v_cache;
+  dst->shared_from = src->shared_from >= 0 ? src->shared_from : src->layer;
+  return succeed();
+}
+
+size_t gemma_attn_prefill_workspace_size(int batch, int s_new, int n_q_heads, int n_kv_heads,
+                                         int head_dim, int window) {
+  if (batch <= 0 || s_new <= 0 || n_q_heads <= 0 || n_kv_heads <= 0 || head_dim <= 0) return 0;
+  size_t off_k;
+  return prefill_ws_parts(batch, s_new, n_q_heads, n_kv_heads, head_dim, window, &off_k);
+}
+
+int gemma_attn_prefill(const void* q, const void* k_new, const void* v_new, void* k_cache, void* v_cache,
+                       int cache_cap, const int32_t* seq_lens_before, int batch, int s_new, int window,
+                       int n_q_heads, int n_kv_heads, int head_dim, float rope_frac, float rope_theta,
+                       float scale, void* out, float* lse, void* workspace, size_t workspace_bytes,
+                       unsigned flags, void* stream) {
+  int rc = check_heads(n_q_heads, n_kv_heads, head_dim, window, rope_frac, rope_theta, scale);
+  if (rc) return rc;
+  if (flags & ~GEMMA_F_SHARED) return fail(GEMMA_ERR_INVALID_ARG, "unknown flags 0x%x", flags);
+  if (batch <= 0 || s_new < 0) return fail(GEMMA_ERR_INVALID_ARG, "batch %d, s_new %d", batch, s_new);
+  const bool shared = flags & GEMMA_F_SHARED;
+  if (shared && (k_new || v_new))
+    return fail(GEMMA_ERR_INVALID_ARG, "GEMMA_F_SHARED: k_new and v_new must be NULL");
+  if (!shared && (!k_new || !v_new))
+    return fail(GEMMA_ERR_INVALID_ARG, "k_new and v_new are required unless GEMMA_F_SHARED");
+  if (!q || !out || !k_cache || !v_cache) return fail(GEMMA_ERR_INVALID_ARG, "null tensor pointer");
+  if (!aligned16(q) || !aligned16(out) || !aligned16(k_cache) || !aligned16(v_cache) ||
+      (k_new && !aligned16(k_new)) || (v_new && !aligned16(v_new)) || !aligned16(workspace))
+    return fail(GEMMA_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
+  if (window > 0) {
+    if (cache_cap != window)
+      return fail(GEMMA_ERR_INVALID_ARG, "local layer: cache_cap %d must equal window %d", cache_cap, window);
+    if (seq_lens_before)
+      return fail(GEMMA_ERR_UNSUPPORTED, "chunked prefill on a local layer is not implemented");
+    if (shared && s_new > window)
+      return fail(GEMMA_ERR_UNSUPPORTED, "shared local layer: prefill longer than the window");
+  } else if (cache_cap < s_new) {
+    return fail(GEMMA_ERR_CAPACITY, "global layer: cache_cap %d < s_new %d", cache_cap, s_new);
+  }
+  if (s_new == 0) return succeed();
+  size_t off_k;
+  size_t need = prefill_ws_parts(batch, s_new, n_q_heads, n_kv_heads, head_dim, window, &off_k);
+  if (!workspace || workspace_bytes < need)
+    return fail(GEMMA_ERR_CAPACITY, "workspace %zu bytes < %zu", workspace_bytes, need);
+  int* status = status_ptr();
+  if (!status) return fail(GEMMA_ERR_CUDA, "no CUDA device");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  unsigned char* ws = static_cast<unsigned char*>(workspace);
+
+  PrefillRopeArgs ra;
+  ra.q = static_cast<const bf16*>(q);
+  ra.k_new = static_cast<const bf16*>(k_new);
+  ra.v_new = static_cast<const bf16*>(v_new);
+  ra.q_rot = reinterpret_cast<bf16*>(ws);
+  ra.k_rot = (window > 0 && !shared) ? reinterpret_cast<bf16*>(ws + off_k) : nullptr;
+  ra.k_cache = static_cast<bf16*>(k_cache);
+  ra.v_cache = static_cast<bf16*>(v_cache);
+  ra.cache_cap = cache_cap;
+  ra.seq_lens_before = seq_lens_before;
+  ra.S = s_new;
+  ra.window = window;
+  ra.Hq = n_q_heads;
+  ra.Hkv = n_kv_heads;
+  ra.n_rot = rope_rotated_pairs(head_dim, rope_frac);
+  ra.log2_theta = std::log2((double)rope_theta);
+  ra.rows_per_cta = 4;
+  ra.status = status;
+  ProfScope p_rope(GEMMA_KERNEL_PREFILL_ROPE, st);
+  cudaError_t e = launch_prefill_rope(ra, batch, head_dim, st);
+  p_rope.done();
+  if (e != cudaSuccess) return cuda_fail(e, "prefill rope launch");
+
+  PrefillAttnArgs aa;
+  aa.q_rot = ra.q_rot;
+  const int64_t D = head_dim;
+  if (window == 0 || shared) {
+    KVView kc = {static_cast<const bf16*>(k_cache), (int64_t)n_kv_heads * cache_cap * D, D, (int64_t)cache_cap * D};
+    KVView vc = {static_cast<const bf16*>(v_cache), kc.stride_b, kc.stride_row, kc.stride_h};
+    aa.k = kc;
+    aa.v = vc;
+    aa.key_cap = cache_cap;
+  } else {
+    KVView kw = {ra.k_rot, (int64_t)s_new * n_kv_heads * D, (int64_t)n_kv_heads * D, D};
+    KVView vw = {static_cast<const bf16*>(v_new), kw.stride_b, kw.stride_row, kw.stride_h};
+    aa.k = kw;
+    aa.v = vw;
+    aa.key_cap = s_new;
+  }
+  aa.seq_lens_before = seq_lens_before;
+  aa.S = s_new;
+  aa.window = window;
+  aa.Hq = n_q_heads;
+  aa.Hkv = n_kv_heads;
+  aa.scale_log2 = (float)((double)scale * 1.4426950408889634);
+  aa.out = static_cast<bf16*>(out);
+  aa.lse = lse;
+  aa.status = status;
+  ProfScope p_attn(GEMMA_KERNEL_PREFILL_ATTN, st);
+  e = launch_prefill_attn(aa, batch, head_dim, st);
+  p_attn.done();
+  if (e != cudaSuccess) return cuda_fail(e, "prefill attention launch");
+  return succeed();
+}
+
+size_t gemma_attn_decode_workspace_size(int batch, int n_q_heads, int n_kv_heads, int head_dim, int window,
+                                        int max_seq_len) {
+  if (batch <= 0 || n_q_heads <= 0 || n_kv_heads <= 0 || head_dim <= 0 || max_seq_len <= 0) return 0;
+  int chunk, n_splits;
+  decode_plan(batch, n_kv_heads, window, max_seq_len, &chunk, &n_splits);
+  size_t a, b;
+  return decode_ws_parts(batch, n_q_heads, head_dim, n_splits, &a, &b);
+}
+
+int gemma_attn_decode(const void* q, const void* k_new, const void* v_new, void* k_cache, void* v_cache,
+                      int cache_cap, const int32_t* seq_lens, int max_seq_len, int batch, int window,
+                      int n_q_heads, int n_kv_heads, int head_dim, float rope_frac, float rope_theta,
+                      float scale, void* out, void* workspace, size_t workspace_bytes, unsigned flags,
+                      void* stream) {
+  int rc = check_heads(n_q_heads, n_kv_heads, head_dim, window, rope_frac, rope_theta, scale);
+  if (rc) return rc;
+  if (flags & ~GEMMA_F_SHARED) return fail(GEMMA_ERR_INVALID_ARG, "unknown flags 0x%x", flags);
+  if (batch <= 0 || max_seq_len <= 0)
+    return fail(GEMMA_ERR_INVALID_ARG, "batch %d, max_seq_len %d", batch, max_seq_len);
+  const bool shared = flags & GEMMA_F_SHARED;
+  if (shared && (k_new || v_new))
+    return fail(GEMMA_ERR_INVALID_ARG, "GEMMA_F_SHARED: k_new and v_new must be NULL");
+  if (!shared && (!k_new || !v_new))
+    return fail(GEMMA_ERR_INVALID_ARG, "k_new and v_new are required unless GEMMA_F_SHARED");
+  if (!q || !out || !k_cache || !v_cache || !seq_lens)
+    return fail(GEMMA_ERR_INVALID_ARG, "null pointer argument");
+  if (!aligned16(q) || !aligned16(out) || !aligned16(k_cache) || !aligned16(v_cache) ||
+      (k_new && !aligned16(k_new)) || (v_new && !aligned16(v_new)) || !aligned16(workspace))
+    return fail(GEMMA_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
+  if (window > 0 && cache_cap != window)
+    return fail(GEMMA_ERR_INVALID_ARG, "local layer: cache_cap %d must equal window %d", cache_cap, window);
+  if (window == 0 && cache_cap < max_seq_len)
+    return fail(GEMMA_ERR_CAPACITY, "global layer: cache_cap %d < max_seq_len %d", cache_cap, max_seq_len);
+  int chunk, n_splits;
+  decode_plan(batch, n_kv_heads, window, max_seq_len, &chunk, &n_splits);
+  size_t off_lse, off_o;
+  size_t need = decode_ws_parts(batch, n_q_heads, head_dim, n_splits, &off_lse, &off_o);
+  if (!workspace || workspace_bytes < need)
+    return fail(GEMMA_ERR_CAPACITY, "workspace %zu bytes < %zu", workspace_bytes, need);
+  int* status = status_ptr();
+  if (!status) return fail(GEMMA_ERR_CUDA, "no CUDA device");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  unsigned char* ws = static_cast<unsigned char*>(workspace);
+
+  DecodeRopeArgs ra;
+  ra.q = static_cast<const bf16*>(q);
+  ra.k_new = static_cast<const bf16*>(k_new);
+  ra.v_new = static_cast<const bf16*>(v_new);
+  ra.q_rot = reinterpret_cast<bf16*>(ws);
+  ra.k_cache = static_cast<bf16*>(k_cache);
+  ra.v_cache = static_cast<bf16*>(v_cache);
+  ra.cache_cap = cache_cap;
+  ra.seq_lens = seq_lens;
+  ra.max_len = max_seq_len;
+  ra.window = window;
+  ra.Hq = n_q_heads;
+  ra.Hkv = n_kv_heads;
+  ra.n_rot = rope_rotated_pairs(head_dim, rope_frac);
+  ra.log2_theta = std::log2((double)rope_theta);
+  ra.status = status;
+  // rotates q; also appends the new K/V unless the layer is shared
+  ProfScope p_app(GEMMA_KERNEL_DECODE_APPEND, st);
+  cudaError_t e = launch_decode_rope_append(ra, batch, head_dim, st);
+  p_app.done();
+  if (e != cudaSuccess) return cuda_fail(e, "decode append launch");
+
+  DecodeAttnArgs da;
+  da.q_rot = ra.q_rot;
+  da.k_cache = static_cast<const bf16*>(k_cache);
+  da.v_cache = static_cast<const bf16*>(v_cache);
+  da.cache_cap = cache_cap;
+  da.seq_lens = seq_lens;
+  da.max_len = max_seq_len;
+  da.window = window;
+  da.Hq = n_q_heads;
+  da.Hkv = n_kv_heads;
+  da.chunk = chunk;
+  da.n_splits = n_splits;
+  da.scale_log2 = (float)((double)scale * 1.4426950408889634);
+  da.part_lse = reinterpret_cast<float*>(ws + off_lse);
+  da.part_o = reinterpret_cast<float*>(ws + off_o);
+  da.out = static_cast<bf16*>(out);
+  da.status = status;
+  da.wait_ns = (unsigned long long)g_wait_ns.load();
+  da.drop_first_copy = g_drop_next.exchange(0);
+  {
+    ProfScope p_split(GEMMA_KERNEL_DECODE_SPLIT, st);
+    e = launch_decode_split(da, batch, head_dim, st);
+    p_split.done();
+  }
+  if (e != cudaSuccess) return cuda_fail(e, "decode attention launch");
+  {
+    ProfScope p_comb(GEMMA_KERNEL_DECODE_COMBINE, st);
+    e = launch_decode_combine(da, batch, head_dim, st);
+    p_comb.done();
+  }
+  if (e != cudaSuccess) return cuda_fail(e, "decode combine launch");
+  return succeed();
+}
+
+int gemma_attn_visible_ranges(const int32_t* seq_lens_before, int batch, int s_new, int window,
+                              int32_t* ranges, void* stream) {
+  if (batch <= 0 || s_new < 0 || window < 0 || !ranges)
+    return fail(GEMMA_ERR_INVALID_ARG, "bad arguments");
+  cudaError_t e = launch_visible_ranges(seq_lens_before, batch, s_new, window, ranges,
+                                        static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "visible ranges launch");
+  return succeed();
+}
+
+int gemma_attn_profile(int enable) {
+  prof_clear();
+  g_prof_on.store(enable != 0);
+  return succeed();
+}
+
+int gemma_attn_profile_read(int kernel, double* total_ms, long long* launches) {
+  if (kernel < 0 || kernel >= GEMMA_KERNEL_KINDS || !total_ms || !launches)
+    return fail(GEMMA_ERR_INVALID_ARG, "bad profile query");
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  double tot = 0.0;
+  long long n = 0;
+  for (auto& r : g_prof) {
+    if (r.kind != kernel) continue;
+    cudaError_t e = cudaEventSynchronize(r.b);
+    if (e != cudaSuccess) return cuda_fail(e, "profile event synchronize");
+    float ms = 0.f;
+    e = cudaEventElapsedTime(&ms, r.a, r.b);
+    if (e != cudaSuccess) return cuda_fail(e, "profile elapsed time");
+    tot += ms;
+    ++n;
+  }
+  *total_ms = tot;
+  *launches = n;
+  return succeed();
+}
+
+int gemma_attn_sync_status(void* stream) {
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "stream synchronize");
+  int v = 0;
+  e = cudaMemcpyFromSymbol(&v, g_status, sizeof v);
+  if (e != cudaSuccess) return cuda_fail(e, "read device status");
+  if (v != 0) {
+    const int zero = 0;
+    e = cudaMemcpyToSymbol(g_status, &zero, sizeof zero);
+    if (e != cudaSuccess) return cuda_fail(e, "clear device status");
+    return fail(v, v == GEMMA_ERR_DEVICE_TIMEOUT ? "a bounded device wait gave up"
+                                                 : "a device-side range check failed");
+  }
+  return succeed();
+}
+
+}  // extern "C"

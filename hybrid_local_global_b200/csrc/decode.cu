@@ -1,0 +1,367 @@
+// decode.cu -- batched single-token decode over the KV cache (split-K
+// flash-decode) and the log-sum-exp combine of the splits.
+//
+// For the new token of sequence b (position len-1) and q head h (KV head
+// g = h / G): out = sum_j softmax_j(scale <q~, k~_j>) v_j over the visible
+// cached keys: every position on a global layer, the ring's last
+// min(len, window) positions on a local layer ("Gemma 4: End-to-End
+// Architecture Walkthrough", 3a/3b; "Gemma 4 Deep Dive" talk: the window
+// bounds what a local layer has to keep). Softmax order does not matter, so
+// ring slots are read in slot order.
+//
+// The step is HBM-bound: every cached K/V byte is read once per KV head and
+// shared by its G query heads. Work unit = (split of `chunk` keys, KV head,
+// sequence). Per CTA:
+//   warp 4      producer: for each 16-key sub-block, one lane arms the slot's
+//               full barrier with the byte count and 32 lanes issue one bulk
+//               copy per K/V row into a ring of padded shared-memory rows
+//               (row stride D*2+16 bytes keeps ldmatrix conflict-free).
+//   warps 0..3  consumers: sub-block t goes to warp t % 4. S = Q K^T with
+//               mma.sync m16n8k16 (A = the G query heads padded to 16 rows,
+//               B = K rows), online softmax in fp32 (log2 domain), then
+//               O^T += V^T P^T with the S accumulators reused directly as the
+//               B fragment of P^T (the GQA group is the MMA's N dimension).
+// The four warps' (m, l, O) merge in shared memory; each split writes its
+// normalised partial and its log2-sum-exp, and the combine kernel merges the
+// splits of a (sequence, head).
+//
+// Every barrier wait is bounded (%globaltimer deadline). On a timeout the
+// CTA raises its abort flag, records GEMMA_ERR_DEVICE_TIMEOUT, waits (again
+// bounded) for its own copies still in flight, and exits without output.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace hlg {
+
+namespace {
+
+template <int D>
+struct DecCfg {
+  static constexpr int KB = 16;                 // keys per sub-block
+  static constexpr int ROW = D + 8;             // padded smem row (elements)
+  static constexpr int ROWB = ROW * 2;          // bytes
+  static constexpr int SLOT_B = 2 * KB * ROWB;  // K rows then V rows
+  static constexpr int NSLOT = (D == 256) ? 6 : 3;
+  static constexpr int RING_B = NSLOT * SLOT_B;
+  static constexpr int Q_B = 8 * ROWB;
+  static constexpr int OSTR = D + 4;            // merge-buffer row (floats)
+  static constexpr int MERGE_B = 4 * 8 * OSTR * 4;
+  static_assert(MERGE_B <= RING_B, "merge buffer must fit in the ring");
+  static constexpr int BAR_OFF = RING_B + Q_B;
+  static constexpr int MISC_OFF = BAR_OFF + 2 * NSLOT * 8;
+  static constexpr int SMEM = MISC_OFF + (1 + 2 * NSLOT + 64) * 4;
+};
+
+__device__ __forceinline__ void ldsm_x2(uint32_t addr, uint32_t& r0, uint32_t& r1) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0,%1}, [%2];"
+               : "=r"(r0), "=r"(r1)
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
+                                        uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
+                                          uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+__device__ __forceinline__ void mma_bf16(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                         uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ void named_bar_sync(int id, int n) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+
+template <int D>
+__global__ void __launch_bounds__(160, 2) k_decode_split(DecodeAttnArgs a) {
+  using C = DecCfg<D>;
+  extern __shared__ __align__(128) unsigned char sm[];
+  unsigned char* ring = sm;
+  bf16* qs = reinterpret_cast<bf16*>(sm + C::RING_B);
+  uint64_t* full = reinterpret_cast<uint64_t*>(sm + C::BAR_OFF);
+  uint64_t* empty = full + C::NSLOT;
+  int* misc = reinterpret_cast<int*>(sm + C::MISC_OFF);
+  volatile int* abort_flag = misc;
+  int* issued = misc + 1;
+  int* consumed = issued + C::NSLOT;
+  float* m_w = reinterpret_cast<float*>(consumed + C::NSLOT);  // [4][8]
+  float* l_w = m_w + 32;                                         // [4][8]
+
+  const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int G = a.Hq / a.Hkv;
+  const int64_t len = a.seq_lens[b];
+  if (len < 1 || len > a.max_len) {
+    if (threadIdx.x == 0 && split == 0 && g == 0) set_status(a.status, GEMMA_ERR_DEVICE_RANGE);
+    return;
+  }
+  const int64_t n_valid = a.window > 0 ? (len < a.window ? len : (int64_t)a.window) : len;
+  const int64_t k_begin = (int64_t)split * a.chunk;
+  if (k_begin >= n_valid) return;
+  const int64_t k_end = (k_begin + a.chunk < n_valid) ? k_begin + a.chunk : n_valid;
+  const int n_sub = (int)((k_end - k_begin + C::KB - 1) / C::KB);
+  const int64_t head_off = ((int64_t)b * a.Hkv + g) * (int64_t)a.cache_cap * D;
+  const bf16* kbase = a.k_cache + head_off;
+  const bf16* vbase = a.v_cache + head_off;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::NSLOT; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+      issued[s] = 0;
+      consumed[s] = 0;
+    }
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  for (int idx = threadIdx.x; idx < 8 * (D / 8); idx += blockDim.x) {
+    const int r = idx / (D / 8), c = (idx % (D / 8)) * 8;
+    uint4 v = make_uint4(0, 0, 0, 0);
+    if (r < G)
+      v = *reinterpret_cast<const uint4*>(a.q_rot + ((int64_t)b * a.Hq + g * G + r) * D + c);
+    *reinterpret_cast<uint4*>(qs + r * C::ROW + c) = v;
+  }
+  __syncthreads();
+  const uint64_t deadline = globaltimer_ns() + a.wait_ns;
+
+  if (warp == 4) {
+    // ---------------- producer ----------------
+    for (int t = 0; t < n_sub; ++t) {
+      const int slot = t % C::NSLOT;
+      bool ok = true;
+      if (lane == 0) {
+        if (t >= C::NSLOT)
+          ok = mbar_wait_bounded(&empty[slot], ((t / C::NSLOT) - 1) & 1, abort_flag, deadline,
+                                 a.status);
+        if (ok && *abort_flag) ok = false;
+      }
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) break;
+      const int64_t key0 = k_begin + (int64_t)t * C::KB;
+      const int nk = (int)((k_end - key0) < C::KB ? (k_end - key0) : C::KB);
+      const bool drop = a.drop_first_copy && t == 0 && split == 0 && g == 0 && b == 0;
+      if (drop) continue;
+      if (lane == 0) {
+        mbar_arrive_expect_tx(&full[slot], (uint32_t)(2 * nk * D * 2));
+        issued[slot] += 1;
+      }
+      __syncwarp();
+      const int r = lane & 15;
+      if (r < nk) {
+        const bool isv = lane >= 16;
+        bulk_g2s(ring + slot * C::SLOT_B + (isv ? C::KB * C::ROWB : 0) + r * C::ROWB,
+                 (isv ? vbase : kbase) + (key0 + r) * D, D * 2, &full[slot]);
+      }
+    }
+  } else {
+    // ---------------- consumers ----------------
+    const int gq = lane >> 2, tg = lane & 3;
+    float o[D / 16][4];
+#pragma unroll
+    for (int mt = 0; mt < D / 16; ++mt) o[mt][0] = o[mt][1] = o[mt][2] = o[mt][3] = 0.f;
+    float m_h = -INFINITY, l_t = 0.f;
+    const uint32_t q_addr = smem_u32(qs) + ((lane & 7) * C::ROW + ((lane >> 3) & 1) * 8) * 2;
+    const uint32_t frag_off = (((lane >> 4) * 8 + (lane & 7)) * C::ROW + ((lane >> 3) & 1) * 8) * 2;
+
+    for (int t = warp; t < n_sub; t += 4) {
+      const int slot = t % C::NSLOT;
+      const bool ok = mbar_wait_bounded(&full[slot], (t / C::NSLOT) & 1, abort_flag, deadline,
+                                        a.status);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      const int64_t key0 = k_begin + (int64_t)t * C::KB;
+      const int nk = (int)((k_end - key0) < C::KB ? (k_end - key0) : C::KB);
+      unsigned char* kslot = ring + slot * C::SLOT_B;
+      unsigned char* vslot = kslot + C::KB * C::ROWB;
+      if (nk < C::KB) {
+        // rows past the end were not copied: make them finite zeros
+        for (int idx = lane; idx < (C::KB - nk) * (D / 8); idx += 32) {
+          const int r = nk + idx / (D / 8), c = (idx % (D / 8)) * 8;
+          *reinterpret_cast<uint4*>(kslot + r * C::ROWB + c * 2) = make_uint4(0, 0, 0, 0);
+          *reinterpret_cast<uint4*>(vslot + r * C::ROWB + c * 2) = make_uint4(0, 0, 0, 0);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+      }
+      // S = Q K^T : rows = query heads (8 real of 16), cols = 16 keys
+      float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
+      const uint32_t k_addr = smem_u32(kslot) + frag_off;
+#pragma unroll 8
+      for (int ks = 0; ks < D / 16; ++ks) {
+        uint32_t qa0, qa2, b0, b1, b2, b3;
+        ldsm_x2(q_addr + ks * 32, qa0, qa2);
+        ldsm_x4(k_addr + ks * 32, b0, b1, b2, b3);
+        mma_bf16(s0, qa0, 0u, qa2, 0u, b0, b1);
+        mma_bf16(s1, qa0, 0u, qa2, 0u, b2, b3);
+      }
+      // online softmax for head gq; this thread holds keys 2tg,2tg+1 and 8+2tg,8+2tg+1
+      float sv[4];
+      sv[0] = (2 * tg < nk) ? s0[0] * a.scale_log2 : -INFINITY;
+      sv[1] = (2 * tg + 1 < nk) ? s0[1] * a.scale_log2 : -INFINITY;
+      sv[2] = (8 + 2 * tg < nk) ? s1[0] * a.scale_log2 : -INFINITY;
+      sv[3] = (9 + 2 * tg < nk) ? s1[1] * a.scale_log2 : -INFINITY;
+      float tmax = fmaxf(fmaxf(sv[0], sv[1]), fmaxf(sv[2], sv[3]));
+      tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 1));
+      tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 2));
+      const float m_new = fmaxf(m_h, tmax);
+      const float base = (m_new == -INFINITY) ? 0.f : m_new;
+      const float alpha = exp2f(m_h - base);
+      float p[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) p[i] = exp2f(sv[i] - base);
+      l_t = l_t * alpha + (p[0] + p[1]) + (p[2] + p[3]);
+      m_h = m_new;
+      const float al0 = __shfl_sync(0xffffffffu, alpha, (2 * tg) * 4);
+      const float al1 = __shfl_sync(0xffffffffu, alpha, (2 * tg + 1) * 4);
+      if (__any_sync(0xffffffffu, al0 != 1.f || al1 != 1.f)) {
+#pragma unroll
+        for (int mt = 0; mt < D / 16; ++mt) {
+          o[mt][0] *= al0;
+          o[mt][1] *= al1;
+          o[mt][2] *= al0;
+          o[mt][3] *= al1;
+        }
+      }
+      const uint32_t pb0 = pack_bf16x2(p[0], p[1]);
+      const uint32_t pb1 = pack_bf16x2(p[2], p[3]);
+      // O^T += V^T P^T : rows = head dims, cols = query heads, k = 16 keys
+      const uint32_t v_addr = smem_u32(vslot) + frag_off;
+#pragma unroll
+      for (int mt = 0; mt < D / 16; ++mt) {
+        uint32_t va0, va1, va2, va3;
+        ldsm_x4_t(v_addr + mt * 32, va0, va1, va2, va3);
+        mma_bf16(o[mt], va0, va1, va2, va3, pb0, pb1);
+      }
+      __syncwarp();
+      if (lane == 0) {
+        consumed[slot] += 1;
+        mbar_arrive(&empty[slot]);
+      }
+    }
+    float l_q = l_t + __shfl_xor_sync(0xffffffffu, l_t, 1);
+    l_q += __shfl_xor_sync(0xffffffffu, l_q, 2);
+    if (tg == 0) {
+      m_w[warp * 8 + gq] = m_h;
+      l_w[warp * 8 + gq] = l_q;
+    }
+    __syncthreads();  // (A) pairs with the producer's (A)
+    if (*abort_flag) return;
+    // scale this warp's O into the merge buffer (overlays the drained ring)
+    float* obuf = reinterpret_cast<float*>(ring);
+    float f[2];
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      const int hh = 2 * tg + j;
+      float M = -INFINITY;
+#pragma unroll
+      for (int w = 0; w < 4; ++w) M = fmaxf(M, m_w[w * 8 + hh]);
+      const float mw = m_w[warp * 8 + hh];
+      f[j] = (mw == -INFINITY) ? 0.f : exp2f(mw - M);
+    }
+#pragma unroll
+    for (int mt = 0; mt < D / 16; ++mt) {
+      float* row0 = obuf + (warp * 8 + 2 * tg) * C::OSTR + mt * 16 + gq;
+      float* row1 = row0 + C::OSTR;
+      row0[0] = o[mt][0] * f[0];
+      row1[0] = o[mt][1] * f[1];
+      row0[8] = o[mt][2] * f[0];
+      row1[8] = o[mt][3] * f[1];
+    }
+    named_bar_sync(1, 128);
+    for (int idx = threadIdx.x; idx < G * D; idx += 128) {
+      const int hh = idx / D, d = idx % D;
+      float M = -INFINITY;
+#pragma unroll
+      for (int w = 0; w < 4; ++w) M = fmaxf(M, m_w[w * 8 + hh]);
+      float L = 0.f, acc = 0.f;
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+        const float mw = m_w[w * 8 + hh];
+        L += (mw == -INFINITY) ? 0.f : l_w[w * 8 + hh] * exp2f(mw - M);
+        acc += obuf[(w * 8 + hh) * C::OSTR + d];
+      }
+      const int64_t pr = ((int64_t)b * a.Hq + g * G + hh) * a.n_splits + split;
+      a.part_o[pr * D + d] = acc / L;
+      if (d == 0) a.part_lse[pr] = M + log2f(L);
+    }
+    return;
+  }
+  // producer reaches here
+  __syncthreads();  // (A)
+  if (*abort_flag && lane == 0) {
+    // drain: wait (bounded) for copies that were issued but never consumed
+    const uint64_t dl = globaltimer_ns() + 200000000ull;
+    volatile int dummy = 0;
+    for (int s = 0; s < C::NSLOT; ++s)
+      if (issued[s] > consumed[s])
+        mbar_wait_bounded(&full[s], (issued[s] - 1) & 1, &dummy, dl, a.status);
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(128) k_decode_combine(DecodeAttnArgs a) {
+  const int h = blockIdx.x, b = blockIdx.y;
+  bf16* dst = a.out + ((int64_t)b * a.Hq + h) * D;
+  const int64_t len = a.seq_lens[b];
+  if (len < 1 || len > a.max_len) {
+    for (int d = threadIdx.x; d < D; d += blockDim.x) dst[d] = __float2bfloat16(0.f);
+    return;
+  }
+  const int64_t n_valid = a.window > 0 ? (len < a.window ? len : (int64_t)a.window) : len;
+  const int n_used = (int)((n_valid + a.chunk - 1) / a.chunk);
+  const int64_t pr0 = ((int64_t)b * a.Hq + h) * a.n_splits;
+  float M = -INFINITY;
+  for (int s = 0; s < n_used; ++s) M = fmaxf(M, a.part_lse[pr0 + s]);
+  float wsum = 0.f;
+  for (int s = 0; s < n_used; ++s) wsum += exp2f(a.part_lse[pr0 + s] - M);
+  const float inv = 1.f / wsum;
+  for (int d = threadIdx.x * 4; d < D; d += blockDim.x * 4) {
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int s = 0; s < n_used; ++s) {
+      const float w = exp2f(a.part_lse[pr0 + s] - M);
+      const float4 v = *reinterpret_cast<const float4*>(a.part_o + (pr0 + s) * D + d);
+      acc.x += w * v.x;
+      acc.y += w * v.y;
+      acc.z += w * v.z;
+      acc.w += w * v.w;
+    }
+    uint2 pk = make_uint2(pack_bf16x2(acc.x * inv, acc.y * inv), pack_bf16x2(acc.z * inv, acc.w * inv));
+    *reinterpret_cast<uint2*>(dst + d) = pk;
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_decode_split(const DecodeAttnArgs& a, int B, int D, cudaStream_t st) {
+  dim3 grid(a.n_splits, a.Hkv, B);
+  if (D == 256) {
+    using C = DecCfg<256>;
+    cudaFuncSetAttribute(k_decode_split<256>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    k_decode_split<256><<<grid, 160, C::SMEM, st>>>(a);
+  } else {
+    using C = DecCfg<512>;
+    cudaFuncSetAttribute(k_decode_split<512>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    k_decode_split<512><<<grid, 160, C::SMEM, st>>>(a);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_decode_combine(const DecodeAttnArgs& a, int B, int D, cudaStream_t st) {
+  dim3 grid(a.Hq, B);
+  if (D == 256)
+    k_decode_combine<256><<<grid, 64, 0, st>>>(a);
+  else
+    k_decode_combine<512><<<grid, 128, 0, st>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace hlg

@@ -1,0 +1,90 @@
+// kernels.h -- launch interfaces between the C ABI (api.cu) and the kernels.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace hlg {
+
+typedef __nv_bfloat16 bf16;
+
+struct PrefillRopeArgs {
+  const bf16* q;       // [B][S][Hq][D]
+  const bf16* k_new;   // [B][S][Hkv][D] or null (shared layer)
+  const bf16* v_new;   // [B][S][Hkv][D] or null
+  bf16* q_rot;         // workspace [B][S][Hq][D]
+  bf16* k_rot;         // workspace [B][S][Hkv][D] (local layers) or null
+  bf16* k_cache;       // [B][Hkv][cap][D]
+  bf16* v_cache;
+  int cache_cap;
+  const int32_t* seq_lens_before;  // device [B] or null
+  int S, window, Hq, Hkv;
+  int n_rot;           // rotated pairs
+  double log2_theta;
+  int rows_per_cta;
+  int* status;
+};
+
+struct DecodeRopeArgs {
+  const bf16* q;       // [B][Hq][D]
+  const bf16* k_new;   // [B][Hkv][D] or null
+  const bf16* v_new;
+  bf16* q_rot;         // workspace [B][Hq][D]
+  bf16* k_cache;
+  bf16* v_cache;
+  int cache_cap;
+  const int32_t* seq_lens;
+  int max_len, window, Hq, Hkv;
+  int n_rot;
+  double log2_theta;
+  int* status;
+};
+
+// Keys/values of one prefill layer as strided 4-D views (b, row, head, d);
+// row = key position. Global layers read the cache, local layers the
+// rotated-K workspace and the caller's V.
+struct KVView {
+  const bf16* ptr;
+  int64_t stride_b, stride_row, stride_h;  // in elements; d is contiguous
+};
+
+struct PrefillAttnArgs {
+  const bf16* q_rot;   // [B][S][Hq][D]
+  KVView k, v;
+  int64_t key_cap;     // rows readable per (batch, head) in the K/V views
+  const int32_t* seq_lens_before;  // device [B] or null
+  int S, window, Hq, Hkv;
+  float scale_log2;    // scale * log2(e)
+  bf16* out;           // [B][S][Hq][D]
+  float* lse;          // [B][Hq][S] or null
+  int* status;
+};
+
+struct DecodeAttnArgs {
+  const bf16* q_rot;       // [B][Hq][D]
+  const bf16* k_cache;     // [B][Hkv][cap][D]
+  const bf16* v_cache;
+  int cache_cap;
+  const int32_t* seq_lens; // device [B]
+  int max_len, window, Hq, Hkv;
+  int chunk;               // keys per split (multiple of 16)
+  int n_splits;
+  float scale_log2;
+  float* part_o;           // [B][Hq][n_splits][D]
+  float* part_lse;         // [B][Hq][n_splits] (log2 domain)
+  bf16* out;               // [B][Hq][D]
+  int* status;
+  unsigned long long wait_ns;
+  int drop_first_copy;     // test hook: skip the first K/V copy of split 0
+};
+
+cudaError_t launch_prefill_rope(const PrefillRopeArgs& a, int B, int D, cudaStream_t st);
+cudaError_t launch_decode_rope_append(const DecodeRopeArgs& a, int B, int D, cudaStream_t st);
+cudaError_t launch_prefill_attn(const PrefillAttnArgs& a, int B, int D, cudaStream_t st);
+cudaError_t launch_decode_split(const DecodeAttnArgs& a, int B, int D, cudaStream_t st);
+cudaError_t launch_decode_combine(const DecodeAttnArgs& a, int B, int D, cudaStream_t st);
+cudaError_t launch_visible_ranges(const int32_t* seq_lens_before, int B, int S, int window,
+                                  int32_t* ranges, cudaStream_t st);
+
+}  // namespace hlg

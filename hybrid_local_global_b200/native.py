@@ -1,0 +1,205 @@
+"""ctypes binding of ``libgemma_attn.so`` -- argument marshalling only.
+
+Every function carries the name of the C entry point it calls (declared in
+``include/gemma_attn.h``). Tensors are torch CUDA tensors; their device
+pointers, the shapes read off them and the current CUDA stream are passed
+through unchanged. There is no fallback: if the shared library is missing
+the import fails.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libgemma_attn.so")
+if not os.path.exists(_LIB_PATH):
+    raise ImportError(
+        "libgemma_attn.so is not built (run `python -m hybrid_local_global_b200.build`); "
+        "there is no fallback implementation")
+_lib = ctypes.CDLL(_LIB_PATH)
+LIB_PATH = _LIB_PATH
+
+GEMMA_OK = 0
+GEMMA_ERR_INVALID_ARG = 1
+GEMMA_ERR_UNSUPPORTED = 2
+GEMMA_ERR_SHARE_MISMATCH = 3
+GEMMA_ERR_CAPACITY = 4
+GEMMA_ERR_CUDA = 5
+GEMMA_ERR_DEVICE_TIMEOUT = 6
+GEMMA_ERR_DEVICE_RANGE = 7
+GEMMA_F_SHARED = 1
+
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+_F = ctypes.c_float
+_SZ = ctypes.c_size_t
+
+
+class gemma_kv_desc(ctypes.Structure):
+    _fields_ = [("k_cache", _P), ("v_cache", _P), ("layer", _I), ("cache_cap", _I),
+                ("window", _I), ("n_kv_heads", _I), ("head_dim", _I), ("rope_frac", _F),
+                ("rope_theta", _F), ("shared_from", _I)]
+
+
+def _sig(name, restype, argtypes):
+    f = getattr(_lib, name)
+    f.restype = restype
+    f.argtypes = argtypes
+    return f
+
+
+_prefill_ws = _sig("gemma_attn_prefill_workspace_size", _SZ, [_I, _I, _I, _I, _I, _I])
+_prefill = _sig("gemma_attn_prefill", _I, [_P, _P, _P, _P, _P, _I, _P, _I, _I, _I, _I, _I, _I,
+                                           _F, _F, _F, _P, _P, _P, _SZ, ctypes.c_uint, _P])
+_decode_ws = _sig("gemma_attn_decode_workspace_size", _SZ, [_I, _I, _I, _I, _I, _I])
+_decode = _sig("gemma_attn_decode", _I, [_P, _P, _P, _P, _P, _I, _P, _I, _I, _I, _I, _I, _I,
+                                         _F, _F, _F, _P, _P, _SZ, ctypes.c_uint, _P])
+_bind = _sig("gemma_kv_share_bind", _I, [ctypes.POINTER(gemma_kv_desc), ctypes.POINTER(gemma_kv_desc)])
+_sched = _sig("gemma_layer_schedule", _I, [_I, _I, _I, ctypes.POINTER(_I), ctypes.POINTER(_I)])
+_ranges = _sig("gemma_attn_visible_ranges", _I, [_P, _I, _I, _I, _P, _P])
+_sync = _sig("gemma_attn_sync_status", _I, [_P])
+_last = _sig("gemma_last_error", ctypes.c_char_p, [])
+_wait = _sig("gemma_attn_set_wait_limit", _I, [ctypes.c_longlong])
+_drop = _sig("gemma_attn_debug_drop_next_copy", _I, [_I])
+
+EXPORTED = ["gemma_attn_prefill_workspace_size", "gemma_attn_prefill",
+            "gemma_attn_decode_workspace_size", "gemma_attn_decode", "gemma_kv_share_bind",
+            "gemma_layer_schedule", "gemma_attn_visible_ranges", "gemma_attn_sync_status",
+            "gemma_last_error", "gemma_attn_set_wait_limit", "gemma_attn_debug_drop_next_copy"]
+
+
+class GemmaError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__("gemma_attn error %d: %s" % (code, msg))
+        self.code = code
+
+
+def _check(rc: int) -> int:
+    if rc != GEMMA_OK:
+        raise GemmaError(rc, gemma_last_error())
+    return rc
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _bf16(t, name):
+    if t is None:
+        return
+    if t.dtype != torch.bfloat16 or not t.is_contiguous() or not t.is_cuda:
+        raise TypeError("%s must be a contiguous bf16 CUDA tensor" % name)
+
+
+def gemma_last_error() -> str:
+    s = _last()
+    return s.decode() if s else ""
+
+
+def gemma_attn_prefill_workspace_size(batch, s_new, n_q_heads, n_kv_heads, head_dim, window) -> int:
+    return int(_prefill_ws(batch, s_new, n_q_heads, n_kv_heads, head_dim, window))
+
+
+def gemma_attn_prefill(q, k_new, v_new, k_cache, v_cache, *, window, rope_frac, rope_theta, scale,
+                       out, seq_lens_before=None, lse=None, workspace=None, flags=0, stream=None):
+    """q [B,S,Hq,D]; k_new/v_new [B,S,Hkv,D] (None if shared); caches [B,Hkv,cap,D]."""
+    for t, n in ((q, "q"), (k_new, "k_new"), (v_new, "v_new"), (k_cache, "k_cache"),
+                 (v_cache, "v_cache"), (out, "out")):
+        _bf16(t, n)
+    B, S, Hq, D = q.shape
+    _, Hkv, cap, _ = k_cache.shape
+    if workspace is None:
+        n = gemma_attn_prefill_workspace_size(B, S, Hq, Hkv, D, window)
+        workspace = torch.empty(max(n, 1), dtype=torch.uint8, device=q.device)
+    return _check(_prefill(_ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_cache), _ptr(v_cache), cap,
+                           _ptr(seq_lens_before), B, S, window, Hq, Hkv, D, rope_frac, rope_theta,
+                           scale, _ptr(out), _ptr(lse), _ptr(workspace), workspace.numel(), flags,
+                           _stream(stream)))
+
+
+def gemma_attn_decode_workspace_size(batch, n_q_heads, n_kv_heads, head_dim, window, max_seq_len) -> int:
+    return int(_decode_ws(batch, n_q_heads, n_kv_heads, head_dim, window, max_seq_len))
+
+
+def gemma_attn_decode(q, k_new, v_new, k_cache, v_cache, *, seq_lens, max_seq_len, window,
+                      rope_frac, rope_theta, scale, out, workspace=None, flags=0, stream=None):
+    """q [B,Hq,D]; k_new/v_new [B,Hkv,D] (None if shared); caches [B,Hkv,cap,D];
+    seq_lens int32 [B] on the device (length including the new token)."""
+    for t, n in ((q, "q"), (k_new, "k_new"), (v_new, "v_new"), (k_cache, "k_cache"),
+                 (v_cache, "v_cache"), (out, "out")):
+        _bf16(t, n)
+    if seq_lens.dtype != torch.int32 or not seq_lens.is_cuda:
+        raise TypeError("seq_lens must be an int32 CUDA tensor")
+    B, Hq, D = q.shape
+    _, Hkv, cap, _ = k_cache.shape
+    if workspace is None:
+        n = gemma_attn_decode_workspace_size(B, Hq, Hkv, D, window, max_seq_len)
+        workspace = torch.empty(max(n, 1), dtype=torch.uint8, device=q.device)
+    return _check(_decode(_ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_cache), _ptr(v_cache), cap,
+                          _ptr(seq_lens), max_seq_len, B, window, Hq, Hkv, D, rope_frac,
+                          rope_theta, scale, _ptr(out), _ptr(workspace), workspace.numel(), flags,
+                          _stream(stream)))
+
+
+def gemma_kv_share_bind(dst: gemma_kv_desc, src: gemma_kv_desc) -> int:
+    return _check(_bind(ctypes.byref(dst), ctypes.byref(src)))
+
+
+def gemma_layer_schedule(n_layers: int, ratio: int, n_shared: int = 0):
+    g = (_I * n_layers)()
+    s = (_I * n_layers)()
+    _check(_sched(n_layers, ratio, n_shared, g, s))
+    return [bool(x) for x in g], [int(x) for x in s]
+
+
+def gemma_attn_visible_ranges(batch, s_new, window, ranges, seq_lens_before=None, stream=None):
+    if ranges.dtype != torch.int32 or not ranges.is_cuda or ranges.numel() < batch * s_new * 3:
+        raise TypeError("ranges must be an int32 CUDA tensor of batch*s_new*3 elements")
+    return _check(_ranges(_ptr(seq_lens_before), batch, s_new, window, _ptr(ranges), _stream(stream)))
+
+
+def gemma_attn_sync_status(stream=None) -> int:
+    """Returns the status code (does not raise)."""
+    return int(_sync(_stream(stream)))
+
+
+def gemma_attn_set_wait_limit(max_ns: int) -> int:
+    return _check(_wait(max_ns))
+
+
+def gemma_attn_debug_drop_next_copy(enable: bool) -> int:
+    return _check(_drop(int(bool(enable))))
+
+
+GEMMA_KERNEL_PREFILL_ROPE = 0
+GEMMA_KERNEL_PREFILL_ATTN = 1
+GEMMA_KERNEL_DECODE_APPEND = 2
+GEMMA_KERNEL_DECODE_SPLIT = 3
+GEMMA_KERNEL_DECODE_COMBINE = 4
+KERNEL_NAMES = {0: "prefill_rope", 1: "prefill_attn", 2: "decode_append", 3: "decode_split",
+                4: "decode_combine"}
+
+_prof = _sig("gemma_attn_profile", _I, [_I])
+_prof_read = _sig("gemma_attn_profile_read", _I, [_I, ctypes.POINTER(ctypes.c_double),
+                                                  ctypes.POINTER(ctypes.c_longlong)])
+EXPORTED += ["gemma_attn_profile", "gemma_attn_profile_read"]
+
+
+def gemma_attn_profile(enable: bool) -> int:
+    return _check(_prof(int(bool(enable))))
+
+
+def gemma_attn_profile_read(kernel: int):
+    """-> (total device ms, launches) of one kernel kind since profiling began."""
+    ms = ctypes.c_double()
+    n = ctypes.c_longlong()
+    _check(_prof_read(kernel, ctypes.byref(ms), ctypes.byref(n)))
+    return float(ms.value), int(n.value)

@@ -1,0 +1,105 @@
+"""A block of interleaved local/global attention layers driven through the C ABI.
+
+The layer schedule and the share map come from ``gemma_layer_schedule``; a
+shared layer's cache descriptor is bound to its source with
+``gemma_kv_share_bind`` (pointer aliasing, no copy) and its calls carry
+``GEMMA_F_SHARED`` so that it neither rotates nor writes K/V. Device memory
+(caches, workspace, outputs) is torch-owned; all compute is in the library.
+"""
+from __future__ import annotations
+
+import torch
+
+from . import native
+from .workloads import LayerType, Workload
+
+
+class AttentionStack:
+    def __init__(self, w: Workload, device="cuda", global_capacity: int | None = None,
+                 alloc_caches: bool = True):
+        self.w = w
+        self.device = torch.device(device)
+        if w.fixed_kinds:
+            self.is_global = [k == "global" for k in w.fixed_kinds]
+            self.share_src = list(range(len(w.fixed_kinds)))
+        else:
+            self.is_global, self.share_src = native.gemma_layer_schedule(w.n_layers, w.ratio, w.n_shared)
+        self.n_layers = len(self.is_global)
+        if global_capacity is None:
+            global_capacity = (w.prior + w.seq) if w.kind == "prefill" else w.len_hi
+        self.global_capacity = global_capacity
+        self.descs: list[native.gemma_kv_desc] = []
+        self.k_cache: list[torch.Tensor] = []
+        self.v_cache: list[torch.Tensor] = []
+        for l in range(self.n_layers):
+            t = self.layer_type(l)
+            cap = t.window if t.window > 0 else global_capacity
+            d = native.gemma_kv_desc()
+            d.layer, d.cache_cap, d.window = l, cap, t.window
+            d.n_kv_heads, d.head_dim = t.n_kv_heads, t.head_dim
+            d.rope_frac, d.rope_theta, d.shared_from = t.rope_frac, t.rope_theta, -1
+            src = self.share_src[l]
+            if src >= 0 and src != l:
+                native.gemma_kv_share_bind(d, self.descs[src])
+                self.k_cache.append(self.k_cache[d.shared_from])
+                self.v_cache.append(self.v_cache[d.shared_from])
+            else:
+                shape = (w.batch, t.n_kv_heads, cap, t.head_dim)
+                if alloc_caches:
+                    kc = torch.empty(shape, dtype=torch.bfloat16, device=self.device)
+                    vc = torch.empty(shape, dtype=torch.bfloat16, device=self.device)
+                    d.k_cache, d.v_cache = kc.data_ptr(), vc.data_ptr()
+                else:
+                    kc = vc = None
+                self.k_cache.append(kc)
+                self.v_cache.append(vc)
+            self.descs.append(d)
+
+    def layer_type(self, l: int) -> LayerType:
+        return self.w.global_ if self.is_global[l] else self.w.local
+
+    def is_shared(self, l: int) -> bool:
+        return self.descs[l].shared_from >= 0
+
+    def owned_cache_bytes(self) -> int:
+        seen, total = set(), 0
+        for l in range(self.n_layers):
+            kc = self.k_cache[l]
+            if kc is None or kc.data_ptr() in seen:
+                continue
+            seen.add(kc.data_ptr())
+            total += 2 * kc.numel() * kc.element_size()
+        return total
+
+    # ------------------------------------------------------------------ prefill
+    def prefill_workspace_bytes(self) -> int:
+        w = self.w
+        return max(native.gemma_attn_prefill_workspace_size(
+            w.batch, w.seq, w.n_q_heads, self.layer_type(l).n_kv_heads, self.layer_type(l).head_dim,
+            self.layer_type(l).window) for l in range(self.n_layers))
+
+    def prefill_layer(self, l: int, q, k, v, out, *, workspace, seq_lens_before=None, lse=None,
+                      stream=None):
+        t = self.layer_type(l)
+        shared = self.is_shared(l)
+        native.gemma_attn_prefill(
+            q, None if shared else k, None if shared else v, self.k_cache[l], self.v_cache[l],
+            window=t.window, rope_frac=t.rope_frac, rope_theta=t.rope_theta, scale=t.scale,
+            out=out, seq_lens_before=seq_lens_before, lse=lse, workspace=workspace,
+            flags=native.GEMMA_F_SHARED if shared else 0, stream=stream)
+
+    # ------------------------------------------------------------------ decode
+    def decode_workspace_bytes(self, max_seq_len: int) -> int:
+        w = self.w
+        return max(native.gemma_attn_decode_workspace_size(
+            w.batch, w.n_q_heads, self.layer_type(l).n_kv_heads, self.layer_type(l).head_dim,
+            self.layer_type(l).window, max_seq_len) for l in range(self.n_layers))
+
+    def decode_layer(self, l: int, q, k, v, out, *, seq_lens, max_seq_len, workspace, stream=None):
+        t = self.layer_type(l)
+        shared = self.is_shared(l)
+        native.gemma_attn_decode(
+            q, None if shared else k, None if shared else v, self.k_cache[l], self.v_cache[l],
+            seq_lens=seq_lens, max_seq_len=max_seq_len, window=t.window, rope_frac=t.rope_frac,
+            rope_theta=t.rope_theta, scale=t.scale, out=out, workspace=workspace,
+            flags=native.GEMMA_F_SHARED if shared else 0, stream=stream)

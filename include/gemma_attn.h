@@ -1,0 +1,229 @@
+/*
+ * gemma_attn.h -- C ABI of libgemma_attn.so: interleaved local (sliding
+ * window) / global causal grouped-query attention with (proportional) RoPE,
+ * a ring-buffer / append KV cache and last-N-layer KV sharing, for NVIDIA
+ * B200 (sm_100a).
+ *
+ * Passages defining the operations (page title, section):
+ *   - "Gemma 4: End-to-End Architecture Walkthrough", 3a "Interleaved
+ *     Local/Global Attention": local layers attend to a fixed recent window,
+ *     global layers to the whole preceding context; r local layers per
+ *     global layer; the final layer is always global.
+ *   - same page, 3b "Making the Expensive Global Layers Cheaper": GQA 8:1 on
+ *     global layers (2:1 on local ones), doubled key dimension; global
+ *     layers cache K/V for the whole context.
+ *   - same page, 3c "p-RoPE", and "Gemma 4 Architecture Reference",
+ *     "Positional Encoding: Proportional RoPE (p-RoPE)": on global layers
+ *     only the first p = 0.25 of the dimension pairs rotate, theta = 1e6.
+ *   - "Gemma 4 Architecture Reference", "Attention Architecture" (window
+ *     512 / 1024, GQA ratios) and "Shared KV Cache" (the last N layers reuse
+ *     K/V of an earlier layer of the same attention type).
+ *
+ * Conventions for every call:
+ *   - Tensors are bf16 (IEEE bfloat16 bit patterns), contiguous, row-major in
+ *     the stated shape, in device memory, 16-byte aligned. fp32 outputs and
+ *     int32 length arrays are device memory too.
+ *   - The caller owns all memory. The library never allocates device memory;
+ *     calls that need scratch take a caller-sized workspace.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream). Calls are
+ *     asynchronous on it; argument errors are reported before anything is
+ *     enqueued and nothing is enqueued on error.
+ *   - Positions are 0-based and absolute. Key j is visible to the query at
+ *     position p iff j <= p and (window == 0 or j > p - window).
+ *   - RoPE pairs dimensions (2i, 2i+1) and turns pair i by the angle
+ *     p * rope_theta^(-2i/head_dim) when i < floor(rope_frac * head_dim / 2);
+ *     other pairs are left as they are. V is never rotated.
+ *   - Cache layout: [batch][n_kv_heads][cache_cap][head_dim]. A global layer
+ *     (window == 0) keeps position p in slot p (cache_cap >= context length).
+ *     A local layer keeps a ring of cache_cap == window slots, position p in
+ *     slot p % window.
+ *   - Return value: a gemma_status. On failure gemma_last_error() gives a
+ *     message (thread-local, valid until the next call on that thread).
+ */
+#ifndef GEMMA_ATTN_H
+#define GEMMA_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define GEMMA_ATTN_ABI_VERSION 1
+
+typedef enum gemma_status {
+    GEMMA_OK = 0,
+    GEMMA_ERR_INVALID_ARG = 1,    /* bad pointer, size, ratio or flag */
+    GEMMA_ERR_UNSUPPORTED = 2,    /* valid request this build does not implement */
+    GEMMA_ERR_SHARE_MISMATCH = 3, /* gemma_kv_share_bind: layers not compatible */
+    GEMMA_ERR_CAPACITY = 4,       /* cache or workspace too small */
+    GEMMA_ERR_CUDA = 5,           /* a CUDA runtime call failed */
+    GEMMA_ERR_DEVICE_TIMEOUT = 6, /* a bounded device wait gave up (see sync_status) */
+    GEMMA_ERR_DEVICE_RANGE = 7    /* a device-side length/capacity check failed */
+} gemma_status;
+
+/* flags */
+#define GEMMA_F_SHARED 1u /* k_cache/v_cache alias an earlier layer (see
+                             gemma_kv_share_bind): k_new and v_new must be NULL;
+                             nothing is rotated or written into the cache. */
+
+/* Supported shapes: head_dim 256 or 512; n_q_heads a multiple of n_kv_heads
+ * with n_q_heads / n_kv_heads <= 8; window 0 (global) or a multiple of 16. */
+
+/* ---------------------------------------------------------------------- */
+/* Prefill: a chunk of s_new tokens per sequence.                          */
+/*                                                                        */
+/* q      [batch][s_new][n_q_heads][head_dim]   pre-RoPE queries           */
+/* k_new  [batch][s_new][n_kv_heads][head_dim]  pre-RoPE keys (NULL if     */
+/* v_new  [batch][s_new][n_kv_heads][head_dim]  values        GEMMA_F_SHARED)*/
+/* k_cache, v_cache [batch][n_kv_heads][cache_cap][head_dim]               */
+/* seq_lens_before  device int32 [batch]: tokens already in the cache per   */
+/*        sequence (the chunk starts at that position), or NULL for 0.     */
+/*        Must be NULL on a local layer (chunked local prefill is not      */
+/*        implemented: GEMMA_ERR_UNSUPPORTED).                              */
+/* out    [batch][s_new][n_q_heads][head_dim]  bf16 attention output        */
+/* lse    optional fp32 [batch][n_q_heads][s_new]: natural-log sum of       */
+/*        exp(scale * q.k) over the visible keys; NULL to skip.            */
+/* workspace: at least gemma_attn_prefill_workspace_size(...) bytes,       */
+/*        256-byte aligned; contents are scratch.                          */
+/*                                                                        */
+/* Effect: rotated K and V of the chunk are written into the cache (global:*/
+/* slots seq_lens_before[b] .. +s_new-1; local: the ring slots of the last */
+/* `window` positions), then every query attends causally (window-limited */
+/* on local layers) to the cached context plus the chunk. On a global     */
+/* layer seq_lens_before[b] + s_new must not exceed cache_cap; a device-   */
+/* side check skips the sequence and reports GEMMA_ERR_DEVICE_RANGE       */
+/* through gemma_attn_sync_status otherwise.                              */
+/* ---------------------------------------------------------------------- */
+size_t gemma_attn_prefill_workspace_size(int batch, int s_new, int n_q_heads,
+                                         int n_kv_heads, int head_dim, int window);
+
+int gemma_attn_prefill(const void* q, const void* k_new, const void* v_new,
+                       void* k_cache, void* v_cache, int cache_cap,
+                       const int32_t* seq_lens_before, int batch, int s_new,
+                       int window, int n_q_heads, int n_kv_heads, int head_dim,
+                       float rope_frac, float rope_theta, float scale,
+                       void* out, float* lse, void* workspace,
+                       size_t workspace_bytes, unsigned flags, void* stream);
+
+/* ---------------------------------------------------------------------- */
+/* Decode: one new token per sequence, batched.                            */
+/*                                                                        */
+/* q      [batch][n_q_heads][head_dim]   pre-RoPE query of the new token   */
+/* k_new, v_new [batch][n_kv_heads][head_dim] pre-RoPE key / value of the  */
+/*        new token (NULL with GEMMA_F_SHARED)                              */
+/* seq_lens device int32 [batch]: sequence length INCLUDING the new token; */
+/*        the new token sits at position seq_lens[b] - 1; every value must */
+/*        be in [1, max_seq_len].                                          */
+/* max_seq_len host upper bound of seq_lens (sizes the split-K grid).      */
+/* out    [batch][n_q_heads][head_dim] bf16.                                */
+/* workspace: at least gemma_attn_decode_workspace_size(...) bytes,        */
+/*        256-byte aligned; contents are scratch.                          */
+/*                                                                        */
+/* Effect: the rotated new key and the new value are written at the slot   */
+/* of position seq_lens[b]-1 (unless shared); then the query attends to   */
+/* every visible cached position (global: all seq_lens[b] positions;      */
+/* local: the last min(seq_lens[b], window) positions held by the ring).  */
+/* The cache before the call must hold rotated keys for earlier positions.*/
+/* ---------------------------------------------------------------------- */
+size_t gemma_attn_decode_workspace_size(int batch, int n_q_heads, int n_kv_heads,
+                                        int head_dim, int window, int max_seq_len);
+
+int gemma_attn_decode(const void* q, const void* k_new, const void* v_new,
+                      void* k_cache, void* v_cache, int cache_cap,
+                      const int32_t* seq_lens, int max_seq_len, int batch,
+                      int window, int n_q_heads, int n_kv_heads, int head_dim,
+                      float rope_frac, float rope_theta, float scale, void* out,
+                      void* workspace, size_t workspace_bytes, unsigned flags,
+                      void* stream);
+
+/* ---------------------------------------------------------------------- */
+/* KV sharing ("Gemma 4 Architecture Reference", "Shared KV Cache").       */
+/* Host only: no device work, no bytes move.                               */
+/* ---------------------------------------------------------------------- */
+typedef struct gemma_kv_desc {
+    void* k_cache;      /* [batch][n_kv_heads][cache_cap][head_dim] bf16 */
+    void* v_cache;
+    int layer;          /* index of the layer in its stack */
+    int cache_cap;
+    int window;         /* 0 = global layer */
+    int n_kv_heads;
+    int head_dim;
+    float rope_frac;
+    float rope_theta;
+    int shared_from;    /* -1: owns its cache; else the layer whose cache it reads */
+} gemma_kv_desc;
+
+/* Makes dst read src's cache: dst->k_cache/v_cache become src's pointers and
+ * dst->shared_from the layer that owns them (a chain resolves to its root).
+ * Requires src->layer < dst->layer and identical window, cache_cap,
+ * n_kv_heads, head_dim, rope_frac and rope_theta (same attention type);
+ * otherwise returns GEMMA_ERR_SHARE_MISMATCH and leaves dst unchanged.
+ * Afterwards call the attention entry points for dst with GEMMA_F_SHARED. */
+int gemma_kv_share_bind(gemma_kv_desc* dst, const gemma_kv_desc* src);
+
+/* Layer schedule of an n_layers stack with `ratio` local layers per global
+ * layer ("Gemma 4: End-to-End Architecture Walkthrough", 3a): layer l is
+ * global iff (l + 1) % (ratio + 1) == 0 or l == n_layers - 1. With the last
+ * n_shared layers shared ("Shared KV Cache"), share_src[l] is the latest
+ * non-shared earlier layer of the same type, l itself for a non-shared
+ * layer, or -1 when a shared layer has no such source (it then keeps its own
+ * cache). Host arrays of n_layers ints; share_src may be NULL. */
+int gemma_layer_schedule(int n_layers, int ratio, int n_shared,
+                         int* is_global, int* share_src);
+
+/* Debug view of the mask logic the kernels use: for every (b, i) of a
+ * prefill chunk writes {lo, hi, count} of the visible key positions to the
+ * device int32 array ranges[batch][s_new][3] (count 0 -> lo > hi).
+ * seq_lens_before as in gemma_attn_prefill. Asynchronous on `stream`. */
+int gemma_attn_visible_ranges(const int32_t* seq_lens_before, int batch, int s_new,
+                              int window, int32_t* ranges, void* stream);
+
+/* Synchronises `stream`, then returns and clears the library's device error
+ * word: GEMMA_OK, GEMMA_ERR_DEVICE_TIMEOUT (a bounded wait inside a kernel
+ * gave up; that kernel's output is invalid), GEMMA_ERR_DEVICE_RANGE, or
+ * GEMMA_ERR_CUDA if the synchronisation itself failed. */
+int gemma_attn_sync_status(void* stream);
+
+/* Message for the last failed call on this thread ("" if none). */
+const char* gemma_last_error(void);
+
+/* Deadline of every bounded device wait (pipeline barriers), in nanoseconds
+ * of %globaltimer from the start of the waiting kernel's work unit. 0
+ * restores the default of one second. Host state, process-wide; affects
+ * launches issued afterwards. */
+int gemma_attn_set_wait_limit(long long max_ns);
+
+/* Test hook for the same path: when `enable` is nonzero, the next
+ * gemma_attn_decode launch does not issue the first key/value copy of its
+ * first work unit, so that unit's consumers wait on a barrier nothing will
+ * complete; their bounded wait runs out, the unit exits without output and
+ * gemma_attn_sync_status reports GEMMA_ERR_DEVICE_TIMEOUT. Nothing faults or
+ * hangs. One-shot: the flag clears when that launch is issued. */
+int gemma_attn_debug_drop_next_copy(int enable);
+
+/* ---------------------------------------------------------------------- */
+/* Measurement hook. While enabled, every launch of the kernels below is   */
+/* bracketed by a pair of CUDA events recorded on the call's stream (event */
+/* objects are created by the library; no device memory is allocated).    */
+/* gemma_attn_profile_read synchronises the recorded events and returns    */
+/* the summed device time and the launch count of one kernel kind since    */
+/* the last gemma_attn_profile(1). gemma_attn_profile(0) stops recording   */
+/* and releases the events.                                                */
+/* ---------------------------------------------------------------------- */
+#define GEMMA_KERNEL_PREFILL_ROPE 0     /* RoPE on Q/K + cache write (prefill) */
+#define GEMMA_KERNEL_PREFILL_ATTN 1     /* prefill attention */
+#define GEMMA_KERNEL_DECODE_APPEND 2    /* RoPE + cache append (decode) */
+#define GEMMA_KERNEL_DECODE_SPLIT 3     /* split-K decode attention */
+#define GEMMA_KERNEL_DECODE_COMBINE 4   /* log-sum-exp combine of the splits */
+#define GEMMA_KERNEL_KINDS 5
+
+int gemma_attn_profile(int enable);
+int gemma_attn_profile_read(int kernel, double* total_ms, long long* launches);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GEMMA_ATTN_H */

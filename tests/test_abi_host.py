@@ -1,0 +1,157 @@
+"""Host-side checks of libgemma_attn.so that need no GPU: the library loads
+and exports every entry point include/gemma_attn.h declares; the layer
+schedule and share map match the oracle; share binding and argument
+validation return the documented codes before touching any pointer."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from hybrid_local_global_b200 import native
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(__file__)), "include", "gemma_attn.h")
+FAKE = 0x10000  # never dereferenced: validation fails before any device work
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?[\w]+\s*\*?\s*(gemma_\w+)\s*\(", src, flags=re.M)))
+
+
+def test_exports_every_declared_symbol():
+    names = declared_functions()
+    assert len(names) >= 11, names
+    lib = ctypes.CDLL(native.LIB_PATH)
+    for n in names:
+        assert hasattr(lib, n), n
+    assert sorted(native.EXPORTED) == names
+
+
+@pytest.mark.parametrize("n,r,ns", [(5, 4, 0), (6, 5, 2), (12, 5, 2), (35, 4, 0), (42, 5, 3),
+                                    (60, 5, 10), (42, 4, 0), (8, 0, 3), (1, 5, 0), (1, 0, 1)])
+def test_schedule_matches_oracle(oracle, n, r, ns):
+    g, s = native.gemma_layer_schedule(n, r, ns)
+    assert g == oracle.layer_schedule(n, r)
+    assert s == [oracle.share_source(n, r, ns, l) for l in range(n)]
+
+
+def test_schedule_rejects_bad_arguments():
+    for args in ((0, 4, 0), (5, -1, 0), (5, 4, 6), (5, 4, -1)):
+        with pytest.raises(native.GemmaError) as e:
+            native.gemma_layer_schedule(*args)
+        assert e.value.code == native.GEMMA_ERR_INVALID_ARG
+
+
+def _desc(layer, window, cap, hkv=4, d=512, frac=0.25, theta=1e6, k=FAKE, v=FAKE + 0x1000):
+    x = native.gemma_kv_desc()
+    x.k_cache, x.v_cache, x.layer, x.cache_cap, x.window = k, v, layer, cap, window
+    x.n_kv_heads, x.head_dim, x.rope_frac, x.rope_theta, x.shared_from = hkv, d, frac, theta, -1
+    return x
+
+
+def test_share_bind_aliases_and_resolves_chains():
+    src = _desc(5, 0, 4096)
+    dst = _desc(11, 0, 4096, k=None, v=None)
+    native.gemma_kv_share_bind(dst, src)
+    assert dst.k_cache == src.k_cache and dst.v_cache == src.v_cache and dst.shared_from == 5
+    dst2 = _desc(13, 0, 4096, k=None, v=None)
+    native.gemma_kv_share_bind(dst2, dst)           # chain resolves to the root
+    assert dst2.shared_from == 5 and dst2.k_cache == src.k_cache
+
+
+@pytest.mark.parametrize("change", ["type", "window", "heads", "dim", "frac", "theta", "order", "cap"])
+def test_share_bind_rejects_mismatch(change):
+    src = _desc(3, 1024, 1024, hkv=16, d=256, frac=1.0, theta=1e4)
+    kw = dict(layer=4, window=1024, cap=1024, hkv=16, d=256, frac=1.0, theta=1e4, k=None, v=None)
+    if change == "type":
+        kw.update(window=0, cap=4096)
+    elif change == "window":
+        kw.update(window=512, cap=512)
+    elif change == "heads":
+        kw.update(hkv=8)
+    elif change == "dim":
+        kw.update(d=512)
+    elif change == "frac":
+        kw.update(frac=0.25)
+    elif change == "theta":
+        kw.update(theta=1e6)
+    elif change == "order":
+        kw.update(layer=2)
+    elif change == "cap":
+        kw.update(cap=2048)
+    dst = _desc(**kw)
+    with pytest.raises(native.GemmaError) as e:
+        native.gemma_kv_share_bind(dst, src)
+    assert e.value.code == native.GEMMA_ERR_SHARE_MISMATCH
+    assert not dst.k_cache and dst.shared_from == -1  # unchanged
+
+
+def _prefill_raw(**over):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, kc=FAKE, vc=FAKE, cap=512, lens=None, B=1, S=16, W=512,
+             Hq=8, Hkv=4, D=256, frac=1.0, theta=1e4, scale=0.0625, out=FAKE, lse=None,
+             ws=FAKE, wsb=1 << 30, flags=0)
+    a.update(over)
+    return native._prefill(a["q"], a["k"], a["v"], a["kc"], a["vc"], a["cap"], a["lens"], a["B"],
+                           a["S"], a["W"], a["Hq"], a["Hkv"], a["D"], a["frac"], a["theta"],
+                           a["scale"], a["out"], a["lse"], a["ws"], a["wsb"], a["flags"], None)
+
+
+def _decode_raw(**over):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, kc=FAKE, vc=FAKE, cap=4096, lens=FAKE, maxlen=4096, B=2, W=0,
+             Hq=32, Hkv=4, D=512, frac=0.25, theta=1e6, scale=0.044, out=FAKE, ws=FAKE,
+             wsb=1 << 30, flags=0)
+    a.update(over)
+    return native._decode(a["q"], a["k"], a["v"], a["kc"], a["vc"], a["cap"], a["lens"], a["maxlen"],
+                          a["B"], a["W"], a["Hq"], a["Hkv"], a["D"], a["frac"], a["theta"],
+                          a["scale"], a["out"], a["ws"], a["wsb"], a["flags"], None)
+
+
+E = native
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(Hq=6), E.GEMMA_ERR_INVALID_ARG),            # Hq not a multiple of Hkv
+    (dict(Hq=64, Hkv=4), E.GEMMA_ERR_UNSUPPORTED),   # 16 q heads per KV head
+    (dict(D=128), E.GEMMA_ERR_UNSUPPORTED),
+    (dict(frac=1.5), E.GEMMA_ERR_INVALID_ARG),
+    (dict(frac=-0.1), E.GEMMA_ERR_INVALID_ARG),
+    (dict(theta=0.0), E.GEMMA_ERR_INVALID_ARG),
+    (dict(W=500, cap=500), E.GEMMA_ERR_INVALID_ARG),  # window not a multiple of 16
+    (dict(cap=1024), E.GEMMA_ERR_INVALID_ARG),        # local ring must hold exactly the window
+    (dict(lens=FAKE), E.GEMMA_ERR_UNSUPPORTED),        # chunked local prefill
+    (dict(W=0, cap=8), E.GEMMA_ERR_CAPACITY),          # global cache shorter than the chunk
+    (dict(k=None), E.GEMMA_ERR_INVALID_ARG),           # unshared layer without new keys
+    (dict(flags=1), E.GEMMA_ERR_INVALID_ARG),          # shared layer with new keys
+    (dict(flags=4), E.GEMMA_ERR_INVALID_ARG),
+    (dict(q=None), E.GEMMA_ERR_INVALID_ARG),
+    (dict(q=FAKE + 8), E.GEMMA_ERR_INVALID_ARG),       # misaligned
+    (dict(wsb=16), E.GEMMA_ERR_CAPACITY),
+    (dict(B=0), E.GEMMA_ERR_INVALID_ARG),
+])
+def test_prefill_validation(over, code):
+    assert _prefill_raw(**over) == code
+    assert native.gemma_last_error()
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(lens=None), E.GEMMA_ERR_INVALID_ARG),
+    (dict(maxlen=0), E.GEMMA_ERR_INVALID_ARG),
+    (dict(cap=1000), E.GEMMA_ERR_CAPACITY),            # global cache < max length
+    (dict(W=1024, cap=4096), E.GEMMA_ERR_INVALID_ARG),
+    (dict(D=384), E.GEMMA_ERR_UNSUPPORTED),
+    (dict(k=None, v=None, flags=0), E.GEMMA_ERR_INVALID_ARG),
+    (dict(wsb=1024), E.GEMMA_ERR_CAPACITY),
+    (dict(out=None), E.GEMMA_ERR_INVALID_ARG),
+])
+def test_decode_validation(over, code):
+    assert _decode_raw(**over) == code
+
+
+def test_workspace_sizes_cover_the_configs():
+    assert native.gemma_attn_prefill_workspace_size(1, 8192, 8, 4, 256, 512) >= 8192 * 8 * 256 * 2 + 8192 * 4 * 256 * 2
+    assert native.gemma_attn_prefill_workspace_size(1, 8192, 8, 1, 512, 0) >= 8192 * 8 * 512 * 2
+    n = native.gemma_attn_decode_workspace_size(64, 32, 4, 512, 0, 131072)
+    assert n >= 64 * 32 * 512 * 2
+    assert native.gemma_attn_decode_workspace_size(0, 32, 4, 512, 0, 131072) == 0

@@ -1,0 +1,245 @@
+"""GPU parity of the prefill path (RoPE + cache write + attention) against the
+fp64 oracle, through the C ABI. Small cases compare every row; the
+full-size workloads compare sampled rows (every attention row is
+independent, so sampled rows are exact)."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from hybrid_local_global_b200 import native, synth
+from hybrid_local_global_b200.stack import AttentionStack
+from hybrid_local_global_b200.workloads import WORKLOADS
+
+from gpu_util import assert_close, gather_rows, sample_rows, to_bits
+
+pytestmark = pytest.mark.gpu
+
+
+def _expected_rotated_bf16(oracle, k_bits_row, pos, frac, theta):
+    y = oracle.rope_bf16(k_bits_row, pos, frac, theta)
+    return torch.from_numpy(y).to(torch.bfloat16)
+
+
+def run_prefill_case(oracle, *, B, S, Hq, Hkv, D, W, frac, theta, seed, prior=None, q_scale=1.0,
+                     k_scale=1.0, tol=(2e-2, 2e-3), check_cache=True, check_lse=True):
+    dev = torch.device("cuda")
+    g = synth.generator(seed)
+    q = synth.randn_bf16((B, S, Hq, D), g, scale=q_scale)
+    k = synth.randn_bf16((B, S, Hkv, D), g, scale=k_scale)
+    v = synth.randn_bf16((B, S, Hkv, D), g)
+    prior = list(prior) if prior else [0] * B
+    T = max(prior) + S
+    cap = W if W else T + 16
+    kc = torch.zeros((B, Hkv, cap, D), dtype=torch.bfloat16)
+    vc = torch.zeros((B, Hkv, cap, D), dtype=torch.bfloat16)
+    for b in range(B):
+        if prior[b]:
+            kc[b, :, :prior[b]] = synth.randn_bf16((Hkv, prior[b], D), g)
+            vc[b, :, :prior[b]] = synth.randn_bf16((Hkv, prior[b], D), g)
+    kc0, vc0 = kc.clone(), vc.clone()
+    qd, kd, vd, kcd, vcd = (x.to(dev) for x in (q, k, v, kc, vc))
+    out = torch.full((B, S, Hq, D), float("nan"), dtype=torch.bfloat16, device=dev)
+    lse = torch.full((B, Hq, S), float("nan"), dtype=torch.float32, device=dev)
+    lens = torch.tensor(prior, dtype=torch.int32, device=dev) if any(prior) else None
+    scale = 1.0 / math.sqrt(D)
+    native.gemma_attn_prefill(qd, kd, vd, kcd, vcd, window=W, rope_frac=frac, rope_theta=theta,
+                              scale=scale, out=out, seq_lens_before=lens, lse=lse)
+    assert native.gemma_attn_sync_status() == 0, native.gemma_last_error()
+
+    # oracle on logical K/V: cached prefix (already rotated) + the new keys
+    k_log = torch.zeros((B, T, Hkv, D), dtype=torch.bfloat16)
+    v_log = torch.zeros((B, T, Hkv, D), dtype=torch.bfloat16)
+    for b in range(B):
+        k_log[b, :prior[b]] = kc0[b, :, :prior[b]].transpose(0, 1)
+        v_log[b, :prior[b]] = vc0[b, :, :prior[b]].transpose(0, 1)
+        k_log[b, prior[b]:prior[b] + S] = k[b]
+        v_log[b, prior[b]:prior[b] + S] = v[b]
+    ref, ref_lse = oracle.attention(to_bits(q), to_bits(k_log), to_bits(v_log), q_pos0=prior,
+                                    n_keys=[p + S for p in prior], rot_from=prior, window=W,
+                                    rope_frac=frac, theta=theta, scale=scale)
+    got = out.float().cpu().double().numpy().transpose(0, 2, 1, 3).reshape(-1, D)  # (b, h, i) rows
+    assert_close(got, ref, *tol, what="prefill out")
+    if check_lse:
+        gl = lse.cpu().double().numpy().reshape(-1)
+        assert np.abs(gl - ref_lse).max() < 2e-2 * max(1.0, q_scale)
+
+    if check_cache:
+        kc1, vc1 = kcd.cpu(), vcd.cpu()
+        for b in range(B):
+            for s in range(S):
+                pos = prior[b] + s
+                if W and s < S - W:
+                    continue
+                slot = pos % W if W else pos
+                assert torch.equal(vc1[b, :, slot], v[b, s]), "V slot %d" % slot
+                for h in range(Hkv):
+                    exp = _expected_rotated_bf16(oracle, to_bits(k[b, s, h]), pos, frac, theta)
+                    got_k = kc1[b, h, slot]
+                    if frac == 0.0:
+                        assert torch.equal(got_k, k[b, s, h])
+                    else:
+                        d = (got_k.float() - exp.float()).abs()
+                        assert (d <= exp.float().abs() * 2 ** -8 + 1e-30).all(), "K slot %d" % slot
+        if W == 0:
+            # untouched slots keep their bytes
+            for b in range(B):
+                assert torch.equal(kc1[b, :, :prior[b]], kc0[b, :, :prior[b]])
+                assert torch.equal(kc1[b, :, prior[b] + S:], kc0[b, :, prior[b] + S:])
+    return out
+
+
+CASES = [
+    dict(B=2, S=1, Hq=8, Hkv=4, D=256, W=512, frac=1.0, theta=1e4, seed=101),
+    dict(B=2, S=200, Hq=4, Hkv=2, D=256, W=48, frac=1.0, theta=1e4, seed=102),
+    dict(B=1, S=300, Hq=8, Hkv=1, D=512, W=0, frac=0.25, theta=1e6, seed=103),
+    dict(B=2, S=130, Hq=2, Hkv=2, D=256, W=0, frac=0.25, theta=1e6, seed=104),
+    dict(B=1, S=257, Hq=8, Hkv=4, D=512, W=64, frac=1.0, theta=1e4, seed=105),
+    dict(B=1, S=96, Hq=4, Hkv=4, D=256, W=16, frac=0.0, theta=1e4, seed=106),
+    dict(B=2, S=100, Hq=8, Hkv=1, D=512, W=0, frac=0.25, theta=1e6, seed=107, prior=[37, 250]),
+    dict(B=1, S=64, Hq=16, Hkv=2, D=256, W=0, frac=1.0, theta=1e4, seed=108, prior=[1000]),
+]
+
+
+@pytest.mark.parametrize("case", CASES, ids=lambda c: "B%dS%dH%d-%dD%dW%d%s" % (
+    c["B"], c["S"], c["Hq"], c["Hkv"], c["D"], c["W"], "P" if c.get("prior") else ""))
+def test_prefill_small(oracle, case):
+    run_prefill_case(oracle, **case)
+
+
+def test_prefill_local_s1024_full(oracle):
+    """Single local layer, B1 S1024 W512 Hq8 Hkv4 D256, full RoPE 1e4, every row."""
+    run_prefill_case(oracle, B=1, S=1024, Hq=8, Hkv=4, D=256, W=512, frac=1.0, theta=1e4, seed=0)
+
+
+@pytest.mark.parametrize("D,W,Hkv,frac,theta", [(256, 512, 4, 1.0, 1e4), (512, 0, 1, 0.25, 1e6)])
+def test_prefill_peaky(oracle, D, W, Hkv, frac, theta):
+    """Queries x8: near one-hot attention, so a wrong mask boundary or a
+    missing key cannot hide behind near-uniform weights. The logits grow 8x,
+    and so does the effect of rounding the rotated q and k to bf16; the
+    tolerance scales with it (see the design notes)."""
+    run_prefill_case(oracle, B=1, S=640, Hq=8, Hkv=Hkv, D=D, W=W, frac=frac, theta=theta, seed=7,
+                     q_scale=8.0, tol=(1e-1, 4e-3), check_cache=False)
+
+
+def test_visible_ranges_bit_exact(oracle):
+    dev = torch.device("cuda")
+    for B, S, W, prior in ((1, 1024, 512, None), (2, 333, 48, None), (2, 100, 0, [0, 4095]),
+                           (1, 4096, 1024, None), (1, 37, 16, None)):
+        r = torch.full((B, S, 3), -7, dtype=torch.int32, device=dev)
+        lens = torch.tensor(prior, dtype=torch.int32, device=dev) if prior else None
+        native.gemma_attn_visible_ranges(B, S, W, r, seq_lens_before=lens)
+        assert native.gemma_attn_sync_status() == 0
+        r = r.cpu().numpy()
+        for b in range(B):
+            p0 = prior[b] if prior else 0
+            for i in range(S):
+                lo, hi, cnt = oracle.visible_range(p0 + i, W, p0 + S)
+                assert tuple(r[b, i]) == (lo, hi, cnt), (b, i)
+
+
+def test_lse_counts_with_zero_queries(oracle):
+    """Q = 0: every visible key weighs the same, so exp(lse) is the visible
+    count; checks the kernel's per-row key set exactly."""
+    dev = torch.device("cuda")
+    for D, W, S, Hkv in ((256, 48, 300, 2), (512, 0, 257, 1)):
+        B, Hq = 1, 8
+        q = torch.zeros((B, S, Hq, D), dtype=torch.bfloat16, device=dev)
+        g = synth.generator(5, "cuda")
+        k = synth.randn_bf16((B, S, Hkv, D), g, "cuda")
+        v = synth.randn_bf16((B, S, Hkv, D), g, "cuda")
+        cap = W if W else S
+        kc = torch.zeros((B, Hkv, cap, D), dtype=torch.bfloat16, device=dev)
+        vc = torch.zeros_like(kc)
+        out = torch.empty((B, S, Hq, D), dtype=torch.bfloat16, device=dev)
+        lse = torch.empty((B, Hq, S), dtype=torch.float32, device=dev)
+        native.gemma_attn_prefill(q, k, v, kc, vc, window=W, rope_frac=1.0, rope_theta=1e4,
+                                  scale=0.1, out=out, lse=lse)
+        assert native.gemma_attn_sync_status() == 0
+        cnt = torch.exp(lse.double()).cpu().numpy()
+        for i in range(S):
+            want = oracle.visible_range(i, W, S)[2]
+            assert np.all(np.rint(cnt[0, :, i]) == want) and np.abs(cnt[0, :, i] - want).max() < 1e-3 * want
+
+
+def test_shared_global_layer_reads_source_and_writes_nothing(oracle):
+    """A shared layer (GEMMA_F_SHARED, no k/v) attends over its source's cache
+    and leaves every cache byte as it was."""
+    dev = torch.device("cuda")
+    B, S, Hq, Hkv, D = 1, 200, 8, 1, 512
+    g = synth.generator(9)
+    q0 = synth.randn_bf16((B, S, Hq, D), g)
+    q1 = synth.randn_bf16((B, S, Hq, D), g)
+    k = synth.randn_bf16((B, S, Hkv, D), g)
+    v = synth.randn_bf16((B, S, Hkv, D), g)
+    kc = torch.zeros((B, Hkv, S, D), dtype=torch.bfloat16, device=dev)
+    vc = torch.zeros_like(kc)
+    out0 = torch.empty((B, S, Hq, D), dtype=torch.bfloat16, device=dev)
+    out1 = torch.empty_like(out0)
+    kw = dict(window=0, rope_frac=0.25, rope_theta=1e6, scale=1 / math.sqrt(D))
+    native.gemma_attn_prefill(q0.to(dev), k.to(dev), v.to(dev), kc, vc, out=out0, **kw)
+    assert native.gemma_attn_sync_status() == 0
+    before = (kc.clone(), vc.clone())
+    native.gemma_attn_prefill(q1.to(dev), None, None, kc, vc, out=out1, flags=native.GEMMA_F_SHARED, **kw)
+    assert native.gemma_attn_sync_status() == 0
+    assert torch.equal(kc, before[0]) and torch.equal(vc, before[1])
+    ref, _ = oracle.attention(to_bits(q1), to_bits(k), to_bits(v), q_pos0=0, n_keys=S, rot_from=0,
+                              window=0, rope_frac=0.25, theta=1e6, scale=1 / math.sqrt(D))
+    got = out1.float().cpu().double().numpy().transpose(0, 2, 1, 3).reshape(-1, D)
+    assert_close(got, ref, what="shared layer")
+
+
+# --------------------------------------------------------------------------- full-size workloads
+def _run_block(oracle, name, n_random=256):
+    w = WORKLOADS[name]
+    dev = torch.device("cuda")
+    st = AttentionStack(w, dev)
+    g = synth.generator(w.seed, "cuda")
+    ws = torch.empty(st.prefill_workspace_bytes(), dtype=torch.uint8, device=dev)
+    lens = None
+    if w.prior:
+        lens = torch.full((w.batch,), w.prior, dtype=torch.int32, device=dev)
+    results = []
+    for l in range(st.n_layers):
+        t = st.layer_type(l)
+        q = synth.randn_bf16((w.batch, w.seq, w.n_q_heads, t.head_dim), g, "cuda")
+        k = synth.randn_bf16((w.batch, w.seq, t.n_kv_heads, t.head_dim), g, "cuda", scale=w.k_scale)
+        v = synth.randn_bf16((w.batch, w.seq, t.n_kv_heads, t.head_dim), g, "cuda")
+        prior_k = prior_v = None
+        if w.prior:
+            # cached context before the chunk: already-rotated keys
+            synth.fill_randn_bf16_(st.k_cache[l][:, :, :w.prior], g)
+            synth.fill_randn_bf16_(st.v_cache[l][:, :, :w.prior], g)
+            prior_k = st.k_cache[l][:, :, :w.prior].clone()
+            prior_v = st.v_cache[l][:, :, :w.prior].clone()
+        out = torch.empty((w.batch, w.seq, w.n_q_heads, t.head_dim), dtype=torch.bfloat16, device=dev)
+        st.prefill_layer(l, q, k, v, out, workspace=ws, seq_lens_before=lens)
+        assert native.gemma_attn_sync_status() == 0, native.gemma_last_error()
+        rows = sample_rows(w.batch, w.n_q_heads, w.seq, n_random, seed=1000 + l, window=t.window,
+                           prior=w.prior)
+        if w.prior:
+            k_log = torch.cat([prior_k.transpose(1, 2), k], dim=1)
+            v_log = torch.cat([prior_v.transpose(1, 2), v], dim=1)
+            del prior_k, prior_v
+        else:
+            k_log, v_log = k, v
+        ref, _ = oracle.attention(to_bits(q), to_bits(k_log), to_bits(v_log), q_pos0=w.prior,
+                                  n_keys=w.prior + w.seq, rot_from=w.prior, window=t.window,
+                                  rope_frac=t.rope_frac, theta=t.rope_theta, scale=t.scale, rows=rows)
+        got = gather_rows(out, rows)
+        results.append(assert_close(got, ref, what="%s layer %d" % (name, l)))
+        del q, k, v, out, k_log, v_log
+    return results
+
+
+def test_prefill_e2b_block_s8192(oracle):
+    _run_block(oracle, "e2b_block_s8192")
+
+
+def test_prefill_31b_block_s32768(oracle):
+    _run_block(oracle, "31b_block_s32768", n_random=128)
+
+
+def test_prefill_global_chunk_256k(oracle):
+    _run_block(oracle, "global_chunk_256k", n_random=48)
