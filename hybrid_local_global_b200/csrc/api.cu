@@ -5,6 +5,7 @@
 #include <atomic>
 #include <cmath>
 #include <cstdarg>
+#include <cstddef>
 #include <cstdio>
 #include <mutex>
 #include <string>
@@ -34,7 +35,7 @@ int succeed() {
   return GEMMA_OK;
 }
 
-__device__ int g_status;  // first device-side failure since the last sync_status
+__device__ DevStatus g_dev;  // device status block (see common.cuh)
 
 std::mutex g_mu;
 int* g_status_ptr[128] = {nullptr};
@@ -55,8 +56,8 @@ int* status_ptr() {
   std::lock_guard<std::mutex> lk(g_mu);
   if (!g_status_ptr[dev]) {
     void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_status) != cudaSuccess) return nullptr;
-    g_status_ptr[dev] = static_cast<int*>(p);
+    if (cudaGetSymbolAddress(&p, g_dev) != cudaSuccess) return nullptr;
+    g_status_ptr[dev] = &static_cast<DevStatus*>(p)->status;
   }
   return g_status_ptr[dev];
 }
@@ -322,8 +323,13 @@ int gemma_attn_prefill(const void* q, const void* k_new, const void* v_new, void
   aa.out = static_cast<bf16*>(out);
   aa.lse = lse;
   aa.status = status;
+  aa.wait_ns = (unsigned long long)g_wait_ns.load();
+  const bool cache_view = (window == 0 || shared);
   ProfScope p_attn(GEMMA_KERNEL_PREFILL_ATTN, st);
-  e = launch_prefill_attn(aa, batch, head_dim, st);
+  if (head_dim == 256)
+    e = launch_prefill_attn_tc(aa, batch, head_dim, cache_view ? cache_cap : s_new, cache_view ? 0 : 1, st);
+  else
+    e = launch_prefill_attn(aa, batch, head_dim, st);
   p_attn.done();
   if (e != cudaSuccess) return cuda_fail(e, "prefill attention launch");
   return succeed();
@@ -439,6 +445,20 @@ int gemma_attn_visible_ranges(const int32_t* seq_lens_before, int batch, int s_n
   return succeed();
 }
 
+int gemma_attn_debug_timeout_info(long long* info8) {
+  if (!info8) return fail(GEMMA_ERR_INVALID_ARG, "null output");
+  DevStatus d;
+  cudaError_t e = cudaMemcpyFromSymbol(&d, g_dev, sizeof d);
+  if (e != cudaSuccess) return cuda_fail(e, "read timeout info");
+  for (int i = 0; i < 8; ++i) info8[i] = (long long)d.info[i];
+  d.timeout_claim = 0;
+  for (int i = 0; i < 8; ++i) d.info[i] = 0;
+  e = cudaMemcpyToSymbol(g_dev, &d.timeout_claim, sizeof(DevStatus) - offsetof(DevStatus, timeout_claim),
+                         offsetof(DevStatus, timeout_claim));
+  if (e != cudaSuccess) return cuda_fail(e, "clear timeout info");
+  return succeed();
+}
+
 int gemma_attn_profile(int enable) {
   prof_clear();
   g_prof_on.store(enable != 0);
@@ -470,11 +490,11 @@ int gemma_attn_sync_status(void* stream) {
   cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "stream synchronize");
   int v = 0;
-  e = cudaMemcpyFromSymbol(&v, g_status, sizeof v);
+  e = cudaMemcpyFromSymbol(&v, g_dev, sizeof v);
   if (e != cudaSuccess) return cuda_fail(e, "read device status");
   if (v != 0) {
     const int zero = 0;
-    e = cudaMemcpyToSymbol(g_status, &zero, sizeof zero);
+    e = cudaMemcpyToSymbol(g_dev, &zero, sizeof zero);
     if (e != cudaSuccess) return cuda_fail(e, "clear device status");
     return fail(v, v == GEMMA_ERR_DEVICE_TIMEOUT ? "a bounded device wait gave up"
                                                  : "a device-side range check failed");

@@ -94,13 +94,40 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Device status block: one per device, owned by the library (api.cu). The
+// `int* status` every kernel receives points at its first member.
+struct DevStatus {
+  int status;                   // first failure code since the last sync_status
+  int timeout_claim;            // set by the first bounded wait that gave up
+  unsigned long long info[8];   // {1, where, a, b, c, barrier word, block id, parity}
+};
+
+__device__ __forceinline__ void record_timeout(int* status, uint64_t* bar, uint32_t parity, int where,
+                                               int a, int b, int c) {
+  if (!status) return;
+  DevStatus* d = reinterpret_cast<DevStatus*>(status);
+  if (atomicCAS(&d->timeout_claim, 0, 1) == 0) {
+    unsigned long long word;
+    asm volatile("ld.shared.b64 %0, [%1];" : "=l"(word) : "r"((uint32_t)__cvta_generic_to_shared(bar)));
+    d->info[0] = 1;
+    d->info[1] = (unsigned long long)(long long)where;
+    d->info[2] = (unsigned long long)(long long)a;
+    d->info[3] = (unsigned long long)(long long)b;
+    d->info[4] = (unsigned long long)(long long)c;
+    d->info[5] = word;
+    d->info[6] = (unsigned long long)blockIdx.x | ((unsigned long long)blockIdx.y << 20) |
+                 ((unsigned long long)blockIdx.z << 40);
+    d->info[7] = parity;
+  }
+}
+
 // Bounded wait: polls until the phase with `parity` completes, until another
 // thread of the CTA raised *abort, or until deadline_ns of %globaltimer has
 // passed; on the deadline it raises *abort and records TIMEOUT. Returns true
 // only when the phase completed.
-__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity,
-                                                  volatile int* abort_flag,
-                                                  uint64_t deadline_ns, int* status) {
+__device__ __forceinline__ bool mbar_wait_bounded_at(uint64_t* bar, uint32_t parity,
+                                                     volatile int* abort_flag, uint64_t deadline_ns,
+                                                     int* status, int where, int a, int b, int c) {
   uint32_t it = 0;
   while (!mbar_try_wait(bar, parity)) {
     if ((++it & 15u) == 0) {
@@ -108,11 +135,18 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
       if (globaltimer_ns() > deadline_ns) {
         *abort_flag = 1;
         set_status(status, GEMMA_ERR_DEVICE_TIMEOUT);
+        record_timeout(status, bar, parity, where, a, b, c);
         return false;
       }
     }
   }
   return true;
+}
+
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity,
+                                                  volatile int* abort_flag,
+                                                  uint64_t deadline_ns, int* status) {
+  return mbar_wait_bounded_at(bar, parity, abort_flag, deadline_ns, status, -1, 0, 0, 0);
 }
 
 // 1-D bulk copy global -> shared, completion signalled as tx bytes on `bar`.

@@ -12,16 +12,20 @@
 // The step is HBM-bound: every cached K/V byte is read once per KV head and
 // shared by its G query heads. Work unit = (split of `chunk` keys, KV head,
 // sequence). Per CTA:
-//   warp 4      producer: for each 16-key sub-block, one lane arms the slot's
+//   warp 3      producer: for each 16-key sub-block, one lane arms the slot's
 //               full barrier with the byte count and 32 lanes issue one bulk
 //               copy per K/V row into a ring of padded shared-memory rows
 //               (row stride D*2+16 bytes keeps ldmatrix conflict-free).
-//   warps 0..3  consumers: sub-block t goes to warp t % 4. S = Q K^T with
+//   warps 0..2  consumers: sub-block t goes to warp t % 3 and ring slot
+//               t % NSLOT, with NSLOT a multiple of 3, so every slot has a
+//               single consumer that waits its phases strictly in order
+//               (two waiters on consecutive phases of one mbarrier would
+//               alias under parity waits). S = Q K^T with
 //               mma.sync m16n8k16 (A = the G query heads padded to 16 rows,
 //               B = K rows), online softmax in fp32 (log2 domain), then
 //               O^T += V^T P^T with the S accumulators reused directly as the
 //               B fragment of P^T (the GQA group is the MMA's N dimension).
-// The four warps' (m, l, O) merge in shared memory; each split writes its
+// The consumer warps' (m, l, O) merge in shared memory; each split writes its
 // normalised partial and its log2-sum-exp, and the combine kernel merges the
 // splits of a (sequence, head).
 //
@@ -35,6 +39,8 @@ namespace hlg {
 
 namespace {
 
+constexpr int NCW = 3;  // consumer warps
+
 template <int D>
 struct DecCfg {
   static constexpr int KB = 16;                 // keys per sub-block
@@ -42,10 +48,11 @@ struct DecCfg {
   static constexpr int ROWB = ROW * 2;          // bytes
   static constexpr int SLOT_B = 2 * KB * ROWB;  // K rows then V rows
   static constexpr int NSLOT = (D == 256) ? 6 : 3;
+  static_assert(NSLOT % NCW == 0, "each ring slot needs a single consumer warp");
   static constexpr int RING_B = NSLOT * SLOT_B;
   static constexpr int Q_B = 8 * ROWB;
   static constexpr int OSTR = D + 4;            // merge-buffer row (floats)
-  static constexpr int MERGE_B = 4 * 8 * OSTR * 4;
+  static constexpr int MERGE_B = NCW * 8 * OSTR * 4;
   static_assert(MERGE_B <= RING_B, "merge buffer must fit in the ring");
   static constexpr int BAR_OFF = RING_B + Q_B;
   static constexpr int MISC_OFF = BAR_OFF + 2 * NSLOT * 8;
@@ -83,7 +90,7 @@ __device__ __forceinline__ void named_bar_sync(int id, int n) {
 }
 
 template <int D>
-__global__ void __launch_bounds__(160, 2) k_decode_split(DecodeAttnArgs a) {
+__global__ void __launch_bounds__(32 * (NCW + 1), 2) k_decode_split(DecodeAttnArgs a) {
   using C = DecCfg<D>;
   extern __shared__ __align__(128) unsigned char sm[];
   unsigned char* ring = sm;
@@ -94,8 +101,8 @@ __global__ void __launch_bounds__(160, 2) k_decode_split(DecodeAttnArgs a) {
   volatile int* abort_flag = misc;
   int* issued = misc + 1;
   int* consumed = issued + C::NSLOT;
-  float* m_w = reinterpret_cast<float*>(consumed + C::NSLOT);  // [4][8]
-  float* l_w = m_w + 32;                                         // [4][8]
+  float* m_w = reinterpret_cast<float*>(consumed + C::NSLOT);  // [NCW][8]
+  float* l_w = m_w + 32;                                         // [NCW][8]
 
   const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -131,18 +138,19 @@ __global__ void __launch_bounds__(160, 2) k_decode_split(DecodeAttnArgs a) {
       v = *reinterpret_cast<const uint4*>(a.q_rot + ((int64_t)b * a.Hq + g * G + r) * D + c);
     *reinterpret_cast<uint4*>(qs + r * C::ROW + c) = v;
   }
+  __syncwarp();
   __syncthreads();
   const uint64_t deadline = globaltimer_ns() + a.wait_ns;
 
-  if (warp == 4) {
+  if (warp == NCW) {
     // ---------------- producer ----------------
     for (int t = 0; t < n_sub; ++t) {
       const int slot = t % C::NSLOT;
       bool ok = true;
       if (lane == 0) {
         if (t >= C::NSLOT)
-          ok = mbar_wait_bounded(&empty[slot], ((t / C::NSLOT) - 1) & 1, abort_flag, deadline,
-                                 a.status);
+          ok = mbar_wait_bounded_at(&empty[slot], ((t / C::NSLOT) - 1) & 1, abort_flag, deadline,
+                                    a.status, 1, t, slot, n_sub);
         if (ok && *abort_flag) ok = false;
       }
       ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -173,10 +181,10 @@ __global__ void __launch_bounds__(160, 2) k_decode_split(DecodeAttnArgs a) {
     const uint32_t q_addr = smem_u32(qs) + ((lane & 7) * C::ROW + ((lane >> 3) & 1) * 8) * 2;
     const uint32_t frag_off = (((lane >> 4) * 8 + (lane & 7)) * C::ROW + ((lane >> 3) & 1) * 8) * 2;
 
-    for (int t = warp; t < n_sub; t += 4) {
+    for (int t = warp; t < n_sub; t += NCW) {
       const int slot = t % C::NSLOT;
-      const bool ok = mbar_wait_bounded(&full[slot], (t / C::NSLOT) & 1, abort_flag, deadline,
-                                        a.status);
+      const bool ok = mbar_wait_bounded_at(&full[slot], (t / C::NSLOT) & 1, abort_flag, deadline,
+                                           a.status, 2, t, slot, warp);
       if (!__all_sync(0xffffffffu, ok)) break;
       const int64_t key0 = k_begin + (int64_t)t * C::KB;
       const int nk = (int)((k_end - key0) < C::KB ? (k_end - key0) : C::KB);
@@ -253,6 +261,7 @@ __global__ void __launch_bounds__(160, 2) k_decode_split(DecodeAttnArgs a) {
       m_w[warp * 8 + gq] = m_h;
       l_w[warp * 8 + gq] = l_q;
     }
+    __syncwarp();
     __syncthreads();  // (A) pairs with the producer's (A)
     if (*abort_flag) return;
     // scale this warp's O into the merge buffer (overlays the drained ring)
@@ -263,7 +272,7 @@ __global__ void __launch_bounds__(160, 2) k_decode_split(DecodeAttnArgs a) {
       const int hh = 2 * tg + j;
       float M = -INFINITY;
 #pragma unroll
-      for (int w = 0; w < 4; ++w) M = fmaxf(M, m_w[w * 8 + hh]);
+      for (int w = 0; w < NCW; ++w) M = fmaxf(M, m_w[w * 8 + hh]);
       const float mw = m_w[warp * 8 + hh];
       f[j] = (mw == -INFINITY) ? 0.f : exp2f(mw - M);
     }
@@ -276,15 +285,16 @@ __global__ void __launch_bounds__(160, 2) k_decode_split(DecodeAttnArgs a) {
       row0[8] = o[mt][2] * f[0];
       row1[8] = o[mt][3] * f[1];
     }
-    named_bar_sync(1, 128);
-    for (int idx = threadIdx.x; idx < G * D; idx += 128) {
+    __syncwarp();
+    named_bar_sync(1, 32 * NCW);
+    for (int idx = threadIdx.x; idx < G * D; idx += 32 * NCW) {
       const int hh = idx / D, d = idx % D;
       float M = -INFINITY;
 #pragma unroll
-      for (int w = 0; w < 4; ++w) M = fmaxf(M, m_w[w * 8 + hh]);
+      for (int w = 0; w < NCW; ++w) M = fmaxf(M, m_w[w * 8 + hh]);
       float L = 0.f, acc = 0.f;
 #pragma unroll
-      for (int w = 0; w < 4; ++w) {
+      for (int w = 0; w < NCW; ++w) {
         const float mw = m_w[w * 8 + hh];
         L += (mw == -INFINITY) ? 0.f : l_w[w * 8 + hh] * exp2f(mw - M);
         acc += obuf[(w * 8 + hh) * C::OSTR + d];
@@ -296,6 +306,7 @@ __global__ void __launch_bounds__(160, 2) k_decode_split(DecodeAttnArgs a) {
     return;
   }
   // producer reaches here
+  __syncwarp();
   __syncthreads();  // (A)
   if (*abort_flag && lane == 0) {
     // drain: wait (bounded) for copies that were issued but never consumed
@@ -303,7 +314,8 @@ __global__ void __launch_bounds__(160, 2) k_decode_split(DecodeAttnArgs a) {
     volatile int dummy = 0;
     for (int s = 0; s < C::NSLOT; ++s)
       if (issued[s] > consumed[s])
-        mbar_wait_bounded(&full[s], (issued[s] - 1) & 1, &dummy, dl, a.status);
+        mbar_wait_bounded_at(&full[s], (issued[s] - 1) & 1, &dummy, dl, a.status, 3, issued[s],
+                             s, consumed[s]);
   }
 }
 
@@ -346,11 +358,11 @@ cudaError_t launch_decode_split(const DecodeAttnArgs& a, int B, int D, cudaStrea
   if (D == 256) {
     using C = DecCfg<256>;
     cudaFuncSetAttribute(k_decode_split<256>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
-    k_decode_split<256><<<grid, 160, C::SMEM, st>>>(a);
+    k_decode_split<256><<<grid, 32 * (NCW + 1), C::SMEM, st>>>(a);
   } else {
     using C = DecCfg<512>;
     cudaFuncSetAttribute(k_decode_split<512>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
-    k_decode_split<512><<<grid, 160, C::SMEM, st>>>(a);
+    k_decode_split<512><<<grid, 32 * (NCW + 1), C::SMEM, st>>>(a);
   }
   return cudaGetLastError();
 }

@@ -59,6 +59,7 @@ struct PrefillAttnArgs {
   bf16* out;           // [B][S][Hq][D]
   float* lse;          // [B][Hq][S] or null
   int* status;
+  unsigned long long wait_ns;
 };
 
 struct DecodeAttnArgs {
@@ -82,6 +83,10 @@ struct DecodeAttnArgs {
 cudaError_t launch_prefill_rope(const PrefillRopeArgs& a, int B, int D, cudaStream_t st);
 cudaError_t launch_decode_rope_append(const DecodeRopeArgs& a, int B, int D, cudaStream_t st);
 cudaError_t launch_prefill_attn(const PrefillAttnArgs& a, int B, int D, cudaStream_t st);
+// tcgen05 prefill (head_dim 256). key_rows_total = rows of the K/V views;
+// kv_token_major: views are [B][rows][Hkv][D] (1) or [B][Hkv][rows][D] (0).
+cudaError_t launch_prefill_attn_tc(const PrefillAttnArgs& a, int B, int D, int key_rows_total,
+                                   int kv_token_major, cudaStream_t st);
 cudaError_t launch_decode_split(const DecodeAttnArgs& a, int B, int D, cudaStream_t st);
 cudaError_t launch_decode_combine(const DecodeAttnArgs& a, int B, int D, cudaStream_t st);
 cudaError_t launch_visible_ranges(const int32_t* seq_lens_before, int B, int S, int window,

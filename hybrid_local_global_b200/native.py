@@ -190,7 +190,15 @@ KERNEL_NAMES = {0: "prefill_rope", 1: "prefill_attn", 2: "decode_append", 3: "de
 _prof = _sig("gemma_attn_profile", _I, [_I])
 _prof_read = _sig("gemma_attn_profile_read", _I, [_I, ctypes.POINTER(ctypes.c_double),
                                                   ctypes.POINTER(ctypes.c_longlong)])
-EXPORTED += ["gemma_attn_profile", "gemma_attn_profile_read"]
+_tinfo = _sig("gemma_attn_debug_timeout_info", _I, [ctypes.POINTER(ctypes.c_longlong)])
+EXPORTED += ["gemma_attn_profile", "gemma_attn_profile_read", "gemma_attn_debug_timeout_info"]
+
+
+def gemma_attn_debug_timeout_info():
+    """-> list of 8 ints describing the first bounded wait that gave up (cleared on read)."""
+    buf = (ctypes.c_longlong * 8)()
+    _check(_tinfo(buf))
+    return [int(x) for x in buf]
 
 
 def gemma_attn_profile(enable: bool) -> int:

@@ -203,6 +203,13 @@ int gemma_attn_set_wait_limit(long long max_ns);
  * hangs. One-shot: the flag clears when that launch is issued. */
 int gemma_attn_debug_drop_next_copy(int enable);
 
+/* Diagnostics of the first bounded device wait that gave up since the last
+ * call: info8[0] = 1 if one did (0 otherwise), [1] = wait site, [2..4] =
+ * site-specific indices (work item, ring slot, stage), [5] = the raw
+ * 64-bit barrier word at give-up time, [6] = block index (x | y << 20 |
+ * z << 40), [7] = awaited phase parity. Reading clears the record. */
+int gemma_attn_debug_timeout_info(long long* info8);
+
 /* ---------------------------------------------------------------------- */
 /* Measurement hook. While enabled, every launch of the kernels below is   */
 /* bracketed by a pair of CUDA events recorded on the call's stream (event */
