@@ -449,8 +449,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-rows-local", type=int, default=256)
     ap.add_argument("--ref-rows-global", type=int, default=256)
-    ap.add_argument("--cpu-rows-local", type=int, default=2048)
-    ap.add_argument("--cpu-rows-global", type=int, default=4096)
+    ap.add_argument("--cpu-rows-local", type=int, default=16384)
+    ap.add_argument("--cpu-rows-global", type=int, default=49152)
     args = ap.parse_args()
 
     world, rank, local = dist_setup(args.gpus)

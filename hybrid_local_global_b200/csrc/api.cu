@@ -326,10 +326,7 @@ int gemma_attn_prefill(const void* q, const void* k_new, const void* v_new, void
   aa.wait_ns = (unsigned long long)g_wait_ns.load();
   const bool cache_view = (window == 0 || shared);
   ProfScope p_attn(GEMMA_KERNEL_PREFILL_ATTN, st);
-  if (head_dim == 256)
-    e = launch_prefill_attn_tc(aa, batch, head_dim, cache_view ? cache_cap : s_new, cache_view ? 0 : 1, st);
-  else
-    e = launch_prefill_attn(aa, batch, head_dim, st);
+  e = launch_prefill_attn_tc(aa, batch, head_dim, cache_view ? cache_cap : s_new, cache_view ? 0 : 1, st);
   p_attn.done();
   if (e != cudaSuccess) return cuda_fail(e, "prefill attention launch");
   return succeed();

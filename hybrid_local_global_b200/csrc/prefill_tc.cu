@@ -24,7 +24,9 @@
 //              write P_j (bf16) over S_j's columns, rescale O in TMEM only
 //              when the running max grows by more than 2^8; epilogue O / l.
 // TMEM columns: O 0..255 (fp32), S/P buffers 256..383 and 384..511.
-// The MMA pipe runs S_{j+1} while the softmax works on S_j, then P_j V_j.
+// The MMA pipe runs P_{j-1} V_{j-1} and S_{j+1} while the softmax works on
+// S_j; the softmax waits for P_{j-1} V_{j-1} only before rescaling O (rare)
+// and before releasing P_j, by which time it has normally completed.
 //
 // Tiles: key tiles [lo(first row), hi(last row)] only (window-aware
 // skipping); per-element masks only on tiles that cross a row's range.
@@ -65,7 +67,7 @@ struct Ctl {
   uint64_t empty[NSTAGE];
   uint64_t s_full[2];
   uint64_t p_ready;
-  uint64_t o_done;
+  uint64_t o_done[2];  // PV_i completes phase i/2 of o_done[i % 2]
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
@@ -146,7 +148,8 @@ __global__ void __launch_bounds__(192, 1)
     mbar_init(&ctl->s_full[0], 1);
     mbar_init(&ctl->s_full[1], 1);
     mbar_init(&ctl->p_ready, 128);
-    mbar_init(&ctl->o_done, 1);
+    mbar_init(&ctl->o_done[0], 1);
+    mbar_init(&ctl->o_done[1], 1);
     mbar_init(&ctl->drain, 1);
     ctl->abort = 0;
     ctl->q_issued = 0;
@@ -288,7 +291,7 @@ __global__ void __launch_bounds__(192, 1)
           __syncwarp();
         }
         if (!ok) break;
-        if (lane == 0) tc::commit(smem_u32(&ctl->o_done));
+        if (lane == 0) tc::commit(smem_u32(&ctl->o_done[(j - 1) & 1]));
       }
     }
     // make sure no MMA is in flight before TMEM can be released
@@ -308,13 +311,10 @@ __global__ void __launch_bounds__(192, 1)
     visible_range(pos0 + (row_valid ? q0 + row : a.S - 1), a.window, n_keys, &lo, &hi);
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
+    int pv_seen = 0;  // P.V products whose completion this thread has consumed
     for (int j = 0; j < n_tiles; ++j) {
       const int64_t kb = (kt0 + j) * BN;
       if (!wait_all(&ctl->s_full[j & 1], (j >> 1) & 1, abort_flag, deadline, a.status, 15, j)) {
-        ok = false;
-        break;
-      }
-      if (j >= 1 && !wait_all(&ctl->o_done, (j - 1) & 1, abort_flag, deadline, a.status, 16, j)) {
         ok = false;
         break;
       }
@@ -351,6 +351,15 @@ __global__ void __launch_bounds__(192, 1)
         m_used = m_new;
       }
       if (j >= 1 && __any_sync(0xffffffffu, need)) {
+        // O must be stable: wait for P_{j-1} V_{j-1}
+        if (pv_seen < j) {
+          if (!wait_all(&ctl->o_done[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag, deadline, a.status, 16, j)) {
+            ok = false;
+            break;
+          }
+          pv_seen = j;
+        }
+        tc::fence_after_sync();
 #pragma unroll 1
         for (int c = 0; c < 8; ++c) {
           uint32_t o[32];
@@ -377,11 +386,22 @@ __global__ void __launch_bounds__(192, 1)
       l += lsum;
       tc::tmem_st32(s_tm, pk[0]);
       tc::tmem_st32(s_tm + 32, pk[1]);
+      // consume P_{j-1} V_{j-1} before P_{j+1} V_{j+1} can complete the next
+      // phase of the same barrier (parity waits must not fall two behind)
+      if (j >= 1 && pv_seen < j) {
+        if (!wait_all(&ctl->o_done[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag, deadline, a.status, 16, j)) {
+          ok = false;
+          break;
+        }
+        pv_seen = j;
+      }
       tc::tmem_wait_st();
       tc::fence_before_sync();
       mbar_arrive(&ctl->p_ready);
     }
-    if (ok) ok = wait_all(&ctl->o_done, (n_tiles - 1) & 1, abort_flag, deadline, a.status, 17, n_tiles);
+    if (ok)
+      ok = wait_all(&ctl->o_done[(n_tiles - 1) & 1], ((n_tiles - 1) >> 1) & 1, abort_flag, deadline,
+                    a.status, 17, n_tiles);
     if (ok) {
       tc::fence_after_sync();
       const float inv = l > 0.f ? 1.f / l : 0.f;

@@ -56,3 +56,22 @@ def gather_rows(out: torch.Tensor, rows: np.ndarray) -> np.ndarray:
     idx_h = torch.as_tensor(rows[:, 1], device=out.device, dtype=torch.long)
     idx_i = torch.as_tensor(rows[:, 2], device=out.device, dtype=torch.long)
     return out[idx_b, idx_i, idx_h].float().cpu().double().numpy()
+
+
+def bf16_ulp(x: torch.Tensor) -> torch.Tensor:
+    """Spacing of bf16 numbers at |x| (8 significant bits)."""
+    a = x.float().abs().clamp_min(2.0 ** -126)
+    return torch.exp2(torch.floor(torch.log2(a)) - 7)
+
+
+def assert_rotated_bf16(got: torch.Tensor, exp: torch.Tensor, x: torch.Tensor, what=""):
+    """Rotated bf16 K against the bf16-rounded fp64 rotation. The kernel rounds
+    its fp32 rotation to nearest, the reference rounds the exact value, so the
+    two differ by at most one bf16 ulp where the values straddle a rounding
+    boundary; the fp32 rotation (x0*c - x1*s with c, s of an fp32-rounded
+    reduced angle) adds about 2^-22 * (|x0| + |x1|), bounded here by 2^-20."""
+    xf = x.float()
+    pair = xf.view(-1, 2).abs().sum(dim=1).repeat_interleave(2)
+    tol = bf16_ulp(exp) + 2 ** -20 * pair
+    d = (got.float() - exp.float()).abs()
+    assert bool((d <= tol).all()), "%s: max excess %.3e" % (what, float((d - tol).max()))

@@ -11,7 +11,7 @@ from hybrid_local_global_b200 import native, synth
 from hybrid_local_global_b200.stack import AttentionStack
 from hybrid_local_global_b200.workloads import WORKLOADS
 
-from gpu_util import assert_close, to_bits
+from gpu_util import assert_close, assert_rotated_bf16, to_bits
 
 pytestmark = pytest.mark.gpu
 
@@ -83,7 +83,7 @@ def run_decode_case(oracle, *, lens, Hq, Hkv, D, W, frac, theta, seed, q_scale=1
     kc1, vc1 = kcd.cpu(), vcd.cpu()
     for b in range(B):
         L = lens[b]
-        kl, vl = logical_kv(kc, vc, L, W, kn[b], vn[b])
+        kl, vl = logical_kv(kc[b], vc[b], L, W, kn[b], vn[b])
         ref, _ = oracle.attention(to_bits(q[b].reshape(1, 1, Hq, D)), to_bits(kl[None]), to_bits(vl[None]),
                                   q_pos0=L - 1, n_keys=L, rot_from=L if shared else L - 1, window=W,
                                   rope_frac=frac, theta=theta, scale=scale)
@@ -96,8 +96,7 @@ def run_decode_case(oracle, *, lens, Hq, Hkv, D, W, frac, theta, seed, q_scale=1
             assert torch.equal(vc1[b, :, slot], vn[b])
             for h in range(Hkv):
                 exp = torch.from_numpy(oracle.rope_bf16(to_bits(kn[b, h]), L - 1, frac, theta)).to(torch.bfloat16)
-                d = (kc1[b, h, slot].float() - exp.float()).abs()
-                assert (d <= exp.float().abs() * 2 ** -8 + 1e-30).all()
+                assert_rotated_bf16(kc1[b, h, slot], exp, kn[b, h], "new K slot")
             other = torch.ones(cap, dtype=torch.bool)
             other[slot] = False
             assert torch.equal(kc1[b][:, other], kc[b][:, other])
@@ -128,7 +127,7 @@ def test_decode_shared_layer(oracle):
 
 def test_decode_peaky(oracle):
     run_decode_case(oracle, lens=[5000, 700], Hq=8, Hkv=1, D=512, W=0, frac=0.25, theta=1e6, seed=209,
-                    q_scale=8.0, tol=(1e-1, 4e-3))
+                    q_scale=8.0, tol=(8 * 2e-2, 2 * 2e-3))
 
 
 def test_decode_range_check_reports_status():

@@ -12,7 +12,7 @@ from hybrid_local_global_b200 import native, synth
 from hybrid_local_global_b200.stack import AttentionStack
 from hybrid_local_global_b200.workloads import WORKLOADS
 
-from gpu_util import assert_close, gather_rows, sample_rows, to_bits
+from gpu_util import assert_close, assert_rotated_bf16, gather_rows, sample_rows, to_bits
 
 pytestmark = pytest.mark.gpu
 
@@ -67,6 +67,7 @@ def run_prefill_case(oracle, *, B, S, Hq, Hkv, D, W, frac, theta, seed, prior=No
 
     if check_cache:
         kc1, vc1 = kcd.cpu(), vcd.cpu()
+        n_same = n_all = 0
         for b in range(B):
             for s in range(S):
                 pos = prior[b] + s
@@ -80,8 +81,11 @@ def run_prefill_case(oracle, *, B, S, Hq, Hkv, D, W, frac, theta, seed, prior=No
                     if frac == 0.0:
                         assert torch.equal(got_k, k[b, s, h])
                     else:
-                        d = (got_k.float() - exp.float()).abs()
-                        assert (d <= exp.float().abs() * 2 ** -8 + 1e-30).all(), "K slot %d" % slot
+                        assert_rotated_bf16(got_k, exp, k[b, s, h], "K slot %d" % slot)
+                        n_same += int((got_k == exp).sum())
+                        n_all += exp.numel()
+        if n_all:
+            assert n_same >= 0.98 * n_all, "only %d of %d rotated K values bit-identical" % (n_same, n_all)
         if W == 0:
             # untouched slots keep their bytes
             for b in range(B):
@@ -116,11 +120,12 @@ def test_prefill_local_s1024_full(oracle):
 @pytest.mark.parametrize("D,W,Hkv,frac,theta", [(256, 512, 4, 1.0, 1e4), (512, 0, 1, 0.25, 1e6)])
 def test_prefill_peaky(oracle, D, W, Hkv, frac, theta):
     """Queries x8: near one-hot attention, so a wrong mask boundary or a
-    missing key cannot hide behind near-uniform weights. The logits grow 8x,
-    and so does the effect of rounding the rotated q and k to bf16; the
-    tolerance scales with it (see the design notes)."""
+    missing key cannot hide behind near-uniform weights (such a bug moves an
+    output by O(1)). The logits grow 8x and so does the logit error from
+    rounding the rotated q and k to bf16, so the max-abs bound is the
+    spec 2e-2 times the query scale and the mean-abs bound doubles."""
     run_prefill_case(oracle, B=1, S=640, Hq=8, Hkv=Hkv, D=D, W=W, frac=frac, theta=theta, seed=7,
-                     q_scale=8.0, tol=(1e-1, 4e-3), check_cache=False)
+                     q_scale=8.0, tol=(8 * 2e-2, 2 * 2e-3), check_cache=False)
 
 
 def test_visible_ranges_bit_exact(oracle):
