@@ -170,6 +170,12 @@ size_t prefill_ws_parts(int B, int S, int Hq, int Hkv, int D, int window, size_t
 
 }  // namespace
 
+namespace hlg {
+// Sets the message gemma_last_error() returns on this thread; for entry
+// points defined in other translation units of the library.
+int record_error(int code, const char* msg) { return fail(code, "%s", msg); }
+}  // namespace hlg
+
 extern "C" {
 
 const char* gemma_last_error(void) { return t_err.c_str(); }

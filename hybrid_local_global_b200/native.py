@@ -211,3 +211,27 @@ def gemma_attn_profile_read(kernel: int):
     n = ctypes.c_longlong()
     _check(_prof_read(kernel, ctypes.byref(ms), ctypes.byref(n)))
     return float(ms.value), int(n.value)
+
+
+_decode_noalloc = _sig("gemma_attn_decode_noalloc", _I, [_P, _P, _P, _P, _P, _I, _P, _I, _I, _I, _I, _I,
+                                                         _I, _F, _F, _F, _P, ctypes.c_uint, _P])
+EXPORTED += ["gemma_attn_decode_noalloc"]
+NOALLOC_SCRATCH_BYTES = 32 << 20
+
+
+def gemma_attn_decode_noalloc(q, k_new, v_new, k_cache, v_cache, *, seq_lens, max_seq_len, window,
+                              rope_frac, rope_theta, scale, out, flags=0, stream=None):
+    """gemma_attn_decode for callers that cannot allocate device memory: the
+    split-K scratch is the library's fixed 32 MiB array (shared by all calls;
+    overlapping calls race). Same arguments as gemma_attn_decode without the
+    workspace."""
+    for t, n in ((q, "q"), (k_new, "k_new"), (v_new, "v_new"), (k_cache, "k_cache"),
+                 (v_cache, "v_cache"), (out, "out")):
+        _bf16(t, n)
+    if seq_lens.dtype != torch.int32 or not seq_lens.is_cuda:
+        raise TypeError("seq_lens must be an int32 CUDA tensor")
+    B, Hq, D = q.shape
+    _, Hkv, cap, _ = k_cache.shape
+    return _check(_decode_noalloc(_ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_cache), _ptr(v_cache), cap,
+                                  _ptr(seq_lens), max_seq_len, B, window, Hq, Hkv, D, rope_frac,
+                                  rope_theta, scale, _ptr(out), flags, _stream(stream)))

@@ -139,6 +139,36 @@ int gemma_attn_decode(const void* q, const void* k_new, const void* v_new,
                       void* stream);
 
 /* ---------------------------------------------------------------------- */
+/* Decode without allocation. The pages have no counterpart for this entry */
+/* point; it exists for callers that cannot obtain device memory for the  */
+/* decode workspace -- e.g. a plugin inside a host runtime that owns all  */
+/* device memory and offers it no allocator, or a latency-critical loop   */
+/* where a cudaMalloc (and its implicit device-wide synchronisation) is   */
+/* not acceptable and no buffer was reserved in advance.                  */
+/*                                                                        */
+/* Same arguments and effect as gemma_attn_decode without the workspace:  */
+/* the split-K scratch comes from a fixed 32 MiB array compiled into the  */
+/* library, which every GPU that loads the library's device code holds    */
+/* until the process exits. The call allocates nothing (no cudaMalloc,    */
+/* no cudaFree, no allocating library routine).                           */
+/*   - A call whose gemma_attn_decode_workspace_size(...) exceeds 32 MiB   */
+/*     returns GEMMA_ERR_CAPACITY with a message and enqueues nothing.     */
+/*   - The first call on a device looks up the array's device address     */
+/*     (cudaGetSymbolAddress) with that device current; make that first   */
+/*     call before any stream capture.                                    */
+/*   - Every call shares the one array and nothing in it needs to start at */
+/*     zero (each call writes the scratch it reads). Calls that overlap on */
+/*     the GPU (other streams, other host threads) race on it: serialise   */
+/*     them.                                                              */
+/* ---------------------------------------------------------------------- */
+int gemma_attn_decode_noalloc(const void* q, const void* k_new, const void* v_new,
+                              void* k_cache, void* v_cache, int cache_cap,
+                              const int32_t* seq_lens, int max_seq_len, int batch,
+                              int window, int n_q_heads, int n_kv_heads, int head_dim,
+                              float rope_frac, float rope_theta, float scale, void* out,
+                              unsigned flags, void* stream);
+
+/* ---------------------------------------------------------------------- */
 /* KV sharing ("Gemma 4 Architecture Reference", "Shared KV Cache").       */
 /* Host only: no device work, no bytes move.                               */
 /* ---------------------------------------------------------------------- */
