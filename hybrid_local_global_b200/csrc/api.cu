@@ -297,6 +297,9 @@ int gemma_attn_prefill(const void* q, const void* k_new, const void* v_new, void
   ra.Hkv = n_kv_heads;
   ra.n_rot = rope_rotated_pairs(head_dim, rope_frac);
   ra.log2_theta = std::log2((double)rope_theta);
+  // queries carry scale * log2(e): the attention kernel's logits are then in
+  // log2 units (one bf16 rounding either way)
+  ra.q_scale = (float)((double)scale * 1.4426950408889634);
   ra.rows_per_cta = 4;
   ra.status = status;
   ProfScope p_rope(GEMMA_KERNEL_PREFILL_ROPE, st);
@@ -325,7 +328,7 @@ int gemma_attn_prefill(const void* q, const void* k_new, const void* v_new, void
   aa.window = window;
   aa.Hq = n_q_heads;
   aa.Hkv = n_kv_heads;
-  aa.scale_log2 = (float)((double)scale * 1.4426950408889634);
+  aa.scale_log2 = 1.0f;  // already applied to the rotated queries
   aa.out = static_cast<bf16*>(out);
   aa.lse = lse;
   aa.status = status;

@@ -22,6 +22,7 @@ struct PrefillRopeArgs {
   int S, window, Hq, Hkv;
   int n_rot;           // rotated pairs
   double log2_theta;
+  float q_scale;       // rotated Q is multiplied by this before the bf16 rounding
   int rows_per_cta;
   int* status;
 };
@@ -82,7 +83,6 @@ struct DecodeAttnArgs {
 
 cudaError_t launch_prefill_rope(const PrefillRopeArgs& a, int B, int D, cudaStream_t st);
 cudaError_t launch_decode_rope_append(const DecodeRopeArgs& a, int B, int D, cudaStream_t st);
-cudaError_t launch_prefill_attn(const PrefillAttnArgs& a, int B, int D, cudaStream_t st);
 // tcgen05 prefill (head_dim 256). key_rows_total = rows of the K/V views;
 // kv_token_major: views are [B][rows][Hkv][D] (1) or [B][Hkv][rows][D] (0).
 cudaError_t launch_prefill_attn_tc(const PrefillAttnArgs& a, int B, int D, int key_rows_total,

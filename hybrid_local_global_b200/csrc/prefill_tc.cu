@@ -324,21 +324,36 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
       for (int c = 0; c < 4; ++c) tc::tmem_ld32(s_tm + c * 32, r[c]);
       tc::tmem_wait_ld();
+      // logits arrive in log2 units (queries carry scale * log2 e); eight
+      // independent max accumulators keep the reduction off one dependency chain
       float v[128];
       const bool full_tile = kb >= lo && kb + BN - 1 <= hi;
-      float tmax = -INFINITY;
+      float mx[8];
 #pragma unroll
-      for (int c = 0; c < 4; ++c)
+      for (int u = 0; u < 8; ++u) mx[u] = -INFINITY;
+      if (full_tile) {
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          float x = __uint_as_float(r[c][e]) * a.scale_log2;
-          if (!full_tile) {
-            const int64_t key = kb + c * 32 + e;
-            x = (key >= lo && key <= hi) ? x : -INFINITY;
+        for (int c = 0; c < 4; ++c)
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const float x = __uint_as_float(r[c][e]);
+            v[c * 32 + e] = x;
+            mx[e & 7] = fmaxf(mx[e & 7], x);
           }
-          v[c * 32 + e] = x;
-          tmax = fmaxf(tmax, x);
-        }
+      } else {
+        const int64_t c_lo = lo - kb, c_hi = hi - kb;  // visible columns of this tile
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const int col = c * 32 + e;
+            const float x = (col >= c_lo && col <= c_hi) ? __uint_as_float(r[c][e]) : -INFINITY;
+            v[col] = x;
+            mx[e & 7] = fmaxf(mx[e & 7], x);
+          }
+      }
+      const float tmax = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                               fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
       const float m_new = fmaxf(m_used, tmax);
       // Rescale when this row's max grew by more than 2^8 (or its first
       // visible key appeared). TMEM loads/stores are warp-collective, so the
@@ -372,7 +387,9 @@ __global__ void __launch_bounds__(192, 1)
         tc::tmem_wait_st();
       }
       const float mb = (m_used == -INFINITY) ? 0.f : m_used;
-      float lsum = 0.f;
+      float ls[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) ls[u] = 0.f;
       uint32_t pk[2][32];
 #pragma unroll
       for (int c = 0; c < 2; ++c)
@@ -380,10 +397,10 @@ __global__ void __launch_bounds__(192, 1)
         for (int e = 0; e < 32; ++e) {
           const float p0 = tc::ex2(v[c * 64 + 2 * e] - mb);
           const float p1 = tc::ex2(v[c * 64 + 2 * e + 1] - mb);
-          lsum += p0 + p1;
+          ls[e & 7] += p0 + p1;
           pk[c][e] = pack_bf16x2(p0, p1);
         }
-      l += lsum;
+      l += ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
       tc::tmem_st32(s_tm, pk[0]);
       tc::tmem_st32(s_tm + 32, pk[1]);
       // consume P_{j-1} V_{j-1} before P_{j+1} V_{j+1} can complete the next

@@ -76,12 +76,30 @@ __device__ __forceinline__ uint4 rotate_chunk(uint4 x, const PairTrig& t, int e0
   return make_uint4(w[0], w[1], w[2], w[3]);
 }
 
+// Rotation followed by a multiplication by `qs`, rounded to bf16 once (the
+// prefill attention kernel takes queries pre-multiplied by scale * log2(e),
+// so its logits come out in log2 units without a per-score multiply).
+__device__ __forceinline__ uint4 rotate_scale_chunk(uint4 x, const PairTrig& t, int e0, int n_rot, float qs) {
+  uint32_t w[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    float2 v = unpack_bf16x2(w[j]);
+    float y0 = v.x, y1 = v.y;
+    if (e0 / 2 + j < n_rot) {
+      y0 = v.x * t.c[j] - v.y * t.s[j];
+      y1 = v.x * t.s[j] + v.y * t.c[j];
+    }
+    w[j] = pack_bf16x2(y0 * qs, y1 * qs);
+  }
+  return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
 __device__ __forceinline__ uint4 ld16(const bf16* p) {
   return __ldg(reinterpret_cast<const uint4*>(p));
 }
 __device__ __forceinline__ void st16(bf16* p, uint4 v) { *reinterpret_cast<uint4*>(p) = v; }
 
-// Prefill: rotate the chunk's Q into q_rot, rotate K and write it (global:
+// Prefill: rotate the chunk's Q into q_rot (times q_scale), rotate K and write it (global:
 // cache slot pos; local: k_rot workspace for the attention kernel, plus the
 // ring slot for the last `window` positions), copy V likewise.
 template <int D>
@@ -106,7 +124,7 @@ __global__ void __launch_bounds__(256) k_prefill_rope(PrefillRopeArgs a) {
     for (int h = threadIdx.y; h < n_heads; h += blockDim.y) {
       if (h < a.Hq) {
         const int64_t off = (row * a.Hq + h) * D + e0;
-        st16(a.q_rot + off, rotate_chunk(ld16(a.q + off), t, e0, a.n_rot));
+        st16(a.q_rot + off, rotate_scale_chunk(ld16(a.q + off), t, e0, a.n_rot, a.q_scale));
         continue;
       }
       const bool is_k = h < a.Hq + a.Hkv;
