@@ -106,6 +106,43 @@ __device__ __forceinline__ bool wait_all(uint64_t* bar, uint32_t parity, volatil
   return __all_sync(0xffffffffu, ok);
 }
 
+// P = 2^(x - mb) over the 128 logits of one row, packed to bf16 pairs, with
+// eight independent partial sums (and, if TRACK, partial maxima) so the
+// reductions do not run down one dependency chain.
+template <bool TRACK>
+__device__ __forceinline__ void exp_row(const uint32_t (&r)[4][32], float mb, uint32_t (&pk)[2][32],
+                                        float (&ls)[8], float (&mx)[8]) {
+#pragma unroll
+  for (int u = 0; u < 8; ++u) {
+    ls[u] = 0.f;
+    if (TRACK) mx[u] = -INFINITY;
+  }
+#pragma unroll
+  for (int i = 0; i < 64; ++i) {
+    const float x0 = __uint_as_float(r[i >> 4][(2 * i) & 31]);
+    const float x1 = __uint_as_float(r[i >> 4][(2 * i + 1) & 31]);
+    if (TRACK) mx[i & 7] = fmaxf(mx[i & 7], fmaxf(x0, x1));
+    const float p0 = tc::ex2(x0 - mb), p1 = tc::ex2(x1 - mb);
+    ls[i & 7] += p0 + p1;
+    pk[i >> 5][i & 31] = pack_bf16x2(p0, p1);
+  }
+}
+
+__device__ __forceinline__ float max8(const float (&mx)[8]) {
+  return fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])), fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+}
+
+__device__ __forceinline__ float max_row(const uint32_t (&r)[4][32]) {
+  float mx[8];
+#pragma unroll
+  for (int u = 0; u < 8; ++u) mx[u] = -INFINITY;
+#pragma unroll
+  for (int c = 0; c < 4; ++c)
+#pragma unroll
+    for (int e = 0; e < 32; ++e) mx[e & 7] = fmaxf(mx[e & 7], __uint_as_float(r[c][e]));
+  return max8(mx);
+}
+
 template <int D>
 __global__ void __launch_bounds__(192, 1)
     k_prefill_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -324,46 +361,49 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
       for (int c = 0; c < 4; ++c) tc::tmem_ld32(s_tm + c * 32, r[c]);
       tc::tmem_wait_ld();
-      // logits arrive in log2 units (queries carry scale * log2 e); eight
-      // independent max accumulators keep the reduction off one dependency chain
-      float v[128];
-      const bool full_tile = kb >= lo && kb + BN - 1 <= hi;
-      float mx[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) mx[u] = -INFINITY;
-      if (full_tile) {
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-#pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const float x = __uint_as_float(r[c][e]);
-            v[c * 32 + e] = x;
-            mx[e & 7] = fmaxf(mx[e & 7], x);
-          }
-      } else {
-        const int64_t c_lo = lo - kb, c_hi = hi - kb;  // visible columns of this tile
+      // Logits arrive in log2 units (queries carry scale * log2 e). Keys this
+      // row cannot see become -inf in place (only tiles that straddle the
+      // visible range need it).
+      if (!(kb >= lo && kb + BN - 1 <= hi)) {
+        const int64_t dlo = lo - kb, dhi = hi - kb;
+        const int c_lo = (int)(dlo < -1 ? -1 : dlo);
+        const int c_hi = (int)(dhi > BN ? BN : dhi);
 #pragma unroll
         for (int c = 0; c < 4; ++c)
 #pragma unroll
           for (int e = 0; e < 32; ++e) {
             const int col = c * 32 + e;
-            const float x = (col >= c_lo && col <= c_hi) ? __uint_as_float(r[c][e]) : -INFINITY;
-            v[col] = x;
-            mx[e & 7] = fmaxf(mx[e & 7], x);
+            if (col < c_lo || col > c_hi) r[c][e] = __float_as_uint(-INFINITY);
           }
       }
-      const float tmax = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                               fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
-      const float m_new = fmaxf(m_used, tmax);
-      // Rescale when this row's max grew by more than 2^8 (or its first
-      // visible key appeared). TMEM loads/stores are warp-collective, so the
-      // warp rescales O together; rows that need nothing use alpha = 1.
-      const bool need = m_new > m_used + RESCALE_LOG2 || (m_used == -INFINITY && m_new != -INFINITY);
+      // The running max m_used only moves when a tile's max exceeds it by more
+      // than 2^8 (or on a row's first visible key), so P = 2^(x - m_used) is
+      // computed in one pass that also takes the tile max, and redone in the
+      // rare case the max moved. A warp with a row that has seen no key yet
+      // takes the max first instead, since its speculation would always fail.
+      float mx[8], ls[8];
+      uint32_t pk[2][32];
+      bool need;
       float alpha = 1.f;
-      if (need) {
-        alpha = (m_used == -INFINITY) ? 0.f : tc::ex2(m_used - m_new);
-        l *= alpha;
-        m_used = m_new;
+      if (__any_sync(0xffffffffu, m_used == -INFINITY)) {
+        const float m_new = fmaxf(m_used, max_row(r));
+        need = m_new > m_used + RESCALE_LOG2 || (m_used == -INFINITY && m_new != -INFINITY);
+        if (need) {
+          alpha = (m_used == -INFINITY) ? 0.f : tc::ex2(m_used - m_new);
+          l *= alpha;
+          m_used = m_new;
+        }
+        exp_row<false>(r, m_used == -INFINITY ? 0.f : m_used, pk, ls, mx);
+      } else {
+        exp_row<true>(r, m_used, pk, ls, mx);
+        const float m_new = fmaxf(m_used, max8(mx));
+        need = m_new > m_used + RESCALE_LOG2;
+        if (need) {
+          alpha = tc::ex2(m_used - m_new);
+          l *= alpha;
+          m_used = m_new;
+          exp_row<false>(r, m_used, pk, ls, mx);
+        }
       }
       if (j >= 1 && __any_sync(0xffffffffu, need)) {
         // O must be stable: wait for P_{j-1} V_{j-1}
@@ -386,20 +426,6 @@ __global__ void __launch_bounds__(192, 1)
         }
         tc::tmem_wait_st();
       }
-      const float mb = (m_used == -INFINITY) ? 0.f : m_used;
-      float ls[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) ls[u] = 0.f;
-      uint32_t pk[2][32];
-#pragma unroll
-      for (int c = 0; c < 2; ++c)
-#pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const float p0 = tc::ex2(v[c * 64 + 2 * e] - mb);
-          const float p1 = tc::ex2(v[c * 64 + 2 * e + 1] - mb);
-          ls[e & 7] += p0 + p1;
-          pk[c][e] = pack_bf16x2(p0, p1);
-        }
       l += ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
       tc::tmem_st32(s_tm, pk[0]);
       tc::tmem_st32(s_tm + 32, pk[1]);
