@@ -50,7 +50,7 @@ def load_peaks():
 
 # --------------------------------------------------------------------------- clocks
 class ClockSampler:
-    """Samples SM clock and clock-event reasons through NVML every 100 ms."""
+    """Samples SM clock and clock-event reasons through NVML every 10 ms."""
     REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
                0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x2: "applications_clocks"}
 
@@ -82,7 +82,7 @@ class ClockSampler:
                         self.reasons.add(name)
             except Exception:
                 pass
-            self._stop.wait(0.1)
+            self._stop.wait(0.01)
 
     def __enter__(self):
         if self._h is not None:
@@ -153,6 +153,22 @@ def make_prefill(w, dev):
     return st, layers, ws, lens
 
 
+def recorded_traffic(kernel, workload=None):
+    """DRAM bytes per launch recorded by an ncu capture under profiles/
+    (``traffic-record:`` lines), keyed by layer type; only records whose
+    kernel-source digest matches the sources built now count."""
+    from hybrid_local_global_b200.profiling import kernel_digest, traffic_records
+    digest = kernel_digest(kernel)
+    out = {}
+    for r in traffic_records(os.path.join(ROOT, "profiles")):
+        if r.get("kernel") != kernel or r.get("digest") != digest:
+            continue
+        if workload is not None and r.get("workload") != workload:
+            continue
+        out[r.get("layer", "")] = r
+    return out
+
+
 def kernel_totals(native):
     res = {}
     for k, name in native.KERNEL_NAMES.items():
@@ -208,6 +224,14 @@ def bench_prefill(args, w, dev, world, peaks):
             else "fallback 1.59 PF/s", "traffic": None,
             "per_launch": "algorithmic FLOPs of all attention launches / their summed device time "
                           "(%d launches, %d per step)" % (attn["launches"], st.n_layers)}
+    rec = recorded_traffic("k_prefill_tc", w.name)
+    kinds = ["global" if g else "local" for g in st.is_global]
+    if all(k in rec for k in kinds):
+        roof["traffic"] = round(sum(float(rec[k]["bytes"]) for k in kinds) / len(kinds))
+        roof["traffic_note"] = ("DRAM read+write bytes per attention launch, mean over the step's layers, "
+                                "from ncu captures in %s" % ", ".join(sorted({rec[k]["file"] for k in kinds})))
+    else:
+        roof["traffic_note"] = "no ncu capture of the current kernel sources for this workload"
     launches = sum(v["launches"] for v in kern.values())
     res = dict(value=value, ms_per_step=dev_ms_max / args.steps, roofline=roof, kernels=kern,
                gpu_launches=launches, clocks=clk.summary(), wall_s=wall, flops_per_step=flops)
@@ -336,6 +360,16 @@ def bench_decode(args, w, dev, world, peaks):
             "peak_source": "%s HBM copy (MEASURED_PEAKS.json)" % peaks[1], "traffic": None,
             "per_launch": "visible K+V bytes of all split launches / their summed device time "
                           "(%d launches, %d per step)" % (sp["launches"], st.n_layers)}
+    rec = recorded_traffic("k_decode_split")
+    if rec:
+        r = next(iter(rec.values()))
+        ratio = float(r["bytes"]) / float(r["units"])
+        roof["traffic"] = round(ratio * kv_bytes / st.n_layers)
+        roof["traffic_note"] = ("DRAM bytes per split launch: visible K+V bytes per launch x %.4f, the "
+                                "traffic/algorithmic ratio of the ncu capture of %s (%s; this block is too "
+                                "large to capture)" % (ratio, r["workload"], r["file"]))
+    else:
+        roof["traffic_note"] = "no ncu capture of the current kernel sources"
     return {"metric": "decode KV GB/s", "value": round(value, 1), "unit": "GB/s",
             "workload": w.name, "description": w.description, "ms_per_step": round(dev_ms / args.steps, 4),
             "bytes_per_step": nbytes, "kv_bytes_per_step": kv_bytes,

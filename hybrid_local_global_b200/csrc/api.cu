@@ -300,7 +300,6 @@ int gemma_attn_prefill(const void* q, const void* k_new, const void* v_new, void
   // queries carry scale * log2(e): the attention kernel's logits are then in
   // log2 units (one bf16 rounding either way)
   ra.q_scale = (float)((double)scale * 1.4426950408889634);
-  ra.rows_per_cta = 4;
   ra.status = status;
   ProfScope p_rope(GEMMA_KERNEL_PREFILL_ROPE, st);
   cudaError_t e = launch_prefill_rope(ra, batch, head_dim, st);

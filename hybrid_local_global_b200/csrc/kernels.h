@@ -23,7 +23,6 @@ struct PrefillRopeArgs {
   int n_rot;           // rotated pairs
   double log2_theta;
   float q_scale;       // rotated Q is multiplied by this before the bf16 rounding
-  int rows_per_cta;
   int* status;
 };
 

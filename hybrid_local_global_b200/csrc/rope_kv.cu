@@ -11,10 +11,11 @@
 // Dive" talk): a global layer appends position p at slot p; a local layer
 // keeps a ring of `window` slots, position p at slot p % window.
 //
-// Precision: the angle pos * inv_freq is formed and reduced modulo 2*pi in
-// fp64 (an fp32 product has an ulp of 1/64 rad near position 2.6e5), then
-// sincosf of the reduced angle; the rotation itself is fp32 and the result
-// is rounded to bf16 (round to nearest even).
+// Precision: the angle pos * inv_freq is formed in half-turns (units of pi)
+// and reduced to [-1, 1] in fp64 (an fp32 product has an ulp of 1/64 rad
+// near position 2.6e5), then sincospif of the reduced angle, which needs no
+// further argument reduction; the rotation itself is fp32 and the result is
+// rounded to bf16 (round to nearest even).
 //
 // Thread map: threadIdx.x owns 8 consecutive elements (4 pairs) of the head
 // vector, so its inverse frequencies are computed once and each angle once
@@ -26,8 +27,7 @@ namespace hlg {
 
 namespace {
 
-constexpr double kTwoPi = 6.283185307179586476925286766559;
-constexpr double kInvTwoPi = 0.15915494309189533576888376337251;
+constexpr double kInvPi = 0.31830988618379067153776752674503;
 
 struct PairTrig {
   float c[4], s[4];
@@ -39,7 +39,8 @@ __device__ __forceinline__ void chunk_inv_freq(int e0, int D, int n_rot, double 
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
     int i = e0 / 2 + j;
-    inv_freq[j] = (i < n_rot) ? exp2(-(2.0 * (double)i / (double)D) * log2_theta) : 0.0;
+    // theta^(-2i/D) radians per position, expressed in half-turns
+    inv_freq[j] = (i < n_rot) ? exp2(-(2.0 * (double)i / (double)D) * log2_theta) * kInvPi : 0.0;
   }
 }
 
@@ -50,9 +51,9 @@ __device__ __forceinline__ PairTrig chunk_trig(int64_t pos, int e0, int n_rot,
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
     if (e0 / 2 + j < n_rot) {
-      double a = (double)pos * inv_freq[j];
-      double r = a - rint(a * kInvTwoPi) * kTwoPi;
-      sincosf((float)r, &t.s[j], &t.c[j]);
+      const double a = (double)pos * inv_freq[j];  // half-turns
+      const double r = a - 2.0 * rint(0.5 * a);     // in [-1, 1]
+      sincospif((float)r, &t.s[j], &t.c[j]);
     } else {
       t.c[j] = 1.f;
       t.s[j] = 0.f;
@@ -99,11 +100,36 @@ __device__ __forceinline__ uint4 ld16(const bf16* p) {
 }
 __device__ __forceinline__ void st16(bf16* p, uint4 v) { *reinterpret_cast<uint4*>(p) = v; }
 
-// Prefill: rotate the chunk's Q into q_rot (times q_scale), rotate K and write it (global:
-// cache slot pos; local: k_rot workspace for the attention kernel, plus the
-// ring slot for the last `window` positions), copy V likewise.
+// Streaming read of an input that is not read again: L2 evict-first, so the
+// rotated outputs that the attention kernel reads next stay in L2.
+__device__ __forceinline__ uint64_t policy_evict_first() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+__device__ __forceinline__ uint4 ld16_stream(const bf16* p, uint64_t pol) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.L2::cache_hint.v4.u32 {%0, %1, %2, %3}, [%4], %5;"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p), "l"(pol));
+  return v;
+}
+
+constexpr int ROPE_HB = 8;     // head vectors loaded before the first store
+constexpr int ROPE_RPT = 2;    // positions per thread
+
+// Prefill: rotate the chunk's Q into q_rot (times q_scale), rotate K and write
+// it (global: cache slot pos; local: the k_rot workspace the attention kernel
+// reads, plus the ring slot for the last `window` positions); V goes to the
+// cache slot (global) or, only for the last `window` positions, the ring
+// (local: the attention kernel reads the caller's V directly).
+//
+// threadIdx.x owns 8 elements of the head vector, threadIdx.y one position
+// (of ROPE_RPT per thread): the angles of a position are formed once and
+// serve all Hq + 2 Hkv head vectors, which are loaded ROPE_HB at a time so
+// several 16-byte loads are in flight per thread.
 template <int D>
-__global__ void __launch_bounds__(256) k_prefill_rope(PrefillRopeArgs a) {
+__global__ void __launch_bounds__(256, 2) k_prefill_rope(PrefillRopeArgs a) {
   const int b = blockIdx.y;
   const int e0 = threadIdx.x * 8;
   const int64_t pos0 = a.seq_lens_before ? (int64_t)a.seq_lens_before[b] : 0;
@@ -112,34 +138,59 @@ __global__ void __launch_bounds__(256) k_prefill_rope(PrefillRopeArgs a) {
       set_status(a.status, GEMMA_ERR_DEVICE_RANGE);
     return;
   }
+  const uint64_t pol = policy_evict_first();
   double inv_freq[4];
   chunk_inv_freq(e0, D, a.n_rot, a.log2_theta, inv_freq);
-  const int n_heads = a.Hq + (a.k_new ? 2 * a.Hkv : 0);
-  const int s_begin = blockIdx.x * a.rows_per_cta;
-  const int s_end = min(a.S, s_begin + a.rows_per_cta);
-  for (int s = s_begin; s < s_end; ++s) {
+#pragma unroll 1
+  for (int rep = 0; rep < ROPE_RPT; ++rep) {
+    const int s = (blockIdx.x * ROPE_RPT + rep) * blockDim.y + threadIdx.y;
+    if (s >= a.S) break;
     const int64_t pos = pos0 + s;
     const PairTrig t = chunk_trig(pos, e0, a.n_rot, inv_freq);
     const int64_t row = (int64_t)b * a.S + s;
-    for (int h = threadIdx.y; h < n_heads; h += blockDim.y) {
-      if (h < a.Hq) {
-        const int64_t off = (row * a.Hq + h) * D + e0;
-        st16(a.q_rot + off, rotate_scale_chunk(ld16(a.q + off), t, e0, a.n_rot, a.q_scale));
-        continue;
-      }
-      const bool is_k = h < a.Hq + a.Hkv;
-      const int kh = is_k ? h - a.Hq : h - a.Hq - a.Hkv;
-      const int64_t src_off = (row * a.Hkv + kh) * D + e0;
-      uint4 v = is_k ? rotate_chunk(ld16(a.k_new + src_off), t, e0, a.n_rot)
-                     : ld16(a.v_new + src_off);
-      bf16* cache = is_k ? a.k_cache : a.v_cache;
-      const int64_t head_base = ((int64_t)b * a.Hkv + kh) * a.cache_cap;
-      if (a.window == 0) {
-        st16(cache + (head_base + pos) * D + e0, v);
-      } else {
-        if (is_k) st16(a.k_rot + src_off, v);
-        if (s >= a.S - a.window) st16(cache + (head_base + pos % a.window) * D + e0, v);
-      }
+    // queries
+#pragma unroll 1
+    for (int h0 = 0; h0 < a.Hq; h0 += ROPE_HB) {
+      uint4 x[ROPE_HB];
+#pragma unroll
+      for (int u = 0; u < ROPE_HB; ++u)
+        if (h0 + u < a.Hq) x[u] = ld16_stream(a.q + (row * a.Hq + h0 + u) * D + e0, pol);
+#pragma unroll
+      for (int u = 0; u < ROPE_HB; ++u)
+        if (h0 + u < a.Hq)
+          st16(a.q_rot + (row * a.Hq + h0 + u) * D + e0, rotate_scale_chunk(x[u], t, e0, a.n_rot, a.q_scale));
+    }
+    if (!a.k_new) continue;  // shared layer: no K/V of its own
+    const bool to_ring = a.window > 0 && s >= a.S - a.window;
+    const int64_t slot = a.window > 0 ? pos % a.window : pos;
+#pragma unroll 1
+    for (int h0 = 0; h0 < a.Hkv; h0 += ROPE_HB / 2) {
+      uint4 kx[ROPE_HB / 2], vx[ROPE_HB / 2];
+      const bool want_v = a.window == 0 || to_ring;
+#pragma unroll
+      for (int u = 0; u < ROPE_HB / 2; ++u)
+        if (h0 + u < a.Hkv) {
+          const int64_t off = (row * a.Hkv + h0 + u) * D + e0;
+          kx[u] = ld16_stream(a.k_new + off, pol);
+          if (want_v) vx[u] = ld16_stream(a.v_new + off, pol);
+        }
+#pragma unroll
+      for (int u = 0; u < ROPE_HB / 2; ++u)
+        if (h0 + u < a.Hkv) {
+          const int kh = h0 + u;
+          const uint4 kr = rotate_chunk(kx[u], t, e0, a.n_rot);
+          const int64_t cslot = (((int64_t)b * a.Hkv + kh) * a.cache_cap + slot) * D + e0;
+          if (a.window == 0) {
+            st16(a.k_cache + cslot, kr);
+            st16(a.v_cache + cslot, vx[u]);
+          } else {
+            st16(a.k_rot + (row * a.Hkv + kh) * D + e0, kr);
+            if (to_ring) {
+              st16(a.k_cache + cslot, kr);
+              st16(a.v_cache + cslot, vx[u]);
+            }
+          }
+        }
     }
   }
 }
@@ -185,7 +236,8 @@ __global__ void __launch_bounds__(256) k_decode_rope_append(DecodeRopeArgs a) {
 cudaError_t launch_prefill_rope(const PrefillRopeArgs& a, int B, int D, cudaStream_t st) {
   const int tx = D / 8;
   dim3 block(tx, 256 / tx);
-  dim3 grid((a.S + a.rows_per_cta - 1) / a.rows_per_cta, B);
+  const int per_cta = block.y * ROPE_RPT;
+  dim3 grid((a.S + per_cta - 1) / per_cta, B);
   if (D == 256)
     k_prefill_rope<256><<<grid, block, 0, st>>>(a);
   else
