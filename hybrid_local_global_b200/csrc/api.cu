@@ -7,6 +7,7 @@
 #include <cstdarg>
 #include <cstddef>
 #include <cstdio>
+#include <cstdlib>
 #include <mutex>
 #include <string>
 #include <vector>
@@ -334,7 +335,18 @@ int gemma_attn_prefill(const void* q, const void* k_new, const void* v_new, void
   aa.wait_ns = (unsigned long long)g_wait_ns.load();
   const bool cache_view = (window == 0 || shared);
   ProfScope p_attn(GEMMA_KERNEL_PREFILL_ATTN, st);
-  e = launch_prefill_attn_tc(aa, batch, head_dim, cache_view ? cache_cap : s_new, cache_view ? 0 : 1, st);
+  // Two query tiles on a CTA pair (cta_group::2) halve each SM's K/V tile
+  // traffic; they win on long head_dim-512 layers (measured on B200: -14% on
+  // a 32K-token global layer) and lose on short or windowed ones, where the
+  // cluster's start/finish overhead dominates. GEMMA_PREFILL_KERNEL=single|pair
+  // overrides the choice.
+  bool use_pair = head_dim == 512 && (cache_view ? cache_cap : s_new) >= 16384;
+  if (const char* v = std::getenv("GEMMA_PREFILL_KERNEL")) {
+    if (std::string(v) == "single") use_pair = false;
+    if (std::string(v) == "pair") use_pair = true;
+  }
+  e = use_pair ? launch_prefill_attn_pair(aa, batch, head_dim, cache_view ? cache_cap : s_new, cache_view ? 0 : 1, st)
+               : launch_prefill_attn_tc(aa, batch, head_dim, cache_view ? cache_cap : s_new, cache_view ? 0 : 1, st);
   p_attn.done();
   if (e != cudaSuccess) return cuda_fail(e, "prefill attention launch");
   return succeed();

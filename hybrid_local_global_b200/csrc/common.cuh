@@ -125,9 +125,24 @@ __device__ __forceinline__ void record_timeout(int* status, uint64_t* bar, uint3
 // thread of the CTA raised *abort, or until deadline_ns of %globaltimer has
 // passed; on the deadline it raises *abort and records TIMEOUT. Returns true
 // only when the phase completed.
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 __device__ __forceinline__ bool mbar_wait_bounded_at(uint64_t* bar, uint32_t parity,
                                                      volatile int* abort_flag, uint64_t deadline_ns,
                                                      int* status, int where, int a, int b, int c) {
+  // a phase that has already completed: the non-blocking test answers
+  // sooner than try_wait (measured on the MMA issue path)
+  if (mbar_test_wait(bar, parity)) return true;
   uint32_t it = 0;
   while (!mbar_try_wait(bar, parity)) {
     if ((++it & 15u) == 0) {

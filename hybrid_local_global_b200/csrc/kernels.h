@@ -82,10 +82,14 @@ struct DecodeAttnArgs {
 
 cudaError_t launch_prefill_rope(const PrefillRopeArgs& a, int B, int D, cudaStream_t st);
 cudaError_t launch_decode_rope_append(const DecodeRopeArgs& a, int B, int D, cudaStream_t st);
-// tcgen05 prefill (head_dim 256). key_rows_total = rows of the K/V views;
-// kv_token_major: views are [B][rows][Hkv][D] (1) or [B][Hkv][rows][D] (0).
+// tcgen05 prefill (head_dim 256 or 512). key_rows_total = rows of the K/V
+// views; kv_token_major: views are [B][rows][Hkv][D] (1) or [B][Hkv][rows][D] (0).
+// _tc: one CTA per 128-row query tile; _pair: two query tiles on a CTA pair
+// sharing each MMA (cta_group::2).
 cudaError_t launch_prefill_attn_tc(const PrefillAttnArgs& a, int B, int D, int key_rows_total,
                                    int kv_token_major, cudaStream_t st);
+cudaError_t launch_prefill_attn_pair(const PrefillAttnArgs& a, int B, int D, int key_rows_total,
+                                     int kv_token_major, cudaStream_t st);
 cudaError_t launch_decode_split(const DecodeAttnArgs& a, int B, int D, cudaStream_t st);
 cudaError_t launch_decode_combine(const DecodeAttnArgs& a, int B, int D, cudaStream_t st);
 cudaError_t launch_visible_ranges(const int32_t* seq_lens_before, int B, int S, int window,

@@ -23,7 +23,7 @@ def _expected_rotated_bf16(oracle, k_bits_row, pos, frac, theta):
 
 
 def run_prefill_case(oracle, *, B, S, Hq, Hkv, D, W, frac, theta, seed, prior=None, q_scale=1.0,
-                     k_scale=1.0, tol=(2e-2, 2e-3), check_cache=True, check_lse=True):
+                     k_scale=1.0, tol=(2e-2, 2e-3), check_cache=True, check_lse=True, cache_fill=0.0):
     dev = torch.device("cuda")
     g = synth.generator(seed)
     q = synth.randn_bf16((B, S, Hq, D), g, scale=q_scale)
@@ -32,8 +32,10 @@ def run_prefill_case(oracle, *, B, S, Hq, Hkv, D, W, frac, theta, seed, prior=No
     prior = list(prior) if prior else [0] * B
     T = max(prior) + S
     cap = W if W else T + 16
-    kc = torch.zeros((B, Hkv, cap, D), dtype=torch.bfloat16)
-    vc = torch.zeros((B, Hkv, cap, D), dtype=torch.bfloat16)
+    # slots past the sequence hold whatever the caller left there: cache_fill
+    # = nan checks that no such value reaches an output
+    kc = torch.full((B, Hkv, cap, D), cache_fill, dtype=torch.bfloat16)
+    vc = torch.full((B, Hkv, cap, D), cache_fill, dtype=torch.bfloat16)
     for b in range(B):
         if prior[b]:
             kc[b, :, :prior[b]] = synth.randn_bf16((Hkv, prior[b], D), g)
@@ -88,9 +90,11 @@ def run_prefill_case(oracle, *, B, S, Hq, Hkv, D, W, frac, theta, seed, prior=No
             assert n_same >= 0.98 * n_all, "only %d of %d rotated K values bit-identical" % (n_same, n_all)
         if W == 0:
             # untouched slots keep their bytes
+            bits = lambda t: t.view(torch.int16)
             for b in range(B):
-                assert torch.equal(kc1[b, :, :prior[b]], kc0[b, :, :prior[b]])
-                assert torch.equal(kc1[b, :, prior[b] + S:], kc0[b, :, prior[b] + S:])
+                for c1, c0 in ((kc1, kc0), (vc1, vc0)):
+                    assert torch.equal(bits(c1[b, :, :prior[b]]), bits(c0[b, :, :prior[b]]))
+                    assert torch.equal(bits(c1[b, :, prior[b] + S:]), bits(c0[b, :, prior[b] + S:]))
     return out
 
 
@@ -109,6 +113,30 @@ CASES = [
 @pytest.mark.parametrize("case", CASES, ids=lambda c: "B%dS%dH%d-%dD%dW%d%s" % (
     c["B"], c["S"], c["Hq"], c["Hkv"], c["D"], c["W"], "P" if c.get("prior") else ""))
 def test_prefill_small(oracle, case):
+    run_prefill_case(oracle, **case)
+
+
+PAIR_CASES = [
+    dict(B=1, S=300, Hq=8, Hkv=1, D=512, W=0, frac=0.25, theta=1e6, seed=111, cache_fill=float("nan")),
+    dict(B=2, S=100, Hq=8, Hkv=1, D=512, W=0, frac=0.25, theta=1e6, seed=112, prior=[37, 250],
+         cache_fill=float("nan")),
+    dict(B=1, S=257, Hq=8, Hkv=4, D=512, W=64, frac=1.0, theta=1e4, seed=113),
+    dict(B=2, S=383, Hq=4, Hkv=2, D=256, W=0, frac=0.25, theta=1e6, seed=114, cache_fill=float("nan")),
+    dict(B=1, S=520, Hq=8, Hkv=4, D=256, W=128, frac=1.0, theta=1e4, seed=115),
+    dict(B=1, S=1, Hq=8, Hkv=4, D=256, W=512, frac=1.0, theta=1e4, seed=116),
+]
+
+
+@pytest.mark.parametrize("kernel", ["single", "pair"])
+@pytest.mark.parametrize("case", PAIR_CASES, ids=lambda c: "B%dS%dH%d-%dD%dW%d%s%s" % (
+    c["B"], c["S"], c["Hq"], c["Hkv"], c["D"], c["W"], "P" if c.get("prior") else "",
+    "nan" if c.get("cache_fill") else ""))
+def test_prefill_each_kernel(oracle, monkeypatch, kernel, case):
+    """Both attention kernels (one query tile per CTA; two per CTA pair on
+    cta_group::2 MMAs) on ragged lengths, odd tile counts, a cached prefix,
+    and caches whose unused slots hold nan (the key tile that crosses the
+    sequence end must not let them reach an output)."""
+    monkeypatch.setenv("GEMMA_PREFILL_KERNEL", kernel)
     run_prefill_case(oracle, **case)
 
 
