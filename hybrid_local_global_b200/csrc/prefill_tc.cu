@@ -146,7 +146,8 @@ __device__ __forceinline__ float max_row(const uint32_t (&r)[4][32]) {
 template <int D>
 __global__ void __launch_bounds__(192, 1)
     k_prefill_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                 const __grid_constant__ CUtensorMap tm_v, const TcArgs a) {
+                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+                 const TcArgs a) {
   using Cfg = TcCfg<D>;
   constexpr int NSTAGE = Cfg::NSTAGE;
   constexpr int Q_B = Cfg::Q_B;
@@ -445,30 +446,43 @@ __global__ void __launch_bounds__(192, 1)
     if (ok)
       ok = wait_all(&ctl->o_done[(n_tiles - 1) & 1], ((n_tiles - 1) >> 1) & 1, abort_flag, deadline,
                     a.status, 17, n_tiles);
+    // Epilogue: O / l as bf16 into the Q buffer (free once the last MMA is
+    // done), laid out as the 128-byte-swizzled boxes of the output map, then
+    // four TMA stores. A thread owns one row, so direct stores would write
+    // 16 bytes per output row per instruction; the staged copy writes whole
+    // rows. Rows past the sequence end are clipped by the store.
+    unsigned char* sO = sm;  // Q buffer
     if (ok) {
       tc::fence_after_sync();
       const float inv = l > 0.f ? 1.f / l : 0.f;
-      bf16* dst = a.out + (((int64_t)b * a.S + q0 + row) * a.Hq + h) * D + vh * DV;
 #pragma unroll 1
       for (int c = 0; c < 8; ++c) {
         uint32_t o[32];
         tc::tmem_ld32(tm + COL_O + c * 32, o);
         tc::tmem_wait_ld();
-        if (row_valid) {
+        unsigned char* box_row = sO + (c >> 1) * CHUNK_B + row * 128;
 #pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            uint4 w;
-            w.x = pack_bf16x2(__uint_as_float(o[u * 8 + 0]) * inv, __uint_as_float(o[u * 8 + 1]) * inv);
-            w.y = pack_bf16x2(__uint_as_float(o[u * 8 + 2]) * inv, __uint_as_float(o[u * 8 + 3]) * inv);
-            w.z = pack_bf16x2(__uint_as_float(o[u * 8 + 4]) * inv, __uint_as_float(o[u * 8 + 5]) * inv);
-            w.w = pack_bf16x2(__uint_as_float(o[u * 8 + 6]) * inv, __uint_as_float(o[u * 8 + 7]) * inv);
-            *reinterpret_cast<uint4*>(dst + c * 32 + u * 8) = w;
-          }
+        for (int u = 0; u < 4; ++u) {
+          uint4 w;
+          w.x = pack_bf16x2(__uint_as_float(o[u * 8 + 0]) * inv, __uint_as_float(o[u * 8 + 1]) * inv);
+          w.y = pack_bf16x2(__uint_as_float(o[u * 8 + 2]) * inv, __uint_as_float(o[u * 8 + 3]) * inv);
+          w.z = pack_bf16x2(__uint_as_float(o[u * 8 + 4]) * inv, __uint_as_float(o[u * 8 + 5]) * inv);
+          w.w = pack_bf16x2(__uint_as_float(o[u * 8 + 6]) * inv, __uint_as_float(o[u * 8 + 7]) * inv);
+          const int unit = ((c & 1) * 4 + u) ^ (row & 7);
+          *reinterpret_cast<uint4*>(box_row + unit * 16) = w;
         }
       }
       if (row_valid && a.lse && vh == 0)
         a.lse[((int64_t)b * a.Hq + h) * a.S + q0 + row] =
             l > 0.f ? (m_used + __log2f(l)) * 0.69314718055994530942f : -INFINITY;
+    }
+    fence_proxy_async_smem();
+    asm volatile("bar.sync 1, 128;" ::: "memory");  // the four softmax warps
+    if (warp == 2 && lane == 0 && !*abort_flag) {
+      for (int c = 0; c < DV / 64; ++c)
+        tc::tma_store_4d(&tm_o, smem_u32(sO + c * CHUNK_B), vh * DV + c * 64, h, q0, b);
+      tc::bulk_commit();
+      tc::bulk_wait_read0();
     }
   }
 
@@ -526,12 +540,13 @@ cudaError_t launch_prefill_attn_tc(const PrefillAttnArgs& a, int B, int D, int k
                                    int kv_token_major, cudaStream_t st) {
   if (D != 256 && D != 512) return cudaErrorInvalidValue;
   const uint64_t E = 2;
-  CUtensorMap mq, mk, mv;
+  CUtensorMap mq, mk, mv, mo;
   {
     const uint64_t dims[4] = {(uint64_t)D, (uint64_t)a.Hq, (uint64_t)a.S, (uint64_t)B};
     const uint64_t str[3] = {(uint64_t)D * E, (uint64_t)a.Hq * D * E, (uint64_t)a.S * a.Hq * D * E};
     const uint32_t box[4] = {64, 1, BM, 1};
     if (!make_map(&mq, a.q_rot, dims, str, box)) return cudaErrorInvalidValue;
+    if (!make_map(&mo, a.out, dims, str, box)) return cudaErrorInvalidValue;
   }
   if (kv_token_major) {
     // [B][rows][Hkv][D]
@@ -573,13 +588,13 @@ cudaError_t launch_prefill_attn_tc(const PrefillAttnArgs& a, int B, int D, int k
     cudaError_t e = cudaFuncSetAttribute(k_prefill_tc<256>, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);
     if (e != cudaSuccess) return e;
     dim3 grid(a.Hq * Cfg::NV, B, t.n_qtiles);
-    k_prefill_tc<256><<<grid, 192, Cfg::SMEM, st>>>(mq, mk, mv, t);
+    k_prefill_tc<256><<<grid, 192, Cfg::SMEM, st>>>(mq, mk, mv, mo, t);
   } else {
     using Cfg = TcCfg<512>;
     cudaError_t e = cudaFuncSetAttribute(k_prefill_tc<512>, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);
     if (e != cudaSuccess) return e;
     dim3 grid(a.Hq * Cfg::NV, B, t.n_qtiles);
-    k_prefill_tc<512><<<grid, 192, Cfg::SMEM, st>>>(mq, mk, mv, t);
+    k_prefill_tc<512><<<grid, 192, Cfg::SMEM, st>>>(mq, mk, mv, mo, t);
   }
   return cudaGetLastError();
 }
