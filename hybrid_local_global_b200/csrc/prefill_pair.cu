@@ -171,7 +171,8 @@ __device__ __forceinline__ void clear_v_tail_pair(uint32_t stage, int r0) {
 template <int D>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
     k_prefill_pair(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                   const __grid_constant__ CUtensorMap tm_v, const PairArgs a) {
+                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+                   const PairArgs a) {
   using Cfg = PairCfg<D>;
   constexpr int NSTAGE = Cfg::NSTAGE;
   constexpr int Q_B = Cfg::Q_B;
@@ -468,30 +469,41 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
     if (ok)
       ok = wait_all(&ctl->o_done[(n_tiles - 1) & 1], ((n_tiles - 1) >> 1) & 1, abort_flag, deadline,
                     a.status, 47, n_tiles);
+    // Epilogue: O / l as bf16 into this CTA's Q buffer (free once the last
+    // MMA is done), as the 128-byte-swizzled boxes of the output map, then
+    // TMA stores of whole rows (rows past the sequence end are clipped).
+    unsigned char* sO = sm;  // Q buffer
     if (ok) {
       tc::fence_after_sync();
       const float inv = l > 0.f ? 1.f / l : 0.f;
-      bf16* dst = a.out + (((int64_t)b * a.S + q0 + row) * a.Hq + h) * D + vh * DV;
 #pragma unroll 1
       for (int c = 0; c < 8; ++c) {
         uint32_t o[32];
         tc::tmem_ld32(tm + COL_O + c * 32, o);
         tc::tmem_wait_ld();
-        if (row_valid) {
+        unsigned char* box_row = sO + (c >> 1) * CHUNK_Q + row * 128;
 #pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            uint4 w;
-            w.x = pack_bf16x2(__uint_as_float(o[u * 8 + 0]) * inv, __uint_as_float(o[u * 8 + 1]) * inv);
-            w.y = pack_bf16x2(__uint_as_float(o[u * 8 + 2]) * inv, __uint_as_float(o[u * 8 + 3]) * inv);
-            w.z = pack_bf16x2(__uint_as_float(o[u * 8 + 4]) * inv, __uint_as_float(o[u * 8 + 5]) * inv);
-            w.w = pack_bf16x2(__uint_as_float(o[u * 8 + 6]) * inv, __uint_as_float(o[u * 8 + 7]) * inv);
-            *reinterpret_cast<uint4*>(dst + c * 32 + u * 8) = w;
-          }
+        for (int u = 0; u < 4; ++u) {
+          uint4 w;
+          w.x = pack_bf16x2(__uint_as_float(o[u * 8 + 0]) * inv, __uint_as_float(o[u * 8 + 1]) * inv);
+          w.y = pack_bf16x2(__uint_as_float(o[u * 8 + 2]) * inv, __uint_as_float(o[u * 8 + 3]) * inv);
+          w.z = pack_bf16x2(__uint_as_float(o[u * 8 + 4]) * inv, __uint_as_float(o[u * 8 + 5]) * inv);
+          w.w = pack_bf16x2(__uint_as_float(o[u * 8 + 6]) * inv, __uint_as_float(o[u * 8 + 7]) * inv);
+          const int unit = ((c & 1) * 4 + u) ^ (row & 7);
+          *reinterpret_cast<uint4*>(box_row + unit * 16) = w;
         }
       }
       if (row_valid && a.lse && vh == 0)
         a.lse[((int64_t)b * a.Hq + h) * a.S + q0 + row] =
             l > 0.f ? (m_used + __log2f(l)) * 0.69314718055994530942f : -INFINITY;
+    }
+    fence_proxy_async_smem();
+    asm volatile("bar.sync 1, 128;" ::: "memory");  // the four softmax warps
+    if (warp == 2 && lane == 0 && !*abort_flag && q0 < a.S) {
+      for (int c = 0; c < DV / 64; ++c)
+        tc::tma_store_4d(&tm_o, smem_u32(sO + c * CHUNK_Q), vh * DV + c * 64, h, q0, b);
+      tc::bulk_commit();
+      tc::bulk_wait_read0();
     }
   }
 
@@ -556,13 +568,13 @@ bool make_map(CUtensorMap* m, const void* ptr, const uint64_t dims[4], const uin
 }
 
 template <int D>
-cudaError_t launch_pair(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const PairArgs& t,
-                        int B, cudaStream_t st) {
+cudaError_t launch_pair(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mo,
+                        const PairArgs& t, int B, cudaStream_t st) {
   using Cfg = PairCfg<D>;
   cudaError_t e = cudaFuncSetAttribute(k_prefill_pair<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);
   if (e != cudaSuccess) return e;
   dim3 grid(2 * t.n_pairs, t.Hq * Cfg::NV, B);
-  k_prefill_pair<D><<<grid, 192, Cfg::SMEM, st>>>(mq, mk, mv, t);
+  k_prefill_pair<D><<<grid, 192, Cfg::SMEM, st>>>(mq, mk, mv, mo, t);
   return cudaGetLastError();
 }
 
@@ -572,12 +584,13 @@ cudaError_t launch_prefill_attn_pair(const PrefillAttnArgs& a, int B, int D, int
                                      int kv_token_major, cudaStream_t st) {
   if (D != 256 && D != 512) return cudaErrorInvalidValue;
   const uint64_t E = 2;
-  CUtensorMap mq, mk, mv;
+  CUtensorMap mq, mk, mv, mo;
   {
     const uint64_t dims[4] = {(uint64_t)D, (uint64_t)a.Hq, (uint64_t)a.S, (uint64_t)B};
     const uint64_t str[3] = {(uint64_t)D * E, (uint64_t)a.Hq * D * E, (uint64_t)a.S * a.Hq * D * E};
     const uint32_t box[4] = {64, 1, BM, 1};
     if (!make_map(&mq, a.q_rot, dims, str, box)) return cudaErrorInvalidValue;
+    if (!make_map(&mo, a.out, dims, str, box)) return cudaErrorInvalidValue;
   }
   if (kv_token_major) {
     // [B][rows][Hkv][D]
@@ -614,7 +627,7 @@ cudaError_t launch_prefill_attn_pair(const PrefillAttnArgs& a, int B, int D, int
   t.kv_token_major = kv_token_major;
   const int n_qtiles = (a.S + BM - 1) / BM;
   t.n_pairs = (n_qtiles + 1) / 2;
-  return D == 256 ? launch_pair<256>(mq, mk, mv, t, B, st) : launch_pair<512>(mq, mk, mv, t, B, st);
+  return D == 256 ? launch_pair<256>(mq, mk, mv, mo, t, B, st) : launch_pair<512>(mq, mk, mv, mo, t, B, st);
 }
 
 }  // namespace hlg
