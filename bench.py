@@ -104,32 +104,22 @@ class ClockSampler:
 
 
 # --------------------------------------------------------------------------- distributed
+RANKS = None  # hybrid_local_global_b200.dist.Ranks of this process
+
+
 def dist_setup(n_gpus):
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if world > 1:
-        import datetime
-        import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
-                                device_id=torch.device("cuda", local))
-    return world, rank, local
+    global RANKS
+    from hybrid_local_global_b200 import dist as hdist
+    RANKS = hdist.setup("nccl")
+    return RANKS.world, RANKS.rank, RANKS.local
 
 
 def barrier(world):
-    if world > 1:
-        import torch.distributed as dist
-        dist.barrier()
+    RANKS.barrier()
 
 
 def max_over_ranks(x: float, world: int) -> float:
-    if world == 1:
-        return x
-    import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    return float(t.item())
+    return RANKS.max_over_ranks(x)
 
 
 # --------------------------------------------------------------------------- prefill (ours)
@@ -487,13 +477,11 @@ def main():
     ap.add_argument("--cpu-rows-global", type=int, default=49152)
     args = ap.parse_args()
 
-    world, rank, local = dist_setup(args.gpus)
     if args.impl == "reference":
-        run_reference(args, world, rank)
-        if world > 1:
-            import torch.distributed as dist
-            dist.destroy_process_group()
+        # the oracle on the host cores: rank 0 alone runs it, no process group
+        run_reference(args, int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")))
         return
+    world, rank, local = dist_setup(args.gpus)
 
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
@@ -534,9 +522,7 @@ def main():
         line["gpu_launches"] += line["decode"]["gpu_launches"]
     if rank == 0:
         print(json.dumps(line))
-    if world > 1:
-        import torch.distributed as dist
-        dist.destroy_process_group()
+    RANKS.close()
 
 
 if __name__ == "__main__":

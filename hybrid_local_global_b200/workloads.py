@@ -76,6 +76,10 @@ WORKLOADS = {
         local=L31B_LOCAL, global_=L31B_GLOBAL, seq=4096, prior=262144 - 4096, seed=4,
         fixed_kinds=("global",),
         description="chunked prefill of 4096 queries at 258048.. against a 256K global cache"),
+    "global_s16384": Workload(
+        "global_s16384", "prefill", batch=1, n_q_heads=32, n_layers=1, ratio=0,
+        local=L31B_LOCAL, global_=L31B_GLOBAL, seq=16384, seed=5, fixed_kinds=("global",),
+        description="one 31B-shaped global layer, B1 S16384 Hq32 Hkv4 D512 (a kernel-profiling case)"),
     "global_decode_256k": Workload(
         "global_decode_256k", "decode", batch=1, n_q_heads=32, n_layers=1, ratio=0,
         local=L31B_LOCAL, global_=L31B_GLOBAL, len_lo=262144, len_hi=262144, seed=4,
