@@ -114,7 +114,7 @@ def rope_bf16(x_bits: np.ndarray, pos: int, rope_frac: float, theta: float) -> n
     return y
 
 
-def attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, *, q_pos0, n_keys, rot_from,
+def attention(q: np.ndarray, k: np.ndarray, v: np.ndarray | None, *, q_pos0, n_keys, rot_from,
               window: int, rope_frac: float, theta: float, scale: float,
               rows: np.ndarray | None = None, n_threads: int = 0):
     """Exact attention rows.
@@ -122,15 +122,17 @@ def attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, *, q_pos0, n_keys, ro
     q: uint16 [B,S,Hq,D]; k, v: uint16 [B,T,Hkv,D] in position order.
     q_pos0[b]: absolute position of query row 0; n_keys[b]: keys 0..n_keys-1
     exist; keys at positions >= rot_from[b] are rotated here, earlier keys
-    arrive rotated. rows: int32 [R,3] (b, h, i); None = every row.
+    arrive rotated. v = None: K = V, the values are the keys as cached
+    (rotated). rows: int32 [R,3] (b, h, i); None = every row.
     Returns (out fp64 [R,D], lse fp64 [R]).
     """
     q = np.ascontiguousarray(q, dtype=np.uint16)
     k = np.ascontiguousarray(k, dtype=np.uint16)
-    v = np.ascontiguousarray(v, dtype=np.uint16)
+    if v is not None:
+        v = np.ascontiguousarray(v, dtype=np.uint16)
     B, S, Hq, D = q.shape
     Bk, T, Hkv, Dk = k.shape
-    if Bk != B or Dk != D or v.shape != k.shape:
+    if Bk != B or Dk != D or (v is not None and v.shape != k.shape):
         raise ValueError("shape mismatch")
     if rows is None:
         bb, hh, ii = np.meshgrid(np.arange(B), np.arange(Hq), np.arange(S), indexing="ij")
@@ -141,7 +143,7 @@ def attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, *, q_pos0, n_keys, ro
     rot_from = np.ascontiguousarray(np.broadcast_to(np.asarray(rot_from, np.int64), (B,)))
     out = np.zeros((rows.shape[0], D), dtype=np.float64)
     lse = np.zeros(rows.shape[0], dtype=np.float64)
-    rc = _load().hlg_attention(_ptr(q), _ptr(k), _ptr(v), _ptr(q_pos0), _ptr(n_keys),
+    rc = _load().hlg_attention(_ptr(q), _ptr(k), _ptr(v) if v is not None else None, _ptr(q_pos0), _ptr(n_keys),
                                _ptr(rot_from), B, S, T, Hq, Hkv, D, window, rope_frac,
                                theta, scale, rows.shape[0], _ptr(rows), _ptr(out), _ptr(lse),
                                n_threads)

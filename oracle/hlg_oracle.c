@@ -171,6 +171,12 @@ void hlg_rope_bf16(const uint16_t* x_bits, double* y, int head_dim,
 /* pre-RoPE) and k~_j = k_j below it (keys that arrive already rotated, as  */
 /* in a filled cache). V is never rotated.                                  */
 /*                                                                          */
+/* K = V ([WALK] 3b "K = V"; [TECH] "Core Model Architecture": global       */
+/* layers cache only K and multiply the attention weights by K, which then  */
+/* serves as V): pass v == NULL and v_j is the key as the cache holds it,   */
+/* k~_j. Reading: the cache holds rotated keys, so the values are the       */
+/* rotated keys.                                                            */
+/*                                                                          */
 /* Layouts: q [B][S][Hq][D], k and v [B][T][Hkv][D] in position order       */
 /* (key j of batch b is row j), all bf16 bits. rows [n_rows][3] int32.      */
 /* out [n_rows][D] fp64, lse [n_rows] fp64 (-inf when nothing is visible).  */
@@ -245,8 +251,14 @@ static void one_row(group_work* w, int64_t r, double* s, double* qrot)
         l += p;
     }
     for (int64_t j = lo; j <= hi; ++j) {
-        const uint16_t* vj = a->v + (((size_t)b * a->T + (size_t)j) * a->Hkv + w->g) * a->D;
         double p = s[j - lo] / l;
+        if (a->v == NULL) {
+            const double* kj = w->krot + (size_t)j * a->D;  /* K serves as V */
+            for (int d = 0; d < a->D; ++d)
+                o[d] += p * kj[d];
+            continue;
+        }
+        const uint16_t* vj = a->v + (((size_t)b * a->T + (size_t)j) * a->Hkv + w->g) * a->D;
         for (int d = 0; d < a->D; ++d)
             o[d] += p * bf16_bits_to_double(vj[d]);
     }

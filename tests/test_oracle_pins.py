@@ -362,3 +362,49 @@ def test_byte_counter_page_figures(oracle):
     a = oracle.stack_cache_bytes(6, 5, 0, 64, **kw)
     b = oracle.stack_cache_bytes(6, 5, 2, 64, **kw)
     assert a - b == oracle.layer_cache_bytes(64, 16, 1024, 256)
+
+
+# --------------------------------------------------------------------------- K = V
+@pytest.mark.parametrize("frac,theta", [(1.0, 1e4), (0.25, 1e6)])
+def test_k_equals_v_matches_sdpa_with_rotated_keys_as_values(oracle, frac, theta):
+    """K = V (v = None): the values are the keys as the cache holds them, i.e.
+    rotated. Equals fp64 SDPA whose keys and values are both the keys rotated
+    by numpy complex multiplication at their own positions (chunk offset P,
+    GQA 4:2)."""
+    B, S, P, Hq, Hkv, D = 1, 5, 7, 4, 2, 16
+    q = rand_bits((B, S, Hq, D), 61)
+    k = rand_bits((B, P + S, Hkv, D), 62)
+    out, lse = oracle.attention(q, k, None, q_pos0=P, n_keys=P + S, rot_from=0, window=0,
+                                rope_frac=frac, theta=theta, scale=0.4)
+    qf, kf = bits_to_f64(q), bits_to_f64(k)
+    qr = np.stack([complex_rope(qf[0, i], P + i, frac, theta) for i in range(S)])[None]
+    kr = np.stack([complex_rope(kf[0, j], j, frac, theta) for j in range(P + S)])[None]
+    qt = qr.transpose(0, 2, 1, 3)
+    kt = np.repeat(kr.transpose(0, 2, 1, 3), Hq // Hkv, axis=1)
+    i = np.arange(S)[:, None] + P
+    j = np.arange(P + S)[None, :]
+    ref = _sdpa(qt, kt, kt, j <= i, 0.4).reshape(-1, D)
+    np.testing.assert_allclose(out, ref, rtol=0, atol=1e-10)
+    # the values differ from the unrotated keys wherever a pair turns
+    plain, _ = oracle.attention(q, k, k, q_pos0=P, n_keys=P + S, rot_from=0, window=0,
+                                rope_frac=frac, theta=theta, scale=0.4)
+    assert np.abs(out - plain).max() > 1e-3
+
+
+def test_k_equals_v_worked_example_and_cached_keys(oracle):
+    """The page's worked example (4 tokens, 8 dims, values set equal to the
+    keys): the output equals the standard computation given V = K explicitly.
+    Keys that arrive rotated (a filled cache, rot_from = T) serve as values
+    exactly as given."""
+    figs = json.load(open(GOLDEN))["k_equals_v_example"]
+    T, D = figs["tokens"], figs["dims"]
+    q = rand_bits((1, T, 1, D), 71)
+    k = rand_bits((1, T, 1, D), 72)
+    kw = dict(q_pos0=0, n_keys=T, window=0, theta=1e4, scale=1 / math.sqrt(D))
+    a, la = oracle.attention(q, k, None, rot_from=0, rope_frac=0.0, **kw)
+    b, lb = oracle.attention(q, k, k, rot_from=0, rope_frac=0.0, **kw)
+    np.testing.assert_array_equal(a, b)
+    np.testing.assert_array_equal(la, lb)
+    c, _ = oracle.attention(q, k, None, rot_from=T, rope_frac=1.0, **kw)
+    d, _ = oracle.attention(q, k, k, rot_from=T, rope_frac=1.0, **kw)
+    np.testing.assert_array_equal(c, d)
