@@ -270,17 +270,25 @@ def e2e_prefill(args, st, layers, ws, lens, flops, world):
 def decode_bytes(w, st, lens_cpu):
     """Algorithmic bytes of one decode step: visible K and V rows read once per
     KV head (every layer, shared ones included: they attend over their
-    source's cache), plus q, the new k/v and the output."""
+    source's cache; K only on a K = V layer), plus q, the new k/v and the
+    output."""
     total = 0
-    L = lens_cpu.to(torch.int64)
     for l in range(st.n_layers):
         t = st.layer_type(l)
-        vis = torch.clamp(L, max=t.window) if t.window else L
-        total += int(vis.sum()) * t.n_kv_heads * t.head_dim * 2 * 2
+        kv = 1 if st.keqv(l) else 2
+        total += visible_kv_bytes(st, l, lens_cpu)
         total += w.batch * w.n_q_heads * t.head_dim * 2 * 2
         if not st.is_shared(l):
-            total += w.batch * t.n_kv_heads * t.head_dim * 2 * 2 * 2
+            total += w.batch * t.n_kv_heads * t.head_dim * 2 * kv
     return total
+
+
+def visible_kv_bytes(st, l, lens_cpu):
+    """Cached K (and V unless K = V) bytes layer l's decode reads."""
+    t = st.layer_type(l)
+    L = lens_cpu.to(torch.int64)
+    vis = torch.clamp(L, max=t.window) if t.window else L
+    return int(vis.sum()) * t.n_kv_heads * t.head_dim * 2 * (1 if st.keqv(l) else 2)
 
 
 def bench_decode(args, w, dev, world, peaks):
@@ -337,10 +345,7 @@ def bench_decode(args, w, dev, world, peaks):
     kern = kernel_totals(native)
     native.gemma_attn_profile(False)
     nbytes = decode_bytes(w, st, lens_cpu)
-    kv_bytes = sum(int((torch.clamp(lens_cpu.to(torch.int64), max=st.layer_type(l).window)
-                        if st.layer_type(l).window else lens_cpu.to(torch.int64)).sum())
-                   * st.layer_type(l).n_kv_heads * st.layer_type(l).head_dim * 4
-                   for l in range(st.n_layers))
+    kv_bytes = sum(visible_kv_bytes(st, l, lens_cpu) for l in range(st.n_layers))
     value = world * nbytes * args.steps / (dev_ms / 1e3) / 1e9
     sp = kern.get("decode_split", {"ms": float("nan"), "launches": 0})
     achieved = kv_bytes * args.steps / (sp["ms"] / 1e3) / 1e9
@@ -348,7 +353,7 @@ def bench_decode(args, w, dev, world, peaks):
     roof = {"bound": "hbm", "kernel": "split-K decode attention", "achieved": round(achieved, 1),
             "peak": peak, "unit": "GB/s", "frac": round(achieved / peak, 4),
             "peak_source": "%s HBM copy (MEASURED_PEAKS.json)" % peaks[1], "traffic": None,
-            "per_launch": "visible K+V bytes of all split launches / their summed device time "
+            "per_launch": "visible K (and V unless K = V) bytes of all split launches / their summed device time "
                           "(%d launches, %d per step)" % (sp["launches"], st.n_layers)}
     rec = recorded_traffic("k_decode_split")
     if rec:

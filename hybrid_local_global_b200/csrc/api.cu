@@ -217,9 +217,32 @@ int gemma_layer_schedule(int n_layers, int ratio, int n_shared, int* is_global, 
   return succeed();
 }
 
+// Checks GEMMA_F_SHARED / GEMMA_F_KEQV and the k_new, v_new and v_cache they
+// imply. On success *v_cache_io is the cache the values are read from: the
+// key cache under K = V.
+static int check_kv_flags(unsigned flags, int window, const void* k_new, const void* v_new, void* k_cache,
+                          void** v_cache_io) {
+  if (flags & ~(GEMMA_F_SHARED | GEMMA_F_KEQV)) return fail(GEMMA_ERR_INVALID_ARG, "unknown flags 0x%x", flags);
+  const bool shared = flags & GEMMA_F_SHARED, keqv = flags & GEMMA_F_KEQV;
+  if (keqv && window > 0)
+    return fail(GEMMA_ERR_UNSUPPORTED, "GEMMA_F_KEQV: K = V is defined for global layers only");
+  if (shared && (k_new || v_new))
+    return fail(GEMMA_ERR_INVALID_ARG, "GEMMA_F_SHARED: k_new and v_new must be NULL");
+  if (keqv && v_new) return fail(GEMMA_ERR_INVALID_ARG, "GEMMA_F_KEQV: v_new must be NULL (the keys are the values)");
+  if (!shared && (!k_new || (!keqv && !v_new)))
+    return fail(GEMMA_ERR_INVALID_ARG, "k_new and v_new are required unless GEMMA_F_SHARED (v_new: unless GEMMA_F_KEQV)");
+  if (keqv) {
+    if (*v_cache_io && *v_cache_io != k_cache)
+      return fail(GEMMA_ERR_INVALID_ARG, "GEMMA_F_KEQV: v_cache must be NULL or equal to k_cache");
+    *v_cache_io = k_cache;
+  }
+  return GEMMA_OK;
+}
+
 int gemma_kv_share_bind(gemma_kv_desc* dst, const gemma_kv_desc* src) {
   if (!dst || !src) return fail(GEMMA_ERR_INVALID_ARG, "null descriptor");
-  if (!src->k_cache || !src->v_cache) return fail(GEMMA_ERR_INVALID_ARG, "source layer has no cache");
+  if (!src->k_cache || (!src->v_cache && !src->k_eq_v))
+    return fail(GEMMA_ERR_INVALID_ARG, "source layer has no cache");
   if (src->layer >= dst->layer)
     return fail(GEMMA_ERR_SHARE_MISMATCH, "source layer %d must precede layer %d", src->layer, dst->layer);
   if ((src->window == 0) != (dst->window == 0))
@@ -227,10 +250,11 @@ int gemma_kv_share_bind(gemma_kv_desc* dst, const gemma_kv_desc* src) {
                 dst->layer);
   if (src->window != dst->window || src->cache_cap != dst->cache_cap ||
       src->n_kv_heads != dst->n_kv_heads || src->head_dim != dst->head_dim ||
-      src->rope_frac != dst->rope_frac || src->rope_theta != dst->rope_theta)
+      src->rope_frac != dst->rope_frac || src->rope_theta != dst->rope_theta ||
+      (src->k_eq_v != 0) != (dst->k_eq_v != 0))
     return fail(GEMMA_ERR_SHARE_MISMATCH,
-                "layers %d and %d differ in window, capacity, KV heads, head_dim or RoPE", src->layer,
-                dst->layer);
+                "layers %d and %d differ in window, capacity, KV heads, head_dim, RoPE or K = V",
+                src->layer, dst->layer);
   dst->k_cache = src->k_cache;
   dst->v_cache = src->v_cache;
   dst->shared_from = src->shared_from >= 0 ? src->shared_from : src->layer;
@@ -251,13 +275,10 @@ int gemma_attn_prefill(const void* q, const void* k_new, const void* v_new, void
                        unsigned flags, void* stream) {
   int rc = check_heads(n_q_heads, n_kv_heads, head_dim, window, rope_frac, rope_theta, scale);
   if (rc) return rc;
-  if (flags & ~GEMMA_F_SHARED) return fail(GEMMA_ERR_INVALID_ARG, "unknown flags 0x%x", flags);
+  rc = check_kv_flags(flags, window, k_new, v_new, k_cache, &v_cache);
+  if (rc) return rc;
   if (batch <= 0 || s_new < 0) return fail(GEMMA_ERR_INVALID_ARG, "batch %d, s_new %d", batch, s_new);
   const bool shared = flags & GEMMA_F_SHARED;
-  if (shared && (k_new || v_new))
-    return fail(GEMMA_ERR_INVALID_ARG, "GEMMA_F_SHARED: k_new and v_new must be NULL");
-  if (!shared && (!k_new || !v_new))
-    return fail(GEMMA_ERR_INVALID_ARG, "k_new and v_new are required unless GEMMA_F_SHARED");
   if (!q || !out || !k_cache || !v_cache) return fail(GEMMA_ERR_INVALID_ARG, "null tensor pointer");
   if (!aligned16(q) || !aligned16(out) || !aligned16(k_cache) || !aligned16(v_cache) ||
       (k_new && !aligned16(k_new)) || (v_new && !aligned16(v_new)) || !aligned16(workspace))
@@ -368,14 +389,10 @@ int gemma_attn_decode(const void* q, const void* k_new, const void* v_new, void*
                       void* stream) {
   int rc = check_heads(n_q_heads, n_kv_heads, head_dim, window, rope_frac, rope_theta, scale);
   if (rc) return rc;
-  if (flags & ~GEMMA_F_SHARED) return fail(GEMMA_ERR_INVALID_ARG, "unknown flags 0x%x", flags);
+  rc = check_kv_flags(flags, window, k_new, v_new, k_cache, &v_cache);
+  if (rc) return rc;
   if (batch <= 0 || max_seq_len <= 0)
     return fail(GEMMA_ERR_INVALID_ARG, "batch %d, max_seq_len %d", batch, max_seq_len);
-  const bool shared = flags & GEMMA_F_SHARED;
-  if (shared && (k_new || v_new))
-    return fail(GEMMA_ERR_INVALID_ARG, "GEMMA_F_SHARED: k_new and v_new must be NULL");
-  if (!shared && (!k_new || !v_new))
-    return fail(GEMMA_ERR_INVALID_ARG, "k_new and v_new are required unless GEMMA_F_SHARED");
   if (!q || !out || !k_cache || !v_cache || !seq_lens)
     return fail(GEMMA_ERR_INVALID_ARG, "null pointer argument");
   if (!aligned16(q) || !aligned16(out) || !aligned16(k_cache) || !aligned16(v_cache) ||
@@ -437,6 +454,7 @@ int gemma_attn_decode(const void* q, const void* k_new, const void* v_new, void*
   da.status = status;
   da.wait_ns = (unsigned long long)g_wait_ns.load();
   da.drop_first_copy = g_drop_next.exchange(0);
+  da.keqv = (flags & GEMMA_F_KEQV) ? 1 : 0;
   {
     ProfScope p_split(GEMMA_KERNEL_DECODE_SPLIT, st);
     e = launch_decode_split(da, batch, head_dim, st);

@@ -25,6 +25,8 @@
 //               B = K rows), online softmax in fp32 (log2 domain), then
 //               O^T += V^T P^T with the S accumulators reused directly as the
 //               B fragment of P^T (the GQA group is the MMA's N dimension).
+// K = V ("Gemma 4: End-to-End Architecture Walkthrough", 3b): only the K
+// rows are copied and the PV product reads them as V, halving the bytes.
 // The consumer warps' (m, l, O) merge in shared memory; each split writes its
 // normalised partial and its log2-sum-exp, and the combine kernel merges the
 // splits of a (sequence, head).
@@ -32,6 +34,8 @@
 // Every barrier wait is bounded (%globaltimer deadline). On a timeout the
 // CTA raises its abort flag, records GEMMA_ERR_DEVICE_TIMEOUT, waits (again
 // bounded) for its own copies still in flight, and exits without output.
+#include <algorithm>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -116,7 +120,10 @@ __global__ void __launch_bounds__(32 * (NCW + 1), 2) k_decode_split(DecodeAttnAr
   const int64_t k_begin = (int64_t)split * a.chunk;
   if (k_begin >= n_valid) return;
   const int64_t k_end = (k_begin + a.chunk < n_valid) ? k_begin + a.chunk : n_valid;
-  const int n_sub = (int)((k_end - k_begin + C::KB - 1) / C::KB);
+  // keys per ring slot: 16 K rows + 16 V rows, or 32 K rows under K = V
+  // (the same bytes per slot, so as many bytes stay in flight)
+  const int kps = a.keqv ? 2 * C::KB : C::KB;
+  const int n_sub = (int)((k_end - k_begin + kps - 1) / kps);
   const int64_t head_off = ((int64_t)b * a.Hkv + g) * (int64_t)a.cache_cap * D;
   const bf16* kbase = a.k_cache + head_off;
   const bf16* vbase = a.v_cache + head_off;
@@ -155,18 +162,18 @@ __global__ void __launch_bounds__(32 * (NCW + 1), 2) k_decode_split(DecodeAttnAr
       }
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) break;
-      const int64_t key0 = k_begin + (int64_t)t * C::KB;
-      const int nk = (int)((k_end - key0) < C::KB ? (k_end - key0) : C::KB);
+      const int64_t key0 = k_begin + (int64_t)t * kps;
+      const int nk = (int)((k_end - key0) < kps ? (k_end - key0) : kps);
       const bool drop = a.drop_first_copy && t == 0 && split == 0 && g == 0 && b == 0;
       if (drop) continue;
       if (lane == 0) {
-        mbar_arrive_expect_tx(&full[slot], (uint32_t)(2 * nk * D * 2));
+        mbar_arrive_expect_tx(&full[slot], (uint32_t)((a.keqv ? 1 : 2) * nk * D * 2));
         issued[slot] += 1;
       }
       __syncwarp();
-      const int r = lane & 15;
+      const int r = a.keqv ? lane : (lane & 15);
       if (r < nk) {
-        const bool isv = lane >= 16;
+        const bool isv = !a.keqv && lane >= 16;  // K = V: 32 K rows, which are the values
         bulk_g2s(ring + slot * C::SLOT_B + (isv ? C::KB * C::ROWB : 0) + r * C::ROWB,
                  (isv ? vbase : kbase) + (key0 + r) * D, D * 2, &full[slot]);
       }
@@ -186,20 +193,25 @@ __global__ void __launch_bounds__(32 * (NCW + 1), 2) k_decode_split(DecodeAttnAr
       const bool ok = mbar_wait_bounded_at(&full[slot], (t / C::NSLOT) & 1, abort_flag, deadline,
                                            a.status, 2, t, slot, warp);
       if (!__all_sync(0xffffffffu, ok)) break;
-      const int64_t key0 = k_begin + (int64_t)t * C::KB;
-      const int nk = (int)((k_end - key0) < C::KB ? (k_end - key0) : C::KB);
-      unsigned char* kslot = ring + slot * C::SLOT_B;
-      unsigned char* vslot = kslot + C::KB * C::ROWB;
-      if (nk < C::KB) {
+      const int64_t key0_slot = k_begin + (int64_t)t * kps;
+      const int nk_slot = (int)((k_end - key0_slot) < kps ? (k_end - key0_slot) : kps);
+      if (nk_slot < kps) {
         // rows past the end were not copied: make them finite zeros
-        for (int idx = lane; idx < (C::KB - nk) * (D / 8); idx += 32) {
-          const int r = nk + idx / (D / 8), c = (idx % (D / 8)) * 8;
-          *reinterpret_cast<uint4*>(kslot + r * C::ROWB + c * 2) = make_uint4(0, 0, 0, 0);
-          *reinterpret_cast<uint4*>(vslot + r * C::ROWB + c * 2) = make_uint4(0, 0, 0, 0);
+        unsigned char* rows = ring + slot * C::SLOT_B;
+        for (int idx = lane; idx < 2 * C::KB * (D / 8); idx += 32) {
+          const int r = idx / (D / 8), c = (idx % (D / 8)) * 8;
+          const int key = a.keqv ? r : (r & (C::KB - 1));  // K rows 0..15, V rows 16..31
+          if (key >= nk_slot) *reinterpret_cast<uint4*>(rows + r * C::ROWB + c * 2) = make_uint4(0, 0, 0, 0);
         }
         fence_proxy_async_smem();
         __syncwarp();
       }
+      // one 16-key sub-block per slot, or two under K = V
+      for (int half = 0; half < (a.keqv ? 2 : 1); ++half) {
+      const int nk = nk_slot - half * C::KB;
+      if (nk <= 0) break;
+      unsigned char* kslot = ring + slot * C::SLOT_B + half * C::KB * C::ROWB;
+      unsigned char* vslot = a.keqv ? kslot : kslot + C::KB * C::ROWB;
       // S = Q K^T : rows = query heads (8 real of 16), cols = 16 keys
       float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
       const uint32_t k_addr = smem_u32(kslot) + frag_off;
@@ -249,6 +261,7 @@ __global__ void __launch_bounds__(32 * (NCW + 1), 2) k_decode_split(DecodeAttnAr
         ldsm_x4_t(v_addr + mt * 32, va0, va1, va2, va3);
         mma_bf16(o[mt], va0, va1, va2, va3, pb0, pb1);
       }
+      }  // half
       __syncwarp();
       if (lane == 0) {
         consumed[slot] += 1;
@@ -319,35 +332,66 @@ __global__ void __launch_bounds__(32 * (NCW + 1), 2) k_decode_split(DecodeAttnAr
   }
 }
 
+// Log-sum-exp merge of the splits of one (sequence, q head): 128 threads =
+// 16 dim quads x 8 split lanes per 64 output dims, so the reads of a
+// split's partial are coalesced and the splits are summed in parallel. The
+// grid's z dimension splits the head dimension when there are few
+// (sequence, head) pairs. Split weights 2^(lse_s - M) are formed once per CTA.
 template <int D>
 __global__ void __launch_bounds__(128) k_decode_combine(DecodeAttnArgs a) {
+  extern __shared__ float w_s[];  // [n_splits]
+  __shared__ __align__(16) float red[8][64];
+  __shared__ float rmax[4], rsum[4];
   const int h = blockIdx.x, b = blockIdx.y;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   bf16* dst = a.out + ((int64_t)b * a.Hq + h) * D;
   const int64_t len = a.seq_lens[b];
   if (len < 1 || len > a.max_len) {
-    for (int d = threadIdx.x; d < D; d += blockDim.x) dst[d] = __float2bfloat16(0.f);
+    for (int d = blockIdx.z * 64 + tid; d < D; d += gridDim.z * 64)
+      if (tid < 64) dst[d] = __float2bfloat16(0.f);
     return;
   }
   const int64_t n_valid = a.window > 0 ? (len < a.window ? len : (int64_t)a.window) : len;
   const int n_used = (int)((n_valid + a.chunk - 1) / a.chunk);
   const int64_t pr0 = ((int64_t)b * a.Hq + h) * a.n_splits;
-  float M = -INFINITY;
-  for (int s = 0; s < n_used; ++s) M = fmaxf(M, a.part_lse[pr0 + s]);
-  float wsum = 0.f;
-  for (int s = 0; s < n_used; ++s) wsum += exp2f(a.part_lse[pr0 + s] - M);
-  const float inv = 1.f / wsum;
-  for (int d = threadIdx.x * 4; d < D; d += blockDim.x * 4) {
+  float m = -INFINITY;
+  for (int s = tid; s < n_used; s += 128) m = fmaxf(m, a.part_lse[pr0 + s]);
+#pragma unroll
+  for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if (lane == 0) rmax[warp] = m;
+  __syncthreads();
+  const float M = fmaxf(fmaxf(rmax[0], rmax[1]), fmaxf(rmax[2], rmax[3]));
+  float sum = 0.f;
+  for (int s = tid; s < n_used; s += 128) {
+    const float w = exp2f(a.part_lse[pr0 + s] - M);
+    w_s[s] = w;
+    sum += w;
+  }
+#pragma unroll
+  for (int o = 16; o; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+  if (lane == 0) rsum[warp] = sum;
+  __syncthreads();
+  const float inv = 1.f / ((rsum[0] + rsum[1]) + (rsum[2] + rsum[3]));
+  const int q = tid & 15, sl = tid >> 4;
+  for (int d0 = blockIdx.z * 64; d0 < D; d0 += gridDim.z * 64) {
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int s = 0; s < n_used; ++s) {
-      const float w = exp2f(a.part_lse[pr0 + s] - M);
-      const float4 v = *reinterpret_cast<const float4*>(a.part_o + (pr0 + s) * D + d);
+    for (int s = sl; s < n_used; s += 8) {
+      const float w = w_s[s];
+      const float4 v = *reinterpret_cast<const float4*>(a.part_o + (pr0 + s) * D + d0 + q * 4);
       acc.x += w * v.x;
       acc.y += w * v.y;
       acc.z += w * v.z;
       acc.w += w * v.w;
     }
-    uint2 pk = make_uint2(pack_bf16x2(acc.x * inv, acc.y * inv), pack_bf16x2(acc.z * inv, acc.w * inv));
-    *reinterpret_cast<uint2*>(dst + d) = pk;
+    *reinterpret_cast<float4*>(&red[sl][q * 4]) = acc;
+    __syncthreads();
+    if (tid < 64) {
+      float t = 0.f;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) t += red[k][tid];
+      dst[d0 + tid] = __float2bfloat16(t * inv);
+    }
+    __syncthreads();  // red is reused by the next 64 dims
   }
 }
 
@@ -368,11 +412,16 @@ cudaError_t launch_decode_split(const DecodeAttnArgs& a, int B, int D, cudaStrea
 }
 
 cudaError_t launch_decode_combine(const DecodeAttnArgs& a, int B, int D, cudaStream_t st) {
-  dim3 grid(a.Hq, B);
+  // enough CTAs for about eight per SM, at most one per 64 output dims
+  const int pairs = a.Hq * B;
+  const int nz = std::max(1, std::min(D / 64, (8 * 148 + pairs - 1) / pairs));
+  dim3 grid(a.Hq, B, nz);
+  const size_t smem = (size_t)a.n_splits * sizeof(float);
+  if (smem > 48 * 1024) return cudaErrorInvalidValue;  // > 12288 splits: not planned by decode_plan
   if (D == 256)
-    k_decode_combine<256><<<grid, 64, 0, st>>>(a);
+    k_decode_combine<256><<<grid, 128, smem, st>>>(a);
   else
-    k_decode_combine<512><<<grid, 128, 0, st>>>(a);
+    k_decode_combine<512><<<grid, 128, smem, st>>>(a);
   return cudaGetLastError();
 }
 

@@ -78,6 +78,7 @@ struct DecodeAttnArgs {
   int* status;
   unsigned long long wait_ns;
   int drop_first_copy;     // test hook: skip the first K/V copy of split 0
+  int keqv;                // K = V: only K rows are loaded and serve as V
 };
 
 cudaError_t launch_prefill_rope(const PrefillRopeArgs& a, int B, int D, cudaStream_t st);

@@ -166,7 +166,7 @@ __global__ void __launch_bounds__(256, 2) k_prefill_rope(PrefillRopeArgs a) {
 #pragma unroll 1
     for (int h0 = 0; h0 < a.Hkv; h0 += ROPE_HB / 2) {
       uint4 kx[ROPE_HB / 2], vx[ROPE_HB / 2];
-      const bool want_v = a.window == 0 || to_ring;
+      const bool want_v = a.v_new && (a.window == 0 || to_ring);  // no v_new: K = V
 #pragma unroll
       for (int u = 0; u < ROPE_HB / 2; ++u)
         if (h0 + u < a.Hkv) {
@@ -182,12 +182,12 @@ __global__ void __launch_bounds__(256, 2) k_prefill_rope(PrefillRopeArgs a) {
           const int64_t cslot = (((int64_t)b * a.Hkv + kh) * a.cache_cap + slot) * D + e0;
           if (a.window == 0) {
             st16(a.k_cache + cslot, kr);
-            st16(a.v_cache + cslot, vx[u]);
+            if (want_v) st16(a.v_cache + cslot, vx[u]);
           } else {
             st16(a.k_rot + (row * a.Hkv + kh) * D + e0, kr);
             if (to_ring) {
               st16(a.k_cache + cslot, kr);
-              st16(a.v_cache + cslot, vx[u]);
+              if (want_v) st16(a.v_cache + cslot, vx[u]);
             }
           }
         }
@@ -214,7 +214,8 @@ __global__ void __launch_bounds__(256) k_decode_rope_append(DecodeRopeArgs a) {
   double inv_freq[4];
   chunk_inv_freq(e0, D, a.n_rot, a.log2_theta, inv_freq);
   const PairTrig t = chunk_trig(pos, e0, a.n_rot, inv_freq);
-  const int n_heads = a.Hq + (a.k_new ? 2 * a.Hkv : 0);
+  // q heads, then K heads, then V heads (none when shared, none for V under K = V)
+  const int n_heads = a.Hq + (a.k_new ? a.Hkv : 0) + (a.v_new ? a.Hkv : 0);
   for (int h = threadIdx.y; h < n_heads; h += blockDim.y) {
     if (h < a.Hq) {
       const int64_t off = ((int64_t)b * a.Hq + h) * D + e0;

@@ -30,6 +30,7 @@ GEMMA_ERR_CUDA = 5
 GEMMA_ERR_DEVICE_TIMEOUT = 6
 GEMMA_ERR_DEVICE_RANGE = 7
 GEMMA_F_SHARED = 1
+GEMMA_F_KEQV = 2  # K = V on a global layer: no v_new, values read from the key cache
 
 _P = ctypes.c_void_p
 _I = ctypes.c_int
@@ -40,7 +41,7 @@ _SZ = ctypes.c_size_t
 class gemma_kv_desc(ctypes.Structure):
     _fields_ = [("k_cache", _P), ("v_cache", _P), ("layer", _I), ("cache_cap", _I),
                 ("window", _I), ("n_kv_heads", _I), ("head_dim", _I), ("rope_frac", _F),
-                ("rope_theta", _F), ("shared_from", _I)]
+                ("rope_theta", _F), ("shared_from", _I), ("k_eq_v", _I)]
 
 
 def _sig(name, restype, argtypes):

@@ -38,6 +38,7 @@ class AttentionStack:
             d.layer, d.cache_cap, d.window = l, cap, t.window
             d.n_kv_heads, d.head_dim = t.n_kv_heads, t.head_dim
             d.rope_frac, d.rope_theta, d.shared_from = t.rope_frac, t.rope_theta, -1
+            d.k_eq_v = int(self.keqv(l))
             src = self.share_src[l]
             if src >= 0 and src != l:
                 native.gemma_kv_share_bind(d, self.descs[src])
@@ -47,8 +48,9 @@ class AttentionStack:
                 shape = (w.batch, t.n_kv_heads, cap, t.head_dim)
                 if alloc_caches:
                     kc = torch.empty(shape, dtype=torch.bfloat16, device=self.device)
-                    vc = torch.empty(shape, dtype=torch.bfloat16, device=self.device)
-                    d.k_cache, d.v_cache = kc.data_ptr(), vc.data_ptr()
+                    # K = V: the key cache is the only cache
+                    vc = kc if d.k_eq_v else torch.empty(shape, dtype=torch.bfloat16, device=self.device)
+                    d.k_cache, d.v_cache = kc.data_ptr(), (0 if d.k_eq_v else vc.data_ptr())
                 else:
                     kc = vc = None
                 self.k_cache.append(kc)
@@ -57,6 +59,10 @@ class AttentionStack:
 
     def layer_type(self, l: int) -> LayerType:
         return self.w.global_ if self.is_global[l] else self.w.local
+
+    def keqv(self, l: int) -> bool:
+        """Global layers of a K = V workload read their values from the key cache."""
+        return bool(self.w.k_eq_v and self.is_global[l])
 
     def is_shared(self, l: int) -> bool:
         return self.descs[l].shared_from >= 0
@@ -68,7 +74,7 @@ class AttentionStack:
             if kc is None or kc.data_ptr() in seen:
                 continue
             seen.add(kc.data_ptr())
-            total += 2 * kc.numel() * kc.element_size()
+            total += (1 if self.keqv(l) else 2) * kc.numel() * kc.element_size()
         return total
 
     # ------------------------------------------------------------------ prefill
@@ -82,11 +88,14 @@ class AttentionStack:
                       stream=None):
         t = self.layer_type(l)
         shared = self.is_shared(l)
+        keqv = self.keqv(l)
         native.gemma_attn_prefill(
-            q, None if shared else k, None if shared else v, self.k_cache[l], self.v_cache[l],
+            q, None if shared else k, None if (shared or keqv) else v, self.k_cache[l],
+            None if keqv else self.v_cache[l],
             window=t.window, rope_frac=t.rope_frac, rope_theta=t.rope_theta, scale=t.scale,
             out=out, seq_lens_before=seq_lens_before, lse=lse, workspace=workspace,
-            flags=native.GEMMA_F_SHARED if shared else 0, stream=stream)
+            flags=(native.GEMMA_F_SHARED if shared else 0) | (native.GEMMA_F_KEQV if keqv else 0),
+            stream=stream)
 
     # ------------------------------------------------------------------ decode
     def decode_workspace_bytes(self, max_seq_len: int) -> int:
@@ -98,8 +107,11 @@ class AttentionStack:
     def decode_layer(self, l: int, q, k, v, out, *, seq_lens, max_seq_len, workspace, stream=None):
         t = self.layer_type(l)
         shared = self.is_shared(l)
+        keqv = self.keqv(l)
         native.gemma_attn_decode(
-            q, None if shared else k, None if shared else v, self.k_cache[l], self.v_cache[l],
+            q, None if shared else k, None if (shared or keqv) else v, self.k_cache[l],
+            None if keqv else self.v_cache[l],
             seq_lens=seq_lens, max_seq_len=max_seq_len, window=t.window, rope_frac=t.rope_frac,
             rope_theta=t.rope_theta, scale=t.scale, out=out, workspace=workspace,
-            flags=native.GEMMA_F_SHARED if shared else 0, stream=stream)
+            flags=(native.GEMMA_F_SHARED if shared else 0) | (native.GEMMA_F_KEQV if keqv else 0),
+            stream=stream)

@@ -45,6 +45,7 @@ class Workload:
     k_scale: float = 1.0         # K drawn as N(0, k_scale^2)
     seed: int = 0
     fixed_kinds: tuple = ()      # overrides the schedule: e.g. ("local",) for one local layer
+    k_eq_v: bool = False         # global layers use K = V (values are the cached keys)
     description: str = field(default="", compare=False)
 
 
@@ -80,6 +81,11 @@ WORKLOADS = {
         "global_s16384", "prefill", batch=1, n_q_heads=32, n_layers=1, ratio=0,
         local=L31B_LOCAL, global_=L31B_GLOBAL, seq=16384, seed=5, fixed_kinds=("global",),
         description="one 31B-shaped global layer, B1 S16384 Hq32 Hkv4 D512 (a kernel-profiling case)"),
+    "global_decode_256k_keqv": Workload(
+        "global_decode_256k_keqv", "decode", batch=1, n_q_heads=32, n_layers=1, ratio=0,
+        local=L31B_LOCAL, global_=L31B_GLOBAL, len_lo=262144, len_hi=262144, seed=6,
+        fixed_kinds=("global",), k_eq_v=True,
+        description="single-token decode at KV length 262144, one global layer with K = V"),
     "global_decode_256k": Workload(
         "global_decode_256k", "decode", batch=1, n_q_heads=32, n_layers=1, ratio=0,
         local=L31B_LOCAL, global_=L31B_GLOBAL, len_lo=262144, len_hi=262144, seed=4,

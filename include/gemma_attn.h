@@ -67,6 +67,14 @@ typedef enum gemma_status {
 #define GEMMA_F_SHARED 1u /* k_cache/v_cache alias an earlier layer (see
                              gemma_kv_share_bind): k_new and v_new must be NULL;
                              nothing is rotated or written into the cache. */
+#define GEMMA_F_KEQV 2u   /* K = V ("Gemma 4: End-to-End Architecture
+                             Walkthrough", 3b "K = V"; "Gemma 4 Technical Report"
+                             summary, Core Model Architecture: only K is cached
+                             and the attention weights multiply K). Global
+                             layers only (window 0, else GEMMA_ERR_UNSUPPORTED).
+                             v_new must be NULL; v_cache must be NULL or equal
+                             k_cache. The values are the keys as the cache holds
+                             them (rotated); nothing is written for V. */
 
 /* Supported shapes: head_dim 256 or 512; n_q_heads a multiple of n_kv_heads
  * with n_q_heads / n_kv_heads <= 8; window 0 (global) or a multiple of 16. */
@@ -183,12 +191,13 @@ typedef struct gemma_kv_desc {
     float rope_frac;
     float rope_theta;
     int shared_from;    /* -1: owns its cache; else the layer whose cache it reads */
+    int k_eq_v;         /* 1: a GEMMA_F_KEQV layer (v_cache may be NULL) */
 } gemma_kv_desc;
 
 /* Makes dst read src's cache: dst->k_cache/v_cache become src's pointers and
  * dst->shared_from the layer that owns them (a chain resolves to its root).
  * Requires src->layer < dst->layer and identical window, cache_cap,
- * n_kv_heads, head_dim, rope_frac and rope_theta (same attention type);
+ * n_kv_heads, head_dim, rope_frac, rope_theta and k_eq_v (same attention type);
  * otherwise returns GEMMA_ERR_SHARE_MISMATCH and leaves dst unchanged.
  * Afterwards call the attention entry points for dst with GEMMA_F_SHARED. */
 int gemma_kv_share_bind(gemma_kv_desc* dst, const gemma_kv_desc* src);

@@ -44,10 +44,11 @@ def test_schedule_rejects_bad_arguments():
         assert e.value.code == native.GEMMA_ERR_INVALID_ARG
 
 
-def _desc(layer, window, cap, hkv=4, d=512, frac=0.25, theta=1e6, k=FAKE, v=FAKE + 0x1000):
+def _desc(layer, window, cap, hkv=4, d=512, frac=0.25, theta=1e6, k=FAKE, v=FAKE + 0x1000, keqv=0):
     x = native.gemma_kv_desc()
     x.k_cache, x.v_cache, x.layer, x.cache_cap, x.window = k, v, layer, cap, window
     x.n_kv_heads, x.head_dim, x.rope_frac, x.rope_theta, x.shared_from = hkv, d, frac, theta, -1
+    x.k_eq_v = keqv
     return x
 
 
@@ -59,6 +60,20 @@ def test_share_bind_aliases_and_resolves_chains():
     dst2 = _desc(13, 0, 4096, k=None, v=None)
     native.gemma_kv_share_bind(dst2, dst)           # chain resolves to the root
     assert dst2.shared_from == 5 and dst2.k_cache == src.k_cache
+
+
+def test_share_bind_k_equals_v():
+    """A K = V source has no value cache; its sharer aliases the key cache,
+    and a K = V layer only aliases a K = V layer."""
+    src = _desc(5, 0, 4096, v=None, keqv=1)
+    dst = _desc(11, 0, 4096, k=None, v=None, keqv=1)
+    native.gemma_kv_share_bind(dst, src)
+    assert dst.k_cache == src.k_cache and not dst.v_cache and dst.shared_from == 5
+    for a, b in ((_desc(5, 0, 4096), _desc(11, 0, 4096, k=None, v=None, keqv=1)),
+                 (_desc(5, 0, 4096, v=None, keqv=1), _desc(11, 0, 4096, k=None, v=None))):
+        with pytest.raises(native.GemmaError) as e:
+            native.gemma_kv_share_bind(b, a)
+        assert e.value.code in (native.GEMMA_ERR_SHARE_MISMATCH, native.GEMMA_ERR_INVALID_ARG)
 
 
 @pytest.mark.parametrize("change", ["type", "window", "heads", "dim", "frac", "theta", "order", "cap"])
@@ -125,6 +140,10 @@ E = native
     (dict(k=None), E.GEMMA_ERR_INVALID_ARG),           # unshared layer without new keys
     (dict(flags=1), E.GEMMA_ERR_INVALID_ARG),          # shared layer with new keys
     (dict(flags=4), E.GEMMA_ERR_INVALID_ARG),
+    (dict(flags=2, v=None), E.GEMMA_ERR_UNSUPPORTED),  # K = V on a local layer
+    (dict(W=0, cap=4096, flags=2), E.GEMMA_ERR_INVALID_ARG),             # K = V with v_new
+    (dict(W=0, cap=4096, flags=2, v=None, vc=FAKE + 256), E.GEMMA_ERR_INVALID_ARG),  # v_cache != k_cache
+    (dict(W=0, cap=4096, flags=3, k=None, v=None, vc=None, wsb=16), E.GEMMA_ERR_CAPACITY),  # shared K = V: flags pass
     (dict(q=None), E.GEMMA_ERR_INVALID_ARG),
     (dict(q=FAKE + 8), E.GEMMA_ERR_INVALID_ARG),       # misaligned
     (dict(wsb=16), E.GEMMA_ERR_CAPACITY),
@@ -144,6 +163,10 @@ def test_prefill_validation(over, code):
     (dict(k=None, v=None, flags=0), E.GEMMA_ERR_INVALID_ARG),
     (dict(wsb=1024), E.GEMMA_ERR_CAPACITY),
     (dict(out=None), E.GEMMA_ERR_INVALID_ARG),
+    (dict(flags=2), E.GEMMA_ERR_INVALID_ARG),                          # K = V with v_new
+    (dict(flags=2, v=None, vc=FAKE + 256), E.GEMMA_ERR_INVALID_ARG),   # v_cache != k_cache
+    (dict(W=1024, cap=1024, flags=2, v=None), E.GEMMA_ERR_UNSUPPORTED),
+    (dict(flags=2, v=None, vc=None, wsb=1024), E.GEMMA_ERR_CAPACITY),  # K = V accepted: v_cache optional
 ])
 def test_decode_validation(over, code):
     assert _decode_raw(**over) == code

@@ -52,7 +52,7 @@ def fill_cache_for_lengths(kc, vc, lens, window, g):
 
 
 def run_decode_case(oracle, *, lens, Hq, Hkv, D, W, frac, theta, seed, q_scale=1.0,
-                    tol=(2e-2, 2e-3), shared=False):
+                    tol=(2e-2, 2e-3), shared=False, keqv=False):
     dev = torch.device("cuda")
     B = len(lens)
     g = synth.generator(seed)
@@ -71,20 +71,25 @@ def run_decode_case(oracle, *, lens, Hq, Hkv, D, W, frac, theta, seed, q_scale=1
             slot = p % W if W else p
             kc[b, :, slot] = kn[b]
             vc[b, :, slot] = vn[b]
-    kcd, vcd = kc.to(dev), vc.to(dev)
+    if keqv:
+        vc, vn = kc, kn  # K = V: one cache; the oracle takes the values from the keys
+    kcd = kc.to(dev)
+    vcd = kcd if keqv else vc.to(dev)
     out = torch.full((B, Hq, D), float("nan"), dtype=torch.bfloat16, device=dev)
     sl = torch.tensor(lens, dtype=torch.int32, device=dev)
     scale = 1.0 / math.sqrt(D)
-    native.gemma_attn_decode(q.to(dev), None if shared else kn.to(dev), None if shared else vn.to(dev),
-                             kcd, vcd, seq_lens=sl, max_seq_len=max_len, window=W, rope_frac=frac,
-                             rope_theta=theta, scale=scale, out=out,
-                             flags=native.GEMMA_F_SHARED if shared else 0)
+    flags = (native.GEMMA_F_SHARED if shared else 0) | (native.GEMMA_F_KEQV if keqv else 0)
+    native.gemma_attn_decode(q.to(dev), None if shared else kn.to(dev),
+                             None if (shared or keqv) else vn.to(dev), kcd, None if keqv else vcd,
+                             seq_lens=sl, max_seq_len=max_len, window=W, rope_frac=frac,
+                             rope_theta=theta, scale=scale, out=out, flags=flags)
     assert native.gemma_attn_sync_status() == 0, native.gemma_last_error()
     kc1, vc1 = kcd.cpu(), vcd.cpu()
     for b in range(B):
         L = lens[b]
         kl, vl = logical_kv(kc[b], vc[b], L, W, kn[b], vn[b])
-        ref, _ = oracle.attention(to_bits(q[b].reshape(1, 1, Hq, D)), to_bits(kl[None]), to_bits(vl[None]),
+        ref, _ = oracle.attention(to_bits(q[b].reshape(1, 1, Hq, D)), to_bits(kl[None]),
+                                  None if keqv else to_bits(vl[None]),
                                   q_pos0=L - 1, n_keys=L, rot_from=L if shared else L - 1, window=W,
                                   rope_frac=frac, theta=theta, scale=scale)
         got = out[b].float().cpu().double().numpy()
@@ -93,7 +98,8 @@ def run_decode_case(oracle, *, lens, Hq, Hkv, D, W, frac, theta, seed, q_scale=1
         if shared:
             assert torch.equal(kc1[b], kc[b]) and torch.equal(vc1[b], vc[b])
         else:
-            assert torch.equal(vc1[b, :, slot], vn[b])
+            if not keqv:
+                assert torch.equal(vc1[b, :, slot], vn[b])
             for h in range(Hkv):
                 exp = torch.from_numpy(oracle.rope_bf16(to_bits(kn[b, h]), L - 1, frac, theta)).to(torch.bfloat16)
                 assert_rotated_bf16(kc1[b, h, slot], exp, kn[b, h], "new K slot")
@@ -123,6 +129,18 @@ def test_decode_shared_layer(oracle):
                     shared=True)
     run_decode_case(oracle, lens=[900, 33], Hq=8, Hkv=4, D=256, W=64, frac=1.0, theta=1e4, seed=208,
                     shared=True)
+
+
+@pytest.mark.parametrize("case", [
+    dict(lens=[1, 37, 300, 2049], Hq=8, Hkv=1, D=512, W=0, frac=0.25, theta=1e6, seed=211),
+    dict(lens=[4097, 2], Hq=32, Hkv=4, D=512, W=0, frac=0.25, theta=1e6, seed=212),
+    dict(lens=[130, 17], Hq=4, Hkv=2, D=256, W=0, frac=1.0, theta=1e4, seed=213),
+], ids=["Hq8", "Hq32", "D256"])
+def test_decode_k_equals_v(oracle, case):
+    """K = V (GEMMA_F_KEQV): only the key is appended and the rotated keys in
+    the cache serve as values; the oracle takes its values from the keys."""
+    run_decode_case(oracle, keqv=True, **case)
+    run_decode_case(oracle, keqv=True, shared=True, **dict(case, seed=case["seed"] + 100))
 
 
 def test_decode_peaky(oracle):
@@ -226,7 +244,8 @@ def _decode_workload(oracle, name, n_sample):
                 kl, vl = logical_kv(kc_b, vc_b, L, t.window, kn[b].cpu(), vn[b].cpu())
                 rot_from = L - 1
             ref, _ = oracle.attention(to_bits(q[b].cpu().reshape(1, 1, w.n_q_heads, D)), to_bits(kl[None]),
-                                      to_bits(vl[None]), q_pos0=L - 1, n_keys=L, rot_from=rot_from,
+                                      None if st.keqv(l) else to_bits(vl[None]),
+                                      q_pos0=L - 1, n_keys=L, rot_from=rot_from,
                                       window=t.window, rope_frac=t.rope_frac, theta=t.rope_theta,
                                       scale=t.scale)
             assert_close(out[b].float().cpu().double().numpy(), ref, what="%s layer %d b=%d" % (name, l, b))
@@ -235,6 +254,10 @@ def _decode_workload(oracle, name, n_sample):
 
 def test_decode_31b_b64(oracle):
     _decode_workload(oracle, "31b_decode_b64", n_sample=8)
+
+
+def test_decode_global_256k_k_equals_v(oracle):
+    _decode_workload(oracle, "global_decode_256k_keqv", n_sample=1)
 
 
 def test_decode_global_256k(oracle):

@@ -23,7 +23,8 @@ def _expected_rotated_bf16(oracle, k_bits_row, pos, frac, theta):
 
 
 def run_prefill_case(oracle, *, B, S, Hq, Hkv, D, W, frac, theta, seed, prior=None, q_scale=1.0,
-                     k_scale=1.0, tol=(2e-2, 2e-3), check_cache=True, check_lse=True, cache_fill=0.0):
+                     k_scale=1.0, tol=(2e-2, 2e-3), check_cache=True, check_lse=True, cache_fill=0.0,
+                     keqv=False):
     dev = torch.device("cuda")
     g = synth.generator(seed)
     q = synth.randn_bf16((B, S, Hq, D), g, scale=q_scale)
@@ -40,14 +41,19 @@ def run_prefill_case(oracle, *, B, S, Hq, Hkv, D, W, frac, theta, seed, prior=No
         if prior[b]:
             kc[b, :, :prior[b]] = synth.randn_bf16((Hkv, prior[b], D), g)
             vc[b, :, :prior[b]] = synth.randn_bf16((Hkv, prior[b], D), g)
+    if keqv:
+        vc = kc  # K = V: one cache, and the values are the cached (rotated) keys
     kc0, vc0 = kc.clone(), vc.clone()
-    qd, kd, vd, kcd, vcd = (x.to(dev) for x in (q, k, v, kc, vc))
+    qd, kd, vd, kcd = (x.to(dev) for x in (q, k, v, kc))
+    vcd = kcd if keqv else vc.to(dev)
     out = torch.full((B, S, Hq, D), float("nan"), dtype=torch.bfloat16, device=dev)
     lse = torch.full((B, Hq, S), float("nan"), dtype=torch.float32, device=dev)
     lens = torch.tensor(prior, dtype=torch.int32, device=dev) if any(prior) else None
     scale = 1.0 / math.sqrt(D)
-    native.gemma_attn_prefill(qd, kd, vd, kcd, vcd, window=W, rope_frac=frac, rope_theta=theta,
-                              scale=scale, out=out, seq_lens_before=lens, lse=lse)
+    native.gemma_attn_prefill(qd, kd, None if keqv else vd, kcd, None if keqv else vcd, window=W,
+                              rope_frac=frac, rope_theta=theta, scale=scale, out=out,
+                              seq_lens_before=lens, lse=lse,
+                              flags=native.GEMMA_F_KEQV if keqv else 0)
     assert native.gemma_attn_sync_status() == 0, native.gemma_last_error()
 
     # oracle on logical K/V: cached prefix (already rotated) + the new keys
@@ -58,7 +64,7 @@ def run_prefill_case(oracle, *, B, S, Hq, Hkv, D, W, frac, theta, seed, prior=No
         v_log[b, :prior[b]] = vc0[b, :, :prior[b]].transpose(0, 1)
         k_log[b, prior[b]:prior[b] + S] = k[b]
         v_log[b, prior[b]:prior[b] + S] = v[b]
-    ref, ref_lse = oracle.attention(to_bits(q), to_bits(k_log), to_bits(v_log), q_pos0=prior,
+    ref, ref_lse = oracle.attention(to_bits(q), to_bits(k_log), None if keqv else to_bits(v_log), q_pos0=prior,
                                     n_keys=[p + S for p in prior], rot_from=prior, window=W,
                                     rope_frac=frac, theta=theta, scale=scale)
     got = out.float().cpu().double().numpy().transpose(0, 2, 1, 3).reshape(-1, D)  # (b, h, i) rows
@@ -76,7 +82,8 @@ def run_prefill_case(oracle, *, B, S, Hq, Hkv, D, W, frac, theta, seed, prior=No
                 if W and s < S - W:
                     continue
                 slot = pos % W if W else pos
-                assert torch.equal(vc1[b, :, slot], v[b, s]), "V slot %d" % slot
+                if not keqv:
+                    assert torch.equal(vc1[b, :, slot], v[b, s]), "V slot %d" % slot
                 for h in range(Hkv):
                     exp = _expected_rotated_bf16(oracle, to_bits(k[b, s, h]), pos, frac, theta)
                     got_k = kc1[b, h, slot]
@@ -138,6 +145,22 @@ def test_prefill_each_kernel(oracle, monkeypatch, kernel, case):
     sequence end must not let them reach an output)."""
     monkeypatch.setenv("GEMMA_PREFILL_KERNEL", kernel)
     run_prefill_case(oracle, **case)
+
+
+KEQV_CASES = [
+    dict(B=1, S=300, Hq=8, Hkv=1, D=512, W=0, frac=0.25, theta=1e6, seed=121, cache_fill=float("nan")),
+    dict(B=2, S=100, Hq=8, Hkv=1, D=512, W=0, frac=0.25, theta=1e6, seed=122, prior=[37, 250]),
+    dict(B=1, S=200, Hq=4, Hkv=2, D=256, W=0, frac=1.0, theta=1e4, seed=123, cache_fill=float("nan")),
+]
+
+
+@pytest.mark.parametrize("kernel", ["single", "pair"])
+@pytest.mark.parametrize("case", KEQV_CASES, ids=["D512", "D512P", "D256"])
+def test_prefill_k_equals_v(oracle, monkeypatch, kernel, case):
+    """K = V (GEMMA_F_KEQV) on global layers: only the rotated keys are written
+    and they serve as values; the oracle takes its values from the keys."""
+    monkeypatch.setenv("GEMMA_PREFILL_KERNEL", kernel)
+    run_prefill_case(oracle, keqv=True, **case)
 
 
 def test_prefill_local_s1024_full(oracle):
