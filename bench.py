@@ -231,22 +231,17 @@ def bench_prefill(args, w, dev, world, peaks):
 
 
 def e2e_prefill(args, st, layers, ws, lens, flops, world):
-    """Same step through the C ABI with host-resident inputs: pinned host ->
-    device copies of every layer's q/k/v and a device -> host read of every
-    output inside the timed region."""
+    """Same step through the public API with host-resident inputs:
+    AttentionStack.prefill_from_host copies every layer's q/k/v from pinned
+    host memory and every output back inside the timed region, overlapping
+    the two copy directions with the attention on separate streams."""
     host_in = [tuple(x.cpu().pin_memory() for x in (q, k, v)) for (q, k, v, _) in layers]
     host_out = [torch.empty(out.shape, dtype=out.dtype, pin_memory=True) for (_, _, _, out) in layers]
     h2d = sum(x.numel() * x.element_size() for t in host_in for x in t)
     d2h = sum(x.numel() * x.element_size() for x in host_out)
 
     def step():
-        for l, ((hq, hk, hv), (q, k, v, out)) in enumerate(zip(host_in, layers)):
-            q.copy_(hq, non_blocking=True)
-            k.copy_(hk, non_blocking=True)
-            v.copy_(hv, non_blocking=True)
-            st.prefill_layer(l, q, k, v, out, workspace=ws, seq_lens_before=lens)
-        for (_, _, _, out), ho in zip(layers, host_out):
-            ho.copy_(out, non_blocking=True)
+        st.prefill_from_host(host_in, host_out, layers, workspace=ws, seq_lens_before=lens)
 
     for _ in range(max(1, args.warmup)):
         step()

@@ -97,6 +97,44 @@ class AttentionStack:
             flags=(native.GEMMA_F_SHARED if shared else 0) | (native.GEMMA_F_KEQV if keqv else 0),
             stream=stream)
 
+    def prefill_from_host(self, host_in, host_out, dev_bufs, *, workspace, seq_lens_before=None):
+        """One prefill pass of every layer on inputs in pinned host memory.
+
+        host_in[l] = (q, k, v) pinned host tensors; host_out[l] a pinned host
+        tensor for layer l's output; dev_bufs[l] = (q, k, v, out) device
+        buffers of the same shapes. The host->device copies of layer l+1's
+        inputs and the device->host copy of layer l-1's output run on their
+        own streams while layer l computes, so the two copy directions and
+        the attention overlap. Work is ordered after everything already on
+        the current stream, and the current stream waits for the last
+        output copy: synchronising the current stream covers the whole pass.
+        """
+        comp = torch.cuda.current_stream(self.device)
+        if not hasattr(self, "_copy_streams"):
+            self._copy_streams = (torch.cuda.Stream(self.device), torch.cuda.Stream(self.device))
+        s_in, s_out = self._copy_streams
+        s_in.wait_stream(comp)   # earlier computes are done with the input buffers
+        s_out.wait_stream(comp)
+        ready = []
+        with torch.cuda.stream(s_in):
+            for (hq, hk, hv), (q, k, v, _) in zip(host_in, dev_bufs):
+                q.copy_(hq, non_blocking=True)
+                k.copy_(hk, non_blocking=True)
+                v.copy_(hv, non_blocking=True)
+                e = torch.cuda.Event()
+                e.record(s_in)
+                ready.append(e)
+        for l, (q, k, v, out) in enumerate(dev_bufs):
+            comp.wait_event(ready[l])
+            self.prefill_layer(l, q, k, v, out, workspace=workspace, seq_lens_before=seq_lens_before,
+                               stream=comp)
+            done = torch.cuda.Event()
+            done.record(comp)
+            s_out.wait_event(done)
+            with torch.cuda.stream(s_out):
+                host_out[l].copy_(out, non_blocking=True)
+        comp.wait_stream(s_out)
+
     # ------------------------------------------------------------------ decode
     def decode_workspace_bytes(self, max_seq_len: int) -> int:
         w = self.w

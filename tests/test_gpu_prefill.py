@@ -299,3 +299,38 @@ def test_prefill_31b_block_s32768(oracle):
 
 def test_prefill_global_chunk_256k(oracle):
     _run_block(oracle, "global_chunk_256k", n_random=48)
+
+
+def test_prefill_from_host_matches_layer_by_layer():
+    """AttentionStack.prefill_from_host (copies on their own streams,
+    overlapped with the attention) gives bit-identical outputs to copying
+    everything first and running the layers one by one."""
+    from hybrid_local_global_b200.workloads import E2B_GLOBAL, E2B_LOCAL, Workload
+    w = Workload("tiny_block", "prefill", batch=1, n_q_heads=8, n_layers=5, ratio=4,
+                 local=E2B_LOCAL, global_=E2B_GLOBAL, seq=700, seed=9)
+    dev = torch.device("cuda")
+    st = AttentionStack(w, dev)
+    g = synth.generator(9)
+    host_in, host_out, bufs = [], [], []
+    for l in range(st.n_layers):
+        t = st.layer_type(l)
+        shp_q = (w.batch, w.seq, w.n_q_heads, t.head_dim)
+        shp_k = (w.batch, w.seq, t.n_kv_heads, t.head_dim)
+        hin = tuple(synth.randn_bf16(s, g).pin_memory() for s in (shp_q, shp_k, shp_k))
+        host_in.append(hin)
+        host_out.append(torch.empty(shp_q, dtype=torch.bfloat16).pin_memory())
+        bufs.append(tuple(torch.empty(x.shape, dtype=x.dtype, device=dev) for x in hin) +
+                    (torch.empty(shp_q, dtype=torch.bfloat16, device=dev),))
+    ws = torch.empty(st.prefill_workspace_bytes(), dtype=torch.uint8, device=dev)
+    for _ in range(2):  # the second pass reuses the buffers of the first
+        st.prefill_from_host(host_in, host_out, bufs, workspace=ws)
+    torch.cuda.current_stream().synchronize()
+    assert native.gemma_attn_sync_status() == 0, native.gemma_last_error()
+    ref = []
+    for l, (hq, hk, hv) in enumerate(host_in):
+        q, k, v = (x.to(dev) for x in (hq, hk, hv))
+        out = torch.empty_like(q)
+        st.prefill_layer(l, q, k, v, out, workspace=ws)
+        ref.append(out.cpu())
+    for l in range(st.n_layers):
+        assert torch.equal(host_out[l].view(torch.int16), ref[l].view(torch.int16)), "layer %d" % l
