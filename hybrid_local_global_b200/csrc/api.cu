@@ -162,11 +162,17 @@ size_t decode_ws_parts(int B, int Hq, int D, int n_splits, size_t* off_lse, size
   return q + lse + o;
 }
 
-size_t prefill_ws_parts(int B, int S, int Hq, int Hkv, int D, int window, size_t* off_k) {
+// Prefill workspace: rotated Q, then on local layers either the rotated K
+// of the chunk (K at off_k) or, for a chunk after cached tokens, the K and V
+// windows of window + S rows (K at off_k, V at *off_vw).
+size_t prefill_ws_parts(int B, int S, int Hq, int Hkv, int D, int window, size_t* off_k,
+                        size_t* off_vw = nullptr) {
   size_t q = align256((size_t)B * S * Hq * D * 2);
   size_t k = window > 0 ? align256((size_t)B * S * Hkv * D * 2) : 0;
+  size_t win = window > 0 ? align256((size_t)B * (window + S) * Hkv * D * 2) : 0;
   *off_k = q;
-  return q + k;
+  if (off_vw) *off_vw = q + win;
+  return q + std::max(k, 2 * win);
 }
 
 }  // namespace
@@ -286,16 +292,20 @@ int gemma_attn_prefill(const void* q, const void* k_new, const void* v_new, void
   if (window > 0) {
     if (cache_cap != window)
       return fail(GEMMA_ERR_INVALID_ARG, "local layer: cache_cap %d must equal window %d", cache_cap, window);
-    if (seq_lens_before)
-      return fail(GEMMA_ERR_UNSUPPORTED, "chunked prefill on a local layer is not implemented");
+    if (shared && seq_lens_before)
+      return fail(GEMMA_ERR_UNSUPPORTED,
+                  "shared local layer after cached tokens: the source's chunk has replaced ring slots it needs");
     if (shared && s_new > window)
       return fail(GEMMA_ERR_UNSUPPORTED, "shared local layer: prefill longer than the window");
   } else if (cache_cap < s_new) {
     return fail(GEMMA_ERR_CAPACITY, "global layer: cache_cap %d < s_new %d", cache_cap, s_new);
   }
   if (s_new == 0) return succeed();
-  size_t off_k;
-  size_t need = prefill_ws_parts(batch, s_new, n_q_heads, n_kv_heads, head_dim, window, &off_k);
+  size_t off_k, off_vw;
+  size_t need = prefill_ws_parts(batch, s_new, n_q_heads, n_kv_heads, head_dim, window, &off_k, &off_vw);
+  // a local layer's chunk after cached tokens attends to a gathered key window
+  const bool chunked_local = window > 0 && seq_lens_before && !shared;
+  const int win_rows = chunked_local ? window + s_new : 0;
   if (!workspace || workspace_bytes < need)
     return fail(GEMMA_ERR_CAPACITY, "workspace %zu bytes < %zu", workspace_bytes, need);
   int* status = status_ptr();
@@ -309,6 +319,15 @@ int gemma_attn_prefill(const void* q, const void* k_new, const void* v_new, void
   ra.v_new = static_cast<const bf16*>(v_new);
   ra.q_rot = reinterpret_cast<bf16*>(ws);
   ra.k_rot = (window > 0 && !shared) ? reinterpret_cast<bf16*>(ws + off_k) : nullptr;
+  ra.v_win = chunked_local ? reinterpret_cast<bf16*>(ws + off_vw) : nullptr;
+  ra.win_rows = win_rows;
+  if (chunked_local) {
+    // before the chunk overwrites ring slots: old keys/values into rows 0..window-1
+    cudaError_t eg = launch_ring_gather(static_cast<const bf16*>(k_cache), static_cast<const bf16*>(v_cache),
+                                        seq_lens_before, batch, n_kv_heads, head_dim, window, win_rows,
+                                        ra.k_rot, ra.v_win, status, st);
+    if (eg != cudaSuccess) return cuda_fail(eg, "ring gather launch");
+  }
   ra.k_cache = static_cast<bf16*>(k_cache);
   ra.v_cache = static_cast<bf16*>(v_cache);
   ra.cache_cap = cache_cap;
@@ -337,6 +356,12 @@ int gemma_attn_prefill(const void* q, const void* k_new, const void* v_new, void
     aa.k = kc;
     aa.v = vc;
     aa.key_cap = cache_cap;
+  } else if (chunked_local) {
+    KVView kw = {ra.k_rot, (int64_t)win_rows * n_kv_heads * D, (int64_t)n_kv_heads * D, D};
+    KVView vw = {ra.v_win, kw.stride_b, kw.stride_row, kw.stride_h};
+    aa.k = kw;
+    aa.v = vw;
+    aa.key_cap = win_rows;
   } else {
     KVView kw = {ra.k_rot, (int64_t)s_new * n_kv_heads * D, (int64_t)n_kv_heads * D, D};
     KVView vw = {static_cast<const bf16*>(v_new), kw.stride_b, kw.stride_row, kw.stride_h};
@@ -344,6 +369,7 @@ int gemma_attn_prefill(const void* q, const void* k_new, const void* v_new, void
     aa.v = vw;
     aa.key_cap = s_new;
   }
+  aa.key_off_window = chunked_local ? 1 : 0;
   aa.seq_lens_before = seq_lens_before;
   aa.S = s_new;
   aa.window = window;
@@ -366,8 +392,9 @@ int gemma_attn_prefill(const void* q, const void* k_new, const void* v_new, void
     if (std::string(v) == "single") use_pair = false;
     if (std::string(v) == "pair") use_pair = true;
   }
-  e = use_pair ? launch_prefill_attn_pair(aa, batch, head_dim, cache_view ? cache_cap : s_new, cache_view ? 0 : 1, st)
-               : launch_prefill_attn_tc(aa, batch, head_dim, cache_view ? cache_cap : s_new, cache_view ? 0 : 1, st);
+  const int key_rows = cache_view ? cache_cap : (int)aa.key_cap;
+  e = use_pair ? launch_prefill_attn_pair(aa, batch, head_dim, key_rows, cache_view ? 0 : 1, st)
+               : launch_prefill_attn_tc(aa, batch, head_dim, key_rows, cache_view ? 0 : 1, st);
   p_attn.done();
   if (e != cudaSuccess) return cuda_fail(e, "prefill attention launch");
   return succeed();

@@ -14,7 +14,10 @@ struct PrefillRopeArgs {
   const bf16* k_new;   // [B][S][Hkv][D] or null (shared layer)
   const bf16* v_new;   // [B][S][Hkv][D] or null
   bf16* q_rot;         // workspace [B][S][Hq][D]
-  bf16* k_rot;         // workspace [B][S][Hkv][D] (local layers) or null
+  bf16* k_rot;         // workspace, local layers: [B][S][Hkv][D], or with win_rows > 0
+                       // [B][win_rows][Hkv][D] with the chunk at rows window.. ; else null
+  bf16* v_win;         // chunked local prefill: V window [B][win_rows][Hkv][D], else null
+  int win_rows;        // 0, or window + S (chunked local prefill)
   bf16* k_cache;       // [B][Hkv][cap][D]
   bf16* v_cache;
   int cache_cap;
@@ -53,6 +56,8 @@ struct PrefillAttnArgs {
   const bf16* q_rot;   // [B][S][Hq][D]
   KVView k, v;
   int64_t key_cap;     // rows readable per (batch, head) in the K/V views
+  int key_off_window;  // 1: view row = position - (seq_lens_before[b] - window) (a key window
+                       // gathered for chunked local prefill); 0: view row = position
   const int32_t* seq_lens_before;  // device [B] or null
   int S, window, Hq, Hkv;
   float scale_log2;    // scale * log2(e)
@@ -82,6 +87,12 @@ struct DecodeAttnArgs {
 };
 
 cudaError_t launch_prefill_rope(const PrefillRopeArgs& a, int B, int D, cudaStream_t st);
+// Chunked local prefill: copies the ring's K/V of positions
+// seq_lens_before[b] - window .. seq_lens_before[b] - 1 into rows 0..window-1
+// of the K and V windows (zeros for negative positions).
+cudaError_t launch_ring_gather(const bf16* k_cache, const bf16* v_cache, const int32_t* seq_lens_before,
+                               int B, int Hkv, int D, int window, int win_rows, bf16* k_win, bf16* v_win,
+                               int* status, cudaStream_t st);
 cudaError_t launch_decode_rope_append(const DecodeRopeArgs& a, int B, int D, cudaStream_t st);
 // tcgen05 prefill (head_dim 256 or 512). key_rows_total = rows of the K/V
 // views; kv_token_major: views are [B][rows][Hkv][D] (1) or [B][Hkv][rows][D] (0).

@@ -96,6 +96,7 @@ struct TcArgs {
   int* status;
   unsigned long long wait_ns;
   int kv_token_major;  // K/V map coordinates: 0 = (d, key, head, b), 1 = (d, head, key, b)
+  int key_off_window;  // 1: K/V view row = position - (pos0 - window), else = position
   int n_qtiles;
 };
 
@@ -168,7 +169,9 @@ __global__ void __launch_bounds__(192, 1)
 
   const int64_t pos0 = a.seq_lens_before ? (int64_t)a.seq_lens_before[b] : 0;
   const int64_t n_keys = pos0 + a.S;
-  if (pos0 < 0 || n_keys > a.key_cap) return;  // reported by the RoPE kernel
+  // view row of a key = its position - koff (a gathered key window starts at pos0 - window)
+  const int64_t koff = a.key_off_window ? pos0 - a.window : 0;
+  if (pos0 < 0 || n_keys - koff > a.key_cap) return;  // reported by the RoPE kernel
   int64_t lo_first, hi_first, lo_last, hi_last;
   visible_range(pos0 + q0, a.window, n_keys, &lo_first, &hi_first);
   visible_range(pos0 + min(q0 + BM - 1, a.S - 1), a.window, n_keys, &lo_last, &hi_last);
@@ -220,7 +223,7 @@ __global__ void __launch_bounds__(192, 1)
       for (int j = 0; j <= n_tiles && ok; ++j) {
         for (int kind = 0; kind < 2 && ok; ++kind) {  // 0: K_j, 1: V_{j-1}
           if ((kind == 0 && j == n_tiles) || (kind == 1 && j == 0)) continue;
-          const int key0 = (int)((kt0 + j - kind) * BN);
+          const int key0 = (int)((kt0 + j - kind) * BN - koff);  // view row
           const int n_st = kind == 0 ? Cfg::K_STAGES : 2;
           for (int half = 0; half < n_st; ++half, ++item) {
             const int s = item % NSTAGE;
@@ -582,6 +585,7 @@ cudaError_t launch_prefill_attn_tc(const PrefillAttnArgs& a, int B, int D, int k
   t.status = a.status;
   t.wait_ns = a.wait_ns;
   t.kv_token_major = kv_token_major;
+  t.key_off_window = a.key_off_window;
   t.n_qtiles = (a.S + BM - 1) / BM;
   if (D == 256) {
     using Cfg = TcCfg<256>;

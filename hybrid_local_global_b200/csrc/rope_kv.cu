@@ -128,7 +128,9 @@ constexpr int ROPE_RPT = 2;    // positions per thread
 // (of ROPE_RPT per thread): the angles of a position are formed once and
 // serve all Hq + 2 Hkv head vectors, which are loaded ROPE_HB at a time so
 // several 16-byte loads are in flight per thread.
-template <int D>
+// WIN: chunked local prefill, where the chunk's rotated K and its V go to
+// rows window.. of the K and V windows (a.win_rows rows per sequence).
+template <int D, bool WIN>
 __global__ void __launch_bounds__(256, 2) k_prefill_rope(PrefillRopeArgs a) {
   const int b = blockIdx.y;
   const int e0 = threadIdx.x * 8;
@@ -166,7 +168,11 @@ __global__ void __launch_bounds__(256, 2) k_prefill_rope(PrefillRopeArgs a) {
 #pragma unroll 1
     for (int h0 = 0; h0 < a.Hkv; h0 += ROPE_HB / 2) {
       uint4 kx[ROPE_HB / 2], vx[ROPE_HB / 2];
-      const bool want_v = a.v_new && (a.window == 0 || to_ring);  // no v_new: K = V
+#pragma unroll
+      for (int u = 0; u < ROPE_HB / 2; ++u) kx[u] = vx[u] = make_uint4(0, 0, 0, 0);
+      // no v_new: K = V; the V window (WIN) takes every position of the chunk
+      const bool want_v = a.v_new && (WIN || a.window == 0 || to_ring);
+      const int64_t wrow = WIN ? (int64_t)b * a.win_rows + a.window + s : row;  // k_rot / V window row
 #pragma unroll
       for (int u = 0; u < ROPE_HB / 2; ++u)
         if (h0 + u < a.Hkv) {
@@ -184,7 +190,8 @@ __global__ void __launch_bounds__(256, 2) k_prefill_rope(PrefillRopeArgs a) {
             st16(a.k_cache + cslot, kr);
             if (want_v) st16(a.v_cache + cslot, vx[u]);
           } else {
-            st16(a.k_rot + (row * a.Hkv + kh) * D + e0, kr);
+            st16(a.k_rot + (wrow * a.Hkv + kh) * D + e0, kr);
+            if (WIN) st16(a.v_win + (wrow * a.Hkv + kh) * D + e0, vx[u]);
             if (to_ring) {
               st16(a.k_cache + cslot, kr);
               if (want_v) st16(a.v_cache + cslot, vx[u]);
@@ -192,6 +199,41 @@ __global__ void __launch_bounds__(256, 2) k_prefill_rope(PrefillRopeArgs a) {
           }
         }
     }
+  }
+}
+
+// Chunked local prefill: before the chunk overwrites ring slots, copy the
+// ring's keys and values of positions pos0-window .. pos0-1 (pos0 =
+// seq_lens_before[b]) into rows 0..window-1 of the K and V windows; the
+// RoPE kernel then writes the chunk at rows window.. . Negative positions
+// become zeros (they are never visible). One CTA per 8 rows of a sequence.
+template <int D>
+__global__ void __launch_bounds__(256) k_ring_gather(const bf16* __restrict__ k_cache,
+                                                     const bf16* __restrict__ v_cache,
+                                                     const int32_t* seq_lens_before, int Hkv, int window,
+                                                     int win_rows, bf16* k_win, bf16* v_win, int* status) {
+  const int b = blockIdx.y;
+  const int64_t pos0 = seq_lens_before[b];
+  if (pos0 < 0) {
+    if (threadIdx.x == 0 && blockIdx.x == 0) set_status(status, GEMMA_ERR_DEVICE_RANGE);
+    return;
+  }
+  constexpr int CH = D / 8;  // 16-byte chunks per head vector
+  const int r0 = blockIdx.x * 8;
+  for (int idx = threadIdx.x; idx < 8 * Hkv * CH; idx += blockDim.x) {
+    const int r = r0 + idx / (Hkv * CH);
+    if (r >= window) break;
+    const int h = (idx / CH) % Hkv, c = (idx % CH) * 8;
+    const int64_t p = pos0 - window + r;
+    uint4 kv = make_uint4(0, 0, 0, 0), vv = make_uint4(0, 0, 0, 0);
+    if (p >= 0) {
+      const int64_t src = (((int64_t)b * Hkv + h) * window + p % window) * D + c;
+      kv = ld16(k_cache + src);
+      vv = ld16(v_cache + src);
+    }
+    const int64_t dst = (((int64_t)b * win_rows + r) * Hkv + h) * D + c;
+    st16(k_win + dst, kv);
+    st16(v_win + dst, vv);
   }
 }
 
@@ -239,10 +281,27 @@ cudaError_t launch_prefill_rope(const PrefillRopeArgs& a, int B, int D, cudaStre
   dim3 block(tx, 256 / tx);
   const int per_cta = block.y * ROPE_RPT;
   dim3 grid((a.S + per_cta - 1) / per_cta, B);
+  const bool win = a.win_rows > 0 && a.v_win;
+  if (D == 256) {
+    if (win) k_prefill_rope<256, true><<<grid, block, 0, st>>>(a);
+    else k_prefill_rope<256, false><<<grid, block, 0, st>>>(a);
+  } else {
+    if (win) k_prefill_rope<512, true><<<grid, block, 0, st>>>(a);
+    else k_prefill_rope<512, false><<<grid, block, 0, st>>>(a);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_ring_gather(const bf16* k_cache, const bf16* v_cache, const int32_t* seq_lens_before,
+                               int B, int Hkv, int D, int window, int win_rows, bf16* k_win, bf16* v_win,
+                               int* status, cudaStream_t st) {
+  dim3 grid((window + 7) / 8, B);
   if (D == 256)
-    k_prefill_rope<256><<<grid, block, 0, st>>>(a);
+    k_ring_gather<256><<<grid, 256, 0, st>>>(k_cache, v_cache, seq_lens_before, Hkv, window, win_rows, k_win,
+                                             v_win, status);
   else
-    k_prefill_rope<512><<<grid, block, 0, st>>>(a);
+    k_ring_gather<512><<<grid, 256, 0, st>>>(k_cache, v_cache, seq_lens_before, Hkv, window, win_rows, k_win,
+                                             v_win, status);
   return cudaGetLastError();
 }
 

@@ -135,7 +135,8 @@ E = native
     (dict(theta=0.0), E.GEMMA_ERR_INVALID_ARG),
     (dict(W=500, cap=500), E.GEMMA_ERR_INVALID_ARG),  # window not a multiple of 16
     (dict(cap=1024), E.GEMMA_ERR_INVALID_ARG),        # local ring must hold exactly the window
-    (dict(lens=FAKE), E.GEMMA_ERR_UNSUPPORTED),        # chunked local prefill
+    (dict(lens=FAKE, wsb=16), E.GEMMA_ERR_CAPACITY),   # chunked local prefill is accepted
+    (dict(lens=FAKE, flags=1, k=None, v=None), E.GEMMA_ERR_UNSUPPORTED),  # ... but not on a shared layer
     (dict(W=0, cap=8), E.GEMMA_ERR_CAPACITY),          # global cache shorter than the chunk
     (dict(k=None), E.GEMMA_ERR_INVALID_ARG),           # unshared layer without new keys
     (dict(flags=1), E.GEMMA_ERR_INVALID_ARG),          # shared layer with new keys

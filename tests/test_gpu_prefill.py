@@ -334,3 +334,64 @@ def test_prefill_from_host_matches_layer_by_layer():
         ref.append(out.cpu())
     for l in range(st.n_layers):
         assert torch.equal(host_out[l].view(torch.int16), ref[l].view(torch.int16)), "layer %d" % l
+
+
+def run_local_chunk_case(oracle, *, B, S, Hq, Hkv, D, W, prior, seed, frac=1.0, theta=1e4,
+                         tol=(2e-2, 2e-3)):
+    """A chunk of S tokens on a local layer after prior[b] cached tokens: the
+    ring holds (rotated) keys and values of the last W cached positions; the
+    chunk's queries attend to those and to the chunk, and the ring ends up
+    holding the last W positions of cache + chunk."""
+    dev = torch.device("cuda")
+    g = synth.generator(seed)
+    q = synth.randn_bf16((B, S, Hq, D), g)
+    k = synth.randn_bf16((B, S, Hkv, D), g)
+    v = synth.randn_bf16((B, S, Hkv, D), g)
+    kc = torch.full((B, Hkv, W, D), float("nan"), dtype=torch.bfloat16)
+    vc = torch.full((B, Hkv, W, D), float("nan"), dtype=torch.bfloat16)
+    T = max(prior) + S
+    k_log = torch.zeros((B, T, Hkv, D), dtype=torch.bfloat16)
+    v_log = torch.zeros((B, T, Hkv, D), dtype=torch.bfloat16)
+    for b in range(B):
+        for p in range(max(0, prior[b] - W), prior[b]):  # what the ring holds
+            kr = synth.randn_bf16((Hkv, D), g)
+            vr = synth.randn_bf16((Hkv, D), g)
+            kc[b, :, p % W], vc[b, :, p % W] = kr, vr
+            k_log[b, p], v_log[b, p] = kr, vr
+        k_log[b, prior[b]:prior[b] + S] = k[b]
+        v_log[b, prior[b]:prior[b] + S] = v[b]
+    kcd, vcd = kc.to(dev), vc.to(dev)
+    out = torch.full((B, S, Hq, D), float("nan"), dtype=torch.bfloat16, device=dev)
+    lens = torch.tensor(prior, dtype=torch.int32, device=dev)
+    scale = 1.0 / math.sqrt(D)
+    native.gemma_attn_prefill(q.to(dev), k.to(dev), v.to(dev), kcd, vcd, window=W, rope_frac=frac,
+                              rope_theta=theta, scale=scale, out=out, seq_lens_before=lens)
+    assert native.gemma_attn_sync_status() == 0, native.gemma_last_error()
+    ref, _ = oracle.attention(to_bits(q), to_bits(k_log), to_bits(v_log), q_pos0=prior,
+                              n_keys=[p + S for p in prior], rot_from=prior, window=W,
+                              rope_frac=frac, theta=theta, scale=scale)
+    got = out.float().cpu().double().numpy().transpose(0, 2, 1, 3).reshape(-1, D)
+    assert_close(got, ref, *tol, what="chunked local prefill")
+    kc1, vc1 = kcd.cpu(), vcd.cpu()
+    for b in range(B):
+        end = prior[b] + S
+        for p in range(max(0, end - W), end):
+            slot = p % W
+            if p >= prior[b]:
+                s_ = p - prior[b]
+                assert torch.equal(vc1[b, :, slot], v[b, s_]), "V slot %d" % slot
+                for h in range(Hkv):
+                    exp = torch.from_numpy(oracle.rope_bf16(to_bits(k[b, s_, h]), p, frac, theta)).to(torch.bfloat16)
+                    assert_rotated_bf16(kc1[b, h, slot], exp, k[b, s_, h], "K slot %d" % slot)
+            else:
+                assert torch.equal(kc1[b, :, slot], kc[b, :, slot]) and torch.equal(vc1[b, :, slot], vc[b, :, slot])
+
+
+@pytest.mark.parametrize("case", [
+    dict(B=2, S=200, Hq=8, Hkv=4, D=256, W=512, prior=[700, 3], seed=131),
+    dict(B=1, S=700, Hq=8, Hkv=4, D=256, W=512, prior=[1000], seed=132),   # chunk longer than the window
+    dict(B=2, S=1, Hq=4, Hkv=2, D=256, W=64, prior=[64, 129], seed=133),   # one-token chunks
+    dict(B=1, S=130, Hq=8, Hkv=4, D=512, W=128, prior=[257], seed=134, frac=0.25, theta=1e6),
+], ids=["S200", "S700", "S1", "D512"])
+def test_prefill_local_chunk_after_cached_tokens(oracle, case):
+    run_local_chunk_case(oracle, **case)
