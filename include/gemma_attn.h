@@ -88,8 +88,10 @@ typedef enum gemma_status {
 /* k_cache, v_cache [batch][n_kv_heads][cache_cap][head_dim]               */
 /* seq_lens_before  device int32 [batch]: tokens already in the cache per   */
 /*        sequence (the chunk starts at that position), or NULL for 0.     */
-/*        Must be NULL on a local layer (chunked local prefill is not      */
-/*        implemented: GEMMA_ERR_UNSUPPORTED).                              */
+/*        On a local layer the chunk also attends to the ring's last       */
+/*        `window` cached positions (read before the chunk overwrites      */
+/*        them); a shared local layer after cached tokens returns          */
+/*        GEMMA_ERR_UNSUPPORTED (its source already replaced those slots). */
 /* out    [batch][s_new][n_q_heads][head_dim]  bf16 attention output        */
 /* lse    optional fp32 [batch][n_q_heads][s_new]: natural-log sum of       */
 /*        exp(scale * q.k) over the visible keys; NULL to skip.            */
