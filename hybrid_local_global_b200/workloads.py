@@ -72,6 +72,11 @@ WORKLOADS = {
         local=L31B_LOCAL, global_=L31B_GLOBAL, len_lo=4096, len_hi=131072, n_shared=2, seed=3,
         description="31B-shaped 6-layer decode: B64, KV length U[4096,131072], ring 1024, "
                     "last 2 layers shared"),
+    "31b_decode_b16_12l_shared": Workload(
+        "31b_decode_b16_12l_shared", "decode", batch=16, n_q_heads=32, n_layers=12, ratio=5,
+        local=L31B_LOCAL, global_=L31B_GLOBAL, len_lo=4096, len_hi=131072, n_shared=2, seed=7,
+        description="31B-shaped 12-layer decode (two 5:1 patterns), last 2 layers shared: "
+                    "10 -> 9 (local), 11 -> 5 (global); B16, KV length U[4096,131072]"),
     "global_chunk_256k": Workload(
         "global_chunk_256k", "prefill", batch=1, n_q_heads=32, n_layers=1, ratio=0,
         local=L31B_LOCAL, global_=L31B_GLOBAL, seq=4096, prior=262144 - 4096, seed=4,

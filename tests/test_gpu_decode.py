@@ -256,6 +256,25 @@ def test_decode_31b_b64(oracle):
     _decode_workload(oracle, "31b_decode_b64", n_sample=8)
 
 
+def test_decode_31b_12_layers_two_shared(oracle):
+    """The 12-layer form of the 31B-shaped decode block: layer 10 reads layer
+    9's ring and layer 11 reads layer 5's global cache (latest earlier layer
+    of the same type), and the owned cache bytes match the oracle's byte
+    counter for that stack."""
+    w = WORKLOADS["31b_decode_b16_12l_shared"]
+    is_global, src = native.gemma_layer_schedule(w.n_layers, w.ratio, w.n_shared)
+    assert [src[l] for l in (10, 11)] == [9, 5]
+    assert [is_global[l] for l in (5, 9, 10, 11)] == [True, False, False, True]
+    st = AttentionStack(w, torch.device("cuda"))
+    expect = oracle.stack_cache_bytes(w.n_layers, w.ratio, w.n_shared, w.batch, local_kv_heads=16,
+                                      local_head_dim=256, local_capacity=1024, global_kv_heads=4,
+                                      global_head_dim=512, global_capacity=w.len_hi, which="all")
+    assert st.owned_cache_bytes() == expect
+    del st
+    torch.cuda.empty_cache()
+    _decode_workload(oracle, "31b_decode_b16_12l_shared", n_sample=3)
+
+
 def test_decode_global_256k_k_equals_v(oracle):
     _decode_workload(oracle, "global_decode_256k_keqv", n_sample=1)
 

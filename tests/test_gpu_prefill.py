@@ -395,3 +395,53 @@ def run_local_chunk_case(oracle, *, B, S, Hq, Hkv, D, W, prior, seed, frac=1.0, 
 ], ids=["S200", "S700", "S1", "D512"])
 def test_prefill_local_chunk_after_cached_tokens(oracle, case):
     run_local_chunk_case(oracle, **case)
+
+
+def test_multi_query_verify_chunk_across_layer_types(oracle):
+    """Speculative verify / multi-query decode: k = 4 new tokens per sequence
+    after a long cached context, through every layer of a 31B-shaped 6-layer
+    stack (5 local with ring caches, 1 global). It is a small chunked
+    prefill: each new token sees the cached context (window-limited on local
+    layers) and the earlier new tokens (causal tail)."""
+    from hybrid_local_global_b200.workloads import L31B_GLOBAL, L31B_LOCAL, Workload
+    prior, kq = [3000, 700], 4
+    w = Workload("verify_k4", "prefill", batch=2, n_q_heads=32, n_layers=6, ratio=5,
+                 local=L31B_LOCAL, global_=L31B_GLOBAL, seq=kq, seed=17)
+    dev = torch.device("cuda")
+    st = AttentionStack(w, dev, global_capacity=max(prior) + kq)
+    g = synth.generator(17)
+    ws = torch.empty(st.prefill_workspace_bytes(), dtype=torch.uint8, device=dev)
+    lens = torch.tensor(prior, dtype=torch.int32, device=dev)
+    T = max(prior) + kq
+    for l in range(st.n_layers):
+        t = st.layer_type(l)
+        Hkv, D, W = t.n_kv_heads, t.head_dim, t.window
+        k_log = torch.zeros((w.batch, T, Hkv, D), dtype=torch.bfloat16)
+        v_log = torch.zeros_like(k_log)
+        kc = torch.full(tuple(st.k_cache[l].shape), float("nan"), dtype=torch.bfloat16)
+        vc = kc.clone()
+        for b in range(w.batch):
+            first = max(0, prior[b] - W) if W else 0
+            kr = synth.randn_bf16((Hkv, prior[b] - first, D), g)
+            vr = synth.randn_bf16((Hkv, prior[b] - first, D), g)
+            for i, p in enumerate(range(first, prior[b])):
+                slot = p % W if W else p
+                kc[b, :, slot], vc[b, :, slot] = kr[:, i], vr[:, i]
+            k_log[b, first:prior[b]] = kr.transpose(0, 1)
+            v_log[b, first:prior[b]] = vr.transpose(0, 1)
+        st.k_cache[l].copy_(kc)
+        st.v_cache[l].copy_(vc)
+        q = synth.randn_bf16((w.batch, kq, w.n_q_heads, D), g)
+        k = synth.randn_bf16((w.batch, kq, Hkv, D), g)
+        v = synth.randn_bf16((w.batch, kq, Hkv, D), g)
+        for b in range(w.batch):
+            k_log[b, prior[b]:prior[b] + kq] = k[b]
+            v_log[b, prior[b]:prior[b] + kq] = v[b]
+        out = torch.full((w.batch, kq, w.n_q_heads, D), float("nan"), dtype=torch.bfloat16, device=dev)
+        st.prefill_layer(l, q.to(dev), k.to(dev), v.to(dev), out, workspace=ws, seq_lens_before=lens)
+        assert native.gemma_attn_sync_status() == 0, native.gemma_last_error()
+        ref, _ = oracle.attention(to_bits(q), to_bits(k_log), to_bits(v_log), q_pos0=prior,
+                                  n_keys=[p + kq for p in prior], rot_from=prior, window=W,
+                                  rope_frac=t.rope_frac, theta=t.rope_theta, scale=t.scale)
+        got = out.float().cpu().double().numpy().transpose(0, 2, 1, 3).reshape(-1, D)
+        assert_close(got, ref, what="verify layer %d (%s)" % (l, "global" if W == 0 else "local"))
