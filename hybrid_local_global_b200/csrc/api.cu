@@ -382,19 +382,30 @@ int gemma_attn_prefill(const void* q, const void* k_new, const void* v_new, void
   aa.wait_ns = (unsigned long long)g_wait_ns.load();
   const bool cache_view = (window == 0 || shared);
   ProfScope p_attn(GEMMA_KERNEL_PREFILL_ATTN, st);
-  // Two query tiles on a CTA pair (cta_group::2) halve each SM's K/V tile
-  // traffic; they win on long head_dim-512 layers (measured on B200: -14% on
-  // a 32K-token global layer) and lose on short or windowed ones, where the
-  // cluster's start/finish overhead dominates. GEMMA_PREFILL_KERNEL=single|pair
-  // overrides the choice.
-  bool use_pair = head_dim == 512 && (cache_view ? cache_cap : s_new) >= 16384;
+  // Head_dim-512 layers run on CTA pairs (cta_group::2, M = 256): each SM
+  // loads and reads from shared memory half of every K and V tile. With an
+  // even number of q heads per KV head the pair takes two q heads of one
+  // query tile (measured on B200: -7% on an 8K-token E2B global layer, -13%
+  // on a 32K-token 31B global layer); otherwise two query tiles of one head,
+  // which only pays from 16K keys. Head_dim 256 stays on one CTA per tile
+  // (both pairings measured slower on local layers).
+  // GEMMA_PREFILL_KERNEL=single|pair|hpair overrides the choice.
+  enum { K_SINGLE, K_PAIR, K_HPAIR } kern = K_SINGLE;
+  if (head_dim == 512) {
+    if ((n_q_heads / n_kv_heads) % 2 == 0)
+      kern = K_HPAIR;
+    else if ((cache_view ? cache_cap : s_new) >= 16384)
+      kern = K_PAIR;
+  }
   if (const char* v = std::getenv("GEMMA_PREFILL_KERNEL")) {
-    if (std::string(v) == "single") use_pair = false;
-    if (std::string(v) == "pair") use_pair = true;
+    if (std::string(v) == "single") kern = K_SINGLE;
+    if (std::string(v) == "pair") kern = K_PAIR;
+    if (std::string(v) == "hpair") kern = K_HPAIR;
   }
   const int key_rows = cache_view ? cache_cap : (int)aa.key_cap;
-  e = use_pair ? launch_prefill_attn_pair(aa, batch, head_dim, key_rows, cache_view ? 0 : 1, st)
-               : launch_prefill_attn_tc(aa, batch, head_dim, key_rows, cache_view ? 0 : 1, st);
+  const int tok_major = cache_view ? 0 : 1;
+  e = kern == K_SINGLE ? launch_prefill_attn_tc(aa, batch, head_dim, key_rows, tok_major, st)
+                       : launch_prefill_attn_pair(aa, batch, head_dim, key_rows, tok_major, kern == K_HPAIR, st);
   p_attn.done();
   if (e != cudaSuccess) return cuda_fail(e, "prefill attention launch");
   return succeed();

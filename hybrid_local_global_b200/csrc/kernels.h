@@ -100,8 +100,10 @@ cudaError_t launch_decode_rope_append(const DecodeRopeArgs& a, int B, int D, cud
 // sharing each MMA (cta_group::2).
 cudaError_t launch_prefill_attn_tc(const PrefillAttnArgs& a, int B, int D, int key_rows_total,
                                    int kv_token_major, cudaStream_t st);
+// head_pair: the pair takes two q heads of one KV head on the same query
+// tile (used when q heads per KV head is even) instead of two query tiles.
 cudaError_t launch_prefill_attn_pair(const PrefillAttnArgs& a, int B, int D, int key_rows_total,
-                                     int kv_token_major, cudaStream_t st);
+                                     int kv_token_major, int head_pair, cudaStream_t st);
 cudaError_t launch_decode_split(const DecodeAttnArgs& a, int B, int D, cudaStream_t st);
 cudaError_t launch_decode_combine(const DecodeAttnArgs& a, int B, int D, cudaStream_t st);
 cudaError_t launch_visible_ranges(const int32_t* seq_lens_before, int B, int S, int window,

@@ -44,12 +44,11 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
-#include <mutex>
-
 #include "common.cuh"
 #include "kernels.h"
 #include "pair.cuh"
 #include "tc.cuh"
+#include "tmap.h"
 
 namespace hlg {
 
@@ -107,7 +106,8 @@ struct PairArgs {
   unsigned long long wait_ns;
   int kv_token_major;  // K/V map coordinates: 0 = (d, key, head, b), 1 = (d, head, key, b)
   int key_off_window;  // 1: K/V view row = position - (pos0 - window), else = position
-  int n_pairs;         // query-tile pairs per (batch, head)
+  int n_pairs;         // query-tile pairs per (batch, head); with head_pair: query tiles
+  int head_pair;       // 1: the CTAs take q heads 2p and 2p+1 of one query tile (same KV head)
 };
 
 __device__ __forceinline__ bool wait_all(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
@@ -188,10 +188,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
 
   const uint32_t rank = pair::cta_rank();
   const bool leader = rank == 0;
-  const int h = blockIdx.y / Cfg::NV, vh = blockIdx.y % Cfg::NV, b = blockIdx.z;
+  const int vh = blockIdx.y % Cfg::NV, b = blockIdx.z;
   const int pq = a.n_pairs - 1 - (int)(blockIdx.x >> 1);  // heaviest pairs first
-  const int pq0 = pq * 2 * BM;                             // first row of the pair
-  const int q0 = pq0 + (int)rank * BM;                     // first row of this CTA
+  // query-tile pairs: rows pq0 .. pq0 + 255 of one head, rank r takes the
+  // r-th 128; head pairs: rows pq0 .. pq0 + 127 of heads 2p and 2p + 1
+  const int pq0 = a.head_pair ? pq * BM : pq * 2 * BM;      // first row of the pair
+  const int span = a.head_pair ? BM : 2 * BM;               // rows the pair covers
+  const int q0 = a.head_pair ? pq0 : pq0 + (int)rank * BM;  // first row of this CTA
+  const int h = a.head_pair ? 2 * (int)(blockIdx.y / Cfg::NV) + (int)rank : (int)(blockIdx.y / Cfg::NV);
   const int g = h / (a.Hq / a.Hkv);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -202,7 +206,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
   if (pos0 < 0 || n_keys - koff > a.key_cap) return;  // reported by the RoPE kernel; same for both CTAs
   int64_t lo_first, hi_first, lo_last, hi_last;
   visible_range(pos0 + pq0, a.window, n_keys, &lo_first, &hi_first);
-  visible_range(pos0 + min(pq0 + 2 * BM - 1, a.S - 1), a.window, n_keys, &lo_last, &hi_last);
+  visible_range(pos0 + min(pq0 + span - 1, a.S - 1), a.window, n_keys, &lo_last, &hi_last);
   const int64_t kt0 = lo_first / BN;
   const int n_tiles = (int)(hi_last / BN - kt0 + 1);
 
@@ -541,42 +545,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
 }
 
 // ---------------------------------------------------------------- host side
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  });
-  return fn;
-}
-
-// bf16 4-D map, dims innermost first, strides in bytes for dims 1..3,
-// box[4], 128-byte swizzle, out-of-range elements read as zero.
-bool make_map(CUtensorMap* m, const void* ptr, const uint64_t dims[4], const uint64_t strides[3],
-              const uint32_t box[4]) {
-  auto fn = encode_fn();
-  if (!fn) return false;
-  cuuint64_t gd[4] = {dims[0], dims[1], dims[2], dims[3]};
-  cuuint64_t gs[3] = {strides[0], strides[1], strides[2]};
-  cuuint32_t bx[4] = {box[0], box[1], box[2], box[3]};
-  cuuint32_t es[4] = {1, 1, 1, 1};
-  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), gd, gs, bx, es,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
-}
-
 template <int D>
 cudaError_t launch_pair(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mo,
                         const PairArgs& t, int B, cudaStream_t st) {
   using Cfg = PairCfg<D>;
   cudaError_t e = cudaFuncSetAttribute(k_prefill_pair<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);
   if (e != cudaSuccess) return e;
-  dim3 grid(2 * t.n_pairs, t.Hq * Cfg::NV, B);
+  dim3 grid(2 * t.n_pairs, (t.head_pair ? t.Hq / 2 : t.Hq) * Cfg::NV, B);
   k_prefill_pair<D><<<grid, 192, Cfg::SMEM, st>>>(mq, mk, mv, mo, t);
   return cudaGetLastError();
 }
@@ -584,38 +559,11 @@ cudaError_t launch_pair(const CUtensorMap& mq, const CUtensorMap& mk, const CUte
 }  // namespace
 
 cudaError_t launch_prefill_attn_pair(const PrefillAttnArgs& a, int B, int D, int key_rows_total,
-                                     int kv_token_major, cudaStream_t st) {
+                                     int kv_token_major, int head_pair, cudaStream_t st) {
   if (D != 256 && D != 512) return cudaErrorInvalidValue;
-  const uint64_t E = 2;
   CUtensorMap mq, mk, mv, mo;
-  {
-    const uint64_t dims[4] = {(uint64_t)D, (uint64_t)a.Hq, (uint64_t)a.S, (uint64_t)B};
-    const uint64_t str[3] = {(uint64_t)D * E, (uint64_t)a.Hq * D * E, (uint64_t)a.S * a.Hq * D * E};
-    const uint32_t box[4] = {64, 1, BM, 1};
-    if (!make_map(&mq, a.q_rot, dims, str, box)) return cudaErrorInvalidValue;
-    if (!make_map(&mo, a.out, dims, str, box)) return cudaErrorInvalidValue;
-  }
-  if (kv_token_major) {
-    // [B][rows][Hkv][D]
-    const uint64_t dims[4] = {(uint64_t)D, (uint64_t)a.Hkv, (uint64_t)key_rows_total, (uint64_t)B};
-    const uint64_t str[3] = {(uint64_t)a.k.stride_h * E, (uint64_t)a.k.stride_row * E,
-                             (uint64_t)a.k.stride_b * E};
-    const uint32_t bk[4] = {64, 1, KH, 1}, bv[4] = {64, 1, BN, 1};
-    if (!make_map(&mk, a.k.ptr, dims, str, bk)) return cudaErrorInvalidValue;
-    const uint64_t strv[3] = {(uint64_t)a.v.stride_h * E, (uint64_t)a.v.stride_row * E,
-                              (uint64_t)a.v.stride_b * E};
-    if (!make_map(&mv, a.v.ptr, dims, strv, bv)) return cudaErrorInvalidValue;
-  } else {
-    // [B][Hkv][rows][D]
-    const uint64_t dims[4] = {(uint64_t)D, (uint64_t)key_rows_total, (uint64_t)a.Hkv, (uint64_t)B};
-    const uint64_t str[3] = {(uint64_t)a.k.stride_row * E, (uint64_t)a.k.stride_h * E,
-                             (uint64_t)a.k.stride_b * E};
-    const uint32_t bk[4] = {64, KH, 1, 1}, bv[4] = {64, BN, 1, 1};
-    if (!make_map(&mk, a.k.ptr, dims, str, bk)) return cudaErrorInvalidValue;
-    const uint64_t strv[3] = {(uint64_t)a.v.stride_row * E, (uint64_t)a.v.stride_h * E,
-                              (uint64_t)a.v.stride_b * E};
-    if (!make_map(&mv, a.v.ptr, dims, strv, bv)) return cudaErrorInvalidValue;
-  }
+  if (!make_prefill_maps(a, B, D, key_rows_total, kv_token_major, BM, KH, BN, &mq, &mk, &mv, &mo))
+    return cudaErrorInvalidValue;
   PairArgs t;
   t.S = a.S;
   t.window = a.window;
@@ -630,7 +578,9 @@ cudaError_t launch_prefill_attn_pair(const PrefillAttnArgs& a, int B, int D, int
   t.kv_token_major = kv_token_major;
   t.key_off_window = a.key_off_window;
   const int n_qtiles = (a.S + BM - 1) / BM;
-  t.n_pairs = (n_qtiles + 1) / 2;
+  // head pairs need an even number of q heads per KV head (both share its K/V)
+  t.head_pair = head_pair && (a.Hq / a.Hkv) % 2 == 0;
+  t.n_pairs = t.head_pair ? n_qtiles : (n_qtiles + 1) / 2;
   return D == 256 ? launch_pair<256>(mq, mk, mv, mo, t, B, st) : launch_pair<512>(mq, mk, mv, mo, t, B, st);
 }
 

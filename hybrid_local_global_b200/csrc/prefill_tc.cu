@@ -39,11 +39,10 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
-#include <mutex>
-
 #include "common.cuh"
 #include "kernels.h"
 #include "tc.cuh"
+#include "tmap.h"
 
 namespace hlg {
 
@@ -507,71 +506,14 @@ __global__ void __launch_bounds__(192, 1)
   }
 }
 
-// ---------------------------------------------------------------- host side
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  });
-  return fn;
-}
-
-// bf16 4-D map, dims innermost first, strides in bytes for dims 1..3,
-// box[4], 128-byte swizzle, out-of-range elements read as zero.
-bool make_map(CUtensorMap* m, const void* ptr, const uint64_t dims[4], const uint64_t strides[3],
-              const uint32_t box[4]) {
-  auto fn = encode_fn();
-  if (!fn) return false;
-  cuuint64_t gd[4] = {dims[0], dims[1], dims[2], dims[3]};
-  cuuint64_t gs[3] = {strides[0], strides[1], strides[2]};
-  cuuint32_t bx[4] = {box[0], box[1], box[2], box[3]};
-  cuuint32_t es[4] = {1, 1, 1, 1};
-  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), gd, gs, bx, es,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
-}
-
 }  // namespace
 
 cudaError_t launch_prefill_attn_tc(const PrefillAttnArgs& a, int B, int D, int key_rows_total,
                                    int kv_token_major, cudaStream_t st) {
   if (D != 256 && D != 512) return cudaErrorInvalidValue;
-  const uint64_t E = 2;
   CUtensorMap mq, mk, mv, mo;
-  {
-    const uint64_t dims[4] = {(uint64_t)D, (uint64_t)a.Hq, (uint64_t)a.S, (uint64_t)B};
-    const uint64_t str[3] = {(uint64_t)D * E, (uint64_t)a.Hq * D * E, (uint64_t)a.S * a.Hq * D * E};
-    const uint32_t box[4] = {64, 1, BM, 1};
-    if (!make_map(&mq, a.q_rot, dims, str, box)) return cudaErrorInvalidValue;
-    if (!make_map(&mo, a.out, dims, str, box)) return cudaErrorInvalidValue;
-  }
-  if (kv_token_major) {
-    // [B][rows][Hkv][D]
-    const uint64_t dims[4] = {(uint64_t)D, (uint64_t)a.Hkv, (uint64_t)key_rows_total, (uint64_t)B};
-    const uint64_t str[3] = {(uint64_t)a.k.stride_h * E, (uint64_t)a.k.stride_row * E,
-                             (uint64_t)a.k.stride_b * E};
-    const uint32_t bk[4] = {64, 1, BN, 1}, bv[4] = {64, 1, 64, 1};
-    if (!make_map(&mk, a.k.ptr, dims, str, bk)) return cudaErrorInvalidValue;
-    const uint64_t strv[3] = {(uint64_t)a.v.stride_h * E, (uint64_t)a.v.stride_row * E,
-                              (uint64_t)a.v.stride_b * E};
-    if (!make_map(&mv, a.v.ptr, dims, strv, bv)) return cudaErrorInvalidValue;
-  } else {
-    // [B][Hkv][rows][D]
-    const uint64_t dims[4] = {(uint64_t)D, (uint64_t)key_rows_total, (uint64_t)a.Hkv, (uint64_t)B};
-    const uint64_t str[3] = {(uint64_t)a.k.stride_row * E, (uint64_t)a.k.stride_h * E,
-                             (uint64_t)a.k.stride_b * E};
-    const uint32_t bk[4] = {64, BN, 1, 1}, bv[4] = {64, 64, 1, 1};
-    if (!make_map(&mk, a.k.ptr, dims, str, bk)) return cudaErrorInvalidValue;
-    const uint64_t strv[3] = {(uint64_t)a.v.stride_row * E, (uint64_t)a.v.stride_h * E,
-                              (uint64_t)a.v.stride_b * E};
-    if (!make_map(&mv, a.v.ptr, dims, strv, bv)) return cudaErrorInvalidValue;
-  }
+  if (!make_prefill_maps(a, B, D, key_rows_total, kv_token_major, BM, BN, 64, &mq, &mk, &mv, &mo))
+    return cudaErrorInvalidValue;
   TcArgs t;
   t.S = a.S;
   t.window = a.window;

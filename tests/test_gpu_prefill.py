@@ -134,15 +134,33 @@ PAIR_CASES = [
 ]
 
 
-@pytest.mark.parametrize("kernel", ["single", "pair"])
+@pytest.mark.parametrize("kernel", ["single", "pair", "hpair"])
 @pytest.mark.parametrize("case", PAIR_CASES, ids=lambda c: "B%dS%dH%d-%dD%dW%d%s%s" % (
     c["B"], c["S"], c["Hq"], c["Hkv"], c["D"], c["W"], "P" if c.get("prior") else "",
     "nan" if c.get("cache_fill") else ""))
 def test_prefill_each_kernel(oracle, monkeypatch, kernel, case):
-    """Both attention kernels (one query tile per CTA; two per CTA pair on
-    cta_group::2 MMAs) on ragged lengths, odd tile counts, a cached prefix,
-    and caches whose unused slots hold nan (the key tile that crosses the
-    sequence end must not let them reach an output)."""
+    """Every attention kernel (one query tile per CTA; two query tiles, or two
+    q heads of one KV head, per CTA pair on cta_group::2 MMAs) on ragged
+    lengths, odd tile counts, a cached prefix, and caches whose unused slots
+    hold nan (the key tile that crosses the sequence end must not let them
+    reach an output)."""
+    monkeypatch.setenv("GEMMA_PREFILL_KERNEL", kernel)
+    run_prefill_case(oracle, **case)
+
+
+WAVE_CASES = [
+    # more work items than SMs: several waves of CTAs or clusters
+    dict(B=2, S=1200, Hq=8, Hkv=4, D=256, W=128, frac=1.0, theta=1e4, seed=141),
+    dict(B=1, S=600, Hq=32, Hkv=4, D=256, W=0, frac=0.25, theta=1e6, seed=142, cache_fill=float("nan")),
+    dict(B=3, S=300, Hq=24, Hkv=12, D=256, W=0, frac=1.0, theta=1e4, seed=143, prior=[0, 129, 700]),
+]
+
+
+@pytest.mark.parametrize("kernel", ["single", "hpair"])
+@pytest.mark.parametrize("case", WAVE_CASES, ids=["W128", "global", "prior"])
+def test_prefill_more_tiles_than_sms(oracle, monkeypatch, kernel, case):
+    """More (query tile, head) items than SMs, so CTAs and CTA pairs run in
+    several waves with unequal key ranges."""
     monkeypatch.setenv("GEMMA_PREFILL_KERNEL", kernel)
     run_prefill_case(oracle, **case)
 
@@ -154,7 +172,7 @@ KEQV_CASES = [
 ]
 
 
-@pytest.mark.parametrize("kernel", ["single", "pair"])
+@pytest.mark.parametrize("kernel", ["single", "pair", "hpair"])
 @pytest.mark.parametrize("case", KEQV_CASES, ids=["D512", "D512P", "D256"])
 def test_prefill_k_equals_v(oracle, monkeypatch, kernel, case):
     """K = V (GEMMA_F_KEQV) on global layers: only the rotated keys are written
@@ -392,8 +410,11 @@ def run_local_chunk_case(oracle, *, B, S, Hq, Hkv, D, W, prior, seed, frac=1.0, 
     dict(B=1, S=700, Hq=8, Hkv=4, D=256, W=512, prior=[1000], seed=132),   # chunk longer than the window
     dict(B=2, S=1, Hq=4, Hkv=2, D=256, W=64, prior=[64, 129], seed=133),   # one-token chunks
     dict(B=1, S=130, Hq=8, Hkv=4, D=512, W=128, prior=[257], seed=134, frac=0.25, theta=1e6),
-], ids=["S200", "S700", "S1", "D512"])
-def test_prefill_local_chunk_after_cached_tokens(oracle, case):
+    dict(B=2, S=400, Hq=24, Hkv=12, D=256, W=512, prior=[1000, 5], seed=135),  # more tiles than SMs
+], ids=["S200", "S700", "S1", "D512", "H24"])
+@pytest.mark.parametrize("kernel", ["single", "hpair"])
+def test_prefill_local_chunk_after_cached_tokens(oracle, monkeypatch, kernel, case):
+    monkeypatch.setenv("GEMMA_PREFILL_KERNEL", kernel)
     run_local_chunk_case(oracle, **case)
 
 
