@@ -135,20 +135,38 @@ int cuda_fail(cudaError_t e, const char* what) {
   return fail(GEMMA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
 }
 
-// Split-K plan of a decode call: keys per split (multiple of 16) and splits
-// per (sequence, KV head). About 2048 keys per unit, the unit count rounded
-// up to whole waves of two CTAs per SM, so equal-length batches fill every
-// wave.
+// Split-K plan of a decode call: keys per split (a multiple of 16) and splits
+// per (sequence, KV head). Each unit is one CTA and two fit on an SM, so with
+// lengths near keys_max a call takes about (waves of units) x (keys per unit
+// + a fixed cost per unit). Long ranges aim at ~2048 keys per unit with the
+// unit count rounded up to whole waves. Ranges that fit in one such unit (a
+// local layer's ring) instead take the split count, 1 to 4 with at least 256
+// keys per unit, that minimises that cost: a batch of 64 sequences x 16 KV
+// heads is 3.46 waves of whole rings but 6.92 waves of half rings.
 void decode_plan(int B, int Hkv, int window, int max_len, int* chunk, int* n_splits) {
   const int64_t keys_max = window > 0 ? std::min<int64_t>(max_len, window) : max_len;
   const int64_t pairs = (int64_t)B * Hkv;
   const int64_t wave = (int64_t)sm_count() * 2;
+  const auto up16 = [](int64_t x) { return ((x + 15) / 16) * 16; };
   int64_t units = (keys_max * pairs + 2047) / 2048;
   units = ((units + wave - 1) / wave) * wave;
   int64_t c = (keys_max * pairs + units - 1) / units;
-  c = ((c + 15) / 16) * 16;
-  c = std::max<int64_t>(c, 256);
-  c = std::min<int64_t>(c, ((keys_max + 15) / 16) * 16);
+  c = std::max<int64_t>(up16(c), 256);
+  if (c >= keys_max) {
+    constexpr int64_t kUnitCost = 128;  // per-unit fixed cost, in keys streamed
+    int64_t best_cost = INT64_MAX;
+    c = up16(keys_max);
+    for (int64_t ns = 1; ns <= 4; ++ns) {
+      const int64_t cc = up16((keys_max + ns - 1) / ns);
+      if (ns > 1 && cc < 256) break;
+      if ((keys_max + cc - 1) / cc != ns) continue;  // same plan as a smaller count
+      const int64_t cost = ((pairs * ns + wave - 1) / wave) * (cc + kUnitCost);
+      if (cost < best_cost) {
+        best_cost = cost;
+        c = cc;
+      }
+    }
+  }
   *chunk = (int)c;
   *n_splits = (int)((keys_max + c - 1) / c);
 }

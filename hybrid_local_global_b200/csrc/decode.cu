@@ -13,9 +13,16 @@
 // shared by its G query heads. Work unit = (split of `chunk` keys, KV head,
 // sequence). Per CTA:
 //   warp 3      producer: for each 16-key sub-block, one lane arms the slot's
-//               full barrier with the byte count and 32 lanes issue one bulk
-//               copy per K/V row into a ring of padded shared-memory rows
-//               (row stride D*2+16 bytes keeps ldmatrix conflict-free).
+//               full barrier with the byte count and the lanes issue one bulk
+//               copy per group of RPC consecutive K or V rows (contiguous in
+//               the cache) into a ring of padded shared-memory row groups
+//               (group stride RPC*D*2+16 bytes). The copy engine takes about
+//               one bulk copy per 44 cycles per SM (measured on B200), which
+//               holds 512-byte rows (head_dim 256) to half the HBM rate, so
+//               head_dim 256 copies row pairs (ldmatrix then reads two rows
+//               per bank group); 1 KB rows (head_dim 512) go one per copy
+//               and stay conflict-free, which K = V, reading every row twice,
+//               needs.
 //   warps 0..2  consumers: sub-block t goes to warp t % 3 and ring slot
 //               t % NSLOT, with NSLOT a multiple of 3, so every slot has a
 //               single consumer that waits its phases strictly in order
@@ -45,12 +52,15 @@ namespace {
 
 constexpr int NCW = 3;  // consumer warps
 
-template <int D>
+template <int D, int RPC_>
 struct DecCfg {
   static constexpr int KB = 16;                 // keys per sub-block
-  static constexpr int ROW = D + 8;             // padded smem row (elements)
+  static constexpr int ROW = D + 8;             // padded smem row of Q (elements)
   static constexpr int ROWB = ROW * 2;          // bytes
-  static constexpr int SLOT_B = 2 * KB * ROWB;  // K rows then V rows
+  static constexpr int RPC = RPC_;                 // rows per bulk copy
+  static constexpr int GROUPB = RPC * D * 2 + 16;  // RPC consecutive K (or V) rows + 16 B pad
+  static constexpr int GPR = KB / RPC;             // row groups per 16-row region
+  static constexpr int SLOT_B = 2 * GPR * GROUPB;  // K region then V region (two K regions under K = V)
   static constexpr int NSLOT = (D == 256) ? 6 : 3;
   static_assert(NSLOT % NCW == 0, "each ring slot needs a single consumer warp");
   static constexpr int RING_B = NSLOT * SLOT_B;
@@ -89,13 +99,20 @@ __device__ __forceinline__ void mma_bf16(float (&c)[4], uint32_t a0, uint32_t a1
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+// byte offset of row r within a run of row groups
+template <int D, int RPC>
+__device__ __forceinline__ int group_row_off(int r) {
+  using C = DecCfg<D, RPC>;
+  return (r / C::RPC) * C::GROUPB + (r % C::RPC) * (D * 2);
+}
+
 __device__ __forceinline__ void named_bar_sync(int id, int n) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
 }
 
-template <int D>
+template <int D, int RPC>
 __global__ void __launch_bounds__(32 * (NCW + 1), 2) k_decode_split(DecodeAttnArgs a) {
-  using C = DecCfg<D>;
+  using C = DecCfg<D, RPC>;
   extern __shared__ __align__(128) unsigned char sm[];
   unsigned char* ring = sm;
   bf16* qs = reinterpret_cast<bf16*>(sm + C::RING_B);
@@ -171,11 +188,17 @@ __global__ void __launch_bounds__(32 * (NCW + 1), 2) k_decode_split(DecodeAttnAr
         issued[slot] += 1;
       }
       __syncwarp();
-      const int r = a.keqv ? lane : (lane & 15);
-      if (r < nk) {
-        const bool isv = !a.keqv && lane >= 16;  // K = V: 32 K rows, which are the values
-        bulk_g2s(ring + slot * C::SLOT_B + (isv ? C::KB * C::ROWB : 0) + r * C::ROWB,
-                 (isv ? vbase : kbase) + (key0 + r) * D, D * 2, &full[slot]);
+      // lanes 0..GPR-1: K row groups, GPR..2*GPR-1: V row groups (K = V:
+      // all 2*GPR lanes copy K rows, which are the values); a short tail
+      // group copies only the rows that exist
+      if (lane < 2 * C::GPR) {
+        const bool isv = !a.keqv && lane >= C::GPR;
+        const int grp = a.keqv ? lane : lane % C::GPR;
+        const int left = nk - grp * C::RPC;
+        if (left > 0)
+          bulk_g2s(ring + slot * C::SLOT_B + (isv ? C::GPR * C::GROUPB : 0) + grp * C::GROUPB,
+                   (isv ? vbase : kbase) + (key0 + grp * C::RPC) * D,
+                   (left >= C::RPC ? C::RPC : left) * D * 2, &full[slot]);
       }
     }
   } else {
@@ -186,7 +209,7 @@ __global__ void __launch_bounds__(32 * (NCW + 1), 2) k_decode_split(DecodeAttnAr
     for (int mt = 0; mt < D / 16; ++mt) o[mt][0] = o[mt][1] = o[mt][2] = o[mt][3] = 0.f;
     float m_h = -INFINITY, l_t = 0.f;
     const uint32_t q_addr = smem_u32(qs) + ((lane & 7) * C::ROW + ((lane >> 3) & 1) * 8) * 2;
-    const uint32_t frag_off = (((lane >> 4) * 8 + (lane & 7)) * C::ROW + ((lane >> 3) & 1) * 8) * 2;
+    const uint32_t frag_off = group_row_off<D, RPC>((lane >> 4) * 8 + (lane & 7)) + ((lane >> 3) & 1) * 16;
 
     for (int t = warp; t < n_sub; t += NCW) {
       const int slot = t % C::NSLOT;
@@ -197,11 +220,13 @@ __global__ void __launch_bounds__(32 * (NCW + 1), 2) k_decode_split(DecodeAttnAr
       const int nk_slot = (int)((k_end - key0_slot) < kps ? (k_end - key0_slot) : kps);
       if (nk_slot < kps) {
         // rows past the end were not copied: make them finite zeros
+        // (slot rows 0..15 are K, 16..31 V; under K = V all 32 are keys,
+        // and either way row r sits at group_row_off(r))
         unsigned char* rows = ring + slot * C::SLOT_B;
         for (int idx = lane; idx < 2 * C::KB * (D / 8); idx += 32) {
           const int r = idx / (D / 8), c = (idx % (D / 8)) * 8;
-          const int key = a.keqv ? r : (r & (C::KB - 1));  // K rows 0..15, V rows 16..31
-          if (key >= nk_slot) *reinterpret_cast<uint4*>(rows + r * C::ROWB + c * 2) = make_uint4(0, 0, 0, 0);
+          const int key = a.keqv ? r : (r & (C::KB - 1));
+          if (key >= nk_slot) *reinterpret_cast<uint4*>(rows + group_row_off<D, RPC>(r) + c * 2) = make_uint4(0, 0, 0, 0);
         }
         fence_proxy_async_smem();
         __syncwarp();
@@ -210,8 +235,8 @@ __global__ void __launch_bounds__(32 * (NCW + 1), 2) k_decode_split(DecodeAttnAr
       for (int half = 0; half < (a.keqv ? 2 : 1); ++half) {
       const int nk = nk_slot - half * C::KB;
       if (nk <= 0) break;
-      unsigned char* kslot = ring + slot * C::SLOT_B + half * C::KB * C::ROWB;
-      unsigned char* vslot = a.keqv ? kslot : kslot + C::KB * C::ROWB;
+      unsigned char* kslot = ring + slot * C::SLOT_B + half * C::GPR * C::GROUPB;
+      unsigned char* vslot = a.keqv ? kslot : kslot + C::GPR * C::GROUPB;
       // S = Q K^T : rows = query heads (8 real of 16), cols = 16 keys
       float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
       const uint32_t k_addr = smem_u32(kslot) + frag_off;
@@ -395,20 +420,26 @@ __global__ void __launch_bounds__(128) k_decode_combine(DecodeAttnArgs a) {
   }
 }
 
+template <int D, int RPC>
+cudaError_t launch_split(const DecodeAttnArgs& a, int B, cudaStream_t st) {
+  using C = DecCfg<D, RPC>;
+  cudaError_t e = cudaFuncSetAttribute(k_decode_split<D, RPC>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  if (e != cudaSuccess) return e;
+  k_decode_split<D, RPC><<<dim3(a.n_splits, a.Hkv, B), 32 * (NCW + 1), C::SMEM, st>>>(a);
+  return cudaGetLastError();
+}
+
 }  // namespace
 
+// Rows per bulk copy (measured on B200): head_dim 256 copies row pairs
+// (local layers of a 64-sequence 31B batch: 364 -> 247 us); head_dim 512
+// copies row pairs too (its 64-sequence global layer: 5.20 -> 4.97 ms),
+// except under K = V, whose consumers read every row twice and lose more to
+// the pairs' 2-way ldmatrix conflicts than they gain (256K tokens: 218 ->
+// 237 us), so there rows go one per copy.
 cudaError_t launch_decode_split(const DecodeAttnArgs& a, int B, int D, cudaStream_t st) {
-  dim3 grid(a.n_splits, a.Hkv, B);
-  if (D == 256) {
-    using C = DecCfg<256>;
-    cudaFuncSetAttribute(k_decode_split<256>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
-    k_decode_split<256><<<grid, 32 * (NCW + 1), C::SMEM, st>>>(a);
-  } else {
-    using C = DecCfg<512>;
-    cudaFuncSetAttribute(k_decode_split<512>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
-    k_decode_split<512><<<grid, 32 * (NCW + 1), C::SMEM, st>>>(a);
-  }
-  return cudaGetLastError();
+  if (D == 256) return launch_split<256, 2>(a, B, st);
+  return a.keqv ? launch_split<512, 1>(a, B, st) : launch_split<512, 2>(a, B, st);
 }
 
 cudaError_t launch_decode_combine(const DecodeAttnArgs& a, int B, int D, cudaStream_t st) {
