@@ -18,11 +18,10 @@
 //               the cache) into a ring of padded shared-memory row groups
 //               (group stride RPC*D*2+16 bytes). The copy engine takes about
 //               one bulk copy per 44 cycles per SM (measured on B200), which
-//               holds 512-byte rows (head_dim 256) to half the HBM rate, so
-//               head_dim 256 copies row pairs (ldmatrix then reads two rows
-//               per bank group); 1 KB rows (head_dim 512) go one per copy
-//               and stay conflict-free, which K = V, reading every row twice,
-//               needs.
+//               held one 512-byte row per copy (head_dim 256) to half the HBM
+//               rate; 2 KB copies (4 rows at head_dim 256, 2 at 512) lift
+//               that. The MMA fragments take the keys of a sub-block in an
+//               order (key_of) that spreads each ldmatrix over row groups.
 //   warps 0..2  consumers: sub-block t goes to warp t % 3 and ring slot
 //               t % NSLOT, with NSLOT a multiple of 3, so every slot has a
 //               single consumer that waits its phases strictly in order
@@ -104,6 +103,17 @@ template <int D, int RPC>
 __device__ __forceinline__ int group_row_off(int r) {
   using C = DecCfg<D, RPC>;
   return (r / C::RPC) * C::GROUPB + (r % C::RPC) * (D * 2);
+}
+
+// The key that MMA index n (0..15) of a 16-key sub-block stands for. S and
+// P.V only need the same order for the K and V fragments and the mask, so
+// the 8 rows each ldmatrix reads are taken from different row groups where
+// possible: rows of one group are D*2 bytes apart and share bank groups,
+// while consecutive groups are shifted by the 16-byte pad.
+template <int RPC>
+__device__ __forceinline__ int key_of(int n) {
+  constexpr int NG = 16 / RPC;  // row groups per 16 keys
+  return (n % NG) * RPC + n / NG;
 }
 
 __device__ __forceinline__ void named_bar_sync(int id, int n) {
@@ -209,7 +219,7 @@ __global__ void __launch_bounds__(32 * (NCW + 1), 2) k_decode_split(DecodeAttnAr
     for (int mt = 0; mt < D / 16; ++mt) o[mt][0] = o[mt][1] = o[mt][2] = o[mt][3] = 0.f;
     float m_h = -INFINITY, l_t = 0.f;
     const uint32_t q_addr = smem_u32(qs) + ((lane & 7) * C::ROW + ((lane >> 3) & 1) * 8) * 2;
-    const uint32_t frag_off = group_row_off<D, RPC>((lane >> 4) * 8 + (lane & 7)) + ((lane >> 3) & 1) * 16;
+    const uint32_t frag_off = group_row_off<D, RPC>(key_of<RPC>((lane >> 4) * 8 + (lane & 7))) + ((lane >> 3) & 1) * 16;
 
     for (int t = warp; t < n_sub; t += NCW) {
       const int slot = t % C::NSLOT;
@@ -248,12 +258,13 @@ __global__ void __launch_bounds__(32 * (NCW + 1), 2) k_decode_split(DecodeAttnAr
         mma_bf16(s0, qa0, 0u, qa2, 0u, b0, b1);
         mma_bf16(s1, qa0, 0u, qa2, 0u, b2, b3);
       }
-      // online softmax for head gq; this thread holds keys 2tg,2tg+1 and 8+2tg,8+2tg+1
+      // online softmax for head gq; this thread holds MMA columns 2tg, 2tg+1,
+      // 8+2tg, 9+2tg, i.e. keys key_of() of those
       float sv[4];
-      sv[0] = (2 * tg < nk) ? s0[0] * a.scale_log2 : -INFINITY;
-      sv[1] = (2 * tg + 1 < nk) ? s0[1] * a.scale_log2 : -INFINITY;
-      sv[2] = (8 + 2 * tg < nk) ? s1[0] * a.scale_log2 : -INFINITY;
-      sv[3] = (9 + 2 * tg < nk) ? s1[1] * a.scale_log2 : -INFINITY;
+      sv[0] = (key_of<RPC>(2 * tg) < nk) ? s0[0] * a.scale_log2 : -INFINITY;
+      sv[1] = (key_of<RPC>(2 * tg + 1) < nk) ? s0[1] * a.scale_log2 : -INFINITY;
+      sv[2] = (key_of<RPC>(8 + 2 * tg) < nk) ? s1[0] * a.scale_log2 : -INFINITY;
+      sv[3] = (key_of<RPC>(9 + 2 * tg) < nk) ? s1[1] * a.scale_log2 : -INFINITY;
       float tmax = fmaxf(fmaxf(sv[0], sv[1]), fmaxf(sv[2], sv[3]));
       tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 1));
       tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 2));
@@ -431,15 +442,13 @@ cudaError_t launch_split(const DecodeAttnArgs& a, int B, cudaStream_t st) {
 
 }  // namespace
 
-// Rows per bulk copy (measured on B200): head_dim 256 copies row pairs
-// (local layers of a 64-sequence 31B batch: 364 -> 247 us); head_dim 512
-// copies row pairs too (its 64-sequence global layer: 5.20 -> 4.97 ms),
-// except under K = V, whose consumers read every row twice and lose more to
-// the pairs' 2-way ldmatrix conflicts than they gain (256K tokens: 218 ->
-// 237 us), so there rows go one per copy.
+// Rows per bulk copy (measured on B200, with key_of's fragment order):
+// head_dim 256 copies groups of 4 rows (2 KB; the local layers of a
+// 64-sequence 31B batch: 348 us at one row per copy, 226 at pairs, 185 at 4,
+// 205 at 8 rows); head_dim 512 copies pairs (2 KB; that batch's global layer
+// 5.20 -> 4.87 ms, 256K tokens with K = V 219 -> 210 us).
 cudaError_t launch_decode_split(const DecodeAttnArgs& a, int B, int D, cudaStream_t st) {
-  if (D == 256) return launch_split<256, 2>(a, B, st);
-  return a.keqv ? launch_split<512, 1>(a, B, st) : launch_split<512, 2>(a, B, st);
+  return D == 256 ? launch_split<256, 4>(a, B, st) : launch_split<512, 2>(a, B, st);
 }
 
 cudaError_t launch_decode_combine(const DecodeAttnArgs& a, int B, int D, cudaStream_t st) {
