@@ -214,7 +214,14 @@ def bench_prefill(args, w, dev, world, peaks):
             else "fallback 1.59 PF/s", "traffic": None,
             "per_launch": "algorithmic FLOPs of all attention launches / their summed device time "
                           "(%d launches, %d per step)" % (attn["launches"], st.n_layers)}
-    rec = recorded_traffic("k_prefill_tc", w.name)
+    # the kernel that runs each layer type: CTA pairs on head_dim 512 (both
+    # model shapes have an even number of q heads per KV head), one CTA per
+    # query tile on head_dim 256
+    rec = {}
+    for kind, lt in (("local", w.local), ("global", w.global_)):
+        r = recorded_traffic("k_prefill_pair" if lt.head_dim == 512 else "k_prefill_tc", w.name)
+        if kind in r:
+            rec[kind] = r[kind]
     kinds = ["global" if g else "local" for g in st.is_global]
     if all(k in rec for k in kinds):
         roof["traffic"] = round(sum(float(rec[k]["bytes"]) for k in kinds) / len(kinds))

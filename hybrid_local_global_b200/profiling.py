@@ -36,8 +36,8 @@ CSRC = os.path.join(os.path.dirname(os.path.abspath(__file__)), "csrc")
 
 # the sources each recorded kernel is built from
 KERNEL_SOURCES = {
-    "k_prefill_tc": ("prefill_tc.cu", "tc.cuh", "common.cuh"),
-    "k_prefill_pair": ("prefill_pair.cu", "pair.cuh", "tc.cuh", "common.cuh"),
+    "k_prefill_tc": ("prefill_tc.cu", "tc.cuh", "common.cuh", "tmap.cu", "tmap.h"),
+    "k_prefill_pair": ("prefill_pair.cu", "pair.cuh", "tc.cuh", "common.cuh", "tmap.cu", "tmap.h"),
     "k_decode_split": ("decode.cu", "common.cuh"),
 }
 
