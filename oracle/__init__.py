@@ -6,7 +6,10 @@ package. The product (``hybrid_local_global_b200``) never imports it and
 shares no code with it; the arithmetic lives in ``hlg_oracle.c`` (plain C,
 fp64, no blocking or reordering beyond the definition).
 
-Inputs are bf16 bit patterns (``numpy.uint16``); outputs are fp64.
+Inputs are bf16 bit patterns (``numpy.uint16``); outputs are fp64. The
+int8 KV pieces (``quantize_rows_u8``, ``dequantize_rows_u8``) take their
+code decision in fp32, and ``attend_rows`` attends over given fp64 keys and
+values (already rotated), e.g. dequantized cache rows.
 Citations of the pages are in the C file next to each function.
 """
 from __future__ import annotations
@@ -59,6 +62,10 @@ def _load():
         lib.hlg_stack_cache_bytes.argtypes = [i32, i32, i32, i64, i32, i32, i32, i64,
                                               i32, i32, i64, i32, i32]
         lib.hlg_stack_cache_bytes.restype = i64
+        lib.hlg_quantize_rows_u8.argtypes = [p, i64, i32, p, p, p]
+        lib.hlg_dequantize_rows_u8.argtypes = [p, p, p, i64, i32, p]
+        lib.hlg_dequantize_rows_u8.restype = None
+        lib.hlg_attend_rows.argtypes = [p, p, p, i64, p, p, i64, i32, f64, p, p]
         _lib = lib
     return _lib
 
@@ -168,3 +175,46 @@ def stack_cache_bytes(n_layers: int, ratio: int, n_shared: int, batch: int, *,
                                              local_kv_heads, local_head_dim, local_capacity,
                                              global_kv_heads, global_head_dim, global_capacity,
                                              int(global_k_equals_v), w))
+
+
+def quantize_rows_u8(x_bits: np.ndarray):
+    """int8 KV rows (see hlg_quantize_rows_u8): x_bits uint16 bf16 [..., D] ->
+    (codes uint8 [..., D], lo float32 [...], step float32 [...])."""
+    x = np.ascontiguousarray(x_bits, dtype=np.uint16)
+    D = x.shape[-1]
+    n = x.size // D
+    codes = np.zeros(x.shape, dtype=np.uint8)
+    lo = np.zeros(x.shape[:-1], dtype=np.float32)
+    step = np.zeros(x.shape[:-1], dtype=np.float32)
+    if _load().hlg_quantize_rows_u8(_ptr(x), n, D, _ptr(codes), _ptr(lo), _ptr(step)) != 0:
+        raise ValueError("oracle rejected the arguments")
+    return codes, lo, step
+
+
+def dequantize_rows_u8(codes: np.ndarray, lo: np.ndarray, step: np.ndarray) -> np.ndarray:
+    """min + code * step, fp64, same shape as codes."""
+    c = np.ascontiguousarray(codes, dtype=np.uint8)
+    lo = np.ascontiguousarray(lo, dtype=np.float32)
+    step = np.ascontiguousarray(step, dtype=np.float32)
+    D = c.shape[-1]
+    out = np.zeros(c.shape, dtype=np.float64)
+    _load().hlg_dequantize_rows_u8(_ptr(c), _ptr(lo), _ptr(step), c.size // D, D, _ptr(out))
+    return out
+
+
+def attend_rows(q: np.ndarray, k: np.ndarray, v: np.ndarray, key_begin, key_count, scale: float):
+    """Attention of fp64 query rows q [R, D] over keys/values k, v [N, D]
+    (fp64, already rotated): row r reads rows key_begin[r] .. +key_count[r].
+    Returns (out fp64 [R, D], lse fp64 [R])."""
+    q = np.ascontiguousarray(q, dtype=np.float64)
+    k = np.ascontiguousarray(k, dtype=np.float64)
+    v = np.ascontiguousarray(v, dtype=np.float64)
+    R, D = q.shape
+    kb = np.ascontiguousarray(np.broadcast_to(np.asarray(key_begin, np.int64), (R,)))
+    kc = np.ascontiguousarray(np.broadcast_to(np.asarray(key_count, np.int64), (R,)))
+    out = np.zeros((R, D), dtype=np.float64)
+    lse = np.zeros(R, dtype=np.float64)
+    if _load().hlg_attend_rows(_ptr(q), _ptr(k), _ptr(v), k.shape[0], _ptr(kb), _ptr(kc), R, D, scale,
+                               _ptr(out), _ptr(lse)) != 0:
+        raise ValueError("oracle rejected the arguments")
+    return out, lse

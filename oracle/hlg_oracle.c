@@ -398,3 +398,98 @@ int64_t hlg_stack_cache_bytes(int n_layers, int ratio, int n_shared,
     }
     return total;
 }
+
+/* ------------------------------------------------------------------------ */
+/* int8 KV cache rows. "Gemma 4 Technical Report", Quantization and        */
+/* Efficiency: a quantizer maps a channel's [min, max] onto the 2^b codes   */
+/* with scale = (2^b - 1) / (max - min) and code = round((x - min) * scale),*/
+/* and the dequantizer returns min + code / scale; Table 3 lists int8 KV    */
+/* caching. Reading: b = 8, one (min, step) pair per cached row (one token, */
+/* one KV head, all D channels), codes 0..255, round half to even, every    */
+/* step of the code decision in fp32, step = (max - min) / 255 stored for   */
+/* the dequantizer (min + code * step), and a constant row gets codes 0 and */
+/* step 0. Inputs are bf16 (the rounded rotated keys, or the values).       */
+/* ------------------------------------------------------------------------ */
+int hlg_quantize_rows_u8(const uint16_t* x_bits, int64_t n_rows, int D, uint8_t* codes,
+                         float* lo_out, float* step_out)
+{
+    if (!x_bits || !codes || !lo_out || !step_out || n_rows < 0 || D <= 0)
+        return 1;
+    for (int64_t r = 0; r < n_rows; ++r) {
+        const uint16_t* x = x_bits + r * D;
+        float lo = (float)bf16_bits_to_double(x[0]), hi = lo;
+        for (int d = 1; d < D; ++d) {
+            float v = (float)bf16_bits_to_double(x[d]);
+            if (v < lo) lo = v;
+            if (v > hi) hi = v;
+        }
+        volatile float range = hi - lo;      /* fp32, rounded once */
+        if (range > 0.0f) {
+            volatile float scale = 255.0f / range;
+            for (int d = 0; d < D; ++d) {
+                volatile float off = (float)bf16_bits_to_double(x[d]) - lo;
+                volatile float t = off * scale;
+                float c = nearbyintf(t);     /* default rounding: to nearest, ties to even */
+                if (c < 0.0f) c = 0.0f;
+                if (c > 255.0f) c = 255.0f;
+                codes[r * D + d] = (uint8_t)c;
+            }
+            step_out[r] = range / 255.0f;
+        } else {
+            for (int d = 0; d < D; ++d)
+                codes[r * D + d] = 0;
+            step_out[r] = 0.0f;
+        }
+        lo_out[r] = lo;
+    }
+    return 0;
+}
+
+/* The dequantized row, in fp64: min + code * step. */
+void hlg_dequantize_rows_u8(const uint8_t* codes, const float* lo, const float* step,
+                            int64_t n_rows, int D, double* out)
+{
+    for (int64_t r = 0; r < n_rows; ++r)
+        for (int d = 0; d < D; ++d)
+            out[r * D + d] = (double)lo[r] + (double)codes[r * D + d] * (double)step[r];
+}
+
+/* Attention of one query row over a given list of keys and values (fp64,   */
+/* already rotated), the definition written out ("Gemma 4: End-to-End       */
+/* Architecture Walkthrough", 3a): s_j = scale <q, k_j>, out = sum_j        */
+/* softmax(s)_j v_j, lse = log sum_j exp(s_j). Row r reads keys             */
+/* key_begin[r] .. key_begin[r] + key_count[r] - 1 of k and v ([n][D]).     */
+int hlg_attend_rows(const double* q, const double* k, const double* v, int64_t n_keys_total,
+                    const int64_t* key_begin, const int64_t* key_count, int64_t n_rows, int D,
+                    double scale, double* out, double* lse)
+{
+    for (int64_t r = 0; r < n_rows; ++r) {
+        int64_t b = key_begin[r], n = key_count[r];
+        if (b < 0 || n < 1 || b + n > n_keys_total)
+            return 1;
+        double* s = (double*)malloc((size_t)n * sizeof(double));
+        if (!s)
+            return 2;
+        double m = -INFINITY;
+        for (int64_t j = 0; j < n; ++j) {
+            double acc = 0.0;
+            for (int d = 0; d < D; ++d)
+                acc += q[r * D + d] * k[(b + j) * D + d];
+            s[j] = scale * acc;
+            if (s[j] > m)
+                m = s[j];
+        }
+        double z = 0.0;
+        for (int64_t j = 0; j < n; ++j)
+            z += exp(s[j] - m);
+        for (int d = 0; d < D; ++d) {
+            double acc = 0.0;
+            for (int64_t j = 0; j < n; ++j)
+                acc += exp(s[j] - m) * v[(b + j) * D + d];
+            out[r * D + d] = acc / z;
+        }
+        lse[r] = m + log(z);
+        free(s);
+    }
+    return 0;
+}
