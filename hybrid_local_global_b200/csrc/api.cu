@@ -171,13 +171,16 @@ void decode_plan(int B, int Hkv, int window, int max_len, int* chunk, int* n_spl
   *n_splits = (int)((keys_max + c - 1) / c);
 }
 
-size_t decode_ws_parts(int B, int Hq, int D, int n_splits, size_t* off_lse, size_t* off_o) {
+size_t decode_ws_parts(int B, int Hq, int Hkv, int D, int n_splits, size_t* off_lse, size_t* off_o,
+                       size_t* off_kst = nullptr) {
   size_t q = align256((size_t)B * Hq * D * 2);
   size_t lse = align256((size_t)B * Hq * n_splits * 4);
   size_t o = align256((size_t)B * Hq * n_splits * D * 4);
+  size_t kst = align256((size_t)B * Hkv * D * 2);  // int8 cache: the rotated new key before quantization
+  if (off_kst) *off_kst = q + lse + o;
   *off_lse = q;
   *off_o = q + lse;
-  return q + lse + o;
+  return q + lse + o + kst;
 }
 
 // Prefill workspace: rotated Q, then on local layers either the rotated K
@@ -186,7 +189,8 @@ size_t decode_ws_parts(int B, int Hq, int D, int n_splits, size_t* off_lse, size
 size_t prefill_ws_parts(int B, int S, int Hq, int Hkv, int D, int window, size_t* off_k,
                         size_t* off_vw = nullptr) {
   size_t q = align256((size_t)B * S * Hq * D * 2);
-  size_t k = window > 0 ? align256((size_t)B * S * Hkv * D * 2) : 0;
+  // rotated K of the chunk: local layers, and global layers with an int8 cache
+  size_t k = align256((size_t)B * S * Hkv * D * 2);
   size_t win = window > 0 ? align256((size_t)B * (window + S) * Hkv * D * 2) : 0;
   *off_k = q;
   if (off_vw) *off_vw = q + win;
@@ -246,7 +250,8 @@ int gemma_layer_schedule(int n_layers, int ratio, int n_shared, int* is_global, 
 // key cache under K = V.
 static int check_kv_flags(unsigned flags, int window, const void* k_new, const void* v_new, void* k_cache,
                           void** v_cache_io) {
-  if (flags & ~(GEMMA_F_SHARED | GEMMA_F_KEQV)) return fail(GEMMA_ERR_INVALID_ARG, "unknown flags 0x%x", flags);
+  if (flags & ~(GEMMA_F_SHARED | GEMMA_F_KEQV | GEMMA_F_KV_INT8))
+    return fail(GEMMA_ERR_INVALID_ARG, "unknown flags 0x%x", flags);
   const bool shared = flags & GEMMA_F_SHARED, keqv = flags & GEMMA_F_KEQV;
   if (keqv && window > 0)
     return fail(GEMMA_ERR_UNSUPPORTED, "GEMMA_F_KEQV: K = V is defined for global layers only");
@@ -275,14 +280,51 @@ int gemma_kv_share_bind(gemma_kv_desc* dst, const gemma_kv_desc* src) {
   if (src->window != dst->window || src->cache_cap != dst->cache_cap ||
       src->n_kv_heads != dst->n_kv_heads || src->head_dim != dst->head_dim ||
       src->rope_frac != dst->rope_frac || src->rope_theta != dst->rope_theta ||
-      (src->k_eq_v != 0) != (dst->k_eq_v != 0))
+      (src->k_eq_v != 0) != (dst->k_eq_v != 0) || (src->kv_int8 != 0) != (dst->kv_int8 != 0))
     return fail(GEMMA_ERR_SHARE_MISMATCH,
-                "layers %d and %d differ in window, capacity, KV heads, head_dim, RoPE or K = V",
+                "layers %d and %d differ in window, capacity, KV heads, head_dim, RoPE, K = V or int8 KV",
                 src->layer, dst->layer);
   dst->k_cache = src->k_cache;
   dst->v_cache = src->v_cache;
   dst->shared_from = src->shared_from >= 0 ? src->shared_from : src->layer;
   return succeed();
+}
+
+size_t gemma_kv_codes_bytes(int batch, int n_kv_heads, int cache_cap, int head_dim) {
+  if (batch <= 0 || n_kv_heads <= 0 || cache_cap <= 0 || head_dim <= 0) return 0;
+  return align256((size_t)batch * n_kv_heads * cache_cap * head_dim);
+}
+
+size_t gemma_kv_cache_bytes(int batch, int n_kv_heads, int cache_cap, int head_dim, unsigned flags) {
+  if (batch <= 0 || n_kv_heads <= 0 || cache_cap <= 0 || head_dim <= 0) return 0;
+  const size_t rows = (size_t)batch * n_kv_heads * cache_cap;
+  if (flags & GEMMA_F_KV_INT8) return gemma_kv_codes_bytes(batch, n_kv_heads, cache_cap, head_dim) + rows * 8;
+  return rows * head_dim * 2;
+}
+
+// int8 cache rows of one call's new tokens: K from the rotated staging rows,
+// V from the caller's values (none under K = V)
+static cudaError_t quantize_kv(const bf16* k_src, const bf16* v_src, void* k_cache, void* v_cache, int batch,
+                               int S, int Hkv, int D, int window, int cache_cap, const int32_t* pos0,
+                               int pos0_minus, int* status, cudaStream_t st) {
+  const size_t off = gemma_kv_codes_bytes(batch, Hkv, cache_cap, D);
+  QuantRowsArgs qa{};
+  qa.S = S;
+  qa.Hkv = Hkv;
+  qa.window = window;
+  qa.cache_cap = cache_cap;
+  qa.pos0 = pos0;
+  qa.pos0_minus = pos0_minus;
+  qa.status = status;
+  qa.src = k_src;
+  qa.codes = static_cast<uint8_t*>(k_cache);
+  qa.params = reinterpret_cast<float2*>(static_cast<uint8_t*>(k_cache) + off);
+  cudaError_t e = launch_quantize_rows(qa, batch, D, st);
+  if (e != cudaSuccess || !v_src) return e;
+  qa.src = v_src;
+  qa.codes = static_cast<uint8_t*>(v_cache);
+  qa.params = reinterpret_cast<float2*>(static_cast<uint8_t*>(v_cache) + off);
+  return launch_quantize_rows(qa, batch, D, st);
 }
 
 size_t gemma_attn_prefill_workspace_size(int batch, int s_new, int n_q_heads, int n_kv_heads,
@@ -303,6 +345,14 @@ int gemma_attn_prefill(const void* q, const void* k_new, const void* v_new, void
   if (rc) return rc;
   if (batch <= 0 || s_new < 0) return fail(GEMMA_ERR_INVALID_ARG, "batch %d, s_new %d", batch, s_new);
   const bool shared = flags & GEMMA_F_SHARED;
+  const bool q8 = flags & GEMMA_F_KV_INT8;
+  const bool keqv = flags & GEMMA_F_KEQV;
+  if (q8) {
+    if (cache_cap % 2) return fail(GEMMA_ERR_INVALID_ARG, "int8 KV: cache_cap %d must be even", cache_cap);
+    if (seq_lens_before)
+      return fail(GEMMA_ERR_UNSUPPORTED, "int8 KV: prefill after cached tokens would read int8 rows");
+    if (shared) return fail(GEMMA_ERR_UNSUPPORTED, "int8 KV: a shared layer's prefill would read int8 rows");
+  }
   if (!q || !out || !k_cache || !v_cache) return fail(GEMMA_ERR_INVALID_ARG, "null tensor pointer");
   if (!aligned16(q) || !aligned16(out) || !aligned16(k_cache) || !aligned16(v_cache) ||
       (k_new && !aligned16(k_new)) || (v_new && !aligned16(v_new)) || !aligned16(workspace))
@@ -331,12 +381,12 @@ int gemma_attn_prefill(const void* q, const void* k_new, const void* v_new, void
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   unsigned char* ws = static_cast<unsigned char*>(workspace);
 
-  PrefillRopeArgs ra;
+  PrefillRopeArgs ra{};
   ra.q = static_cast<const bf16*>(q);
   ra.k_new = static_cast<const bf16*>(k_new);
   ra.v_new = static_cast<const bf16*>(v_new);
   ra.q_rot = reinterpret_cast<bf16*>(ws);
-  ra.k_rot = (window > 0 && !shared) ? reinterpret_cast<bf16*>(ws + off_k) : nullptr;
+  ra.k_rot = ((window > 0 && !shared) || q8) ? reinterpret_cast<bf16*>(ws + off_k) : nullptr;
   ra.v_win = chunked_local ? reinterpret_cast<bf16*>(ws + off_vw) : nullptr;
   ra.win_rows = win_rows;
   if (chunked_local) {
@@ -359,16 +409,20 @@ int gemma_attn_prefill(const void* q, const void* k_new, const void* v_new, void
   // queries carry scale * log2(e): the attention kernel's logits are then in
   // log2 units (one bf16 rounding either way)
   ra.q_scale = (float)((double)scale * 1.4426950408889634);
+  ra.quant = q8 ? 1 : 0;
   ra.status = status;
   ProfScope p_rope(GEMMA_KERNEL_PREFILL_ROPE, st);
   cudaError_t e = launch_prefill_rope(ra, batch, head_dim, st);
+  if (e == cudaSuccess && q8)
+    e = quantize_kv(ra.k_rot, keqv ? nullptr : ra.v_new, k_cache, v_cache, batch, s_new, n_kv_heads, head_dim,
+                    window, cache_cap, nullptr, 0, status, st);
   p_rope.done();
   if (e != cudaSuccess) return cuda_fail(e, "prefill rope launch");
 
-  PrefillAttnArgs aa;
+  PrefillAttnArgs aa{};
   aa.q_rot = ra.q_rot;
   const int64_t D = head_dim;
-  if (window == 0 || shared) {
+  if ((window == 0 || shared) && !q8) {
     KVView kc = {static_cast<const bf16*>(k_cache), (int64_t)n_kv_heads * cache_cap * D, D, (int64_t)cache_cap * D};
     KVView vc = {static_cast<const bf16*>(v_cache), kc.stride_b, kc.stride_row, kc.stride_h};
     aa.k = kc;
@@ -381,8 +435,9 @@ int gemma_attn_prefill(const void* q, const void* k_new, const void* v_new, void
     aa.v = vw;
     aa.key_cap = win_rows;
   } else {
+    // the chunk's rotated K and the caller's V (K = V: the rotated K again)
     KVView kw = {ra.k_rot, (int64_t)s_new * n_kv_heads * D, (int64_t)n_kv_heads * D, D};
-    KVView vw = {static_cast<const bf16*>(v_new), kw.stride_b, kw.stride_row, kw.stride_h};
+    KVView vw = {keqv ? ra.k_rot : static_cast<const bf16*>(v_new), kw.stride_b, kw.stride_row, kw.stride_h};
     aa.k = kw;
     aa.v = vw;
     aa.key_cap = s_new;
@@ -398,7 +453,7 @@ int gemma_attn_prefill(const void* q, const void* k_new, const void* v_new, void
   aa.lse = lse;
   aa.status = status;
   aa.wait_ns = (unsigned long long)g_wait_ns.load();
-  const bool cache_view = (window == 0 || shared);
+  const bool cache_view = (window == 0 || shared) && !q8;
   ProfScope p_attn(GEMMA_KERNEL_PREFILL_ATTN, st);
   // Head_dim-512 layers run on CTA pairs (cta_group::2, M = 256): each SM
   // loads and reads from shared memory half of every K and V tile. With an
@@ -435,7 +490,7 @@ size_t gemma_attn_decode_workspace_size(int batch, int n_q_heads, int n_kv_heads
   int chunk, n_splits;
   decode_plan(batch, n_kv_heads, window, max_seq_len, &chunk, &n_splits);
   size_t a, b;
-  return decode_ws_parts(batch, n_q_heads, head_dim, n_splits, &a, &b);
+  return decode_ws_parts(batch, n_q_heads, n_kv_heads, head_dim, n_splits, &a, &b);
 }
 
 int gemma_attn_decode(const void* q, const void* k_new, const void* v_new, void* k_cache, void* v_cache,
@@ -458,10 +513,12 @@ int gemma_attn_decode(const void* q, const void* k_new, const void* v_new, void*
     return fail(GEMMA_ERR_INVALID_ARG, "local layer: cache_cap %d must equal window %d", cache_cap, window);
   if (window == 0 && cache_cap < max_seq_len)
     return fail(GEMMA_ERR_CAPACITY, "global layer: cache_cap %d < max_seq_len %d", cache_cap, max_seq_len);
+  const bool q8 = flags & GEMMA_F_KV_INT8;
+  if (q8 && cache_cap % 2) return fail(GEMMA_ERR_INVALID_ARG, "int8 KV: cache_cap %d must be even", cache_cap);
   int chunk, n_splits;
   decode_plan(batch, n_kv_heads, window, max_seq_len, &chunk, &n_splits);
-  size_t off_lse, off_o;
-  size_t need = decode_ws_parts(batch, n_q_heads, head_dim, n_splits, &off_lse, &off_o);
+  size_t off_lse, off_o, off_kst;
+  size_t need = decode_ws_parts(batch, n_q_heads, n_kv_heads, head_dim, n_splits, &off_lse, &off_o, &off_kst);
   if (!workspace || workspace_bytes < need)
     return fail(GEMMA_ERR_CAPACITY, "workspace %zu bytes < %zu", workspace_bytes, need);
   int* status = status_ptr();
@@ -469,7 +526,7 @@ int gemma_attn_decode(const void* q, const void* k_new, const void* v_new, void*
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   unsigned char* ws = static_cast<unsigned char*>(workspace);
 
-  DecodeRopeArgs ra;
+  DecodeRopeArgs ra{};
   ra.q = static_cast<const bf16*>(q);
   ra.k_new = static_cast<const bf16*>(k_new);
   ra.v_new = static_cast<const bf16*>(v_new);
@@ -484,14 +541,19 @@ int gemma_attn_decode(const void* q, const void* k_new, const void* v_new, void*
   ra.Hkv = n_kv_heads;
   ra.n_rot = rope_rotated_pairs(head_dim, rope_frac);
   ra.log2_theta = std::log2((double)rope_theta);
+  ra.k_stage = q8 ? reinterpret_cast<bf16*>(ws + off_kst) : nullptr;
   ra.status = status;
-  // rotates q; also appends the new K/V unless the layer is shared
+  // rotates q; also appends the new K/V unless the layer is shared (int8:
+  // the rotated key is staged, then both rows are quantized into the cache)
   ProfScope p_app(GEMMA_KERNEL_DECODE_APPEND, st);
   cudaError_t e = launch_decode_rope_append(ra, batch, head_dim, st);
+  if (e == cudaSuccess && q8 && k_new)
+    e = quantize_kv(ra.k_stage, (flags & GEMMA_F_KEQV) ? nullptr : ra.v_new, k_cache, v_cache, batch, 1,
+                    n_kv_heads, head_dim, window, cache_cap, seq_lens, 1, status, st);
   p_app.done();
   if (e != cudaSuccess) return cuda_fail(e, "decode append launch");
 
-  DecodeAttnArgs da;
+  DecodeAttnArgs da{};
   da.q_rot = ra.q_rot;
   da.k_cache = static_cast<const bf16*>(k_cache);
   da.v_cache = static_cast<const bf16*>(v_cache);
@@ -511,9 +573,16 @@ int gemma_attn_decode(const void* q, const void* k_new, const void* v_new, void*
   da.wait_ns = (unsigned long long)g_wait_ns.load();
   da.drop_first_copy = g_drop_next.exchange(0);
   da.keqv = (flags & GEMMA_F_KEQV) ? 1 : 0;
+  if (q8) {
+    const size_t off = gemma_kv_codes_bytes(batch, n_kv_heads, cache_cap, head_dim);
+    da.k_codes = static_cast<const uint8_t*>(k_cache);
+    da.v_codes = static_cast<const uint8_t*>(v_cache);
+    da.k_params = reinterpret_cast<const float2*>(static_cast<const uint8_t*>(k_cache) + off);
+    da.v_params = reinterpret_cast<const float2*>(static_cast<const uint8_t*>(v_cache) + off);
+  }
   {
     ProfScope p_split(GEMMA_KERNEL_DECODE_SPLIT, st);
-    e = launch_decode_split(da, batch, head_dim, st);
+    e = q8 ? launch_decode_split_q8(da, batch, head_dim, st) : launch_decode_split(da, batch, head_dim, st);
     p_split.done();
   }
   if (e != cudaSuccess) return cuda_fail(e, "decode attention launch");

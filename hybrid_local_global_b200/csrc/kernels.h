@@ -26,6 +26,8 @@ struct PrefillRopeArgs {
   int n_rot;           // rotated pairs
   double log2_theta;
   float q_scale;       // rotated Q is multiplied by this before the bf16 rounding
+  int quant;           // int8 cache: rotated K goes to k_rot ([B][S][Hkv][D]) on every layer
+                       // type and nothing is written into the cache (launch_quantize_rows does)
   int* status;
 };
 
@@ -36,11 +38,29 @@ struct DecodeRopeArgs {
   bf16* q_rot;         // workspace [B][Hq][D]
   bf16* k_cache;
   bf16* v_cache;
+  bf16* k_stage;       // int8 cache: the rotated new key goes here ([B][Hkv][D]) and nothing
+                       // is written into the cache (launch_quantize_rows does); else null
   int cache_cap;
   const int32_t* seq_lens;
   int max_len, window, Hq, Hkv;
   int n_rot;
   double log2_theta;
+  int* status;
+};
+
+// int8 cache rows: the bf16 rows src + ((b * S + s) * Hkv + h) * D (b < B,
+// s < S, h < Hkv) at positions pos = pos0[b] - pos0_minus + s are quantized
+// (per row: min, step = (max - min) / 255, codes round((x - min) * 255 /
+// (max - min)), fp32) into slot pos (global) or pos % window (local, only
+// the last `window` rows of the chunk) of codes [B][Hkv][cap][D] and
+// params [B][Hkv][cap] (min, step).
+struct QuantRowsArgs {
+  const bf16* src;
+  int S, Hkv, window, cache_cap;
+  const int32_t* pos0;  // device [B], or null for 0
+  int pos0_minus;
+  uint8_t* codes;
+  float2* params;
   int* status;
 };
 
@@ -84,6 +104,11 @@ struct DecodeAttnArgs {
   unsigned long long wait_ns;
   int drop_first_copy;     // test hook: skip the first K/V copy of split 0
   int keqv;                // K = V: only K rows are loaded and serve as V
+  // int8 cache (k_cache/v_cache unused): codes [B][Hkv][cap][D] and per-row (min, step)
+  const uint8_t* k_codes;
+  const uint8_t* v_codes;
+  const float2* k_params;
+  const float2* v_params;
 };
 
 cudaError_t launch_prefill_rope(const PrefillRopeArgs& a, int B, int D, cudaStream_t st);
@@ -94,6 +119,7 @@ cudaError_t launch_ring_gather(const bf16* k_cache, const bf16* v_cache, const i
                                int B, int Hkv, int D, int window, int win_rows, bf16* k_win, bf16* v_win,
                                int* status, cudaStream_t st);
 cudaError_t launch_decode_rope_append(const DecodeRopeArgs& a, int B, int D, cudaStream_t st);
+cudaError_t launch_quantize_rows(const QuantRowsArgs& a, int B, int D, cudaStream_t st);
 // tcgen05 prefill (head_dim 256 or 512). key_rows_total = rows of the K/V
 // views; kv_token_major: views are [B][rows][Hkv][D] (1) or [B][Hkv][rows][D] (0).
 // _tc: one CTA per 128-row query tile; _pair: two query tiles on a CTA pair
@@ -105,6 +131,8 @@ cudaError_t launch_prefill_attn_tc(const PrefillAttnArgs& a, int B, int D, int k
 cudaError_t launch_prefill_attn_pair(const PrefillAttnArgs& a, int B, int D, int key_rows_total,
                                      int kv_token_major, int head_pair, cudaStream_t st);
 cudaError_t launch_decode_split(const DecodeAttnArgs& a, int B, int D, cudaStream_t st);
+// int8 cache: the same split-K decode reading codes and (min, step) rows
+cudaError_t launch_decode_split_q8(const DecodeAttnArgs& a, int B, int D, cudaStream_t st);
 cudaError_t launch_decode_combine(const DecodeAttnArgs& a, int B, int D, cudaStream_t st);
 cudaError_t launch_visible_ranges(const int32_t* seq_lens_before, int B, int S, int window,
                                   int32_t* ranges, cudaStream_t st);

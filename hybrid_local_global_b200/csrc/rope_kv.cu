@@ -122,7 +122,9 @@ constexpr int ROPE_RPT = 2;    // positions per thread
 // it (global: cache slot pos; local: the k_rot workspace the attention kernel
 // reads, plus the ring slot for the last `window` positions); V goes to the
 // cache slot (global) or, only for the last `window` positions, the ring
-// (local: the attention kernel reads the caller's V directly).
+// (local: the attention kernel reads the caller's V directly). With an int8
+// cache (a.quant) every layer type writes only k_rot; the quantize kernel
+// fills the cache from k_rot and the caller's V.
 //
 // threadIdx.x owns 8 elements of the head vector, threadIdx.y one position
 // (of ROPE_RPT per thread): the angles of a position are formed once and
@@ -163,7 +165,7 @@ __global__ void __launch_bounds__(256, 2) k_prefill_rope(PrefillRopeArgs a) {
           st16(a.q_rot + (row * a.Hq + h0 + u) * D + e0, rotate_scale_chunk(x[u], t, e0, a.n_rot, a.q_scale));
     }
     if (!a.k_new) continue;  // shared layer: no K/V of its own
-    const bool to_ring = a.window > 0 && s >= a.S - a.window;
+    const bool to_ring = a.window > 0 && s >= a.S - a.window && !a.quant;
     const int64_t slot = a.window > 0 ? pos % a.window : pos;
 #pragma unroll 1
     for (int h0 = 0; h0 < a.Hkv; h0 += ROPE_HB / 2) {
@@ -171,7 +173,7 @@ __global__ void __launch_bounds__(256, 2) k_prefill_rope(PrefillRopeArgs a) {
 #pragma unroll
       for (int u = 0; u < ROPE_HB / 2; ++u) kx[u] = vx[u] = make_uint4(0, 0, 0, 0);
       // no v_new: K = V; the V window (WIN) takes every position of the chunk
-      const bool want_v = a.v_new && (WIN || a.window == 0 || to_ring);
+      const bool want_v = a.v_new && !a.quant && (WIN || a.window == 0 || to_ring);
       const int64_t wrow = WIN ? (int64_t)b * a.win_rows + a.window + s : row;  // k_rot / V window row
 #pragma unroll
       for (int u = 0; u < ROPE_HB / 2; ++u)
@@ -186,7 +188,7 @@ __global__ void __launch_bounds__(256, 2) k_prefill_rope(PrefillRopeArgs a) {
           const int kh = h0 + u;
           const uint4 kr = rotate_chunk(kx[u], t, e0, a.n_rot);
           const int64_t cslot = (((int64_t)b * a.Hkv + kh) * a.cache_cap + slot) * D + e0;
-          if (a.window == 0) {
+          if (a.window == 0 && !a.quant) {
             st16(a.k_cache + cslot, kr);
             if (want_v) st16(a.v_cache + cslot, vx[u]);
           } else {
@@ -256,8 +258,9 @@ __global__ void __launch_bounds__(256) k_decode_rope_append(DecodeRopeArgs a) {
   double inv_freq[4];
   chunk_inv_freq(e0, D, a.n_rot, a.log2_theta, inv_freq);
   const PairTrig t = chunk_trig(pos, e0, a.n_rot, inv_freq);
-  // q heads, then K heads, then V heads (none when shared, none for V under K = V)
-  const int n_heads = a.Hq + (a.k_new ? a.Hkv : 0) + (a.v_new ? a.Hkv : 0);
+  // q heads, then K heads, then V heads (none when shared, none for V under
+  // K = V, none with an int8 cache: the quantize kernel reads the caller's V)
+  const int n_heads = a.Hq + (a.k_new ? a.Hkv : 0) + ((a.v_new && !a.k_stage) ? a.Hkv : 0);
   for (int h = threadIdx.y; h < n_heads; h += blockDim.y) {
     if (h < a.Hq) {
       const int64_t off = ((int64_t)b * a.Hq + h) * D + e0;
@@ -269,12 +272,98 @@ __global__ void __launch_bounds__(256) k_decode_rope_append(DecodeRopeArgs a) {
     const int64_t src_off = ((int64_t)b * a.Hkv + kh) * D + e0;
     uint4 v = is_k ? rotate_chunk(ld16(a.k_new + src_off), t, e0, a.n_rot)
                    : ld16(a.v_new + src_off);
+    if (a.k_stage) {  // int8 cache: the rotated key waits for the quantize kernel
+      st16(a.k_stage + src_off, v);
+      continue;
+    }
     bf16* cache = is_k ? a.k_cache : a.v_cache;
     st16(cache + (((int64_t)b * a.Hkv + kh) * a.cache_cap + slot) * D + e0, v);
   }
 }
 
+// int8 cache rows ("Gemma 4 Technical Report", Quantization and Efficiency:
+// code = round((x - min) * (2^b - 1) / (max - min)), value min + code /
+// scale; here b = 8 and one (min, step) per cached row). One warp per row,
+// D / 32 elements per lane; every step of the code decision is fp32 with
+// round-to-nearest (IEEE division, no contraction), ties to even; a
+// constant row gets codes 0 and step 0.
+template <int D>
+__global__ void __launch_bounds__(256) k_quantize_rows(QuantRowsArgs a, int n_rows) {
+  constexpr int E = D / 32;  // 8 or 16
+  const int row = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  if (row >= n_rows) return;
+  const int h = row % a.Hkv;
+  const int s = (row / a.Hkv) % a.S;
+  const int b = row / (a.Hkv * a.S);
+  const int64_t pos = (a.pos0 ? (int64_t)a.pos0[b] - a.pos0_minus : 0) + s;
+  if (pos < 0) {
+    if (lane == 0) set_status(a.status, GEMMA_ERR_DEVICE_RANGE);
+    return;
+  }
+  if (a.window > 0 && s < a.S - a.window) return;  // only the chunk's last `window` rows reach the ring
+  const int64_t slot = a.window > 0 ? pos % a.window : pos;
+  if (slot >= a.cache_cap) {
+    if (lane == 0) set_status(a.status, GEMMA_ERR_DEVICE_RANGE);
+    return;
+  }
+  const bf16* src = a.src + (((int64_t)b * a.S + s) * a.Hkv + h) * D + lane * E;
+  float x[E];
+#pragma unroll
+  for (int c = 0; c < E / 8; ++c) {
+    const uint4 u = ld16(src + c * 8);
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float2 f = unpack_bf16x2(w[j]);
+      x[c * 8 + 2 * j] = f.x;
+      x[c * 8 + 2 * j + 1] = f.y;
+    }
+  }
+  float lo = x[0], hi = x[0];
+#pragma unroll
+  for (int e = 1; e < E; ++e) {
+    lo = fminf(lo, x[e]);
+    hi = fmaxf(hi, x[e]);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+    hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+  }
+  const float range = __fsub_rn(hi, lo);
+  uint32_t packed[E / 4];
+#pragma unroll
+  for (int i = 0; i < E / 4; ++i) packed[i] = 0;
+  if (range > 0.f) {
+    const float scale = __fdiv_rn(255.f, range);
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      int c = __float2int_rn(__fmul_rn(__fsub_rn(x[e], lo), scale));
+      c = c < 0 ? 0 : (c > 255 ? 255 : c);
+      packed[e / 4] |= (uint32_t)c << (8 * (e % 4));
+    }
+  }
+  const int64_t crow = ((int64_t)b * a.Hkv + h) * a.cache_cap + slot;
+  uint8_t* dst = a.codes + crow * D + lane * E;
+  if (E == 8)
+    *reinterpret_cast<uint2*>(dst) = make_uint2(packed[0], packed[1]);
+  else
+    *reinterpret_cast<uint4*>(dst) = make_uint4(packed[0], packed[1], packed[E / 4 > 2 ? 2 : 0], packed[E / 4 > 3 ? 3 : 0]);
+  if (lane == 0) a.params[crow] = make_float2(lo, range > 0.f ? __fdiv_rn(range, 255.f) : 0.f);
+}
+
 }  // namespace
+
+cudaError_t launch_quantize_rows(const QuantRowsArgs& a, int B, int D, cudaStream_t st) {
+  const int n_rows = B * a.S * a.Hkv;
+  if (n_rows <= 0) return cudaSuccess;
+  const int grid = (n_rows + 7) / 8;
+  if (D == 256)
+    k_quantize_rows<256><<<grid, 256, 0, st>>>(a, n_rows);
+  else
+    k_quantize_rows<512><<<grid, 256, 0, st>>>(a, n_rows);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_prefill_rope(const PrefillRopeArgs& a, int B, int D, cudaStream_t st) {
   const int tx = D / 8;

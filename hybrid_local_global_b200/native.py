@@ -31,6 +31,7 @@ GEMMA_ERR_DEVICE_TIMEOUT = 6
 GEMMA_ERR_DEVICE_RANGE = 7
 GEMMA_F_SHARED = 1
 GEMMA_F_KEQV = 2  # K = V on a global layer: no v_new, values read from the key cache
+GEMMA_F_KV_INT8 = 4  # int8 KV cache (Int8KVCache buffers); added automatically for those
 
 _P = ctypes.c_void_p
 _I = ctypes.c_int
@@ -41,7 +42,7 @@ _SZ = ctypes.c_size_t
 class gemma_kv_desc(ctypes.Structure):
     _fields_ = [("k_cache", _P), ("v_cache", _P), ("layer", _I), ("cache_cap", _I),
                 ("window", _I), ("n_kv_heads", _I), ("head_dim", _I), ("rope_frac", _F),
-                ("rope_theta", _F), ("shared_from", _I), ("k_eq_v", _I)]
+                ("rope_theta", _F), ("shared_from", _I), ("k_eq_v", _I), ("kv_int8", _I)]
 
 
 def _sig(name, restype, argtypes):
@@ -64,11 +65,14 @@ _sync = _sig("gemma_attn_sync_status", _I, [_P])
 _last = _sig("gemma_last_error", ctypes.c_char_p, [])
 _wait = _sig("gemma_attn_set_wait_limit", _I, [ctypes.c_longlong])
 _drop = _sig("gemma_attn_debug_drop_next_copy", _I, [_I])
+_kv_bytes = _sig("gemma_kv_cache_bytes", _SZ, [_I, _I, _I, _I, ctypes.c_uint])
+_kv_codes = _sig("gemma_kv_codes_bytes", _SZ, [_I, _I, _I, _I])
 
 EXPORTED = ["gemma_attn_prefill_workspace_size", "gemma_attn_prefill",
             "gemma_attn_decode_workspace_size", "gemma_attn_decode", "gemma_kv_share_bind",
             "gemma_layer_schedule", "gemma_attn_visible_ranges", "gemma_attn_sync_status",
-            "gemma_last_error", "gemma_attn_set_wait_limit", "gemma_attn_debug_drop_next_copy"]
+            "gemma_last_error", "gemma_attn_set_wait_limit", "gemma_attn_debug_drop_next_copy",
+            "gemma_kv_cache_bytes", "gemma_kv_codes_bytes"]
 
 
 class GemmaError(RuntimeError):
@@ -87,6 +91,38 @@ def _ptr(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
+def gemma_kv_cache_bytes(batch, n_kv_heads, cache_cap, head_dim, flags=0) -> int:
+    return int(_kv_bytes(batch, n_kv_heads, cache_cap, head_dim, flags))
+
+
+def gemma_kv_codes_bytes(batch, n_kv_heads, cache_cap, head_dim) -> int:
+    return int(_kv_codes(batch, n_kv_heads, cache_cap, head_dim))
+
+
+class Int8KVCache:
+    """One layer's int8 K (or V) cache buffer (GEMMA_F_KV_INT8 layout):
+    ``codes`` uint8 [B, Hkv, cap, D], then ``params`` float32 [B, Hkv, cap, 2]
+    = (min, step) per row, a row's value being min + code * step."""
+
+    def __init__(self, batch, n_kv_heads, cache_cap, head_dim, device, fill=0):
+        n = gemma_kv_cache_bytes(batch, n_kv_heads, cache_cap, head_dim, GEMMA_F_KV_INT8)
+        if n == 0:
+            raise ValueError("bad int8 cache shape")
+        self.shape = (batch, n_kv_heads, cache_cap, head_dim)
+        self.buf = torch.full((n,), fill, dtype=torch.uint8, device=device)
+        rows = batch * n_kv_heads * cache_cap
+        off = gemma_kv_codes_bytes(batch, n_kv_heads, cache_cap, head_dim)
+        self.codes = self.buf[:rows * head_dim].view(batch, n_kv_heads, cache_cap, head_dim)
+        self.params = self.buf[off:off + rows * 8].view(torch.float32).view(batch, n_kv_heads, cache_cap, 2)
+        self.device = self.buf.device
+
+    def data_ptr(self):
+        return self.buf.data_ptr()
+
+    def numel(self):
+        return self.buf.numel()
+
+
 def _stream(stream):
     if stream is None:
         stream = torch.cuda.current_stream()
@@ -94,7 +130,7 @@ def _stream(stream):
 
 
 def _bf16(t, name):
-    if t is None:
+    if t is None or isinstance(t, Int8KVCache):
         return
     if t.dtype != torch.bfloat16 or not t.is_contiguous() or not t.is_cuda:
         raise TypeError("%s must be a contiguous bf16 CUDA tensor" % name)
@@ -117,6 +153,8 @@ def gemma_attn_prefill(q, k_new, v_new, k_cache, v_cache, *, window, rope_frac, 
         _bf16(t, n)
     B, S, Hq, D = q.shape
     _, Hkv, cap, _ = k_cache.shape
+    if isinstance(k_cache, Int8KVCache):
+        flags |= GEMMA_F_KV_INT8
     if workspace is None:
         n = gemma_attn_prefill_workspace_size(B, S, Hq, Hkv, D, window)
         workspace = torch.empty(max(n, 1), dtype=torch.uint8, device=q.device)
@@ -141,6 +179,8 @@ def gemma_attn_decode(q, k_new, v_new, k_cache, v_cache, *, seq_lens, max_seq_le
         raise TypeError("seq_lens must be an int32 CUDA tensor")
     B, Hq, D = q.shape
     _, Hkv, cap, _ = k_cache.shape
+    if isinstance(k_cache, Int8KVCache):
+        flags |= GEMMA_F_KV_INT8
     if workspace is None:
         n = gemma_attn_decode_workspace_size(B, Hq, Hkv, D, window, max_seq_len)
         workspace = torch.empty(max(n, 1), dtype=torch.uint8, device=q.device)

@@ -75,6 +75,34 @@ typedef enum gemma_status {
                              v_new must be NULL; v_cache must be NULL or equal
                              k_cache. The values are the keys as the cache holds
                              them (rotated); nothing is written for V. */
+#define GEMMA_F_KV_INT8 4u /* int8 KV cache ("Gemma 4 Technical Report",
+                             Quantization and Efficiency, and its Table 3
+                             "+KV int8"). Each cache buffer holds
+                               codes  uint8 [batch][n_kv_heads][cache_cap][head_dim]
+                             followed, at byte offset
+                             gemma_kv_codes_bytes(batch, n_kv_heads, cache_cap,
+                             head_dim), by
+                               params float2 [batch][n_kv_heads][cache_cap] = (min, step)
+                             per cached row; the row's value is
+                             min + code * step. A row is quantized after
+                             (p-)RoPE and the bf16 rounding: min/max over its
+                             head_dim channels, code = round((x - min) * 255 /
+                             (max - min)) to nearest even, in fp32; a constant
+                             row gets codes 0 and step 0. Size the buffers with
+                             gemma_kv_cache_bytes(..., GEMMA_F_KV_INT8);
+                             cache_cap must be even. Prefill attends with the
+                             chunk's own bf16 K/V and writes codes; decode
+                             reads codes. Prefill after cached tokens
+                             (seq_lens_before != NULL) or with GEMMA_F_SHARED
+                             returns GEMMA_ERR_UNSUPPORTED. Combines with
+                             GEMMA_F_KEQV and, for decode, GEMMA_F_SHARED. */
+
+/* Bytes of one layer's K (or V) cache buffer: batch * n_kv_heads *
+ * cache_cap * head_dim * 2 for bf16; with GEMMA_F_KV_INT8 the codes, padded
+ * to 256 bytes, plus 8 bytes of (min, step) per row. 0 on bad arguments. */
+size_t gemma_kv_cache_bytes(int batch, int n_kv_heads, int cache_cap, int head_dim, unsigned flags);
+/* Offset of the (min, step) array in an int8 cache buffer. */
+size_t gemma_kv_codes_bytes(int batch, int n_kv_heads, int cache_cap, int head_dim);
 
 /* Supported shapes: head_dim 256 or 512; n_q_heads a multiple of n_kv_heads
  * with n_q_heads / n_kv_heads <= 8; window 0 (global) or a multiple of 16. */
@@ -194,12 +222,13 @@ typedef struct gemma_kv_desc {
     float rope_theta;
     int shared_from;    /* -1: owns its cache; else the layer whose cache it reads */
     int k_eq_v;         /* 1: a GEMMA_F_KEQV layer (v_cache may be NULL) */
+    int kv_int8;        /* 1: the caches are GEMMA_F_KV_INT8 buffers */
 } gemma_kv_desc;
 
 /* Makes dst read src's cache: dst->k_cache/v_cache become src's pointers and
  * dst->shared_from the layer that owns them (a chain resolves to its root).
  * Requires src->layer < dst->layer and identical window, cache_cap,
- * n_kv_heads, head_dim, rope_frac, rope_theta and k_eq_v (same attention type);
+ * n_kv_heads, head_dim, rope_frac, rope_theta, k_eq_v and kv_int8 (same attention type);
  * otherwise returns GEMMA_ERR_SHARE_MISMATCH and leaves dst unchanged.
  * Afterwards call the attention entry points for dst with GEMMA_F_SHARED. */
 int gemma_kv_share_bind(gemma_kv_desc* dst, const gemma_kv_desc* src);

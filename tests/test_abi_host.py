@@ -76,7 +76,7 @@ def test_share_bind_k_equals_v():
         assert e.value.code in (native.GEMMA_ERR_SHARE_MISMATCH, native.GEMMA_ERR_INVALID_ARG)
 
 
-@pytest.mark.parametrize("change", ["type", "window", "heads", "dim", "frac", "theta", "order", "cap"])
+@pytest.mark.parametrize("change", ["type", "window", "heads", "dim", "frac", "theta", "order", "cap", "int8"])
 def test_share_bind_rejects_mismatch(change):
     src = _desc(3, 1024, 1024, hkv=16, d=256, frac=1.0, theta=1e4)
     kw = dict(layer=4, window=1024, cap=1024, hkv=16, d=256, frac=1.0, theta=1e4, k=None, v=None)
@@ -97,6 +97,8 @@ def test_share_bind_rejects_mismatch(change):
     elif change == "cap":
         kw.update(cap=2048)
     dst = _desc(**kw)
+    if change == "int8":
+        dst.kv_int8 = 1
     with pytest.raises(native.GemmaError) as e:
         native.gemma_kv_share_bind(dst, src)
     assert e.value.code == native.GEMMA_ERR_SHARE_MISMATCH
@@ -140,7 +142,12 @@ E = native
     (dict(W=0, cap=8), E.GEMMA_ERR_CAPACITY),          # global cache shorter than the chunk
     (dict(k=None), E.GEMMA_ERR_INVALID_ARG),           # unshared layer without new keys
     (dict(flags=1), E.GEMMA_ERR_INVALID_ARG),          # shared layer with new keys
-    (dict(flags=4), E.GEMMA_ERR_INVALID_ARG),
+    (dict(flags=8), E.GEMMA_ERR_INVALID_ARG),          # unknown flag
+    (dict(flags=4, wsb=16), E.GEMMA_ERR_CAPACITY),     # int8 KV: accepted
+    (dict(flags=4, W=0, cap=4095, wsb=16), E.GEMMA_ERR_INVALID_ARG),   # int8 KV: odd capacity
+    (dict(flags=4, lens=FAKE), E.GEMMA_ERR_UNSUPPORTED),               # int8 KV after cached tokens
+    (dict(flags=5, k=None, v=None), E.GEMMA_ERR_UNSUPPORTED),          # int8 KV on a shared layer's prefill
+    (dict(W=0, cap=4096, flags=6, v=None, wsb=16), E.GEMMA_ERR_CAPACITY),  # int8 K = V: accepted
     (dict(flags=2, v=None), E.GEMMA_ERR_UNSUPPORTED),  # K = V on a local layer
     (dict(W=0, cap=4096, flags=2), E.GEMMA_ERR_INVALID_ARG),             # K = V with v_new
     (dict(W=0, cap=4096, flags=2, v=None, vc=FAKE + 256), E.GEMMA_ERR_INVALID_ARG),  # v_cache != k_cache
@@ -168,6 +175,10 @@ def test_prefill_validation(over, code):
     (dict(flags=2, v=None, vc=FAKE + 256), E.GEMMA_ERR_INVALID_ARG),   # v_cache != k_cache
     (dict(W=1024, cap=1024, flags=2, v=None), E.GEMMA_ERR_UNSUPPORTED),
     (dict(flags=2, v=None, vc=None, wsb=1024), E.GEMMA_ERR_CAPACITY),  # K = V accepted: v_cache optional
+    (dict(flags=4, wsb=1024), E.GEMMA_ERR_CAPACITY),                   # int8 KV accepted
+    (dict(flags=4, cap=4097, maxlen=4097, wsb=1024), E.GEMMA_ERR_INVALID_ARG),  # int8 KV: odd capacity
+    (dict(flags=5, k=None, v=None, wsb=1024), E.GEMMA_ERR_CAPACITY),   # int8 KV on a shared layer: accepted
+    (dict(flags=8), E.GEMMA_ERR_INVALID_ARG),                          # unknown flag
 ])
 def test_decode_validation(over, code):
     assert _decode_raw(**over) == code
@@ -179,3 +190,17 @@ def test_workspace_sizes_cover_the_configs():
     n = native.gemma_attn_decode_workspace_size(64, 32, 4, 512, 0, 131072)
     assert n >= 64 * 32 * 512 * 2
     assert native.gemma_attn_decode_workspace_size(0, 32, 4, 512, 0, 131072) == 0
+
+
+def test_kv_cache_bytes():
+    """bf16: one element per (row, dim); int8: the codes padded to 256 bytes,
+    then one (min, step) float pair per row."""
+    assert native.gemma_kv_cache_bytes(2, 4, 4096, 512) == 2 * 4 * 4096 * 512 * 2
+    codes = native.gemma_kv_codes_bytes(2, 4, 4096, 512)
+    assert codes == 2 * 4 * 4096 * 512
+    assert native.gemma_kv_cache_bytes(2, 4, 4096, 512, native.GEMMA_F_KV_INT8) == codes + 2 * 4 * 4096 * 8
+    assert native.gemma_kv_codes_bytes(1, 1, 2, 256) == 512
+    assert native.gemma_kv_codes_bytes(1, 3, 2, 16) == 256        # 96 bytes of codes, padded
+    assert native.gemma_kv_cache_bytes(1, 3, 2, 16, native.GEMMA_F_KV_INT8) == 256 + 6 * 8
+    assert native.gemma_kv_cache_bytes(0, 4, 4096, 512) == 0
+    assert native.gemma_kv_codes_bytes(1, 1, 0, 256) == 0

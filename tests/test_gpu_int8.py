@@ -1,0 +1,244 @@
+"""GPU parity of the int8 KV cache (GEMMA_F_KV_INT8) against the oracle,
+through the C ABI: the codes and (min, step) rows that prefill and decode
+write, and decode attention over an int8 cache.
+
+Cached rows are quantized by the oracle (oracle.quantize_rows_u8) from seeded
+bf16 rows; the expected attention is the oracle's over the dequantized rows
+(oracle.attend_rows). Where the GPU's input to a code decision is exactly the
+oracle's (values, and keys without RoPE) codes and rows must be bit-exact;
+rotated keys come from fp32 (GPU) and fp64 (oracle) rotations that agree up
+to a bf16 rounding, so their rows are compared within one code step.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from hybrid_local_global_b200 import native, synth
+
+from gpu_util import assert_close, to_bits
+
+pytestmark = pytest.mark.gpu
+
+SENTINEL = 0xAB
+
+
+def f64_to_bf16(x: np.ndarray) -> torch.Tensor:
+    return torch.from_numpy(np.asarray(x, dtype=np.float64)).to(torch.bfloat16)
+
+
+def quantize(oracle, rows: torch.Tensor):
+    """bf16 rows [..., D] -> (codes uint8 tensor, params float32 [..., 2]) from the oracle."""
+    c, lo, st = oracle.quantize_rows_u8(to_bits(rows.contiguous()))
+    return torch.from_numpy(c), torch.from_numpy(np.stack([lo, st], axis=-1))
+
+
+def dequant(oracle, codes: torch.Tensor, params: torch.Tensor) -> np.ndarray:
+    p = params.numpy()
+    return oracle.dequantize_rows_u8(codes.numpy(), p[..., 0], p[..., 1])
+
+
+def rotated_bf16(oracle, x: torch.Tensor, pos, frac, theta) -> torch.Tensor:
+    """[..., D] bf16 -> the oracle's (p-)RoPE at `pos`, rounded to bf16."""
+    flat = x.reshape(-1, x.shape[-1])
+    rows = [f64_to_bf16(oracle.rope_bf16(to_bits(r), pos, frac, theta)) for r in flat]
+    return torch.stack(rows).reshape(x.shape)
+
+
+def assert_rows_within_step(oracle, codes, params, exp_codes, exp_params, what):
+    """Rotated keys: the dequantized rows agree within one code step (the bf16
+    rotated inputs of the two sides may differ in a last bit)."""
+    got = dequant(oracle, codes, params)
+    exp = dequant(oracle, exp_codes, exp_params)
+    step = np.maximum(params[..., 1].numpy(), exp_params[..., 1].numpy())[..., None].astype(np.float64)
+    tol = 1.01 * step + 2.0 ** -7 * np.abs(exp)
+    assert (np.abs(got - exp) <= tol).all(), what
+    same = (codes == exp_codes).reshape(-1, codes.shape[-1]).all(dim=1).float().mean().item()
+    assert same >= 0.5, "%s: only %.0f%% of rows bit-identical" % (what, 100 * same)
+
+
+# ---------------------------------------------------------------------- prefill
+PREFILL_CASES = [
+    dict(B=2, S=200, Hq=8, Hkv=1, D=512, W=0, frac=0.25, theta=1e6, seed=301),
+    dict(B=1, S=300, Hq=8, Hkv=4, D=256, W=128, frac=1.0, theta=1e4, seed=302),
+    dict(B=2, S=96, Hq=4, Hkv=2, D=256, W=0, frac=0.0, theta=1e4, seed=303),      # NoPE: K codes exact
+    dict(B=1, S=130, Hq=8, Hkv=1, D=512, W=0, frac=0.25, theta=1e6, seed=304, keqv=True),
+    dict(B=1, S=40, Hq=8, Hkv=4, D=256, W=64, frac=0.0, theta=1e4, seed=305),      # chunk shorter than the ring
+]
+
+
+@pytest.mark.parametrize("case", PREFILL_CASES, ids=["global", "local", "nope", "keqv", "short"])
+def test_prefill_writes_int8_rows(oracle, case):
+    case = dict(case)
+    keqv = case.pop("keqv", False)
+    B, S, Hq, Hkv, D, W = (case[k] for k in ("B", "S", "Hq", "Hkv", "D", "W"))
+    frac, theta = case["frac"], case["theta"]
+    dev = torch.device("cuda")
+    g = synth.generator(case["seed"])
+    q = synth.randn_bf16((B, S, Hq, D), g)
+    k = synth.randn_bf16((B, S, Hkv, D), g)
+    v = synth.randn_bf16((B, S, Hkv, D), g)
+    cap = W if W else S + 16
+    kc = native.Int8KVCache(B, Hkv, cap, D, dev, fill=SENTINEL)
+    vc = kc if keqv else native.Int8KVCache(B, Hkv, cap, D, dev, fill=SENTINEL)
+    out8 = torch.full((B, S, Hq, D), float("nan"), dtype=torch.bfloat16, device=dev)
+    scale = 1.0 / math.sqrt(D)
+    flags = native.GEMMA_F_KEQV if keqv else 0
+    kw = dict(window=W, rope_frac=frac, rope_theta=theta, scale=scale, flags=flags)
+    native.gemma_attn_prefill(q.to(dev), k.to(dev), None if keqv else v.to(dev), kc, None if keqv else vc,
+                              out=out8, **kw)
+    assert native.gemma_attn_sync_status() == 0, native.gemma_last_error()
+    # the attention itself is the bf16 path's: same kernels, same rotated chunk
+    kb = torch.zeros((B, Hkv, cap, D), dtype=torch.bfloat16, device=dev)
+    vb = kb if keqv else torch.zeros_like(kb)
+    outb = torch.full_like(out8, float("nan"))
+    native.gemma_attn_prefill(q.to(dev), k.to(dev), None if keqv else v.to(dev), kb, None if keqv else vb,
+                              out=outb, **kw)
+    assert native.gemma_attn_sync_status() == 0, native.gemma_last_error()
+    assert torch.equal(out8.view(torch.int16), outb.view(torch.int16))
+    codes_k, par_k = kc.codes.cpu(), kc.params.cpu()
+    codes_v, par_v = vc.codes.cpu(), vc.params.cpu()
+    written = torch.zeros((B, cap), dtype=torch.bool)
+    first = max(0, S - W) if W else 0
+    for b in range(B):
+        for p in range(first, S):
+            slot = p % W if W else p
+            written[b, slot] = True
+            if not keqv:
+                ec, ep = quantize(oracle, v[b, p])
+                assert torch.equal(codes_v[b, :, slot], ec), "V codes b=%d p=%d" % (b, p)
+                assert torch.equal(par_v[b, :, slot], ep), "V (min, step) b=%d p=%d" % (b, p)
+            ec, ep = quantize(oracle, rotated_bf16(oracle, k[b, p], p, frac, theta))
+            if frac == 0.0:
+                assert torch.equal(codes_k[b, :, slot], ec), "K codes b=%d p=%d" % (b, p)
+                assert torch.equal(par_k[b, :, slot], ep), "K (min, step) b=%d p=%d" % (b, p)
+            else:
+                assert_rows_within_step(oracle, codes_k[b, :, slot], par_k[b, :, slot], ec, ep,
+                                        "K rows b=%d p=%d" % (b, p))
+    untouched = ~written
+    for c in (codes_k, codes_v):
+        assert (c.permute(0, 2, 1, 3)[untouched] == SENTINEL).all()
+    for par in (par_k, par_v):
+        raw = par.view(torch.int32).permute(0, 2, 1, 3)[untouched]
+        assert (raw == int(np.uint32(0xABABABAB).view(np.int32))).all()
+
+
+# ----------------------------------------------------------------------- decode
+def run_decode_int8(oracle, *, lens, Hq, Hkv, D, W, frac, theta, seed, keqv=False, shared=False,
+                    v_scale=1.0, tol=(2e-2, 2e-3)):
+    dev = torch.device("cuda")
+    B = len(lens)
+    g = synth.generator(seed)
+    max_len = max(lens)
+    cap = W if W else max_len + 16 + (max_len % 2)
+    # cached rows (already rotated), quantized by the oracle, at their slots
+    k_rows = synth.randn_bf16((B, Hkv, cap, D), g)
+    v_rows = synth.randn_bf16((B, Hkv, cap, D), g, scale=v_scale)
+    q = synth.randn_bf16((B, Hq, D), g)
+    kn = synth.randn_bf16((B, Hkv, D), g)
+    vn = synth.randn_bf16((B, Hkv, D), g, scale=v_scale)
+    if keqv:
+        v_rows, vn = k_rows, kn
+    ck, pk = quantize(oracle, k_rows)
+    cv, pv = (ck, pk) if keqv else quantize(oracle, v_rows)
+    if shared:
+        # the new token's rows are already in the (source layer's) cache
+        for b in range(B):
+            slot = (lens[b] - 1) % W if W else lens[b] - 1
+            ck[b, :, slot], pk[b, :, slot] = quantize(oracle, kn[b])
+            if not keqv:
+                cv[b, :, slot], pv[b, :, slot] = quantize(oracle, vn[b])
+            else:
+                cv, pv = ck, pk
+    kc = native.Int8KVCache(B, Hkv, cap, D, dev)
+    kc.codes.copy_(ck)
+    kc.params.copy_(pk)
+    vc = kc
+    if not keqv:
+        vc = native.Int8KVCache(B, Hkv, cap, D, dev)
+        vc.codes.copy_(cv)
+        vc.params.copy_(pv)
+    out = torch.full((B, Hq, D), float("nan"), dtype=torch.bfloat16, device=dev)
+    sl = torch.tensor(lens, dtype=torch.int32, device=dev)
+    scale = 1.0 / math.sqrt(D)
+    flags = (native.GEMMA_F_SHARED if shared else 0) | (native.GEMMA_F_KEQV if keqv else 0)
+    native.gemma_attn_decode(q.to(dev), None if shared else kn.to(dev),
+                             None if (shared or keqv) else vn.to(dev), kc, None if keqv else vc,
+                             seq_lens=sl, max_seq_len=max_len, window=W, rope_frac=frac, rope_theta=theta,
+                             scale=scale, out=out, flags=flags)
+    assert native.gemma_attn_sync_status() == 0, native.gemma_last_error()
+    ck1, pk1, cv1, pv1 = kc.codes.cpu(), kc.params.cpu(), vc.codes.cpu(), vc.params.cpu()
+    G = Hq // Hkv
+    for b in range(B):
+        L = lens[b]
+        slot_new = (L - 1) % W if W else L - 1
+        # the new token's rows as the oracle writes them
+        if shared:
+            nk_c, nk_p = ck[b, :, slot_new], pk[b, :, slot_new]
+            nv_c, nv_p = cv[b, :, slot_new], pv[b, :, slot_new]
+        else:
+            nk_c, nk_p = quantize(oracle, rotated_bf16(oracle, kn[b], L - 1, frac, theta))
+            nv_c, nv_p = (nk_c, nk_p) if keqv else quantize(oracle, vn[b])
+            if not keqv:
+                assert torch.equal(cv1[b, :, slot_new], nv_c) and torch.equal(pv1[b, :, slot_new], nv_p)
+            if frac == 0.0:
+                assert torch.equal(ck1[b, :, slot_new], nk_c) and torch.equal(pk1[b, :, slot_new], nk_p)
+            else:
+                assert_rows_within_step(oracle, ck1[b, :, slot_new], pk1[b, :, slot_new], nk_c, nk_p,
+                                        "new K row b=%d" % b)
+            other = torch.ones(cap, dtype=torch.bool)
+            other[slot_new] = False
+            assert torch.equal(ck1[b][:, other], ck[b][:, other])
+        first = max(0, L - W) if W else 0
+        positions = list(range(first, L))
+        keys = np.zeros((Hkv, len(positions), D))
+        vals = np.zeros((Hkv, len(positions), D))
+        for i, p in enumerate(positions):
+            if p == L - 1:
+                keys[:, i] = dequant(oracle, nk_c, nk_p)
+                vals[:, i] = dequant(oracle, nv_c, nv_p)
+            else:
+                s = p % W if W else p
+                keys[:, i] = dequant(oracle, ck[b, :, s], pk[b, :, s])
+                vals[:, i] = dequant(oracle, cv[b, :, s], pv[b, :, s])
+        n = len(positions)
+        qrot = np.stack([oracle.rope_bf16(to_bits(q[b, h]), L - 1, frac, theta) for h in range(Hq)])
+        ref, _ = oracle.attend_rows(qrot, keys.reshape(Hkv * n, D), vals.reshape(Hkv * n, D),
+                                    [(h // G) * n for h in range(Hq)], [n] * Hq, scale)
+        assert_close(out[b].float().cpu().double().numpy(), ref, *tol, what="int8 decode b=%d len=%d" % (b, L))
+
+
+DECODE_CASES = [
+    dict(lens=[1, 37, 300, 4097], Hq=8, Hkv=1, D=512, W=0, frac=0.25, theta=1e6, seed=311),
+    dict(lens=[1, 5, 64, 65, 1000], Hq=8, Hkv=4, D=256, W=64, frac=1.0, theta=1e4, seed=312),
+    dict(lens=[17, 16, 15, 33], Hq=32, Hkv=16, D=256, W=16, frac=0.0, theta=1e4, seed=313),
+    dict(lens=[7777, 123], Hq=32, Hkv=4, D=512, W=0, frac=0.25, theta=1e6, seed=314),
+    dict(lens=[3000, 900], Hq=32, Hkv=16, D=256, W=1024, frac=1.0, theta=1e4, seed=315),
+    dict(lens=[2, 129], Hq=8, Hkv=4, D=256, W=0, frac=0.0, theta=1e4, seed=316),   # NoPE: new K row exact
+]
+
+
+@pytest.mark.parametrize("case", DECODE_CASES, ids=lambda c: "L%s_H%d-%dD%dW%d" % (
+    "_".join(map(str, c["lens"])), c["Hq"], c["Hkv"], c["D"], c["W"]))
+def test_decode_int8(oracle, case):
+    run_decode_int8(oracle, **case)
+
+
+def test_decode_int8_k_equals_v(oracle):
+    run_decode_int8(oracle, lens=[1, 37, 300, 2049], Hq=8, Hkv=1, D=512, W=0, frac=0.25, theta=1e6, seed=321,
+                    keqv=True)
+
+
+@pytest.mark.parametrize("W,D,Hkv", [(0, 512, 1), (64, 256, 4)])
+def test_decode_int8_shared_layer(oracle, W, D, Hkv):
+    run_decode_int8(oracle, lens=[900, 33], Hq=8, Hkv=Hkv, D=D, W=W, frac=0.25 if W == 0 else 1.0,
+                    theta=1e6 if W == 0 else 1e4, seed=322, shared=True)
+
+
+@pytest.mark.parametrize("v_scale", [1e-3, 40.0])
+def test_decode_int8_value_ranges(oracle, v_scale):
+    """Rows whose steps are far from 1: the fp16 weights of the codes are
+    scaled by a power of two that keeps them in range."""
+    run_decode_int8(oracle, lens=[300, 1500], Hq=8, Hkv=1, D=512, W=0, frac=0.25, theta=1e6, seed=323,
+                    v_scale=v_scale, tol=(2e-2 * v_scale, 2e-3 * v_scale))
