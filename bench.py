@@ -3,6 +3,7 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload NAME] [--decode-workload NAME|none]
+                    [--decode-int8-workload NAME|none]
 
 One JSON line on rank 0. A step is one pass of the prefill block named by
 --workload (default: the E2B-shaped 5-layer block, B1 S8192: layer schedule,
@@ -10,7 +11,10 @@ RoPE + cache write, attention for every layer) over resident synthetic
 inputs; `value` is its algorithmic TFLOP/s (4*B*Hq*D per visible query-key
 pair, masked pairs not counted) over all ranks. The `decode` object measures
 the batched decode block named by --decode-workload (default: 31B-shaped,
-6 layers, B64, KV lengths U[4096,131072], last two layers shared) in KV GB/s.
+6 layers, B64, KV lengths U[4096,131072], last two layers shared) in KV GB/s;
+`decode_int8` the same block on int8 KV caches (GB/s of the int8 rows read,
+and `bf16_equivalent_gbs`: the bf16 bytes the same keys would take, per
+second).
 
 --impl reference times the fp64 CPU oracle (the path's reference
 implementation here) on the host cores, each step a bounded sample of rows
@@ -285,12 +289,15 @@ def decode_bytes(w, st, lens_cpu):
     return total
 
 
-def visible_kv_bytes(st, l, lens_cpu):
-    """Cached K (and V unless K = V) bytes layer l's decode reads."""
+def visible_kv_bytes(st, l, lens_cpu, bf16_equivalent=False):
+    """Cached K (and V unless K = V) bytes layer l's decode reads: head_dim
+    bf16 per key, or on int8 caches head_dim codes plus an 8-byte (min,
+    step) pair (bf16_equivalent: the bf16 bytes of the same keys)."""
     t = st.layer_type(l)
     L = lens_cpu.to(torch.int64)
     vis = torch.clamp(L, max=t.window) if t.window else L
-    return int(vis.sum()) * t.n_kv_heads * t.head_dim * 2 * (1 if st.keqv(l) else 2)
+    row = t.head_dim + 8 if (st.w.kv_int8 and not bf16_equivalent) else t.head_dim * 2
+    return int(vis.sum()) * t.n_kv_heads * row * (1 if st.keqv(l) else 2)
 
 
 def bench_decode(args, w, dev, world, peaks):
@@ -310,8 +317,9 @@ def bench_decode(args, w, dev, world, peaks):
         if kc.data_ptr() in seen:
             continue
         seen.add(kc.data_ptr())
-        synth.fill_randn_bf16_(kc, g)
-        synth.fill_randn_bf16_(st.v_cache[l], g)
+        synth.fill_cache_(kc, g)
+        if st.v_cache[l] is not kc:
+            synth.fill_cache_(st.v_cache[l], g)
     layers = []
     for l in range(st.n_layers):
         t = st.layer_type(l)
@@ -357,7 +365,7 @@ def bench_decode(args, w, dev, world, peaks):
             "peak_source": "%s HBM copy (MEASURED_PEAKS.json)" % peaks[1], "traffic": None,
             "per_launch": "visible K (and V unless K = V) bytes of all split launches / their summed device time "
                           "(%d launches, %d per step)" % (sp["launches"], st.n_layers)}
-    rec = recorded_traffic("k_decode_split")
+    rec = recorded_traffic("k_decode_split_q8" if w.kv_int8 else "k_decode_split")
     if rec:
         r = next(iter(rec.values()))
         ratio = float(r["bytes"]) / float(r["units"])
@@ -367,7 +375,7 @@ def bench_decode(args, w, dev, world, peaks):
                                 "large to capture)" % (ratio, r["workload"], r["file"]))
     else:
         roof["traffic_note"] = "no ncu capture of the current kernel sources"
-    return {"metric": "decode KV GB/s", "value": round(value, 1), "unit": "GB/s",
+    res = {"metric": "decode KV GB/s", "value": round(value, 1), "unit": "GB/s",
             "workload": w.name, "description": w.description, "ms_per_step": round(dev_ms / args.steps, 4),
             "bytes_per_step": nbytes, "kv_bytes_per_step": kv_bytes,
             "kv_lengths": {"min": int(lens_cpu.min()), "max": max_len, "sum": int(lens_cpu.sum())},
@@ -375,6 +383,12 @@ def bench_decode(args, w, dev, world, peaks):
             "cache_bytes_owned": st.owned_cache_bytes(),
             "roofline": roof, "kernels": kern, "clocks": clk.summary(),
             "gpu_launches": sum(v["launches"] for v in kern.values())}
+    if w.kv_int8:
+        eq = sum(visible_kv_bytes(st, l, lens_cpu, bf16_equivalent=True) for l in range(st.n_layers))
+        res["bf16_equivalent_gbs"] = round(world * eq * args.steps / (dev_ms / 1e3) / 1e9, 1)
+        res["bf16_equivalent_note"] = ("bf16 bytes of the same visible keys per second of the whole step: "
+                                       "the bandwidth a bf16 cache would need to match this step time")
+    return res
 
 
 # --------------------------------------------------------------------------- oracle (CPU)
@@ -476,6 +490,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="e2b_block_s8192", choices=sorted(WORKLOADS))
     ap.add_argument("--decode-workload", default="31b_decode_b64")
+    ap.add_argument("--decode-int8-workload", default="31b_decode_b64_int8")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-rows-local", type=int, default=256)
@@ -527,6 +542,10 @@ def main():
         dw = WORKLOADS[args.decode_workload]
         line["decode"] = bench_decode(args, dw, dev, world, peaks)
         line["gpu_launches"] += line["decode"]["gpu_launches"]
+    if args.decode_int8_workload != "none":
+        dw = WORKLOADS[args.decode_int8_workload]
+        line["decode_int8"] = bench_decode(args, dw, dev, world, peaks)
+        line["gpu_launches"] += line["decode_int8"]["gpu_launches"]
     if rank == 0:
         print(json.dumps(line))
     RANKS.close()

@@ -8,24 +8,23 @@
 // Walkthrough", 3a/3b), computed without dequantizing element by element:
 //   s_j = <q, min_j + step_j c_j> = step_j <q, c_j> + min_j sum(q)
 //   o   = sum_j p_j (min_j + step_j c_j) = sum_j (p_j step_j) c_j + sum_j p_j min_j
-// so the MMAs multiply the codes themselves (exact in fp16), and the affine
-// part is applied per key (S) and as one scalar per head (O).
+// so the MMAs multiply the codes themselves (exact in fp16, offset by 1024),
+// and the affine part and the offset are applied per key (S) and as one
+// scalar per head (O).
 //
-// Per CTA = (split, KV head, sequence), 128 threads:
-//   warp 3      producer: per 16-key sub-block, four bulk copies into a ring
-//               slot: the K codes (16 rows x D bytes, contiguous in the
-//               cache), the V codes, and their (min, step) rows.
+// Per CTA = (split, KV head, sequence), 128 threads, two CTAs per SM:
+//   warp 3      producer: per 16-key sub-block, one bulk copy per pair of
+//               consecutive K (or V) code rows (contiguous in the cache) into
+//               padded row pairs of a ring slot, plus one copy each of the K
+//               and V (min, step) rows.
 //   warps 0..2  consumers: sub-block t goes to warp t % 3 (and ring slot
-//               t % NSLOT). The warp widens its slot's codes to fp16 in its
-//               own padded staging rows (a byte permute puts each code in
-//               the mantissa of 1024.0, and subtracting 1024 leaves the code
-//               exactly), releases the slot, then runs the mma.sync path of
-//               decode.cu in fp16: S = Q C_K^T, then O^T += C_V^T P'^T.
-// Scaling: Q is staged as fp16 times 2^-eq with max|q| <= 1, and P' = p *
-// step_j * 2^-ev with 2^ev >= every step of the CTA's key range (read in a
-// pre-pass over the (min, step) rows), so neither leaves fp16's range; both
-// powers of two are undone exactly in fp32.
-//
+//               t % NSLOT). The MMA fragments (mma.sync m16n8k16, fp16) come
+//               straight from the code rows: a byte permute puts a code in
+//               the mantissa of fp16 1024.0 and subtracting 1024 leaves it
+//               exactly. The k positions of S and the output rows of P.V
+//               stand for dims in an order that makes each lane's codes 16
+//               contiguous bytes, and a fixed key order (key_at) spreads the
+//               rows a quarter warp reads over different banks.
 // Every barrier wait is bounded (%globaltimer deadline); on a timeout the CTA
 // raises its abort flag, records GEMMA_ERR_DEVICE_TIMEOUT, waits (bounded)
 // for its own copies in flight, and exits without output.
@@ -46,35 +45,49 @@ constexpr int NCW = 3;  // consumer warps
 template <int D>
 struct Q8Cfg {
   static constexpr int KB = 16;                      // keys per sub-block
-  static constexpr int CODES_B = 2 * KB * D;         // K codes [16][D], then V codes (K = V: 32 K rows)
-  static constexpr int RAW_B = CODES_B + 2 * KB * 8; // then K (min, step) [16], V [16] (K = V: 32 K)
+  static constexpr int PAIRB = 2 * D + 16;           // two consecutive code rows + 16 B pad
+  static constexpr int REGION_B = (KB / 2) * PAIRB;  // 16 code rows as 8 padded pairs
+  static constexpr int PAR_OFF = 2 * REGION_B;       // K region, V region (K = V: 32 K rows), then
+  static constexpr int RAW_B = PAR_OFF + 2 * KB * 8; // K (min, step) [16], V [16] (K = V: 32 K)
   static constexpr int NSLOT = 6;
   static_assert(NSLOT % NCW == 0, "each ring slot needs a single consumer warp");
-  static constexpr int ROW = D + 8;                  // fp16 staging row (elements), 16 B pad
-  static constexpr int ROWB = ROW * 2;
-  static constexpr int STG_B = 2 * KB * ROWB;        // per consumer warp: 32 rows
+  static constexpr int ROW = D + 8;                  // fp16 Q row (elements), 16 B pad
   static constexpr int RING_B = NSLOT * RAW_B;
-  static constexpr int STG_OFF = RING_B;
-  static constexpr int Q_OFF = STG_OFF + NCW * STG_B;
-  static constexpr int Q_B = 8 * ROWB;
+  static constexpr int Q_OFF = RING_B;
+  static constexpr int Q_B = 8 * ROW * 2;
   static constexpr int QSUM_OFF = Q_OFF + Q_B;       // float [8] sum of each head's staged q
   static constexpr int BAR_OFF = QSUM_OFF + 64;
   static constexpr int MISC_OFF = BAR_OFF + 2 * NSLOT * 8;
   static constexpr int SMEM = MISC_OFF + (4 + 2 * NSLOT + 64) * 4;
   static constexpr int OSTR = D + 4;                 // merge-buffer row (floats)
   static constexpr int MERGE_B = NCW * 8 * OSTR * 4;
-  static_assert(MERGE_B <= NCW * STG_B, "merge buffer must fit in the staging rows");
-  static_assert(RAW_B % 16 == 0 && ROWB % 16 == 0 && STG_OFF % 16 == 0, "16-byte alignment");
-  static constexpr int MIN_BLOCKS = (SMEM * 2 <= 227 * 1024) ? 2 : 1;
+  static_assert(MERGE_B <= RING_B, "merge buffer must fit in the drained ring");
+  static_assert(PAIRB % 16 == 0 && RAW_B % 16 == 0 && Q_OFF % 16 == 0, "16-byte alignment");
+  static_assert(2 * SMEM <= 227 * 1024, "two CTAs per SM");
+  static constexpr int VCH = D / 128;                // 16-dim chunks of V per lane (D/8 dims per lane)
 };
 
-// Two codes (bytes `sel` picks) -> fp16x2 holding them exactly.
-__device__ __forceinline__ uint32_t codes_to_h2(uint32_t w, uint32_t sel) {
-  uint32_t h = __byte_perm(w, 0x64u, sel);  // bytes c, 0x64, c', 0x64: fp16 1024 + c, 1024 + c'
-  __half2 v = *reinterpret_cast<__half2*>(&h);
-  v = __hsub2(v, __half2half2(__ushort_as_half((unsigned short)0x6400)));
-  return *reinterpret_cast<uint32_t*>(&v);
+// Byte offset of code row r (0..31) in a slot: rows go in padded pairs.
+template <int D>
+__device__ __forceinline__ int code_row_off(int r) {
+  return (r >> 1) * Q8Cfg<D>::PAIRB + (r & 1) * D;
 }
+
+// The key (0..15 within a 16-key half) that MMA column / P.V index j stands
+// for. The S fragments read rows key_at(gq) and key_at(8 + gq) with the 8
+// lanes of a quarter warp on two of them, the P.V fragments rows key_at(2tg)
+// .. key_at(9 + 2tg) with four lanes on four rows; this order puts each such
+// set of rows in row pairs whose 16-byte pads shift them onto disjoint banks
+// (head_dim 512; head_dim 256 keeps a 2-way overlap on the P.V side).
+__device__ __forceinline__ int key_at(int j) {
+  const int q = (j & 7) >> 1;
+  return (j & 8) ? ((j & 1) ? 9 + 2 * q : 2 * q + 1) : ((j & 1) ? 8 + 2 * q : 2 * q);
+}
+
+// Two codes (bytes `sel` picks) -> fp16x2 (1024 + c, 1024 + c'), exactly:
+// the code lands in the mantissa of 1024.0. The MMAs take the codes with
+// this offset and the 1024 comes off once per key (S) and per head (O).
+__device__ __forceinline__ uint32_t codes_h2(uint32_t w, uint32_t sel) { return __byte_perm(w, 0x64u, sel); }
 
 __device__ __forceinline__ uint32_t pack_h2(float lo, float hi) {
   __half2 v = __floats2half2_rn(lo, hi);
@@ -91,11 +104,10 @@ __device__ __forceinline__ float pow2_ceil(float x) {
 }
 
 template <int D>
-__global__ void __launch_bounds__(32 * (NCW + 1), Q8Cfg<D>::MIN_BLOCKS) k_decode_split_q8(DecodeAttnArgs a) {
+__global__ void __launch_bounds__(32 * (NCW + 1), 2) k_decode_split_q8(DecodeAttnArgs a) {
   using C = Q8Cfg<D>;
   extern __shared__ __align__(128) unsigned char sm[];
   unsigned char* ring = sm;
-  unsigned char* stg_all = sm + C::STG_OFF;
   __half* qs = reinterpret_cast<__half*>(sm + C::Q_OFF);
   float* qsum = reinterpret_cast<float*>(sm + C::QSUM_OFF);
   uint64_t* full = reinterpret_cast<uint64_t*>(sm + C::BAR_OFF);
@@ -139,58 +151,7 @@ __global__ void __launch_bounds__(32 * (NCW + 1), Q8Cfg<D>::MIN_BLOCKS) k_decode
     *abort_flag = 0;
     fence_barrier_init();
   }
-  // max |q| over the group's heads and the largest V step of this split's
-  // keys: both become powers of two that keep the fp16 operands in range
-  float qmax = 0.f, vmax = 0.f;
-  for (int idx = threadIdx.x; idx < G * (D / 8); idx += blockDim.x) {
-    const int r = idx / (D / 8), c = (idx % (D / 8)) * 8;
-    const uint4 u = *reinterpret_cast<const uint4*>(a.q_rot + ((int64_t)b * a.Hq + g * G + r) * D + c);
-    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const float2 f = unpack_bf16x2(w[j]);
-      qmax = fmaxf(qmax, fmaxf(fabsf(f.x), fabsf(f.y)));
-    }
-  }
-  for (int64_t k = k_begin + threadIdx.x; k < k_end; k += blockDim.x) vmax = fmaxf(vmax, vpar[k].y);
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    qmax = fmaxf(qmax, __shfl_xor_sync(0xffffffffu, qmax, o));
-    vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, o));
-  }
-  if (lane == 0) {
-    red[warp] = qmax;
-    red[4 + warp] = vmax;
-  }
-  __syncthreads();
-  qmax = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
-  vmax = fmaxf(fmaxf(red[4], red[5]), fmaxf(red[6], red[7]));
-  const float fq = pow2_ceil(qmax), fv = pow2_ceil(vmax);
-  const float inv_fq = 1.f / fq, inv_fv = 1.f / fv;  // exact: powers of two
-  for (int idx = threadIdx.x; idx < 8 * (D / 8); idx += blockDim.x) {
-    const int r = idx / (D / 8), c = (idx % (D / 8)) * 8;
-    uint4 u = make_uint4(0, 0, 0, 0);
-    if (r < G) u = *reinterpret_cast<const uint4*>(a.q_rot + ((int64_t)b * a.Hq + g * G + r) * D + c);
-    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-    uint32_t h[4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const float2 f = unpack_bf16x2(w[j]);
-      h[j] = pack_h2(f.x * inv_fq, f.y * inv_fq);
-    }
-    *reinterpret_cast<uint4*>(qs + r * C::ROW + c) = make_uint4(h[0], h[1], h[2], h[3]);
-  }
-  __syncthreads();
-  // sum of each head's staged q (the same fp16 values the MMA reads)
-  for (int r = warp; r < 8; r += NCW + 1) {
-    float acc = 0.f;
-    for (int d = lane; d < D; d += 32) acc += __half2float(qs[r * C::ROW + d]);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-    if (lane == 0) qsum[r] = acc;
-  }
-  __syncwarp();
-  __syncthreads();
+  __syncthreads();  // the barriers exist before the producer arms them
   const uint64_t deadline = globaltimer_ns() + a.wait_ns;
 
   if (warp == NCW) {
@@ -220,25 +181,103 @@ __global__ void __launch_bounds__(32 * (NCW + 1), Q8Cfg<D>::MIN_BLOCKS) k_decode
         issued[slot] += 1;
       }
       __syncwarp();
-      if (lane == 0) bulk_g2s(dst, kcode + key0 * D, (uint32_t)(nk * D), &full[slot]);
-      if (lane == 1) bulk_g2s(dst + C::CODES_B, kpar + key0, (uint32_t)(np * 8), &full[slot]);
-      if (!a.keqv) {
-        if (lane == 2) bulk_g2s(dst + C::KB * D, vcode + key0 * D, (uint32_t)(nk * D), &full[slot]);
-        if (lane == 3) bulk_g2s(dst + C::CODES_B + C::KB * 8, vpar + key0, (uint32_t)(np * 8), &full[slot]);
+      // lanes 0..7: K row pairs, 8..15: V row pairs (K = V: lanes 0..15, the
+      // 16 pairs of 32 K rows); lanes 16, 17: the (min, step) rows
+      if (lane < 16) {
+        const bool isv = !a.keqv && lane >= 8;
+        const int pr = a.keqv ? lane : (lane & 7);
+        const int left = nk - 2 * pr;
+        if (left > 0)
+          bulk_g2s(dst + (isv ? C::REGION_B : 0) + pr * C::PAIRB, (isv ? vcode : kcode) + (key0 + 2 * pr) * D,
+                   (uint32_t)((left >= 2 ? 2 : 1) * D), &full[slot]);
+      } else if (lane == 16) {
+        bulk_g2s(dst + C::PAR_OFF, kpar + key0, (uint32_t)(np * 8), &full[slot]);
+      } else if (lane == 17 && !a.keqv) {
+        bulk_g2s(dst + C::PAR_OFF + C::KB * 8, vpar + key0, (uint32_t)(np * 8), &full[slot]);
       }
     }
   } else {
     // ---------------- consumers ----------------
+    // Consumer prologue, overlapping the producer's first copies: max |q|
+    // over the group's heads and the largest V step of this split's keys
+    // become powers of two that keep the fp16 operands in range; then Q
+    // (scaled) in fp16 and each head's sum of it.
+    float qmax = 0.f, vmax = 0.f;
+    for (int idx = threadIdx.x; idx < G * (D / 8); idx += 32 * NCW) {
+      const int r = idx / (D / 8), c = (idx % (D / 8)) * 8;
+      const uint4 u = *reinterpret_cast<const uint4*>(a.q_rot + ((int64_t)b * a.Hq + g * G + r) * D + c);
+      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float2 f = unpack_bf16x2(w[j]);
+        qmax = fmaxf(qmax, fmaxf(fabsf(f.x), fabsf(f.y)));
+      }
+    }
+    for (int64_t k = k_begin + threadIdx.x; k < k_end; k += 32 * NCW) vmax = fmaxf(vmax, vpar[k].y);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      qmax = fmaxf(qmax, __shfl_xor_sync(0xffffffffu, qmax, o));
+      vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, o));
+    }
+    if (lane == 0) {
+      red[warp] = qmax;
+      red[4 + warp] = vmax;
+    }
+    named_bar_sync(1, 32 * NCW);
+    qmax = fmaxf(fmaxf(red[0], red[1]), red[2]);
+    vmax = fmaxf(fmaxf(red[4], red[5]), red[6]);
+    const float fq = pow2_ceil(qmax), fv = pow2_ceil(vmax);
+    const float inv_fq = 1.f / fq, inv_fv = 1.f / fv;  // exact: powers of two
+    for (int idx = threadIdx.x; idx < 8 * (D / 8); idx += 32 * NCW) {
+      const int r = idx / (D / 8), c = (idx % (D / 8)) * 8;
+      uint4 u = make_uint4(0, 0, 0, 0);
+      if (r < G) u = *reinterpret_cast<const uint4*>(a.q_rot + ((int64_t)b * a.Hq + g * G + r) * D + c);
+      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+      uint32_t h[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float2 f = unpack_bf16x2(w[j]);
+        h[j] = pack_h2(f.x * inv_fq, f.y * inv_fq);
+      }
+      *reinterpret_cast<uint4*>(qs + r * C::ROW + c) = make_uint4(h[0], h[1], h[2], h[3]);
+    }
+    named_bar_sync(1, 32 * NCW);
+    // sum of each head's fp16 q (the values the MMAs read)
+    for (int r = warp; r < 8; r += NCW) {
+      float acc = 0.f;
+      for (int d = lane; d < D; d += 32) acc += __half2float(qs[r * C::ROW + d]);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+      if (lane == 0) qsum[r] = acc;
+    }
+    named_bar_sync(1, 32 * NCW);
+    // The MMA fragments come straight from the copied code rows. S: the 16
+    // k positions of k-step s of 64-dim group grp stand for dims
+    // 64 grp + 16 tg' + 4 s + {0, 1} (k = 2tg', 2tg'+1) and + {2, 3} (k = 8+2tg',
+    // 9+2tg'), so a lane's K codes for four k-steps are 16 contiguous bytes,
+    // and its Q fragments 16 contiguous fp16. P.V: output row m of m-tile mt
+    // is dim (D/8) gq' + 16 (mt / 8) + 2 (mt % 8) (+1 for row m + 8), so a
+    // lane's V codes for eight m-tiles are 16 contiguous bytes of each of its
+    // four key rows; the merge puts the dims back in order.
     const int gq = lane >> 2, tg = lane & 3;
-    unsigned char* stg = stg_all + warp * C::STG_B;  // rows 0..15 K, 16..31 V (K = V: 32 K rows)
     float o[D / 16][4];
 #pragma unroll
     for (int mt = 0; mt < D / 16; ++mt) o[mt][0] = o[mt][1] = o[mt][2] = o[mt][3] = 0.f;
-    float m_h = -INFINITY, l_t = 0.f, corr = 0.f;  // corr: sum of p * min of V over this lane's keys
+    // corr: sum of p * min of V over this lane's keys; psum: sum of the fp16
+    // weights P' the MMAs used (the codes carry +1024)
+    float m_h = -INFINITY, l_t = 0.f, corr = 0.f, psum = 0.f;
     const float qsum_h = qsum[gq] * fq;           // sum of head gq's q
     const float sl_fq = a.scale_log2 * fq;
-    const uint32_t q_addr = smem_u32(qs) + ((lane & 7) * C::ROW + ((lane >> 3) & 1) * 8) * 2;
-    const uint32_t frag_off = (((lane >> 4) * 8 + (lane & 7)) * C::ROW + ((lane >> 3) & 1) * 8) * 2;
+    const unsigned char* q_row = reinterpret_cast<const unsigned char*>(qs) + (gq * C::ROW + 16 * tg) * 2;
+    // this lane's keys: S columns / P.V positions 2tg, 2tg+1, 8+2tg, 9+2tg
+    int key_l[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) key_l[i] = key_at(i < 2 ? 2 * tg + i : 8 + 2 * tg + (i - 2));
+    const int kro_a = code_row_off<D>(key_at(gq)) + 16 * tg;       // S rows: n-tile 0
+    const int kro_b = code_row_off<D>(key_at(8 + gq)) + 16 * tg;   // n-tile 1
+    int vro[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) vro[i] = code_row_off<D>(key_l[i]) + (D / 8) * gq;
 
     for (int t = warp; t < n_sub; t += NCW) {
       const int slot = t % C::NSLOT;
@@ -248,67 +287,49 @@ __global__ void __launch_bounds__(32 * (NCW + 1), Q8Cfg<D>::MIN_BLOCKS) k_decode
       const int64_t key0_slot = k_begin + (int64_t)t * kps;
       const int nk_slot = (int)((k_end - key0_slot) < kps ? (k_end - key0_slot) : kps);
       const unsigned char* raw = ring + slot * C::RAW_B;
-      // widen the codes to fp16 staging rows; rows past the end become zeros
-      constexpr int CPR = D / 16;  // 16-code chunks per row
-      for (int idx = lane; idx < 2 * C::KB * CPR; idx += 32) {
-        const int r = idx / CPR, c = idx % CPR;
-        const int key = a.keqv ? r : (r & (C::KB - 1));
-        uint4 lo4 = make_uint4(0, 0, 0, 0), hi4 = make_uint4(0, 0, 0, 0);
-        if (key < nk_slot) {
-          const uint4 u = *reinterpret_cast<const uint4*>(raw + r * D + c * 16);
-          lo4 = make_uint4(codes_to_h2(u.x, 0x4140), codes_to_h2(u.x, 0x4342), codes_to_h2(u.y, 0x4140),
-                           codes_to_h2(u.y, 0x4342));
-          hi4 = make_uint4(codes_to_h2(u.z, 0x4140), codes_to_h2(u.z, 0x4342), codes_to_h2(u.w, 0x4140),
-                           codes_to_h2(u.w, 0x4342));
-        }
-        uint4* d = reinterpret_cast<uint4*>(stg + r * C::ROWB + c * 32);
-        d[0] = lo4;
-        d[1] = hi4;
-      }
-      // this lane's keys of each 16-key half: 2tg, 2tg+1, 8+2tg, 9+2tg
-      const float2* praw = reinterpret_cast<const float2*>(raw + C::CODES_B);  // K [16] then V [16] (K = V: 32 K)
-      float2 kp[2][4], vp[2][4];
-#pragma unroll
-      for (int half = 0; half < 2; ++half)
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int j = (i < 2 ? 2 * tg + i : 8 + 2 * tg + (i - 2));
-          const int kk = half * C::KB + j;
-          const bool have = a.keqv ? kk < nk_slot : (half == 0 && j < nk_slot);
-          kp[half][i] = have ? praw[kk] : make_float2(0.f, 0.f);
-          vp[half][i] = have ? (a.keqv ? kp[half][i] : praw[C::KB + j]) : make_float2(0.f, 0.f);
-        }
-      // the codes and rows are in registers and staging: the slot can refill
-      __syncwarp();
-      if (lane == 0) {
-        consumed[slot] += 1;
-        mbar_arrive(&empty[slot]);
-      }
+      const float2* praw = reinterpret_cast<const float2*>(raw + C::PAR_OFF);  // K [16], V [16] (K = V: 32 K)
       for (int half = 0; half < (a.keqv ? 2 : 1); ++half) {
         const int nk = nk_slot - half * C::KB;
         if (nk <= 0) break;
-        unsigned char* kst = stg + half * C::KB * C::ROWB;
-        unsigned char* vst = a.keqv ? kst : stg + C::KB * C::ROWB;
-        // raw S = Q' C^T (Q' = q / fq): rows = query heads (8 real of 16), cols = 16 keys
-        float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
-        const uint32_t k_addr = smem_u32(kst) + frag_off;
-#pragma unroll 8
-        for (int ks = 0; ks < D / 16; ++ks) {
-          uint32_t qa0, qa2, b0, b1, b2, b3;
-          ldsm_x2(q_addr + ks * 32, qa0, qa2);
-          ldsm_x4(k_addr + ks * 32, b0, b1, b2, b3);
-          mma_f16(s0, qa0, 0u, qa2, 0u, b0, b1);
-          mma_f16(s1, qa0, 0u, qa2, 0u, b2, b3);
-        }
-        // s_j = step_j <q, c_j> + min_j sum(q), in log2 units
-        const float raw_s[4] = {s0[0], s0[1], s1[0], s1[1]};
-        float sv[4];
+        const unsigned char* kreg = raw + half * C::REGION_B;
+        const unsigned char* vreg = a.keqv ? kreg : raw + C::REGION_B;
+        float2 kp[4], vp[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          const int j = (i < 2 ? 2 * tg + i : 8 + 2 * tg + (i - 2));
-          sv[i] = (j < nk) ? (kp[half][i].y * raw_s[i] * sl_fq + kp[half][i].x * qsum_h * a.scale_log2)
-                           : -INFINITY;
+          const bool have = key_l[i] < nk;  // rows past the end hold stale (finite) codes: masked below
+          kp[i] = have ? praw[half * C::KB + key_l[i]] : make_float2(0.f, 0.f);
+          vp[i] = have ? (a.keqv ? kp[i] : praw[C::KB + key_l[i]]) : make_float2(0.f, 0.f);
         }
+        // S' = Q' (1024 + C)^T (Q' = q / fq): rows = query heads (8 real of 16),
+        // cols = 16 keys; even and odd k-steps accumulate apart
+        float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
+        float s2[4] = {0.f, 0.f, 0.f, 0.f}, s3[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 2
+        for (int grp = 0; grp < D / 64; ++grp) {
+          const uint4 qa = *reinterpret_cast<const uint4*>(q_row + grp * 128);
+          const uint4 qb = *reinterpret_cast<const uint4*>(q_row + grp * 128 + 16);
+          const uint4 ka = *reinterpret_cast<const uint4*>(kreg + kro_a + grp * 64);
+          const uint4 kb = *reinterpret_cast<const uint4*>(kreg + kro_b + grp * 64);
+          const uint32_t qw[8] = {qa.x, qa.y, qa.z, qa.w, qb.x, qb.y, qb.z, qb.w};
+          const uint32_t kwa[4] = {ka.x, ka.y, ka.z, ka.w}, kwb[4] = {kb.x, kb.y, kb.z, kb.w};
+#pragma unroll
+          for (int st = 0; st < 4; st += 2) {
+            mma_f16(s0, qw[2 * st], 0u, qw[2 * st + 1], 0u, codes_h2(kwa[st], 0x4140), codes_h2(kwa[st], 0x4342));
+            mma_f16(s1, qw[2 * st], 0u, qw[2 * st + 1], 0u, codes_h2(kwb[st], 0x4140), codes_h2(kwb[st], 0x4342));
+            mma_f16(s2, qw[2 * st + 2], 0u, qw[2 * st + 3], 0u, codes_h2(kwa[st + 1], 0x4140),
+                    codes_h2(kwa[st + 1], 0x4342));
+            mma_f16(s3, qw[2 * st + 2], 0u, qw[2 * st + 3], 0u, codes_h2(kwb[st + 1], 0x4140),
+                    codes_h2(kwb[st + 1], 0x4342));
+          }
+        }
+        // s_j = step_j <q, c_j> + min_j sum(q) = step_j fq S'_j + (min_j - 1024 step_j) sum(q),
+        // in log2 units
+        const float raw_s[4] = {s0[0] + s2[0], s0[1] + s2[1], s1[0] + s3[0], s1[1] + s3[1]};
+        float sv[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          sv[i] = (key_l[i] < nk) ? (kp[i].y * raw_s[i] * sl_fq + (kp[i].x - 1024.f * kp[i].y) * qsum_h * a.scale_log2)
+                                  : -INFINITY;
         float tmax = fmaxf(fmaxf(sv[0], sv[1]), fmaxf(sv[2], sv[3]));
         tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 1));
         tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 2));
@@ -319,8 +340,8 @@ __global__ void __launch_bounds__(32 * (NCW + 1), Q8Cfg<D>::MIN_BLOCKS) k_decode
 #pragma unroll
         for (int i = 0; i < 4; ++i) p[i] = exp2f(sv[i] - base);
         l_t = l_t * alpha + (p[0] + p[1]) + (p[2] + p[3]);
-        corr = corr * alpha + ((p[0] * vp[half][0].x + p[1] * vp[half][1].x) +
-                               (p[2] * vp[half][2].x + p[3] * vp[half][3].x));
+        corr = corr * alpha + ((p[0] * vp[0].x + p[1] * vp[1].x) + (p[2] * vp[2].x + p[3] * vp[3].x));
+        psum *= alpha;
         m_h = m_new;
         const float al0 = __shfl_sync(0xffffffffu, alpha, (2 * tg) * 4);
         const float al1 = __shfl_sync(0xffffffffu, alpha, (2 * tg + 1) * 4);
@@ -334,23 +355,47 @@ __global__ void __launch_bounds__(32 * (NCW + 1), Q8Cfg<D>::MIN_BLOCKS) k_decode
           }
         }
         // P' = p * step_j / fv: the codes' weights, within fp16's range
-        const uint32_t pb0 = pack_h2(p[0] * (vp[half][0].y * inv_fv), p[1] * (vp[half][1].y * inv_fv));
-        const uint32_t pb1 = pack_h2(p[2] * (vp[half][2].y * inv_fv), p[3] * (vp[half][3].y * inv_fv));
+        const uint32_t pb0 = pack_h2(p[0] * (vp[0].y * inv_fv), p[1] * (vp[1].y * inv_fv));
+        const uint32_t pb1 = pack_h2(p[2] * (vp[2].y * inv_fv), p[3] * (vp[3].y * inv_fv));
+        {
+          const float2 f0 = __half22float2(*reinterpret_cast<const __half2*>(&pb0));
+          const float2 f1 = __half22float2(*reinterpret_cast<const __half2*>(&pb1));
+          psum += (f0.x + f0.y) + (f1.x + f1.y);
+        }
         // O'^T += C_V^T P'^T : rows = head dims, cols = query heads, k = 16 keys
-        const uint32_t v_addr = smem_u32(vst) + frag_off;
 #pragma unroll
-        for (int mt = 0; mt < D / 16; ++mt) {
-          uint32_t va0, va1, va2, va3;
-          ldsm_x4_t(v_addr + mt * 32, va0, va1, va2, va3);
-          mma_f16(o[mt], va0, va1, va2, va3, pb0, pb1);
+        for (int c = 0; c < C::VCH; ++c) {
+          const uint4 r0 = *reinterpret_cast<const uint4*>(vreg + vro[0] + 16 * c);
+          const uint4 r1 = *reinterpret_cast<const uint4*>(vreg + vro[1] + 16 * c);
+          const uint4 r2 = *reinterpret_cast<const uint4*>(vreg + vro[2] + 16 * c);
+          const uint4 r3 = *reinterpret_cast<const uint4*>(vreg + vro[3] + 16 * c);
+          const uint32_t w0[4] = {r0.x, r0.y, r0.z, r0.w}, w1[4] = {r1.x, r1.y, r1.z, r1.w};
+          const uint32_t w2[4] = {r2.x, r2.y, r2.z, r2.w}, w3[4] = {r3.x, r3.y, r3.z, r3.w};
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            // keys (2tg, 2tg+1) and (8+2tg, 9+2tg) interleaved per dim
+            const uint32_t t01 = __byte_perm(w0[i], w1[i], 0x5140), t23 = __byte_perm(w0[i], w1[i], 0x7362);
+            const uint32_t u01 = __byte_perm(w2[i], w3[i], 0x5140), u23 = __byte_perm(w2[i], w3[i], 0x7362);
+            mma_f16(o[8 * c + 2 * i], codes_h2(t01, 0x4140), codes_h2(t01, 0x4342),
+                    codes_h2(u01, 0x4140), codes_h2(u01, 0x4342), pb0, pb1);
+            mma_f16(o[8 * c + 2 * i + 1], codes_h2(t23, 0x4140), codes_h2(t23, 0x4342),
+                    codes_h2(u23, 0x4140), codes_h2(u23, 0x4342), pb0, pb1);
+          }
         }
       }  // half
-      __syncwarp();  // the staging rows are rewritten by this warp's next slot
+      // every lane is done with the slot's rows: it can refill
+      __syncwarp();
+      if (lane == 0) {
+        consumed[slot] += 1;
+        mbar_arrive(&empty[slot]);
+      }
     }
     // per head: the sum over the 4 lanes holding its keys
     float l_q = l_t + __shfl_xor_sync(0xffffffffu, l_t, 1);
     l_q += __shfl_xor_sync(0xffffffffu, l_q, 2);
-    float corr_h = corr + __shfl_xor_sync(0xffffffffu, corr, 1);
+    // O = fv (O' - 1024 sum P') + sum p min: the offset goes into the per-head term
+    float corr_h = corr - 1024.f * fv * psum;
+    corr_h += __shfl_xor_sync(0xffffffffu, corr_h, 1);
     corr_h += __shfl_xor_sync(0xffffffffu, corr_h, 2);
     const float c0 = __shfl_sync(0xffffffffu, corr_h, (2 * tg) * 4);      // head 2tg
     const float c1 = __shfl_sync(0xffffffffu, corr_h, (2 * tg + 1) * 4);  // head 2tg + 1
@@ -361,8 +406,8 @@ __global__ void __launch_bounds__(32 * (NCW + 1), Q8Cfg<D>::MIN_BLOCKS) k_decode
     __syncwarp();
     __syncthreads();  // (A) pairs with the producer's (A)
     if (*abort_flag) return;
-    // this warp's O = fv * O' + corr, scaled into the merge buffer (over the staging rows)
-    float* obuf = reinterpret_cast<float*>(stg_all);
+    // this warp's O = fv * O' + corr, scaled into the merge buffer (over the drained ring)
+    float* obuf = reinterpret_cast<float*>(ring);
     float f[2];
 #pragma unroll
     for (int j = 0; j < 2; ++j) {
@@ -375,12 +420,13 @@ __global__ void __launch_bounds__(32 * (NCW + 1), Q8Cfg<D>::MIN_BLOCKS) k_decode
     }
 #pragma unroll
     for (int mt = 0; mt < D / 16; ++mt) {
-      float* row0 = obuf + (warp * 8 + 2 * tg) * C::OSTR + mt * 16 + gq;
+      const int dim = (D / 8) * gq + 16 * (mt / 8) + 2 * (mt % 8);  // row gq of m-tile mt; row gq+8 is dim+1
+      float* row0 = obuf + (warp * 8 + 2 * tg) * C::OSTR + dim;
       float* row1 = row0 + C::OSTR;
       row0[0] = (o[mt][0] * fv + c0) * f[0];
       row1[0] = (o[mt][1] * fv + c1) * f[1];
-      row0[8] = (o[mt][2] * fv + c0) * f[0];
-      row1[8] = (o[mt][3] * fv + c1) * f[1];
+      row0[1] = (o[mt][2] * fv + c0) * f[0];
+      row1[1] = (o[mt][3] * fv + c1) * f[1];
     }
     __syncwarp();
     named_bar_sync(1, 32 * NCW);

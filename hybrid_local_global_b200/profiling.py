@@ -38,7 +38,8 @@ CSRC = os.path.join(os.path.dirname(os.path.abspath(__file__)), "csrc")
 KERNEL_SOURCES = {
     "k_prefill_tc": ("prefill_tc.cu", "tc.cuh", "common.cuh", "tmap.cu", "tmap.h"),
     "k_prefill_pair": ("prefill_pair.cu", "pair.cuh", "tc.cuh", "common.cuh", "tmap.cu", "tmap.h"),
-    "k_decode_split": ("decode.cu", "common.cuh"),
+    "k_decode_split": ("decode.cu", "mma_sync.cuh", "common.cuh"),
+    "k_decode_split_q8": ("decode_q8.cu", "mma_sync.cuh", "common.cuh"),
 }
 
 
@@ -197,8 +198,9 @@ def run(workload: str, reps: int, layers: list[int] | None) -> None:
         max_len = int(lens_cpu.max())
         for l in todo:
             if not st.is_shared(l):
-                synth.fill_randn_bf16_(st.k_cache[l], g)
-                synth.fill_randn_bf16_(st.v_cache[l], g)
+                synth.fill_cache_(st.k_cache[l], g)
+                if st.v_cache[l] is not st.k_cache[l]:
+                    synth.fill_cache_(st.v_cache[l], g)
         ws = torch.empty(st.decode_workspace_bytes(max_len), dtype=torch.uint8, device=dev)
         bufs = {}
         for l in todo:

@@ -39,6 +39,7 @@ class AttentionStack:
             d.n_kv_heads, d.head_dim = t.n_kv_heads, t.head_dim
             d.rope_frac, d.rope_theta, d.shared_from = t.rope_frac, t.rope_theta, -1
             d.k_eq_v = int(self.keqv(l))
+            d.kv_int8 = int(w.kv_int8)
             src = self.share_src[l]
             if src >= 0 and src != l:
                 native.gemma_kv_share_bind(d, self.descs[src])
@@ -47,9 +48,15 @@ class AttentionStack:
             else:
                 shape = (w.batch, t.n_kv_heads, cap, t.head_dim)
                 if alloc_caches:
-                    kc = torch.empty(shape, dtype=torch.bfloat16, device=self.device)
+                    if w.kv_int8:
+                        def new_cache():
+                            return native.Int8KVCache(*shape, self.device)
+                    else:
+                        def new_cache():
+                            return torch.empty(shape, dtype=torch.bfloat16, device=self.device)
+                    kc = new_cache()
                     # K = V: the key cache is the only cache
-                    vc = kc if d.k_eq_v else torch.empty(shape, dtype=torch.bfloat16, device=self.device)
+                    vc = kc if d.k_eq_v else new_cache()
                     d.k_cache, d.v_cache = kc.data_ptr(), (0 if d.k_eq_v else vc.data_ptr())
                 else:
                     kc = vc = None
@@ -74,7 +81,8 @@ class AttentionStack:
             if kc is None or kc.data_ptr() in seen:
                 continue
             seen.add(kc.data_ptr())
-            total += (1 if self.keqv(l) else 2) * kc.numel() * kc.element_size()
+            per = kc.numel() * (1 if isinstance(kc, native.Int8KVCache) else kc.element_size())
+            total += (1 if self.keqv(l) else 2) * per
         return total
 
     # ------------------------------------------------------------------ prefill

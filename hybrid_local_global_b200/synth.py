@@ -35,6 +35,28 @@ def fill_randn_bf16_(t: torch.Tensor, gen: torch.Generator, scale: float = 1.0) 
     return t
 
 
+def fill_int8_cache_(cache, gen: torch.Generator):
+    """Synthetic int8 cache rows: codes uniform on 0..255 and (min, step)
+    near those of a N(0, 1) row of a few hundred channels (min about -3,
+    step about 6 / 255), drawn from `gen` one leading slice at a time."""
+    codes, params = cache.codes, cache.params
+    for i in range(codes.shape[0]):
+        c = torch.randint(0, 256, tuple(codes.shape[1:]), generator=gen, device=codes.device, dtype=torch.int32)
+        codes[i].copy_(c)
+        n = torch.randn(tuple(params.shape[1:]), generator=gen, device=params.device, dtype=torch.float32)
+        params[i, ..., 0].copy_(-3.0 + 0.2 * n[..., 0])
+        params[i, ..., 1].copy_((6.0 / 255.0) * (1.0 + 0.05 * n[..., 1]))
+    return cache
+
+
+def fill_cache_(cache, gen: torch.Generator):
+    """A layer's cache buffer filled with synthetic rows: bf16 N(0, 1), or
+    int8 rows (fill_int8_cache_) for an int8 cache object."""
+    if isinstance(cache, torch.Tensor):
+        return fill_randn_bf16_(cache, gen)
+    return fill_int8_cache_(cache, gen)
+
+
 def decode_lengths(batch: int, lo: int, hi: int, seed: int) -> torch.Tensor:
     """Per-sequence KV lengths uniform on [lo, hi] (int32, CPU)."""
     g = generator(seed)

@@ -46,6 +46,7 @@ class Workload:
     seed: int = 0
     fixed_kinds: tuple = ()      # overrides the schedule: e.g. ("local",) for one local layer
     k_eq_v: bool = False         # global layers use K = V (values are the cached keys)
+    kv_int8: bool = False        # int8 KV caches (codes + (min, step) per row)
     description: str = field(default="", compare=False)
 
 
@@ -72,6 +73,12 @@ WORKLOADS = {
         local=L31B_LOCAL, global_=L31B_GLOBAL, len_lo=4096, len_hi=131072, n_shared=2, seed=3,
         description="31B-shaped 6-layer decode: B64, KV length U[4096,131072], ring 1024, "
                     "last 2 layers shared"),
+    "31b_decode_b64_int8": Workload(
+        "31b_decode_b64_int8", "decode", batch=64, n_q_heads=32, n_layers=6, ratio=5,
+        local=L31B_LOCAL, global_=L31B_GLOBAL, len_lo=4096, len_hi=131072, n_shared=2, seed=3,
+        kv_int8=True,
+        description="31B-shaped 6-layer decode on int8 KV caches: B64, KV length U[4096,131072], "
+                    "ring 1024, last 2 layers shared"),
     "31b_decode_b16_12l_shared": Workload(
         "31b_decode_b16_12l_shared", "decode", batch=16, n_q_heads=32, n_layers=12, ratio=5,
         local=L31B_LOCAL, global_=L31B_GLOBAL, len_lo=4096, len_hi=131072, n_shared=2, seed=7,
@@ -96,6 +103,16 @@ WORKLOADS = {
         local=L31B_LOCAL, global_=L31B_GLOBAL, len_lo=262144, len_hi=262144, seed=4,
         fixed_kinds=("global",),
         description="single-token decode at KV length 262144, one global layer"),
+    "local_decode_b64_int8": Workload(
+        "local_decode_b64_int8", "decode", batch=64, n_q_heads=32, n_layers=1, ratio=0,
+        local=L31B_LOCAL, global_=L31B_GLOBAL, len_lo=4096, len_hi=131072, seed=3,
+        fixed_kinds=("local",), kv_int8=True,
+        description="one 31B-shaped local layer's decode on an int8 ring: B64, ring 1024"),
+    "global_decode_256k_int8": Workload(
+        "global_decode_256k_int8", "decode", batch=1, n_q_heads=32, n_layers=1, ratio=0,
+        local=L31B_LOCAL, global_=L31B_GLOBAL, len_lo=262144, len_hi=262144, seed=4,
+        fixed_kinds=("global",), kv_int8=True,
+        description="single-token decode at KV length 262144 on an int8 KV cache, one global layer"),
 }
 
 
