@@ -334,11 +334,32 @@ size_t gemma_attn_prefill_workspace_size(int batch, int s_new, int n_q_heads, in
   return prefill_ws_parts(batch, s_new, n_q_heads, n_kv_heads, head_dim, window, &off_k);
 }
 
-int gemma_attn_prefill(const void* q, const void* k_new, const void* v_new, void* k_cache, void* v_cache,
-                       int cache_cap, const int32_t* seq_lens_before, int batch, int s_new, int window,
-                       int n_q_heads, int n_kv_heads, int head_dim, float rope_frac, float rope_theta,
-                       float scale, void* out, float* lse, void* workspace, size_t workspace_bytes,
-                       unsigned flags, void* stream) {
+// Where a layer's cache rows live (see cache_row): a contiguous cache, or
+// the pages of a pool named by a page table (global layers).
+struct CacheLayout {
+  const int32_t* page_table;  // [batch][pages_per_seq], or null
+  int page_size, pages_per_seq, n_pages;
+};
+
+static CacheLayout contiguous(int cache_cap, int batch) { return CacheLayout{nullptr, cache_cap, 1, batch}; }
+
+static int check_paged(const int32_t* page_table, int page_size, int pages_per_seq, int n_pages, unsigned flags) {
+  if (!page_table) return fail(GEMMA_ERR_INVALID_ARG, "paged cache: null page table");
+  if (page_size <= 0 || page_size % 128)
+    return fail(GEMMA_ERR_INVALID_ARG, "paged cache: page_size %d must be a positive multiple of 128", page_size);
+  if (pages_per_seq <= 0 || n_pages <= 0)
+    return fail(GEMMA_ERR_INVALID_ARG, "paged cache: pages_per_seq %d, n_pages %d", pages_per_seq, n_pages);
+  if ((int64_t)pages_per_seq * page_size > INT32_MAX)
+    return fail(GEMMA_ERR_INVALID_ARG, "paged cache: pages_per_seq * page_size exceeds 2^31");
+  if (flags & GEMMA_F_KV_INT8) return fail(GEMMA_ERR_UNSUPPORTED, "paged cache: int8 rows are not paged in this build");
+  return GEMMA_OK;
+}
+
+static int prefill_impl(const void* q, const void* k_new, const void* v_new, void* k_cache, void* v_cache,
+                        int cache_cap, const int32_t* seq_lens_before, int batch, int s_new, int window,
+                        int n_q_heads, int n_kv_heads, int head_dim, float rope_frac, float rope_theta,
+                        float scale, void* out, float* lse, void* workspace, size_t workspace_bytes,
+                        unsigned flags, void* stream, const CacheLayout& L) {
   int rc = check_heads(n_q_heads, n_kv_heads, head_dim, window, rope_frac, rope_theta, scale);
   if (rc) return rc;
   rc = check_kv_flags(flags, window, k_new, v_new, k_cache, &v_cache);
@@ -410,6 +431,10 @@ int gemma_attn_prefill(const void* q, const void* k_new, const void* v_new, void
   // log2 units (one bf16 rounding either way)
   ra.q_scale = (float)((double)scale * 1.4426950408889634);
   ra.quant = q8 ? 1 : 0;
+  ra.page_table = L.page_table;
+  ra.page_size = L.page_size;
+  ra.pages_per_seq = L.pages_per_seq;
+  ra.n_pages = L.n_pages;
   ra.status = status;
   ProfScope p_rope(GEMMA_KERNEL_PREFILL_ROPE, st);
   cudaError_t e = launch_prefill_rope(ra, batch, head_dim, st);
@@ -423,7 +448,10 @@ int gemma_attn_prefill(const void* q, const void* k_new, const void* v_new, void
   aa.q_rot = ra.q_rot;
   const int64_t D = head_dim;
   if ((window == 0 || shared) && !q8) {
-    KVView kc = {static_cast<const bf16*>(k_cache), (int64_t)n_kv_heads * cache_cap * D, D, (int64_t)cache_cap * D};
+    // head-major views of the cache's pages (a contiguous cache: one page of
+    // cache_cap rows per sequence)
+    const int64_t ps = L.page_size;
+    KVView kc = {static_cast<const bf16*>(k_cache), (int64_t)n_kv_heads * ps * D, D, ps * D};
     KVView vc = {static_cast<const bf16*>(v_cache), kc.stride_b, kc.stride_row, kc.stride_h};
     aa.k = kc;
     aa.v = vc;
@@ -454,6 +482,10 @@ int gemma_attn_prefill(const void* q, const void* k_new, const void* v_new, void
   aa.status = status;
   aa.wait_ns = (unsigned long long)g_wait_ns.load();
   const bool cache_view = (window == 0 || shared) && !q8;
+  aa.page_table = cache_view ? L.page_table : nullptr;
+  aa.page_size = L.page_size;
+  aa.pages_per_seq = L.pages_per_seq;
+  aa.n_pages = cache_view ? L.n_pages : batch;
   ProfScope p_attn(GEMMA_KERNEL_PREFILL_ATTN, st);
   // Head_dim-512 layers run on CTA pairs (cta_group::2, M = 256): each SM
   // loads and reads from shared memory half of every K and V tile. With an
@@ -475,13 +507,36 @@ int gemma_attn_prefill(const void* q, const void* k_new, const void* v_new, void
     if (std::string(v) == "pair") kern = K_PAIR;
     if (std::string(v) == "hpair") kern = K_HPAIR;
   }
-  const int key_rows = cache_view ? cache_cap : (int)aa.key_cap;
+  const int key_rows = cache_view ? L.page_size : (int)aa.key_cap;
   const int tok_major = cache_view ? 0 : 1;
   e = kern == K_SINGLE ? launch_prefill_attn_tc(aa, batch, head_dim, key_rows, tok_major, st)
                        : launch_prefill_attn_pair(aa, batch, head_dim, key_rows, tok_major, kern == K_HPAIR, st);
   p_attn.done();
   if (e != cudaSuccess) return cuda_fail(e, "prefill attention launch");
   return succeed();
+}
+
+int gemma_attn_prefill(const void* q, const void* k_new, const void* v_new, void* k_cache, void* v_cache,
+                       int cache_cap, const int32_t* seq_lens_before, int batch, int s_new, int window,
+                       int n_q_heads, int n_kv_heads, int head_dim, float rope_frac, float rope_theta,
+                       float scale, void* out, float* lse, void* workspace, size_t workspace_bytes,
+                       unsigned flags, void* stream) {
+  return prefill_impl(q, k_new, v_new, k_cache, v_cache, cache_cap, seq_lens_before, batch, s_new, window,
+                      n_q_heads, n_kv_heads, head_dim, rope_frac, rope_theta, scale, out, lse, workspace,
+                      workspace_bytes, flags, stream, contiguous(cache_cap, batch));
+}
+
+int gemma_attn_prefill_paged(const void* q, const void* k_new, const void* v_new, void* k_pool, void* v_pool,
+                             const int32_t* page_table, int page_size, int pages_per_seq, int n_pages,
+                             const int32_t* seq_lens_before, int batch, int s_new, int n_q_heads,
+                             int n_kv_heads, int head_dim, float rope_frac, float rope_theta, float scale,
+                             void* out, float* lse, void* workspace, size_t workspace_bytes, unsigned flags,
+                             void* stream) {
+  int rc = check_paged(page_table, page_size, pages_per_seq, n_pages, flags);
+  if (rc) return rc;
+  return prefill_impl(q, k_new, v_new, k_pool, v_pool, pages_per_seq * page_size, seq_lens_before, batch, s_new,
+                      0, n_q_heads, n_kv_heads, head_dim, rope_frac, rope_theta, scale, out, lse, workspace,
+                      workspace_bytes, flags, stream, CacheLayout{page_table, page_size, pages_per_seq, n_pages});
 }
 
 size_t gemma_attn_decode_workspace_size(int batch, int n_q_heads, int n_kv_heads, int head_dim, int window,
@@ -493,11 +548,11 @@ size_t gemma_attn_decode_workspace_size(int batch, int n_q_heads, int n_kv_heads
   return decode_ws_parts(batch, n_q_heads, n_kv_heads, head_dim, n_splits, &a, &b);
 }
 
-int gemma_attn_decode(const void* q, const void* k_new, const void* v_new, void* k_cache, void* v_cache,
-                      int cache_cap, const int32_t* seq_lens, int max_seq_len, int batch, int window,
-                      int n_q_heads, int n_kv_heads, int head_dim, float rope_frac, float rope_theta,
-                      float scale, void* out, void* workspace, size_t workspace_bytes, unsigned flags,
-                      void* stream) {
+static int decode_impl(const void* q, const void* k_new, const void* v_new, void* k_cache, void* v_cache,
+                       int cache_cap, const int32_t* seq_lens, int max_seq_len, int batch, int window,
+                       int n_q_heads, int n_kv_heads, int head_dim, float rope_frac, float rope_theta,
+                       float scale, void* out, void* workspace, size_t workspace_bytes, unsigned flags,
+                       void* stream, const CacheLayout& L) {
   int rc = check_heads(n_q_heads, n_kv_heads, head_dim, window, rope_frac, rope_theta, scale);
   if (rc) return rc;
   rc = check_kv_flags(flags, window, k_new, v_new, k_cache, &v_cache);
@@ -542,6 +597,10 @@ int gemma_attn_decode(const void* q, const void* k_new, const void* v_new, void*
   ra.n_rot = rope_rotated_pairs(head_dim, rope_frac);
   ra.log2_theta = std::log2((double)rope_theta);
   ra.k_stage = q8 ? reinterpret_cast<bf16*>(ws + off_kst) : nullptr;
+  ra.page_table = L.page_table;
+  ra.page_size = L.page_size;
+  ra.pages_per_seq = L.pages_per_seq;
+  ra.n_pages = L.n_pages;
   ra.status = status;
   // rotates q; also appends the new K/V unless the layer is shared (int8:
   // the rotated key is staged, then both rows are quantized into the cache)
@@ -573,6 +632,10 @@ int gemma_attn_decode(const void* q, const void* k_new, const void* v_new, void*
   da.wait_ns = (unsigned long long)g_wait_ns.load();
   da.drop_first_copy = g_drop_next.exchange(0);
   da.keqv = (flags & GEMMA_F_KEQV) ? 1 : 0;
+  da.page_table = L.page_table;
+  da.page_size = L.page_size;
+  da.pages_per_seq = L.pages_per_seq;
+  da.n_pages = L.n_pages;
   if (q8) {
     const size_t off = gemma_kv_codes_bytes(batch, n_kv_heads, cache_cap, head_dim);
     da.k_codes = static_cast<const uint8_t*>(k_cache);
@@ -593,6 +656,28 @@ int gemma_attn_decode(const void* q, const void* k_new, const void* v_new, void*
   }
   if (e != cudaSuccess) return cuda_fail(e, "decode combine launch");
   return succeed();
+}
+
+int gemma_attn_decode(const void* q, const void* k_new, const void* v_new, void* k_cache, void* v_cache,
+                      int cache_cap, const int32_t* seq_lens, int max_seq_len, int batch, int window,
+                      int n_q_heads, int n_kv_heads, int head_dim, float rope_frac, float rope_theta,
+                      float scale, void* out, void* workspace, size_t workspace_bytes, unsigned flags,
+                      void* stream) {
+  return decode_impl(q, k_new, v_new, k_cache, v_cache, cache_cap, seq_lens, max_seq_len, batch, window, n_q_heads,
+                     n_kv_heads, head_dim, rope_frac, rope_theta, scale, out, workspace, workspace_bytes, flags,
+                     stream, contiguous(cache_cap, batch));
+}
+
+int gemma_attn_decode_paged(const void* q, const void* k_new, const void* v_new, void* k_pool, void* v_pool,
+                            const int32_t* page_table, int page_size, int pages_per_seq, int n_pages,
+                            const int32_t* seq_lens, int max_seq_len, int batch, int n_q_heads, int n_kv_heads,
+                            int head_dim, float rope_frac, float rope_theta, float scale, void* out,
+                            void* workspace, size_t workspace_bytes, unsigned flags, void* stream) {
+  int rc = check_paged(page_table, page_size, pages_per_seq, n_pages, flags);
+  if (rc) return rc;
+  return decode_impl(q, k_new, v_new, k_pool, v_pool, pages_per_seq * page_size, seq_lens, max_seq_len, batch, 0,
+                     n_q_heads, n_kv_heads, head_dim, rope_frac, rope_theta, scale, out, workspace, workspace_bytes,
+                     flags, stream, CacheLayout{page_table, page_size, pages_per_seq, n_pages});
 }
 
 int gemma_attn_visible_ranges(const int32_t* seq_lens_before, int batch, int s_new, int window,

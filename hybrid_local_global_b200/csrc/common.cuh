@@ -28,6 +28,18 @@ __host__ __device__ __forceinline__ int64_t visible_range(int64_t pos, int windo
   return b >= a ? b - a + 1 : 0;
 }
 
+// Cache addressing. A layer's cache is a pool of pages [n_pages][Hkv][ps][D];
+// position (or ring slot) p of sequence b lives at row p % ps of page
+// table[b * pps + p / ps]. A contiguous cache [B][Hkv][cap][D] is the case
+// table == null: page b, ps = cap. Returns the row index into the pool
+// (in units of D elements), or -1 when the page index is outside the pool.
+__host__ __device__ __forceinline__ int64_t cache_row(const int32_t* table, int pps, int ps, int n_pages,
+                                                      int Hkv, int b, int h, int64_t p) {
+  const int64_t page = table ? (int64_t)table[(int64_t)b * pps + p / ps] : (int64_t)b;
+  if (page < 0 || page >= n_pages) return -1;
+  return (page * Hkv + h) * ps + p % ps;
+}
+
 // Number of rotated pairs under (p-)RoPE: floor(rope_frac * head_dim / 2).
 __host__ __forceinline__ int rope_rotated_pairs(int head_dim, float rope_frac) {
   double v = (double)rope_frac * (double)(head_dim / 2);

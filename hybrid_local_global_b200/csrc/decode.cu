@@ -124,9 +124,8 @@ __global__ void __launch_bounds__(32 * (NCW + 1), 2) k_decode_split(DecodeAttnAr
   // (the same bytes per slot, so as many bytes stay in flight)
   const int kps = a.keqv ? 2 * C::KB : C::KB;
   const int n_sub = (int)((k_end - k_begin + kps - 1) / kps);
-  const int64_t head_off = ((int64_t)b * a.Hkv + g) * (int64_t)a.cache_cap * D;
-  const bf16* kbase = a.k_cache + head_off;
-  const bf16* vbase = a.v_cache + head_off;
+  // a sub-block's rows are contiguous: pages hold a multiple of 32 rows and
+  // sub-blocks start at multiples of 16 (32 under K = V)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::NSLOT; ++s) {
@@ -166,6 +165,13 @@ __global__ void __launch_bounds__(32 * (NCW + 1), 2) k_decode_split(DecodeAttnAr
       const int nk = (int)((k_end - key0) < kps ? (k_end - key0) : kps);
       const bool drop = a.drop_first_copy && t == 0 && split == 0 && g == 0 && b == 0;
       if (drop) continue;
+      int64_t brow = cache_row(a.page_table, a.pages_per_seq, a.page_size, a.n_pages, a.Hkv, b, g, key0);
+      if (brow < 0) {  // a page outside the pool: report it and read pool row 0 (finite, wrong)
+        if (lane == 0) set_status(a.status, GEMMA_ERR_DEVICE_RANGE);
+        brow = 0;
+      }
+      const bf16* kbase = a.k_cache + brow * D;
+      const bf16* vbase = a.v_cache + brow * D;
       if (lane == 0) {
         mbar_arrive_expect_tx(&full[slot], (uint32_t)((a.keqv ? 1 : 2) * nk * D * 2));
         issued[slot] += 1;
@@ -180,7 +186,7 @@ __global__ void __launch_bounds__(32 * (NCW + 1), 2) k_decode_split(DecodeAttnAr
         const int left = nk - grp * C::RPC;
         if (left > 0)
           bulk_g2s(ring + slot * C::SLOT_B + (isv ? C::GPR * C::GROUPB : 0) + grp * C::GROUPB,
-                   (isv ? vbase : kbase) + (key0 + grp * C::RPC) * D,
+                   (isv ? vbase : kbase) + (int64_t)grp * C::RPC * D,
                    (left >= C::RPC ? C::RPC : left) * D * 2, &full[slot]);
       }
     }

@@ -28,6 +28,10 @@ struct PrefillRopeArgs {
   float q_scale;       // rotated Q is multiplied by this before the bf16 rounding
   int quant;           // int8 cache: rotated K goes to k_rot ([B][S][Hkv][D]) on every layer
                        // type and nothing is written into the cache (launch_quantize_rows does)
+  // cache pages (see cache_row): table [B][pages_per_seq] or null for a
+  // contiguous cache (page_size = cache_cap, n_pages = B)
+  const int32_t* page_table;
+  int page_size, pages_per_seq, n_pages;
   int* status;
 };
 
@@ -45,6 +49,10 @@ struct DecodeRopeArgs {
   int max_len, window, Hq, Hkv;
   int n_rot;
   double log2_theta;
+  // cache pages (see cache_row): table [B][pages_per_seq] or null for a
+  // contiguous cache (page_size = cache_cap, n_pages = B)
+  const int32_t* page_table;
+  int page_size, pages_per_seq, n_pages;
   int* status;
 };
 
@@ -85,6 +93,11 @@ struct PrefillAttnArgs {
   float* lse;          // [B][Hq][S] or null
   int* status;
   unsigned long long wait_ns;
+  // cache pages (see cache_row): table [B][pages_per_seq] or null for a
+  // contiguous cache; a paged cache is read through head-major
+  // views of the pool: view row = position % page_size, view batch = page
+  const int32_t* page_table;
+  int page_size, pages_per_seq, n_pages;
 };
 
 struct DecodeAttnArgs {
@@ -109,6 +122,10 @@ struct DecodeAttnArgs {
   const uint8_t* v_codes;
   const float2* k_params;
   const float2* v_params;
+  // cache pages (see cache_row): table [B][pages_per_seq] or null for a
+  // contiguous cache (page_size = cache_cap, n_pages = B)
+  const int32_t* page_table;
+  int page_size, pages_per_seq, n_pages;
 };
 
 cudaError_t launch_prefill_rope(const PrefillRopeArgs& a, int B, int D, cudaStream_t st);

@@ -107,6 +107,10 @@ struct PairArgs {
   int kv_token_major;  // K/V map coordinates: 0 = (d, key, head, b), 1 = (d, head, key, b)
   int key_off_window;  // 1: K/V view row = position - (pos0 - window), else = position
   int n_pairs;         // query-tile pairs per (batch, head); with head_pair: query tiles
+  // paged cache (head-major views of the pool): view row = position % page_size,
+  // view batch = page_table[b * pages_per_seq + position / page_size]; null: contiguous
+  const int32_t* page_table;
+  int page_size, pages_per_seq, n_pages;
   int head_pair;       // 1: the CTAs take q heads 2p and 2p+1 of one query tile (same KV head)
 };
 
@@ -256,7 +260,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
       for (int j = 0; j <= n_tiles && ok; ++j) {
         for (int kind = 0; kind < 2 && ok; ++kind) {  // 0: K_j, 1: V_{j-1}
           if ((kind == 0 && j == n_tiles) || (kind == 1 && j == 0)) continue;
-          const int key0 = (int)((kt0 + j - kind) * BN - koff);  // view row
+          int key0 = (int)((kt0 + j - kind) * BN - koff);  // view row
+          int kb = b;                                           // view batch
+          if (a.page_table) {
+            // tiles never straddle a page (page_size is a multiple of 128); a
+            // tile past the sequence's pages holds no visible key: any page
+            const int pi = key0 / a.page_size;
+            kb = pi < a.pages_per_seq ? a.page_table[(int64_t)b * a.pages_per_seq + pi] : 0;
+            if (kb < 0 || kb >= a.n_pages) {
+              if ((int64_t)key0 < n_keys) set_status(a.status, GEMMA_ERR_DEVICE_RANGE);
+              kb = 0;
+            }
+            key0 -= pi * a.page_size;
+          }
           const int n_st = kind == 0 ? Cfg::K_STAGES : 1;
           for (int hs = 0; hs < n_st; ++hs, ++item) {
             const int s = item % NSTAGE;
@@ -275,17 +291,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
               for (int cc = 0; cc < 4; ++cc) {
                 const int d0 = (hs * 4 + cc) * 64;
                 if (a.kv_token_major)
-                  pair::tma_load_4d_pair(dst + cc * CHUNK_K, &tm_k, d0, g, k0, b, bar);
+                  pair::tma_load_4d_pair(dst + cc * CHUNK_K, &tm_k, d0, g, k0, kb, bar);
                 else
-                  pair::tma_load_4d_pair(dst + cc * CHUNK_K, &tm_k, d0, k0, g, b, bar);
+                  pair::tma_load_4d_pair(dst + cc * CHUNK_K, &tm_k, d0, k0, g, kb, bar);
               }
             } else {
               const int c0 = vh * DV + (int)rank * VH;  // this CTA's 128 output columns
               for (int c = 0; c < 2; ++c) {
                 if (a.kv_token_major)
-                  pair::tma_load_4d_pair(dst + c * CHUNK_V, &tm_v, c0 + c * 64, g, key0, b, bar);
+                  pair::tma_load_4d_pair(dst + c * CHUNK_V, &tm_v, c0 + c * 64, g, key0, kb, bar);
                 else
-                  pair::tma_load_4d_pair(dst + c * CHUNK_V, &tm_v, c0 + c * 64, key0, g, b, bar);
+                  pair::tma_load_4d_pair(dst + c * CHUNK_V, &tm_v, c0 + c * 64, key0, g, kb, bar);
               }
             }
           }
@@ -577,6 +593,10 @@ cudaError_t launch_prefill_attn_pair(const PrefillAttnArgs& a, int B, int D, int
   t.wait_ns = a.wait_ns;
   t.kv_token_major = kv_token_major;
   t.key_off_window = a.key_off_window;
+  t.page_table = a.page_table;
+  t.page_size = a.page_size;
+  t.pages_per_seq = a.pages_per_seq;
+  t.n_pages = a.n_pages;
   const int n_qtiles = (a.S + BM - 1) / BM;
   // head pairs need an even number of q heads per KV head (both share its K/V)
   t.head_pair = head_pair && (a.Hq / a.Hkv) % 2 == 0;

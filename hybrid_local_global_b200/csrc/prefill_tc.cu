@@ -97,6 +97,10 @@ struct TcArgs {
   int kv_token_major;  // K/V map coordinates: 0 = (d, key, head, b), 1 = (d, head, key, b)
   int key_off_window;  // 1: K/V view row = position - (pos0 - window), else = position
   int n_qtiles;
+  // paged cache (head-major views of the pool): view row = position % page_size,
+  // view batch = page_table[b * pages_per_seq + position / page_size]; null: contiguous
+  const int32_t* page_table;
+  int page_size, pages_per_seq, n_pages;
 };
 
 __device__ __forceinline__ bool wait_all(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
@@ -222,7 +226,19 @@ __global__ void __launch_bounds__(192, 1)
       for (int j = 0; j <= n_tiles && ok; ++j) {
         for (int kind = 0; kind < 2 && ok; ++kind) {  // 0: K_j, 1: V_{j-1}
           if ((kind == 0 && j == n_tiles) || (kind == 1 && j == 0)) continue;
-          const int key0 = (int)((kt0 + j - kind) * BN - koff);  // view row
+          int key0 = (int)((kt0 + j - kind) * BN - koff);  // view row
+          int kb = b;                                           // view batch
+          if (a.page_table) {
+            // tiles never straddle a page (page_size is a multiple of 128); a
+            // tile past the sequence's pages holds no visible key: any page
+            const int pi = key0 / a.page_size;
+            kb = pi < a.pages_per_seq ? a.page_table[(int64_t)b * a.pages_per_seq + pi] : 0;
+            if (kb < 0 || kb >= a.n_pages) {
+              if ((int64_t)key0 < n_keys) set_status(a.status, GEMMA_ERR_DEVICE_RANGE);
+              kb = 0;
+            }
+            key0 -= pi * a.page_size;
+          }
           const int n_st = kind == 0 ? Cfg::K_STAGES : 2;
           for (int half = 0; half < n_st; ++half, ++item) {
             const int s = item % NSTAGE;
@@ -240,17 +256,17 @@ __global__ void __launch_bounds__(192, 1)
               for (int cc = 0; cc < 2; ++cc) {
                 const int d0 = (half * 2 + cc) * 64;
                 if (a.kv_token_major)
-                  tc::tma_load_4d(dst + cc * CHUNK_B, &tm_k, d0, g, key0, b, bar);
+                  tc::tma_load_4d(dst + cc * CHUNK_B, &tm_k, d0, g, key0, kb, bar);
                 else
-                  tc::tma_load_4d(dst + cc * CHUNK_B, &tm_k, d0, key0, g, b, bar);
+                  tc::tma_load_4d(dst + cc * CHUNK_B, &tm_k, d0, key0, g, kb, bar);
               }
             } else {
               const int k0 = key0 + half * 64;
               for (int c = 0; c < 4; ++c) {
                 if (a.kv_token_major)
-                  tc::tma_load_4d(dst + c * 8192, &tm_v, vh * DV + c * 64, g, k0, b, bar);
+                  tc::tma_load_4d(dst + c * 8192, &tm_v, vh * DV + c * 64, g, k0, kb, bar);
                 else
-                  tc::tma_load_4d(dst + c * 8192, &tm_v, vh * DV + c * 64, k0, g, b, bar);
+                  tc::tma_load_4d(dst + c * 8192, &tm_v, vh * DV + c * 64, k0, g, kb, bar);
               }
             }
           }
@@ -528,6 +544,10 @@ cudaError_t launch_prefill_attn_tc(const PrefillAttnArgs& a, int B, int D, int k
   t.wait_ns = a.wait_ns;
   t.kv_token_major = kv_token_major;
   t.key_off_window = a.key_off_window;
+  t.page_table = a.page_table;
+  t.page_size = a.page_size;
+  t.pages_per_seq = a.pages_per_seq;
+  t.n_pages = a.n_pages;
   t.n_qtiles = (a.S + BM - 1) / BM;
   if (D == 256) {
     using Cfg = TcCfg<256>;

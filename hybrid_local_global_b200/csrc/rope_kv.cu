@@ -187,7 +187,15 @@ __global__ void __launch_bounds__(256, 2) k_prefill_rope(PrefillRopeArgs a) {
         if (h0 + u < a.Hkv) {
           const int kh = h0 + u;
           const uint4 kr = rotate_chunk(kx[u], t, e0, a.n_rot);
-          const int64_t cslot = (((int64_t)b * a.Hkv + kh) * a.cache_cap + slot) * D + e0;
+          int64_t crow = 0;
+          if ((a.window == 0 && !a.quant) || to_ring) {
+            crow = cache_row(a.page_table, a.pages_per_seq, a.page_size, a.n_pages, a.Hkv, b, kh, slot);
+            if (crow < 0) {  // a page outside the pool: report, write nothing
+              set_status(a.status, GEMMA_ERR_DEVICE_RANGE);
+              continue;
+            }
+          }
+          const int64_t cslot = crow * D + e0;
           if (a.window == 0 && !a.quant) {
             st16(a.k_cache + cslot, kr);
             if (want_v) st16(a.v_cache + cslot, vx[u]);
@@ -277,7 +285,12 @@ __global__ void __launch_bounds__(256) k_decode_rope_append(DecodeRopeArgs a) {
       continue;
     }
     bf16* cache = is_k ? a.k_cache : a.v_cache;
-    st16(cache + (((int64_t)b * a.Hkv + kh) * a.cache_cap + slot) * D + e0, v);
+    const int64_t crow = cache_row(a.page_table, a.pages_per_seq, a.page_size, a.n_pages, a.Hkv, b, kh, slot);
+    if (crow < 0) {  // a page outside the pool: report, write nothing
+      set_status(a.status, GEMMA_ERR_DEVICE_RANGE);
+      continue;
+    }
+    st16(cache + crow * D + e0, v);
   }
 }
 

@@ -58,7 +58,10 @@ bool make_prefill_maps(const PrefillAttnArgs& a, int B, int D, int key_rows_tota
     const uint32_t bk[4] = {64, 1, k_rows, 1}, bv[4] = {64, 1, v_rows, 1};
     return make_map_bf16_4d(mk, a.k.ptr, dims, strk, bk) && make_map_bf16_4d(mv, a.v.ptr, dims, strv, bv);
   }
-  const uint64_t dims[4] = {(uint64_t)D, (uint64_t)key_rows_total, (uint64_t)a.Hkv, (uint64_t)B};
+  // head-major views are cache views: pages of key_rows_total rows (a
+  // contiguous cache is n_pages = B pages of its capacity)
+  const uint64_t dims[4] = {(uint64_t)D, (uint64_t)key_rows_total, (uint64_t)a.Hkv,
+                            (uint64_t)(a.n_pages > 0 ? a.n_pages : B)};
   const uint64_t strk[3] = {(uint64_t)a.k.stride_row * E, (uint64_t)a.k.stride_h * E,
                             (uint64_t)a.k.stride_b * E};
   const uint64_t strv[3] = {(uint64_t)a.v.stride_row * E, (uint64_t)a.v.stride_h * E,

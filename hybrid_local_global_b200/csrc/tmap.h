@@ -18,7 +18,8 @@ bool make_map_bf16_4d(CUtensorMap* m, const void* ptr, const uint64_t dims[4], c
 //   q, o  [B][S][Hq][D], box 64 dims x 1 head x q_rows x 1;
 //   k     the K view, box 64 dims x k_rows keys;
 //   v     the V view, box 64 dims x v_rows keys;
-// the K/V views are [B][rows][Hkv][D] (kv_token_major) or [B][Hkv][rows][D].
+// the K/V views are [B][rows][Hkv][D] (kv_token_major) or [pages][Hkv][rows][D]
+// (a cache: a.n_pages pages of key_rows_total rows; n_pages = B when contiguous).
 bool make_prefill_maps(const PrefillAttnArgs& a, int B, int D, int key_rows_total, int kv_token_major,
                        uint32_t q_rows, uint32_t k_rows, uint32_t v_rows, CUtensorMap* mq, CUtensorMap* mk,
                        CUtensorMap* mv, CUtensorMap* mo);

@@ -66,13 +66,18 @@ _last = _sig("gemma_last_error", ctypes.c_char_p, [])
 _wait = _sig("gemma_attn_set_wait_limit", _I, [ctypes.c_longlong])
 _drop = _sig("gemma_attn_debug_drop_next_copy", _I, [_I])
 _kv_bytes = _sig("gemma_kv_cache_bytes", _SZ, [_I, _I, _I, _I, ctypes.c_uint])
+_prefill_paged = _sig("gemma_attn_prefill_paged", _I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _P, _I, _I, _I, _I,
+                                                       _I, _F, _F, _F, _P, _P, _P, _SZ, ctypes.c_uint, _P])
+_decode_paged = _sig("gemma_attn_decode_paged", _I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _P, _I, _I, _I, _I, _I,
+                                                     _F, _F, _F, _P, _P, _SZ, ctypes.c_uint, _P])
 _kv_codes = _sig("gemma_kv_codes_bytes", _SZ, [_I, _I, _I, _I])
 
 EXPORTED = ["gemma_attn_prefill_workspace_size", "gemma_attn_prefill",
             "gemma_attn_decode_workspace_size", "gemma_attn_decode", "gemma_kv_share_bind",
             "gemma_layer_schedule", "gemma_attn_visible_ranges", "gemma_attn_sync_status",
             "gemma_last_error", "gemma_attn_set_wait_limit", "gemma_attn_debug_drop_next_copy",
-            "gemma_kv_cache_bytes", "gemma_kv_codes_bytes"]
+            "gemma_kv_cache_bytes", "gemma_kv_codes_bytes", "gemma_attn_prefill_paged",
+            "gemma_attn_decode_paged"]
 
 
 class GemmaError(RuntimeError):
@@ -188,6 +193,50 @@ def gemma_attn_decode(q, k_new, v_new, k_cache, v_cache, *, seq_lens, max_seq_le
                           _ptr(seq_lens), max_seq_len, B, window, Hq, Hkv, D, rope_frac,
                           rope_theta, scale, _ptr(out), _ptr(workspace), workspace.numel(), flags,
                           _stream(stream)))
+
+
+def _paged_args(k_pool, page_table):
+    if page_table.dtype != torch.int32 or not page_table.is_cuda or page_table.dim() != 2:
+        raise TypeError("page_table must be an int32 CUDA tensor [batch, pages_per_seq]")
+    n_pages, Hkv, page_size, _ = k_pool.shape
+    return n_pages, Hkv, page_size, page_table.shape[1]
+
+
+def gemma_attn_prefill_paged(q, k_new, v_new, k_pool, v_pool, page_table, *, rope_frac, rope_theta, scale, out,
+                             seq_lens_before=None, lse=None, workspace=None, flags=0, stream=None):
+    """Global layer on a paged cache: pools [n_pages, Hkv, page_size, D]
+    (bf16), page_table int32 [B, pages_per_seq] on the device."""
+    for t, n in ((q, "q"), (k_new, "k_new"), (v_new, "v_new"), (k_pool, "k_pool"), (v_pool, "v_pool"),
+                 (out, "out")):
+        _bf16(t, n)
+    B, S, Hq, D = q.shape
+    n_pages, Hkv, ps, pps = _paged_args(k_pool, page_table)
+    if workspace is None:
+        n = gemma_attn_prefill_workspace_size(B, S, Hq, Hkv, D, 0)
+        workspace = torch.empty(max(n, 1), dtype=torch.uint8, device=q.device)
+    return _check(_prefill_paged(_ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_pool), _ptr(v_pool), _ptr(page_table),
+                                 ps, pps, n_pages, _ptr(seq_lens_before), B, S, Hq, Hkv, D, rope_frac, rope_theta,
+                                 scale, _ptr(out), _ptr(lse), _ptr(workspace), workspace.numel(), flags,
+                                 _stream(stream)))
+
+
+def gemma_attn_decode_paged(q, k_new, v_new, k_pool, v_pool, page_table, *, seq_lens, max_seq_len, rope_frac,
+                            rope_theta, scale, out, workspace=None, flags=0, stream=None):
+    """Global-layer decode on a paged cache (see gemma_attn_prefill_paged)."""
+    for t, n in ((q, "q"), (k_new, "k_new"), (v_new, "v_new"), (k_pool, "k_pool"), (v_pool, "v_pool"),
+                 (out, "out")):
+        _bf16(t, n)
+    if seq_lens.dtype != torch.int32 or not seq_lens.is_cuda:
+        raise TypeError("seq_lens must be an int32 CUDA tensor")
+    B, Hq, D = q.shape
+    n_pages, Hkv, ps, pps = _paged_args(k_pool, page_table)
+    if workspace is None:
+        n = gemma_attn_decode_workspace_size(B, Hq, Hkv, D, 0, max_seq_len)
+        workspace = torch.empty(max(n, 1), dtype=torch.uint8, device=q.device)
+    return _check(_decode_paged(_ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_pool), _ptr(v_pool), _ptr(page_table),
+                                ps, pps, n_pages, _ptr(seq_lens), max_seq_len, B, Hq, Hkv, D, rope_frac,
+                                rope_theta, scale, _ptr(out), _ptr(workspace), workspace.numel(), flags,
+                                _stream(stream)))
 
 
 def gemma_kv_share_bind(dst: gemma_kv_desc, src: gemma_kv_desc) -> int:

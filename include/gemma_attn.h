@@ -177,6 +177,42 @@ int gemma_attn_decode(const void* q, const void* k_new, const void* v_new,
                       void* stream);
 
 /* ---------------------------------------------------------------------- */
+/* Paged global cache ("Gemma 4: End-to-End Architecture Walkthrough", 3b: */
+/* a global layer caches K/V for the whole context; paging lets the pool   */
+/* grow with the tokens actually held instead of a per-sequence capacity). */
+/* Global layers only (window 0); same arguments and behaviour as          */
+/* gemma_attn_prefill / gemma_attn_decode except the cache:                */
+/* k_pool, v_pool  [n_pages][n_kv_heads][page_size][head_dim] bf16: pages  */
+/*        of page_size consecutive positions of one sequence.             */
+/* page_table device int32 [batch][pages_per_seq]: position p of sequence */
+/*        b is row p % page_size of page page_table[b][p / page_size].    */
+/*        Entries for every page a call reads or writes (positions below  */
+/*        seq_lens_before + s_new, or below seq_lens) must name a page of  */
+/*        the pool; a device-side check reports any other as              */
+/*        GEMMA_ERR_DEVICE_RANGE (nothing is written for it). Shared      */
+/*        layers pass their source's pool and table. The caller owns the  */
+/*        pool, the table and page allocation.                            */
+/* page_size: a multiple of 128. pages_per_seq * page_size is the         */
+/*        per-sequence capacity (the bound on seq_lens). GEMMA_F_KV_INT8   */
+/*        returns GEMMA_ERR_UNSUPPORTED.                                  */
+/* ---------------------------------------------------------------------- */
+int gemma_attn_prefill_paged(const void* q, const void* k_new, const void* v_new,
+                             void* k_pool, void* v_pool, const int32_t* page_table,
+                             int page_size, int pages_per_seq, int n_pages,
+                             const int32_t* seq_lens_before, int batch, int s_new,
+                             int n_q_heads, int n_kv_heads, int head_dim, float rope_frac,
+                             float rope_theta, float scale, void* out, float* lse,
+                             void* workspace, size_t workspace_bytes, unsigned flags,
+                             void* stream);
+int gemma_attn_decode_paged(const void* q, const void* k_new, const void* v_new,
+                            void* k_pool, void* v_pool, const int32_t* page_table,
+                            int page_size, int pages_per_seq, int n_pages,
+                            const int32_t* seq_lens, int max_seq_len, int batch,
+                            int n_q_heads, int n_kv_heads, int head_dim, float rope_frac,
+                            float rope_theta, float scale, void* out, void* workspace,
+                            size_t workspace_bytes, unsigned flags, void* stream);
+
+/* ---------------------------------------------------------------------- */
 /* Decode without allocation. The pages have no counterpart for this entry */
 /* point; it exists for callers that cannot obtain device memory for the  */
 /* decode workspace -- e.g. a plugin inside a host runtime that owns all  */

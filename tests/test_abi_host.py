@@ -204,3 +204,52 @@ def test_kv_cache_bytes():
     assert native.gemma_kv_cache_bytes(1, 3, 2, 16, native.GEMMA_F_KV_INT8) == 256 + 6 * 8
     assert native.gemma_kv_cache_bytes(0, 4, 4096, 512) == 0
     assert native.gemma_kv_codes_bytes(1, 1, 0, 256) == 0
+
+
+def _prefill_paged_raw(**over):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, kc=FAKE, vc=FAKE, table=FAKE, ps=128, pps=64, npages=256, lens=None, B=2,
+             S=16, Hq=8, Hkv=1, D=512, frac=0.25, theta=1e6, scale=0.044, out=FAKE, lse=None, ws=FAKE,
+             wsb=1 << 30, flags=0)
+    a.update(over)
+    return native._prefill_paged(a["q"], a["k"], a["v"], a["kc"], a["vc"], a["table"], a["ps"], a["pps"],
+                                 a["npages"], a["lens"], a["B"], a["S"], a["Hq"], a["Hkv"], a["D"], a["frac"],
+                                 a["theta"], a["scale"], a["out"], a["lse"], a["ws"], a["wsb"], a["flags"], None)
+
+
+def _decode_paged_raw(**over):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, kc=FAKE, vc=FAKE, table=FAKE, ps=256, pps=32, npages=64, lens=FAKE,
+             maxlen=4096, B=2, Hq=32, Hkv=4, D=512, frac=0.25, theta=1e6, scale=0.044, out=FAKE, ws=FAKE,
+             wsb=1 << 30, flags=0)
+    a.update(over)
+    return native._decode_paged(a["q"], a["k"], a["v"], a["kc"], a["vc"], a["table"], a["ps"], a["pps"],
+                                a["npages"], a["lens"], a["maxlen"], a["B"], a["Hq"], a["Hkv"], a["D"], a["frac"],
+                                a["theta"], a["scale"], a["out"], a["ws"], a["wsb"], a["flags"], None)
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(wsb=16), E.GEMMA_ERR_CAPACITY),                  # accepted
+    (dict(table=None), E.GEMMA_ERR_INVALID_ARG),
+    (dict(ps=100), E.GEMMA_ERR_INVALID_ARG),               # not a multiple of 128
+    (dict(ps=0), E.GEMMA_ERR_INVALID_ARG),
+    (dict(pps=0), E.GEMMA_ERR_INVALID_ARG),
+    (dict(npages=0), E.GEMMA_ERR_INVALID_ARG),
+    (dict(flags=4), E.GEMMA_ERR_UNSUPPORTED),              # int8 rows are not paged
+    (dict(pps=1, S=200), E.GEMMA_ERR_CAPACITY),            # chunk beyond pages_per_seq * page_size
+    (dict(flags=2, v=None, vc=None, wsb=16), E.GEMMA_ERR_CAPACITY),   # K = V accepted
+])
+def test_prefill_paged_validation(over, code):
+    assert _prefill_paged_raw(**over) == code
+    assert native.gemma_last_error()
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(wsb=1024), E.GEMMA_ERR_CAPACITY),                # accepted
+    (dict(table=None), E.GEMMA_ERR_INVALID_ARG),
+    (dict(ps=192), E.GEMMA_ERR_INVALID_ARG),
+    (dict(flags=4), E.GEMMA_ERR_UNSUPPORTED),
+    (dict(pps=8), E.GEMMA_ERR_CAPACITY),                   # 8 pages of 256 < max_seq_len 4096
+    (dict(flags=1, k=None, v=None, wsb=1024), E.GEMMA_ERR_CAPACITY),  # shared layer accepted
+])
+def test_decode_paged_validation(over, code):
+    assert _decode_paged_raw(**over) == code
+    assert native.gemma_last_error()
