@@ -13,18 +13,22 @@
 // scalar per head (O).
 //
 // Per CTA = (split, KV head, sequence), 128 threads, two CTAs per SM:
-//   warp 3      producer: per 16-key sub-block, one bulk copy per pair of
-//               consecutive K (or V) code rows (contiguous in the cache) into
-//               padded row pairs of a ring slot, plus one copy each of the K
-//               and V (min, step) rows.
+//   warp 3      producer: per 16-key sub-block, the K and the V code rows
+//               arrive as TMA tiles of 16 rows x 128 bytes (one per 128-byte
+//               column chunk), 128-byte swizzled, plus one bulk copy each of
+//               the K and V (min, step) rows: 6 copies (head_dim 256) or 10
+//               (head_dim 512) per 16 keys. The copy engine takes about one
+//               copy per 44 cycles per SM, so copies of one or two rows
+//               would bound the stream well below HBM.
 //   warps 0..2  consumers: sub-block t goes to warp t % 3 (and ring slot
 //               t % NSLOT). The MMA fragments (mma.sync m16n8k16, fp16) come
 //               straight from the code rows: a byte permute puts a code in
 //               the mantissa of fp16 1024.0 and subtracting 1024 leaves it
 //               exactly. The k positions of S and the output rows of P.V
 //               stand for dims in an order that makes each lane's codes 16
-//               contiguous bytes, and a fixed key order (key_at) spreads the
-//               rows a quarter warp reads over different banks.
+//               contiguous bytes, and a fixed key order (key_at) puts the
+//               rows a quarter warp reads on swizzle phases that land its
+//               eight 16-byte reads on disjoint banks.
 // Every barrier wait is bounded (%globaltimer deadline); on a timeout the CTA
 // raises its abort flag, records GEMMA_ERR_DEVICE_TIMEOUT, waits (bounded)
 // for its own copies in flight, and exits without output.
@@ -33,6 +37,8 @@
 #include "common.cuh"
 #include "kernels.h"
 #include "mma_sync.cuh"
+#include "tc.cuh"
+#include "tmap.h"
 
 namespace hlg {
 
@@ -45,43 +51,56 @@ constexpr int NCW = 3;  // consumer warps
 template <int D>
 struct Q8Cfg {
   static constexpr int KB = 16;                      // keys per sub-block
-  static constexpr int PAIRB = 2 * D + 16;           // two consecutive code rows + 16 B pad
-  static constexpr int REGION_B = (KB / 2) * PAIRB;  // 16 code rows as 8 padded pairs
-  static constexpr int PAR_OFF = 2 * REGION_B;       // K region, V region (K = V: 32 K rows), then
-  static constexpr int RAW_B = PAR_OFF + 2 * KB * 8; // K (min, step) [16], V [16] (K = V: 32 K)
-  static constexpr int NSLOT = 6;
+  static constexpr int NCH = D / 128;                // 128-byte column chunks of a code row
+  static constexpr int BOX_B = KB * 128;             // one TMA tile: 16 rows x 128 bytes
+  static constexpr int REGION_B = NCH * BOX_B;       // 16 code rows, chunk-major, swizzled
+  static constexpr int SLOT_B = 2 * REGION_B;        // K region, V region (K = V: 32 K rows)
+  static constexpr int NSLOT = D == 512 ? 6 : 12;
   static_assert(NSLOT % NCW == 0, "each ring slot needs a single consumer warp");
+  static constexpr int RING_B = NSLOT * SLOT_B;
+  static constexpr int PAR_B = 2 * KB * 8;           // K (min, step) [16], V [16] (K = V: 32 K)
+  static constexpr int PAR_OFF = RING_B;
   static constexpr int ROW = D + 8;                  // fp16 Q row (elements), 16 B pad
-  static constexpr int RING_B = NSLOT * RAW_B;
-  static constexpr int Q_OFF = RING_B;
+  static constexpr int Q_OFF = PAR_OFF + NSLOT * PAR_B;
   static constexpr int Q_B = 8 * ROW * 2;
   static constexpr int QSUM_OFF = Q_OFF + Q_B;       // float [8] sum of each head's staged q
   static constexpr int BAR_OFF = QSUM_OFF + 64;
   static constexpr int MISC_OFF = BAR_OFF + 2 * NSLOT * 8;
-  static constexpr int SMEM = MISC_OFF + (4 + 2 * NSLOT + 64) * 4;
+  static constexpr int ALIGN_B = 1024;               // 128-byte swizzle: tiles on 1024-byte boundaries
+  static constexpr int SMEM = ALIGN_B + MISC_OFF + (4 + 2 * NSLOT + 64) * 4;
   static constexpr int OSTR = D + 4;                 // merge-buffer row (floats)
   static constexpr int MERGE_B = NCW * 8 * OSTR * 4;
   static_assert(MERGE_B <= RING_B, "merge buffer must fit in the drained ring");
-  static_assert(PAIRB % 16 == 0 && RAW_B % 16 == 0 && Q_OFF % 16 == 0, "16-byte alignment");
-  static_assert(2 * SMEM <= 227 * 1024, "two CTAs per SM");
-  static constexpr int VCH = D / 128;                // 16-dim chunks of V per lane (D/8 dims per lane)
+  static_assert(BOX_B % 1024 == 0 && SLOT_B % 1024 == 0 && Q_OFF % 16 == 0, "alignment");
+  static_assert(2 * (SMEM + 1024) <= 228 * 1024, "two CTAs per SM");
+  static constexpr int VCH = D / 128;                // 16-byte units of V codes per lane and key row
+  static constexpr int PPL = 4 / VCH;                // lane pairs per 128-byte line (P.V reads)
 };
 
-// Byte offset of code row r (0..31) in a slot: rows go in padded pairs.
-template <int D>
-__device__ __forceinline__ int code_row_off(int r) {
-  return (r >> 1) * Q8Cfg<D>::PAIRB + (r & 1) * D;
+// The key (0..15 within a 16-key half) that MMA column / P.V index j stands
+// for: j = 8a + 2t + e holds row t + 4e + 8a. The S fragments read rows
+// key_at(2i) and key_at(2i + 1) with the 8 lanes of a quarter warp, whose
+// swizzle phases (row mod 8) then differ in bit 2; the P.V fragments read
+// rows key_at(2t + s), t = 0..3, whose phases differ mod 4. With the
+// 16-byte units each lane reads (code_unit, pv_off) every quarter warp
+// touches eight distinct units of a 128-byte line: no bank conflicts.
+__device__ __forceinline__ int key_at(int j) { return ((j >> 1) & 3) | ((j & 1) << 2) | (j & 8); }
+
+// Byte address, within a region, of the 16-byte unit `u` (0..7) of 128-byte
+// chunk `ch` of code row `r`: TMA's 128-byte swizzle XORs the unit with the
+// row's line index mod 8 (each tile is 16 lines of 128 bytes).
+__device__ __forceinline__ int code_unit(int ch, int r, int u) {
+  return ch * (16 * 128) + r * 128 + ((u ^ (r & 7)) << 4);
 }
 
-// The key (0..15 within a 16-key half) that MMA column / P.V index j stands
-// for. The S fragments read rows key_at(gq) and key_at(8 + gq) with the 8
-// lanes of a quarter warp on two of them, the P.V fragments rows key_at(2tg)
-// .. key_at(9 + 2tg) with four lanes on four rows; this order puts each such
-// set of rows in row pairs whose 16-byte pads shift them onto disjoint banks
-// (head_dim 512; head_dim 256 keeps a 2-way overlap on the P.V side).
-__device__ __forceinline__ int key_at(int j) {
-  const int q = (j & 7) >> 1;
-  return (j & 8) ? ((j & 1) ? 9 + 2 * q : 2 * q + 1) : ((j & 1) ? 8 + 2 * q : 2 * q);
+// Dim (= byte offset in a code row) of the first of the 16 codes lane group
+// gq reads for P.V unit c (0..VCH-1). Lanes 2p and 2p + 1 take units u and
+// u ^ 4 of one 128-byte line; every dim is covered once.
+template <int D>
+__host__ __device__ __forceinline__ int pv_off(int gq, int c) {
+  using C = Q8Cfg<D>;
+  const int p = gq >> 1, h = gq & 1;
+  return (p / C::PPL) * 128 + 16 * (4 * h + C::VCH * (p % C::PPL) + c);
 }
 
 // Two codes (bytes `sel` picks) -> fp16x2 (1024 + c, 1024 + c'), exactly:
@@ -104,10 +123,15 @@ __device__ __forceinline__ float pow2_ceil(float x) {
 }
 
 template <int D>
-__global__ void __launch_bounds__(32 * (NCW + 1), 2) k_decode_split_q8(DecodeAttnArgs a) {
+__global__ void __launch_bounds__(32 * (NCW + 1), 2)
+    k_decode_split_q8(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                      DecodeAttnArgs a) {
   using C = Q8Cfg<D>;
-  extern __shared__ __align__(128) unsigned char sm[];
+  extern __shared__ __align__(128) unsigned char sm_raw[];
+  const uint32_t raw_u32 = smem_u32(sm_raw);
+  unsigned char* sm = sm_raw + (((raw_u32 + C::ALIGN_B - 1) & ~uint32_t(C::ALIGN_B - 1)) - raw_u32);
   unsigned char* ring = sm;
+  unsigned char* pring = sm + C::PAR_OFF;
   __half* qs = reinterpret_cast<__half*>(sm + C::Q_OFF);
   float* qsum = reinterpret_cast<float*>(sm + C::QSUM_OFF);
   uint64_t* full = reinterpret_cast<uint64_t*>(sm + C::BAR_OFF);
@@ -136,8 +160,6 @@ __global__ void __launch_bounds__(32 * (NCW + 1), 2) k_decode_split_q8(DecodeAtt
   const int kps = a.keqv ? 2 * C::KB : C::KB;
   const int n_sub = (int)((k_end - k_begin + kps - 1) / kps);
   const int64_t row0 = ((int64_t)b * a.Hkv + g) * (int64_t)a.cache_cap;  // first cache row of (b, g)
-  const uint8_t* kcode = a.k_codes + row0 * D;
-  const uint8_t* vcode = a.v_codes + row0 * D;
   const float2* kpar = a.k_params + row0;
   const float2* vpar = a.keqv ? kpar : a.v_params + row0;
 
@@ -156,44 +178,41 @@ __global__ void __launch_bounds__(32 * (NCW + 1), 2) k_decode_split_q8(DecodeAtt
 
   if (warp == NCW) {
     // ---------------- producer ----------------
-    for (int t = 0; t < n_sub; ++t) {
-      const int slot = t % C::NSLOT;
-      bool ok = true;
-      if (lane == 0) {
-        if (t >= C::NSLOT)
-          ok = mbar_wait_bounded_at(&empty[slot], ((t / C::NSLOT) - 1) & 1, abort_flag, deadline,
-                                    a.status, 1, t, slot, n_sub);
-        if (ok && *abort_flag) ok = false;
-      }
-      ok = __shfl_sync(0xffffffffu, ok, 0);
-      if (!ok) break;
-      const int64_t key0 = k_begin + (int64_t)t * kps;
-      const int nk = (int)((k_end - key0) < kps ? (k_end - key0) : kps);
-      // (min, step) rows go in pairs (16-byte copies): key0 is a multiple of 16
-      // and the cache capacity is even, so the pair of an odd last row exists
-      const int np = (nk + 1) & ~1;
-      const bool drop = a.drop_first_copy && t == 0 && split == 0 && g == 0 && b == 0;
-      if (drop) continue;
-      unsigned char* dst = ring + slot * C::RAW_B;
-      if (lane == 0) {
-        const uint32_t bytes = a.keqv ? (uint32_t)(nk * D + np * 8) : (uint32_t)(2 * (nk * D + np * 8));
+    if (lane == 0) {
+      tc::prefetch_tmap(&tm_k);
+      tc::prefetch_tmap(&tm_v);
+      for (int t = 0; t < n_sub; ++t) {
+        const int slot = t % C::NSLOT;
+        if (t >= C::NSLOT &&
+            !mbar_wait_bounded_at(&empty[slot], ((t / C::NSLOT) - 1) & 1, abort_flag, deadline, a.status, 1, t,
+                                  slot, n_sub))
+          break;
+        if (*abort_flag) break;
+        const int64_t key0 = k_begin + (int64_t)t * kps;
+        const int nk = (int)((k_end - key0) < kps ? (k_end - key0) : kps);
+        // (min, step) rows go in pairs (16-byte copies): key0 is a multiple of 16
+        // and the cache capacity is even, so the pair of an odd last row exists
+        const int np = (nk + 1) & ~1;
+        const bool drop = a.drop_first_copy && t == 0 && split == 0 && g == 0 && b == 0;
+        if (drop) continue;
+        // regions that hold rows: K and V, or (K = V) the first 16 K rows and,
+        // when there are more, the next 16
+        const int n_reg = a.keqv ? (nk > C::KB ? 2 : 1) : 2;
+        const uint32_t bytes = (uint32_t)(n_reg * C::REGION_B) + (uint32_t)((a.keqv ? 1 : 2) * np * 8);
         mbar_arrive_expect_tx(&full[slot], bytes);
         issued[slot] += 1;
-      }
-      __syncwarp();
-      // lanes 0..7: K row pairs, 8..15: V row pairs (K = V: lanes 0..15, the
-      // 16 pairs of 32 K rows); lanes 16, 17: the (min, step) rows
-      if (lane < 16) {
-        const bool isv = !a.keqv && lane >= 8;
-        const int pr = a.keqv ? lane : (lane & 7);
-        const int left = nk - 2 * pr;
-        if (left > 0)
-          bulk_g2s(dst + (isv ? C::REGION_B : 0) + pr * C::PAIRB, (isv ? vcode : kcode) + (key0 + 2 * pr) * D,
-                   (uint32_t)((left >= 2 ? 2 : 1) * D), &full[slot]);
-      } else if (lane == 16) {
-        bulk_g2s(dst + C::PAR_OFF, kpar + key0, (uint32_t)(np * 8), &full[slot]);
-      } else if (lane == 17 && !a.keqv) {
-        bulk_g2s(dst + C::PAR_OFF + C::KB * 8, vpar + key0, (uint32_t)(np * 8), &full[slot]);
+        const uint32_t dst = smem_u32(ring + slot * C::SLOT_B);
+        const uint32_t bar = smem_u32(&full[slot]);
+        for (int r = 0; r < n_reg; ++r) {
+          const CUtensorMap* m = (a.keqv || r == 0) ? &tm_k : &tm_v;
+          const int y = (int)key0 + (a.keqv ? r * C::KB : 0);  // rows past the capacity read as 0
+#pragma unroll
+          for (int ch = 0; ch < C::NCH; ++ch)
+            tc::tma_load_4d(dst + r * C::REGION_B + ch * C::BOX_B, m, ch * 128, y, g, b, bar);
+        }
+        unsigned char* pdst = pring + slot * C::PAR_B;
+        bulk_g2s(pdst, kpar + key0, (uint32_t)(np * 8), &full[slot]);
+        if (!a.keqv) bulk_g2s(pdst + C::KB * 8, vpar + key0, (uint32_t)(np * 8), &full[slot]);
       }
     }
   } else {
@@ -273,11 +292,17 @@ __global__ void __launch_bounds__(32 * (NCW + 1), 2) k_decode_split_q8(DecodeAtt
     int key_l[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) key_l[i] = key_at(i < 2 ? 2 * tg + i : 8 + 2 * tg + (i - 2));
-    const int kro_a = code_row_off<D>(key_at(gq)) + 16 * tg;       // S rows: n-tile 0
-    const int kro_b = code_row_off<D>(key_at(8 + gq)) + 16 * tg;   // n-tile 1
-    int vro[4];
+    // S rows (n-tile 0: key_at(gq), n-tile 1: key_at(8 + gq)): 64-dim group
+    // 2 ch + hb of a row is units 4 hb + tg of chunk ch
+    const int ra = key_at(gq), rb = key_at(8 + gq);
+    const int ka_lo = code_unit(0, ra, tg), ka_hi = code_unit(0, ra, 4 + tg);
+    const int kb_lo = code_unit(0, rb, tg), kb_hi = code_unit(0, rb, 4 + tg);
+    // P.V rows key_l[i]: units pv_off(gq, c) of each
+    const int pv0 = pv_off<D>(gq, 0);
+    int vrow[4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) vro[i] = code_row_off<D>(key_l[i]) + (D / 8) * gq;
+    for (int i = 0; i < 4; ++i) vrow[i] = (pv0 >> 7) * C::BOX_B + key_l[i] * 128;
+    const int pv_u = (pv0 >> 4) & 7;  // unit of c = 0; unit c is pv_u + c
 
     for (int t = warp; t < n_sub; t += NCW) {
       const int slot = t % C::NSLOT;
@@ -286,8 +311,8 @@ __global__ void __launch_bounds__(32 * (NCW + 1), 2) k_decode_split_q8(DecodeAtt
       if (!__all_sync(0xffffffffu, ok)) break;
       const int64_t key0_slot = k_begin + (int64_t)t * kps;
       const int nk_slot = (int)((k_end - key0_slot) < kps ? (k_end - key0_slot) : kps);
-      const unsigned char* raw = ring + slot * C::RAW_B;
-      const float2* praw = reinterpret_cast<const float2*>(raw + C::PAR_OFF);  // K [16], V [16] (K = V: 32 K)
+      const unsigned char* raw = ring + slot * C::SLOT_B;
+      const float2* praw = reinterpret_cast<const float2*>(pring + slot * C::PAR_B);  // K [16], V [16] (K = V: 32 K)
       for (int half = 0; half < (a.keqv ? 2 : 1); ++half) {
         const int nk = nk_slot - half * C::KB;
         if (nk <= 0) break;
@@ -308,8 +333,9 @@ __global__ void __launch_bounds__(32 * (NCW + 1), 2) k_decode_split_q8(DecodeAtt
         for (int grp = 0; grp < D / 64; ++grp) {
           const uint4 qa = *reinterpret_cast<const uint4*>(q_row + grp * 128);
           const uint4 qb = *reinterpret_cast<const uint4*>(q_row + grp * 128 + 16);
-          const uint4 ka = *reinterpret_cast<const uint4*>(kreg + kro_a + grp * 64);
-          const uint4 kb = *reinterpret_cast<const uint4*>(kreg + kro_b + grp * 64);
+          const unsigned char* kch = kreg + (grp >> 1) * C::BOX_B;
+          const uint4 ka = *reinterpret_cast<const uint4*>(kch + ((grp & 1) ? ka_hi : ka_lo));
+          const uint4 kb = *reinterpret_cast<const uint4*>(kch + ((grp & 1) ? kb_hi : kb_lo));
           const uint32_t qw[8] = {qa.x, qa.y, qa.z, qa.w, qb.x, qb.y, qb.z, qb.w};
           const uint32_t kwa[4] = {ka.x, ka.y, ka.z, ka.w}, kwb[4] = {kb.x, kb.y, kb.z, kb.w};
 #pragma unroll
@@ -365,10 +391,10 @@ __global__ void __launch_bounds__(32 * (NCW + 1), 2) k_decode_split_q8(DecodeAtt
         // O'^T += C_V^T P'^T : rows = head dims, cols = query heads, k = 16 keys
 #pragma unroll
         for (int c = 0; c < C::VCH; ++c) {
-          const uint4 r0 = *reinterpret_cast<const uint4*>(vreg + vro[0] + 16 * c);
-          const uint4 r1 = *reinterpret_cast<const uint4*>(vreg + vro[1] + 16 * c);
-          const uint4 r2 = *reinterpret_cast<const uint4*>(vreg + vro[2] + 16 * c);
-          const uint4 r3 = *reinterpret_cast<const uint4*>(vreg + vro[3] + 16 * c);
+          const uint4 r0 = *reinterpret_cast<const uint4*>(vreg + vrow[0] + (((pv_u + c) ^ (key_l[0] & 7)) << 4));
+          const uint4 r1 = *reinterpret_cast<const uint4*>(vreg + vrow[1] + (((pv_u + c) ^ (key_l[1] & 7)) << 4));
+          const uint4 r2 = *reinterpret_cast<const uint4*>(vreg + vrow[2] + (((pv_u + c) ^ (key_l[2] & 7)) << 4));
+          const uint4 r3 = *reinterpret_cast<const uint4*>(vreg + vrow[3] + (((pv_u + c) ^ (key_l[3] & 7)) << 4));
           const uint32_t w0[4] = {r0.x, r0.y, r0.z, r0.w}, w1[4] = {r1.x, r1.y, r1.z, r1.w};
           const uint32_t w2[4] = {r2.x, r2.y, r2.z, r2.w}, w3[4] = {r3.x, r3.y, r3.z, r3.w};
 #pragma unroll
@@ -420,7 +446,7 @@ __global__ void __launch_bounds__(32 * (NCW + 1), 2) k_decode_split_q8(DecodeAtt
     }
 #pragma unroll
     for (int mt = 0; mt < D / 16; ++mt) {
-      const int dim = (D / 8) * gq + 16 * (mt / 8) + 2 * (mt % 8);  // row gq of m-tile mt; row gq+8 is dim+1
+      const int dim = pv_off<D>(gq, mt / 8) + 2 * (mt % 8);  // row gq of m-tile mt; row gq+8 is dim+1
       float* row0 = obuf + (warp * 8 + 2 * tg) * C::OSTR + dim;
       float* row1 = row0 + C::OSTR;
       row0[0] = (o[mt][0] * fv + c0) * f[0];
@@ -465,9 +491,20 @@ __global__ void __launch_bounds__(32 * (NCW + 1), 2) k_decode_split_q8(DecodeAtt
 template <int D>
 cudaError_t launch_q8(const DecodeAttnArgs& a, int B, cudaStream_t st) {
   using C = Q8Cfg<D>;
+  // codes [B][Hkv][cap][D] bytes as 4-D maps (dims innermost first), tiles of
+  // 128 bytes x 16 rows
+  CUtensorMap mk, mv;
+  const uint64_t dims[4] = {(uint64_t)D, (uint64_t)a.cache_cap, (uint64_t)a.Hkv, (uint64_t)B};
+  const uint64_t str[3] = {(uint64_t)D, (uint64_t)a.cache_cap * D, (uint64_t)a.Hkv * a.cache_cap * D};
+  const uint32_t box[4] = {128, (uint32_t)C::KB, 1, 1};
+  if (!make_map_u8_4d(&mk, a.k_codes, dims, str, box)) return cudaErrorInvalidValue;
+  if (a.keqv)
+    mv = mk;
+  else if (!make_map_u8_4d(&mv, a.v_codes, dims, str, box))
+    return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(k_decode_split_q8<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
-  k_decode_split_q8<D><<<dim3(a.n_splits, a.Hkv, B), 32 * (NCW + 1), C::SMEM, st>>>(a);
+  k_decode_split_q8<D><<<dim3(a.n_splits, a.Hkv, B), 32 * (NCW + 1), C::SMEM, st>>>(mk, mv, a);
   return cudaGetLastError();
 }
 

@@ -1,4 +1,4 @@
-// tmap.cu -- host-side TMA tensor maps for the prefill kernels.
+// tmap.cu -- host-side TMA tensor maps (prefill attention, int8 decode).
 #include <cudaTypedefs.h>
 
 #include <mutex>
@@ -22,20 +22,30 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-}  // namespace
-
-bool make_map_bf16_4d(CUtensorMap* m, const void* ptr, const uint64_t dims[4], const uint64_t strides[3],
-                      const uint32_t box[4]) {
+bool make_map_4d(CUtensorMap* m, CUtensorMapDataType type, const void* ptr, const uint64_t dims[4],
+                 const uint64_t strides[3], const uint32_t box[4]) {
   auto fn = encode_fn();
   if (!fn) return false;
   cuuint64_t gd[4] = {dims[0], dims[1], dims[2], dims[3]};
   cuuint64_t gs[3] = {strides[0], strides[1], strides[2]};
   cuuint32_t bx[4] = {box[0], box[1], box[2], box[3]};
   cuuint32_t es[4] = {1, 1, 1, 1};
-  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), gd, gs, bx, es,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  CUresult r = fn(m, type, 4, const_cast<void*>(ptr), gd, gs, bx, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+bool make_map_bf16_4d(CUtensorMap* m, const void* ptr, const uint64_t dims[4], const uint64_t strides[3],
+                      const uint32_t box[4]) {
+  return make_map_4d(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, ptr, dims, strides, box);
+}
+
+bool make_map_u8_4d(CUtensorMap* m, const void* ptr, const uint64_t dims[4], const uint64_t strides[3],
+                    const uint32_t box[4]) {
+  return make_map_4d(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, ptr, dims, strides, box);
 }
 
 bool make_prefill_maps(const PrefillAttnArgs& a, int B, int D, int key_rows_total, int kv_token_major,

@@ -1,4 +1,4 @@
-// tmap.h -- host-side TMA tensor maps for the prefill kernels.
+// tmap.h -- host-side TMA tensor maps (prefill attention, int8 decode).
 #pragma once
 
 #include <cuda.h>
@@ -13,6 +13,9 @@ namespace hlg {
 // the driver entry point is missing or rejects the layout.
 bool make_map_bf16_4d(CUtensorMap* m, const void* ptr, const uint64_t dims[4], const uint64_t strides[3],
                       const uint32_t box[4]);
+// The same for a uint8 tensor (int8 KV codes); box[0] <= 128 bytes.
+bool make_map_u8_4d(CUtensorMap* m, const void* ptr, const uint64_t dims[4], const uint64_t strides[3],
+                    const uint32_t box[4]);
 
 // The four maps of one prefill attention launch:
 //   q, o  [B][S][Hq][D], box 64 dims x 1 head x q_rows x 1;
