@@ -367,12 +367,18 @@ def bench_decode(args, w, dev, world, peaks):
                           "(%d launches, %d per step)" % (sp["launches"], st.n_layers)}
     rec = recorded_traffic("k_decode_split_q8" if w.kv_int8 else "k_decode_split")
     if rec:
-        r = next(iter(rec.values()))
-        ratio = float(r["bytes"]) / float(r["units"])
-        roof["traffic"] = round(ratio * kv_bytes / st.n_layers)
-        roof["traffic_note"] = ("DRAM bytes per split launch: visible K+V bytes per launch x %.4f, the "
-                                "traffic/algorithmic ratio of the ncu capture of %s (%s; this block is too "
-                                "large to capture)" % (ratio, r["workload"], r["file"]))
+        # each layer takes the traffic/algorithmic ratio captured for its layer
+        # type (or the other type's, when only one was captured)
+        ratio = {k: float(r["bytes"]) / float(r["units"]) for k, r in rec.items()}
+        any_ratio = next(iter(ratio.values()))
+        per_layer = [ratio.get("global" if st.layer_type(l).window == 0 else "local", any_ratio)
+                     * visible_kv_bytes(st, l, lens_cpu) for l in range(st.n_layers)]
+        roof["traffic"] = round(sum(per_layer) / st.n_layers)
+        roof["traffic_note"] = ("DRAM bytes per split launch: each layer's visible K+V bytes x the "
+                                "traffic/algorithmic ratio of the ncu capture for its layer type (%s), mean "
+                                "over the block's launches; this block is too large to capture"
+                                % ", ".join("%s %.4f: %s in %s" % (k, ratio[k], rec[k]["workload"], rec[k]["file"])
+                                            for k in sorted(rec)))
     else:
         roof["traffic_note"] = "no ncu capture of the current kernel sources"
     res = {"metric": "decode KV GB/s", "value": round(value, 1), "unit": "GB/s",
