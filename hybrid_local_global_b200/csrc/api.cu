@@ -187,11 +187,15 @@ size_t decode_ws_parts(int B, int Hq, int Hkv, int D, int n_splits, size_t* off_
 // of the chunk (K at off_k) or, for a chunk after cached tokens, the K and V
 // windows of window + S rows (K at off_k, V at *off_vw).
 size_t prefill_ws_parts(int B, int S, int Hq, int Hkv, int D, int window, size_t* off_k,
-                        size_t* off_vw = nullptr) {
+                        size_t* off_vw = nullptr, int prefix_rows = 0) {
   size_t q = align256((size_t)B * S * Hq * D * 2);
   // rotated K of the chunk: local layers, and global layers with an int8 cache
   size_t k = align256((size_t)B * S * Hkv * D * 2);
-  size_t win = window > 0 ? align256((size_t)B * (window + S) * Hkv * D * 2) : 0;
+  // K and V windows: chunked local prefill (window + S rows), or the
+  // dequantized prefix plus chunk of an int8 global layer (prefix_rows rows)
+  size_t win = window > 0     ? align256((size_t)B * (window + S) * Hkv * D * 2)
+               : prefix_rows ? align256((size_t)B * prefix_rows * Hkv * D * 2)
+                             : 0;
   *off_k = q;
   if (off_vw) *off_vw = q + win;
   return q + std::max(k, 2 * win);
@@ -304,11 +308,16 @@ size_t gemma_kv_cache_bytes(int batch, int n_kv_heads, int cache_cap, int head_d
 
 // int8 cache rows of one call's new tokens: K from the rotated staging rows,
 // V from the caller's values (none under K = V)
-static cudaError_t quantize_kv(const bf16* k_src, const bf16* v_src, void* k_cache, void* v_cache, int batch,
-                               int S, int Hkv, int D, int window, int cache_cap, const int32_t* pos0,
-                               int pos0_minus, int* status, cudaStream_t st) {
+// Quantize a chunk's rows into an int8 cache. Sources are [B][rows][Hkv][D]
+// with chunk token s at row s (mode 0), window + s (1) or its position (2);
+// V from the caller's layout [B][S][Hkv][D] (null under K = V).
+static cudaError_t quantize_kv(const bf16* k_src, int k_rows, int k_mode, const bf16* v_src, void* k_cache,
+                               void* v_cache, int batch, int S, int Hkv, int D, int window, int cache_cap,
+                               const int32_t* pos0, int pos0_minus, int* status, cudaStream_t st) {
   const size_t off = gemma_kv_codes_bytes(batch, Hkv, cache_cap, D);
   QuantRowsArgs qa{};
+  qa.src_rows = k_rows;
+  qa.src_row_mode = k_mode;
   qa.S = S;
   qa.Hkv = Hkv;
   qa.window = window;
@@ -322,6 +331,8 @@ static cudaError_t quantize_kv(const bf16* k_src, const bf16* v_src, void* k_cac
   cudaError_t e = launch_quantize_rows(qa, batch, D, st);
   if (e != cudaSuccess || !v_src) return e;
   qa.src = v_src;
+  qa.src_rows = S;
+  qa.src_row_mode = 0;
   qa.codes = static_cast<uint8_t*>(v_cache);
   qa.params = reinterpret_cast<float2*>(static_cast<uint8_t*>(v_cache) + off);
   return launch_quantize_rows(qa, batch, D, st);
@@ -332,6 +343,16 @@ size_t gemma_attn_prefill_workspace_size(int batch, int s_new, int n_q_heads, in
   if (batch <= 0 || s_new <= 0 || n_q_heads <= 0 || n_kv_heads <= 0 || head_dim <= 0) return 0;
   size_t off_k;
   return prefill_ws_parts(batch, s_new, n_q_heads, n_kv_heads, head_dim, window, &off_k);
+}
+
+size_t gemma_attn_prefill_workspace_size_cached(int batch, int s_new, int n_q_heads, int n_kv_heads,
+                                                int head_dim, int window, int cache_cap, unsigned flags) {
+  if (batch <= 0 || s_new <= 0 || n_q_heads <= 0 || n_kv_heads <= 0 || head_dim <= 0 || cache_cap <= 0)
+    return 0;
+  size_t off_k;
+  const bool prefix = (flags & GEMMA_F_KV_INT8) && window == 0;
+  return prefill_ws_parts(batch, s_new, n_q_heads, n_kv_heads, head_dim, window, &off_k, nullptr,
+                          prefix ? cache_cap : 0);
 }
 
 // Where a layer's cache rows live (see cache_row): a contiguous cache, or
@@ -370,8 +391,6 @@ static int prefill_impl(const void* q, const void* k_new, const void* v_new, voi
   const bool keqv = flags & GEMMA_F_KEQV;
   if (q8) {
     if (cache_cap % 2) return fail(GEMMA_ERR_INVALID_ARG, "int8 KV: cache_cap %d must be even", cache_cap);
-    if (seq_lens_before)
-      return fail(GEMMA_ERR_UNSUPPORTED, "int8 KV: prefill after cached tokens would read int8 rows");
     if (shared) return fail(GEMMA_ERR_UNSUPPORTED, "int8 KV: a shared layer's prefill would read int8 rows");
   }
   if (!q || !out || !k_cache || !v_cache) return fail(GEMMA_ERR_INVALID_ARG, "null tensor pointer");
@@ -390,11 +409,15 @@ static int prefill_impl(const void* q, const void* k_new, const void* v_new, voi
     return fail(GEMMA_ERR_CAPACITY, "global layer: cache_cap %d < s_new %d", cache_cap, s_new);
   }
   if (s_new == 0) return succeed();
-  size_t off_k, off_vw;
-  size_t need = prefill_ws_parts(batch, s_new, n_q_heads, n_kv_heads, head_dim, window, &off_k, &off_vw);
-  // a local layer's chunk after cached tokens attends to a gathered key window
+  // a local layer's chunk after cached tokens attends to a gathered key
+  // window; so does a global layer's on an int8 cache (the dequantized
+  // prefix, with the chunk at the rows of its positions)
   const bool chunked_local = window > 0 && seq_lens_before && !shared;
-  const int win_rows = chunked_local ? window + s_new : 0;
+  const bool prefix_q8 = q8 && window == 0 && seq_lens_before;
+  const int win_rows = chunked_local ? window + s_new : prefix_q8 ? cache_cap : 0;
+  size_t off_k, off_vw;
+  size_t need = prefill_ws_parts(batch, s_new, n_q_heads, n_kv_heads, head_dim, window, &off_k, &off_vw,
+                                 prefix_q8 ? cache_cap : 0);
   if (!workspace || workspace_bytes < need)
     return fail(GEMMA_ERR_CAPACITY, "workspace %zu bytes < %zu", workspace_bytes, need);
   int* status = status_ptr();
@@ -408,9 +431,21 @@ static int prefill_impl(const void* q, const void* k_new, const void* v_new, voi
   ra.v_new = static_cast<const bf16*>(v_new);
   ra.q_rot = reinterpret_cast<bf16*>(ws);
   ra.k_rot = ((window > 0 && !shared) || q8) ? reinterpret_cast<bf16*>(ws + off_k) : nullptr;
-  ra.v_win = chunked_local ? reinterpret_cast<bf16*>(ws + off_vw) : nullptr;
+  ra.v_win = (chunked_local || prefix_q8) ? reinterpret_cast<bf16*>(ws + off_vw) : nullptr;
   ra.win_rows = win_rows;
-  if (chunked_local) {
+  ra.win_at_pos = prefix_q8 ? 1 : 0;
+  const size_t codes_off = q8 ? gemma_kv_codes_bytes(batch, n_kv_heads, cache_cap, head_dim) : 0;
+  if (q8 && (chunked_local || prefix_q8)) {
+    // before the chunk's rows are quantized into the cache: the cached rows
+    // it attends to, dequantized, into the windows (K = V: K only)
+    const uint8_t* kc8 = static_cast<const uint8_t*>(k_cache);
+    const uint8_t* vc8 = keqv ? nullptr : static_cast<const uint8_t*>(v_cache);
+    cudaError_t eg = launch_gather_q8(kc8, reinterpret_cast<const float2*>(kc8 + codes_off), vc8,
+                                      vc8 ? reinterpret_cast<const float2*>(vc8 + codes_off) : nullptr,
+                                      seq_lens_before, batch, n_kv_heads, head_dim, window, cache_cap, win_rows,
+                                      ra.k_rot, ra.v_win, status, st);
+    if (eg != cudaSuccess) return cuda_fail(eg, "int8 window gather launch");
+  } else if (chunked_local) {
     // before the chunk overwrites ring slots: old keys/values into rows 0..window-1
     cudaError_t eg = launch_ring_gather(static_cast<const bf16*>(k_cache), static_cast<const bf16*>(v_cache),
                                         seq_lens_before, batch, n_kv_heads, head_dim, window, win_rows,
@@ -439,8 +474,9 @@ static int prefill_impl(const void* q, const void* k_new, const void* v_new, voi
   ProfScope p_rope(GEMMA_KERNEL_PREFILL_ROPE, st);
   cudaError_t e = launch_prefill_rope(ra, batch, head_dim, st);
   if (e == cudaSuccess && q8)
-    e = quantize_kv(ra.k_rot, keqv ? nullptr : ra.v_new, k_cache, v_cache, batch, s_new, n_kv_heads, head_dim,
-                    window, cache_cap, nullptr, 0, status, st);
+    e = quantize_kv(ra.k_rot, win_rows ? win_rows : s_new, prefix_q8 ? 2 : chunked_local ? 1 : 0,
+                    keqv ? nullptr : ra.v_new, k_cache, v_cache, batch, s_new, n_kv_heads, head_dim, window,
+                    cache_cap, seq_lens_before, 0, status, st);
   p_rope.done();
   if (e != cudaSuccess) return cuda_fail(e, "prefill rope launch");
 
@@ -456,9 +492,9 @@ static int prefill_impl(const void* q, const void* k_new, const void* v_new, voi
     aa.k = kc;
     aa.v = vc;
     aa.key_cap = cache_cap;
-  } else if (chunked_local) {
+  } else if (chunked_local || prefix_q8) {
     KVView kw = {ra.k_rot, (int64_t)win_rows * n_kv_heads * D, (int64_t)n_kv_heads * D, D};
-    KVView vw = {ra.v_win, kw.stride_b, kw.stride_row, kw.stride_h};
+    KVView vw = {keqv ? ra.k_rot : ra.v_win, kw.stride_b, kw.stride_row, kw.stride_h};
     aa.k = kw;
     aa.v = vw;
     aa.key_cap = win_rows;
@@ -499,7 +535,7 @@ static int prefill_impl(const void* q, const void* k_new, const void* v_new, voi
   if (head_dim == 512) {
     if ((n_q_heads / n_kv_heads) % 2 == 0)
       kern = K_HPAIR;
-    else if ((cache_view ? cache_cap : s_new) >= 16384)
+    else if ((cache_view || prefix_q8 ? cache_cap : s_new) >= 16384)
       kern = K_PAIR;
   }
   if (const char* v = std::getenv("GEMMA_PREFILL_KERNEL")) {
@@ -607,7 +643,7 @@ static int decode_impl(const void* q, const void* k_new, const void* v_new, void
   ProfScope p_app(GEMMA_KERNEL_DECODE_APPEND, st);
   cudaError_t e = launch_decode_rope_append(ra, batch, head_dim, st);
   if (e == cudaSuccess && q8 && k_new)
-    e = quantize_kv(ra.k_stage, (flags & GEMMA_F_KEQV) ? nullptr : ra.v_new, k_cache, v_cache, batch, 1,
+    e = quantize_kv(ra.k_stage, 1, 0, (flags & GEMMA_F_KEQV) ? nullptr : ra.v_new, k_cache, v_cache, batch, 1,
                     n_kv_heads, head_dim, window, cache_cap, seq_lens, 1, status, st);
   p_app.done();
   if (e != cudaSuccess) return cuda_fail(e, "decode append launch");

@@ -33,11 +33,15 @@ __host__ __device__ __forceinline__ int64_t visible_range(int64_t pos, int windo
 // table[b * pps + p / ps]. A contiguous cache [B][Hkv][cap][D] is the case
 // table == null: page b, ps = cap. Returns the row index into the pool
 // (in units of D elements), or -1 when the page index is outside the pool.
+// Positions are below the int capacity, so pages take 32-bit division; a
+// contiguous cache takes none (this sits on the decode producer's path).
 __host__ __device__ __forceinline__ int64_t cache_row(const int32_t* table, int pps, int ps, int n_pages,
                                                       int Hkv, int b, int h, int64_t p) {
-  const int64_t page = table ? (int64_t)table[(int64_t)b * pps + p / ps] : (int64_t)b;
+  if (!table) return ((int64_t)b * Hkv + h) * ps + p;
+  const int pi = (int)p / ps;
+  const int64_t page = table[(int64_t)b * pps + pi];
   if (page < 0 || page >= n_pages) return -1;
-  return (page * Hkv + h) * ps + p % ps;
+  return (page * Hkv + h) * ps + ((int)p - pi * ps);
 }
 
 // Number of rotated pairs under (p-)RoPE: floor(rope_frac * head_dim / 2).

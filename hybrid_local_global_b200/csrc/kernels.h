@@ -15,9 +15,12 @@ struct PrefillRopeArgs {
   const bf16* v_new;   // [B][S][Hkv][D] or null
   bf16* q_rot;         // workspace [B][S][Hq][D]
   bf16* k_rot;         // workspace, local layers: [B][S][Hkv][D], or with win_rows > 0
-                       // [B][win_rows][Hkv][D] with the chunk at rows window.. ; else null
-  bf16* v_win;         // chunked local prefill: V window [B][win_rows][Hkv][D], else null
-  int win_rows;        // 0, or window + S (chunked local prefill)
+                       // [B][win_rows][Hkv][D] with the chunk at rows window.. (or, with
+                       // win_at_pos, at rows seq_lens_before[b]..); else null
+  bf16* v_win;         // key windows (chunked prefill): V window [B][win_rows][Hkv][D], else null
+  int win_rows;        // 0, or the window rows per sequence: window + S (chunked local prefill)
+                       // or cache_cap (int8 global prefill after cached tokens)
+  int win_at_pos;      // 1: a chunk token's window row is its position
   bf16* k_cache;       // [B][Hkv][cap][D]
   bf16* v_cache;
   int cache_cap;
@@ -63,7 +66,9 @@ struct DecodeRopeArgs {
 // the last `window` rows of the chunk) of codes [B][Hkv][cap][D] and
 // params [B][Hkv][cap] (min, step).
 struct QuantRowsArgs {
-  const bf16* src;
+  const bf16* src;     // [B][src_rows][Hkv][D]; chunk token s at row s (src_row_mode 0),
+  int src_rows;        // window + s (1) or its position (2)
+  int src_row_mode;
   int S, Hkv, window, cache_cap;
   const int32_t* pos0;  // device [B], or null for 0
   int pos0_minus;
@@ -135,6 +140,14 @@ cudaError_t launch_prefill_rope(const PrefillRopeArgs& a, int B, int D, cudaStre
 cudaError_t launch_ring_gather(const bf16* k_cache, const bf16* v_cache, const int32_t* seq_lens_before,
                                int B, int Hkv, int D, int window, int win_rows, bf16* k_win, bf16* v_win,
                                int* status, cudaStream_t st);
+// Int8 caches: dequantize cached rows (min + code * step, rounded to bf16)
+// into key windows [B][win_rows][Hkv][D]. window > 0: the ring's positions
+// pos0-window .. pos0-1 into rows 0..window-1 (negative positions: zeros);
+// window 0: positions 0 .. pos0-1 into rows 0..pos0-1. v_codes null: K only.
+cudaError_t launch_gather_q8(const uint8_t* k_codes, const float2* k_params, const uint8_t* v_codes,
+                             const float2* v_params, const int32_t* seq_lens_before, int B, int Hkv, int D,
+                             int window, int cache_cap, int win_rows, bf16* k_win, bf16* v_win, int* status,
+                             cudaStream_t st);
 cudaError_t launch_decode_rope_append(const DecodeRopeArgs& a, int B, int D, cudaStream_t st);
 cudaError_t launch_quantize_rows(const QuantRowsArgs& a, int B, int D, cudaStream_t st);
 // tcgen05 prefill (head_dim 256 or 512). key_rows_total = rows of the K/V

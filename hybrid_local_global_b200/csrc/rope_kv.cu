@@ -20,6 +20,8 @@
 // Thread map: threadIdx.x owns 8 consecutive elements (4 pairs) of the head
 // vector, so its inverse frequencies are computed once and each angle once
 // per position, then reused for every Q and K head of that position.
+#include <algorithm>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -173,8 +175,9 @@ __global__ void __launch_bounds__(256, 2) k_prefill_rope(PrefillRopeArgs a) {
 #pragma unroll
       for (int u = 0; u < ROPE_HB / 2; ++u) kx[u] = vx[u] = make_uint4(0, 0, 0, 0);
       // no v_new: K = V; the V window (WIN) takes every position of the chunk
-      const bool want_v = a.v_new && !a.quant && (WIN || a.window == 0 || to_ring);
-      const int64_t wrow = WIN ? (int64_t)b * a.win_rows + a.window + s : row;  // k_rot / V window row
+      const bool want_v = a.v_new && (WIN || (!a.quant && (a.window == 0 || to_ring)));
+      // k_rot / V window row
+      const int64_t wrow = WIN ? (int64_t)b * a.win_rows + (a.win_at_pos ? pos : a.window + s) : row;
 #pragma unroll
       for (int u = 0; u < ROPE_HB / 2; ++u)
         if (h0 + u < a.Hkv) {
@@ -244,6 +247,75 @@ __global__ void __launch_bounds__(256) k_ring_gather(const bf16* __restrict__ k_
     const int64_t dst = (((int64_t)b * win_rows + r) * Hkv + h) * D + c;
     st16(k_win + dst, kv);
     st16(v_win + dst, vv);
+  }
+}
+
+// Int8 caches: the key windows of a prefill after cached tokens, from the
+// codes. A warp dequantizes one cached row (one position, one KV head):
+// value = min + code * step in fp32, rounded to bf16. window > 0: rows
+// 0..window-1 take the ring's positions pos0-window .. pos0-1 (slot p mod
+// window; negative positions give zeros, never visible); window 0: rows
+// 0..pos0-1 take positions 0..pos0-1 (slot = position).
+template <int D>
+__global__ void __launch_bounds__(256) k_gather_q8(const uint8_t* __restrict__ k_codes,
+                                                   const float2* __restrict__ k_params,
+                                                   const uint8_t* __restrict__ v_codes,
+                                                   const float2* __restrict__ v_params,
+                                                   const int32_t* seq_lens_before, int Hkv, int window,
+                                                   int cache_cap, int win_rows, bf16* k_win, bf16* v_win,
+                                                   int* status) {
+  constexpr int E = D / 32;  // codes per lane: 8 or 16
+  const int b = blockIdx.y;
+  const int64_t pos0 = seq_lens_before[b];
+  if (pos0 < 0 || (window == 0 && pos0 > cache_cap)) {
+    if (threadIdx.x == 0 && blockIdx.x == 0) set_status(status, GEMMA_ERR_DEVICE_RANGE);
+    return;
+  }
+  const int64_t rows = window > 0 ? window : pos0;
+  const int lane = threadIdx.x & 31;
+  const int64_t n_items = rows * Hkv;
+  for (int64_t it = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5); it < n_items; it += (int64_t)gridDim.x * 8) {
+    const int64_t r = it / Hkv;
+    const int h = (int)(it % Hkv);
+    const int64_t p = window > 0 ? pos0 - window + r : r;
+    const int64_t dst = (((int64_t)b * win_rows + r) * Hkv + h) * D + lane * E;
+    for (int kv = 0; kv < (v_codes ? 2 : 1); ++kv) {
+      bf16* out = (kv ? v_win : k_win) + dst;
+      uint32_t packed[E / 2];
+      if (p < 0) {
+#pragma unroll
+        for (int i = 0; i < E / 2; ++i) packed[i] = 0;
+      } else {
+        const int64_t crow = ((int64_t)b * Hkv + h) * cache_cap + (window > 0 ? p % window : p);
+        const float2 mp = (kv ? v_params : k_params)[crow];
+        const uint8_t* cp = (kv ? v_codes : k_codes) + crow * D + lane * E;
+        uint32_t w[E / 4];
+        if constexpr (E == 8) {
+          const uint2 u = *reinterpret_cast<const uint2*>(cp);
+          w[0] = u.x;
+          w[1] = u.y;
+        } else {
+          const uint4 u = *reinterpret_cast<const uint4*>(cp);
+          w[0] = u.x;
+          w[1] = u.y;
+          w[2] = u.z;
+          w[3] = u.w;
+        }
+#pragma unroll
+        for (int i = 0; i < E / 2; ++i) {
+          const uint32_t word = w[i / 2];
+          const float c0 = (float)((word >> (16 * (i % 2))) & 0xffu);
+          const float c1 = (float)((word >> (16 * (i % 2) + 8)) & 0xffu);
+          packed[i] = pack_bf16x2(__fmaf_rn(c0, mp.y, mp.x), __fmaf_rn(c1, mp.y, mp.x));
+        }
+      }
+      if constexpr (E == 8) {
+        *reinterpret_cast<uint4*>(out) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+      } else {
+        *reinterpret_cast<uint4*>(out) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+        *reinterpret_cast<uint4*>(out + 8) = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+      }
+    }
   }
 }
 
@@ -319,7 +391,8 @@ __global__ void __launch_bounds__(256) k_quantize_rows(QuantRowsArgs a, int n_ro
     if (lane == 0) set_status(a.status, GEMMA_ERR_DEVICE_RANGE);
     return;
   }
-  const bf16* src = a.src + (((int64_t)b * a.S + s) * a.Hkv + h) * D + lane * E;
+  const int64_t srow = a.src_row_mode == 0 ? s : a.src_row_mode == 1 ? (int64_t)a.window + s : pos;
+  const bf16* src = a.src + (((int64_t)b * a.src_rows + srow) * a.Hkv + h) * D + lane * E;
   float x[E];
 #pragma unroll
   for (int c = 0; c < E / 8; ++c) {
@@ -404,6 +477,22 @@ cudaError_t launch_ring_gather(const bf16* k_cache, const bf16* v_cache, const i
   else
     k_ring_gather<512><<<grid, 256, 0, st>>>(k_cache, v_cache, seq_lens_before, Hkv, window, win_rows, k_win,
                                              v_win, status);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gather_q8(const uint8_t* k_codes, const float2* k_params, const uint8_t* v_codes,
+                             const float2* v_params, const int32_t* seq_lens_before, int B, int Hkv, int D,
+                             int window, int cache_cap, int win_rows, bf16* k_win, bf16* v_win, int* status,
+                             cudaStream_t st) {
+  const int64_t rows = window > 0 ? window : cache_cap;  // an upper bound; blocks stride over the rest
+  const int64_t blocks = std::min<int64_t>((rows * Hkv + 7) / 8, 1184);
+  dim3 grid((unsigned)std::max<int64_t>(blocks, 1), B);
+  if (D == 256)
+    k_gather_q8<256><<<grid, 256, 0, st>>>(k_codes, k_params, v_codes, v_params, seq_lens_before, Hkv, window,
+                                           cache_cap, win_rows, k_win, v_win, status);
+  else
+    k_gather_q8<512><<<grid, 256, 0, st>>>(k_codes, k_params, v_codes, v_params, seq_lens_before, Hkv, window,
+                                           cache_cap, win_rows, k_win, v_win, status);
   return cudaGetLastError();
 }
 

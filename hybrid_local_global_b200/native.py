@@ -53,6 +53,8 @@ def _sig(name, restype, argtypes):
 
 
 _prefill_ws = _sig("gemma_attn_prefill_workspace_size", _SZ, [_I, _I, _I, _I, _I, _I])
+_prefill_ws_cached = _sig("gemma_attn_prefill_workspace_size_cached", _SZ,
+                          [_I, _I, _I, _I, _I, _I, _I, ctypes.c_uint])
 _prefill = _sig("gemma_attn_prefill", _I, [_P, _P, _P, _P, _P, _I, _P, _I, _I, _I, _I, _I, _I,
                                            _F, _F, _F, _P, _P, _P, _SZ, ctypes.c_uint, _P])
 _decode_ws = _sig("gemma_attn_decode_workspace_size", _SZ, [_I, _I, _I, _I, _I, _I])
@@ -77,7 +79,7 @@ EXPORTED = ["gemma_attn_prefill_workspace_size", "gemma_attn_prefill",
             "gemma_layer_schedule", "gemma_attn_visible_ranges", "gemma_attn_sync_status",
             "gemma_last_error", "gemma_attn_set_wait_limit", "gemma_attn_debug_drop_next_copy",
             "gemma_kv_cache_bytes", "gemma_kv_codes_bytes", "gemma_attn_prefill_paged",
-            "gemma_attn_decode_paged"]
+            "gemma_attn_decode_paged", "gemma_attn_prefill_workspace_size_cached"]
 
 
 class GemmaError(RuntimeError):
@@ -150,6 +152,11 @@ def gemma_attn_prefill_workspace_size(batch, s_new, n_q_heads, n_kv_heads, head_
     return int(_prefill_ws(batch, s_new, n_q_heads, n_kv_heads, head_dim, window))
 
 
+def gemma_attn_prefill_workspace_size_cached(batch, s_new, n_q_heads, n_kv_heads, head_dim, window, cache_cap,
+                                             flags=0) -> int:
+    return int(_prefill_ws_cached(batch, s_new, n_q_heads, n_kv_heads, head_dim, window, cache_cap, flags))
+
+
 def gemma_attn_prefill(q, k_new, v_new, k_cache, v_cache, *, window, rope_frac, rope_theta, scale,
                        out, seq_lens_before=None, lse=None, workspace=None, flags=0, stream=None):
     """q [B,S,Hq,D]; k_new/v_new [B,S,Hkv,D] (None if shared); caches [B,Hkv,cap,D]."""
@@ -161,7 +168,8 @@ def gemma_attn_prefill(q, k_new, v_new, k_cache, v_cache, *, window, rope_frac, 
     if isinstance(k_cache, Int8KVCache):
         flags |= GEMMA_F_KV_INT8
     if workspace is None:
-        n = gemma_attn_prefill_workspace_size(B, S, Hq, Hkv, D, window)
+        n = (gemma_attn_prefill_workspace_size_cached(B, S, Hq, Hkv, D, window, cap, flags)
+             if seq_lens_before is not None else gemma_attn_prefill_workspace_size(B, S, Hq, Hkv, D, window))
         workspace = torch.empty(max(n, 1), dtype=torch.uint8, device=q.device)
     return _check(_prefill(_ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_cache), _ptr(v_cache), cap,
                            _ptr(seq_lens_before), B, S, window, Hq, Hkv, D, rope_frac, rope_theta,

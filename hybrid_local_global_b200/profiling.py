@@ -39,7 +39,7 @@ KERNEL_SOURCES = {
     "k_prefill_tc": ("prefill_tc.cu", "tc.cuh", "common.cuh", "tmap.cu", "tmap.h"),
     "k_prefill_pair": ("prefill_pair.cu", "pair.cuh", "tc.cuh", "common.cuh", "tmap.cu", "tmap.h"),
     "k_decode_split": ("decode.cu", "mma_sync.cuh", "common.cuh"),
-    "k_decode_split_q8": ("decode_q8.cu", "mma_sync.cuh", "common.cuh"),
+    "k_decode_split_q8": ("decode_q8.cu", "mma_sync.cuh", "tc.cuh", "common.cuh", "tmap.cu", "tmap.h"),
 }
 
 

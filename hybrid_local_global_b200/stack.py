@@ -86,11 +86,24 @@ class AttentionStack:
         return total
 
     # ------------------------------------------------------------------ prefill
-    def prefill_workspace_bytes(self) -> int:
+    def prefill_workspace_bytes(self, after_cached: bool | None = None) -> int:
+        """Workspace for one prefill layer call; after_cached (default: the
+        workload has cached tokens) sizes it for chunks after cached tokens."""
         w = self.w
-        return max(native.gemma_attn_prefill_workspace_size(
-            w.batch, w.seq, w.n_q_heads, self.layer_type(l).n_kv_heads, self.layer_type(l).head_dim,
-            self.layer_type(l).window) for l in range(self.n_layers))
+        if after_cached is None:
+            after_cached = w.prior > 0
+        flags = native.GEMMA_F_KV_INT8 if w.kv_int8 else 0
+        sizes = []
+        for l in range(self.n_layers):
+            t = self.layer_type(l)
+            if after_cached:
+                cap = t.window if t.window > 0 else self.global_capacity
+                sizes.append(native.gemma_attn_prefill_workspace_size_cached(
+                    w.batch, w.seq, w.n_q_heads, t.n_kv_heads, t.head_dim, t.window, cap, flags))
+            else:
+                sizes.append(native.gemma_attn_prefill_workspace_size(
+                    w.batch, w.seq, w.n_q_heads, t.n_kv_heads, t.head_dim, t.window))
+        return max(sizes)
 
     def prefill_layer(self, l: int, q, k, v, out, *, workspace, seq_lens_before=None, lse=None,
                       stream=None):

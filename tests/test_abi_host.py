@@ -126,6 +126,8 @@ def _decode_raw(**over):
 
 
 E = native
+# the plain workspace of the prefill harness's shapes on a global layer
+PLAIN_WS_GLOBAL = native.gemma_attn_prefill_workspace_size(1, 16, 8, 4, 256, 0)
 
 
 @pytest.mark.parametrize("over,code", [
@@ -145,7 +147,9 @@ E = native
     (dict(flags=8), E.GEMMA_ERR_INVALID_ARG),          # unknown flag
     (dict(flags=4, wsb=16), E.GEMMA_ERR_CAPACITY),     # int8 KV: accepted
     (dict(flags=4, W=0, cap=4095, wsb=16), E.GEMMA_ERR_INVALID_ARG),   # int8 KV: odd capacity
-    (dict(flags=4, lens=FAKE), E.GEMMA_ERR_UNSUPPORTED),               # int8 KV after cached tokens
+    (dict(flags=4, lens=FAKE, wsb=16), E.GEMMA_ERR_CAPACITY),          # int8 KV after cached tokens: accepted
+    (dict(flags=4, W=0, cap=16384, lens=FAKE, wsb=PLAIN_WS_GLOBAL), E.GEMMA_ERR_CAPACITY),  # ... whose global
+                                                                        # layers need the larger workspace
     (dict(flags=5, k=None, v=None), E.GEMMA_ERR_UNSUPPORTED),          # int8 KV on a shared layer's prefill
     (dict(W=0, cap=4096, flags=6, v=None, wsb=16), E.GEMMA_ERR_CAPACITY),  # int8 K = V: accepted
     (dict(flags=2, v=None), E.GEMMA_ERR_UNSUPPORTED),  # K = V on a local layer
@@ -182,6 +186,22 @@ def test_prefill_validation(over, code):
 ])
 def test_decode_validation(over, code):
     assert _decode_raw(**over) == code
+
+
+def test_cached_prefill_workspace_sizes():
+    """Only an int8 global layer after cached tokens needs more: its keys and
+    values up to the capacity in bf16."""
+    for W in (512, 0):
+        for D, Hkv in ((256, 4), (512, 1)):
+            plain = native.gemma_attn_prefill_workspace_size(2, 1024, 8, Hkv, D, W)
+            assert native.gemma_attn_prefill_workspace_size_cached(2, 1024, 8, Hkv, D, W, 16384, 0) == plain
+            q8 = native.gemma_attn_prefill_workspace_size_cached(2, 1024, 8, Hkv, D, W, 16384,
+                                                                 native.GEMMA_F_KV_INT8)
+            if W:
+                assert q8 == plain
+            else:
+                assert q8 >= 2 * 1024 * 8 * D * 2 + 2 * (2 * 16384 * Hkv * D * 2)
+    assert native.gemma_attn_prefill_workspace_size_cached(2, 1024, 8, 4, 256, 0, 0, 0) == 0
 
 
 def test_workspace_sizes_cover_the_configs():

@@ -242,3 +242,110 @@ def test_decode_int8_value_ranges(oracle, v_scale):
     scaled by a power of two that keeps them in range."""
     run_decode_int8(oracle, lens=[300, 1500], Hq=8, Hkv=1, D=512, W=0, frac=0.25, theta=1e6, seed=323,
                     v_scale=v_scale, tol=(2e-2 * v_scale, 2e-3 * v_scale))
+
+
+# ------------------------------------------------- prefill after cached tokens
+def run_prefill_int8_chunk(oracle, *, before, S, Hq, Hkv, D, W, frac, theta, seed, keqv=False):
+    """A chunk of S tokens after `before[b]` cached tokens on an int8 cache.
+
+    The cached rows are the oracle's quantization of seeded (already rotated)
+    rows; the chunk attends to them dequantized (min + code * step) and to
+    its own keys and values; its rows are then quantized into the cache."""
+    dev = torch.device("cuda")
+    B = len(before)
+    g = synth.generator(seed)
+    cap = W if W else max(before) + S + 16 + (max(before) + S) % 2
+    k_rows = synth.randn_bf16((B, Hkv, cap, D), g)
+    v_rows = k_rows if keqv else synth.randn_bf16((B, Hkv, cap, D), g)
+    q = synth.randn_bf16((B, S, Hq, D), g)
+    kn = synth.randn_bf16((B, S, Hkv, D), g)
+    vn = kn if keqv else synth.randn_bf16((B, S, Hkv, D), g)
+    ck, pk = quantize(oracle, k_rows)
+    cv, pv = (ck, pk) if keqv else quantize(oracle, v_rows)
+    kc = native.Int8KVCache(B, Hkv, cap, D, dev)
+    kc.codes.copy_(ck)
+    kc.params.copy_(pk)
+    vc = kc
+    if not keqv:
+        vc = native.Int8KVCache(B, Hkv, cap, D, dev)
+        vc.codes.copy_(cv)
+        vc.params.copy_(pv)
+    out = torch.full((B, S, Hq, D), float("nan"), dtype=torch.bfloat16, device=dev)
+    lse = torch.full((B, Hq, S), float("nan"), dtype=torch.float32, device=dev)
+    scale = 1.0 / math.sqrt(D)
+    native.gemma_attn_prefill(q.to(dev), kn.to(dev), None if keqv else vn.to(dev), kc, None if keqv else vc,
+                              window=W, rope_frac=frac, rope_theta=theta, scale=scale, out=out, lse=lse,
+                              seq_lens_before=torch.tensor(before, dtype=torch.int32, device=dev),
+                              flags=native.GEMMA_F_KEQV if keqv else 0)
+    assert native.gemma_attn_sync_status() == 0, native.gemma_last_error()
+    ck1, pk1, cv1, pv1 = kc.codes.cpu(), kc.params.cpu(), vc.codes.cpu(), vc.params.cpu()
+    G = Hq // Hkv
+    out_c, lse_c = out.float().cpu().double().numpy(), lse.cpu().double().numpy()
+    for b in range(B):
+        P0 = before[b]
+        lo = max(0, P0 - W) if W else 0
+        positions = list(range(lo, P0 + S))
+        n = len(positions)
+        keys = np.zeros((Hkv, n, D))
+        vals = np.zeros((Hkv, n, D))
+        written = torch.zeros(cap, dtype=torch.bool)
+        for idx, p in enumerate(positions):
+            if p < P0:  # cached: the rows the cache held before the call
+                s = p % W if W else p
+                keys[:, idx] = dequant(oracle, ck[b, :, s], pk[b, :, s])
+                vals[:, idx] = dequant(oracle, cv[b, :, s], pv[b, :, s])
+            else:       # the chunk's own rotated key and value
+                i = p - P0
+                keys[:, idx] = np.stack([oracle.rope_bf16(to_bits(kn[b, i, h]), p, frac, theta)
+                                         for h in range(Hkv)])
+                # K = V: the values are the rotated keys
+                vals[:, idx] = keys[:, idx] if keqv else vn[b, i].double().numpy()
+                if W and i < S - W:
+                    continue  # overwritten later in the same chunk: never reaches the ring
+                s = p % W if W else p
+                written[s] = True
+                ec, ep = quantize(oracle, rotated_bf16(oracle, kn[b, i], p, frac, theta))
+                if frac == 0.0:
+                    assert torch.equal(ck1[b, :, s], ec) and torch.equal(pk1[b, :, s], ep)
+                else:
+                    assert_rows_within_step(oracle, ck1[b, :, s], pk1[b, :, s], ec, ep, "K b=%d p=%d" % (b, p))
+                if not keqv:
+                    ec, ep = quantize(oracle, vn[b, i])
+                    assert torch.equal(cv1[b, :, s], ec) and torch.equal(pv1[b, :, s], ep), "V b=%d p=%d" % (b, p)
+        # rows the chunk does not write keep their codes
+        assert torch.equal(ck1[b][:, ~written], ck[b][:, ~written])
+        assert torch.equal(pk1[b][:, ~written], pk[b][:, ~written])
+        rows_q, begin, count = [], [], []
+        for i in range(S):
+            P = P0 + i
+            vis_lo = max(lo, P - W + 1) if W else 0
+            for h in range(Hq):
+                rows_q.append(oracle.rope_bf16(to_bits(q[b, i, h]), P, frac, theta))
+                begin.append((h // G) * n + (vis_lo - lo))
+                count.append(P - vis_lo + 1)
+        ref, ref_lse = oracle.attend_rows(np.array(rows_q), keys.reshape(Hkv * n, D), vals.reshape(Hkv * n, D),
+                                          begin, count, scale)
+        assert_close(out_c[b].reshape(S * Hq, D), ref, 2e-2, 2e-3, what="int8 chunk b=%d before=%d" % (b, P0))
+        got_lse = lse_c[b].transpose(1, 0).reshape(S * Hq)
+        assert np.abs(got_lse - ref_lse).max() < 2e-2, "lse b=%d" % b
+
+
+CHUNK_CASES = [
+    dict(before=[300, 0, 1000], S=200, Hq=8, Hkv=1, D=512, W=0, frac=0.25, theta=1e6, seed=331),
+    dict(before=[4096], S=256, Hq=32, Hkv=4, D=512, W=0, frac=0.25, theta=1e6, seed=332),
+    dict(before=[77, 200], S=96, Hq=4, Hkv=2, D=256, W=0, frac=0.0, theta=1e4, seed=333),
+    dict(before=[50, 300, 0], S=100, Hq=8, Hkv=4, D=256, W=128, frac=1.0, theta=1e4, seed=334),
+    dict(before=[500, 3], S=300, Hq=8, Hkv=4, D=256, W=128, frac=1.0, theta=1e4, seed=335),
+    dict(before=[64, 65], S=4, Hq=32, Hkv=16, D=256, W=64, frac=0.0, theta=1e4, seed=336),
+]
+
+
+@pytest.mark.parametrize("case", CHUNK_CASES, ids=["global", "global_h32", "global_d256_nope", "local",
+                                                   "local_long_chunk", "local_verify4"])
+def test_prefill_int8_after_cached_tokens(oracle, case):
+    run_prefill_int8_chunk(oracle, **case)
+
+
+def test_prefill_int8_after_cached_tokens_k_equals_v(oracle):
+    run_prefill_int8_chunk(oracle, before=[129, 700], S=130, Hq=8, Hkv=1, D=512, W=0, frac=0.25, theta=1e6,
+                           seed=337, keqv=True)
