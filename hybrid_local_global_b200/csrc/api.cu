@@ -391,7 +391,6 @@ static int prefill_impl(const void* q, const void* k_new, const void* v_new, voi
   const bool keqv = flags & GEMMA_F_KEQV;
   if (q8) {
     if (cache_cap % 2) return fail(GEMMA_ERR_INVALID_ARG, "int8 KV: cache_cap %d must be even", cache_cap);
-    if (shared) return fail(GEMMA_ERR_UNSUPPORTED, "int8 KV: a shared layer's prefill would read int8 rows");
   }
   if (!q || !out || !k_cache || !v_cache) return fail(GEMMA_ERR_INVALID_ARG, "null tensor pointer");
   if (!aligned16(q) || !aligned16(out) || !aligned16(k_cache) || !aligned16(v_cache) ||
@@ -410,11 +409,13 @@ static int prefill_impl(const void* q, const void* k_new, const void* v_new, voi
   }
   if (s_new == 0) return succeed();
   // a local layer's chunk after cached tokens attends to a gathered key
-  // window; so does a global layer's on an int8 cache (the dequantized
-  // prefix, with the chunk at the rows of its positions)
+  // window. On an int8 cache so does every chunk that reads cached rows
+  // (after cached tokens, or a shared layer's): the rows are dequantized
+  // into the window; a global layer's window rows are positions.
   const bool chunked_local = window > 0 && seq_lens_before && !shared;
-  const bool prefix_q8 = q8 && window == 0 && seq_lens_before;
-  const int win_rows = chunked_local ? window + s_new : prefix_q8 ? cache_cap : 0;
+  const bool win_local = chunked_local || (q8 && window > 0 && shared);
+  const bool prefix_q8 = q8 && window == 0 && (seq_lens_before || shared);
+  const int win_rows = win_local ? window + s_new : prefix_q8 ? cache_cap : 0;
   size_t off_k, off_vw;
   size_t need = prefill_ws_parts(batch, s_new, n_q_heads, n_kv_heads, head_dim, window, &off_k, &off_vw,
                                  prefix_q8 ? cache_cap : 0);
@@ -431,19 +432,20 @@ static int prefill_impl(const void* q, const void* k_new, const void* v_new, voi
   ra.v_new = static_cast<const bf16*>(v_new);
   ra.q_rot = reinterpret_cast<bf16*>(ws);
   ra.k_rot = ((window > 0 && !shared) || q8) ? reinterpret_cast<bf16*>(ws + off_k) : nullptr;
-  ra.v_win = (chunked_local || prefix_q8) ? reinterpret_cast<bf16*>(ws + off_vw) : nullptr;
+  ra.v_win = (win_local || prefix_q8) ? reinterpret_cast<bf16*>(ws + off_vw) : nullptr;
   ra.win_rows = win_rows;
   ra.win_at_pos = prefix_q8 ? 1 : 0;
   const size_t codes_off = q8 ? gemma_kv_codes_bytes(batch, n_kv_heads, cache_cap, head_dim) : 0;
-  if (q8 && (chunked_local || prefix_q8)) {
+  if (q8 && (win_local || prefix_q8)) {
     // before the chunk's rows are quantized into the cache: the cached rows
-    // it attends to, dequantized, into the windows (K = V: K only)
+    // it attends to, dequantized, into the windows (K = V: K only). A shared
+    // layer's chunk is in the cache already: its positions come along.
     const uint8_t* kc8 = static_cast<const uint8_t*>(k_cache);
     const uint8_t* vc8 = keqv ? nullptr : static_cast<const uint8_t*>(v_cache);
     cudaError_t eg = launch_gather_q8(kc8, reinterpret_cast<const float2*>(kc8 + codes_off), vc8,
                                       vc8 ? reinterpret_cast<const float2*>(vc8 + codes_off) : nullptr,
-                                      seq_lens_before, batch, n_kv_heads, head_dim, window, cache_cap, win_rows,
-                                      ra.k_rot, ra.v_win, status, st);
+                                      seq_lens_before, shared ? s_new : 0, batch, n_kv_heads, head_dim, window,
+                                      cache_cap, win_rows, ra.k_rot, ra.v_win, status, st);
     if (eg != cudaSuccess) return cuda_fail(eg, "int8 window gather launch");
   } else if (chunked_local) {
     // before the chunk overwrites ring slots: old keys/values into rows 0..window-1
@@ -473,7 +475,7 @@ static int prefill_impl(const void* q, const void* k_new, const void* v_new, voi
   ra.status = status;
   ProfScope p_rope(GEMMA_KERNEL_PREFILL_ROPE, st);
   cudaError_t e = launch_prefill_rope(ra, batch, head_dim, st);
-  if (e == cudaSuccess && q8)
+  if (e == cudaSuccess && q8 && !shared)
     e = quantize_kv(ra.k_rot, win_rows ? win_rows : s_new, prefix_q8 ? 2 : chunked_local ? 1 : 0,
                     keqv ? nullptr : ra.v_new, k_cache, v_cache, batch, s_new, n_kv_heads, head_dim, window,
                     cache_cap, seq_lens_before, 0, status, st);
@@ -492,7 +494,7 @@ static int prefill_impl(const void* q, const void* k_new, const void* v_new, voi
     aa.k = kc;
     aa.v = vc;
     aa.key_cap = cache_cap;
-  } else if (chunked_local || prefix_q8) {
+  } else if (win_local || prefix_q8) {
     KVView kw = {ra.k_rot, (int64_t)win_rows * n_kv_heads * D, (int64_t)n_kv_heads * D, D};
     KVView vw = {keqv ? ra.k_rot : ra.v_win, kw.stride_b, kw.stride_row, kw.stride_h};
     aa.k = kw;
@@ -506,7 +508,7 @@ static int prefill_impl(const void* q, const void* k_new, const void* v_new, voi
     aa.v = vw;
     aa.key_cap = s_new;
   }
-  aa.key_off_window = chunked_local ? 1 : 0;
+  aa.key_off_window = win_local ? 1 : 0;
   aa.seq_lens_before = seq_lens_before;
   aa.S = s_new;
   aa.window = window;

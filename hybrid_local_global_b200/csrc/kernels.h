@@ -141,13 +141,15 @@ cudaError_t launch_ring_gather(const bf16* k_cache, const bf16* v_cache, const i
                                int B, int Hkv, int D, int window, int win_rows, bf16* k_win, bf16* v_win,
                                int* status, cudaStream_t st);
 // Int8 caches: dequantize cached rows (min + code * step, rounded to bf16)
-// into key windows [B][win_rows][Hkv][D]. window > 0: the ring's positions
-// pos0-window .. pos0-1 into rows 0..window-1 (negative positions: zeros);
-// window 0: positions 0 .. pos0-1 into rows 0..pos0-1. v_codes null: K only.
+// into key windows [B][win_rows][Hkv][D]; pos0 = seq_lens_before[b] (0 if
+// null), plus `extra` positions (a shared layer's chunk). window > 0: the
+// ring's positions pos0-window .. pos0+extra-1 into rows 0.. (negative
+// positions: zeros); window 0: positions 0 .. pos0+extra-1 into rows 0.. .
+// v_codes null: K only.
 cudaError_t launch_gather_q8(const uint8_t* k_codes, const float2* k_params, const uint8_t* v_codes,
-                             const float2* v_params, const int32_t* seq_lens_before, int B, int Hkv, int D,
-                             int window, int cache_cap, int win_rows, bf16* k_win, bf16* v_win, int* status,
-                             cudaStream_t st);
+                             const float2* v_params, const int32_t* seq_lens_before, int extra, int B, int Hkv,
+                             int D, int window, int cache_cap, int win_rows, bf16* k_win, bf16* v_win,
+                             int* status, cudaStream_t st);
 cudaError_t launch_decode_rope_append(const DecodeRopeArgs& a, int B, int D, cudaStream_t st);
 cudaError_t launch_quantize_rows(const QuantRowsArgs& a, int B, int D, cudaStream_t st);
 // tcgen05 prefill (head_dim 256 or 512). key_rows_total = rows of the K/V

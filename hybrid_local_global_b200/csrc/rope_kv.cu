@@ -250,28 +250,30 @@ __global__ void __launch_bounds__(256) k_ring_gather(const bf16* __restrict__ k_
   }
 }
 
-// Int8 caches: the key windows of a prefill after cached tokens, from the
-// codes. A warp dequantizes one cached row (one position, one KV head):
-// value = min + code * step in fp32, rounded to bf16. window > 0: rows
-// 0..window-1 take the ring's positions pos0-window .. pos0-1 (slot p mod
-// window; negative positions give zeros, never visible); window 0: rows
-// 0..pos0-1 take positions 0..pos0-1 (slot = position).
+// Int8 caches: the key windows of a prefill that reads cached rows, from
+// the codes. A warp dequantizes one cached row (one position, one KV head):
+// value = min + code * step in fp32, rounded to bf16. With pos0 =
+// seq_lens_before[b] (0 if null) and `extra` more positions (a shared
+// layer's chunk, already in the cache): window > 0: rows 0..window+extra-1
+// take positions pos0-window .. pos0+extra-1 (slot p mod window; negative
+// positions give zeros, never visible); window 0: rows 0..pos0+extra-1 take
+// positions 0..pos0+extra-1 (slot = position).
 template <int D>
 __global__ void __launch_bounds__(256) k_gather_q8(const uint8_t* __restrict__ k_codes,
                                                    const float2* __restrict__ k_params,
                                                    const uint8_t* __restrict__ v_codes,
                                                    const float2* __restrict__ v_params,
-                                                   const int32_t* seq_lens_before, int Hkv, int window,
-                                                   int cache_cap, int win_rows, bf16* k_win, bf16* v_win,
-                                                   int* status) {
+                                                   const int32_t* seq_lens_before, int extra, int Hkv,
+                                                   int window, int cache_cap, int win_rows, bf16* k_win,
+                                                   bf16* v_win, int* status) {
   constexpr int E = D / 32;  // codes per lane: 8 or 16
   const int b = blockIdx.y;
-  const int64_t pos0 = seq_lens_before[b];
-  if (pos0 < 0 || (window == 0 && pos0 > cache_cap)) {
+  const int64_t pos0 = seq_lens_before ? (int64_t)seq_lens_before[b] : 0;
+  const int64_t rows = window > 0 ? (int64_t)window + extra : pos0 + extra;
+  if (pos0 < 0 || rows > win_rows || (window == 0 && rows > cache_cap)) {
     if (threadIdx.x == 0 && blockIdx.x == 0) set_status(status, GEMMA_ERR_DEVICE_RANGE);
     return;
   }
-  const int64_t rows = window > 0 ? window : pos0;
   const int lane = threadIdx.x & 31;
   const int64_t n_items = rows * Hkv;
   for (int64_t it = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5); it < n_items; it += (int64_t)gridDim.x * 8) {
@@ -481,18 +483,18 @@ cudaError_t launch_ring_gather(const bf16* k_cache, const bf16* v_cache, const i
 }
 
 cudaError_t launch_gather_q8(const uint8_t* k_codes, const float2* k_params, const uint8_t* v_codes,
-                             const float2* v_params, const int32_t* seq_lens_before, int B, int Hkv, int D,
-                             int window, int cache_cap, int win_rows, bf16* k_win, bf16* v_win, int* status,
-                             cudaStream_t st) {
-  const int64_t rows = window > 0 ? window : cache_cap;  // an upper bound; blocks stride over the rest
+                             const float2* v_params, const int32_t* seq_lens_before, int extra, int B, int Hkv,
+                             int D, int window, int cache_cap, int win_rows, bf16* k_win, bf16* v_win,
+                             int* status, cudaStream_t st) {
+  const int64_t rows = win_rows;  // an upper bound; blocks stride over the rest
   const int64_t blocks = std::min<int64_t>((rows * Hkv + 7) / 8, 1184);
   dim3 grid((unsigned)std::max<int64_t>(blocks, 1), B);
   if (D == 256)
-    k_gather_q8<256><<<grid, 256, 0, st>>>(k_codes, k_params, v_codes, v_params, seq_lens_before, Hkv, window,
-                                           cache_cap, win_rows, k_win, v_win, status);
+    k_gather_q8<256><<<grid, 256, 0, st>>>(k_codes, k_params, v_codes, v_params, seq_lens_before, extra, Hkv,
+                                           window, cache_cap, win_rows, k_win, v_win, status);
   else
-    k_gather_q8<512><<<grid, 256, 0, st>>>(k_codes, k_params, v_codes, v_params, seq_lens_before, Hkv, window,
-                                           cache_cap, win_rows, k_win, v_win, status);
+    k_gather_q8<512><<<grid, 256, 0, st>>>(k_codes, k_params, v_codes, v_params, seq_lens_before, extra, Hkv,
+                                           window, cache_cap, win_rows, k_win, v_win, status);
   return cudaGetLastError();
 }
 

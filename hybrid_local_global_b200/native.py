@@ -169,7 +169,8 @@ def gemma_attn_prefill(q, k_new, v_new, k_cache, v_cache, *, window, rope_frac, 
         flags |= GEMMA_F_KV_INT8
     if workspace is None:
         n = (gemma_attn_prefill_workspace_size_cached(B, S, Hq, Hkv, D, window, cap, flags)
-             if seq_lens_before is not None else gemma_attn_prefill_workspace_size(B, S, Hq, Hkv, D, window))
+             if seq_lens_before is not None or flags & GEMMA_F_SHARED
+             else gemma_attn_prefill_workspace_size(B, S, Hq, Hkv, D, window))
         workspace = torch.empty(max(n, 1), dtype=torch.uint8, device=q.device)
     return _check(_prefill(_ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_cache), _ptr(v_cache), cap,
                            _ptr(seq_lens_before), B, S, window, Hq, Hkv, D, rope_frac, rope_theta,

@@ -91,7 +91,8 @@ class AttentionStack:
         workload has cached tokens) sizes it for chunks after cached tokens."""
         w = self.w
         if after_cached is None:
-            after_cached = w.prior > 0
+            # int8 caches: a shared layer's prefill reads cached rows too
+            after_cached = w.prior > 0 or (w.kv_int8 and any(self.is_shared(l) for l in range(self.n_layers)))
         flags = native.GEMMA_F_KV_INT8 if w.kv_int8 else 0
         sizes = []
         for l in range(self.n_layers):

@@ -91,15 +91,15 @@ typedef enum gemma_status {
                              row gets codes 0 and step 0. Size the buffers with
                              gemma_kv_cache_bytes(..., GEMMA_F_KV_INT8);
                              cache_cap must be even. Prefill attends with the
-                             chunk's own bf16 K/V and writes codes; after
-                             cached tokens (seq_lens_before != NULL) the
-                             cached rows it also attends to are read back as
-                             min + code * step rounded to bf16 (a global
-                             layer then needs the larger workspace of
+                             chunk's own bf16 K/V and writes codes; the cached
+                             rows a chunk also attends to (after cached
+                             tokens, or every row on a GEMMA_F_SHARED layer)
+                             are read back as min + code * step rounded to
+                             bf16 (a global layer then needs the larger
+                             workspace of
                              gemma_attn_prefill_workspace_size_cached).
-                             Decode reads codes. Prefill with GEMMA_F_SHARED
-                             returns GEMMA_ERR_UNSUPPORTED. Combines with
-                             GEMMA_F_KEQV and, for decode, GEMMA_F_SHARED. */
+                             Decode reads codes. Combines with GEMMA_F_KEQV
+                             and GEMMA_F_SHARED. */
 
 /* Bytes of one layer's K (or V) cache buffer: batch * n_kv_heads *
  * cache_cap * head_dim * 2 for bf16; with GEMMA_F_KV_INT8 the codes, padded
@@ -140,11 +140,12 @@ size_t gemma_kv_codes_bytes(int batch, int n_kv_heads, int cache_cap, int head_d
 /* ---------------------------------------------------------------------- */
 size_t gemma_attn_prefill_workspace_size(int batch, int s_new, int n_q_heads,
                                          int n_kv_heads, int head_dim, int window);
-/* Workspace of a prefill after cached tokens (seq_lens_before != NULL) on  */
-/* a cache of capacity cache_cap: equal to the above, except that an int8  */
-/* global layer (GEMMA_F_KV_INT8 in flags, window 0) also holds its keys   */
-/* and values up to cache_cap rows in bf16 (2 * batch * cache_cap *        */
-/* n_kv_heads * head_dim * 2 bytes more). 0 on bad arguments.              */
+/* Workspace of a prefill that reads cached rows (seq_lens_before != NULL, */
+/* or a GEMMA_F_SHARED layer) on a cache of capacity cache_cap: equal to   */
+/* the above, except that an int8 global layer (GEMMA_F_KV_INT8 in flags,  */
+/* window 0) also holds its keys and values up to cache_cap rows in bf16   */
+/* (2 * batch * cache_cap * n_kv_heads * head_dim * 2 bytes more). 0 on    */
+/* bad arguments.                                                          */
 size_t gemma_attn_prefill_workspace_size_cached(int batch, int s_new, int n_q_heads,
                                                 int n_kv_heads, int head_dim, int window,
                                                 int cache_cap, unsigned flags);

@@ -150,7 +150,7 @@ PLAIN_WS_GLOBAL = native.gemma_attn_prefill_workspace_size(1, 16, 8, 4, 256, 0)
     (dict(flags=4, lens=FAKE, wsb=16), E.GEMMA_ERR_CAPACITY),          # int8 KV after cached tokens: accepted
     (dict(flags=4, W=0, cap=16384, lens=FAKE, wsb=PLAIN_WS_GLOBAL), E.GEMMA_ERR_CAPACITY),  # ... whose global
                                                                         # layers need the larger workspace
-    (dict(flags=5, k=None, v=None), E.GEMMA_ERR_UNSUPPORTED),          # int8 KV on a shared layer's prefill
+    (dict(flags=5, k=None, v=None, wsb=16), E.GEMMA_ERR_CAPACITY),     # int8 KV on a shared layer: accepted
     (dict(W=0, cap=4096, flags=6, v=None, wsb=16), E.GEMMA_ERR_CAPACITY),  # int8 K = V: accepted
     (dict(flags=2, v=None), E.GEMMA_ERR_UNSUPPORTED),  # K = V on a local layer
     (dict(W=0, cap=4096, flags=2), E.GEMMA_ERR_INVALID_ARG),             # K = V with v_new

@@ -349,3 +349,79 @@ def test_prefill_int8_after_cached_tokens(oracle, case):
 def test_prefill_int8_after_cached_tokens_k_equals_v(oracle):
     run_prefill_int8_chunk(oracle, before=[129, 700], S=130, Hq=8, Hkv=1, D=512, W=0, frac=0.25, theta=1e6,
                            seed=337, keqv=True)
+
+
+# ------------------------------------------------------- shared layer's prefill
+def run_prefill_int8_shared(oracle, *, before, S, Hq, Hkv, D, W, frac, theta, seed, keqv=False):
+    """A KV-shared layer's prefill on an int8 cache: its source has already
+    quantized every row, the chunk's included; the layer attends to all of
+    them dequantized and writes nothing."""
+    dev = torch.device("cuda")
+    B = len(before)
+    g = synth.generator(seed)
+    cap = W if W else max(before) + S + 16 + (max(before) + S) % 2
+    k_rows = synth.randn_bf16((B, Hkv, cap, D), g)
+    v_rows = k_rows if keqv else synth.randn_bf16((B, Hkv, cap, D), g)
+    q = synth.randn_bf16((B, S, Hq, D), g)
+    ck, pk = quantize(oracle, k_rows)
+    cv, pv = (ck, pk) if keqv else quantize(oracle, v_rows)
+    kc = native.Int8KVCache(B, Hkv, cap, D, dev)
+    kc.codes.copy_(ck)
+    kc.params.copy_(pk)
+    vc = kc
+    if not keqv:
+        vc = native.Int8KVCache(B, Hkv, cap, D, dev)
+        vc.codes.copy_(cv)
+        vc.params.copy_(pv)
+    out = torch.full((B, S, Hq, D), float("nan"), dtype=torch.bfloat16, device=dev)
+    scale = 1.0 / math.sqrt(D)
+    lens = torch.tensor(before, dtype=torch.int32, device=dev) if any(before) else None
+    native.gemma_attn_prefill(q.to(dev), None, None, kc, None if keqv else vc, window=W, rope_frac=frac,
+                              rope_theta=theta, scale=scale, out=out, seq_lens_before=lens,
+                              flags=native.GEMMA_F_SHARED | (native.GEMMA_F_KEQV if keqv else 0))
+    assert native.gemma_attn_sync_status() == 0, native.gemma_last_error()
+    assert torch.equal(kc.codes.cpu(), ck) and torch.equal(kc.params.cpu(), pk), "a shared layer writes nothing"
+    if not keqv:
+        assert torch.equal(vc.codes.cpu(), cv) and torch.equal(vc.params.cpu(), pv)
+    G = Hq // Hkv
+    out_c = out.float().cpu().double().numpy()
+    for b in range(B):
+        P0 = before[b]
+        lo = max(0, P0 - W) if W else 0
+        positions = list(range(lo, P0 + S))
+        n = len(positions)
+        keys = np.zeros((Hkv, n, D))
+        vals = np.zeros((Hkv, n, D))
+        for idx, p in enumerate(positions):
+            s = p % W if W else p
+            keys[:, idx] = dequant(oracle, ck[b, :, s], pk[b, :, s])
+            vals[:, idx] = dequant(oracle, cv[b, :, s], pv[b, :, s])
+        rows_q, begin, count = [], [], []
+        for i in range(S):
+            P = P0 + i
+            vis_lo = max(lo, P - W + 1) if W else 0
+            for h in range(Hq):
+                rows_q.append(oracle.rope_bf16(to_bits(q[b, i, h]), P, frac, theta))
+                begin.append((h // G) * n + (vis_lo - lo))
+                count.append(P - vis_lo + 1)
+        ref, _ = oracle.attend_rows(np.array(rows_q), keys.reshape(Hkv * n, D), vals.reshape(Hkv * n, D),
+                                    begin, count, scale)
+        assert_close(out_c[b].reshape(S * Hq, D), ref, 2e-2, 2e-3, what="int8 shared b=%d before=%d" % (b, P0))
+
+
+SHARED_CASES = [
+    dict(before=[300, 0], S=200, Hq=8, Hkv=1, D=512, W=0, frac=0.25, theta=1e6, seed=341),
+    dict(before=[0], S=300, Hq=32, Hkv=4, D=512, W=0, frac=0.25, theta=1e6, seed=342),
+    dict(before=[0, 0], S=100, Hq=8, Hkv=4, D=256, W=128, frac=1.0, theta=1e4, seed=343),
+    dict(before=[0], S=64, Hq=32, Hkv=16, D=256, W=64, frac=1.0, theta=1e4, seed=344),
+]
+
+
+@pytest.mark.parametrize("case", SHARED_CASES, ids=["global_prior", "global", "local", "local_full_ring"])
+def test_prefill_int8_shared_layer(oracle, case):
+    run_prefill_int8_shared(oracle, **case)
+
+
+def test_prefill_int8_shared_layer_k_equals_v(oracle):
+    run_prefill_int8_shared(oracle, before=[129], S=130, Hq=8, Hkv=1, D=512, W=0, frac=0.25, theta=1e6,
+                            seed=345, keqv=True)
