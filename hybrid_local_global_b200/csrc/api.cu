@@ -308,14 +308,29 @@ size_t gemma_kv_cache_bytes(int batch, int n_kv_heads, int cache_cap, int head_d
 
 // int8 cache rows of one call's new tokens: K from the rotated staging rows,
 // V from the caller's values (none under K = V)
+// Where a layer's cache rows live (see cache_row): a contiguous cache, or
+// the pages of a pool named by a page table (global layers).
+struct CacheLayout {
+  const int32_t* page_table;  // [batch][pages_per_seq], or null
+  int page_size, pages_per_seq, n_pages;
+};
+
+static CacheLayout contiguous(int cache_cap, int batch) { return CacheLayout{nullptr, cache_cap, 1, batch}; }
+
 // Quantize a chunk's rows into an int8 cache. Sources are [B][rows][Hkv][D]
 // with chunk token s at row s (mode 0), window + s (1) or its position (2);
 // V from the caller's layout [B][S][Hkv][D] (null under K = V).
 static cudaError_t quantize_kv(const bf16* k_src, int k_rows, int k_mode, const bf16* v_src, void* k_cache,
                                void* v_cache, int batch, int S, int Hkv, int D, int window, int cache_cap,
-                               const int32_t* pos0, int pos0_minus, int* status, cudaStream_t st) {
-  const size_t off = gemma_kv_codes_bytes(batch, Hkv, cache_cap, D);
+                               const int32_t* pos0, int pos0_minus, const CacheLayout& L, int* status,
+                               cudaStream_t st) {
+  // an int8 pool is laid out as an int8 cache of n_pages "sequences" of page_size rows
+  const size_t off = gemma_kv_codes_bytes(L.n_pages, Hkv, L.page_size, D);
   QuantRowsArgs qa{};
+  qa.page_table = L.page_table;
+  qa.page_size = L.page_size;
+  qa.pages_per_seq = L.pages_per_seq;
+  qa.n_pages = L.n_pages;
   qa.src_rows = k_rows;
   qa.src_row_mode = k_mode;
   qa.S = S;
@@ -355,15 +370,6 @@ size_t gemma_attn_prefill_workspace_size_cached(int batch, int s_new, int n_q_he
                           prefix ? cache_cap : 0);
 }
 
-// Where a layer's cache rows live (see cache_row): a contiguous cache, or
-// the pages of a pool named by a page table (global layers).
-struct CacheLayout {
-  const int32_t* page_table;  // [batch][pages_per_seq], or null
-  int page_size, pages_per_seq, n_pages;
-};
-
-static CacheLayout contiguous(int cache_cap, int batch) { return CacheLayout{nullptr, cache_cap, 1, batch}; }
-
 static int check_paged(const int32_t* page_table, int page_size, int pages_per_seq, int n_pages, unsigned flags) {
   if (!page_table) return fail(GEMMA_ERR_INVALID_ARG, "paged cache: null page table");
   if (page_size <= 0 || page_size % 128)
@@ -372,7 +378,6 @@ static int check_paged(const int32_t* page_table, int page_size, int pages_per_s
     return fail(GEMMA_ERR_INVALID_ARG, "paged cache: pages_per_seq %d, n_pages %d", pages_per_seq, n_pages);
   if ((int64_t)pages_per_seq * page_size > INT32_MAX)
     return fail(GEMMA_ERR_INVALID_ARG, "paged cache: pages_per_seq * page_size exceeds 2^31");
-  if (flags & GEMMA_F_KV_INT8) return fail(GEMMA_ERR_UNSUPPORTED, "paged cache: int8 rows are not paged in this build");
   return GEMMA_OK;
 }
 
@@ -435,7 +440,7 @@ static int prefill_impl(const void* q, const void* k_new, const void* v_new, voi
   ra.v_win = (win_local || prefix_q8) ? reinterpret_cast<bf16*>(ws + off_vw) : nullptr;
   ra.win_rows = win_rows;
   ra.win_at_pos = prefix_q8 ? 1 : 0;
-  const size_t codes_off = q8 ? gemma_kv_codes_bytes(batch, n_kv_heads, cache_cap, head_dim) : 0;
+  const size_t codes_off = q8 ? gemma_kv_codes_bytes(L.n_pages, n_kv_heads, L.page_size, head_dim) : 0;
   if (q8 && (win_local || prefix_q8)) {
     // before the chunk's rows are quantized into the cache: the cached rows
     // it attends to, dequantized, into the windows (K = V: K only). A shared
@@ -445,7 +450,8 @@ static int prefill_impl(const void* q, const void* k_new, const void* v_new, voi
     cudaError_t eg = launch_gather_q8(kc8, reinterpret_cast<const float2*>(kc8 + codes_off), vc8,
                                       vc8 ? reinterpret_cast<const float2*>(vc8 + codes_off) : nullptr,
                                       seq_lens_before, shared ? s_new : 0, batch, n_kv_heads, head_dim, window,
-                                      cache_cap, win_rows, ra.k_rot, ra.v_win, status, st);
+                                      cache_cap, L.page_table, L.page_size, L.pages_per_seq, L.n_pages, win_rows,
+                                      ra.k_rot, ra.v_win, status, st);
     if (eg != cudaSuccess) return cuda_fail(eg, "int8 window gather launch");
   } else if (chunked_local) {
     // before the chunk overwrites ring slots: old keys/values into rows 0..window-1
@@ -478,7 +484,7 @@ static int prefill_impl(const void* q, const void* k_new, const void* v_new, voi
   if (e == cudaSuccess && q8 && !shared)
     e = quantize_kv(ra.k_rot, win_rows ? win_rows : s_new, prefix_q8 ? 2 : chunked_local ? 1 : 0,
                     keqv ? nullptr : ra.v_new, k_cache, v_cache, batch, s_new, n_kv_heads, head_dim, window,
-                    cache_cap, seq_lens_before, 0, status, st);
+                    cache_cap, seq_lens_before, 0, L, status, st);
   p_rope.done();
   if (e != cudaSuccess) return cuda_fail(e, "prefill rope launch");
 
@@ -646,7 +652,7 @@ static int decode_impl(const void* q, const void* k_new, const void* v_new, void
   cudaError_t e = launch_decode_rope_append(ra, batch, head_dim, st);
   if (e == cudaSuccess && q8 && k_new)
     e = quantize_kv(ra.k_stage, 1, 0, (flags & GEMMA_F_KEQV) ? nullptr : ra.v_new, k_cache, v_cache, batch, 1,
-                    n_kv_heads, head_dim, window, cache_cap, seq_lens, 1, status, st);
+                    n_kv_heads, head_dim, window, cache_cap, seq_lens, 1, L, status, st);
   p_app.done();
   if (e != cudaSuccess) return cuda_fail(e, "decode append launch");
 
@@ -675,7 +681,7 @@ static int decode_impl(const void* q, const void* k_new, const void* v_new, void
   da.pages_per_seq = L.pages_per_seq;
   da.n_pages = L.n_pages;
   if (q8) {
-    const size_t off = gemma_kv_codes_bytes(batch, n_kv_heads, cache_cap, head_dim);
+    const size_t off = gemma_kv_codes_bytes(L.n_pages, n_kv_heads, L.page_size, head_dim);
     da.k_codes = static_cast<const uint8_t*>(k_cache);
     da.v_codes = static_cast<const uint8_t*>(v_cache);
     da.k_params = reinterpret_cast<const float2*>(static_cast<const uint8_t*>(k_cache) + off);

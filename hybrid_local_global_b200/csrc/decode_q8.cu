@@ -159,9 +159,10 @@ __global__ void __launch_bounds__(32 * (NCW + 1), 2)
   // keys per ring slot: 16 K rows + 16 V rows, or 32 K rows under K = V
   const int kps = a.keqv ? 2 * C::KB : C::KB;
   const int n_sub = (int)((k_end - k_begin + kps - 1) / kps);
-  const int64_t row0 = ((int64_t)b * a.Hkv + g) * (int64_t)a.cache_cap;  // first cache row of (b, g)
-  const float2* kpar = a.k_params + row0;
-  const float2* vpar = a.keqv ? kpar : a.v_params + row0;
+  // (min, step) rows, addressed like the codes by cache_row (a paged pool
+  // or, without a table, the contiguous cache)
+  const float2* kpar = a.k_params;
+  const float2* vpar = a.keqv ? kpar : a.v_params;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::NSLOT; ++s) {
@@ -195,6 +196,20 @@ __global__ void __launch_bounds__(32 * (NCW + 1), 2)
         const int np = (nk + 1) & ~1;
         const bool drop = a.drop_first_copy && t == 0 && split == 0 && g == 0 && b == 0;
         if (drop) continue;
+        // the slot's page and first row in it (a slot never straddles a page:
+        // pages hold a multiple of 128 rows, slots start at multiples of 16/32)
+        int pg = b;
+        int prow = (int)key0;
+        if (a.page_table) {
+          const int pi = (int)key0 / a.page_size;
+          pg = a.page_table[(int64_t)b * a.pages_per_seq + pi];
+          prow = (int)key0 - pi * a.page_size;
+          if (pg < 0 || pg >= a.n_pages) {  // a page outside the pool: report it, read page 0
+            set_status(a.status, GEMMA_ERR_DEVICE_RANGE);
+            pg = 0;
+          }
+        }
+        const int64_t par0 = ((int64_t)pg * a.Hkv + g) * a.page_size + prow;
         // regions that hold rows: K and V, or (K = V) the first 16 K rows and,
         // when there are more, the next 16
         const int n_reg = a.keqv ? (nk > C::KB ? 2 : 1) : 2;
@@ -205,14 +220,14 @@ __global__ void __launch_bounds__(32 * (NCW + 1), 2)
         const uint32_t bar = smem_u32(&full[slot]);
         for (int r = 0; r < n_reg; ++r) {
           const CUtensorMap* m = (a.keqv || r == 0) ? &tm_k : &tm_v;
-          const int y = (int)key0 + (a.keqv ? r * C::KB : 0);  // rows past the capacity read as 0
+          const int y = prow + (a.keqv ? r * C::KB : 0);  // rows past the page read as 0
 #pragma unroll
           for (int ch = 0; ch < C::NCH; ++ch)
-            tc::tma_load_4d(dst + r * C::REGION_B + ch * C::BOX_B, m, ch * 128, y, g, b, bar);
+            tc::tma_load_4d(dst + r * C::REGION_B + ch * C::BOX_B, m, ch * 128, y, g, pg, bar);
         }
         unsigned char* pdst = pring + slot * C::PAR_B;
-        bulk_g2s(pdst, kpar + key0, (uint32_t)(np * 8), &full[slot]);
-        if (!a.keqv) bulk_g2s(pdst + C::KB * 8, vpar + key0, (uint32_t)(np * 8), &full[slot]);
+        bulk_g2s(pdst, kpar + par0, (uint32_t)(np * 8), &full[slot]);
+        if (!a.keqv) bulk_g2s(pdst + C::KB * 8, vpar + par0, (uint32_t)(np * 8), &full[slot]);
       }
     }
   } else {
@@ -232,7 +247,10 @@ __global__ void __launch_bounds__(32 * (NCW + 1), 2)
         qmax = fmaxf(qmax, fmaxf(fabsf(f.x), fabsf(f.y)));
       }
     }
-    for (int64_t k = k_begin + threadIdx.x; k < k_end; k += 32 * NCW) vmax = fmaxf(vmax, vpar[k].y);
+    for (int64_t k = k_begin + threadIdx.x; k < k_end; k += 32 * NCW) {
+      const int64_t r = cache_row(a.page_table, a.pages_per_seq, a.page_size, a.n_pages, a.Hkv, b, g, k);
+      if (r >= 0) vmax = fmaxf(vmax, vpar[r].y);  // (a page outside the pool: the producer reports it)
+    }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
       qmax = fmaxf(qmax, __shfl_xor_sync(0xffffffffu, qmax, o));
@@ -491,11 +509,13 @@ __global__ void __launch_bounds__(32 * (NCW + 1), 2)
 template <int D>
 cudaError_t launch_q8(const DecodeAttnArgs& a, int B, cudaStream_t st) {
   using C = Q8Cfg<D>;
-  // codes [B][Hkv][cap][D] bytes as 4-D maps (dims innermost first), tiles of
-  // 128 bytes x 16 rows
+  // codes [pages][Hkv][page_size][D] bytes (a contiguous cache: B pages of
+  // its capacity) as 4-D maps (dims innermost first), tiles of 128 bytes x
+  // 16 rows
   CUtensorMap mk, mv;
-  const uint64_t dims[4] = {(uint64_t)D, (uint64_t)a.cache_cap, (uint64_t)a.Hkv, (uint64_t)B};
-  const uint64_t str[3] = {(uint64_t)D, (uint64_t)a.cache_cap * D, (uint64_t)a.Hkv * a.cache_cap * D};
+  const uint64_t ps = (uint64_t)a.page_size;
+  const uint64_t dims[4] = {(uint64_t)D, ps, (uint64_t)a.Hkv, (uint64_t)a.n_pages};
+  const uint64_t str[3] = {(uint64_t)D, ps * D, (uint64_t)a.Hkv * ps * D};
   const uint32_t box[4] = {128, (uint32_t)C::KB, 1, 1};
   if (!make_map_u8_4d(&mk, a.k_codes, dims, str, box)) return cudaErrorInvalidValue;
   if (a.keqv)

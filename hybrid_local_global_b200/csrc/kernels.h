@@ -69,11 +69,13 @@ struct QuantRowsArgs {
   const bf16* src;     // [B][src_rows][Hkv][D]; chunk token s at row s (src_row_mode 0),
   int src_rows;        // window + s (1) or its position (2)
   int src_row_mode;
-  int S, Hkv, window, cache_cap;
+  int S, Hkv, window, cache_cap;  // cache_cap: positions per sequence (range check)
   const int32_t* pos0;  // device [B], or null for 0
   int pos0_minus;
-  uint8_t* codes;
+  uint8_t* codes;       // rows addressed by cache_row (codes [rows][D], params [rows])
   float2* params;
+  const int32_t* page_table;  // null: contiguous (page_size = cache_cap, n_pages = B)
+  int page_size, pages_per_seq, n_pages;
   int* status;
 };
 
@@ -146,9 +148,12 @@ cudaError_t launch_ring_gather(const bf16* k_cache, const bf16* v_cache, const i
 // ring's positions pos0-window .. pos0+extra-1 into rows 0.. (negative
 // positions: zeros); window 0: positions 0 .. pos0+extra-1 into rows 0.. .
 // v_codes null: K only.
+// Cached rows are addressed by cache_row (page_table null: contiguous,
+// page_size = cache_cap, n_pages = B).
 cudaError_t launch_gather_q8(const uint8_t* k_codes, const float2* k_params, const uint8_t* v_codes,
                              const float2* v_params, const int32_t* seq_lens_before, int extra, int B, int Hkv,
-                             int D, int window, int cache_cap, int win_rows, bf16* k_win, bf16* v_win,
+                             int D, int window, int cache_cap, const int32_t* page_table, int page_size,
+                             int pages_per_seq, int n_pages, int win_rows, bf16* k_win, bf16* v_win,
                              int* status, cudaStream_t st);
 cudaError_t launch_decode_rope_append(const DecodeRopeArgs& a, int B, int D, cudaStream_t st);
 cudaError_t launch_quantize_rows(const QuantRowsArgs& a, int B, int D, cudaStream_t st);

@@ -264,8 +264,9 @@ __global__ void __launch_bounds__(256) k_gather_q8(const uint8_t* __restrict__ k
                                                    const uint8_t* __restrict__ v_codes,
                                                    const float2* __restrict__ v_params,
                                                    const int32_t* seq_lens_before, int extra, int Hkv,
-                                                   int window, int cache_cap, int win_rows, bf16* k_win,
-                                                   bf16* v_win, int* status) {
+                                                   int window, int cache_cap, const int32_t* page_table,
+                                                   int page_size, int pages_per_seq, int n_pages, int win_rows,
+                                                   bf16* k_win, bf16* v_win, int* status) {
   constexpr int E = D / 32;  // codes per lane: 8 or 16
   const int b = blockIdx.y;
   const int64_t pos0 = seq_lens_before ? (int64_t)seq_lens_before[b] : 0;
@@ -284,11 +285,13 @@ __global__ void __launch_bounds__(256) k_gather_q8(const uint8_t* __restrict__ k
     for (int kv = 0; kv < (v_codes ? 2 : 1); ++kv) {
       bf16* out = (kv ? v_win : k_win) + dst;
       uint32_t packed[E / 2];
-      if (p < 0) {
+      const int64_t crow =
+          p < 0 ? -1 : cache_row(page_table, pages_per_seq, page_size, n_pages, Hkv, b, h, window > 0 ? p % window : p);
+      if (p >= 0 && crow < 0 && lane == 0) set_status(status, GEMMA_ERR_DEVICE_RANGE);  // page outside the pool
+      if (crow < 0) {
 #pragma unroll
         for (int i = 0; i < E / 2; ++i) packed[i] = 0;
       } else {
-        const int64_t crow = ((int64_t)b * Hkv + h) * cache_cap + (window > 0 ? p % window : p);
         const float2 mp = (kv ? v_params : k_params)[crow];
         const uint8_t* cp = (kv ? v_codes : k_codes) + crow * D + lane * E;
         uint32_t w[E / 4];
@@ -431,7 +434,11 @@ __global__ void __launch_bounds__(256) k_quantize_rows(QuantRowsArgs a, int n_ro
       packed[e / 4] |= (uint32_t)c << (8 * (e % 4));
     }
   }
-  const int64_t crow = ((int64_t)b * a.Hkv + h) * a.cache_cap + slot;
+  const int64_t crow = cache_row(a.page_table, a.pages_per_seq, a.page_size, a.n_pages, a.Hkv, b, h, slot);
+  if (crow < 0) {  // a page outside the pool: report, write nothing
+    if (lane == 0) set_status(a.status, GEMMA_ERR_DEVICE_RANGE);
+    return;
+  }
   uint8_t* dst = a.codes + crow * D + lane * E;
   if (E == 8)
     *reinterpret_cast<uint2*>(dst) = make_uint2(packed[0], packed[1]);
@@ -484,17 +491,20 @@ cudaError_t launch_ring_gather(const bf16* k_cache, const bf16* v_cache, const i
 
 cudaError_t launch_gather_q8(const uint8_t* k_codes, const float2* k_params, const uint8_t* v_codes,
                              const float2* v_params, const int32_t* seq_lens_before, int extra, int B, int Hkv,
-                             int D, int window, int cache_cap, int win_rows, bf16* k_win, bf16* v_win,
+                             int D, int window, int cache_cap, const int32_t* page_table, int page_size,
+                             int pages_per_seq, int n_pages, int win_rows, bf16* k_win, bf16* v_win,
                              int* status, cudaStream_t st) {
   const int64_t rows = win_rows;  // an upper bound; blocks stride over the rest
   const int64_t blocks = std::min<int64_t>((rows * Hkv + 7) / 8, 1184);
   dim3 grid((unsigned)std::max<int64_t>(blocks, 1), B);
   if (D == 256)
     k_gather_q8<256><<<grid, 256, 0, st>>>(k_codes, k_params, v_codes, v_params, seq_lens_before, extra, Hkv,
-                                           window, cache_cap, win_rows, k_win, v_win, status);
+                                           window, cache_cap, page_table, page_size, pages_per_seq, n_pages,
+                                           win_rows, k_win, v_win, status);
   else
     k_gather_q8<512><<<grid, 256, 0, st>>>(k_codes, k_params, v_codes, v_params, seq_lens_before, extra, Hkv,
-                                           window, cache_cap, win_rows, k_win, v_win, status);
+                                           window, cache_cap, page_table, page_size, pages_per_seq, n_pages,
+                                           win_rows, k_win, v_win, status);
   return cudaGetLastError();
 }
 

@@ -214,14 +214,19 @@ def _paged_args(k_pool, page_table):
 def gemma_attn_prefill_paged(q, k_new, v_new, k_pool, v_pool, page_table, *, rope_frac, rope_theta, scale, out,
                              seq_lens_before=None, lse=None, workspace=None, flags=0, stream=None):
     """Global layer on a paged cache: pools [n_pages, Hkv, page_size, D]
-    (bf16), page_table int32 [B, pages_per_seq] on the device."""
+    (bf16, or Int8KVCache(n_pages, Hkv, page_size, D) buffers), page_table
+    int32 [B, pages_per_seq] on the device."""
     for t, n in ((q, "q"), (k_new, "k_new"), (v_new, "v_new"), (k_pool, "k_pool"), (v_pool, "v_pool"),
                  (out, "out")):
         _bf16(t, n)
     B, S, Hq, D = q.shape
     n_pages, Hkv, ps, pps = _paged_args(k_pool, page_table)
+    if isinstance(k_pool, Int8KVCache):
+        flags |= GEMMA_F_KV_INT8
     if workspace is None:
-        n = gemma_attn_prefill_workspace_size(B, S, Hq, Hkv, D, 0)
+        n = (gemma_attn_prefill_workspace_size_cached(B, S, Hq, Hkv, D, 0, ps * pps, flags)
+             if seq_lens_before is not None or flags & GEMMA_F_SHARED
+             else gemma_attn_prefill_workspace_size(B, S, Hq, Hkv, D, 0))
         workspace = torch.empty(max(n, 1), dtype=torch.uint8, device=q.device)
     return _check(_prefill_paged(_ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_pool), _ptr(v_pool), _ptr(page_table),
                                  ps, pps, n_pages, _ptr(seq_lens_before), B, S, Hq, Hkv, D, rope_frac, rope_theta,
@@ -239,6 +244,8 @@ def gemma_attn_decode_paged(q, k_new, v_new, k_pool, v_pool, page_table, *, seq_
         raise TypeError("seq_lens must be an int32 CUDA tensor")
     B, Hq, D = q.shape
     n_pages, Hkv, ps, pps = _paged_args(k_pool, page_table)
+    if isinstance(k_pool, Int8KVCache):
+        flags |= GEMMA_F_KV_INT8
     if workspace is None:
         n = gemma_attn_decode_workspace_size(B, Hq, Hkv, D, 0, max_seq_len)
         workspace = torch.empty(max(n, 1), dtype=torch.uint8, device=q.device)

@@ -206,8 +206,13 @@ int gemma_attn_decode(const void* q, const void* k_new, const void* v_new,
 /*        layers pass their source's pool and table. The caller owns the  */
 /*        pool, the table and page allocation.                            */
 /* page_size: a multiple of 128. pages_per_seq * page_size is the         */
-/*        per-sequence capacity (the bound on seq_lens). GEMMA_F_KV_INT8   */
-/*        returns GEMMA_ERR_UNSUPPORTED.                                  */
+/*        per-sequence capacity (the bound on seq_lens).                   */
+/* GEMMA_F_KV_INT8: each pool is an int8 cache buffer of n_pages           */
+/*        "sequences" of page_size rows: codes [n_pages][n_kv_heads]       */
+/*        [page_size][head_dim], then (min, step) at byte offset           */
+/*        gemma_kv_codes_bytes(n_pages, n_kv_heads, page_size, head_dim);  */
+/*        size it with gemma_kv_cache_bytes(n_pages, n_kv_heads,           */
+/*        page_size, head_dim, GEMMA_F_KV_INT8).                           */
 /* ---------------------------------------------------------------------- */
 int gemma_attn_prefill_paged(const void* q, const void* k_new, const void* v_new,
                              void* k_pool, void* v_pool, const int32_t* page_table,

@@ -226,6 +226,10 @@ def test_kv_cache_bytes():
     assert native.gemma_kv_codes_bytes(1, 1, 0, 256) == 0
 
 
+# the plain workspace of the paged prefill harness's shapes
+PAGED_PLAIN_WS = native.gemma_attn_prefill_workspace_size(2, 16, 8, 1, 512, 0)
+
+
 def _prefill_paged_raw(**over):
     a = dict(q=FAKE, k=FAKE, v=FAKE, kc=FAKE, vc=FAKE, table=FAKE, ps=128, pps=64, npages=256, lens=None, B=2,
              S=16, Hq=8, Hkv=1, D=512, frac=0.25, theta=1e6, scale=0.044, out=FAKE, lse=None, ws=FAKE,
@@ -253,7 +257,9 @@ def _decode_paged_raw(**over):
     (dict(ps=0), E.GEMMA_ERR_INVALID_ARG),
     (dict(pps=0), E.GEMMA_ERR_INVALID_ARG),
     (dict(npages=0), E.GEMMA_ERR_INVALID_ARG),
-    (dict(flags=4), E.GEMMA_ERR_UNSUPPORTED),              # int8 rows are not paged
+    (dict(flags=4, wsb=16), E.GEMMA_ERR_CAPACITY),         # int8 pools accepted
+    (dict(flags=4, lens=FAKE, wsb=PAGED_PLAIN_WS), E.GEMMA_ERR_CAPACITY),  # ... after cached tokens they
+                                                                          # need the larger workspace
     (dict(pps=1, S=200), E.GEMMA_ERR_CAPACITY),            # chunk beyond pages_per_seq * page_size
     (dict(flags=2, v=None, vc=None, wsb=16), E.GEMMA_ERR_CAPACITY),   # K = V accepted
 ])
@@ -266,7 +272,7 @@ def test_prefill_paged_validation(over, code):
     (dict(wsb=1024), E.GEMMA_ERR_CAPACITY),                # accepted
     (dict(table=None), E.GEMMA_ERR_INVALID_ARG),
     (dict(ps=192), E.GEMMA_ERR_INVALID_ARG),
-    (dict(flags=4), E.GEMMA_ERR_UNSUPPORTED),
+    (dict(flags=4, wsb=1024), E.GEMMA_ERR_CAPACITY),      # int8 pools accepted
     (dict(pps=8), E.GEMMA_ERR_CAPACITY),                   # 8 pages of 256 < max_seq_len 4096
     (dict(flags=1, k=None, v=None, wsb=1024), E.GEMMA_ERR_CAPACITY),  # shared layer accepted
 ])

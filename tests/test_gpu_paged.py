@@ -222,3 +222,95 @@ def test_page_outside_the_pool_is_reported():
                                    rope_theta=1e6, scale=0.044, out=out)
     assert native.gemma_attn_sync_status() == 0, native.gemma_last_error()
     assert torch.isfinite(out.float()).all()
+
+
+# ------------------------------------------------------------- int8 pools
+def int8_pool_from(cache, table, ps, n_pages, dev):
+    """An Int8KVCache pool (n_pages "sequences" of ps rows) holding, page by
+    page, the rows of a contiguous Int8KVCache; other pages hold 0xAB."""
+    B, Hkv, cap, D = cache.shape
+    pool = native.Int8KVCache(n_pages, Hkv, ps, D, dev, fill=0xAB)
+    codes, params = cache.codes.cpu(), cache.params.cpu()
+    pc, pp = pool.codes.cpu(), pool.params.cpu()
+    for b in range(B):
+        for p in range(table.shape[1]):
+            pc[int(table[b, p])] = codes[b, :, p * ps:(p + 1) * ps]
+            pp[int(table[b, p])] = params[b, :, p * ps:(p + 1) * ps]
+    pool.codes.copy_(pc)
+    pool.params.copy_(pp)
+    return pool
+
+
+def assert_int8_pool_matches(pool, cache, table, ps, n_pages):
+    pc, pp = pool.codes.cpu(), pool.params.cpu()
+    assert torch.equal(from_pool(pc, table, ps), cache.codes.cpu())
+    assert torch.equal(from_pool(pp, table, ps).view(torch.int32), cache.params.cpu().view(torch.int32))
+    free = ~owned_mask(table, n_pages)
+    assert (pc[free] == 0xAB).all()
+
+
+def seeded_int8_cache(oracle, B, Hkv, cap, D, g, dev):
+    """A contiguous int8 cache holding the oracle's quantization of seeded rows."""
+    c = native.Int8KVCache(B, Hkv, cap, D, dev)
+    codes, lo, step = oracle.quantize_rows_u8(to_bits(synth.randn_bf16((B, Hkv, cap, D), g)))
+    c.codes.copy_(torch.from_numpy(codes))
+    c.params.copy_(torch.from_numpy(np.stack([lo, step], axis=-1)))
+    return c
+
+
+@pytest.mark.parametrize("keqv", [False, True], ids=["kv", "keqv"])
+def test_decode_paged_int8_matches_contiguous(oracle, keqv):
+    dev = torch.device("cuda")
+    lens, Hq, Hkv, D, ps = [1, 300, 4097, 129], 32, 4, 512, 256
+    B = len(lens)
+    g = synth.generator(421)
+    pps = (max(lens) + ps - 1) // ps + 1
+    cap, n_pages = pps * ps, B * pps + 3
+    kc = seeded_int8_cache(oracle, B, Hkv, cap, D, g, dev)
+    vc = kc if keqv else seeded_int8_cache(oracle, B, Hkv, cap, D, g, dev)
+    table = make_table(B, pps, n_pages, 421)
+    kp = int8_pool_from(kc, table, ps, n_pages, dev)
+    vp = kp if keqv else int8_pool_from(vc, table, ps, n_pages, dev)
+    q = synth.randn_bf16((B, Hq, D), g).to(dev)
+    kn = synth.randn_bf16((B, Hkv, D), g).to(dev)
+    vn = None if keqv else synth.randn_bf16((B, Hkv, D), g).to(dev)
+    sl = torch.tensor(lens, dtype=torch.int32, device=dev)
+    kw = dict(seq_lens=sl, max_seq_len=max(lens), rope_frac=0.25, rope_theta=1e6, scale=1 / math.sqrt(D),
+              flags=native.GEMMA_F_KEQV if keqv else 0)
+    out_c = torch.full((B, Hq, D), float("nan"), dtype=torch.bfloat16, device=dev)
+    out_p = torch.full_like(out_c, float("nan"))
+    native.gemma_attn_decode(q, kn, vn, kc, None if keqv else vc, window=0, out=out_c, **kw)
+    native.gemma_attn_decode_paged(q, kn, vn, kp, None if keqv else vp, table.to(dev), out=out_p, **kw)
+    assert native.gemma_attn_sync_status() == 0, native.gemma_last_error()
+    assert torch.equal(bits(out_p), bits(out_c))
+    assert_int8_pool_matches(kp, kc, table, ps, n_pages)
+    if not keqv:
+        assert_int8_pool_matches(vp, vc, table, ps, n_pages)
+
+
+@pytest.mark.parametrize("prior", [None, [700, 0, 129]], ids=["fresh", "after_cached"])
+def test_prefill_paged_int8_matches_contiguous(oracle, prior):
+    dev = torch.device("cuda")
+    B, S, Hq, Hkv, D, ps = 3, 200, 8, 1, 512, 128
+    before = prior or [0] * B
+    g = synth.generator(422)
+    pps = (max(before) + S + ps - 1) // ps + 1
+    cap, n_pages = pps * ps, B * pps + 2
+    kc = seeded_int8_cache(oracle, B, Hkv, cap, D, g, dev)
+    vc = seeded_int8_cache(oracle, B, Hkv, cap, D, g, dev)
+    table = make_table(B, pps, n_pages, 422)
+    kp = int8_pool_from(kc, table, ps, n_pages, dev)
+    vp = int8_pool_from(vc, table, ps, n_pages, dev)
+    q = synth.randn_bf16((B, S, Hq, D), g).to(dev)
+    k = synth.randn_bf16((B, S, Hkv, D), g).to(dev)
+    v = synth.randn_bf16((B, S, Hkv, D), g).to(dev)
+    lens = torch.tensor(prior, dtype=torch.int32, device=dev) if prior else None
+    kw = dict(rope_frac=0.25, rope_theta=1e6, scale=1 / math.sqrt(D), seq_lens_before=lens)
+    out_c = torch.full((B, S, Hq, D), float("nan"), dtype=torch.bfloat16, device=dev)
+    out_p = torch.full_like(out_c, float("nan"))
+    native.gemma_attn_prefill(q, k, v, kc, vc, window=0, out=out_c, **kw)
+    native.gemma_attn_prefill_paged(q, k, v, kp, vp, table.to(dev), out=out_p, **kw)
+    assert native.gemma_attn_sync_status() == 0, native.gemma_last_error()
+    assert torch.equal(bits(out_p), bits(out_c))
+    assert_int8_pool_matches(kp, kc, table, ps, n_pages)
+    assert_int8_pool_matches(vp, vc, table, ps, n_pages)
