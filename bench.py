@@ -16,6 +16,12 @@ the batched decode block named by --decode-workload (default: 31B-shaped,
 and `bf16_equivalent_gbs`: the bf16 bytes the same keys would take, per
 second).
 
+Each part runs two timed passes of the same steps, both bracketed by a
+barrier and a synchronize and timed with CUDA events on the stream: the step
+time comes from an uninstrumented pass; the per-kernel device times of the
+roofline (`kernels`, `roofline.achieved`) come from the second pass, where
+the library records events around every launch.
+
 --impl reference times the fp64 CPU oracle (the path's reference
 implementation here) on the host cores, each step a bounded sample of rows
 of the same workload.
@@ -172,6 +178,45 @@ def kernel_totals(native):
     return res
 
 
+def timed_passes(native, step, args, world, dev, before_step=None):
+    """Two timed passes of args.steps steps each, bracketed by a barrier and a
+    synchronize: the first, uninstrumented, gives the step time (`value`);
+    the second records the library's CUDA events around each launch
+    (gemma_attn_profile) for the per-kernel device times of the roofline.
+    The events cost a few microseconds of serialisation per launch, so they
+    stay out of the step time. -> (step ms summed over steps, max over ranks;
+    wall seconds of the first pass; per-kernel totals; clock record)."""
+    def run(evs):
+        barrier(world)
+        torch.cuda.synchronize()
+        t0 = time.perf_counter()
+        for a, b in evs:
+            if before_step is not None:
+                before_step()
+            a.record()
+            step()
+            b.record()
+        torch.cuda.synchronize()
+        wall = time.perf_counter() - t0
+        barrier(world)
+        return wall
+
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    evs2 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            for _ in range(args.steps)]
+    with ClockSampler(dev.index or 0) as clk:
+        wall = run(evs)
+        native.gemma_attn_profile(True)
+        run(evs2)
+    rc = native.gemma_attn_sync_status()
+    assert rc == 0, native.gemma_last_error()
+    dev_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in evs), world)
+    kern = kernel_totals(native)
+    native.gemma_attn_profile(False)
+    return dev_ms, wall, kern, clk
+
+
 def bench_prefill(args, w, dev, world, peaks):
     from hybrid_local_global_b200 import native
     st, layers, ws, lens = make_prefill(w, dev)
@@ -186,27 +231,7 @@ def bench_prefill(args, w, dev, world, peaks):
         step()
     torch.cuda.synchronize()
     assert native.gemma_attn_sync_status() == 0, native.gemma_last_error()
-    native.gemma_attn_profile(True)
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in range(args.steps)]
-    with ClockSampler(dev.index or 0) as clk:
-        barrier(world)
-        torch.cuda.synchronize()
-        t0 = time.perf_counter()
-        for a, b in evs:
-            flush.zero_()
-            a.record()
-            step()
-            b.record()
-        torch.cuda.synchronize()
-        wall = time.perf_counter() - t0
-        barrier(world)
-    rc = native.gemma_attn_sync_status()
-    assert rc == 0, native.gemma_last_error()
-    dev_ms = sum(a.elapsed_time(b) for a, b in evs)
-    kern = kernel_totals(native)
-    native.gemma_attn_profile(False)
-    dev_ms_max = max_over_ranks(dev_ms, world)
+    dev_ms_max, wall, kern, clk = timed_passes(native, step, args, world, dev, before_step=flush.zero_)
     flops = prefill_flops(w, st.is_global)
     value = world * flops * args.steps / (dev_ms_max / 1e3) / 1e12
     attn = kern.get("prefill_attn", {"ms": float("nan"), "launches": 0})
@@ -217,7 +242,8 @@ def bench_prefill(args, w, dev, world, peaks):
             "peak_source": "%s bf16 burst (MEASURED_PEAKS.json)" % peaks[1] if peaks[1] == "measured"
             else "fallback 1.59 PF/s", "traffic": None,
             "per_launch": "algorithmic FLOPs of all attention launches / their summed device time "
-                          "(%d launches, %d per step)" % (attn["launches"], st.n_layers)}
+                          "(%d launches, %d per step; CUDA events around each launch, in a second timed "
+                          "pass of the same steps)" % (attn["launches"], st.n_layers)}
     # the kernel that runs each layer type: CTA pairs on head_dim 512 (both
     # model shapes have an even number of q heads per KV head), one CTA per
     # query tile on head_dim 256
@@ -338,22 +364,7 @@ def bench_decode(args, w, dev, world, peaks):
         step()
     torch.cuda.synchronize()
     assert native.gemma_attn_sync_status() == 0, native.gemma_last_error()
-    native.gemma_attn_profile(True)
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in range(args.steps)]
-    with ClockSampler(dev.index or 0) as clk:
-        barrier(world)
-        torch.cuda.synchronize()
-        for a, b in evs:
-            a.record()
-            step()
-            b.record()
-        torch.cuda.synchronize()
-        barrier(world)
-    assert native.gemma_attn_sync_status() == 0, native.gemma_last_error()
-    dev_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in evs), world)
-    kern = kernel_totals(native)
-    native.gemma_attn_profile(False)
+    dev_ms, _, kern, clk = timed_passes(native, step, args, world, dev)
     nbytes = decode_bytes(w, st, lens_cpu)
     kv_bytes = sum(visible_kv_bytes(st, l, lens_cpu) for l in range(st.n_layers))
     value = world * nbytes * args.steps / (dev_ms / 1e3) / 1e9
@@ -364,7 +375,8 @@ def bench_decode(args, w, dev, world, peaks):
             "peak": peak, "unit": "GB/s", "frac": round(achieved / peak, 4),
             "peak_source": "%s HBM copy (MEASURED_PEAKS.json)" % peaks[1], "traffic": None,
             "per_launch": "visible K (and V unless K = V) bytes of all split launches / their summed device time "
-                          "(%d launches, %d per step)" % (sp["launches"], st.n_layers)}
+                          "(%d launches, %d per step; CUDA events around each launch, in a second timed pass "
+                          "of the same steps)" % (sp["launches"], st.n_layers)}
     rec = recorded_traffic("k_decode_split_q8" if w.kv_int8 else "k_decode_split")
     if rec:
         # each layer takes the traffic/algorithmic ratio captured for its layer
