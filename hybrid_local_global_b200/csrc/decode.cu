@@ -93,7 +93,9 @@ __device__ __forceinline__ int key_of(int n) {
   return (n % NG) * RPC + n / NG;
 }
 
-template <int D, int RPC>
+// PAGED: the cache is a pool named by a.page_table (see cache_row); the
+// contiguous instance keeps the plain row arithmetic of one (b, g) range.
+template <int D, int RPC, bool PAGED>
 __global__ void __launch_bounds__(32 * (NCW + 1), 2) k_decode_split(DecodeAttnArgs a) {
   using C = DecCfg<D, RPC>;
   extern __shared__ __align__(128) unsigned char sm[];
@@ -126,6 +128,7 @@ __global__ void __launch_bounds__(32 * (NCW + 1), 2) k_decode_split(DecodeAttnAr
   const int n_sub = (int)((k_end - k_begin + kps - 1) / kps);
   // a sub-block's rows are contiguous: pages hold a multiple of 32 rows and
   // sub-blocks start at multiples of 16 (32 under K = V)
+  const int64_t head_off = PAGED ? 0 : ((int64_t)b * a.Hkv + g) * (int64_t)a.cache_cap * D;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::NSLOT; ++s) {
@@ -165,13 +168,17 @@ __global__ void __launch_bounds__(32 * (NCW + 1), 2) k_decode_split(DecodeAttnAr
       const int nk = (int)((k_end - key0) < kps ? (k_end - key0) : kps);
       const bool drop = a.drop_first_copy && t == 0 && split == 0 && g == 0 && b == 0;
       if (drop) continue;
-      int64_t brow = cache_row(a.page_table, a.pages_per_seq, a.page_size, a.n_pages, a.Hkv, b, g, key0);
-      if (brow < 0) {  // a page outside the pool: report it and read pool row 0 (finite, wrong)
-        if (lane == 0) set_status(a.status, GEMMA_ERR_DEVICE_RANGE);
-        brow = 0;
+      int64_t boff = head_off + key0 * D;  // element offset of the sub-block's first row
+      if constexpr (PAGED) {
+        int64_t brow = cache_row(a.page_table, a.pages_per_seq, a.page_size, a.n_pages, a.Hkv, b, g, key0);
+        if (brow < 0) {  // a page outside the pool: report it and read pool row 0 (finite, wrong)
+          if (lane == 0) set_status(a.status, GEMMA_ERR_DEVICE_RANGE);
+          brow = 0;
+        }
+        boff = brow * D;
       }
-      const bf16* kbase = a.k_cache + brow * D;
-      const bf16* vbase = a.v_cache + brow * D;
+      const bf16* kbase = a.k_cache + boff;
+      const bf16* vbase = a.v_cache + boff;
       if (lane == 0) {
         mbar_arrive_expect_tx(&full[slot], (uint32_t)((a.keqv ? 1 : 2) * nk * D * 2));
         issued[slot] += 1;
@@ -410,13 +417,19 @@ __global__ void __launch_bounds__(128) k_decode_combine(DecodeAttnArgs a) {
   }
 }
 
+template <int D, int RPC, bool PAGED>
+cudaError_t launch_split_as(const DecodeAttnArgs& a, int B, cudaStream_t st) {
+  using C = DecCfg<D, RPC>;
+  cudaError_t e = cudaFuncSetAttribute(k_decode_split<D, RPC, PAGED>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       C::SMEM);
+  if (e != cudaSuccess) return e;
+  k_decode_split<D, RPC, PAGED><<<dim3(a.n_splits, a.Hkv, B), 32 * (NCW + 1), C::SMEM, st>>>(a);
+  return cudaGetLastError();
+}
+
 template <int D, int RPC>
 cudaError_t launch_split(const DecodeAttnArgs& a, int B, cudaStream_t st) {
-  using C = DecCfg<D, RPC>;
-  cudaError_t e = cudaFuncSetAttribute(k_decode_split<D, RPC>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
-  if (e != cudaSuccess) return e;
-  k_decode_split<D, RPC><<<dim3(a.n_splits, a.Hkv, B), 32 * (NCW + 1), C::SMEM, st>>>(a);
-  return cudaGetLastError();
+  return a.page_table ? launch_split_as<D, RPC, true>(a, B, st) : launch_split_as<D, RPC, false>(a, B, st);
 }
 
 }  // namespace

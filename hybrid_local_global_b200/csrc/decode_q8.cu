@@ -122,7 +122,9 @@ __device__ __forceinline__ float pow2_ceil(float x) {
   return ldexpf(1.f, m == 0.5f ? e - 1 : e);
 }
 
-template <int D>
+// PAGED: the cache is a pool named by a.page_table (see cache_row); the
+// contiguous instance keeps the plain row arithmetic of one (b, g) range.
+template <int D, bool PAGED>
 __global__ void __launch_bounds__(32 * (NCW + 1), 2)
     k_decode_split_q8(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                       DecodeAttnArgs a) {
@@ -159,10 +161,11 @@ __global__ void __launch_bounds__(32 * (NCW + 1), 2)
   // keys per ring slot: 16 K rows + 16 V rows, or 32 K rows under K = V
   const int kps = a.keqv ? 2 * C::KB : C::KB;
   const int n_sub = (int)((k_end - k_begin + kps - 1) / kps);
-  // (min, step) rows, addressed like the codes by cache_row (a paged pool
-  // or, without a table, the contiguous cache)
-  const float2* kpar = a.k_params;
-  const float2* vpar = a.keqv ? kpar : a.v_params;
+  // (min, step) rows, addressed like the codes: from the first row of (b, g)
+  // in a contiguous cache, through cache_row in a pool
+  const int64_t row0 = PAGED ? 0 : ((int64_t)b * a.Hkv + g) * (int64_t)a.cache_cap;
+  const float2* kpar = a.k_params + row0;
+  const float2* vpar = (a.keqv ? a.k_params : a.v_params) + row0;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::NSLOT; ++s) {
@@ -200,7 +203,8 @@ __global__ void __launch_bounds__(32 * (NCW + 1), 2)
         // pages hold a multiple of 128 rows, slots start at multiples of 16/32)
         int pg = b;
         int prow = (int)key0;
-        if (a.page_table) {
+        int64_t par0 = key0;  // (min, step) row of key0, from kpar / vpar
+        if constexpr (PAGED) {
           const int pi = (int)key0 / a.page_size;
           pg = a.page_table[(int64_t)b * a.pages_per_seq + pi];
           prow = (int)key0 - pi * a.page_size;
@@ -208,8 +212,8 @@ __global__ void __launch_bounds__(32 * (NCW + 1), 2)
             set_status(a.status, GEMMA_ERR_DEVICE_RANGE);
             pg = 0;
           }
+          par0 = ((int64_t)pg * a.Hkv + g) * a.page_size + prow;
         }
-        const int64_t par0 = ((int64_t)pg * a.Hkv + g) * a.page_size + prow;
         // regions that hold rows: K and V, or (K = V) the first 16 K rows and,
         // when there are more, the next 16
         const int n_reg = a.keqv ? (nk > C::KB ? 2 : 1) : 2;
@@ -248,8 +252,12 @@ __global__ void __launch_bounds__(32 * (NCW + 1), 2)
       }
     }
     for (int64_t k = k_begin + threadIdx.x; k < k_end; k += 32 * NCW) {
-      const int64_t r = cache_row(a.page_table, a.pages_per_seq, a.page_size, a.n_pages, a.Hkv, b, g, k);
-      if (r >= 0) vmax = fmaxf(vmax, vpar[r].y);  // (a page outside the pool: the producer reports it)
+      if constexpr (PAGED) {
+        const int64_t r = cache_row(a.page_table, a.pages_per_seq, a.page_size, a.n_pages, a.Hkv, b, g, k);
+        if (r >= 0) vmax = fmaxf(vmax, vpar[r].y);  // (a page outside the pool: the producer reports it)
+      } else {
+        vmax = fmaxf(vmax, vpar[k].y);
+      }
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
@@ -522,9 +530,10 @@ cudaError_t launch_q8(const DecodeAttnArgs& a, int B, cudaStream_t st) {
     mv = mk;
   else if (!make_map_u8_4d(&mv, a.v_codes, dims, str, box))
     return cudaErrorInvalidValue;
-  cudaError_t e = cudaFuncSetAttribute(k_decode_split_q8<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  auto kern = a.page_table ? k_decode_split_q8<D, true> : k_decode_split_q8<D, false>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
-  k_decode_split_q8<D><<<dim3(a.n_splits, a.Hkv, B), 32 * (NCW + 1), C::SMEM, st>>>(mk, mv, a);
+  kern<<<dim3(a.n_splits, a.Hkv, B), 32 * (NCW + 1), C::SMEM, st>>>(mk, mv, a);
   return cudaGetLastError();
 }
 
