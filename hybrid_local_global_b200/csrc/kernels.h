@@ -29,8 +29,9 @@ struct PrefillRopeArgs {
   int n_rot;           // rotated pairs
   double log2_theta;
   float q_scale;       // rotated Q is multiplied by this before the bf16 rounding
-  int quant;           // int8 cache: rotated K goes to k_rot ([B][S][Hkv][D]) on every layer
-                       // type and nothing is written into the cache (launch_quantize_rows does)
+  int quant;           // int8 cache: rotated K goes to k_rot ([B][S][Hkv][D], or its window rows
+                       // with win_rows > 0) on every layer type and nothing is written into the
+                       // cache (launch_quantize_rows does)
   // cache pages (see cache_row): table [B][pages_per_seq] or null for a
   // contiguous cache (page_size = cache_cap, n_pages = B)
   const int32_t* page_table;
@@ -109,9 +110,9 @@ struct PrefillAttnArgs {
 
 struct DecodeAttnArgs {
   const bf16* q_rot;       // [B][Hq][D]
-  const bf16* k_cache;     // [B][Hkv][cap][D]
+  const bf16* k_cache;     // [B][Hkv][cap][D], or a pool [n_pages][Hkv][page_size][D]
   const bf16* v_cache;
-  int cache_cap;
+  int cache_cap;           // positions per sequence
   const int32_t* seq_lens; // device [B]
   int max_len, window, Hq, Hkv;
   int chunk;               // keys per split (multiple of 16)
@@ -124,7 +125,8 @@ struct DecodeAttnArgs {
   unsigned long long wait_ns;
   int drop_first_copy;     // test hook: skip the first K/V copy of split 0
   int keqv;                // K = V: only K rows are loaded and serve as V
-  // int8 cache (k_cache/v_cache unused): codes [B][Hkv][cap][D] and per-row (min, step)
+  // int8 cache (k_cache/v_cache unused): codes [B][Hkv][cap][D] and per-row (min, step),
+  // or the same over the pages of a pool
   const uint8_t* k_codes;
   const uint8_t* v_codes;
   const float2* k_params;
