@@ -425,3 +425,73 @@ def test_prefill_int8_shared_layer(oracle, case):
 def test_prefill_int8_shared_layer_k_equals_v(oracle):
     run_prefill_int8_shared(oracle, before=[129], S=130, Hq=8, Hkv=1, D=512, W=0, frac=0.25, theta=1e6,
                             seed=345, keqv=True)
+
+
+# ------------------------------------------------- the benchmarked int8 block
+def test_decode_31b_b64_int8_sampled(oracle):
+    """The 31B-shaped decode block on int8 caches, as bench.py times it (B64,
+    KV lengths U[4096,131072], 5 local + 1 global layer, layer 4 sharing
+    layer 3), with seeded synthetic codes and (min, step) rows. Sampled
+    sequences (rows are independent) are held to the oracle over the
+    dequantized rows; global-layer samples are kept to at most 40000 keys so
+    that the fp64 key arrays stay small."""
+    from hybrid_local_global_b200.stack import AttentionStack
+    from hybrid_local_global_b200.workloads import WORKLOADS
+    w = WORKLOADS["31b_decode_b64_int8"]
+    dev = torch.device("cuda")
+    st = AttentionStack(w, dev)
+    lens_cpu = synth.decode_lengths(w.batch, w.len_lo, w.len_hi, seed=w.seed)
+    lens = lens_cpu.to(dev)
+    max_len = int(lens_cpu.max())
+    g = synth.generator(w.seed, "cuda")
+    owned = set()
+    for l in range(st.n_layers):
+        if not st.is_shared(l) and st.k_cache[l].data_ptr() not in owned:
+            owned.add(st.k_cache[l].data_ptr())
+            synth.fill_int8_cache_(st.k_cache[l], g)
+            if st.v_cache[l] is not st.k_cache[l]:
+                synth.fill_int8_cache_(st.v_cache[l], g)
+    ws = torch.empty(st.decode_workspace_bytes(max_len), dtype=torch.uint8, device=dev)
+    rng = np.random.default_rng(w.seed)
+    pick = set(rng.choice(w.batch, size=4, replace=False).tolist()) | {int(lens_cpu.argmin())}
+    for l in range(st.n_layers):
+        t = st.layer_type(l)
+        D, Hkv, W = t.head_dim, t.n_kv_heads, t.window
+        G = w.n_q_heads // Hkv
+        q = synth.randn_bf16((w.batch, w.n_q_heads, D), g, "cuda")
+        kn = synth.randn_bf16((w.batch, Hkv, D), g, "cuda")
+        vn = synth.randn_bf16((w.batch, Hkv, D), g, "cuda")
+        shared = st.is_shared(l)
+        checked = [b for b in sorted(pick) if W or int(lens_cpu[b]) <= 40000]
+        kc, vc = st.k_cache[l], st.v_cache[l]
+        snaps = {}
+        for b in checked:
+            n = min(kc.shape[2], int(lens_cpu[b]))
+            snaps[b] = (kc.codes[b, :, :n].cpu(), kc.params[b, :, :n].cpu(),
+                        vc.codes[b, :, :n].cpu(), vc.params[b, :, :n].cpu())
+        out = torch.empty((w.batch, w.n_q_heads, D), dtype=torch.bfloat16, device=dev)
+        st.decode_layer(l, q, kn, vn, out, seq_lens=lens, max_seq_len=max_len, workspace=ws)
+        assert native.gemma_attn_sync_status() == 0, native.gemma_last_error()
+        for b in checked:
+            L = int(lens_cpu[b])
+            ck, pk, cv, pv = snaps[b]
+            slot_new = (L - 1) % W if W else L - 1
+            if shared:  # the source layer has appended this step's rows already
+                nk_c, nk_p, nv_c, nv_p = ck[:, slot_new], pk[:, slot_new], cv[:, slot_new], pv[:, slot_new]
+            else:
+                nk_c, nk_p = quantize(oracle, rotated_bf16(oracle, kn[b].cpu(), L - 1, t.rope_frac, t.rope_theta))
+                nv_c, nv_p = quantize(oracle, vn[b].cpu())
+            positions = np.arange(max(0, L - W) if W else 0, L)
+            n = len(positions)
+            slots = torch.from_numpy(positions % W if W else positions)
+            keys = dequant(oracle, ck[:, slots], pk[:, slots])  # [Hkv, n, D]
+            vals = dequant(oracle, cv[:, slots], pv[:, slots])
+            keys[:, n - 1] = dequant(oracle, nk_c, nk_p)          # position L - 1: this step's rows
+            vals[:, n - 1] = dequant(oracle, nv_c, nv_p)
+            qrot = np.stack([oracle.rope_bf16(to_bits(q[b, h].cpu()), L - 1, t.rope_frac, t.rope_theta)
+                             for h in range(w.n_q_heads)])
+            ref, _ = oracle.attend_rows(qrot, keys.reshape(Hkv * n, D), vals.reshape(Hkv * n, D),
+                                        [(h // G) * n for h in range(w.n_q_heads)], [n] * w.n_q_heads, t.scale)
+            assert_close(out[b].float().cpu().double().numpy(), ref,
+                         what="31b int8 layer %d b=%d len=%d" % (l, b, L))
+        del snaps
