@@ -370,7 +370,7 @@ size_t gemma_attn_prefill_workspace_size_cached(int batch, int s_new, int n_q_he
                           prefix ? cache_cap : 0);
 }
 
-static int check_paged(const int32_t* page_table, int page_size, int pages_per_seq, int n_pages, unsigned flags) {
+static int check_paged(const int32_t* page_table, int page_size, int pages_per_seq, int n_pages) {
   if (!page_table) return fail(GEMMA_ERR_INVALID_ARG, "paged cache: null page table");
   if (page_size <= 0 || page_size % 128)
     return fail(GEMMA_ERR_INVALID_ARG, "paged cache: page_size %d must be a positive multiple of 128", page_size);
@@ -576,7 +576,7 @@ int gemma_attn_prefill_paged(const void* q, const void* k_new, const void* v_new
                              int n_kv_heads, int head_dim, float rope_frac, float rope_theta, float scale,
                              void* out, float* lse, void* workspace, size_t workspace_bytes, unsigned flags,
                              void* stream) {
-  int rc = check_paged(page_table, page_size, pages_per_seq, n_pages, flags);
+  int rc = check_paged(page_table, page_size, pages_per_seq, n_pages);
   if (rc) return rc;
   return prefill_impl(q, k_new, v_new, k_pool, v_pool, pages_per_seq * page_size, seq_lens_before, batch, s_new,
                       0, n_q_heads, n_kv_heads, head_dim, rope_frac, rope_theta, scale, out, lse, workspace,
@@ -717,7 +717,7 @@ int gemma_attn_decode_paged(const void* q, const void* k_new, const void* v_new,
                             const int32_t* seq_lens, int max_seq_len, int batch, int n_q_heads, int n_kv_heads,
                             int head_dim, float rope_frac, float rope_theta, float scale, void* out,
                             void* workspace, size_t workspace_bytes, unsigned flags, void* stream) {
-  int rc = check_paged(page_table, page_size, pages_per_seq, n_pages, flags);
+  int rc = check_paged(page_table, page_size, pages_per_seq, n_pages);
   if (rc) return rc;
   return decode_impl(q, k_new, v_new, k_pool, v_pool, pages_per_seq * page_size, seq_lens, max_seq_len, batch, 0,
                      n_q_heads, n_kv_heads, head_dim, rope_frac, rope_theta, scale, out, workspace, workspace_bytes,
