@@ -495,3 +495,28 @@ def test_decode_31b_b64_int8_sampled(oracle):
             assert_close(out[b].float().cpu().double().numpy(), ref,
                          what="31b int8 layer %d b=%d len=%d" % (l, b, L))
         del snaps
+
+
+def test_decode_int8_bounded_wait_times_out_and_context_survives(oracle):
+    """The int8 decode's first copy is not issued, so a barrier is never
+    completed: the bounded wait gives up after its deadline, the status says
+    so, and the next calls on the same context are correct."""
+    native.gemma_attn_set_wait_limit(20_000_000)  # 20 ms
+    try:
+        native.gemma_attn_debug_drop_next_copy(True)
+        dev = torch.device("cuda")
+        B, Hq, Hkv, D, L = 1, 8, 1, 512, 2000
+        g = synth.generator(350, "cuda")
+        kc = synth.fill_int8_cache_(native.Int8KVCache(B, Hkv, L + 16, D, dev), g)
+        vc = synth.fill_int8_cache_(native.Int8KVCache(B, Hkv, L + 16, D, dev), g)
+        q = synth.randn_bf16((B, Hq, D), g, "cuda")
+        kn = synth.randn_bf16((B, Hkv, D), g, "cuda")
+        vn = synth.randn_bf16((B, Hkv, D), g, "cuda")
+        out = torch.empty((B, Hq, D), dtype=torch.bfloat16, device=dev)
+        sl = torch.tensor([L], dtype=torch.int32, device=dev)
+        native.gemma_attn_decode(q, kn, vn, kc, vc, seq_lens=sl, max_seq_len=L, window=0, rope_frac=0.25,
+                                 rope_theta=1e6, scale=0.05, out=out)
+        assert native.gemma_attn_sync_status() == native.GEMMA_ERR_DEVICE_TIMEOUT
+    finally:
+        native.gemma_attn_set_wait_limit(0)
+    run_decode_int8(oracle, lens=[2000, 37], Hq=8, Hkv=1, D=512, W=0, frac=0.25, theta=1e6, seed=351)
