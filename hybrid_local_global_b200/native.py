@@ -130,6 +130,15 @@ class Int8KVCache:
         return self.buf.numel()
 
 
+def _kv_kind(k_cache, v_cache) -> int:
+    """GEMMA_F_KV_INT8 when the caches are Int8KVCache buffers, else 0; both
+    caches (v_cache may be None under K = V) must be of one kind."""
+    q8 = isinstance(k_cache, Int8KVCache)
+    if v_cache is not None and isinstance(v_cache, Int8KVCache) != q8:
+        raise TypeError("k_cache and v_cache must both be Int8KVCache buffers or both bf16 tensors")
+    return GEMMA_F_KV_INT8 if q8 else 0
+
+
 def _stream(stream):
     if stream is None:
         stream = torch.cuda.current_stream()
@@ -165,8 +174,7 @@ def gemma_attn_prefill(q, k_new, v_new, k_cache, v_cache, *, window, rope_frac, 
         _bf16(t, n)
     B, S, Hq, D = q.shape
     _, Hkv, cap, _ = k_cache.shape
-    if isinstance(k_cache, Int8KVCache):
-        flags |= GEMMA_F_KV_INT8
+    flags |= _kv_kind(k_cache, v_cache)
     if workspace is None:
         n = (gemma_attn_prefill_workspace_size_cached(B, S, Hq, Hkv, D, window, cap, flags)
              if seq_lens_before is not None or flags & GEMMA_F_SHARED
@@ -193,8 +201,7 @@ def gemma_attn_decode(q, k_new, v_new, k_cache, v_cache, *, seq_lens, max_seq_le
         raise TypeError("seq_lens must be an int32 CUDA tensor")
     B, Hq, D = q.shape
     _, Hkv, cap, _ = k_cache.shape
-    if isinstance(k_cache, Int8KVCache):
-        flags |= GEMMA_F_KV_INT8
+    flags |= _kv_kind(k_cache, v_cache)
     if workspace is None:
         n = gemma_attn_decode_workspace_size(B, Hq, Hkv, D, window, max_seq_len)
         workspace = torch.empty(max(n, 1), dtype=torch.uint8, device=q.device)
@@ -221,8 +228,7 @@ def gemma_attn_prefill_paged(q, k_new, v_new, k_pool, v_pool, page_table, *, rop
         _bf16(t, n)
     B, S, Hq, D = q.shape
     n_pages, Hkv, ps, pps = _paged_args(k_pool, page_table)
-    if isinstance(k_pool, Int8KVCache):
-        flags |= GEMMA_F_KV_INT8
+    flags |= _kv_kind(k_pool, v_pool)
     if workspace is None:
         n = (gemma_attn_prefill_workspace_size_cached(B, S, Hq, Hkv, D, 0, ps * pps, flags)
              if seq_lens_before is not None or flags & GEMMA_F_SHARED
@@ -244,8 +250,7 @@ def gemma_attn_decode_paged(q, k_new, v_new, k_pool, v_pool, page_table, *, seq_
         raise TypeError("seq_lens must be an int32 CUDA tensor")
     B, Hq, D = q.shape
     n_pages, Hkv, ps, pps = _paged_args(k_pool, page_table)
-    if isinstance(k_pool, Int8KVCache):
-        flags |= GEMMA_F_KV_INT8
+    flags |= _kv_kind(k_pool, v_pool)
     if workspace is None:
         n = gemma_attn_decode_workspace_size(B, Hq, Hkv, D, 0, max_seq_len)
         workspace = torch.empty(max(n, 1), dtype=torch.uint8, device=q.device)

@@ -279,3 +279,17 @@ def test_prefill_paged_validation(over, code):
 def test_decode_paged_validation(over, code):
     assert _decode_paged_raw(**over) == code
     assert native.gemma_last_error()
+
+
+def test_binding_rejects_mixed_cache_kinds():
+    """An int8 key cache with a bf16 value cache (or the reverse) would be read
+    with the wrong layout: the binding refuses it before any call."""
+    import torch
+    i8 = native.Int8KVCache(1, 1, 16, 256, "cpu")
+    bf = torch.zeros((1, 1, 16, 256), dtype=torch.bfloat16)
+    assert native._kv_kind(i8, i8) == native.GEMMA_F_KV_INT8
+    assert native._kv_kind(i8, None) == native.GEMMA_F_KV_INT8   # K = V
+    assert native._kv_kind(bf, bf) == 0
+    for k, v in ((i8, bf), (bf, i8)):
+        with pytest.raises(TypeError):
+            native._kv_kind(k, v)
