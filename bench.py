@@ -2,19 +2,27 @@
 """Benchmark of the interleaved local/global attention path on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload NAME] [--decode-workload NAME|none]
-                    [--decode-int8-workload NAME|none]
+                    [--workload NAME] [--extra-prefill A,B|none]
+                    [--decode-workload NAME|none] [--decode-int8-workload NAME|none]
+                    [--extra-decode A,B|none]
 
 One JSON line on rank 0. A step is one pass of the prefill block named by
---workload (default: the E2B-shaped 5-layer block, B1 S8192: layer schedule,
-RoPE + cache write, attention for every layer) over resident synthetic
-inputs; `value` is its algorithmic TFLOP/s (4*B*Hq*D per visible query-key
-pair, masked pairs not counted) over all ranks. The `decode` object measures
-the batched decode block named by --decode-workload (default: 31B-shaped,
-6 layers, B64, KV lengths U[4096,131072], last two layers shared) in KV GB/s;
-`decode_int8` the same block on int8 KV caches (GB/s of the int8 rows read,
-and `bf16_equivalent_gbs`: the bf16 bytes the same keys would take, per
-second).
+--workload (default: the 31B-shaped 6-layer block, B2 S32768, 5 local + 1
+global: layer schedule, RoPE + cache write, attention for every layer) over
+resident synthetic inputs; `value` is its algorithmic TFLOP/s (4*B*Hq*D per
+visible query-key pair, masked pairs not counted) over all ranks.
+
+Every other workload shape gets an object of its own, with its step time,
+roofline and oracle baseline:
+  configs.<name>  the prefill workloads of --extra-prefill (default: the
+                  single local layer B1 S1024, the E2B-shaped block B1 S8192,
+                  the 4096-query chunk against a 256K global cache) and the
+                  decode workloads of --extra-decode (default: single-token
+                  decode at 256K), in TFLOP/s or KV GB/s;
+  decode          the 31B-shaped batched decode block (B64, KV lengths
+                  U[4096,131072], 6 layers, last two shared) in KV GB/s;
+  decode_int8     the same block on int8 KV caches (GB/s of the int8 rows
+                  read, and `bf16_equivalent_gbs`).
 
 Each part runs two timed passes of the same steps, both bracketed by a
 barrier and a synchronize and timed with CUDA events on the stream: the step
@@ -22,13 +30,15 @@ time comes from an uninstrumented pass; the per-kernel device times of the
 roofline (`kernels`, `roofline.achieved`) come from the second pass, where
 the library records events around every launch.
 
---impl reference times the fp64 CPU oracle (the path's reference
-implementation here) on the host cores, each step a bounded sample of rows
-of the same workload.
+`cpu_baseline` objects time the fp64 CPU oracle on the host cores over a
+bounded, seeded sample of rows (prefill) or sequences (decode) of the same
+workload and inputs. --impl reference times the oracle alone, on the
+headline workload, each step a bounded sample of its rows.
 """
 from __future__ import annotations
 
 import argparse
+import concurrent.futures as cf
 import json
 import os
 import statistics
@@ -48,6 +58,9 @@ from hybrid_local_global_b200.workloads import WORKLOADS, prefill_flops, visible
 
 METRIC = "attention prefill TFLOP/s and decode KV GB/s on 1 B200, as % of roofline"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+HEADLINE = "31b_block_s32768"
+EXTRA_PREFILL = "local_s1024,e2b_block_s8192,global_chunk_256k"
+EXTRA_DECODE = "global_decode_256k"
 
 
 def load_peaks():
@@ -56,6 +69,19 @@ def load_peaks():
         d = json.load(open(p))
         return d, "measured"
     return dict(FALLBACK_PEAKS), "fallback"
+
+
+# A timed pass this long runs the tensor cores under the 1 kW power cap, as
+# the sustained GEMM loop of the measured peaks did; shorter passes compare
+# with the burst figure.
+SUSTAINED_AFTER_S = 1.0
+
+
+def tensor_peak(peaks, timed_s):
+    d, src = peaks
+    if timed_s >= SUSTAINED_AFTER_S and "bf16_tflops_sustained" in d:
+        return d["bf16_tflops_sustained"], "%s bf16 sustained (MEASURED_PEAKS.json; timed pass %.1f s)" % (src, timed_s)
+    return d["bf16_tflops"], "%s bf16 burst (MEASURED_PEAKS.json; timed pass %.2f s)" % (src, timed_s)
 
 
 # --------------------------------------------------------------------------- clocks
@@ -132,18 +158,24 @@ def max_over_ranks(x: float, world: int) -> float:
     return RANKS.max_over_ranks(x)
 
 
-# --------------------------------------------------------------------------- prefill (ours)
+# --------------------------------------------------------------------------- inputs
+def draw_prefill_layer(w, t, g, dev):
+    """One layer's q, k, v (k scaled by the workload's k_scale), drawn in the
+    workload's order: q, then k, then v."""
+    q = synth.randn_bf16((w.batch, w.seq, w.n_q_heads, t.head_dim), g, dev)
+    k = synth.randn_bf16((w.batch, w.seq, t.n_kv_heads, t.head_dim), g, dev, scale=w.k_scale)
+    v = synth.randn_bf16((w.batch, w.seq, t.n_kv_heads, t.head_dim), g, dev)
+    return q, k, v
+
+
 def make_prefill(w, dev):
     from hybrid_local_global_b200.stack import AttentionStack
     st = AttentionStack(w, dev)
     g = synth.generator(w.seed, dev)
     layers = []
     for l in range(st.n_layers):
-        t = st.layer_type(l)
-        q = synth.randn_bf16((w.batch, w.seq, w.n_q_heads, t.head_dim), g, dev)
-        k = synth.randn_bf16((w.batch, w.seq, t.n_kv_heads, t.head_dim), g, dev, scale=w.k_scale)
-        v = synth.randn_bf16((w.batch, w.seq, t.n_kv_heads, t.head_dim), g, dev)
-        out = torch.empty((w.batch, w.seq, w.n_q_heads, t.head_dim), dtype=torch.bfloat16, device=dev)
+        q, k, v = draw_prefill_layer(w, st.layer_type(l), g, dev)
+        out = torch.empty_like(q)
         if w.prior and not st.is_shared(l):
             synth.fill_randn_bf16_(st.k_cache[l][:, :, :w.prior], g)
             synth.fill_randn_bf16_(st.v_cache[l][:, :, :w.prior], g)
@@ -217,7 +249,8 @@ def timed_passes(native, step, args, world, dev, before_step=None):
     return dev_ms, wall, kern, clk
 
 
-def bench_prefill(args, w, dev, world, peaks):
+# --------------------------------------------------------------------------- prefill (ours)
+def bench_prefill(args, w, dev, world, peaks, e2e=False, cpu=False):
     from hybrid_local_global_b200 import native
     st, layers, ws, lens = make_prefill(w, dev)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
@@ -236,11 +269,11 @@ def bench_prefill(args, w, dev, world, peaks):
     value = world * flops * args.steps / (dev_ms_max / 1e3) / 1e12
     attn = kern.get("prefill_attn", {"ms": float("nan"), "launches": 0})
     achieved = flops * args.steps / (attn["ms"] / 1e3) / 1e12
-    peak = peaks[0]["bf16_tflops"]
+    peak, peak_source = tensor_peak(peaks, dev_ms_max / 1e3)
+    burst = peaks[0]["bf16_tflops"]
     roof = {"bound": "tensor", "kernel": "prefill attention", "achieved": round(achieved, 2),
-            "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
-            "peak_source": "%s bf16 burst (MEASURED_PEAKS.json)" % peaks[1] if peaks[1] == "measured"
-            else "fallback 1.59 PF/s", "traffic": None,
+            "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4), "peak_source": peak_source,
+            "frac_of_burst": round(achieved / burst, 4), "traffic": None,
             "per_launch": "algorithmic FLOPs of all attention launches / their summed device time "
                           "(%d launches, %d per step; CUDA events around each launch, in a second timed "
                           "pass of the same steps)" % (attn["launches"], st.n_layers)}
@@ -260,11 +293,19 @@ def bench_prefill(args, w, dev, world, peaks):
     else:
         roof["traffic_note"] = "no ncu capture of the current kernel sources for this workload"
     launches = sum(v["launches"] for v in kern.values())
-    res = dict(value=value, ms_per_step=dev_ms_max / args.steps, roofline=roof, kernels=kern,
-               gpu_launches=launches, clocks=clk.summary(), wall_s=wall, flops_per_step=flops)
-    if not args.no_e2e:
+    res = {"metric": "prefill attention TFLOP/s", "value": round(value, 3), "unit": "TFLOP/s",
+           "workload": w.name, "description": w.description,
+           "ms_per_step": round(dev_ms_max / args.steps, 4), "flops_per_step": flops,
+           "layers": ["global" if g else "local" for g in st.is_global],
+           "roofline": roof, "kernels": kern, "gpu_launches": launches, "clocks": clk.summary(),
+           "wall_s": round(wall, 3)}
+    if e2e:
         res["e2e"] = e2e_prefill(args, st, layers, ws, lens, flops, world)
-    return res, st, layers
+    if cpu:
+        res["cpu_baseline"] = prefill_cpu_baseline(w, st.is_global, layers, st, args.cpu_flops)
+    del layers, st, ws, flush
+    torch.cuda.empty_cache()
+    return res
 
 
 def e2e_prefill(args, st, layers, ws, lens, flops, world):
@@ -272,15 +313,22 @@ def e2e_prefill(args, st, layers, ws, lens, flops, world):
     AttentionStack.prefill_from_host copies every layer's q/k/v from pinned
     host memory and every output back inside the timed region, overlapping
     the two copy directions with the attention on separate streams."""
-    host_in = [tuple(x.cpu().pin_memory() for x in (q, k, v)) for (q, k, v, _) in layers]
-    host_out = [torch.empty(out.shape, dtype=out.dtype, pin_memory=True) for (_, _, _, out) in layers]
+    host_in, host_out = [], []
+    for (q, k, v, out) in layers:
+        hs = []
+        for x in (q, k, v):
+            h = torch.empty(x.shape, dtype=x.dtype, pin_memory=True)
+            h.copy_(x)
+            hs.append(h)
+        host_in.append(tuple(hs))
+        host_out.append(torch.empty(out.shape, dtype=out.dtype, pin_memory=True))
     h2d = sum(x.numel() * x.element_size() for t in host_in for x in t)
     d2h = sum(x.numel() * x.element_size() for x in host_out)
 
     def step():
         st.prefill_from_host(host_in, host_out, layers, workspace=ws, seq_lens_before=lens)
 
-    for _ in range(max(1, args.warmup)):
+    for _ in range(max(1, min(args.warmup, 2))):
         step()
     torch.cuda.synchronize()
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
@@ -293,9 +341,83 @@ def e2e_prefill(args, st, layers, ws, lens, flops, world):
     torch.cuda.synchronize()
     barrier(world)
     ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in evs), world)
+    del host_in, host_out
     return {"value": round(world * flops * args.steps / (ms / 1e3) / 1e12, 3), "unit": "TFLOP/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
             "ms_per_step": round(ms / args.steps, 4)}
+
+
+# --------------------------------------------------------------------------- oracle on prefill rows
+def rows_for_budget(w, is_global, flops_budget):
+    """Sampled rows per layer so that the oracle's work is about flops_budget
+    (split evenly over the layers), capped at every row of the layer."""
+    per_layer = flops_budget / max(1, len(is_global))
+    total_rows = w.batch * w.n_q_heads * w.seq
+    out = []
+    for g in is_global:
+        t = w.global_ if g else w.local
+        per_row = 4 * t.head_dim * visible_pairs_prefill(w.seq, w.prior, t.window) / w.seq
+        out.append(int(min(total_rows, max(64, per_layer // per_row))))
+    return out
+
+
+def sample_rows(w, n, seed):
+    """n seeded rows (b, h, i), uniform over the layer's rows; every row when
+    n covers them all."""
+    total = w.batch * w.n_q_heads * w.seq
+    if n >= total:
+        bb, hh, ii = np.meshgrid(np.arange(w.batch), np.arange(w.n_q_heads), np.arange(w.seq), indexing="ij")
+        return np.stack([bb.ravel(), hh.ravel(), ii.ravel()], axis=1).astype(np.int32)
+    rng = np.random.default_rng(seed)
+    return np.stack([rng.integers(0, w.batch, n), rng.integers(0, w.n_q_heads, n),
+                     rng.integers(0, w.seq, n)], axis=1).astype(np.int32)
+
+
+def oracle_prefill_rows(w, t, q, k, v, rows):
+    """Times the oracle on `rows` of one layer (q [B,S,Hq,D], k/v [B,T,Hkv,D]
+    bf16 bits in position order, the first w.prior keys already rotated);
+    returns (seconds, algorithmic FLOPs of those rows)."""
+    import oracle
+    t0 = time.perf_counter()
+    oracle.attention(q, k, v, q_pos0=w.prior, n_keys=w.prior + w.seq, rot_from=w.prior,
+                     window=t.window, rope_frac=t.rope_frac, theta=t.rope_theta, scale=t.scale, rows=rows)
+    secs = time.perf_counter() - t0
+    pos = w.prior + rows[:, 2].astype(np.int64)
+    vis = np.minimum(pos + 1, t.window) if t.window else pos + 1
+    return secs, int(4 * t.head_dim * vis.sum())
+
+
+def layer_bits_for_oracle(w, st, l, q, k, v):
+    """Host bf16 bits of one layer's inputs as the oracle takes them: keys and
+    values in position order, a cached prefix (already rotated) first."""
+    if w.prior:
+        kc, vc = st.k_cache[l], st.v_cache[l]
+        k = torch.cat([kc[:, :, :w.prior].transpose(1, 2), k], dim=1)
+        v = torch.cat([vc[:, :, :w.prior].transpose(1, 2), v], dim=1)
+    return synth.bits(q), synth.bits(k), synth.bits(v)
+
+
+def prefill_cpu_baseline(w, is_global, layers, st, flops_budget):
+    """The oracle on a bounded, seeded sample of each layer's rows, on the
+    inputs the GPU steps used (rows are independent, so the sample's rate is
+    the workload's)."""
+    import oracle
+    n_rows = rows_for_budget(w, is_global, flops_budget)
+    secs, flops = 0.0, 0
+    for l, g in enumerate(is_global):
+        t = w.global_ if g else w.local
+        q, k, v, _ = layers[l]
+        qb, kb, vb = layer_bits_for_oracle(w, st, l, q, k, v)
+        s, f = oracle_prefill_rows(w, t, qb, kb, vb, sample_rows(w, n_rows[l], seed=77 + l))
+        secs += s
+        flops += f
+    n_all = w.batch * w.n_q_heads * w.seq
+    return {"value": round(flops / secs / 1e12, 6), "unit": "TFLOP/s", "cores": oracle.default_threads(),
+            "kind": "oracle", "seconds": round(secs, 2),
+            "sample": ("every row of every layer" if all(n >= n_all for n in n_rows) else
+                       "%s seeded random rows (b, h, i) of the layers [%s] of the same workload and inputs "
+                       "(rows are independent, so the rate is the workload's)"
+                       % ("/".join(str(n) for n in n_rows), ",".join("G" if g else "L" for g in is_global)))}
 
 
 # --------------------------------------------------------------------------- decode (ours)
@@ -315,18 +437,85 @@ def decode_bytes(w, st, lens_cpu):
     return total
 
 
-def visible_kv_bytes(st, l, lens_cpu, bf16_equivalent=False):
+def visible_kv_bytes(st, l, lens_cpu, bf16_equivalent=False, seqs=None):
     """Cached K (and V unless K = V) bytes layer l's decode reads: head_dim
     bf16 per key, or on int8 caches head_dim codes plus an 8-byte (min,
-    step) pair (bf16_equivalent: the bf16 bytes of the same keys)."""
+    step) pair (bf16_equivalent: the bf16 bytes of the same keys); `seqs`
+    restricts the count to those sequences."""
     t = st.layer_type(l)
     L = lens_cpu.to(torch.int64)
+    if seqs is not None:
+        L = L[list(seqs)]
     vis = torch.clamp(L, max=t.window) if t.window else L
     row = t.head_dim + 8 if (st.w.kv_int8 and not bf16_equivalent) else t.head_dim * 2
     return int(vis.sum()) * t.n_kv_heads * row * (1 if st.keqv(l) else 2)
 
 
-def bench_decode(args, w, dev, world, peaks):
+def decode_cpu_baseline(w, st, layers, lens_cpu, n_random=2):
+    """The oracle on a seeded sample of sequences (the shortest, the longest
+    and n_random others) of every layer, after the GPU steps: each sampled
+    sequence's q rotated by the oracle at its position, attending over the
+    sequence's visible cached rows (the new token included), dequantized by
+    the oracle on int8 caches. Rate = the sample's visible K+V bytes per
+    second of oracle time."""
+    import oracle
+    from hybrid_local_global_b200 import native
+    lens = [int(x) for x in lens_cpu]
+    rng = np.random.default_rng(99)
+    pick = {int(np.argmin(lens)), int(np.argmax(lens))}
+    others = [b for b in range(len(lens)) if b not in pick]
+    pick |= set(int(x) for x in rng.choice(others, size=min(n_random, len(others)), replace=False)) if others else set()
+    seqs = sorted(pick)
+    threads = oracle.default_threads()
+    secs, nbytes = 0.0, 0
+    with cf.ThreadPoolExecutor(max_workers=threads) as ex:
+        for l in range(st.n_layers):
+            t = st.layer_type(l)
+            q = layers[l][0]
+            kc, vc = st.k_cache[l], st.v_cache[l]
+            keqv = st.keqv(l)
+            G = w.n_q_heads // t.n_kv_heads
+            for b in seqs:
+                L = lens[b]
+                first = max(0, L - t.window) if t.window else 0
+                slots = [(p % t.window) if t.window else p for p in range(first, L)]
+                qbits = synth.bits(q[b])
+                qrot = np.stack([oracle.rope_bf16(qbits[h], L - 1, t.rope_frac, t.rope_theta)
+                                 for h in range(w.n_q_heads)])
+                idx = torch.as_tensor(slots, dtype=torch.long, device=q.device)
+                t0 = time.perf_counter()
+                if isinstance(kc, native.Int8KVCache):
+                    def rows_of(c):
+                        codes = c.codes[b].index_select(1, idx).cpu().numpy()
+                        prm = c.params[b].index_select(1, idx).cpu().numpy()
+                        return codes, prm
+                    kcod, kprm = rows_of(kc)
+                    vcod, vprm = (kcod, kprm) if keqv else rows_of(vc)
+                    t0 = time.perf_counter()
+                    kf = oracle.dequantize_rows_u8(kcod, kprm[..., 0], kprm[..., 1])
+                    vf = kf if keqv else oracle.dequantize_rows_u8(vcod, vprm[..., 0], vprm[..., 1])
+                    deq = time.perf_counter() - t0
+                else:
+                    kf = kc[b].index_select(1, idx).double().cpu().numpy()
+                    vf = kf if keqv else vc[b].index_select(1, idx).double().cpu().numpy()
+                    deq = 0.0
+                n = len(slots)
+                t0 = time.perf_counter()
+                futs = [ex.submit(oracle.attend_rows, qrot[h:h + 1], kf[h // G], vf[h // G], 0, n, t.scale)
+                        for h in range(w.n_q_heads)]
+                for f in futs:
+                    f.result()
+                secs += time.perf_counter() - t0 + deq
+                del kf, vf
+            nbytes += visible_kv_bytes(st, l, lens_cpu, seqs=seqs)
+    return {"value": round(nbytes / secs / 1e9, 3), "unit": "GB/s", "cores": threads, "kind": "oracle",
+            "seconds": round(secs, 2),
+            "sample": "sequences %s (%s) of every layer, all q heads; bytes = their visible K+V cache bytes"
+                      % (seqs, "the only one" if len(lens) == 1 else
+                         "shortest, longest and %d seeded others" % (len(seqs) - 2))}
+
+
+def bench_decode(args, w, dev, world, peaks, cpu=False):
     from hybrid_local_global_b200 import native
     from hybrid_local_global_b200.stack import AttentionStack
     st = AttentionStack(w, dev)
@@ -388,84 +577,46 @@ def bench_decode(args, w, dev, world, peaks):
         roof["traffic"] = round(sum(per_layer) / st.n_layers)
         roof["traffic_note"] = ("DRAM bytes per split launch: each layer's visible K+V bytes x the "
                                 "traffic/algorithmic ratio of the ncu capture for its layer type (%s), mean "
-                                "over the block's launches; this block is too large to capture"
-                                % ", ".join("%s %.4f: %s in %s" % (k, ratio[k], rec[k]["workload"], rec[k]["file"])
-                                            for k in sorted(rec)))
+                                "over the block's launches" % ", ".join(
+                                    "%s %.4f: %s in %s" % (k, ratio[k], rec[k]["workload"], rec[k]["file"])
+                                    for k in sorted(rec)))
     else:
         roof["traffic_note"] = "no ncu capture of the current kernel sources"
     res = {"metric": "decode KV GB/s", "value": round(value, 1), "unit": "GB/s",
-            "workload": w.name, "description": w.description, "ms_per_step": round(dev_ms / args.steps, 4),
-            "bytes_per_step": nbytes, "kv_bytes_per_step": kv_bytes,
-            "kv_lengths": {"min": int(lens_cpu.min()), "max": max_len, "sum": int(lens_cpu.sum())},
-            "shared_layers": [l for l in range(st.n_layers) if st.is_shared(l)],
-            "cache_bytes_owned": st.owned_cache_bytes(),
-            "roofline": roof, "kernels": kern, "clocks": clk.summary(),
-            "gpu_launches": sum(v["launches"] for v in kern.values())}
+           "workload": w.name, "description": w.description, "ms_per_step": round(dev_ms / args.steps, 4),
+           "bytes_per_step": nbytes, "kv_bytes_per_step": kv_bytes,
+           "kv_lengths": {"min": int(lens_cpu.min()), "max": max_len, "sum": int(lens_cpu.sum())},
+           "shared_layers": [l for l in range(st.n_layers) if st.is_shared(l)],
+           "cache_bytes_owned": st.owned_cache_bytes(),
+           "roofline": roof, "kernels": kern, "clocks": clk.summary(),
+           "gpu_launches": sum(v["launches"] for v in kern.values())}
     if w.kv_int8:
         eq = sum(visible_kv_bytes(st, l, lens_cpu, bf16_equivalent=True) for l in range(st.n_layers))
         res["bf16_equivalent_gbs"] = round(world * eq * args.steps / (dev_ms / 1e3) / 1e9, 1)
         res["bf16_equivalent_note"] = ("bf16 bytes of the same visible keys per second of the whole step: "
                                        "the bandwidth a bf16 cache would need to match this step time")
+    if cpu:
+        res["cpu_baseline"] = decode_cpu_baseline(w, st, layers, lens_cpu)
+    del layers, st, ws
+    torch.cuda.empty_cache()
     return res
 
 
-# --------------------------------------------------------------------------- oracle (CPU)
-def oracle_sample_rows(w, is_global, rows_per_layer, seed):
-    """A bounded, seeded sample of attention rows for each layer."""
-    rng = np.random.default_rng(seed)
-    sample = []
-    for l, g in enumerate(is_global):
-        n = rows_per_layer[1] if g else rows_per_layer[0]
-        r = np.stack([rng.integers(0, w.batch, n), rng.integers(0, w.n_q_heads, n),
-                      rng.integers(0, w.seq, n)], axis=1).astype(np.int32)
-        sample.append(r)
-    return sample
-
-
-def time_oracle(w, layers_bits, is_global, sample):
-    """Runs the oracle on the sampled rows; returns (seconds, algorithmic FLOPs)."""
-    import oracle
-    secs, flops = 0.0, 0
-    for l, g in enumerate(is_global):
-        t = w.global_ if g else w.local
-        q, k, v = layers_bits[l]
-        rows = sample[l]
-        t0 = time.perf_counter()
-        oracle.attention(q, k, v, q_pos0=w.prior, n_keys=w.prior + w.seq, rot_from=w.prior,
-                         window=t.window, rope_frac=t.rope_frac, theta=t.rope_theta, scale=t.scale,
-                         rows=rows)
-        secs += time.perf_counter() - t0
-        pos = w.prior + rows[:, 2].astype(np.int64)
-        vis = np.minimum(pos + 1, t.window) if t.window else pos + 1
-        flops += int(4 * t.head_dim * vis.sum())
-    return secs, flops
-
-
-def host_layers_bits(w, layers):
-    return [(synth.bits(q), synth.bits(k), synth.bits(v)) for (q, k, v, _) in layers]
-
-
-def cpu_layers_bits(w, is_global):
-    """Workload inputs drawn on the CPU (for the reference arm, no GPU needed)."""
-    g = synth.generator(w.seed)
-    out = []
-    for gl in is_global:
-        t = w.global_ if gl else w.local
-        q = synth.randn_bf16((w.batch, w.seq, w.n_q_heads, t.head_dim), g)
-        k = synth.randn_bf16((w.batch, w.seq, t.n_kv_heads, t.head_dim), g, scale=w.k_scale)
-        v = synth.randn_bf16((w.batch, w.seq, t.n_kv_heads, t.head_dim), g)
-        out.append((synth.bits(q), synth.bits(k), synth.bits(v)))
-    return out
-
-
+# --------------------------------------------------------------------------- reference arm (the oracle)
 def schedule_of(w):
+    """The oracle's layer schedule (the reference arm takes nothing from the
+    product library)."""
     if w.fixed_kinds:
         return [k == "global" for k in w.fixed_kinds]
-    from hybrid_local_global_b200 import native
-    return native.gemma_layer_schedule(w.n_layers, w.ratio, w.n_shared)[0]
+    import oracle
+    return oracle.layer_schedule(w.n_layers, w.ratio)
 
 
 def run_reference(args, world, rank):
+    """Times the oracle on the headline workload: every step a seeded sample
+    of rows of every layer. The inputs are the workload's own (drawn on the
+    GPU with the workload's seed when one is present, else on the CPU), copied
+    to the host one layer at a time; only the oracle's time is counted."""
     import oracle
     if rank != 0:
         return
@@ -475,20 +626,30 @@ def run_reference(args, world, rank):
                           "prefill workloads without a cached prefix"}))
         return
     is_global = schedule_of(w)
-    layers = cpu_layers_bits(w, is_global)
+    dev = torch.device("cuda", 0) if torch.cuda.is_available() else torch.device("cpu")
+    g = synth.generator(w.seed, dev)
     cores = oracle.default_threads()
     per = (args.ref_rows_local, args.ref_rows_global)
-    for i in range(args.warmup):
-        time_oracle(w, layers, is_global, oracle_sample_rows(w, is_global, per, seed=i))
-    secs, flops = 0.0, 0
-    for i in range(args.steps):
-        s, f = time_oracle(w, layers, is_global, oracle_sample_rows(w, is_global, per, seed=1000 + i))
-        secs += s
-        flops += f
-    value = flops / secs / 1e12
-    sample = "%d rows per local layer + %d rows of the global layer per step, seeded uniform over (b, h, i)" % per
+    secs = [0.0] * args.steps
+    flops = [0] * args.steps
+    for l, gl in enumerate(is_global):
+        t = w.global_ if gl else w.local
+        q, k, v = draw_prefill_layer(w, t, g, dev)
+        qb, kb, vb = synth.bits(q), synth.bits(k), synth.bits(v)
+        del q, k, v
+        n = per[1] if gl else per[0]
+        for i in range(args.warmup):
+            oracle_prefill_rows(w, t, qb, kb, vb, sample_rows(w, n, seed=100 * l + i))
+        for i in range(args.steps):
+            s, f = oracle_prefill_rows(w, t, qb, kb, vb, sample_rows(w, n, seed=100000 + 100 * l + i))
+            secs[i] += s
+            flops[i] += f
+        del qb, kb, vb
+    value = sum(flops) / sum(secs) / 1e12
+    sample = ("%d rows per local layer + %d rows of each global layer per step, seeded uniform over "
+              "(b, h, i)" % per)
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": secs * 1e3 / args.steps,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": sum(secs) * 1e3 / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic: bf16 ~N(0,1), seeded",
             "config": {"workload": w.name, "description": w.description, "batch": w.batch, "seq_len": w.seq,
@@ -500,21 +661,27 @@ def run_reference(args, world, rank):
 
 
 # --------------------------------------------------------------------------- main
+def names(arg):
+    return [] if arg in ("", "none") else [x for x in arg.split(",") if x]
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="e2b_block_s8192", choices=sorted(WORKLOADS))
+    ap.add_argument("--workload", default=HEADLINE, choices=sorted(WORKLOADS))
+    ap.add_argument("--extra-prefill", default=EXTRA_PREFILL)
     ap.add_argument("--decode-workload", default="31b_decode_b64")
     ap.add_argument("--decode-int8-workload", default="31b_decode_b64_int8")
+    ap.add_argument("--extra-decode", default=EXTRA_DECODE)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-flops", type=float, default=4e11,
+                    help="oracle work per prefill cpu_baseline (FLOPs of the sampled rows)")
     ap.add_argument("--ref-rows-local", type=int, default=256)
     ap.add_argument("--ref-rows-global", type=int, default=256)
-    ap.add_argument("--cpu-rows-local", type=int, default=16384)
-    ap.add_argument("--cpu-rows-global", type=int, default=49152)
     args = ap.parse_args()
 
     if args.impl == "reference":
@@ -526,44 +693,38 @@ def main():
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     peaks = load_peaks()
+    cpu = rank == 0 and world == 1 and not args.no_cpu_baseline
     w = WORKLOADS[args.workload]
-    pre, st, layers = bench_prefill(args, w, dev, world, peaks)
-    line = {"metric": METRIC, "value": round(pre["value"], 3), "unit": "TFLOP/s", "n_gpus": world,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(pre["ms_per_step"], 4),
+    pre = bench_prefill(args, w, dev, world, peaks, e2e=not args.no_e2e, cpu=cpu)
+    line = {"metric": METRIC, "value": pre["value"], "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": pre["ms_per_step"],
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic: bf16 ~N(0,1) Q/K/V, seeded per workload (no dataset)",
             "config": {"workload": w.name, "description": w.description, "batch": w.batch,
-                       "seq_len": w.seq, "n_q_heads": w.n_q_heads,
-                       "layers": ["global" if g else "local" for g in st.is_global],
+                       "seq_len": w.seq, "n_q_heads": w.n_q_heads, "layers": pre["layers"],
                        "parallelism": "independent replica per GPU (dp%d)" % world,
                        "l2": "flushed between timed steps (256 MiB write, outside the step events)"},
             "roofline": pre["roofline"], "gpu_launches": pre["gpu_launches"], "clocks": pre["clocks"],
             "kernels": pre["kernels"], "flops_per_step": pre["flops_per_step"]}
-    if "e2e" in pre:
-        line["e2e"] = pre["e2e"]
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        import oracle
-        is_global = st.is_global
-        bits_layers = host_layers_bits(w, layers)
-        sample = oracle_sample_rows(w, is_global, (args.cpu_rows_local, args.cpu_rows_global), seed=77)
-        secs, flops = time_oracle(w, bits_layers, is_global, sample)
-        line["cpu_baseline"] = {
-            "value": round(flops / secs / 1e12, 6), "unit": "TFLOP/s", "cores": oracle.default_threads(),
-            "kind": "oracle", "seconds": round(secs, 2),
-            "sample": "%d seeded random rows per local layer and %d of the global layer of the same "
-                      "workload (rows are independent, so the rate is the workload's)" % (
-                          args.cpu_rows_local, args.cpu_rows_global)}
-        del bits_layers
-    del layers, st
-    torch.cuda.empty_cache()
+    for key in ("e2e", "cpu_baseline"):
+        if key in pre:
+            line[key] = pre[key]
+    configs = {}
+    for name in names(args.extra_prefill):
+        if name == w.name:
+            continue
+        configs[name] = bench_prefill(args, WORKLOADS[name], dev, world, peaks, cpu=cpu)
     if args.decode_workload != "none":
-        dw = WORKLOADS[args.decode_workload]
-        line["decode"] = bench_decode(args, dw, dev, world, peaks)
-        line["gpu_launches"] += line["decode"]["gpu_launches"]
+        line["decode"] = bench_decode(args, WORKLOADS[args.decode_workload], dev, world, peaks, cpu=cpu)
     if args.decode_int8_workload != "none":
-        dw = WORKLOADS[args.decode_int8_workload]
-        line["decode_int8"] = bench_decode(args, dw, dev, world, peaks)
-        line["gpu_launches"] += line["decode_int8"]["gpu_launches"]
+        line["decode_int8"] = bench_decode(args, WORKLOADS[args.decode_int8_workload], dev, world, peaks, cpu=cpu)
+    for name in names(args.extra_decode):
+        configs[name] = bench_decode(args, WORKLOADS[name], dev, world, peaks, cpu=cpu)
+    if configs:
+        line["configs"] = configs
+    for obj in list(configs.values()) + [line.get("decode"), line.get("decode_int8")]:
+        if obj:
+            line["gpu_launches"] += obj["gpu_launches"]
     if rank == 0:
         print(json.dumps(line))
     RANKS.close()

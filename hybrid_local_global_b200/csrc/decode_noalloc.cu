@@ -32,7 +32,9 @@ void* g_noalloc_ptr[128] = {nullptr};
 
 // Device address of the scratch array on the current device. In host code
 // the array's name is only a host-side stand-in, so the address is looked up
-// once per device with that device current.
+// once per device with that device current and kept for the life of the
+// process; a device reset may move the array, so the header asks processes
+// that reset a device not to call this entry point on it again.
 int noalloc_scratch(void** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);

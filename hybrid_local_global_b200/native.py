@@ -343,6 +343,7 @@ def gemma_attn_decode_noalloc(q, k_new, v_new, k_cache, v_cache, *, seq_lens, ma
         raise TypeError("seq_lens must be an int32 CUDA tensor")
     B, Hq, D = q.shape
     _, Hkv, cap, _ = k_cache.shape
+    flags |= _kv_kind(k_cache, v_cache)
     return _check(_decode_noalloc(_ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_cache), _ptr(v_cache), cap,
                                   _ptr(seq_lens), max_seq_len, B, window, Hq, Hkv, D, rope_frac,
                                   rope_theta, scale, _ptr(out), flags, _stream(stream)))

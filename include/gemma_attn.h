@@ -247,7 +247,10 @@ int gemma_attn_decode_paged(const void* q, const void* k_new, const void* v_new,
 /*     returns GEMMA_ERR_CAPACITY with a message and enqueues nothing.     */
 /*   - The first call on a device looks up the array's device address     */
 /*     (cudaGetSymbolAddress) with that device current; make that first   */
-/*     call before any stream capture.                                    */
+/*     call before any stream capture. The address is kept for the life   */
+/*     of the process: after a cudaDeviceReset (or any teardown of the    */
+/*     device's context) the array may move, so a process that resets a  */
+/*     device must not call this entry point on it again.                 */
 /*   - Every call shares the one array and nothing in it needs to start at */
 /*     zero (each call writes the scratch it reads). Calls that overlap on */
 /*     the GPU (other streams, other host threads) race on it: serialise   */

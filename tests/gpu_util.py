@@ -75,3 +75,38 @@ def assert_rotated_bf16(got: torch.Tensor, exp: torch.Tensor, x: torch.Tensor, w
     tol = bf16_ulp(exp) + 2 ** -20 * pair
     d = (got.float() - exp.float()).abs()
     assert bool((d <= tol).all()), "%s: max excess %.3e" % (what, float((d - tol).max()))
+
+
+# The prefill kernels take queries rotated and pre-multiplied by the logit
+# scale in log2 units (scale * log2 e, an fp32 constant), rounded to bf16 once;
+# decode rounds the rotated query itself. Keys are rotated and rounded to bf16
+# by both.
+LOG2E = 1.4426950408889634
+
+
+def prefill_query_multiplier(scale: float) -> float:
+    """The fp32 constant the prefill path multiplies rotated queries by."""
+    return float(np.float32(np.float64(np.float32(scale)) * LOG2E))
+
+
+def rotate_round(oracle, x: "torch.Tensor", pos, frac, theta, mult=1.0):
+    """bf16 rows [B, S, H, D] -> the oracle's (p-)RoPE of row (b, s, h) at
+    position pos[b] + s, times `mult`, rounded to bf16: the operands as the
+    GPU path rounds them."""
+    import torch
+    B, S, H, D = x.shape
+    xb = to_bits(x)
+    y = np.empty((B, S, H, D), dtype=np.float64)
+    for b in range(B):
+        for s_ in range(S):
+            for h in range(H):
+                y[b, s_, h] = oracle.rope_bf16(xb[b, s_, h], int(pos[b]) + s_, frac, theta)
+    return torch.from_numpy(y * mult).to(torch.bfloat16)
+
+
+def derived_bound(model: np.ndarray, exact: np.ndarray, max_abs=MAX_ABS, mean_abs=MEAN_ABS):
+    """Bound on |gpu - exact| when the GPU is held to (max_abs, mean_abs)
+    against `model` (the exact attention of the rounded operands): by the
+    triangle inequality, the model's own error plus that tolerance."""
+    e = np.abs(model - exact)
+    return float(e.max()) + max_abs, float(e.mean()) + mean_abs

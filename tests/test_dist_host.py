@@ -96,7 +96,8 @@ def test_single_process_needs_no_group():
 def test_reference_arm_runs_on_rank_zero_only(rank):
     env = dict(os.environ, RANK=str(rank), WORLD_SIZE="2", LOCAL_RANK=str(rank))
     cmd = [sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--gpus", "2",
-           "--steps", "1", "--warmup", "0", "--ref-rows-local", "2", "--ref-rows-global", "2"]
+           "--steps", "1", "--warmup", "0", "--ref-rows-local", "2", "--ref-rows-global", "2",
+           "--workload", "local_s1024"]
     p = subprocess.run(cmd, env=env, capture_output=True, text=True, timeout=600)
     assert p.returncode == 0, p.stderr[-2000:]
     lines = [l for l in p.stdout.splitlines() if l.startswith("{")]

@@ -5,9 +5,11 @@ afford cudaMalloc). Its split-K scratch is the library's fixed 32 MiB array.
 
 The test calls it through the C ABI twice in a row, with different inputs,
 and checks each result against gemma_attn_decode given a caller-allocated
-workspace, within the tolerance the other parity tests use. The second call
-would expose scratch left over from the first. The file is named to be
-collected last, and it passes both alone in a fresh process and after the
+workspace. Both calls run the same kernels with the same split plan (the plan
+does not depend on the workspace size), so the outputs must be bit-identical;
+the second call would expose scratch left over from the first. The int8 case
+goes through the Python binding's cache-kind detection. The file is named to
+be collected last, and it passes both alone in a fresh process and after the
 other tests.
 """
 import math
@@ -17,19 +19,21 @@ import torch
 
 from hybrid_local_global_b200 import native, synth
 
-from gpu_util import assert_close
-
 pytestmark = pytest.mark.gpu
 
 
-def _case(seed, lens, Hq, Hkv, D, W, frac, theta):
+def _case(seed, lens, Hq, Hkv, D, W, frac, theta, int8=False):
     dev = torch.device("cuda")
     g = synth.generator(seed, "cuda")
     B = len(lens)
     max_len = max(lens)
     cap = W if W else max_len
-    kc = synth.randn_bf16((B, Hkv, cap, D), g, "cuda")
-    vc = synth.randn_bf16((B, Hkv, cap, D), g, "cuda")
+    if int8:
+        kc = synth.fill_int8_cache_(native.Int8KVCache(B, Hkv, cap, D, dev), g)
+        vc = synth.fill_int8_cache_(native.Int8KVCache(B, Hkv, cap, D, dev), g)
+    else:
+        kc = synth.randn_bf16((B, Hkv, cap, D), g, "cuda")
+        vc = synth.randn_bf16((B, Hkv, cap, D), g, "cuda")
     q = synth.randn_bf16((B, Hq, D), g, "cuda")
     kn = synth.randn_bf16((B, Hkv, D), g, "cuda")
     vn = synth.randn_bf16((B, Hkv, D), g, "cuda")
@@ -39,10 +43,27 @@ def _case(seed, lens, Hq, Hkv, D, W, frac, theta):
     return (q, kn, vn, kc, vc), kw
 
 
+def _bits(t):
+    return t.view(torch.int16)
+
+
+def _clone_cache(c):
+    if isinstance(c, native.Int8KVCache):
+        d = native.Int8KVCache(*c.shape, c.device)
+        d.buf.copy_(c.buf)
+        return d
+    return c.clone()
+
+
+def _cache_bytes(c):
+    return c.buf if isinstance(c, native.Int8KVCache) else _bits(c)
+
+
 @pytest.mark.parametrize("shape", [
     dict(lens=[3000, 9001, 17, 12000], Hq=32, Hkv=4, D=512, W=0, frac=0.25, theta=1e6),
     dict(lens=[5000, 700, 1024], Hq=32, Hkv=16, D=256, W=1024, frac=1.0, theta=1e4),
-])
+    dict(lens=[4000, 33, 2049], Hq=32, Hkv=4, D=512, W=0, frac=0.25, theta=1e6, int8=True),
+], ids=["global", "local", "global_int8"])
 def test_noalloc_decode_matches_workspace_decode_twice(shape):
     for call, seed in enumerate((301, 302)):
         (q, kn, vn, kc, vc), kw = _case(seed, **shape)
@@ -50,16 +71,17 @@ def test_noalloc_decode_matches_workspace_decode_twice(shape):
                                                        kw["window"], kw["max_seq_len"])
         assert 0 < need <= native.NOALLOC_SCRATCH_BYTES
         ref = torch.empty_like(q)
-        kc_ref, vc_ref = kc.clone(), vc.clone()
+        kc_ref, vc_ref = _clone_cache(kc), _clone_cache(vc)
         native.gemma_attn_decode(q, kn, vn, kc_ref, vc_ref, out=ref, **kw)
         assert native.gemma_attn_sync_status() == 0, native.gemma_last_error()
         out = torch.full_like(q, float("nan"))
         native.gemma_attn_decode_noalloc(q, kn, vn, kc, vc, out=out, **kw)
         assert native.gemma_attn_sync_status() == 0, native.gemma_last_error()
-        assert_close(out.float().cpu().double().numpy(), ref.float().cpu().double().numpy(),
-                     what="no-alloc decode, call %d" % (call + 1))
+        # same kernels, same split plan: bit-identical outputs
+        assert torch.equal(_bits(out), _bits(ref)), "no-alloc decode differs, call %d" % (call + 1)
         # the cache append is the same operation
-        assert torch.equal(kc, kc_ref) and torch.equal(vc, vc_ref)
+        assert torch.equal(_cache_bytes(kc), _cache_bytes(kc_ref))
+        assert torch.equal(_cache_bytes(vc), _cache_bytes(vc_ref))
 
 
 def test_noalloc_decode_rejects_more_scratch_than_it_has():
