@@ -210,17 +210,49 @@ def test_prefill_peaky(oracle, monkeypatch, kernel, D, W, Hkv, frac, theta):
     q = synth.randn_bf16((B, S, Hq, D), g, scale=8.0)
     k = synth.randn_bf16((B, S, Hkv, D), g)
     v = synth.randn_bf16((B, S, Hkv, D), g)
+    assert_matches_rounded_model(oracle, out, q, k, v, W, frac, theta, "prefill peaky")
+
+
+def assert_matches_rounded_model(oracle, out, q, k, v, W, frac, theta, what):
+    """GPU output against the exact attention of the operands rounded as the
+    prefill kernels round them (spec tolerance), and against the exact
+    oracle within that model's error plus the tolerance."""
+    B, S, Hq, D = q.shape
     scale = 1.0 / math.sqrt(D)
     c = prefill_query_multiplier(scale)
-    qr = rotate_round(oracle, q, [0], frac, theta, mult=c)
-    kr = rotate_round(oracle, k, [0], frac, theta)
+    qr = rotate_round(oracle, q, [0] * B, frac, theta, mult=c)
+    kr = rotate_round(oracle, k, [0] * B, frac, theta)
     model, _ = oracle.attention(to_bits(qr), to_bits(kr), to_bits(v), q_pos0=0, n_keys=S, rot_from=S, window=W,
                                 rope_frac=0.0, theta=theta, scale=scale / c)
     exact, _ = oracle.attention(to_bits(q), to_bits(k), to_bits(v), q_pos0=0, n_keys=S, rot_from=0, window=W,
                                 rope_frac=frac, theta=theta, scale=scale)
     got = out.float().cpu().double().numpy().transpose(0, 2, 1, 3).reshape(-1, D)
-    assert_close(got, model, what="prefill peaky vs rounded-operand model")
-    assert_close(got, exact, *derived_bound(model, exact), what="prefill peaky vs exact")
+    assert_close(got, model, what="%s vs rounded-operand model" % what)
+    assert_close(got, exact, *derived_bound(model, exact), what="%s vs exact" % what)
+
+
+@pytest.mark.parametrize("kernel", ["single", "hpair"])
+def test_prefill_growing_logits(oracle, monkeypatch, kernel):
+    """Keys scaled up along the sequence (x1 at the start to x3 at the end)
+    and queries x3: every later key tile holds larger logits, so the running
+    row maximum keeps moving and O is rescaled in TMEM several times per
+    row."""
+    monkeypatch.setenv("GEMMA_PREFILL_KERNEL", kernel)
+    B, S, Hq, Hkv, D, frac, theta = 2, 1000, 8, 1, 512, 0.25, 1e6
+    dev = torch.device("cuda")
+    g = synth.generator(151)
+    q = synth.randn_bf16((B, S, Hq, D), g, scale=3.0)
+    k0 = synth.randn_bf16((B, S, Hkv, D), g)
+    v = synth.randn_bf16((B, S, Hkv, D), g)
+    ramp = (1.0 + 2.0 * torch.arange(S, dtype=torch.float32) / S).view(1, S, 1, 1)
+    k = (k0.float() * ramp).to(torch.bfloat16)
+    kc = torch.zeros((B, Hkv, S, D), dtype=torch.bfloat16, device=dev)
+    vc = torch.zeros_like(kc)
+    out = torch.full((B, S, Hq, D), float("nan"), dtype=torch.bfloat16, device=dev)
+    native.gemma_attn_prefill(q.to(dev), k.to(dev), v.to(dev), kc, vc, window=0, rope_frac=frac, rope_theta=theta,
+                              scale=1.0 / math.sqrt(D), out=out)
+    assert native.gemma_attn_sync_status() == 0, native.gemma_last_error()
+    assert_matches_rounded_model(oracle, out, q, k, v, 0, frac, theta, "growing logits")
 
 
 def test_visible_ranges_bit_exact(oracle):
