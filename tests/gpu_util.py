@@ -104,9 +104,26 @@ def rotate_round(oracle, x: "torch.Tensor", pos, frac, theta, mult=1.0):
     return torch.from_numpy(y * mult).to(torch.bfloat16)
 
 
-def derived_bound(model: np.ndarray, exact: np.ndarray, max_abs=MAX_ABS, mean_abs=MEAN_ABS):
-    """Bound on |gpu - exact| when the GPU is held to (max_abs, mean_abs)
-    against `model` (the exact attention of the rounded operands): by the
-    triangle inequality, the model's own error plus that tolerance."""
+# bf16 unit roundoff (8 significant bits, round to nearest)
+BF16_U = 2.0 ** -8
+
+
+def rounding_bound(model: np.ndarray, v_absmax: float) -> float:
+    """Largest |gpu - model| that the GPU's own bf16 roundings allow, the
+    operands rounded as in `model`: every weight p_j is rounded to bf16
+    (relative error <= u) and normalised by the sum of the unrounded
+    weights, which moves an output by at most u * sum_j w_j |v_j| <=
+    u * max|v|; the output itself is rounded to bf16 (<= u * |o|). A slack
+    of 2^-10 covers the fp32 accumulations and the exp2 approximation."""
+    return BF16_U * (v_absmax + float(np.abs(model).max())) + 2.0 ** -10
+
+
+def assert_close_to_model(gpu, model, exact, v_absmax, what=""):
+    """GPU output against the exact attention of its rounded operands within
+    the rounding bound above (mean-abs within the benchmark spec's 2e-3), and
+    against the exact oracle within the model's own error plus that bound
+    (the triangle inequality)."""
+    tol = rounding_bound(model, v_absmax)
+    assert_close(gpu, model, tol, MEAN_ABS, what="%s vs rounded-operand model" % what)
     e = np.abs(model - exact)
-    return float(e.max()) + max_abs, float(e.mean()) + mean_abs
+    assert_close(gpu, exact, float(e.max()) + tol, float(e.mean()) + MEAN_ABS, what="%s vs exact" % what)
