@@ -54,7 +54,8 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 from hybrid_local_global_b200 import synth  # noqa: E402
-from hybrid_local_global_b200.workloads import WORKLOADS, prefill_flops, visible_pairs_prefill  # noqa: E402
+from hybrid_local_global_b200.workloads import (WORKLOADS, layer_shape_tag, prefill_attn_bytes,  # noqa: E402
+                                                prefill_flops, visible_pairs_prefill)
 
 METRIC = "attention prefill TFLOP/s and decode KV GB/s on 1 B200, as % of roofline"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -185,19 +186,23 @@ def make_prefill(w, dev):
     return st, layers, ws, lens
 
 
-def recorded_traffic(kernel, workload=None):
-    """DRAM bytes per launch recorded by an ncu capture under profiles/
-    (``traffic-record:`` lines), keyed by layer type; only records whose
-    kernel-source digest matches the sources built now count."""
+def current_records(kernel):
+    """DRAM bytes per launch recorded by ncu captures under profiles/
+    (``traffic-record:`` lines) for a kernel whose sources still have the
+    digest recorded with them."""
     from hybrid_local_global_b200.profiling import kernel_digest, traffic_records
     digest = kernel_digest(kernel)
+    return [r for r in traffic_records(os.path.join(ROOT, "profiles"))
+            if r.get("kernel") == kernel and r.get("digest") == digest]
+
+
+def recorded_traffic(kernel, workload=None):
+    """current_records of one workload (or of any, the last per layer type),
+    keyed by layer type."""
     out = {}
-    for r in traffic_records(os.path.join(ROOT, "profiles")):
-        if r.get("kernel") != kernel or r.get("digest") != digest:
-            continue
-        if workload is not None and r.get("workload") != workload:
-            continue
-        out[r.get("layer", "")] = r
+    for r in current_records(kernel):
+        if workload is None or r.get("workload") == workload:
+            out[r.get("layer", "")] = r
     return out
 
 
@@ -277,21 +282,29 @@ def bench_prefill(args, w, dev, world, peaks, e2e=False, cpu=False):
             "per_launch": "algorithmic FLOPs of all attention launches / their summed device time "
                           "(%d launches, %d per step; CUDA events around each launch, in a second timed "
                           "pass of the same steps)" % (attn["launches"], st.n_layers)}
-    # the kernel that runs each layer type: CTA pairs on head_dim 512 (both
-    # model shapes have an even number of q heads per KV head), one CTA per
-    # query tile on head_dim 256
-    rec = {}
+    # DRAM traffic of each layer type's launch: a capture of this workload, or
+    # of a smaller one of the same per-head shape scaled by the bytes moved
+    # (traffic / algorithmic bytes of the captured launch x this launch's)
+    per_kind, files = {}, set()
     for kind, lt in (("local", w.local), ("global", w.global_)):
-        r = recorded_traffic("k_prefill_pair" if lt.head_dim == 512 else "k_prefill_tc", w.name)
-        if kind in r:
-            rec[kind] = r[kind]
+        kname = "k_prefill_pair" if lt.head_dim == 512 else "k_prefill_tc"
+        exact = recorded_traffic(kname, w.name)
+        if kind in exact:
+            per_kind[kind] = (float(exact[kind]["bytes"]), "%s (this workload)" % exact[kind]["file"])
+            continue
+        for r in current_records(kname):
+            if r.get("shape") == layer_shape_tag(w, lt) and "units" in r and r.get("layer") == kind:
+                ratio = float(r["bytes"]) / float(r["units"])
+                per_kind[kind] = (ratio * prefill_attn_bytes(w, lt),
+                                  "%s (%s, %.3f x the algorithmic bytes)" % (r["file"], r["workload"], ratio))
+                break
     kinds = ["global" if g else "local" for g in st.is_global]
-    if all(k in rec for k in kinds):
-        roof["traffic"] = round(sum(float(rec[k]["bytes"]) for k in kinds) / len(kinds))
-        roof["traffic_note"] = ("DRAM read+write bytes per attention launch, mean over the step's layers, "
-                                "from ncu captures in %s" % ", ".join(sorted({rec[k]["file"] for k in kinds})))
+    if all(k in per_kind for k in kinds):
+        roof["traffic"] = round(sum(per_kind[k][0] for k in kinds) / len(kinds))
+        roof["traffic_note"] = ("DRAM read+write bytes per attention launch, mean over the step's layers, from "
+                                "ncu captures: %s" % "; ".join(sorted({per_kind[k][1] for k in kinds})))
     else:
-        roof["traffic_note"] = "no ncu capture of the current kernel sources for this workload"
+        roof["traffic_note"] = "no ncu capture of the current kernel sources for this layer shape"
     launches = sum(v["launches"] for v in kern.values())
     res = {"metric": "prefill attention TFLOP/s", "value": round(value, 3), "unit": "TFLOP/s",
            "workload": w.name, "description": w.description,

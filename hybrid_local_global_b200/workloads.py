@@ -89,6 +89,16 @@ WORKLOADS = {
         local=L31B_LOCAL, global_=L31B_GLOBAL, seq=4096, prior=262144 - 4096, seed=4,
         fixed_kinds=("global",),
         description="chunked prefill of 4096 queries at 258048.. against a 256K global cache"),
+    "31b_local_s8192": Workload(
+        "31b_local_s8192", "prefill", batch=1, n_q_heads=32, n_layers=1, ratio=0,
+        local=L31B_LOCAL, global_=L31B_GLOBAL, seq=8192, k_scale=0.5, seed=2, fixed_kinds=("local",),
+        description="one 31B-shaped local layer, B1 S8192 Hq32 Hkv16 D256 W1024 (a kernel-profiling case)"),
+    "global_chunk_64k": Workload(
+        "global_chunk_64k", "prefill", batch=1, n_q_heads=32, n_layers=1, ratio=0,
+        local=L31B_LOCAL, global_=L31B_GLOBAL, seq=1024, prior=65536 - 1024, seed=4,
+        fixed_kinds=("global",),
+        description="chunked prefill of 1024 queries at 64512.. against a 64K global cache "
+                    "(a kernel-profiling case)"),
     "global_s16384": Workload(
         "global_s16384", "prefill", batch=1, n_q_heads=32, n_layers=1, ratio=0,
         local=L31B_LOCAL, global_=L31B_GLOBAL, seq=16384, seed=5, fixed_kinds=("global",),
@@ -138,3 +148,24 @@ def prefill_flops(w: Workload, is_global: list[bool]) -> int:
         t = w.global_ if g else w.local
         total += 4 * w.batch * w.n_q_heads * t.head_dim * visible_pairs_prefill(w.seq, w.prior, t.window)
     return total
+
+
+def prefill_attn_bytes(w: Workload, t: LayerType) -> int:
+    """Algorithmic DRAM bytes of one prefill attention launch of layer type t:
+    the queries read and the outputs written, the chunk's keys and values
+    read (rotated keys from the cache or the workspace, values from the
+    caller), and on a chunk after cached tokens the cached prefix's keys and
+    values, each element once (bf16)."""
+    q = w.batch * w.seq * w.n_q_heads * t.head_dim * 2
+    kv = w.batch * w.seq * t.n_kv_heads * t.head_dim * 2
+    if w.prior:
+        vis_prior = min(w.prior, t.window) if t.window else w.prior
+        kv += w.batch * vis_prior * t.n_kv_heads * t.head_dim * 2
+    return 2 * q + (1 if w.k_eq_v else 2) * kv
+
+
+def layer_shape_tag(w: Workload, t: LayerType) -> str:
+    """Per-(batch, head) shape of a layer's attention: q heads, KV heads, head
+    dim, window, and whether the chunk follows cached tokens (c) or not (f).
+    Traffic records of one shape scale with the bytes moved."""
+    return "%d-%d-%d-%d-%s" % (w.n_q_heads, t.n_kv_heads, t.head_dim, t.window, "c" if w.prior else "f")
