@@ -201,6 +201,47 @@ size_t prefill_ws_parts(int B, int S, int Hq, int Hkv, int D, int window, size_t
   return q + std::max(k, 2 * win);
 }
 
+// Multi-token decode on the tensor-core kernel: a global bf16 layer on a
+// contiguous cache whose G q heads x tokens rows fit one 128-row tile.
+bool verify_fast(int tokens, int window, int n_q_heads, int n_kv_heads, int head_dim, unsigned flags, bool paged) {
+  return window == 0 && !(flags & GEMMA_F_KV_INT8) && !paged && (head_dim == 256 || head_dim == 512) &&
+         (n_q_heads / n_kv_heads) * tokens <= 128;
+}
+
+// Keys per split of the multi-token kernel: a multiple of 128 between 1024
+// and 8192, aiming at eight CTAs per SM over the planned length (a CTA's
+// fixed cost, the Q tile and the partials, is then a few percent of its
+// streaming time). The 128-row-tile kernel runs head_dim / 256 CTAs per KV
+// head and split, the transposed one a single CTA.
+void verify_plan(int B, int Hq, int Hkv, int tokens, int head_dim, int max_len, int* chunk, int* n_splits) {
+  const int per_head = verify_tc_rows(Hq, Hkv, tokens, head_dim) ? 1 : head_dim / 256;
+  const int64_t ctas_per_split = (int64_t)B * Hkv * per_head;
+  const int64_t target = (int64_t)sm_count() * 8;
+  int64_t c = ((int64_t)max_len * ctas_per_split + target - 1) / target;
+  c = ((c + 127) / 128) * 128;
+  c = std::min<int64_t>(std::max<int64_t>(c, 1024), 8192);
+  *chunk = (int)c;
+  *n_splits = (int)((max_len + c - 1) / c);
+}
+
+// fast path: rotated Q, split log2-sum-exps, split partial O
+size_t verify_ws_parts(int B, int tokens, int Hq, int D, int n_splits, size_t* off_lse, size_t* off_o) {
+  const size_t rows = (size_t)B * tokens * Hq;
+  const size_t q = align256(rows * D * 2);
+  const size_t lse = align256(rows * n_splits * 4);
+  *off_lse = q;
+  *off_o = q + lse;
+  return q + lse + align256(rows * n_splits * D * 4);
+}
+
+// other layers: lengths before the new tokens, then the chunked-prefill workspace
+size_t verify_route_ws(int B, int tokens, int Hq, int Hkv, int D, int window, int cache_cap, unsigned flags) {
+  size_t off_k;
+  const bool prefix = (flags & GEMMA_F_KV_INT8) && window == 0;
+  return align256((size_t)B * 4) +
+         prefill_ws_parts(B, tokens, Hq, Hkv, D, window, &off_k, nullptr, prefix ? cache_cap : 0);
+}
+
 }  // namespace
 
 namespace hlg {
@@ -385,7 +426,11 @@ static int prefill_impl(const void* q, const void* k_new, const void* v_new, voi
                         int cache_cap, const int32_t* seq_lens_before, int batch, int s_new, int window,
                         int n_q_heads, int n_kv_heads, int head_dim, float rope_frac, float rope_theta,
                         float scale, void* out, float* lse, void* workspace, size_t workspace_bytes,
-                        unsigned flags, void* stream, const CacheLayout& L) {
+                        unsigned flags, void* stream, const CacheLayout& L,
+                        const int32_t* lens_after = nullptr) {
+  // lens_after (multi-token decode): lengths including the chunk; once the
+  // arguments have passed, seq_lens_before (then a device buffer of batch
+  // ints) receives lens_after - s_new
   int rc = check_heads(n_q_heads, n_kv_heads, head_dim, window, rope_frac, rope_theta, scale);
   if (rc) return rc;
   rc = check_kv_flags(flags, window, k_new, v_new, k_cache, &v_cache);
@@ -430,6 +475,10 @@ static int prefill_impl(const void* q, const void* k_new, const void* v_new, voi
   if (!status) return fail(GEMMA_ERR_CUDA, "no CUDA device");
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   unsigned char* ws = static_cast<unsigned char*>(workspace);
+  if (lens_after) {
+    cudaError_t el = launch_lens_minus(lens_after, const_cast<int32_t*>(seq_lens_before), batch, s_new, st);
+    if (el != cudaSuccess) return cuda_fail(el, "length launch");
+  }
 
   PrefillRopeArgs ra{};
   ra.q = static_cast<const bf16*>(q);
@@ -626,6 +675,8 @@ static int decode_impl(const void* q, const void* k_new, const void* v_new, void
   unsigned char* ws = static_cast<unsigned char*>(workspace);
 
   DecodeRopeArgs ra{};
+  ra.tokens = 1;
+  ra.q_scale = 1.f;
   ra.q = static_cast<const bf16*>(q);
   ra.k_new = static_cast<const bf16*>(k_new);
   ra.v_new = static_cast<const bf16*>(v_new);
@@ -657,6 +708,7 @@ static int decode_impl(const void* q, const void* k_new, const void* v_new, void
   if (e != cudaSuccess) return cuda_fail(e, "decode append launch");
 
   DecodeAttnArgs da{};
+  da.tokens = 1;
   da.q_rot = ra.q_rot;
   da.k_cache = static_cast<const bf16*>(k_cache);
   da.v_cache = static_cast<const bf16*>(v_cache);
@@ -722,6 +774,135 @@ int gemma_attn_decode_paged(const void* q, const void* k_new, const void* v_new,
   return decode_impl(q, k_new, v_new, k_pool, v_pool, pages_per_seq * page_size, seq_lens, max_seq_len, batch, 0,
                      n_q_heads, n_kv_heads, head_dim, rope_frac, rope_theta, scale, out, workspace, workspace_bytes,
                      flags, stream, CacheLayout{page_table, page_size, pages_per_seq, n_pages});
+}
+
+size_t gemma_attn_decode_multi_workspace_size(int batch, int tokens, int n_q_heads, int n_kv_heads, int head_dim,
+                                              int window, int max_seq_len, int cache_cap, unsigned flags) {
+  if (batch <= 0 || tokens <= 0 || n_q_heads <= 0 || n_kv_heads <= 0 || head_dim <= 0 || max_seq_len <= 0 ||
+      cache_cap <= 0)
+    return 0;
+  if (verify_fast(tokens, window, n_q_heads, n_kv_heads, head_dim, flags, false)) {
+    int chunk, n_splits;
+    verify_plan(batch, n_q_heads, n_kv_heads, tokens, head_dim, max_seq_len, &chunk, &n_splits);
+    size_t a, b;
+    return verify_ws_parts(batch, tokens, n_q_heads, head_dim, n_splits, &a, &b);
+  }
+  return verify_route_ws(batch, tokens, n_q_heads, n_kv_heads, head_dim, window, cache_cap, flags);
+}
+
+int gemma_attn_decode_multi(const void* q, const void* k_new, const void* v_new, void* k_cache, void* v_cache,
+                            int cache_cap, const int32_t* seq_lens, int max_seq_len, int batch, int tokens,
+                            int window, int n_q_heads, int n_kv_heads, int head_dim, float rope_frac,
+                            float rope_theta, float scale, void* out, void* workspace, size_t workspace_bytes,
+                            unsigned flags, void* stream) {
+  int rc = check_heads(n_q_heads, n_kv_heads, head_dim, window, rope_frac, rope_theta, scale);
+  if (rc) return rc;
+  if (batch <= 0 || tokens <= 0 || max_seq_len <= 0)
+    return fail(GEMMA_ERR_INVALID_ARG, "batch %d, tokens %d, max_seq_len %d", batch, tokens, max_seq_len);
+  if (!seq_lens) return fail(GEMMA_ERR_INVALID_ARG, "null seq_lens");
+  if (window == 0 && cache_cap < max_seq_len)
+    return fail(GEMMA_ERR_CAPACITY, "global layer: cache_cap %d < max_seq_len %d", cache_cap, max_seq_len);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  unsigned char* ws = static_cast<unsigned char*>(workspace);
+  if (!verify_fast(tokens, window, n_q_heads, n_kv_heads, head_dim, flags, false)) {
+    // the new tokens as a chunk after seq_lens - tokens cached tokens
+    const size_t need = verify_route_ws(batch, tokens, n_q_heads, n_kv_heads, head_dim, window, cache_cap, flags);
+    if (!workspace || workspace_bytes < need)
+      return fail(GEMMA_ERR_CAPACITY, "workspace %zu bytes < %zu", workspace_bytes, need);
+    if (!aligned16(workspace)) return fail(GEMMA_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
+    int32_t* before = reinterpret_cast<int32_t*>(ws);
+    const size_t head = align256((size_t)batch * 4);
+    return prefill_impl(q, k_new, v_new, k_cache, v_cache, cache_cap, before, batch, tokens, window, n_q_heads,
+                        n_kv_heads, head_dim, rope_frac, rope_theta, scale, out, nullptr, ws + head,
+                        workspace_bytes - head, flags, stream, contiguous(cache_cap, batch), seq_lens);
+  }
+  rc = check_kv_flags(flags, window, k_new, v_new, k_cache, &v_cache);
+  if (rc) return rc;
+  if (!q || !out || !k_cache || !v_cache) return fail(GEMMA_ERR_INVALID_ARG, "null tensor pointer");
+  if (!aligned16(q) || !aligned16(out) || !aligned16(k_cache) || !aligned16(v_cache) ||
+      (k_new && !aligned16(k_new)) || (v_new && !aligned16(v_new)) || !aligned16(workspace))
+    return fail(GEMMA_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
+  int chunk, n_splits;
+  verify_plan(batch, n_q_heads, n_kv_heads, tokens, head_dim, max_seq_len, &chunk, &n_splits);
+  size_t off_lse, off_o;
+  const size_t need = verify_ws_parts(batch, tokens, n_q_heads, head_dim, n_splits, &off_lse, &off_o);
+  if (!workspace || workspace_bytes < need)
+    return fail(GEMMA_ERR_CAPACITY, "workspace %zu bytes < %zu", workspace_bytes, need);
+  int* status = status_ptr();
+  if (!status) return fail(GEMMA_ERR_CUDA, "no CUDA device");
+
+  DecodeRopeArgs ra{};
+  ra.tokens = tokens;
+  // queries carry scale * log2(e), as in prefill: logits arrive in log2 units
+  ra.q_scale = (float)((double)scale * 1.4426950408889634);
+  ra.q = static_cast<const bf16*>(q);
+  ra.k_new = static_cast<const bf16*>(k_new);
+  ra.v_new = static_cast<const bf16*>(v_new);
+  ra.q_rot = reinterpret_cast<bf16*>(ws);
+  ra.k_cache = static_cast<bf16*>(k_cache);
+  ra.v_cache = static_cast<bf16*>(v_cache);
+  ra.cache_cap = cache_cap;
+  ra.seq_lens = seq_lens;
+  ra.max_len = max_seq_len;
+  ra.window = 0;
+  ra.Hq = n_q_heads;
+  ra.Hkv = n_kv_heads;
+  ra.n_rot = rope_rotated_pairs(head_dim, rope_frac);
+  ra.log2_theta = std::log2((double)rope_theta);
+  ra.k_stage = nullptr;
+  ra.page_table = nullptr;
+  ra.page_size = cache_cap;
+  ra.pages_per_seq = 1;
+  ra.n_pages = batch;
+  ra.status = status;
+  ProfScope p_app(GEMMA_KERNEL_DECODE_APPEND, st);
+  cudaError_t e = launch_decode_rope_append(ra, batch, head_dim, st);
+  p_app.done();
+  if (e != cudaSuccess) return cuda_fail(e, "decode append launch");
+
+  const int64_t D = head_dim;
+  VerifyAttnArgs va{};
+  va.q_rot = ra.q_rot;
+  va.k = KVView{static_cast<const bf16*>(k_cache), (int64_t)n_kv_heads * cache_cap * D, D, (int64_t)cache_cap * D};
+  va.v = KVView{static_cast<const bf16*>(v_cache), va.k.stride_b, va.k.stride_row, va.k.stride_h};
+  va.cache_cap = cache_cap;
+  va.seq_lens = seq_lens;
+  va.tokens = tokens;
+  va.Hq = n_q_heads;
+  va.Hkv = n_kv_heads;
+  va.chunk = chunk;
+  va.n_splits = n_splits;
+  va.part_o = reinterpret_cast<float*>(ws + off_o);
+  va.part_lse = reinterpret_cast<float*>(ws + off_lse);
+  va.status = status;
+  va.wait_ns = (unsigned long long)g_wait_ns.load();
+  {
+    ProfScope p_split(GEMMA_KERNEL_DECODE_SPLIT, st);
+    e = launch_verify_attn_tc(va, batch, head_dim, st);
+    p_split.done();
+  }
+  if (e != cudaSuccess) return cuda_fail(e, "multi-token attention launch");
+
+  DecodeAttnArgs da{};
+  da.tokens = tokens;
+  da.seq_lens = seq_lens;
+  da.max_len = max_seq_len;
+  da.window = 0;
+  da.Hq = n_q_heads;
+  da.Hkv = n_kv_heads;
+  da.chunk = chunk;
+  da.n_splits = n_splits;
+  da.part_lse = va.part_lse;
+  da.part_o = va.part_o;
+  da.out = static_cast<bf16*>(out);
+  da.status = status;
+  {
+    ProfScope p_comb(GEMMA_KERNEL_DECODE_COMBINE, st);
+    e = launch_decode_combine(da, batch, head_dim, st);
+    p_comb.done();
+  }
+  if (e != cudaSuccess) return cuda_fail(e, "decode combine launch");
+  return succeed();
 }
 
 int gemma_attn_visible_ranges(const int32_t* seq_lens_before, int batch, int s_new, int window,

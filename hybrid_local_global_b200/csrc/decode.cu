@@ -354,7 +354,8 @@ __global__ void __launch_bounds__(32 * (NCW + 1), 2) k_decode_split(DecodeAttnAr
   }
 }
 
-// Log-sum-exp merge of the splits of one (sequence, q head): 128 threads =
+// Log-sum-exp merge of the splits of one (sequence, query token, q head)
+// (decode: one token per sequence): 128 threads =
 // 16 dim quads x 8 split lanes per 64 output dims, so the reads of a
 // split's partial are coalesced and the splits are summed in parallel. The
 // grid's z dimension splits the head dimension when there are few
@@ -364,18 +365,19 @@ __global__ void __launch_bounds__(128) k_decode_combine(DecodeAttnArgs a) {
   extern __shared__ float w_s[];  // [n_splits]
   __shared__ __align__(16) float red[8][64];
   __shared__ float rmax[4], rsum[4];
-  const int h = blockIdx.x, b = blockIdx.y;
+  // blockIdx.y = b * tokens + t: the row of (sequence b, query token t)
+  const int h = blockIdx.x, bt = blockIdx.y, b = bt / a.tokens;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  bf16* dst = a.out + ((int64_t)b * a.Hq + h) * D;
+  bf16* dst = a.out + ((int64_t)bt * a.Hq + h) * D;
   const int64_t len = a.seq_lens[b];
-  if (len < 1 || len > a.max_len) {
+  if (len < a.tokens || len > a.max_len) {
     for (int d = blockIdx.z * 64 + tid; d < D; d += gridDim.z * 64)
       if (tid < 64) dst[d] = __float2bfloat16(0.f);
     return;
   }
   const int64_t n_valid = a.window > 0 ? (len < a.window ? len : (int64_t)a.window) : len;
   const int n_used = (int)((n_valid + a.chunk - 1) / a.chunk);
-  const int64_t pr0 = ((int64_t)b * a.Hq + h) * a.n_splits;
+  const int64_t pr0 = ((int64_t)bt * a.Hq + h) * a.n_splits;
   float m = -INFINITY;
   for (int s = tid; s < n_used; s += 128) m = fmaxf(m, a.part_lse[pr0 + s]);
 #pragma unroll
@@ -445,9 +447,10 @@ cudaError_t launch_decode_split(const DecodeAttnArgs& a, int B, int D, cudaStrea
 
 cudaError_t launch_decode_combine(const DecodeAttnArgs& a, int B, int D, cudaStream_t st) {
   // enough CTAs for about eight per SM, at most one per 64 output dims
-  const int pairs = a.Hq * B;
+  if (a.tokens < 1) return cudaErrorInvalidValue;
+  const int pairs = a.Hq * B * a.tokens;
   const int nz = std::max(1, std::min(D / 64, (8 * 148 + pairs - 1) / pairs));
-  dim3 grid(a.Hq, B, nz);
+  dim3 grid(a.Hq, B * a.tokens, nz);
   const size_t smem = (size_t)a.n_splits * sizeof(float);
   if (smem > 48 * 1024) return cudaErrorInvalidValue;  // > 12288 splits: not planned by decode_plan
   if (D == 256)

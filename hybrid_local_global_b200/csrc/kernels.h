@@ -40,10 +40,12 @@ struct PrefillRopeArgs {
 };
 
 struct DecodeRopeArgs {
-  const bf16* q;       // [B][Hq][D]
-  const bf16* k_new;   // [B][Hkv][D] or null
+  const bf16* q;       // [B][tokens][Hq][D]
+  const bf16* k_new;   // [B][tokens][Hkv][D] or null
   const bf16* v_new;
-  bf16* q_rot;         // workspace [B][Hq][D]
+  bf16* q_rot;         // workspace [B][tokens][Hq][D]
+  int tokens;          // new tokens per sequence, at positions len - tokens .. len - 1 (decode: 1)
+  float q_scale;       // rotated q is multiplied by this before the bf16 rounding (decode: 1)
   bf16* k_cache;
   bf16* v_cache;
   bf16* k_stage;       // int8 cache: the rotated new key goes here ([B][Hkv][D]) and nothing
@@ -118,9 +120,10 @@ struct DecodeAttnArgs {
   int chunk;               // keys per split (multiple of 16)
   int n_splits;
   float scale_log2;
-  float* part_o;           // [B][Hq][n_splits][D]
-  float* part_lse;         // [B][Hq][n_splits] (log2 domain)
-  bf16* out;               // [B][Hq][D]
+  float* part_o;           // [B][tokens][Hq][n_splits][D]
+  float* part_lse;         // [B][tokens][Hq][n_splits] (log2 domain)
+  bf16* out;               // [B][tokens][Hq][D]
+  int tokens;              // query tokens per sequence (decode: 1; the combine's rows)
   int* status;
   unsigned long long wait_ns;
   int drop_first_copy;     // test hook: skip the first K/V copy of split 0
@@ -158,6 +161,31 @@ cudaError_t launch_gather_q8(const uint8_t* k_codes, const float2* k_params, con
                              int pages_per_seq, int n_pages, int win_rows, bf16* k_win, bf16* v_win,
                              int* status, cudaStream_t st);
 cudaError_t launch_decode_rope_append(const DecodeRopeArgs& a, int B, int D, cudaStream_t st);
+cudaError_t launch_lens_minus(const int32_t* seq_lens, int32_t* lens_before, int B, int tokens, cudaStream_t st);
+
+// Multi-token decode on a global layer (several new tokens per sequence, each
+// seeing the cache and the earlier new tokens), over splits of `chunk` keys,
+// writing per-split partials for launch_decode_combine. Up to 64 query rows
+// (G q heads x tokens) a KV head: the transposed tensor-core kernel (query
+// rows as the MMA's N, one CTA per KV head and split); more: the prefill
+// kernel's 128-row tile over those rows (launch_verify_attn_rows; two CTAs
+// per KV head at head_dim 512). verify_tc_rows gives the first kernel's
+// padded row count, 0 when the second one runs.
+struct VerifyAttnArgs {
+  const bf16* q_rot;        // [B][tokens][Hq][D], times scale * log2(e)
+  KVView k, v;              // head-major cache views [B][Hkv][cap][D]
+  int cache_cap;
+  const int32_t* seq_lens;  // device [B], including the new tokens
+  int tokens, Hq, Hkv;
+  int chunk, n_splits;      // keys per split (a multiple of 128), splits planned
+  float* part_o;            // [B][tokens][Hq][n_splits][D]
+  float* part_lse;          // [B][tokens][Hq][n_splits] (log2 domain)
+  int* status;
+  unsigned long long wait_ns;
+};
+cudaError_t launch_verify_attn_tc(const VerifyAttnArgs& a, int B, int D, cudaStream_t st);
+cudaError_t launch_verify_attn_rows(const VerifyAttnArgs& a, int B, int D, cudaStream_t st);
+int verify_tc_rows(int Hq, int Hkv, int tokens, int D);
 cudaError_t launch_quantize_rows(const QuantRowsArgs& a, int B, int D, cudaStream_t st);
 // tcgen05 prefill (head_dim 256 or 512). key_rows_total = rows of the K/V
 // views; kv_token_major: views are [B][rows][Hkv][D] (1) or [B][Hkv][rows][D] (0).

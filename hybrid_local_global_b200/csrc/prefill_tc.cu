@@ -101,6 +101,12 @@ struct TcArgs {
   // view batch = page_table[b * pages_per_seq + position / page_size]; null: contiguous
   const int32_t* page_table;
   int page_size, pages_per_seq, n_pages;
+  // multi-token decode (VF instances): rows (token t, q head g * G + i) = t * G + i
+  // of KV head g, keys [split * chunk, +chunk) of the sequence's seq_lens[b]
+  const int32_t* seq_lens;
+  int tokens, chunk, n_splits;
+  float* part_o;
+  float* part_lse;
 };
 
 __device__ __forceinline__ bool wait_all(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
@@ -147,7 +153,12 @@ __device__ __forceinline__ float max_row(const uint32_t (&r)[4][32]) {
   return max8(mx);
 }
 
-template <int D>
+// VF: the multi-token decode instance (see launch_verify_attn_rows): a CTA is
+// (KV head g and output half, sequence b, key split); its 128-row tile holds
+// the G q heads of g for each of the `tokens` new tokens (rows past G *
+// tokens see no key), and it writes fp32 partials O / l and log2-sum-exp for
+// the combine instead of bf16 rows.
+template <int D, bool VF>
 __global__ void __launch_bounds__(192, 1)
     k_prefill_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
@@ -164,22 +175,39 @@ __global__ void __launch_bounds__(192, 1)
   Ctl<NSTAGE>* ctl = reinterpret_cast<Ctl<NSTAGE>*>(sm + Q_B + NSTAGE * STAGE_B);
   volatile int* abort_flag = &ctl->abort;
 
-  const int h = blockIdx.x / Cfg::NV, vh = blockIdx.x % Cfg::NV, b = blockIdx.y;
-  const int qt = a.n_qtiles - 1 - (int)blockIdx.z;
-  const int q0 = qt * BM;
-  const int g = h / (a.Hq / a.Hkv);
+  const int G = a.Hq / a.Hkv;
+  const int vh = blockIdx.x % Cfg::NV, b = blockIdx.y;
+  const int h = VF ? 0 : (int)blockIdx.x / Cfg::NV;  // VF: per row, g * G + row % G
+  const int g = VF ? (int)blockIdx.x / Cfg::NV : h / G;
+  const int q0 = VF ? 0 : (a.n_qtiles - 1 - (int)blockIdx.z) * BM;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  const int64_t pos0 = a.seq_lens_before ? (int64_t)a.seq_lens_before[b] : 0;
-  const int64_t n_keys = pos0 + a.S;
+  int64_t pos0, n_keys, kt0;
+  int n_tiles;
+  if (VF) {
+    // token t sits at position seq_lens[b] - tokens + t; this CTA reads keys
+    // [split * chunk, min(+chunk, seq_lens[b]))
+    n_keys = a.seq_lens[b];
+    pos0 = n_keys - a.tokens;
+    const int64_t k_begin = (int64_t)blockIdx.z * a.chunk;
+    if (pos0 < 0 || n_keys > a.key_cap || k_begin >= n_keys) return;  // range reported by the append kernel
+    const int64_t k_end = k_begin + a.chunk < n_keys ? k_begin + a.chunk : n_keys;
+    kt0 = k_begin / BN;
+    n_tiles = (int)((k_end - 1) / BN - kt0 + 1);
+  } else {
+    pos0 = a.seq_lens_before ? (int64_t)a.seq_lens_before[b] : 0;
+    n_keys = pos0 + a.S;
+  }
   // view row of a key = its position - koff (a gathered key window starts at pos0 - window)
-  const int64_t koff = a.key_off_window ? pos0 - a.window : 0;
-  if (pos0 < 0 || n_keys - koff > a.key_cap) return;  // reported by the RoPE kernel
-  int64_t lo_first, hi_first, lo_last, hi_last;
-  visible_range(pos0 + q0, a.window, n_keys, &lo_first, &hi_first);
-  visible_range(pos0 + min(q0 + BM - 1, a.S - 1), a.window, n_keys, &lo_last, &hi_last);
-  const int64_t kt0 = lo_first / BN;
-  const int n_tiles = (int)(hi_last / BN - kt0 + 1);
+  const int64_t koff = (!VF && a.key_off_window) ? pos0 - a.window : 0;
+  if (!VF) {
+    if (pos0 < 0 || n_keys - koff > a.key_cap) return;  // reported by the RoPE kernel
+    int64_t lo_first, hi_first, lo_last, hi_last;
+    visible_range(pos0 + q0, a.window, n_keys, &lo_first, &hi_first);
+    visible_range(pos0 + min(q0 + BM - 1, a.S - 1), a.window, n_keys, &lo_last, &hi_last);
+    kt0 = lo_first / BN;
+    n_tiles = (int)(hi_last / BN - kt0 + 1);
+  }
 
   if (threadIdx.x == 0) {
     mbar_init(&ctl->q_full, 1);
@@ -217,9 +245,16 @@ __global__ void __launch_bounds__(192, 1)
       tc::prefetch_tmap(&tm_q);
       tc::prefetch_tmap(&tm_k);
       tc::prefetch_tmap(&tm_v);
-      mbar_arrive_expect_tx(&ctl->q_full, Q_B);
-      for (int c = 0; c < D / 64; ++c)
-        tc::tma_load_4d(sQ + c * CHUNK_B, &tm_q, c * 64, h, q0, b, smem_u32(&ctl->q_full));
+      if (VF) {
+        // G heads x tokens rows; the tile's other rows are never stored
+        mbar_arrive_expect_tx(&ctl->q_full, (uint32_t)(D * 2 * G * a.tokens));
+        for (int c = 0; c < D / 64; ++c)
+          tc::tma_load_4d(sQ + c * CHUNK_B, &tm_q, c * 64, g * G, 0, b, smem_u32(&ctl->q_full));
+      } else {
+        mbar_arrive_expect_tx(&ctl->q_full, Q_B);
+        for (int c = 0; c < D / 64; ++c)
+          tc::tma_load_4d(sQ + c * CHUNK_B, &tm_q, c * 64, h, q0, b, smem_u32(&ctl->q_full));
+      }
       ctl->q_issued = 1;
       int item = 0;
       bool ok = true;
@@ -362,9 +397,15 @@ __global__ void __launch_bounds__(192, 1)
     const int wq = warp & 3;
     const int row = wq * 32 + lane;
     const uint32_t tm = tmem + ((uint32_t)(wq * 32) << 16);
-    const bool row_valid = q0 + row < a.S;
+    const bool row_valid = VF ? row < G * a.tokens : q0 + row < a.S;
     int64_t lo, hi;
-    visible_range(pos0 + (row_valid ? q0 + row : a.S - 1), a.window, n_keys, &lo, &hi);
+    if (VF) {
+      // keys up to the row's token (global layer); a row past the tokens sees none
+      lo = row_valid ? 0 : 1;
+      hi = row_valid ? pos0 + row / G : 0;
+    } else {
+      visible_range(pos0 + (row_valid ? q0 + row : a.S - 1), a.window, n_keys, &lo, &hi);
+    }
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
     int pv_seen = 0;  // P.V products whose completion this thread has consumed
@@ -470,7 +511,30 @@ __global__ void __launch_bounds__(192, 1)
     // 16 bytes per output row per instruction; the staged copy writes whole
     // rows. Rows past the sequence end are clipped by the store.
     unsigned char* sO = sm;  // Q buffer
-    if (ok) {
+    if (VF) {
+      // fp32 partial O / l of this split and its log2-sum-exp, for the combine
+      if (ok) {
+        tc::fence_after_sync();
+        const float inv = l > 0.f ? 1.f / l : 0.f;
+        const int t = row / G;
+        const int64_t pr = (((int64_t)b * a.tokens + t) * a.Hq + g * G + row % G) * a.n_splits + blockIdx.z;
+        float* dst = a.part_o + pr * D + vh * DV;
+#pragma unroll 1
+        for (int c = 0; c < 8; ++c) {
+          uint32_t o[32];
+          tc::tmem_ld32(tm + COL_O + c * 32, o);  // every lane: the load is warp-wide
+          tc::tmem_wait_ld();
+          if (row_valid) {
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+              *reinterpret_cast<float4*>(dst + c * 32 + u * 4) =
+                  make_float4(__uint_as_float(o[u * 4 + 0]) * inv, __uint_as_float(o[u * 4 + 1]) * inv,
+                              __uint_as_float(o[u * 4 + 2]) * inv, __uint_as_float(o[u * 4 + 3]) * inv);
+          }
+        }
+        if (row_valid && vh == 0) a.part_lse[pr] = l > 0.f ? m_used + __log2f(l) : -INFINITY;
+      }
+    } else if (ok) {
       tc::fence_after_sync();
       const float inv = l > 0.f ? 1.f / l : 0.f;
 #pragma unroll 1
@@ -496,7 +560,7 @@ __global__ void __launch_bounds__(192, 1)
     }
     fence_proxy_async_smem();
     asm volatile("bar.sync 1, 128;" ::: "memory");  // the four softmax warps
-    if (warp == 2 && lane == 0 && !*abort_flag) {
+    if (!VF && warp == 2 && lane == 0 && !*abort_flag) {
       for (int c = 0; c < DV / 64; ++c)
         tc::tma_store_4d(&tm_o, smem_u32(sO + c * CHUNK_B), vh * DV + c * 64, h, q0, b);
       tc::bulk_commit();
@@ -551,18 +615,83 @@ cudaError_t launch_prefill_attn_tc(const PrefillAttnArgs& a, int B, int D, int k
   t.n_qtiles = (a.S + BM - 1) / BM;
   if (D == 256) {
     using Cfg = TcCfg<256>;
-    cudaError_t e = cudaFuncSetAttribute(k_prefill_tc<256>, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);
+    cudaError_t e =
+        cudaFuncSetAttribute(k_prefill_tc<256, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);
     if (e != cudaSuccess) return e;
     dim3 grid(a.Hq * Cfg::NV, B, t.n_qtiles);
-    k_prefill_tc<256><<<grid, 192, Cfg::SMEM, st>>>(mq, mk, mv, mo, t);
+    k_prefill_tc<256, false><<<grid, 192, Cfg::SMEM, st>>>(mq, mk, mv, mo, t);
   } else {
     using Cfg = TcCfg<512>;
-    cudaError_t e = cudaFuncSetAttribute(k_prefill_tc<512>, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);
+    cudaError_t e =
+        cudaFuncSetAttribute(k_prefill_tc<512, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);
     if (e != cudaSuccess) return e;
     dim3 grid(a.Hq * Cfg::NV, B, t.n_qtiles);
-    k_prefill_tc<512><<<grid, 192, Cfg::SMEM, st>>>(mq, mk, mv, mo, t);
+    k_prefill_tc<512, false><<<grid, 192, Cfg::SMEM, st>>>(mq, mk, mv, mo, t);
   }
   return cudaGetLastError();
+}
+
+namespace {
+template <int D>
+cudaError_t launch_verify_as(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const TcArgs& t,
+                             int B, cudaStream_t st) {
+  using Cfg = TcCfg<D>;
+  cudaError_t e = cudaFuncSetAttribute(k_prefill_tc<D, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);
+  if (e != cudaSuccess) return e;
+  dim3 grid(t.Hkv * Cfg::NV, B, t.n_splits);
+  k_prefill_tc<D, true><<<grid, 192, Cfg::SMEM, st>>>(mq, mk, mv, mq, t);
+  return cudaGetLastError();
+}
+}  // namespace
+
+cudaError_t launch_verify_attn_rows(const VerifyAttnArgs& a, int B, int D, cudaStream_t st) {
+  const int G = a.Hq / a.Hkv;
+  if ((D != 256 && D != 512) || a.tokens < 1 || G * a.tokens > BM || a.chunk % BN || a.n_splits < 1)
+    return cudaErrorInvalidValue;
+  const uint64_t E = 2;
+  CUtensorMap mq, mk, mv;
+  {
+    // q_rot [B][tokens][Hq][D]: a box is the G heads of one KV head for every token
+    const uint64_t dims[4] = {(uint64_t)D, (uint64_t)a.Hq, (uint64_t)a.tokens, (uint64_t)B};
+    const uint64_t str[3] = {(uint64_t)D * E, (uint64_t)a.Hq * D * E, (uint64_t)a.tokens * a.Hq * D * E};
+    const uint32_t box[4] = {64, (uint32_t)G, (uint32_t)a.tokens, 1};
+    if (!make_map_bf16_4d(&mq, a.q_rot, dims, str, box)) return cudaErrorInvalidValue;
+  }
+  {
+    // head-major cache views: (d, key, head, b), K boxes of 128 keys, V boxes of 64
+    const uint64_t dims[4] = {(uint64_t)D, (uint64_t)a.cache_cap, (uint64_t)a.Hkv, (uint64_t)B};
+    const uint64_t strk[3] = {(uint64_t)a.k.stride_row * E, (uint64_t)a.k.stride_h * E, (uint64_t)a.k.stride_b * E};
+    const uint64_t strv[3] = {(uint64_t)a.v.stride_row * E, (uint64_t)a.v.stride_h * E, (uint64_t)a.v.stride_b * E};
+    const uint32_t bk[4] = {64, (uint32_t)BN, 1, 1}, bv[4] = {64, 64, 1, 1};
+    if (!make_map_bf16_4d(&mk, a.k.ptr, dims, strk, bk) || !make_map_bf16_4d(&mv, a.v.ptr, dims, strv, bv))
+      return cudaErrorInvalidValue;
+  }
+  TcArgs t{};
+  t.S = a.tokens;
+  t.window = 0;
+  t.Hq = a.Hq;
+  t.Hkv = a.Hkv;
+  t.key_cap = a.cache_cap;
+  t.seq_lens_before = nullptr;
+  t.scale_log2 = 1.f;
+  t.out = nullptr;
+  t.lse = nullptr;
+  t.status = a.status;
+  t.wait_ns = a.wait_ns;
+  t.kv_token_major = 0;
+  t.key_off_window = 0;
+  t.n_qtiles = 1;
+  t.page_table = nullptr;
+  t.page_size = a.cache_cap;
+  t.pages_per_seq = 1;
+  t.n_pages = B;
+  t.seq_lens = a.seq_lens;
+  t.tokens = a.tokens;
+  t.chunk = a.chunk;
+  t.n_splits = a.n_splits;
+  t.part_o = a.part_o;
+  t.part_lse = a.part_lse;
+  return D == 256 ? launch_verify_as<256>(mq, mk, mv, t, B, st) : launch_verify_as<512>(mq, mk, mv, t, B, st);
 }
 
 }  // namespace hlg

@@ -327,14 +327,17 @@ __global__ void __launch_bounds__(256) k_gather_q8(const uint8_t* __restrict__ k
 // Decode: one token per sequence at position seq_lens[b]-1.
 template <int D>
 __global__ void __launch_bounds__(256) k_decode_rope_append(DecodeRopeArgs a) {
-  const int b = blockIdx.x;
+  // one block per (sequence, new token): bt = b * tokens + t, the layout of
+  // q, k_new, v_new and q_rot
+  const int bt = blockIdx.x;
+  const int b = bt / a.tokens;
   const int e0 = threadIdx.x * 8;
   const int64_t len = a.seq_lens[b];
-  if (len < 1 || len > a.max_len) {
+  if (len < a.tokens || len > a.max_len) {
     if (threadIdx.x == 0 && threadIdx.y == 0) set_status(a.status, GEMMA_ERR_DEVICE_RANGE);
     return;
   }
-  const int64_t pos = len - 1;
+  const int64_t pos = len - a.tokens + bt % a.tokens;
   const int64_t slot = a.window > 0 ? pos % a.window : pos;
   if (slot >= a.cache_cap) {
     if (threadIdx.x == 0 && threadIdx.y == 0) set_status(a.status, GEMMA_ERR_DEVICE_RANGE);
@@ -348,13 +351,15 @@ __global__ void __launch_bounds__(256) k_decode_rope_append(DecodeRopeArgs a) {
   const int n_heads = a.Hq + (a.k_new ? a.Hkv : 0) + ((a.v_new && !a.k_stage) ? a.Hkv : 0);
   for (int h = threadIdx.y; h < n_heads; h += blockDim.y) {
     if (h < a.Hq) {
-      const int64_t off = ((int64_t)b * a.Hq + h) * D + e0;
-      st16(a.q_rot + off, rotate_chunk(ld16(a.q + off), t, e0, a.n_rot));
+      const int64_t off = ((int64_t)bt * a.Hq + h) * D + e0;
+      const uint4 x = ld16(a.q + off);
+      st16(a.q_rot + off, a.q_scale == 1.f ? rotate_chunk(x, t, e0, a.n_rot)
+                                           : rotate_scale_chunk(x, t, e0, a.n_rot, a.q_scale));
       continue;
     }
     const bool is_k = h < a.Hq + a.Hkv;
     const int kh = is_k ? h - a.Hq : h - a.Hq - a.Hkv;
-    const int64_t src_off = ((int64_t)b * a.Hkv + kh) * D + e0;
+    const int64_t src_off = ((int64_t)bt * a.Hkv + kh) * D + e0;
     uint4 v = is_k ? rotate_chunk(ld16(a.k_new + src_off), t, e0, a.n_rot)
                    : ld16(a.v_new + src_off);
     if (a.k_stage) {  // int8 cache: the rotated key waits for the quantize kernel
@@ -508,13 +513,27 @@ cudaError_t launch_gather_q8(const uint8_t* k_codes, const float2* k_params, con
   return cudaGetLastError();
 }
 
+// lens_before[b] = seq_lens[b] - tokens: the cached length before a
+// multi-token step, for the chunked-prefill route of such a step.
+__global__ void k_lens_minus(const int32_t* __restrict__ seq_lens, int32_t* __restrict__ lens_before, int B,
+                             int tokens) {
+  const int b = blockIdx.x * blockDim.x + threadIdx.x;
+  if (b < B) lens_before[b] = seq_lens[b] - tokens;
+}
+
+cudaError_t launch_lens_minus(const int32_t* seq_lens, int32_t* lens_before, int B, int tokens, cudaStream_t st) {
+  k_lens_minus<<<(B + 127) / 128, 128, 0, st>>>(seq_lens, lens_before, B, tokens);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_decode_rope_append(const DecodeRopeArgs& a, int B, int D, cudaStream_t st) {
   const int tx = D / 8;
   dim3 block(tx, 256 / tx);
+  if (a.tokens < 1) return cudaErrorInvalidValue;
   if (D == 256)
-    k_decode_rope_append<256><<<B, block, 0, st>>>(a);
+    k_decode_rope_append<256><<<B * a.tokens, block, 0, st>>>(a);
   else
-    k_decode_rope_append<512><<<B, block, 0, st>>>(a);
+    k_decode_rope_append<512><<<B * a.tokens, block, 0, st>>>(a);
   return cudaGetLastError();
 }
 

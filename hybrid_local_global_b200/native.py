@@ -73,6 +73,9 @@ _prefill_paged = _sig("gemma_attn_prefill_paged", _I, [_P, _P, _P, _P, _P, _P, _
 _decode_paged = _sig("gemma_attn_decode_paged", _I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _P, _I, _I, _I, _I, _I,
                                                      _F, _F, _F, _P, _P, _SZ, ctypes.c_uint, _P])
 _kv_codes = _sig("gemma_kv_codes_bytes", _SZ, [_I, _I, _I, _I])
+_multi_ws = _sig("gemma_attn_decode_multi_workspace_size", _SZ, [_I, _I, _I, _I, _I, _I, _I, _I, ctypes.c_uint])
+_multi = _sig("gemma_attn_decode_multi", _I, [_P, _P, _P, _P, _P, _I, _P, _I, _I, _I, _I, _I, _I, _I,
+                                              _F, _F, _F, _P, _P, _SZ, ctypes.c_uint, _P])
 
 EXPORTED = ["gemma_attn_prefill_workspace_size", "gemma_attn_prefill",
             "gemma_attn_decode_workspace_size", "gemma_attn_decode", "gemma_kv_share_bind",
@@ -211,6 +214,32 @@ def gemma_attn_decode(q, k_new, v_new, k_cache, v_cache, *, seq_lens, max_seq_le
                           _stream(stream)))
 
 
+def gemma_attn_decode_multi_workspace_size(batch, tokens, n_q_heads, n_kv_heads, head_dim, window, max_seq_len,
+                                           cache_cap, flags=0) -> int:
+    return int(_multi_ws(batch, tokens, n_q_heads, n_kv_heads, head_dim, window, max_seq_len, cache_cap, flags))
+
+
+def gemma_attn_decode_multi(q, k_new, v_new, k_cache, v_cache, *, seq_lens, max_seq_len, window,
+                            rope_frac, rope_theta, scale, out, workspace=None, flags=0, stream=None):
+    """q [B,T,Hq,D]; k_new/v_new [B,T,Hkv,D] (None if shared); caches [B,Hkv,cap,D];
+    seq_lens int32 [B] on the device (length including the T new tokens)."""
+    for t, n in ((q, "q"), (k_new, "k_new"), (v_new, "v_new"), (k_cache, "k_cache"),
+                 (v_cache, "v_cache"), (out, "out")):
+        _bf16(t, n)
+    if seq_lens.dtype != torch.int32 or not seq_lens.is_cuda:
+        raise TypeError("seq_lens must be an int32 CUDA tensor")
+    B, T, Hq, D = q.shape
+    _, Hkv, cap, _ = k_cache.shape
+    flags |= _kv_kind(k_cache, v_cache)
+    if workspace is None:
+        n = gemma_attn_decode_multi_workspace_size(B, T, Hq, Hkv, D, window, max_seq_len, cap, flags)
+        workspace = torch.empty(max(n, 1), dtype=torch.uint8, device=q.device)
+    return _check(_multi(_ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_cache), _ptr(v_cache), cap,
+                         _ptr(seq_lens), max_seq_len, B, T, window, Hq, Hkv, D, rope_frac,
+                         rope_theta, scale, _ptr(out), _ptr(workspace), workspace.numel(), flags,
+                         _stream(stream)))
+
+
 def _paged_args(k_pool, page_table):
     if page_table.dtype != torch.int32 or not page_table.is_cuda or page_table.dim() != 2:
         raise TypeError("page_table must be an int32 CUDA tensor [batch, pages_per_seq]")
@@ -326,7 +355,7 @@ def gemma_attn_profile_read(kernel: int):
 
 _decode_noalloc = _sig("gemma_attn_decode_noalloc", _I, [_P, _P, _P, _P, _P, _I, _P, _I, _I, _I, _I, _I,
                                                          _I, _F, _F, _F, _P, ctypes.c_uint, _P])
-EXPORTED += ["gemma_attn_decode_noalloc"]
+EXPORTED += ["gemma_attn_decode_noalloc", "gemma_attn_decode_multi_workspace_size", "gemma_attn_decode_multi"]
 NOALLOC_SCRATCH_BYTES = 32 << 20
 
 

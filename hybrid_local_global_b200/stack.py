@@ -175,3 +175,29 @@ class AttentionStack:
             rope_theta=t.rope_theta, scale=t.scale, out=out, workspace=workspace,
             flags=(native.GEMMA_F_SHARED if shared else 0) | (native.GEMMA_F_KEQV if keqv else 0),
             stream=stream)
+
+    # ------------------------------------------------------- multi-token decode
+    def decode_multi_workspace_bytes(self, tokens: int, max_seq_len: int) -> int:
+        w = self.w
+        flags = native.GEMMA_F_KV_INT8 if w.kv_int8 else 0
+        sizes = []
+        for l in range(self.n_layers):
+            t = self.layer_type(l)
+            cap = t.window if t.window > 0 else self.global_capacity
+            sizes.append(native.gemma_attn_decode_multi_workspace_size(
+                w.batch, tokens, w.n_q_heads, t.n_kv_heads, t.head_dim, t.window, max_seq_len, cap, flags))
+        return max(sizes)
+
+    def decode_multi_layer(self, l: int, q, k, v, out, *, seq_lens, max_seq_len, workspace, stream=None):
+        """tokens = q.shape[1] new tokens per sequence (a drafter's proposals
+        being checked); seq_lens counts them."""
+        t = self.layer_type(l)
+        shared = self.is_shared(l)
+        keqv = self.keqv(l)
+        native.gemma_attn_decode_multi(
+            q, None if shared else k, None if (shared or keqv) else v, self.k_cache[l],
+            None if keqv else self.v_cache[l],
+            seq_lens=seq_lens, max_seq_len=max_seq_len, window=t.window, rope_frac=t.rope_frac,
+            rope_theta=t.rope_theta, scale=t.scale, out=out, workspace=workspace,
+            flags=(native.GEMMA_F_SHARED if shared else 0) | (native.GEMMA_F_KEQV if keqv else 0),
+            stream=stream)

@@ -190,6 +190,48 @@ int gemma_attn_decode(const void* q, const void* k_new, const void* v_new,
                       void* stream);
 
 /* ---------------------------------------------------------------------- */
+/* Multi-token decode: `tokens` new tokens per sequence, each attending to */
+/* the cache and to the earlier new tokens -- the target model's pass that */
+/* checks a drafter's proposals in speculative decoding ("Gemma 4: End-to- */
+/* End Architecture Walkthrough", Phase 4, multi-token prediction drafters;*/
+/* "Gemma 4: Architecture, Training and Local Deployment", 3.4). The       */
+/* result equals tokens consecutive gemma_attn_decode calls (or a         */
+/* gemma_attn_prefill of the tokens after seq_lens - tokens cached ones).  */
+/*                                                                        */
+/* q      [batch][tokens][n_q_heads][head_dim] pre-RoPE queries            */
+/* k_new, v_new [batch][tokens][n_kv_heads][head_dim] pre-RoPE keys /      */
+/*        values (NULL with GEMMA_F_SHARED; v_new NULL with GEMMA_F_KEQV)  */
+/* seq_lens device int32 [batch]: sequence length INCLUDING the new        */
+/*        tokens; token t sits at position seq_lens[b] - tokens + t. Every */
+/*        value must be in [tokens, max_seq_len]; a device-side check      */
+/*        reports others as GEMMA_ERR_DEVICE_RANGE.                        */
+/* max_seq_len host upper bound of seq_lens (sizes the split grid).        */
+/* out    [batch][tokens][n_q_heads][head_dim] bf16.                       */
+/* workspace: gemma_attn_decode_multi_workspace_size(...) bytes, 256-byte  */
+/*        aligned; scratch.                                                */
+/*                                                                        */
+/* A global bf16 layer on a contiguous cache with (n_q_heads / n_kv_heads) */
+/* * tokens <= 128 runs one tensor-core kernel per split of the cached    */
+/* keys whose tile holds every q head of a KV head for all the tokens, so */
+/* the cache is streamed once per step as in single-token decode. Other   */
+/* layers (local, int8) run as a chunked prefill; a shared local layer is */
+/* GEMMA_ERR_UNSUPPORTED there, as in gemma_attn_prefill after cached     */
+/* tokens. Cache effects: the rotated new keys and the values are written */
+/* at their positions' slots, unless the layer is shared.                 */
+/* ---------------------------------------------------------------------- */
+size_t gemma_attn_decode_multi_workspace_size(int batch, int tokens, int n_q_heads,
+                                              int n_kv_heads, int head_dim, int window,
+                                              int max_seq_len, int cache_cap, unsigned flags);
+
+int gemma_attn_decode_multi(const void* q, const void* k_new, const void* v_new,
+                            void* k_cache, void* v_cache, int cache_cap,
+                            const int32_t* seq_lens, int max_seq_len, int batch, int tokens,
+                            int window, int n_q_heads, int n_kv_heads, int head_dim,
+                            float rope_frac, float rope_theta, float scale, void* out,
+                            void* workspace, size_t workspace_bytes, unsigned flags,
+                            void* stream);
+
+/* ---------------------------------------------------------------------- */
 /* Paged global cache ("Gemma 4: End-to-End Architecture Walkthrough", 3b: */
 /* a global layer caches K/V for the whole context; paging lets the pool   */
 /* grow with the tokens actually held instead of a per-sequence capacity). */

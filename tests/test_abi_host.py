@@ -188,6 +188,57 @@ def test_decode_validation(over, code):
     assert _decode_raw(**over) == code
 
 
+def _multi_raw(**over):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, kc=FAKE, vc=FAKE, cap=4096, lens=FAKE, maxlen=4096, B=2, T=4, W=0,
+             Hq=32, Hkv=4, D=512, frac=0.25, theta=1e6, scale=0.044, out=FAKE, ws=FAKE,
+             wsb=16, flags=0)
+    a.update(over)
+    return native._multi(a["q"], a["k"], a["v"], a["kc"], a["vc"], a["cap"], a["lens"], a["maxlen"],
+                         a["B"], a["T"], a["W"], a["Hq"], a["Hkv"], a["D"], a["frac"], a["theta"],
+                         a["scale"], a["out"], a["ws"], a["wsb"], a["flags"], None)
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(), E.GEMMA_ERR_CAPACITY),                                   # the tensor-core path: accepted
+    (dict(T=0), E.GEMMA_ERR_INVALID_ARG),
+    (dict(lens=None), E.GEMMA_ERR_INVALID_ARG),
+    (dict(maxlen=0), E.GEMMA_ERR_INVALID_ARG),
+    (dict(cap=1000), E.GEMMA_ERR_CAPACITY),                           # global cache < max length
+    (dict(D=384), E.GEMMA_ERR_UNSUPPORTED),
+    (dict(k=None, v=None), E.GEMMA_ERR_INVALID_ARG),                  # unshared layer without new keys
+    (dict(flags=1), E.GEMMA_ERR_INVALID_ARG),                         # shared layer with new keys
+    (dict(flags=1, k=None, v=None), E.GEMMA_ERR_CAPACITY),            # shared global: accepted
+    (dict(flags=2), E.GEMMA_ERR_INVALID_ARG),                         # K = V with v_new
+    (dict(flags=2, v=None, vc=None), E.GEMMA_ERR_CAPACITY),           # K = V: accepted
+    (dict(q=FAKE + 8, wsb=1 << 30), E.GEMMA_ERR_INVALID_ARG),         # misaligned
+    (dict(out=None, wsb=1 << 30), E.GEMMA_ERR_INVALID_ARG),
+    (dict(T=17), E.GEMMA_ERR_CAPACITY),                               # 8 x 17 rows: the prefill route
+    (dict(T=17, out=None, wsb=1 << 30), E.GEMMA_ERR_INVALID_ARG),     # ... which validates as prefill
+    (dict(W=1024, cap=1024, Hkv=16, D=256, frac=1.0, theta=1e4), E.GEMMA_ERR_CAPACITY),  # local: route
+    (dict(W=1024, cap=4096, Hkv=16, D=256, frac=1.0, theta=1e4, wsb=1 << 30), E.GEMMA_ERR_INVALID_ARG),
+    (dict(W=1024, cap=1024, Hkv=16, D=256, frac=1.0, theta=1e4, flags=1, k=None, v=None, wsb=1 << 30),
+     E.GEMMA_ERR_UNSUPPORTED),                                        # shared local after cached tokens
+    (dict(flags=4), E.GEMMA_ERR_CAPACITY),                            # int8: route
+])
+def test_decode_multi_validation(over, code):
+    assert _multi_raw(**over) == code
+    assert native.gemma_last_error()
+
+
+def test_decode_multi_workspace_sizes():
+    """The tensor-core path holds the rotated queries and fp32 split
+    partials; the routed layers a length buffer plus the chunked-prefill
+    workspace."""
+    n = native.gemma_attn_decode_multi_workspace_size(64, 4, 32, 4, 512, 0, 131072, 131072, 0)
+    assert n >= 64 * 4 * 32 * 512 * (2 + 4)
+    loc = native.gemma_attn_decode_multi_workspace_size(64, 4, 32, 16, 256, 1024, 131072, 1024, 0)
+    assert loc >= 256 + native.gemma_attn_prefill_workspace_size_cached(64, 4, 32, 16, 256, 1024, 1024, 0)
+    q8 = native.gemma_attn_decode_multi_workspace_size(2, 4, 32, 4, 512, 0, 4096, 4096, native.GEMMA_F_KV_INT8)
+    assert q8 >= native.gemma_attn_prefill_workspace_size_cached(2, 4, 32, 4, 512, 0, 4096, native.GEMMA_F_KV_INT8)
+    assert native.gemma_attn_decode_multi_workspace_size(0, 4, 32, 4, 512, 0, 4096, 4096, 0) == 0
+    assert native.gemma_attn_decode_multi_workspace_size(2, 0, 32, 4, 512, 0, 4096, 4096, 0) == 0
+
+
 def test_cached_prefill_workspace_sizes():
     """Only an int8 global layer after cached tokens needs more: its keys and
     values up to the capacity in bf16."""

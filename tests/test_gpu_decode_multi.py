@@ -1,0 +1,270 @@
+"""GPU parity of multi-token decode (several new tokens per sequence, as when
+the target model checks a drafter's proposals in speculative decoding)
+against the fp64 oracle, through the C ABI: the tensor-core path of global
+bf16 layers (q heads x tokens packed in one tile, split over the cached
+keys, combined), and the chunked-prefill route of local and int8 layers;
+cache slots written, KV sharing, K = V and the device range check."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from hybrid_local_global_b200 import native, synth
+from hybrid_local_global_b200.stack import AttentionStack
+from hybrid_local_global_b200.workloads import L31B_GLOBAL, L31B_LOCAL, Workload
+
+from gpu_util import assert_close, assert_rotated_bf16, to_bits
+
+pytestmark = pytest.mark.gpu
+
+
+def run_multi_case(oracle, *, lens, T, Hq, Hkv, D, W, frac, theta, seed, shared=False, keqv=False,
+                   cap_extra=16):
+    dev = torch.device("cuda")
+    B = len(lens)
+    g = synth.generator(seed)
+    max_len = max(lens)
+    cap = W if W else max_len + cap_extra
+    kc = torch.full((B, Hkv, cap, D), float("nan"), dtype=torch.bfloat16)
+    vc = kc.clone()
+    k_log = torch.zeros((B, max_len, Hkv, D), dtype=torch.bfloat16)
+    v_log = torch.zeros_like(k_log)
+    for b in range(B):
+        n = lens[b] - T
+        first = max(0, n - W) if W else 0
+        kr = synth.randn_bf16((Hkv, n - first, D), g)
+        vr = synth.randn_bf16((Hkv, n - first, D), g)
+        for i, p in enumerate(range(first, n)):
+            slot = p % W if W else p
+            kc[b, :, slot], vc[b, :, slot] = kr[:, i], vr[:, i]
+        k_log[b, first:n] = kr.transpose(0, 1)
+        v_log[b, first:n] = vr.transpose(0, 1)
+    q = synth.randn_bf16((B, T, Hq, D), g)
+    kn = synth.randn_bf16((B, T, Hkv, D), g)
+    vn = synth.randn_bf16((B, T, Hkv, D), g)
+    for b in range(B):
+        n = lens[b] - T
+        k_log[b, n:lens[b]] = kn[b]
+        v_log[b, n:lens[b]] = vn[b]
+        if shared:
+            # the new tokens' K/V are in the (source layer's) cache already, rotated
+            for t in range(T):
+                slot = (n + t) % W if W else n + t
+                kc[b, :, slot], vc[b, :, slot] = kn[b, t], vn[b, t]
+    if keqv:
+        vc, vn, v_log = kc, kn, None
+    kcd = kc.to(dev)
+    vcd = kcd if keqv else vc.to(dev)
+    out = torch.full((B, T, Hq, D), float("nan"), dtype=torch.bfloat16, device=dev)
+    sl = torch.tensor(lens, dtype=torch.int32, device=dev)
+    scale = 1.0 / math.sqrt(D)
+    flags = (native.GEMMA_F_SHARED if shared else 0) | (native.GEMMA_F_KEQV if keqv else 0)
+    native.gemma_attn_decode_multi(q.to(dev), None if shared else kn.to(dev),
+                                   None if (shared or keqv) else vn.to(dev), kcd, None if keqv else vcd,
+                                   seq_lens=sl, max_seq_len=max_len, window=W, rope_frac=frac,
+                                   rope_theta=theta, scale=scale, out=out, flags=flags)
+    assert native.gemma_attn_sync_status() == 0, native.gemma_last_error()
+    before = [L - T for L in lens]
+    ref, _ = oracle.attention(to_bits(q), to_bits(k_log), None if keqv else to_bits(v_log), q_pos0=before,
+                              n_keys=lens, rot_from=lens if shared else before, window=W,
+                              rope_frac=frac, theta=theta, scale=scale)
+    got = out.float().cpu().double().numpy().transpose(0, 2, 1, 3).reshape(-1, D)
+    assert_close(got, ref, what="multi-token decode T=%d" % T)
+    kc1, vc1 = kcd.cpu(), vcd.cpu()
+    for b in range(B):
+        written = torch.zeros(cap, dtype=torch.bool)
+        for t in range(T):
+            p = before[b] + t
+            slot = p % W if W else p
+            if W and p < lens[b] - W:
+                continue  # overwritten later in the same call by a newer token
+            written[slot] = True
+            if shared:
+                continue
+            if not keqv:
+                assert torch.equal(vc1[b, :, slot], vn[b, t]), "V slot %d" % slot
+            for h in range(Hkv):
+                exp = torch.from_numpy(oracle.rope_bf16(to_bits(kn[b, t, h]), p, frac, theta)).to(torch.bfloat16)
+                assert_rotated_bf16(kc1[b, h, slot], exp, kn[b, t, h], "K slot %d" % slot)
+        keep = ~written if not shared else torch.ones(cap, dtype=torch.bool)
+        # unwritten slots keep their bytes (NaN included)
+        assert torch.equal(kc1[b][:, keep].view(torch.int16), kc[b][:, keep].view(torch.int16))
+        assert torch.equal(vc1[b][:, keep].view(torch.int16), vc[b][:, keep].view(torch.int16))
+    return out
+
+
+GLOBAL_CASES = [
+    dict(lens=[3000, 700], T=4, Hq=32, Hkv=4, D=512, seed=301),            # 31B global shape, 3 splits
+    dict(lens=[4], T=4, Hq=32, Hkv=4, D=512, seed=302),                    # the tokens are the sequence
+    dict(lens=[1, 2000], T=1, Hq=8, Hkv=1, D=512, seed=303),               # one token (= decode)
+    dict(lens=[2500, 130, 9], T=2, Hq=8, Hkv=1, D=512, seed=304),          # E2B global shape
+    dict(lens=[5000, 1031], T=8, Hq=32, Hkv=4, D=512, seed=305),           # 64 rows a tile
+    dict(lens=[1500, 16], T=16, Hq=32, Hkv=4, D=512, seed=306),            # 128 rows: the full tile
+    dict(lens=[2049, 300], T=3, Hq=8, Hkv=4, D=256, seed=307, frac=1.0, theta=1e4),  # head_dim 256
+    dict(lens=[1024, 1025], T=5, Hq=12, Hkv=2, D=512, seed=308),           # split edges, G = 6
+]
+
+
+@pytest.mark.parametrize("case", GLOBAL_CASES,
+                         ids=["31b", "LeqT", "T1", "e2b", "T8", "T16", "D256", "edges"])
+def test_multi_global_tensor_core(oracle, case):
+    case = dict(case)
+    run_multi_case(oracle, W=0, frac=case.pop("frac", 0.25), theta=case.pop("theta", 1e6), **case)
+
+
+def test_multi_global_shared(oracle):
+    run_multi_case(oracle, lens=[2100, 77], T=4, Hq=32, Hkv=4, D=512, W=0, frac=0.25, theta=1e6, seed=311,
+                   shared=True)
+
+
+def test_multi_global_keqv(oracle):
+    run_multi_case(oracle, lens=[1800, 5], T=4, Hq=32, Hkv=4, D=512, W=0, frac=0.25, theta=1e6, seed=312,
+                   keqv=True)
+
+
+def test_multi_global_exact_capacity(oracle):
+    """The last key sits in the last cache row (no padding past the sequence)."""
+    run_multi_case(oracle, lens=[1280, 1000], T=4, Hq=8, Hkv=1, D=512, W=0, frac=0.25, theta=1e6, seed=313,
+                   cap_extra=0)
+
+
+@pytest.mark.parametrize("case", [
+    dict(lens=[3000, 700, 4], T=4, Hq=32, Hkv=16, D=256, W=1024, seed=321),    # 31B local shape
+    dict(lens=[600, 65], T=3, Hq=8, Hkv=4, D=256, W=64, seed=322),             # ring wraps inside the call
+    dict(lens=[40], T=40, Hq=4, Hkv=2, D=256, W=16, seed=323),                 # more tokens than the window
+    dict(lens=[3000, 700], T=17, Hq=32, Hkv=4, D=512, W=0, seed=324, frac=0.25, theta=1e6),  # 136 rows: route
+], ids=["31b_local", "wrap", "T_gt_W", "global_route"])
+def test_multi_routed_layers(oracle, case):
+    case = dict(case)
+    run_multi_case(oracle, frac=case.pop("frac", 1.0), theta=case.pop("theta", 1e4), **case)
+
+
+def test_multi_int8_global_matches_prefill_route(oracle):
+    """An int8 global layer goes through the chunked prefill: the result is
+    bit-identical to gemma_attn_prefill after seq_lens - tokens cached tokens
+    on a copy of the same cache."""
+    dev = torch.device("cuda")
+    B, T, Hq, Hkv, D, lens = 2, 4, 32, 4, 512, [1500, 300]
+    cap = 1600
+    g = synth.generator(331, "cuda")
+    kc = synth.fill_int8_cache_(native.Int8KVCache(B, Hkv, cap, D, dev), g)
+    vc = synth.fill_int8_cache_(native.Int8KVCache(B, Hkv, cap, D, dev), g)
+    kc2, vc2 = native.Int8KVCache(B, Hkv, cap, D, dev), native.Int8KVCache(B, Hkv, cap, D, dev)
+    kc2.buf.copy_(kc.buf)
+    vc2.buf.copy_(vc.buf)
+    q = synth.randn_bf16((B, T, Hq, D), g, "cuda")
+    kn = synth.randn_bf16((B, T, Hkv, D), g, "cuda")
+    vn = synth.randn_bf16((B, T, Hkv, D), g, "cuda")
+    sl = torch.tensor(lens, dtype=torch.int32, device=dev)
+    before = torch.tensor([L - T for L in lens], dtype=torch.int32, device=dev)
+    kw = dict(rope_frac=0.25, rope_theta=1e6, scale=1.0 / math.sqrt(D))
+    o1 = torch.empty((B, T, Hq, D), dtype=torch.bfloat16, device=dev)
+    o2 = torch.empty_like(o1)
+    native.gemma_attn_decode_multi(q, kn, vn, kc, vc, seq_lens=sl, max_seq_len=max(lens), window=0, out=o1, **kw)
+    native.gemma_attn_prefill(q, kn, vn, kc2, vc2, window=0, out=o2, seq_lens_before=before, **kw)
+    assert native.gemma_attn_sync_status() == 0, native.gemma_last_error()
+    assert torch.equal(o1.view(torch.int16), o2.view(torch.int16))
+    assert torch.equal(kc.buf, kc2.buf) and torch.equal(vc.buf, vc2.buf)
+
+
+def test_multi_equals_consecutive_decodes(oracle):
+    """T tokens in one call against T single-token decode calls on a copy of
+    the cache: the same rows within the benchmark spec's tolerance (the two paths
+    round the query scaling differently), and the same cache bytes."""
+    dev = torch.device("cuda")
+    B, T, Hq, Hkv, D, lens = 3, 4, 32, 4, 512, [2000, 37, 4100]
+    cap = max(lens) + 8
+    g = synth.generator(341)
+    kc = synth.randn_bf16((B, Hkv, cap, D), g).to(dev)
+    vc = synth.randn_bf16((B, Hkv, cap, D), g).to(dev)
+    kc2, vc2 = kc.clone(), vc.clone()
+    q = synth.randn_bf16((B, T, Hq, D), g).to(dev)
+    kn = synth.randn_bf16((B, T, Hkv, D), g).to(dev)
+    vn = synth.randn_bf16((B, T, Hkv, D), g).to(dev)
+    kw = dict(window=0, rope_frac=0.25, rope_theta=1e6, scale=1.0 / math.sqrt(D))
+    o1 = torch.empty((B, T, Hq, D), dtype=torch.bfloat16, device=dev)
+    native.gemma_attn_decode_multi(q, kn, vn, kc, vc, seq_lens=torch.tensor(lens, dtype=torch.int32, device=dev),
+                                   max_seq_len=max(lens), out=o1, **kw)
+    o2 = torch.empty_like(o1)
+    for t in range(T):
+        sl = torch.tensor([L - T + t + 1 for L in lens], dtype=torch.int32, device=dev)
+        ot = torch.empty((B, Hq, D), dtype=torch.bfloat16, device=dev)
+        native.gemma_attn_decode(q[:, t].contiguous(), kn[:, t].contiguous(), vn[:, t].contiguous(), kc2, vc2,
+                                 seq_lens=sl, max_seq_len=max(lens), out=ot, **kw)
+        o2[:, t] = ot
+    assert native.gemma_attn_sync_status() == 0, native.gemma_last_error()
+    assert torch.equal(kc.view(torch.int16), kc2.view(torch.int16))
+    assert torch.equal(vc.view(torch.int16), vc2.view(torch.int16))
+    assert_close(o1.float().cpu().numpy(), o2.float().cpu().numpy(), what="one call vs T decode calls")
+
+
+def test_multi_range_check_reports(oracle):
+    """seq_lens below the token count: the device check reports
+    GEMMA_ERR_DEVICE_RANGE, writes zeros for that sequence, and the other
+    sequences are unaffected."""
+    dev = torch.device("cuda")
+    B, T, Hq, Hkv, D = 2, 4, 8, 1, 512
+    cap = 512
+    g = synth.generator(351)
+    kc = synth.randn_bf16((B, Hkv, cap, D), g).to(dev)
+    vc = synth.randn_bf16((B, Hkv, cap, D), g).to(dev)
+    q = synth.randn_bf16((B, T, Hq, D), g).to(dev)
+    kn = synth.randn_bf16((B, T, Hkv, D), g).to(dev)
+    vn = synth.randn_bf16((B, T, Hkv, D), g).to(dev)
+    out = torch.full((B, T, Hq, D), float("nan"), dtype=torch.bfloat16, device=dev)
+    sl = torch.tensor([300, 3], dtype=torch.int32, device=dev)
+    native.gemma_attn_decode_multi(q, kn, vn, kc, vc, seq_lens=sl, max_seq_len=300, window=0, rope_frac=0.25,
+                                   rope_theta=1e6, scale=1.0 / math.sqrt(D), out=out)
+    assert native.gemma_attn_sync_status() == native.GEMMA_ERR_DEVICE_RANGE
+    assert torch.count_nonzero(out[1].float()) == 0
+    assert torch.isfinite(out[0].float()).all()
+    assert native.gemma_attn_sync_status() == 0  # reading the status clears it
+
+
+def test_multi_stack_31b_block(oracle):
+    """k = 4 tokens per sequence through every layer of a 31B-shaped
+    6-layer stack (5 local with ring caches, 1 global) with the stack's
+    multi-token decode call."""
+    prior, kq = [3000, 700], 4
+    w = Workload("verify_k4", "decode", batch=2, n_q_heads=32, n_layers=6, ratio=5,
+                 local=L31B_LOCAL, global_=L31B_GLOBAL, len_lo=1, len_hi=max(prior) + kq, seed=17)
+    dev = torch.device("cuda")
+    st = AttentionStack(w, dev)
+    g = synth.generator(17)
+    lens_l = [p + kq for p in prior]
+    ws = torch.empty(st.decode_multi_workspace_bytes(kq, max(lens_l)), dtype=torch.uint8, device=dev)
+    lens = torch.tensor(lens_l, dtype=torch.int32, device=dev)
+    T = max(lens_l)
+    for l in range(st.n_layers):
+        t = st.layer_type(l)
+        Hkv, D, W = t.n_kv_heads, t.head_dim, t.window
+        k_log = torch.zeros((w.batch, T, Hkv, D), dtype=torch.bfloat16)
+        v_log = torch.zeros_like(k_log)
+        kc = torch.full(tuple(st.k_cache[l].shape), float("nan"), dtype=torch.bfloat16)
+        vc = kc.clone()
+        for b in range(w.batch):
+            first = max(0, prior[b] - W) if W else 0
+            kr = synth.randn_bf16((Hkv, prior[b] - first, D), g)
+            vr = synth.randn_bf16((Hkv, prior[b] - first, D), g)
+            for i, p in enumerate(range(first, prior[b])):
+                slot = p % W if W else p
+                kc[b, :, slot], vc[b, :, slot] = kr[:, i], vr[:, i]
+            k_log[b, first:prior[b]] = kr.transpose(0, 1)
+            v_log[b, first:prior[b]] = vr.transpose(0, 1)
+        st.k_cache[l].copy_(kc)
+        st.v_cache[l].copy_(vc)
+        q = synth.randn_bf16((w.batch, kq, w.n_q_heads, D), g)
+        k = synth.randn_bf16((w.batch, kq, Hkv, D), g)
+        v = synth.randn_bf16((w.batch, kq, Hkv, D), g)
+        for b in range(w.batch):
+            k_log[b, prior[b]:prior[b] + kq] = k[b]
+            v_log[b, prior[b]:prior[b] + kq] = v[b]
+        out = torch.full((w.batch, kq, w.n_q_heads, D), float("nan"), dtype=torch.bfloat16, device=dev)
+        st.decode_multi_layer(l, q.to(dev), k.to(dev), v.to(dev), out, seq_lens=lens, max_seq_len=T, workspace=ws)
+        assert native.gemma_attn_sync_status() == 0, native.gemma_last_error()
+        ref, _ = oracle.attention(to_bits(q), to_bits(k_log), to_bits(v_log), q_pos0=prior,
+                                  n_keys=lens_l, rot_from=prior, window=W,
+                                  rope_frac=t.rope_frac, theta=t.rope_theta, scale=t.scale)
+        got = out.float().cpu().double().numpy().transpose(0, 2, 1, 3).reshape(-1, D)
+        assert_close(got, ref, what="verify layer %d (%s)" % (l, "global" if W == 0 else "local"))
