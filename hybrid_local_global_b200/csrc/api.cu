@@ -201,11 +201,14 @@ size_t prefill_ws_parts(int B, int S, int Hq, int Hkv, int D, int window, size_t
   return q + std::max(k, 2 * win);
 }
 
-// Multi-token decode on the tensor-core kernel: a global bf16 layer on a
-// contiguous cache whose G q heads x tokens rows fit one 128-row tile.
+// Multi-token decode on the tensor-core kernels (bf16, contiguous cache):
+// a global layer whose G q heads x tokens rows fit one 128-row tile, or an
+// unshared local layer with at most 64 such rows and tokens <= window.
 bool verify_fast(int tokens, int window, int n_q_heads, int n_kv_heads, int head_dim, unsigned flags, bool paged) {
-  return window == 0 && !(flags & GEMMA_F_KV_INT8) && !paged && (head_dim == 256 || head_dim == 512) &&
-         (n_q_heads / n_kv_heads) * tokens <= 128;
+  if ((flags & GEMMA_F_KV_INT8) || paged || (head_dim != 256 && head_dim != 512)) return false;
+  if (window == 0) return (n_q_heads / n_kv_heads) * tokens <= 128;
+  return !(flags & GEMMA_F_SHARED) && tokens <= window && tokens <= 128 &&
+         verify_tc_rows(n_q_heads, n_kv_heads, tokens, head_dim) != 0;
 }
 
 // Keys per split of the multi-token kernel: a multiple of 128 between 1024
@@ -213,7 +216,18 @@ bool verify_fast(int tokens, int window, int n_q_heads, int n_kv_heads, int head
 // fixed cost, the Q tile and the partials, is then a few percent of its
 // streaming time). The 128-row-tile kernel runs head_dim / 256 CTAs per KV
 // head and split, the transposed one a single CTA.
-void verify_plan(int B, int Hq, int Hkv, int tokens, int head_dim, int max_len, int* chunk, int* n_splits) {
+// A local layer splits its ring only when its B x Hkv CTAs fill fewer than
+// two waves.
+void verify_plan(int B, int Hq, int Hkv, int tokens, int head_dim, int window, int max_len, int* chunk,
+                 int* n_splits) {
+  if (window > 0) {
+    const int64_t ctas = (int64_t)B * Hkv, wave2 = (int64_t)sm_count() * 2;
+    int64_t c = ctas >= wave2 ? window : ((int64_t)window * ctas + wave2 - 1) / wave2;
+    c = std::min<int64_t>(((std::max<int64_t>(c, 1) + 127) / 128) * 128, ((window + 127) / 128) * 128);
+    *chunk = (int)c;
+    *n_splits = (int)((window + c - 1) / c);
+    return;
+  }
   const int per_head = verify_tc_rows(Hq, Hkv, tokens, head_dim) ? 1 : head_dim / 256;
   const int64_t ctas_per_split = (int64_t)B * Hkv * per_head;
   const int64_t target = (int64_t)sm_count() * 8;
@@ -224,14 +238,18 @@ void verify_plan(int B, int Hq, int Hkv, int tokens, int head_dim, int max_len, 
   *n_splits = (int)((max_len + c - 1) / c);
 }
 
-// fast path: rotated Q, split log2-sum-exps, split partial O
-size_t verify_ws_parts(int B, int tokens, int Hq, int D, int n_splits, size_t* off_lse, size_t* off_o) {
+// fast path: rotated Q, split log2-sum-exps, split partial O; local layers
+// also the new tokens' rotated keys (the ring is written after attention)
+size_t verify_ws_parts(int B, int tokens, int Hq, int Hkv, int D, int window, int n_splits, size_t* off_lse,
+                       size_t* off_o, size_t* off_kst) {
   const size_t rows = (size_t)B * tokens * Hq;
   const size_t q = align256(rows * D * 2);
   const size_t lse = align256(rows * n_splits * 4);
+  const size_t o = align256(rows * n_splits * D * 4);
   *off_lse = q;
   *off_o = q + lse;
-  return q + lse + align256(rows * n_splits * D * 4);
+  *off_kst = q + lse + o;
+  return q + lse + o + (window > 0 ? align256((size_t)B * tokens * Hkv * D * 2) : 0);
 }
 
 // other layers: lengths before the new tokens, then the chunked-prefill workspace
@@ -783,9 +801,9 @@ size_t gemma_attn_decode_multi_workspace_size(int batch, int tokens, int n_q_hea
     return 0;
   if (verify_fast(tokens, window, n_q_heads, n_kv_heads, head_dim, flags, false)) {
     int chunk, n_splits;
-    verify_plan(batch, n_q_heads, n_kv_heads, tokens, head_dim, max_seq_len, &chunk, &n_splits);
-    size_t a, b;
-    return verify_ws_parts(batch, tokens, n_q_heads, head_dim, n_splits, &a, &b);
+    verify_plan(batch, n_q_heads, n_kv_heads, tokens, head_dim, window, max_seq_len, &chunk, &n_splits);
+    size_t a, b, c;
+    return verify_ws_parts(batch, tokens, n_q_heads, n_kv_heads, head_dim, window, n_splits, &a, &b, &c);
   }
   return verify_route_ws(batch, tokens, n_q_heads, n_kv_heads, head_dim, window, cache_cap, flags);
 }
@@ -822,10 +840,13 @@ int gemma_attn_decode_multi(const void* q, const void* k_new, const void* v_new,
   if (!aligned16(q) || !aligned16(out) || !aligned16(k_cache) || !aligned16(v_cache) ||
       (k_new && !aligned16(k_new)) || (v_new && !aligned16(v_new)) || !aligned16(workspace))
     return fail(GEMMA_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
+  if (window > 0 && cache_cap != window)
+    return fail(GEMMA_ERR_INVALID_ARG, "local layer: cache_cap %d must equal window %d", cache_cap, window);
   int chunk, n_splits;
-  verify_plan(batch, n_q_heads, n_kv_heads, tokens, head_dim, max_seq_len, &chunk, &n_splits);
-  size_t off_lse, off_o;
-  const size_t need = verify_ws_parts(batch, tokens, n_q_heads, head_dim, n_splits, &off_lse, &off_o);
+  verify_plan(batch, n_q_heads, n_kv_heads, tokens, head_dim, window, max_seq_len, &chunk, &n_splits);
+  size_t off_lse, off_o, off_kst;
+  const size_t need =
+      verify_ws_parts(batch, tokens, n_q_heads, n_kv_heads, head_dim, window, n_splits, &off_lse, &off_o, &off_kst);
   if (!workspace || workspace_bytes < need)
     return fail(GEMMA_ERR_CAPACITY, "workspace %zu bytes < %zu", workspace_bytes, need);
   int* status = status_ptr();
@@ -844,12 +865,15 @@ int gemma_attn_decode_multi(const void* q, const void* k_new, const void* v_new,
   ra.cache_cap = cache_cap;
   ra.seq_lens = seq_lens;
   ra.max_len = max_seq_len;
-  ra.window = 0;
+  ra.window = window;
   ra.Hq = n_q_heads;
   ra.Hkv = n_kv_heads;
   ra.n_rot = rope_rotated_pairs(head_dim, rope_frac);
   ra.log2_theta = std::log2((double)rope_theta);
-  ra.k_stage = nullptr;
+  // a local layer's new rows would overwrite ring slots that the earlier new
+  // tokens still see: its rotated keys wait in the workspace, and the ring
+  // is written once the attention is done
+  ra.k_stage = window > 0 ? reinterpret_cast<bf16*>(ws + off_kst) : nullptr;
   ra.page_table = nullptr;
   ra.page_size = cache_cap;
   ra.pages_per_seq = 1;
@@ -866,6 +890,9 @@ int gemma_attn_decode_multi(const void* q, const void* k_new, const void* v_new,
   va.k = KVView{static_cast<const bf16*>(k_cache), (int64_t)n_kv_heads * cache_cap * D, D, (int64_t)cache_cap * D};
   va.v = KVView{static_cast<const bf16*>(v_cache), va.k.stride_b, va.k.stride_row, va.k.stride_h};
   va.cache_cap = cache_cap;
+  va.window = window;
+  va.k_tail = ra.k_stage;
+  va.v_tail = ra.v_new;
   va.seq_lens = seq_lens;
   va.tokens = tokens;
   va.Hq = n_q_heads;
@@ -882,12 +909,22 @@ int gemma_attn_decode_multi(const void* q, const void* k_new, const void* v_new,
     p_split.done();
   }
   if (e != cudaSuccess) return cuda_fail(e, "multi-token attention launch");
+  if (window > 0) {
+    DecodeRopeArgs rb = ra;
+    rb.skip_q = 1;
+    rb.k_stage = nullptr;
+    ProfScope p_app2(GEMMA_KERNEL_DECODE_APPEND, st);
+    e = launch_decode_rope_append(rb, batch, head_dim, st);
+    p_app2.done();
+    if (e != cudaSuccess) return cuda_fail(e, "decode append launch");
+  }
 
   DecodeAttnArgs da{};
   da.tokens = tokens;
+  da.every_split = window > 0 ? 1 : 0;
   da.seq_lens = seq_lens;
   da.max_len = max_seq_len;
-  da.window = 0;
+  da.window = window;
   da.Hq = n_q_heads;
   da.Hkv = n_kv_heads;
   da.chunk = chunk;

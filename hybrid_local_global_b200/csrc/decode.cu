@@ -376,7 +376,7 @@ __global__ void __launch_bounds__(128) k_decode_combine(DecodeAttnArgs a) {
     return;
   }
   const int64_t n_valid = a.window > 0 ? (len < a.window ? len : (int64_t)a.window) : len;
-  const int n_used = (int)((n_valid + a.chunk - 1) / a.chunk);
+  const int n_used = a.every_split ? a.n_splits : (int)((n_valid + a.chunk - 1) / a.chunk);
   const int64_t pr0 = ((int64_t)bt * a.Hq + h) * a.n_splits;
   float m = -INFINITY;
   for (int s = tid; s < n_used; s += 128) m = fmaxf(m, a.part_lse[pr0 + s]);

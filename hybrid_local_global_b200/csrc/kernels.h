@@ -46,6 +46,7 @@ struct DecodeRopeArgs {
   bf16* q_rot;         // workspace [B][tokens][Hq][D]
   int tokens;          // new tokens per sequence, at positions len - tokens .. len - 1 (decode: 1)
   float q_scale;       // rotated q is multiplied by this before the bf16 rounding (decode: 1)
+  int skip_q;          // 1: the new K/V only (q and q_rot are not touched)
   bf16* k_cache;
   bf16* v_cache;
   bf16* k_stage;       // int8 cache: the rotated new key goes here ([B][Hkv][D]) and nothing
@@ -127,6 +128,7 @@ struct DecodeAttnArgs {
   int* status;
   unsigned long long wait_ns;
   int drop_first_copy;     // test hook: skip the first K/V copy of split 0
+  int every_split;         // 1: every planned split wrote a partial (multi-token local layers)
   int keqv;                // K = V: only K rows are loaded and serve as V
   // int8 cache (k_cache/v_cache unused): codes [B][Hkv][cap][D] and per-row (min, step),
   // or the same over the pages of a pool
@@ -175,6 +177,13 @@ struct VerifyAttnArgs {
   const bf16* q_rot;        // [B][tokens][Hq][D], times scale * log2(e)
   KVView k, v;              // head-major cache views [B][Hkv][cap][D]
   int cache_cap;
+  // window > 0 (local layer, transposed kernel only): the cache is the ring
+  // of `window` slots as it was before the new tokens (slot = position %
+  // window); the new tokens' rotated keys and values are read from k_tail /
+  // v_tail [B][tokens][Hkv][D], and every split writes a partial.
+  int window;
+  const bf16* k_tail;
+  const bf16* v_tail;
   const int32_t* seq_lens;  // device [B], including the new tokens
   int tokens, Hq, Hkv;
   int chunk, n_splits;      // keys per split (a multiple of 128), splits planned

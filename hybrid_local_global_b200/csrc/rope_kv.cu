@@ -349,7 +349,7 @@ __global__ void __launch_bounds__(256) k_decode_rope_append(DecodeRopeArgs a) {
   // q heads, then K heads, then V heads (none when shared, none for V under
   // K = V, none with an int8 cache: the quantize kernel reads the caller's V)
   const int n_heads = a.Hq + (a.k_new ? a.Hkv : 0) + ((a.v_new && !a.k_stage) ? a.Hkv : 0);
-  for (int h = threadIdx.y; h < n_heads; h += blockDim.y) {
+  for (int h = threadIdx.y + (a.skip_q ? a.Hq : 0); h < n_heads; h += blockDim.y) {
     if (h < a.Hq) {
       const int64_t off = ((int64_t)bt * a.Hq + h) * D + e0;
       const uint4 x = ld16(a.q + off);

@@ -95,6 +95,7 @@ struct VCfg {
 
 struct VArgs {
   int Hq, Hkv, tokens, chunk, n_splits;
+  int window;  // LOCAL: ring slots
   int64_t key_cap;
   const int32_t* seq_lens;
   float* part_o;
@@ -145,10 +146,16 @@ __device__ __forceinline__ float reduce_columns(float (&x)[32], int lane) {
   return x[0];
 }
 
-template <int D, int NQ>
+// LOCAL: a local layer. The K/V maps are the ring as it was before the new
+// tokens (slot s holds the latest position p < pos0 with p % window == s,
+// if p >= 0); split z takes the slots [z * chunk, +chunk), and the last
+// split also a tail tile of the new tokens' keys and values (tm_kt / tm_vt,
+// [B][tokens][Hkv][D]). Every split writes a partial.
+template <int D, int NQ, bool LOCAL>
 __global__ void __launch_bounds__(192, 1)
     k_verify_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                const __grid_constant__ CUtensorMap tm_v, const VArgs a) {
+                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_kt,
+                const __grid_constant__ CUtensorMap tm_vt, const VArgs a) {
   using C = VCfg<D, NQ>;
   constexpr int NSTAGE = C::NSTAGE;
   constexpr int MT = C::MT;
@@ -170,14 +177,19 @@ __global__ void __launch_bounds__(192, 1)
   const int nvalid = G * a.tokens;  // query rows: row t * G + i = (token t, q head g * G + i)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  // token t sits at position pos0 + t; this CTA reads keys [k_begin, k_end)
+  // token t sits at position pos0 + t; this CTA reads keys (global) or ring
+  // slots (LOCAL) [k_begin, k_end), tile j starting at k_begin + j * BN
   const int64_t n_keys = a.seq_lens[b];
   const int64_t pos0 = n_keys - a.tokens;
   const int64_t k_begin = (int64_t)split * a.chunk;
-  if (pos0 < 0 || n_keys > a.key_cap || k_begin >= n_keys) return;  // lengths are checked by the append kernel
-  const int64_t k_end = k_begin + a.chunk < n_keys ? k_begin + a.chunk : n_keys;
-  const int64_t kt0 = k_begin / BN;
-  const int n_tiles = (int)((k_end - 1) / BN - kt0 + 1);
+  const int64_t k_stop = LOCAL ? (int64_t)a.window : n_keys;
+  if (pos0 < 0 || (!LOCAL && n_keys > a.key_cap) || k_begin >= k_stop) return;  // checked by the append kernel
+  const int64_t k_end = k_begin + a.chunk < k_stop ? k_begin + a.chunk : k_stop;
+  const int n_ring = (int)((k_end - k_begin + BN - 1) / BN);
+  const int n_tiles = n_ring + ((LOCAL && split == a.n_splits - 1) ? 1 : 0);  // LOCAL: + the tail tile
+  // keys of a tile that hold data (V rows past them are zeroed): global,
+  // up to the sequence end; ring, the slots already written
+  const int64_t data_end = LOCAL ? (pos0 < a.window ? pos0 : (int64_t)a.window) : n_keys;
 
   if (threadIdx.x == 0) {
     mbar_init(&ctl->q_full, 1);
@@ -225,6 +237,10 @@ __global__ void __launch_bounds__(192, 1)
       tc::prefetch_tmap(&tm_q);
       tc::prefetch_tmap(&tm_k);
       tc::prefetch_tmap(&tm_v);
+      if (LOCAL) {
+        tc::prefetch_tmap(&tm_kt);
+        tc::prefetch_tmap(&tm_vt);
+      }
       mbar_arrive_expect_tx(&ctl->q_full, (uint32_t)(D * 2 * nvalid));
       for (int c = 0; c < D / 64; ++c)
         tc::tma_load_4d(sQ + c * C::Q_CH, &tm_q, c * 64, g * G, 0, b, smem_u32(&ctl->q_full));
@@ -234,8 +250,10 @@ __global__ void __launch_bounds__(192, 1)
       for (int j = 0; j <= n_tiles && ok; ++j) {
         for (int kind = 0; kind < 2 && ok; ++kind) {  // 0: K_j, 1: V_{j-1}
           if ((kind == 0 && j == n_tiles) || (kind == 1 && j == 0)) continue;
-          const int key0 = (int)((kt0 + j - kind) * BN);
-          const CUtensorMap* map = kind == 0 ? &tm_k : &tm_v;
+          const int jt = j - kind;
+          const bool tail = LOCAL && jt == n_ring;
+          const int key0 = (int)(k_begin + (int64_t)jt * BN);
+          const CUtensorMap* map = tail ? (kind == 0 ? &tm_kt : &tm_vt) : (kind == 0 ? &tm_k : &tm_v);
           for (int h = 0; h < MT; ++h, ++item) {
             const int s = item % NSTAGE;
             if (item >= NSTAGE &&
@@ -248,7 +266,12 @@ __global__ void __launch_bounds__(192, 1)
             const uint32_t bar = smem_u32(&ctl->full[s]);
             mbar_arrive_expect_tx(&ctl->full[s], STAGE_B);
             ctl->issued[s] += 1;
-            for (int cc = 0; cc < 2; ++cc) tc::tma_load_4d(dst + cc * CH_B, map, h * 128 + cc * 64, key0, g, b, bar);
+            for (int cc = 0; cc < 2; ++cc) {
+              if (tail)  // (d, head, token, b): tokens past the last are zeros
+                tc::tma_load_4d(dst + cc * CH_B, map, h * 128 + cc * 64, g, 0, b, bar);
+              else
+                tc::tma_load_4d(dst + cc * CH_B, map, h * 128 + cc * 64, key0, g, b, bar);
+            }
           }
         }
       }
@@ -292,7 +315,8 @@ __global__ void __launch_bounds__(192, 1)
           ok = false;
           break;
         }
-        const int64_t rows_valid = n_keys - (kt0 + j - 1) * BN;
+        const int64_t rows_valid =
+            (LOCAL && j - 1 == n_ring) ? BN : data_end - (k_begin + (int64_t)(j - 1) * BN);
         const uint32_t pb = sP + (uint32_t)((j - 1) & 1) * C::P_BUF;
         for (int m = 0; m < MT; ++m, ++item) {
           const int s = item % NSTAGE;
@@ -367,13 +391,28 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
         for (int n = 0; n < NQ; ++n) v[n] = __uint_as_float(r[n / 32][n % 32]);
       }
-      // row t * G + i sees keys up to pos0 + t; rows past nvalid see none
-      const int64_t dk = (kt0 + j) * BN + kl - pos0;
-      const int n_first = dk <= 0 ? 0 : dk >= a.tokens ? NQ : (int)dk * G;
-      if (n_first > 0 || nvalid < NQ) {
+      // visible rows [n_lo, n_hi) for this thread's key. Global, and the
+      // tail tile: row t * G + i sees keys up to pos0 + t. Ring: token t sees
+      // the positions after pos0 + t - window, so slot s, at distance
+      // d = (pos0 - 1 - s) mod window below pos0, is seen by tokens
+      // t <= window - 2 - d (none if the slot is unwritten or past the ring).
+      // Rows past nvalid see nothing.
+      int n_lo = 0, n_hi = nvalid;
+      if (LOCAL && j < n_ring) {
+        const int64_t slot = k_begin + (int64_t)j * BN + kl;
+        const int64_t d = (pos0 - 1 - slot) % a.window;
+        const int64_t dd = d < 0 ? d + a.window : d;
+        const bool written = slot < a.window && dd <= pos0 - 1;
+        const int64_t t_max1 = a.window - 1 - dd;  // tokens 0 .. t_max1 - 1 see the slot
+        n_hi = !written ? 0 : t_max1 >= a.tokens ? nvalid : (int)t_max1 * G;
+      } else {
+        const int64_t dk = LOCAL ? (int64_t)kl : k_begin + (int64_t)j * BN + kl - pos0;
+        n_lo = dk <= 0 ? 0 : dk >= a.tokens ? NQ : (int)dk * G;
+      }
+      if (n_lo > 0 || n_hi < NQ) {
 #pragma unroll
         for (int n = 0; n < NQ; ++n)
-          if (n < n_first || n >= nvalid) v[n] = -INFINITY;
+          if (n < n_lo || n >= n_hi) v[n] = -INFINITY;
       }
       bool need = false;
 #pragma unroll
@@ -519,14 +558,19 @@ __global__ void __launch_bounds__(192, 1)
   }
 }
 
-template <int D, int NQ>
-cudaError_t launch_as(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const VArgs& v, int B,
-                      cudaStream_t st) {
+template <int D, int NQ, bool LOCAL>
+cudaError_t launch_as(const CUtensorMap (&m)[5], const VArgs& v, int B, cudaStream_t st) {
   using C = VCfg<D, NQ>;
-  cudaError_t e = cudaFuncSetAttribute(k_verify_tc<D, NQ>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  cudaError_t e =
+      cudaFuncSetAttribute(k_verify_tc<D, NQ, LOCAL>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
-  k_verify_tc<D, NQ><<<dim3(v.Hkv, B, v.n_splits), 192, C::SMEM, st>>>(mq, mk, mv, v);
+  k_verify_tc<D, NQ, LOCAL><<<dim3(v.Hkv, B, v.n_splits), 192, C::SMEM, st>>>(m[0], m[1], m[2], m[3], m[4], v);
   return cudaGetLastError();
+}
+
+template <int D, int NQ>
+cudaError_t launch_nq(const CUtensorMap (&m)[5], const VArgs& v, int B, cudaStream_t st) {
+  return v.window > 0 ? launch_as<D, NQ, true>(m, v, B, st) : launch_as<D, NQ, false>(m, v, B, st);
 }
 
 }  // namespace
@@ -540,10 +584,13 @@ int verify_tc_rows(int Hq, int Hkv, int tokens, int D) {
 cudaError_t launch_verify_attn_tc(const VerifyAttnArgs& a, int B, int D, cudaStream_t st) {
   const int G = a.Hq / a.Hkv;
   const int NQ = verify_tc_rows(a.Hq, a.Hkv, a.tokens, D);
-  if (NQ == 0) return launch_verify_attn_rows(a, B, D, st);  // more than 64 query rows a KV head
-  if (a.tokens < 1 || a.chunk % BN || a.n_splits < 1 || G * a.tokens > NQ) return cudaErrorInvalidValue;
+  if (NQ == 0 && a.window == 0) return launch_verify_attn_rows(a, B, D, st);  // more than 64 query rows
+  if (NQ == 0 || a.tokens < 1 || a.chunk % BN || a.n_splits < 1 || G * a.tokens > NQ) return cudaErrorInvalidValue;
+  if (a.window > 0 && (a.tokens > BN || !a.k_tail || !a.v_tail || a.cache_cap != a.window))
+    return cudaErrorInvalidValue;
   const uint64_t E = 2;
-  CUtensorMap mq, mk, mv;
+  CUtensorMap maps[5];
+  CUtensorMap &mq = maps[0], &mk = maps[1], &mv = maps[2];
   {
     // q_rot [B][tokens][Hq][D]: a box is the G heads of one KV head for every token
     const uint64_t dims[4] = {(uint64_t)D, (uint64_t)a.Hq, (uint64_t)a.tokens, (uint64_t)B};
@@ -560,7 +607,19 @@ cudaError_t launch_verify_attn_tc(const VerifyAttnArgs& a, int B, int D, cudaStr
     if (!make_map_bf16_4d(&mk, a.k.ptr, dims, strk, box) || !make_map_bf16_4d(&mv, a.v.ptr, dims, strv, box))
       return cudaErrorInvalidValue;
   }
+  if (a.window > 0) {
+    // the new tokens' rows (d, head, token, b); boxes of 64 dims x 128 tokens
+    const uint64_t dims[4] = {(uint64_t)D, (uint64_t)a.Hkv, (uint64_t)a.tokens, (uint64_t)B};
+    const uint64_t str[3] = {(uint64_t)D * E, (uint64_t)a.Hkv * D * E, (uint64_t)a.tokens * a.Hkv * D * E};
+    const uint32_t box[4] = {64, 1, (uint32_t)BN, 1};
+    if (!make_map_bf16_4d(&maps[3], a.k_tail, dims, str, box) || !make_map_bf16_4d(&maps[4], a.v_tail, dims, str, box))
+      return cudaErrorInvalidValue;
+  } else {
+    maps[3] = mk;
+    maps[4] = mv;
+  }
   VArgs v{};
+  v.window = a.window;
   v.Hq = a.Hq;
   v.Hkv = a.Hkv;
   v.tokens = a.tokens;
@@ -572,8 +631,8 @@ cudaError_t launch_verify_attn_tc(const VerifyAttnArgs& a, int B, int D, cudaStr
   v.part_lse = a.part_lse;
   v.status = a.status;
   v.wait_ns = a.wait_ns;
-  if (D == 256) return NQ == 32 ? launch_as<256, 32>(mq, mk, mv, v, B, st) : launch_as<256, 64>(mq, mk, mv, v, B, st);
-  return NQ == 32 ? launch_as<512, 32>(mq, mk, mv, v, B, st) : launch_as<512, 64>(mq, mk, mv, v, B, st);
+  if (D == 256) return NQ == 32 ? launch_nq<256, 32>(maps, v, B, st) : launch_nq<256, 64>(maps, v, B, st);
+  return NQ == 32 ? launch_nq<512, 32>(maps, v, B, st) : launch_nq<512, 64>(maps, v, B, st);
 }
 
 }  // namespace hlg

@@ -214,7 +214,7 @@ def _multi_raw(**over):
     (dict(out=None, wsb=1 << 30), E.GEMMA_ERR_INVALID_ARG),
     (dict(T=17), E.GEMMA_ERR_CAPACITY),                               # 8 x 17 rows: the prefill route
     (dict(T=17, out=None, wsb=1 << 30), E.GEMMA_ERR_INVALID_ARG),     # ... which validates as prefill
-    (dict(W=1024, cap=1024, Hkv=16, D=256, frac=1.0, theta=1e4), E.GEMMA_ERR_CAPACITY),  # local: route
+    (dict(W=1024, cap=1024, Hkv=16, D=256, frac=1.0, theta=1e4), E.GEMMA_ERR_CAPACITY),  # local: accepted
     (dict(W=1024, cap=4096, Hkv=16, D=256, frac=1.0, theta=1e4, wsb=1 << 30), E.GEMMA_ERR_INVALID_ARG),
     (dict(W=1024, cap=1024, Hkv=16, D=256, frac=1.0, theta=1e4, flags=1, k=None, v=None, wsb=1 << 30),
      E.GEMMA_ERR_UNSUPPORTED),                                        # shared local after cached tokens
@@ -227,12 +227,16 @@ def test_decode_multi_validation(over, code):
 
 def test_decode_multi_workspace_sizes():
     """The tensor-core path holds the rotated queries and fp32 split
-    partials; the routed layers a length buffer plus the chunked-prefill
-    workspace."""
+    partials (local layers also the new tokens' rotated keys); the routed
+    layers a length buffer plus the chunked-prefill workspace."""
     n = native.gemma_attn_decode_multi_workspace_size(64, 4, 32, 4, 512, 0, 131072, 131072, 0)
     assert n >= 64 * 4 * 32 * 512 * (2 + 4)
     loc = native.gemma_attn_decode_multi_workspace_size(64, 4, 32, 16, 256, 1024, 131072, 1024, 0)
-    assert loc >= 256 + native.gemma_attn_prefill_workspace_size_cached(64, 4, 32, 16, 256, 1024, 1024, 0)
+    assert loc >= 64 * 4 * 32 * 256 * (2 + 4) + 64 * 4 * 16 * 256 * 2
+    routed = native.gemma_attn_decode_multi_workspace_size(1, 40, 32, 16, 256, 1024, 4096, 1024, 0)  # 80 rows
+    assert routed >= 256 + native.gemma_attn_prefill_workspace_size_cached(1, 40, 32, 16, 256, 1024, 1024, 0)
+    shared = native.gemma_attn_decode_multi_workspace_size(1, 4, 32, 16, 256, 1024, 4096, 1024, native.GEMMA_F_SHARED)
+    assert shared >= 256 + native.gemma_attn_prefill_workspace_size_cached(1, 4, 32, 16, 256, 1024, 1024, 0)
     q8 = native.gemma_attn_decode_multi_workspace_size(2, 4, 32, 4, 512, 0, 4096, 4096, native.GEMMA_F_KV_INT8)
     assert q8 >= native.gemma_attn_prefill_workspace_size_cached(2, 4, 32, 4, 512, 0, 4096, native.GEMMA_F_KV_INT8)
     assert native.gemma_attn_decode_multi_workspace_size(0, 4, 32, 4, 512, 0, 4096, 4096, 0) == 0

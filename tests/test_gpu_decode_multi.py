@@ -130,11 +130,25 @@ def test_multi_global_exact_capacity(oracle):
 
 
 @pytest.mark.parametrize("case", [
-    dict(lens=[3000, 700, 4], T=4, Hq=32, Hkv=16, D=256, W=1024, seed=321),    # 31B local shape
+    dict(lens=[3000, 700, 4], T=4, Hq=32, Hkv=16, D=256, W=1024, seed=321),    # 31B local shape, 4 ring splits
+    dict(lens=[3000], T=4, Hq=32, Hkv=16, D=256, W=1024, seed=325),            # one sequence: 8 ring splits
+    dict(lens=[1028, 1027, 1029, 5], T=4, Hq=32, Hkv=16, D=256, W=1024, seed=326),  # ring just full / not
     dict(lens=[600, 65], T=3, Hq=8, Hkv=4, D=256, W=64, seed=322),             # ring wraps inside the call
+    dict(lens=[900, 8], T=8, Hq=32, Hkv=4, D=256, W=512, seed=327),            # 64 query rows
+    dict(lens=[300, 17], T=16, Hq=8, Hkv=4, D=512, W=16, seed=328, frac=0.25, theta=1e6),  # T = window
+])
+def test_multi_local_tensor_core(oracle, case):
+    """Local layers: the ring as it was, plus a tail tile of the new tokens;
+    the ring is written after the attention."""
+    case = dict(case)
+    run_multi_case(oracle, frac=case.pop("frac", 1.0), theta=case.pop("theta", 1e4), **case)
+
+
+@pytest.mark.parametrize("case", [
     dict(lens=[40], T=40, Hq=4, Hkv=2, D=256, W=16, seed=323),                 # more tokens than the window
+    dict(lens=[700, 90], T=40, Hq=4, Hkv=2, D=256, W=64, seed=329),            # 80 query rows
     dict(lens=[3000, 700], T=17, Hq=32, Hkv=4, D=512, W=0, seed=324, frac=0.25, theta=1e6),  # 136 rows: route
-], ids=["31b_local", "wrap", "T_gt_W", "global_route"])
+], ids=["T_gt_W", "local_rows80", "global_route"])
 def test_multi_routed_layers(oracle, case):
     case = dict(case)
     run_multi_case(oracle, frac=case.pop("frac", 1.0), theta=case.pop("theta", 1e4), **case)
