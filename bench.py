@@ -528,16 +528,15 @@ def decode_cpu_baseline(w, st, layers, lens_cpu, n_random=2):
                          "shortest, longest and %d seeded others" % (len(seqs) - 2))}
 
 
-def bench_decode(args, w, dev, world, peaks, cpu=False):
-    from hybrid_local_global_b200 import native
+def make_decode_stack(w, dev):
+    """A decode workload's stack with every owned cache filled from the
+    workload's seed, and its per-sequence lengths (CPU and device)."""
     from hybrid_local_global_b200.stack import AttentionStack
     st = AttentionStack(w, dev)
     if w.len_lo == w.len_hi:
         lens_cpu = torch.full((w.batch,), w.len_hi, dtype=torch.int32)
     else:
         lens_cpu = synth.decode_lengths(w.batch, w.len_lo, w.len_hi, seed=w.seed)
-    lens = lens_cpu.to(dev)
-    max_len = int(lens_cpu.max())
     g = synth.generator(w.seed, dev)
     seen = set()
     for l in range(st.n_layers):
@@ -548,6 +547,12 @@ def bench_decode(args, w, dev, world, peaks, cpu=False):
         synth.fill_cache_(kc, g)
         if st.v_cache[l] is not kc:
             synth.fill_cache_(st.v_cache[l], g)
+    return st, lens_cpu, lens_cpu.to(dev), int(lens_cpu.max()), g
+
+
+def bench_decode(args, w, dev, world, peaks, cpu=False):
+    from hybrid_local_global_b200 import native
+    st, lens_cpu, lens, max_len, g = make_decode_stack(w, dev)
     layers = []
     for l in range(st.n_layers):
         t = st.layer_type(l)
@@ -611,6 +616,152 @@ def bench_decode(args, w, dev, world, peaks, cpu=False):
     if cpu:
         res["cpu_baseline"] = decode_cpu_baseline(w, st, layers, lens_cpu)
     del layers, st, ws
+    torch.cuda.empty_cache()
+    return res
+
+
+# --------------------------------------------------------------------------- multi-token decode (ours)
+def verify_kv_bytes(st, l, lens_cpu, T, seqs=None):
+    """K (and V unless K = V) bytes one multi-token decode of layer l reads:
+    a global layer every position of the sequence, a local layer the ring's
+    written slots before the T new tokens plus the T new rows."""
+    t = st.layer_type(l)
+    L = lens_cpu.to(torch.int64)
+    if seqs is not None:
+        L = L[list(seqs)]
+    keys = (torch.clamp(L - T, max=t.window) + T) if t.window else L
+    return int(keys.sum()) * t.n_kv_heads * t.head_dim * 2 * (1 if st.keqv(l) else 2)
+
+
+def verify_cpu_baseline(w, st, layers, lens_cpu, n_random=1):
+    """The oracle on a seeded sample of sequences (the shortest, the longest
+    and n_random others) of every layer, after the GPU steps: each of the T
+    new tokens' q rows rotated by the oracle at its position, attending over
+    its visible positions among the rows cached after the step (on a local
+    layer the ring then holds the last `window` positions, so an early token
+    sees up to T - 1 fewer keys than on the GPU). Rate = the sample's K+V
+    bytes as counted for the GPU per second of oracle time."""
+    import oracle
+    T = w.tokens
+    lens = [int(x) for x in lens_cpu]
+    rng = np.random.default_rng(99)
+    pick = {int(np.argmin(lens)), int(np.argmax(lens))}
+    others = [b for b in range(len(lens)) if b not in pick]
+    pick |= set(int(x) for x in rng.choice(others, size=min(n_random, len(others)), replace=False)) if others else set()
+    seqs = sorted(pick)
+    threads = oracle.default_threads()
+    secs, nbytes = 0.0, 0
+    with cf.ThreadPoolExecutor(max_workers=threads) as ex:
+        for l in range(st.n_layers):
+            t = st.layer_type(l)
+            q = layers[l][0]
+            kc, vc = st.k_cache[l], st.v_cache[l]
+            keqv = st.keqv(l)
+            G = w.n_q_heads // t.n_kv_heads
+            for b in seqs:
+                L = lens[b]
+                first = max(0, L - t.window) if t.window else 0
+                slots = [(p % t.window) if t.window else p for p in range(first, L)]
+                idx = torch.as_tensor(slots, dtype=torch.long, device=q.device)
+                kf = kc[b].index_select(1, idx).double().cpu().numpy()
+                vf = kf if keqv else vc[b].index_select(1, idx).double().cpu().numpy()
+                qbits = synth.bits(q[b])  # [T, Hq, D]
+                t0 = time.perf_counter()
+                qr = np.stack([np.stack([oracle.rope_bf16(qbits[tok, h], L - T + tok, t.rope_frac, t.rope_theta)
+                                         for h in range(w.n_q_heads)]) for tok in range(T)])  # [T, Hq, D]
+                lo = np.array([max(0, L - T + tok - t.window + 1 - first) if t.window else 0 for tok in range(T)])
+                hi = np.array([L - T + tok + 1 - first for tok in range(T)])
+                futs = [ex.submit(oracle.attend_rows, qr[tok, hk * G:(hk + 1) * G], kf[hk], vf[hk], lo[tok],
+                                  hi[tok] - lo[tok], t.scale)
+                        for hk in range(t.n_kv_heads) for tok in range(T)]
+                for f in futs:
+                    f.result()
+                secs += time.perf_counter() - t0
+                del kf, vf
+            nbytes += verify_kv_bytes(st, l, lens_cpu, T, seqs=seqs)
+    return {"value": round(nbytes / secs / 1e9, 3), "unit": "GB/s", "cores": threads, "kind": "oracle",
+            "seconds": round(secs, 2),
+            "sample": "sequences %s (shortest, longest and %d seeded other) of every layer, all q heads and "
+                      "all %d new tokens; bytes = their K+V bytes as counted for the GPU"
+                      % (seqs, len(seqs) - 2, T)}
+
+
+def bench_verify(args, w, dev, world, peaks, cpu=False):
+    """Multi-token decode (w.tokens new tokens per sequence) through every
+    layer of the stack, and a single-token decode step of the same stack
+    for the ratio."""
+    from hybrid_local_global_b200 import native
+    st, lens_cpu, lens, max_len, g = make_decode_stack(w, dev)
+    T = w.tokens
+    layers, dlayers = [], []
+    for l in range(st.n_layers):
+        t = st.layer_type(l)
+        q = synth.randn_bf16((w.batch, T, w.n_q_heads, t.head_dim), g, dev)
+        k = synth.randn_bf16((w.batch, T, t.n_kv_heads, t.head_dim), g, dev)
+        v = synth.randn_bf16((w.batch, T, t.n_kv_heads, t.head_dim), g, dev)
+        layers.append((q, k, v, torch.empty_like(q)))
+        dlayers.append(tuple(x[:, 0].contiguous() for x in (q, k, v)) + (torch.empty_like(q[:, 0]),))
+    ws = torch.empty(max(st.decode_multi_workspace_bytes(T, max_len), st.decode_workspace_bytes(max_len)),
+                     dtype=torch.uint8, device=dev)
+
+    def step():
+        for l, (q, k, v, out) in enumerate(layers):
+            st.decode_multi_layer(l, q, k, v, out, seq_lens=lens, max_seq_len=max_len, workspace=ws)
+
+    def dstep():
+        for l, (q, k, v, out) in enumerate(dlayers):
+            st.decode_layer(l, q, k, v, out, seq_lens=lens, max_seq_len=max_len, workspace=ws)
+
+    for fn in (dstep, step):
+        for _ in range(args.warmup):
+            fn()
+    torch.cuda.synchronize()
+    assert native.gemma_attn_sync_status() == 0, native.gemma_last_error()
+    d_ms, _, dkern, _ = timed_passes(native, dstep, args, world, dev)
+    dev_ms, _, kern, clk = timed_passes(native, step, args, world, dev)
+    kv_bytes = sum(verify_kv_bytes(st, l, lens_cpu, T) for l in range(st.n_layers))
+    io_bytes = sum(w.batch * T * (w.n_q_heads * st.layer_type(l).head_dim * 2 * 2 +
+                                  st.layer_type(l).n_kv_heads * st.layer_type(l).head_dim * 2 * 2)
+                   for l in range(st.n_layers))
+    nbytes = kv_bytes + io_bytes
+    value = world * nbytes * args.steps / (dev_ms / 1e3) / 1e9
+    sp = kern.get("decode_split", {"ms": float("nan"), "launches": 0})
+    achieved = kv_bytes * args.steps / (sp["ms"] / 1e3) / 1e9
+    peak = peaks[0]["hbm_gbs"]
+    roof = {"bound": "hbm", "kernel": "multi-token decode attention (transposed tensor-core kernel)",
+            "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s", "frac": round(achieved / peak, 4),
+            "peak_source": "%s HBM copy (MEASURED_PEAKS.json)" % peaks[1], "traffic": None,
+            "per_launch": "K (and V unless K = V) bytes of all attention launches / their summed device time "
+                          "(%d launches, %d per step; CUDA events around each launch, in a second timed pass "
+                          "of the same steps)" % (sp["launches"], st.n_layers)}
+    rec = recorded_traffic("k_verify_tc")
+    if rec:
+        ratio = {k: float(r["bytes"]) / float(r["units"]) for k, r in rec.items()}
+        any_ratio = next(iter(ratio.values()))
+        per_layer = [ratio.get("global" if st.layer_type(l).window == 0 else "local", any_ratio)
+                     * verify_kv_bytes(st, l, lens_cpu, T) for l in range(st.n_layers)]
+        roof["traffic"] = round(sum(per_layer) / st.n_layers)
+        roof["traffic_note"] = ("DRAM bytes per attention launch: each layer's K+V bytes x the traffic/algorithmic "
+                                "ratio of the ncu capture for its layer type (%s), mean over the block's launches"
+                                % ", ".join("%s %.4f: %s in %s" % (k, ratio[k], rec[k]["workload"], rec[k]["file"])
+                                            for k in sorted(rec)))
+    else:
+        roof["traffic_note"] = "no ncu capture of the current kernel sources"
+    res = {"metric": "multi-token decode KV GB/s", "value": round(value, 1), "unit": "GB/s",
+           "workload": w.name, "description": w.description, "tokens": T,
+           "ms_per_step": round(dev_ms / args.steps, 4),
+           "decode_ms_per_step": round(d_ms / args.steps, 4),
+           "ratio_to_decode_step": round(dev_ms / d_ms, 4),
+           "ratio_note": "one multi-token step (T tokens per sequence) / one single-token decode step of the "
+                         "same stack, lengths and inputs (the first of the T tokens)",
+           "bytes_per_step": nbytes, "kv_bytes_per_step": kv_bytes,
+           "kv_lengths": {"min": int(lens_cpu.min()), "max": max_len, "sum": int(lens_cpu.sum())},
+           "roofline": roof, "kernels": kern, "decode_kernels": dkern, "clocks": clk.summary(),
+           "gpu_launches": sum(v["launches"] for v in kern.values()) +
+                           sum(v["launches"] for v in dkern.values())}
+    if cpu:
+        res["cpu_baseline"] = verify_cpu_baseline(w, st, layers, lens_cpu)
+    del layers, dlayers, st, ws
     torch.cuda.empty_cache()
     return res
 
@@ -689,6 +840,7 @@ def main():
     ap.add_argument("--decode-workload", default="31b_decode_b64")
     ap.add_argument("--decode-int8-workload", default="31b_decode_b64_int8")
     ap.add_argument("--extra-decode", default=EXTRA_DECODE)
+    ap.add_argument("--verify-workload", default="31b_verify_b64_k4")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-flops", type=float, default=4e11,
@@ -733,9 +885,13 @@ def main():
         line["decode_int8"] = bench_decode(args, WORKLOADS[args.decode_int8_workload], dev, world, peaks, cpu=cpu)
     for name in names(args.extra_decode):
         configs[name] = bench_decode(args, WORKLOADS[name], dev, world, peaks, cpu=cpu)
+    if args.verify_workload != "none":
+        vw = WORKLOADS[args.verify_workload]
+        line["verify_k%d" % vw.tokens] = bench_verify(args, vw, dev, world, peaks, cpu=cpu)
     if configs:
         line["configs"] = configs
-    for obj in list(configs.values()) + [line.get("decode"), line.get("decode_int8")]:
+    for obj in list(configs.values()) + [line.get("decode"), line.get("decode_int8")] + \
+            [v for k, v in line.items() if k.startswith("verify_k")]:
         if obj:
             line["gpu_launches"] += obj["gpu_launches"]
     if rank == 0:

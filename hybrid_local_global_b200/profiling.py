@@ -40,6 +40,7 @@ KERNEL_SOURCES = {
     "k_prefill_pair": ("prefill_pair.cu", "pair.cuh", "tc.cuh", "common.cuh", "tmap.cu", "tmap.h"),
     "k_decode_split": ("decode.cu", "mma_sync.cuh", "common.cuh"),
     "k_decode_split_q8": ("decode_q8.cu", "mma_sync.cuh", "tc.cuh", "common.cuh", "tmap.cu", "tmap.h"),
+    "k_verify_tc": ("verify_tc.cu", "tc.cuh", "common.cuh", "tmap.cu", "tmap.h"),
 }
 
 
@@ -201,18 +202,22 @@ def run(workload: str, reps: int, layers: list[int] | None) -> None:
                 synth.fill_cache_(st.k_cache[l], g)
                 if st.v_cache[l] is not st.k_cache[l]:
                     synth.fill_cache_(st.v_cache[l], g)
-        ws = torch.empty(st.decode_workspace_bytes(max_len), dtype=torch.uint8, device=dev)
+        T = w.tokens  # > 1: multi-token decode
+        ws_bytes = st.decode_multi_workspace_bytes(T, max_len) if T > 1 else st.decode_workspace_bytes(max_len)
+        ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+        tok = (T,) if T > 1 else ()
         bufs = {}
         for l in todo:
             t = st.layer_type(l)
-            q = synth.randn_bf16((w.batch, w.n_q_heads, t.head_dim), g, dev)
-            k = synth.randn_bf16((w.batch, t.n_kv_heads, t.head_dim), g, dev)
-            v = synth.randn_bf16((w.batch, t.n_kv_heads, t.head_dim), g, dev)
+            q = synth.randn_bf16((w.batch,) + tok + (w.n_q_heads, t.head_dim), g, dev)
+            k = synth.randn_bf16((w.batch,) + tok + (t.n_kv_heads, t.head_dim), g, dev)
+            v = synth.randn_bf16((w.batch,) + tok + (t.n_kv_heads, t.head_dim), g, dev)
             bufs[l] = (q, k, v, torch.empty_like(q))
+        layer_call = st.decode_multi_layer if T > 1 else st.decode_layer
         for _ in range(reps):
             for l in todo:
                 q, k, v, out = bufs[l]
-                st.decode_layer(l, q, k, v, out, seq_lens=lens, max_seq_len=max_len, workspace=ws)
+                layer_call(l, q, k, v, out, seq_lens=lens, max_seq_len=max_len, workspace=ws)
     torch.cuda.synchronize()
     rc = native.gemma_attn_sync_status()
     if rc != 0:

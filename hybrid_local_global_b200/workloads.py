@@ -47,6 +47,7 @@ class Workload:
     fixed_kinds: tuple = ()      # overrides the schedule: e.g. ("local",) for one local layer
     k_eq_v: bool = False         # global layers use K = V (values are the cached keys)
     kv_int8: bool = False        # int8 KV caches (codes + (min, step) per row)
+    tokens: int = 1              # decode: new tokens per sequence (> 1: multi-token decode)
     description: str = field(default="", compare=False)
 
 
@@ -73,6 +74,16 @@ WORKLOADS = {
         local=L31B_LOCAL, global_=L31B_GLOBAL, len_lo=4096, len_hi=131072, n_shared=2, seed=3,
         description="31B-shaped 6-layer decode: B64, KV length U[4096,131072], ring 1024, "
                     "last 2 layers shared"),
+    "31b_verify_b64_k4": Workload(
+        "31b_verify_b64_k4", "decode", batch=64, n_q_heads=32, n_layers=6, ratio=5,
+        local=L31B_LOCAL, global_=L31B_GLOBAL, len_lo=4096, len_hi=131072, seed=3, tokens=4,
+        description="31B-shaped 6-layer multi-token decode (checking k = 4 drafted tokens): B64, "
+                    "KV length U[4096,131072] including the 4 new tokens, ring 1024, no shared layers"),
+    "31b_verify_b8_k4": Workload(
+        "31b_verify_b8_k4", "decode", batch=8, n_q_heads=32, n_layers=6, ratio=5,
+        local=L31B_LOCAL, global_=L31B_GLOBAL, len_lo=16384, len_hi=32768, seed=5, tokens=4,
+        description="31B-shaped 6-layer multi-token decode, k = 4, B8, KV length U[16384,32768] "
+                    "(a capture-sized case: every layer's K+V above the L2 size)"),
     "31b_decode_b64_int8": Workload(
         "31b_decode_b64_int8", "decode", batch=64, n_q_heads=32, n_layers=6, ratio=5,
         local=L31B_LOCAL, global_=L31B_GLOBAL, len_lo=4096, len_hi=131072, n_shared=2, seed=3,
