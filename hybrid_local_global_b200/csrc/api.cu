@@ -205,7 +205,8 @@ size_t prefill_ws_parts(int B, int S, int Hq, int Hkv, int D, int window, size_t
 // a global layer whose G q heads x tokens rows fit one 128-row tile, or an
 // unshared local layer with at most 64 such rows and tokens <= window.
 bool verify_fast(int tokens, int window, int n_q_heads, int n_kv_heads, int head_dim, unsigned flags, bool paged) {
-  if ((flags & GEMMA_F_KV_INT8) || paged || (head_dim != 256 && head_dim != 512)) return false;
+  if ((flags & (GEMMA_F_KV_INT8 | GEMMA_F_SOURCE_WINDOW)) || paged || (head_dim != 256 && head_dim != 512))
+    return false;
   if (window == 0) return (n_q_heads / n_kv_heads) * tokens <= 128;
   return !(flags & GEMMA_F_SHARED) && tokens <= window && tokens <= 128 &&
          verify_tc_rows(n_q_heads, n_kv_heads, tokens, head_dim) != 0;
@@ -313,7 +314,7 @@ int gemma_layer_schedule(int n_layers, int ratio, int n_shared, int* is_global, 
 // key cache under K = V.
 static int check_kv_flags(unsigned flags, int window, const void* k_new, const void* v_new, void* k_cache,
                           void** v_cache_io) {
-  if (flags & ~(GEMMA_F_SHARED | GEMMA_F_KEQV | GEMMA_F_KV_INT8))
+  if (flags & ~(GEMMA_F_SHARED | GEMMA_F_KEQV | GEMMA_F_KV_INT8 | GEMMA_F_SOURCE_WINDOW))
     return fail(GEMMA_ERR_INVALID_ARG, "unknown flags 0x%x", flags);
   const bool shared = flags & GEMMA_F_SHARED, keqv = flags & GEMMA_F_KEQV;
   if (keqv && window > 0)
@@ -457,9 +458,12 @@ static int prefill_impl(const void* q, const void* k_new, const void* v_new, voi
   const bool shared = flags & GEMMA_F_SHARED;
   const bool q8 = flags & GEMMA_F_KV_INT8;
   const bool keqv = flags & GEMMA_F_KEQV;
+  const bool src_win = flags & GEMMA_F_SOURCE_WINDOW;
   if (q8) {
     if (cache_cap % 2) return fail(GEMMA_ERR_INVALID_ARG, "int8 KV: cache_cap %d must be even", cache_cap);
   }
+  if (src_win && (window == 0 || !seq_lens_before))
+    return fail(GEMMA_ERR_INVALID_ARG, "GEMMA_F_SOURCE_WINDOW: local layers after cached tokens only");
   if (!q || !out || !k_cache || !v_cache) return fail(GEMMA_ERR_INVALID_ARG, "null tensor pointer");
   if (!aligned16(q) || !aligned16(out) || !aligned16(k_cache) || !aligned16(v_cache) ||
       (k_new && !aligned16(k_new)) || (v_new && !aligned16(v_new)) || !aligned16(workspace))
@@ -467,9 +471,10 @@ static int prefill_impl(const void* q, const void* k_new, const void* v_new, voi
   if (window > 0) {
     if (cache_cap != window)
       return fail(GEMMA_ERR_INVALID_ARG, "local layer: cache_cap %d must equal window %d", cache_cap, window);
-    if (shared && seq_lens_before)
+    if (shared && seq_lens_before && !src_win)
       return fail(GEMMA_ERR_UNSUPPORTED,
-                  "shared local layer after cached tokens: the source's chunk has replaced ring slots it needs");
+                  "shared local layer after cached tokens: the source's chunk has replaced ring slots it needs "
+                  "(GEMMA_F_SOURCE_WINDOW reads the window its source's call left in the workspace)");
     if (shared && s_new > window)
       return fail(GEMMA_ERR_UNSUPPORTED, "shared local layer: prefill longer than the window");
   } else if (cache_cap < s_new) {
@@ -481,7 +486,11 @@ static int prefill_impl(const void* q, const void* k_new, const void* v_new, voi
   // (after cached tokens, or a shared layer's): the rows are dequantized
   // into the window; a global layer's window rows are positions.
   const bool chunked_local = window > 0 && seq_lens_before && !shared;
-  const bool win_local = chunked_local || (q8 && window > 0 && shared);
+  // a shared local layer after cached tokens attends to the window its
+  // source's call left in this workspace (int8: the chunk's rows are read
+  // back from the codes over it, as a shared layer reads every row)
+  const bool reuse_local = window > 0 && seq_lens_before && shared && src_win;
+  const bool win_local = chunked_local || reuse_local || (q8 && window > 0 && shared);
   const bool prefix_q8 = q8 && window == 0 && (seq_lens_before || shared);
   const int win_rows = win_local ? window + s_new : prefix_q8 ? cache_cap : 0;
   size_t off_k, off_vw;
@@ -518,7 +527,7 @@ static int prefill_impl(const void* q, const void* k_new, const void* v_new, voi
                                       vc8 ? reinterpret_cast<const float2*>(vc8 + codes_off) : nullptr,
                                       seq_lens_before, shared ? s_new : 0, batch, n_kv_heads, head_dim, window,
                                       cache_cap, L.page_table, L.page_size, L.pages_per_seq, L.n_pages, win_rows,
-                                      ra.k_rot, ra.v_win, status, st);
+                                      reuse_local ? window : 0, ra.k_rot, ra.v_win, status, st);
     if (eg != cudaSuccess) return cuda_fail(eg, "int8 window gather launch");
   } else if (chunked_local) {
     // before the chunk overwrites ring slots: old keys/values into rows 0..window-1
@@ -558,7 +567,8 @@ static int prefill_impl(const void* q, const void* k_new, const void* v_new, voi
   PrefillAttnArgs aa{};
   aa.q_rot = ra.q_rot;
   const int64_t D = head_dim;
-  if ((window == 0 || shared) && !q8) {
+  const bool cache_view = (window == 0 || shared) && !q8 && !reuse_local;
+  if (cache_view) {
     // head-major views of the cache's pages (a contiguous cache: one page of
     // cache_cap rows per sequence)
     const int64_t ps = L.page_size;
@@ -568,8 +578,9 @@ static int prefill_impl(const void* q, const void* k_new, const void* v_new, voi
     aa.v = vc;
     aa.key_cap = cache_cap;
   } else if (win_local || prefix_q8) {
-    KVView kw = {ra.k_rot, (int64_t)win_rows * n_kv_heads * D, (int64_t)n_kv_heads * D, D};
-    KVView vw = {keqv ? ra.k_rot : ra.v_win, kw.stride_b, kw.stride_row, kw.stride_h};
+    const bf16* k_win = reinterpret_cast<const bf16*>(ws + off_k);
+    KVView kw = {k_win, (int64_t)win_rows * n_kv_heads * D, (int64_t)n_kv_heads * D, D};
+    KVView vw = {keqv ? k_win : ra.v_win, kw.stride_b, kw.stride_row, kw.stride_h};
     aa.k = kw;
     aa.v = vw;
     aa.key_cap = win_rows;
@@ -592,7 +603,6 @@ static int prefill_impl(const void* q, const void* k_new, const void* v_new, voi
   aa.lse = lse;
   aa.status = status;
   aa.wait_ns = (unsigned long long)g_wait_ns.load();
-  const bool cache_view = (window == 0 || shared) && !q8;
   aa.page_table = cache_view ? L.page_table : nullptr;
   aa.page_size = L.page_size;
   aa.pages_per_seq = L.pages_per_seq;
@@ -668,6 +678,9 @@ static int decode_impl(const void* q, const void* k_new, const void* v_new, void
   if (rc) return rc;
   rc = check_kv_flags(flags, window, k_new, v_new, k_cache, &v_cache);
   if (rc) return rc;
+  if (flags & GEMMA_F_SOURCE_WINDOW)
+    return fail(GEMMA_ERR_INVALID_ARG, "GEMMA_F_SOURCE_WINDOW: a prefill / multi-token flag (one new token "
+                                       "never needs a slot its source replaced)");
   if (batch <= 0 || max_seq_len <= 0)
     return fail(GEMMA_ERR_INVALID_ARG, "batch %d, max_seq_len %d", batch, max_seq_len);
   if (!q || !out || !k_cache || !v_cache || !seq_lens)

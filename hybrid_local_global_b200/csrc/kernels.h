@@ -154,13 +154,13 @@ cudaError_t launch_ring_gather(const bf16* k_cache, const bf16* v_cache, const i
 // null), plus `extra` positions (a shared layer's chunk). window > 0: the
 // ring's positions pos0-window .. pos0+extra-1 into rows 0.. (negative
 // positions: zeros); window 0: positions 0 .. pos0+extra-1 into rows 0.. .
-// v_codes null: K only.
+// Rows below first_row are not written. v_codes null: K only.
 // Cached rows are addressed by cache_row (page_table null: contiguous,
 // page_size = cache_cap, n_pages = B).
 cudaError_t launch_gather_q8(const uint8_t* k_codes, const float2* k_params, const uint8_t* v_codes,
                              const float2* v_params, const int32_t* seq_lens_before, int extra, int B, int Hkv,
                              int D, int window, int cache_cap, const int32_t* page_table, int page_size,
-                             int pages_per_seq, int n_pages, int win_rows, bf16* k_win, bf16* v_win,
+                             int pages_per_seq, int n_pages, int win_rows, int first_row, bf16* k_win, bf16* v_win,
                              int* status, cudaStream_t st);
 cudaError_t launch_decode_rope_append(const DecodeRopeArgs& a, int B, int D, cudaStream_t st);
 cudaError_t launch_lens_minus(const int32_t* seq_lens, int32_t* lens_before, int B, int tokens, cudaStream_t st);

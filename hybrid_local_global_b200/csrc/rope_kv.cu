@@ -257,7 +257,8 @@ __global__ void __launch_bounds__(256) k_ring_gather(const bf16* __restrict__ k_
 // layer's chunk, already in the cache): window > 0: rows 0..window+extra-1
 // take positions pos0-window .. pos0+extra-1 (slot p mod window; negative
 // positions give zeros, never visible); window 0: rows 0..pos0+extra-1 take
-// positions 0..pos0+extra-1 (slot = position).
+// positions 0..pos0+extra-1 (slot = position). Rows below first_row are
+// left as they are (a shared layer's chunk re-read over its source's window).
 template <int D>
 __global__ void __launch_bounds__(256) k_gather_q8(const uint8_t* __restrict__ k_codes,
                                                    const float2* __restrict__ k_params,
@@ -266,7 +267,7 @@ __global__ void __launch_bounds__(256) k_gather_q8(const uint8_t* __restrict__ k
                                                    const int32_t* seq_lens_before, int extra, int Hkv,
                                                    int window, int cache_cap, const int32_t* page_table,
                                                    int page_size, int pages_per_seq, int n_pages, int win_rows,
-                                                   bf16* k_win, bf16* v_win, int* status) {
+                                                   int first_row, bf16* k_win, bf16* v_win, int* status) {
   constexpr int E = D / 32;  // codes per lane: 8 or 16
   const int b = blockIdx.y;
   const int64_t pos0 = seq_lens_before ? (int64_t)seq_lens_before[b] : 0;
@@ -277,7 +278,8 @@ __global__ void __launch_bounds__(256) k_gather_q8(const uint8_t* __restrict__ k
   }
   const int lane = threadIdx.x & 31;
   const int64_t n_items = rows * Hkv;
-  for (int64_t it = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5); it < n_items; it += (int64_t)gridDim.x * 8) {
+  for (int64_t it = (int64_t)first_row * Hkv + (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5); it < n_items;
+       it += (int64_t)gridDim.x * 8) {
     const int64_t r = it / Hkv;
     const int h = (int)(it % Hkv);
     const int64_t p = window > 0 ? pos0 - window + r : r;
@@ -497,19 +499,20 @@ cudaError_t launch_ring_gather(const bf16* k_cache, const bf16* v_cache, const i
 cudaError_t launch_gather_q8(const uint8_t* k_codes, const float2* k_params, const uint8_t* v_codes,
                              const float2* v_params, const int32_t* seq_lens_before, int extra, int B, int Hkv,
                              int D, int window, int cache_cap, const int32_t* page_table, int page_size,
-                             int pages_per_seq, int n_pages, int win_rows, bf16* k_win, bf16* v_win,
-                             int* status, cudaStream_t st) {
-  const int64_t rows = win_rows;  // an upper bound; blocks stride over the rest
+                             int pages_per_seq, int n_pages, int win_rows, int first_row, bf16* k_win,
+                             bf16* v_win, int* status, cudaStream_t st) {
+  if (first_row < 0) return cudaErrorInvalidValue;
+  const int64_t rows = std::max(win_rows - first_row, 1);  // an upper bound; blocks stride over the rest
   const int64_t blocks = std::min<int64_t>((rows * Hkv + 7) / 8, 1184);
   dim3 grid((unsigned)std::max<int64_t>(blocks, 1), B);
   if (D == 256)
     k_gather_q8<256><<<grid, 256, 0, st>>>(k_codes, k_params, v_codes, v_params, seq_lens_before, extra, Hkv,
                                            window, cache_cap, page_table, page_size, pages_per_seq, n_pages,
-                                           win_rows, k_win, v_win, status);
+                                           win_rows, first_row, k_win, v_win, status);
   else
     k_gather_q8<512><<<grid, 256, 0, st>>>(k_codes, k_params, v_codes, v_params, seq_lens_before, extra, Hkv,
                                            window, cache_cap, page_table, page_size, pages_per_seq, n_pages,
-                                           win_rows, k_win, v_win, status);
+                                           win_rows, first_row, k_win, v_win, status);
   return cudaGetLastError();
 }
 

@@ -32,6 +32,7 @@ GEMMA_ERR_DEVICE_RANGE = 7
 GEMMA_F_SHARED = 1
 GEMMA_F_KEQV = 2  # K = V on a global layer: no v_new, values read from the key cache
 GEMMA_F_KV_INT8 = 4  # int8 KV cache (Int8KVCache buffers); added automatically for those
+GEMMA_F_SOURCE_WINDOW = 8  # shared local layer after cached tokens: attend to the source call's window
 
 _P = ctypes.c_void_p
 _I = ctypes.c_int

@@ -106,17 +106,51 @@ class AttentionStack:
                     w.batch, w.seq, w.n_q_heads, t.n_kv_heads, t.head_dim, t.window))
         return max(sizes)
 
+    # ---------------------------------------------- windows of shared local layers
+    def _has_sharers(self, l: int) -> bool:
+        return any(self.descs[m].shared_from == l for m in range(self.n_layers))
+
+    def _window_source(self, l: int, chunked: bool):
+        """For a local layer's chunk after cached tokens on a stack whose
+        local layers share K/V: the source layer whose call leaves the K/V
+        window in its own workspace (GEMMA_F_SOURCE_WINDOW), else None."""
+        if not chunked or self.layer_type(l).window == 0:
+            return None
+        if self.is_shared(l):
+            return self.descs[l].shared_from
+        return l if self._has_sharers(l) else None
+
+    def _window_workspace(self, src: int, nbytes: int):
+        """The workspace a source layer and its sharers use for one chunk
+        (kept per source: layers in between must not write it)."""
+        if not hasattr(self, "_win_ws"):
+            self._win_ws = {}
+        buf = self._win_ws.get(src)
+        if buf is None or buf.numel() < nbytes:
+            buf = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=self.device)
+            self._win_ws[src] = buf
+        return buf
+
     def prefill_layer(self, l: int, q, k, v, out, *, workspace, seq_lens_before=None, lse=None,
                       stream=None):
+        """One layer's chunk. A local layer after cached tokens whose K/V
+        are shared runs, with its sharers, on a workspace of its own."""
         t = self.layer_type(l)
         shared = self.is_shared(l)
         keqv = self.keqv(l)
+        flags = (native.GEMMA_F_SHARED if shared else 0) | (native.GEMMA_F_KEQV if keqv else 0)
+        src = self._window_source(l, seq_lens_before is not None)
+        if src is not None:
+            flags |= native.GEMMA_F_SOURCE_WINDOW
+            n = native.gemma_attn_prefill_workspace_size_cached(
+                q.shape[0], q.shape[1], q.shape[2], t.n_kv_heads, t.head_dim, t.window, t.window,
+                native.GEMMA_F_KV_INT8 if self.w.kv_int8 else 0)
+            workspace = self._window_workspace(src, n)
         native.gemma_attn_prefill(
             q, None if shared else k, None if (shared or keqv) else v, self.k_cache[l],
             None if keqv else self.v_cache[l],
             window=t.window, rope_frac=t.rope_frac, rope_theta=t.rope_theta, scale=t.scale,
-            out=out, seq_lens_before=seq_lens_before, lse=lse, workspace=workspace,
-            flags=(native.GEMMA_F_SHARED if shared else 0) | (native.GEMMA_F_KEQV if keqv else 0),
+            out=out, seq_lens_before=seq_lens_before, lse=lse, workspace=workspace, flags=flags,
             stream=stream)
 
     def prefill_from_host(self, host_in, host_out, dev_bufs, *, workspace, seq_lens_before=None):
@@ -190,14 +224,23 @@ class AttentionStack:
 
     def decode_multi_layer(self, l: int, q, k, v, out, *, seq_lens, max_seq_len, workspace, stream=None):
         """tokens = q.shape[1] new tokens per sequence (a drafter's proposals
-        being checked); seq_lens counts them."""
+        being checked); seq_lens counts them. Local layers whose K/V are
+        shared run, with their sharers, as a chunk after the cached tokens
+        on a workspace of their own (GEMMA_F_SOURCE_WINDOW)."""
         t = self.layer_type(l)
         shared = self.is_shared(l)
         keqv = self.keqv(l)
+        flags = (native.GEMMA_F_SHARED if shared else 0) | (native.GEMMA_F_KEQV if keqv else 0)
+        src = self._window_source(l, True)
+        if src is not None:
+            flags |= native.GEMMA_F_SOURCE_WINDOW
+            n = native.gemma_attn_decode_multi_workspace_size(
+                q.shape[0], q.shape[1], q.shape[2], t.n_kv_heads, t.head_dim, t.window, max_seq_len, t.window,
+                flags | (native.GEMMA_F_KV_INT8 if self.w.kv_int8 else 0))
+            workspace = self._window_workspace(src, n)
         native.gemma_attn_decode_multi(
             q, None if shared else k, None if (shared or keqv) else v, self.k_cache[l],
             None if keqv else self.v_cache[l],
             seq_lens=seq_lens, max_seq_len=max_seq_len, window=t.window, rope_frac=t.rope_frac,
-            rope_theta=t.rope_theta, scale=t.scale, out=out, workspace=workspace,
-            flags=(native.GEMMA_F_SHARED if shared else 0) | (native.GEMMA_F_KEQV if keqv else 0),
+            rope_theta=t.rope_theta, scale=t.scale, out=out, workspace=workspace, flags=flags,
             stream=stream)

@@ -101,6 +101,30 @@ typedef enum gemma_status {
                              Decode reads codes. Combines with GEMMA_F_KEQV
                              and GEMMA_F_SHARED. */
 
+#define GEMMA_F_SOURCE_WINDOW 8u /* KV-shared local layers after cached tokens
+                             ("Gemma 4 Architecture Reference", Shared KV Cache:
+                             the last layers reuse an earlier local layer's
+                             K/V). A chunk after cached tokens on an unshared
+                             local layer leaves in its workspace the keys and
+                             values it attended to: the ring's last `window`
+                             positions before the chunk, then the chunk. With
+                             GEMMA_F_SHARED | GEMMA_F_SOURCE_WINDOW a shared
+                             local layer's call attends to them; its workspace
+                             must be the one of its source layer's call for the
+                             same chunk (same batch, s_new, head counts,
+                             head_dim, window and seq_lens_before), not written
+                             since except by other such shared calls. Without
+                             the flag that call is GEMMA_ERR_UNSUPPORTED: the
+                             source's chunk has replaced ring slots that the
+                             chunk's earlier queries still see. On an int8
+                             cache the chunk's own rows are read back from the
+                             codes, as a shared layer reads every row. In
+                             gemma_attn_decode_multi the flag on an unshared
+                             local layer selects the chunked-prefill path, so
+                             that the call leaves that window. Only for local
+                             layers after cached tokens (else
+                             GEMMA_ERR_INVALID_ARG). */
+
 /* Bytes of one layer's K (or V) cache buffer: batch * n_kv_heads *
  * cache_cap * head_dim * 2 for bf16; with GEMMA_F_KV_INT8 the codes, padded
  * to 256 bytes, plus 8 bytes of (min, step) per row. 0 on bad arguments. */
@@ -122,8 +146,9 @@ size_t gemma_kv_codes_bytes(int batch, int n_kv_heads, int cache_cap, int head_d
 /*        sequence (the chunk starts at that position), or NULL for 0.     */
 /*        On a local layer the chunk also attends to the ring's last       */
 /*        `window` cached positions (read before the chunk overwrites      */
-/*        them); a shared local layer after cached tokens returns          */
-/*        GEMMA_ERR_UNSUPPORTED (its source already replaced those slots). */
+/*        them); a shared local layer after cached tokens needs            */
+/*        GEMMA_F_SOURCE_WINDOW (else GEMMA_ERR_UNSUPPORTED: its source     */
+/*        already replaced those slots).                                   */
 /* out    [batch][s_new][n_q_heads][head_dim]  bf16 attention output        */
 /* lse    optional fp32 [batch][n_q_heads][s_new]: natural-log sum of       */
 /*        exp(scale * q.k) over the visible keys; NULL to skip.            */
@@ -210,14 +235,18 @@ int gemma_attn_decode(const void* q, const void* k_new, const void* v_new,
 /* workspace: gemma_attn_decode_multi_workspace_size(...) bytes, 256-byte  */
 /*        aligned; scratch.                                                */
 /*                                                                        */
-/* A global bf16 layer on a contiguous cache with (n_q_heads / n_kv_heads) */
-/* * tokens <= 128 runs one tensor-core kernel per split of the cached    */
-/* keys whose tile holds every q head of a KV head for all the tokens, so */
-/* the cache is streamed once per step as in single-token decode. Other   */
-/* layers (local, int8) run as a chunked prefill; a shared local layer is */
-/* GEMMA_ERR_UNSUPPORTED there, as in gemma_attn_prefill after cached     */
-/* tokens. Cache effects: the rotated new keys and the values are written */
-/* at their positions' slots, unless the layer is shared.                 */
+/* bf16 layers on a contiguous cache run one tensor-core kernel per split */
+/* of the cached keys whose tile holds every q head of a KV head for all  */
+/* the tokens, so the cache is streamed once per step as in single-token  */
+/* decode: global layers with (n_q_heads / n_kv_heads) * tokens <= 128,   */
+/* unshared local layers with that product <= 64 and tokens <= window     */
+/* (the ring is read as it was, plus the new rows; it is written after).  */
+/* Other layers (int8, shared local, larger products) run as a chunked    */
+/* prefill of the tokens after seq_lens - tokens cached ones; a shared    */
+/* local layer needs GEMMA_F_SOURCE_WINDOW, with its source layer's call  */
+/* passing it too (see that flag). Cache effects: the rotated new keys    */
+/* and the values are written at their positions' slots, unless the layer */
+/* is shared.                                                             */
 /* ---------------------------------------------------------------------- */
 size_t gemma_attn_decode_multi_workspace_size(int batch, int tokens, int n_q_heads,
                                               int n_kv_heads, int head_dim, int window,

@@ -141,10 +141,15 @@ PLAIN_WS_GLOBAL = native.gemma_attn_prefill_workspace_size(1, 16, 8, 4, 256, 0)
     (dict(cap=1024), E.GEMMA_ERR_INVALID_ARG),        # local ring must hold exactly the window
     (dict(lens=FAKE, wsb=16), E.GEMMA_ERR_CAPACITY),   # chunked local prefill is accepted
     (dict(lens=FAKE, flags=1, k=None, v=None), E.GEMMA_ERR_UNSUPPORTED),  # ... but not on a shared layer
+    (dict(lens=FAKE, flags=9, k=None, v=None, wsb=16), E.GEMMA_ERR_CAPACITY),  # ... unless on its source's window
+    (dict(lens=FAKE, flags=8, wsb=16), E.GEMMA_ERR_CAPACITY),          # the source's own call may pass the flag
+    (dict(flags=9, k=None, v=None), E.GEMMA_ERR_INVALID_ARG),          # the flag needs cached tokens
+    (dict(W=0, cap=4096, lens=FAKE, flags=9, k=None, v=None), E.GEMMA_ERR_INVALID_ARG),  # ... and a local layer
+    (dict(lens=FAKE, flags=13, k=None, v=None, wsb=16), E.GEMMA_ERR_CAPACITY),  # int8 shared, source window
     (dict(W=0, cap=8), E.GEMMA_ERR_CAPACITY),          # global cache shorter than the chunk
     (dict(k=None), E.GEMMA_ERR_INVALID_ARG),           # unshared layer without new keys
     (dict(flags=1), E.GEMMA_ERR_INVALID_ARG),          # shared layer with new keys
-    (dict(flags=8), E.GEMMA_ERR_INVALID_ARG),          # unknown flag
+    (dict(flags=16), E.GEMMA_ERR_INVALID_ARG),         # unknown flag
     (dict(flags=4, wsb=16), E.GEMMA_ERR_CAPACITY),     # int8 KV: accepted
     (dict(flags=4, W=0, cap=4095, wsb=16), E.GEMMA_ERR_INVALID_ARG),   # int8 KV: odd capacity
     (dict(flags=4, lens=FAKE, wsb=16), E.GEMMA_ERR_CAPACITY),          # int8 KV after cached tokens: accepted
@@ -182,7 +187,8 @@ def test_prefill_validation(over, code):
     (dict(flags=4, wsb=1024), E.GEMMA_ERR_CAPACITY),                   # int8 KV accepted
     (dict(flags=4, cap=4097, maxlen=4097, wsb=1024), E.GEMMA_ERR_INVALID_ARG),  # int8 KV: odd capacity
     (dict(flags=5, k=None, v=None, wsb=1024), E.GEMMA_ERR_CAPACITY),   # int8 KV on a shared layer: accepted
-    (dict(flags=8), E.GEMMA_ERR_INVALID_ARG),                          # unknown flag
+    (dict(flags=8), E.GEMMA_ERR_INVALID_ARG),                          # the source-window flag is not for decode
+    (dict(flags=16), E.GEMMA_ERR_INVALID_ARG),                         # unknown flag
 ])
 def test_decode_validation(over, code):
     assert _decode_raw(**over) == code
@@ -217,7 +223,10 @@ def _multi_raw(**over):
     (dict(W=1024, cap=1024, Hkv=16, D=256, frac=1.0, theta=1e4), E.GEMMA_ERR_CAPACITY),  # local: accepted
     (dict(W=1024, cap=4096, Hkv=16, D=256, frac=1.0, theta=1e4, wsb=1 << 30), E.GEMMA_ERR_INVALID_ARG),
     (dict(W=1024, cap=1024, Hkv=16, D=256, frac=1.0, theta=1e4, flags=1, k=None, v=None, wsb=1 << 30),
-     E.GEMMA_ERR_UNSUPPORTED),                                        # shared local after cached tokens
+     E.GEMMA_ERR_UNSUPPORTED),                                        # shared local after cached tokens ...
+    (dict(W=1024, cap=1024, Hkv=16, D=256, frac=1.0, theta=1e4, flags=9, k=None, v=None),
+     E.GEMMA_ERR_CAPACITY),                                           # ... on its source's window: routed
+    (dict(flags=8, wsb=1 << 30), E.GEMMA_ERR_INVALID_ARG),            # the source-window flag on a global layer
     (dict(flags=4), E.GEMMA_ERR_CAPACITY),                            # int8: route
 ])
 def test_decode_multi_validation(over, code):
