@@ -12,7 +12,11 @@
 // and the affine part and the offset are applied per key (S) and as one
 // scalar per head (O).
 //
-// Per CTA = (split, KV head, sequence), 128 threads, two CTAs per SM:
+// Per CTA = (split, KV head, sequence), 128 threads; four CTAs per SM at
+// head_dim 256 (measured on the 31B-shaped local layer, B64, ring 1024:
+// 154 us with two CTAs of a 12-slot ring, 132 with three, 126 with four of
+// a 6-slot ring: the short local splits are latency-bound, so more resident
+// warps pay), two at head_dim 512, whose O accumulators need the registers:
 //   warp 3      producer: per 16-key sub-block, the K and the V code rows
 //               arrive as TMA tiles of 16 rows x 128 bytes (one per 128-byte
 //               column chunk), 128-byte swizzled, plus one bulk copy each of
@@ -55,7 +59,7 @@ struct Q8Cfg {
   static constexpr int BOX_B = KB * 128;             // one TMA tile: 16 rows x 128 bytes
   static constexpr int REGION_B = NCH * BOX_B;       // 16 code rows, chunk-major, swizzled
   static constexpr int SLOT_B = 2 * REGION_B;        // K region, V region (K = V: 32 K rows)
-  static constexpr int NSLOT = D == 512 ? 6 : 12;
+  static constexpr int NSLOT = 6;
   static_assert(NSLOT % NCW == 0, "each ring slot needs a single consumer warp");
   static constexpr int RING_B = NSLOT * SLOT_B;
   static constexpr int PAR_B = 2 * KB * 8;           // K (min, step) [16], V [16] (K = V: 32 K)
@@ -72,7 +76,8 @@ struct Q8Cfg {
   static constexpr int MERGE_B = NCW * 8 * OSTR * 4;
   static_assert(MERGE_B <= RING_B, "merge buffer must fit in the drained ring");
   static_assert(BOX_B % 1024 == 0 && SLOT_B % 1024 == 0 && Q_OFF % 16 == 0, "alignment");
-  static_assert(2 * (SMEM + 1024) <= 228 * 1024, "two CTAs per SM");
+  static constexpr int CTAS_PER_SM = D == 256 ? 4 : 2;  // see the launch bounds
+  static_assert(CTAS_PER_SM * (SMEM + 1024) <= 228 * 1024, "resident CTAs per SM");
   static constexpr int VCH = D / 128;                // 16-byte units of V codes per lane and key row
   static constexpr int PPL = 4 / VCH;                // lane pairs per 128-byte line (P.V reads)
 };
@@ -125,7 +130,7 @@ __device__ __forceinline__ float pow2_ceil(float x) {
 // PAGED: the cache is a pool named by a.page_table (see cache_row); the
 // contiguous instance keeps the plain row arithmetic of one (b, g) range.
 template <int D, bool PAGED>
-__global__ void __launch_bounds__(32 * (NCW + 1), 2)
+__global__ void __launch_bounds__(32 * (NCW + 1), Q8Cfg<D>::CTAS_PER_SM)
     k_decode_split_q8(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                       DecodeAttnArgs a) {
   using C = Q8Cfg<D>;
