@@ -201,12 +201,12 @@ size_t prefill_ws_parts(int B, int S, int Hq, int Hkv, int D, int window, size_t
   return q + std::max(k, 2 * win);
 }
 
-// Multi-token decode on the tensor-core kernels (bf16, contiguous cache):
-// a global layer whose G q heads x tokens rows fit one 128-row tile, or an
-// unshared local layer with at most 64 such rows and tokens <= window.
-bool verify_fast(int tokens, int window, int n_q_heads, int n_kv_heads, int head_dim, unsigned flags, bool paged) {
-  if ((flags & (GEMMA_F_KV_INT8 | GEMMA_F_SOURCE_WINDOW)) || paged || (head_dim != 256 && head_dim != 512))
-    return false;
+// Multi-token decode on the tensor-core kernels (bf16 caches): a global
+// layer (contiguous or paged) whose G q heads x tokens rows fit one 128-row
+// tile, or an unshared local layer with at most 64 such rows and
+// tokens <= window.
+bool verify_fast(int tokens, int window, int n_q_heads, int n_kv_heads, int head_dim, unsigned flags) {
+  if ((flags & (GEMMA_F_KV_INT8 | GEMMA_F_SOURCE_WINDOW)) || (head_dim != 256 && head_dim != 512)) return false;
   if (window == 0) return (n_q_heads / n_kv_heads) * tokens <= 128;
   return !(flags & GEMMA_F_SHARED) && tokens <= window && tokens <= 128 &&
          verify_tc_rows(n_q_heads, n_kv_heads, tokens, head_dim) != 0;
@@ -812,7 +812,7 @@ size_t gemma_attn_decode_multi_workspace_size(int batch, int tokens, int n_q_hea
   if (batch <= 0 || tokens <= 0 || n_q_heads <= 0 || n_kv_heads <= 0 || head_dim <= 0 || max_seq_len <= 0 ||
       cache_cap <= 0)
     return 0;
-  if (verify_fast(tokens, window, n_q_heads, n_kv_heads, head_dim, flags, false)) {
+  if (verify_fast(tokens, window, n_q_heads, n_kv_heads, head_dim, flags)) {
     int chunk, n_splits;
     verify_plan(batch, n_q_heads, n_kv_heads, tokens, head_dim, window, max_seq_len, &chunk, &n_splits);
     size_t a, b, c;
@@ -821,11 +821,11 @@ size_t gemma_attn_decode_multi_workspace_size(int batch, int tokens, int n_q_hea
   return verify_route_ws(batch, tokens, n_q_heads, n_kv_heads, head_dim, window, cache_cap, flags);
 }
 
-int gemma_attn_decode_multi(const void* q, const void* k_new, const void* v_new, void* k_cache, void* v_cache,
-                            int cache_cap, const int32_t* seq_lens, int max_seq_len, int batch, int tokens,
-                            int window, int n_q_heads, int n_kv_heads, int head_dim, float rope_frac,
-                            float rope_theta, float scale, void* out, void* workspace, size_t workspace_bytes,
-                            unsigned flags, void* stream) {
+static int multi_impl(const void* q, const void* k_new, const void* v_new, void* k_cache, void* v_cache,
+                      int cache_cap, const int32_t* seq_lens, int max_seq_len, int batch, int tokens, int window,
+                      int n_q_heads, int n_kv_heads, int head_dim, float rope_frac, float rope_theta, float scale,
+                      void* out, void* workspace, size_t workspace_bytes, unsigned flags, void* stream,
+                      const CacheLayout& L) {
   int rc = check_heads(n_q_heads, n_kv_heads, head_dim, window, rope_frac, rope_theta, scale);
   if (rc) return rc;
   if (batch <= 0 || tokens <= 0 || max_seq_len <= 0)
@@ -835,7 +835,7 @@ int gemma_attn_decode_multi(const void* q, const void* k_new, const void* v_new,
     return fail(GEMMA_ERR_CAPACITY, "global layer: cache_cap %d < max_seq_len %d", cache_cap, max_seq_len);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   unsigned char* ws = static_cast<unsigned char*>(workspace);
-  if (!verify_fast(tokens, window, n_q_heads, n_kv_heads, head_dim, flags, false)) {
+  if (!verify_fast(tokens, window, n_q_heads, n_kv_heads, head_dim, flags)) {
     // the new tokens as a chunk after seq_lens - tokens cached tokens
     const size_t need = verify_route_ws(batch, tokens, n_q_heads, n_kv_heads, head_dim, window, cache_cap, flags);
     if (!workspace || workspace_bytes < need)
@@ -845,7 +845,7 @@ int gemma_attn_decode_multi(const void* q, const void* k_new, const void* v_new,
     const size_t head = align256((size_t)batch * 4);
     return prefill_impl(q, k_new, v_new, k_cache, v_cache, cache_cap, before, batch, tokens, window, n_q_heads,
                         n_kv_heads, head_dim, rope_frac, rope_theta, scale, out, nullptr, ws + head,
-                        workspace_bytes - head, flags, stream, contiguous(cache_cap, batch), seq_lens);
+                        workspace_bytes - head, flags, stream, L, seq_lens);
   }
   rc = check_kv_flags(flags, window, k_new, v_new, k_cache, &v_cache);
   if (rc) return rc;
@@ -887,10 +887,10 @@ int gemma_attn_decode_multi(const void* q, const void* k_new, const void* v_new,
   // tokens still see: its rotated keys wait in the workspace, and the ring
   // is written once the attention is done
   ra.k_stage = window > 0 ? reinterpret_cast<bf16*>(ws + off_kst) : nullptr;
-  ra.page_table = nullptr;
-  ra.page_size = cache_cap;
-  ra.pages_per_seq = 1;
-  ra.n_pages = batch;
+  ra.page_table = L.page_table;
+  ra.page_size = L.page_size;
+  ra.pages_per_seq = L.pages_per_seq;
+  ra.n_pages = L.n_pages;
   ra.status = status;
   ProfScope p_app(GEMMA_KERNEL_DECODE_APPEND, st);
   cudaError_t e = launch_decode_rope_append(ra, batch, head_dim, st);
@@ -900,9 +900,14 @@ int gemma_attn_decode_multi(const void* q, const void* k_new, const void* v_new,
   const int64_t D = head_dim;
   VerifyAttnArgs va{};
   va.q_rot = ra.q_rot;
-  va.k = KVView{static_cast<const bf16*>(k_cache), (int64_t)n_kv_heads * cache_cap * D, D, (int64_t)cache_cap * D};
+  const int64_t ps = L.page_size;  // rows of a view: a page, or a sequence's cache
+  va.k = KVView{static_cast<const bf16*>(k_cache), (int64_t)n_kv_heads * ps * D, D, ps * D};
   va.v = KVView{static_cast<const bf16*>(v_cache), va.k.stride_b, va.k.stride_row, va.k.stride_h};
   va.cache_cap = cache_cap;
+  va.page_table = L.page_table;
+  va.page_size = L.page_size;
+  va.pages_per_seq = L.pages_per_seq;
+  va.n_pages = L.n_pages;
   va.window = window;
   va.k_tail = ra.k_stage;
   va.v_tail = ra.v_new;
@@ -953,6 +958,29 @@ int gemma_attn_decode_multi(const void* q, const void* k_new, const void* v_new,
   }
   if (e != cudaSuccess) return cuda_fail(e, "decode combine launch");
   return succeed();
+}
+
+int gemma_attn_decode_multi(const void* q, const void* k_new, const void* v_new, void* k_cache, void* v_cache,
+                            int cache_cap, const int32_t* seq_lens, int max_seq_len, int batch, int tokens,
+                            int window, int n_q_heads, int n_kv_heads, int head_dim, float rope_frac,
+                            float rope_theta, float scale, void* out, void* workspace, size_t workspace_bytes,
+                            unsigned flags, void* stream) {
+  return multi_impl(q, k_new, v_new, k_cache, v_cache, cache_cap, seq_lens, max_seq_len, batch, tokens, window,
+                    n_q_heads, n_kv_heads, head_dim, rope_frac, rope_theta, scale, out, workspace, workspace_bytes,
+                    flags, stream, contiguous(cache_cap, batch));
+}
+
+int gemma_attn_decode_multi_paged(const void* q, const void* k_new, const void* v_new, void* k_pool, void* v_pool,
+                                  const int32_t* page_table, int page_size, int pages_per_seq, int n_pages,
+                                  const int32_t* seq_lens, int max_seq_len, int batch, int tokens, int n_q_heads,
+                                  int n_kv_heads, int head_dim, float rope_frac, float rope_theta, float scale,
+                                  void* out, void* workspace, size_t workspace_bytes, unsigned flags,
+                                  void* stream) {
+  int rc = check_paged(page_table, page_size, pages_per_seq, n_pages);
+  if (rc) return rc;
+  return multi_impl(q, k_new, v_new, k_pool, v_pool, pages_per_seq * page_size, seq_lens, max_seq_len, batch, tokens,
+                    0, n_q_heads, n_kv_heads, head_dim, rope_frac, rope_theta, scale, out, workspace,
+                    workspace_bytes, flags, stream, CacheLayout{page_table, page_size, pages_per_seq, n_pages});
 }
 
 int gemma_attn_visible_ranges(const int32_t* seq_lens_before, int batch, int s_new, int window,

@@ -184,6 +184,12 @@ struct VerifyAttnArgs {
   int window;
   const bf16* k_tail;
   const bf16* v_tail;
+  // cache pages (global layers): k / v are head-major views of a pool of
+  // n_pages pages of page_size rows, position p of sequence b at row
+  // p % page_size of page page_table[b][p / page_size]; page_table null:
+  // contiguous (page_size = cache_cap, n_pages = B)
+  const int32_t* page_table;
+  int page_size, pages_per_seq, n_pages;
   const int32_t* seq_lens;  // device [B], including the new tokens
   int tokens, Hq, Hkv;
   int chunk, n_splits;      // keys per split (a multiple of 128), splits planned

@@ -658,8 +658,9 @@ cudaError_t launch_verify_attn_rows(const VerifyAttnArgs& a, int B, int D, cudaS
     if (!make_map_bf16_4d(&mq, a.q_rot, dims, str, box)) return cudaErrorInvalidValue;
   }
   {
-    // head-major cache views: (d, key, head, b), K boxes of 128 keys, V boxes of 64
-    const uint64_t dims[4] = {(uint64_t)D, (uint64_t)a.cache_cap, (uint64_t)a.Hkv, (uint64_t)B};
+    // head-major views (d, row, head, page) of the cache (a page per sequence
+    // when contiguous), K boxes of 128 rows, V boxes of 64
+    const uint64_t dims[4] = {(uint64_t)D, (uint64_t)a.page_size, (uint64_t)a.Hkv, (uint64_t)a.n_pages};
     const uint64_t strk[3] = {(uint64_t)a.k.stride_row * E, (uint64_t)a.k.stride_h * E, (uint64_t)a.k.stride_b * E};
     const uint64_t strv[3] = {(uint64_t)a.v.stride_row * E, (uint64_t)a.v.stride_h * E, (uint64_t)a.v.stride_b * E};
     const uint32_t bk[4] = {64, (uint32_t)BN, 1, 1}, bv[4] = {64, 64, 1, 1};
@@ -681,10 +682,10 @@ cudaError_t launch_verify_attn_rows(const VerifyAttnArgs& a, int B, int D, cudaS
   t.kv_token_major = 0;
   t.key_off_window = 0;
   t.n_qtiles = 1;
-  t.page_table = nullptr;
-  t.page_size = a.cache_cap;
-  t.pages_per_seq = 1;
-  t.n_pages = B;
+  t.page_table = a.page_table;
+  t.page_size = a.page_size;
+  t.pages_per_seq = a.pages_per_seq;
+  t.n_pages = a.n_pages;
   t.seq_lens = a.seq_lens;
   t.tokens = a.tokens;
   t.chunk = a.chunk;

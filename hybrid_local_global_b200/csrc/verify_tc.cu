@@ -97,6 +97,8 @@ struct VArgs {
   int Hq, Hkv, tokens, chunk, n_splits;
   int window;  // LOCAL: ring slots
   int64_t key_cap;
+  const int32_t* page_table;  // global layers on a paged pool (see VerifyAttnArgs); else null
+  int page_size, pages_per_seq, n_pages;
   const int32_t* seq_lens;
   float* part_o;
   float* part_lse;
@@ -254,6 +256,18 @@ __global__ void __launch_bounds__(192, 1)
           const bool tail = LOCAL && jt == n_ring;
           const int key0 = (int)(k_begin + (int64_t)jt * BN);
           const CUtensorMap* map = tail ? (kind == 0 ? &tm_kt : &tm_vt) : (kind == 0 ? &tm_k : &tm_v);
+          // view row and batch of the tile: a page of the pool (a tile never
+          // straddles a page: page_size is a multiple of 128), or the sequence
+          int row = key0, page = b;
+          if (!LOCAL && a.page_table) {
+            const int pi = key0 / a.page_size;
+            page = pi < a.pages_per_seq ? a.page_table[(int64_t)b * a.pages_per_seq + pi] : 0;
+            if (page < 0 || page >= a.n_pages) {  // a page outside the pool: report, read page 0
+              set_status(a.status, GEMMA_ERR_DEVICE_RANGE);
+              page = 0;
+            }
+            row = key0 - pi * a.page_size;
+          }
           for (int h = 0; h < MT; ++h, ++item) {
             const int s = item % NSTAGE;
             if (item >= NSTAGE &&
@@ -270,7 +284,7 @@ __global__ void __launch_bounds__(192, 1)
               if (tail)  // (d, head, token, b): tokens past the last are zeros
                 tc::tma_load_4d(dst + cc * CH_B, map, h * 128 + cc * 64, g, 0, b, bar);
               else
-                tc::tma_load_4d(dst + cc * CH_B, map, h * 128 + cc * 64, key0, g, b, bar);
+                tc::tma_load_4d(dst + cc * CH_B, map, h * 128 + cc * 64, row, g, page, bar);
             }
           }
         }
@@ -598,9 +612,11 @@ cudaError_t launch_verify_attn_tc(const VerifyAttnArgs& a, int B, int D, cudaStr
     const uint32_t box[4] = {64, (uint32_t)G, (uint32_t)a.tokens, 1};
     if (!make_map_bf16_4d(&mq, a.q_rot, dims, str, box)) return cudaErrorInvalidValue;
   }
+  if (a.window > 0 && a.page_table) return cudaErrorInvalidValue;  // rings are not paged
   {
-    // head-major cache views (d, key, head, b); boxes of 64 dims x 128 keys
-    const uint64_t dims[4] = {(uint64_t)D, (uint64_t)a.cache_cap, (uint64_t)a.Hkv, (uint64_t)B};
+    // head-major views (d, row, head, page) of the cache (a page per
+    // sequence when contiguous); boxes of 64 dims x 128 rows
+    const uint64_t dims[4] = {(uint64_t)D, (uint64_t)a.page_size, (uint64_t)a.Hkv, (uint64_t)a.n_pages};
     const uint64_t strk[3] = {(uint64_t)a.k.stride_row * E, (uint64_t)a.k.stride_h * E, (uint64_t)a.k.stride_b * E};
     const uint64_t strv[3] = {(uint64_t)a.v.stride_row * E, (uint64_t)a.v.stride_h * E, (uint64_t)a.v.stride_b * E};
     const uint32_t box[4] = {64, (uint32_t)BN, 1, 1};
@@ -620,6 +636,10 @@ cudaError_t launch_verify_attn_tc(const VerifyAttnArgs& a, int B, int D, cudaStr
   }
   VArgs v{};
   v.window = a.window;
+  v.page_table = a.page_table;
+  v.page_size = a.page_size;
+  v.pages_per_seq = a.pages_per_seq;
+  v.n_pages = a.n_pages;
   v.Hq = a.Hq;
   v.Hkv = a.Hkv;
   v.tokens = a.tokens;

@@ -77,6 +77,8 @@ _kv_codes = _sig("gemma_kv_codes_bytes", _SZ, [_I, _I, _I, _I])
 _multi_ws = _sig("gemma_attn_decode_multi_workspace_size", _SZ, [_I, _I, _I, _I, _I, _I, _I, _I, ctypes.c_uint])
 _multi = _sig("gemma_attn_decode_multi", _I, [_P, _P, _P, _P, _P, _I, _P, _I, _I, _I, _I, _I, _I, _I,
                                               _F, _F, _F, _P, _P, _SZ, ctypes.c_uint, _P])
+_multi_paged = _sig("gemma_attn_decode_multi_paged", _I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _P, _I, _I, _I, _I,
+                                                          _I, _I, _F, _F, _F, _P, _P, _SZ, ctypes.c_uint, _P])
 
 EXPORTED = ["gemma_attn_prefill_workspace_size", "gemma_attn_prefill",
             "gemma_attn_decode_workspace_size", "gemma_attn_decode", "gemma_kv_share_bind",
@@ -290,6 +292,27 @@ def gemma_attn_decode_paged(q, k_new, v_new, k_pool, v_pool, page_table, *, seq_
                                 _stream(stream)))
 
 
+def gemma_attn_decode_multi_paged(q, k_new, v_new, k_pool, v_pool, page_table, *, seq_lens, max_seq_len, rope_frac,
+                                  rope_theta, scale, out, workspace=None, flags=0, stream=None):
+    """Multi-token decode of a global layer on a paged cache: q [B,T,Hq,D],
+    k_new/v_new [B,T,Hkv,D]; pools and page table as gemma_attn_prefill_paged."""
+    for t, n in ((q, "q"), (k_new, "k_new"), (v_new, "v_new"), (k_pool, "k_pool"), (v_pool, "v_pool"),
+                 (out, "out")):
+        _bf16(t, n)
+    if seq_lens.dtype != torch.int32 or not seq_lens.is_cuda:
+        raise TypeError("seq_lens must be an int32 CUDA tensor")
+    B, T, Hq, D = q.shape
+    n_pages, Hkv, ps, pps = _paged_args(k_pool, page_table)
+    flags |= _kv_kind(k_pool, v_pool)
+    if workspace is None:
+        n = gemma_attn_decode_multi_workspace_size(B, T, Hq, Hkv, D, 0, max_seq_len, ps * pps, flags)
+        workspace = torch.empty(max(n, 1), dtype=torch.uint8, device=q.device)
+    return _check(_multi_paged(_ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_pool), _ptr(v_pool), _ptr(page_table),
+                               ps, pps, n_pages, _ptr(seq_lens), max_seq_len, B, T, Hq, Hkv, D, rope_frac,
+                               rope_theta, scale, _ptr(out), _ptr(workspace), workspace.numel(), flags,
+                               _stream(stream)))
+
+
 def gemma_kv_share_bind(dst: gemma_kv_desc, src: gemma_kv_desc) -> int:
     return _check(_bind(ctypes.byref(dst), ctypes.byref(src)))
 
@@ -356,7 +379,8 @@ def gemma_attn_profile_read(kernel: int):
 
 _decode_noalloc = _sig("gemma_attn_decode_noalloc", _I, [_P, _P, _P, _P, _P, _I, _P, _I, _I, _I, _I, _I,
                                                          _I, _F, _F, _F, _P, ctypes.c_uint, _P])
-EXPORTED += ["gemma_attn_decode_noalloc", "gemma_attn_decode_multi_workspace_size", "gemma_attn_decode_multi"]
+EXPORTED += ["gemma_attn_decode_noalloc", "gemma_attn_decode_multi_workspace_size", "gemma_attn_decode_multi",
+             "gemma_attn_decode_multi_paged"]
 NOALLOC_SCRATCH_BYTES = 32 << 20
 
 

@@ -300,6 +300,17 @@ int gemma_attn_decode_paged(const void* q, const void* k_new, const void* v_new,
                             int n_q_heads, int n_kv_heads, int head_dim, float rope_frac,
                             float rope_theta, float scale, void* out, void* workspace,
                             size_t workspace_bytes, unsigned flags, void* stream);
+/* Multi-token decode (gemma_attn_decode_multi) on a paged global cache;   */
+/* the workspace is gemma_attn_decode_multi_workspace_size(batch, tokens,  */
+/* n_q_heads, n_kv_heads, head_dim, 0, max_seq_len, pages_per_seq *        */
+/* page_size, flags).                                                      */
+int gemma_attn_decode_multi_paged(const void* q, const void* k_new, const void* v_new,
+                                  void* k_pool, void* v_pool, const int32_t* page_table,
+                                  int page_size, int pages_per_seq, int n_pages,
+                                  const int32_t* seq_lens, int max_seq_len, int batch, int tokens,
+                                  int n_q_heads, int n_kv_heads, int head_dim, float rope_frac,
+                                  float rope_theta, float scale, void* out, void* workspace,
+                                  size_t workspace_bytes, unsigned flags, void* stream);
 
 /* ---------------------------------------------------------------------- */
 /* Decode without allocation. The pages have no counterpart for this entry */
