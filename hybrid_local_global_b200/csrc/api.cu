@@ -261,6 +261,30 @@ size_t verify_route_ws(int B, int tokens, int Hq, int Hkv, int D, int window, in
          prefill_ws_parts(B, tokens, Hq, Hkv, D, window, &off_k, nullptr, prefix ? cache_cap : 0);
 }
 
+// Multi-token decode on an int8 global layer: the tokens one at a time
+// through single-token decode, which is what the call computes (a chunked
+// prefill would dequantize the whole cached prefix into the workspace).
+// Workspace: per-token lengths, the decode workspace, then one token's q,
+// new K and V, and output.
+bool verify_by_decode(int window, unsigned flags) { return window == 0 && (flags & GEMMA_F_KV_INT8); }
+
+size_t verify_decode_ws(int B, int Hq, int Hkv, int D, int max_len, size_t* off_dec, size_t* off_q,
+                        size_t* off_k, size_t* off_v, size_t* off_o) {
+  int chunk, n_splits;
+  decode_plan(B, Hkv, 0, max_len, &chunk, &n_splits);
+  size_t a, b, o = align256((size_t)B * 4);
+  *off_dec = o;
+  o += align256(decode_ws_parts(B, Hq, Hkv, D, n_splits, &a, &b));
+  *off_q = o;
+  o += align256((size_t)B * Hq * D * 2);
+  *off_k = o;
+  o += align256((size_t)B * Hkv * D * 2);
+  *off_v = o;
+  o += align256((size_t)B * Hkv * D * 2);
+  *off_o = o;
+  return o + align256((size_t)B * Hq * D * 2);
+}
+
 }  // namespace
 
 namespace hlg {
@@ -812,6 +836,10 @@ size_t gemma_attn_decode_multi_workspace_size(int batch, int tokens, int n_q_hea
   if (batch <= 0 || tokens <= 0 || n_q_heads <= 0 || n_kv_heads <= 0 || head_dim <= 0 || max_seq_len <= 0 ||
       cache_cap <= 0)
     return 0;
+  if (verify_by_decode(window, flags)) {
+    size_t a, b, c, d, e;
+    return verify_decode_ws(batch, n_q_heads, n_kv_heads, head_dim, max_seq_len, &a, &b, &c, &d, &e);
+  }
   if (verify_fast(tokens, window, n_q_heads, n_kv_heads, head_dim, flags)) {
     int chunk, n_splits;
     verify_plan(batch, n_q_heads, n_kv_heads, tokens, head_dim, window, max_seq_len, &chunk, &n_splits);
@@ -835,6 +863,49 @@ static int multi_impl(const void* q, const void* k_new, const void* v_new, void*
     return fail(GEMMA_ERR_CAPACITY, "global layer: cache_cap %d < max_seq_len %d", cache_cap, max_seq_len);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   unsigned char* ws = static_cast<unsigned char*>(workspace);
+  if (verify_by_decode(window, flags)) {
+    rc = check_kv_flags(flags, window, k_new, v_new, k_cache, &v_cache);
+    if (rc) return rc;
+    if (flags & GEMMA_F_SOURCE_WINDOW)
+      return fail(GEMMA_ERR_INVALID_ARG, "GEMMA_F_SOURCE_WINDOW: local layers after cached tokens only");
+    if (!q || !out || !k_cache || !v_cache) return fail(GEMMA_ERR_INVALID_ARG, "null tensor pointer");
+    if (!aligned16(q) || !aligned16(out) || !aligned16(k_cache) || !aligned16(v_cache) ||
+        (k_new && !aligned16(k_new)) || (v_new && !aligned16(v_new)) || !aligned16(workspace))
+      return fail(GEMMA_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
+    if (cache_cap % 2) return fail(GEMMA_ERR_INVALID_ARG, "int8 KV: cache_cap %d must be even", cache_cap);
+    size_t off_dec, off_q, off_k, off_v, off_o;
+    const size_t need =
+        verify_decode_ws(batch, n_q_heads, n_kv_heads, head_dim, max_seq_len, &off_dec, &off_q, &off_k, &off_v, &off_o);
+    if (!workspace || workspace_bytes < need)
+      return fail(GEMMA_ERR_CAPACITY, "workspace %zu bytes < %zu", workspace_bytes, need);
+    // token t of every sequence: its rows out of [B][tokens][..] into the
+    // workspace, a decode at length seq_lens - (tokens - 1 - t), its output back
+    int32_t* lens_t = reinterpret_cast<int32_t*>(ws);
+    const size_t qrow = (size_t)n_q_heads * head_dim * 2, kvrow = (size_t)n_kv_heads * head_dim * 2;
+    const size_t dec_bytes = off_q - off_dec;
+    for (int t = 0; t < tokens; ++t) {
+      cudaError_t e = launch_lens_minus(seq_lens, lens_t, batch, tokens - 1 - t, st);
+      if (e == cudaSuccess)
+        e = cudaMemcpy2DAsync(ws + off_q, qrow, static_cast<const unsigned char*>(q) + t * qrow, tokens * qrow, qrow,
+                              batch, cudaMemcpyDeviceToDevice, st);
+      if (e == cudaSuccess && k_new)
+        e = cudaMemcpy2DAsync(ws + off_k, kvrow, static_cast<const unsigned char*>(k_new) + t * kvrow,
+                              tokens * kvrow, kvrow, batch, cudaMemcpyDeviceToDevice, st);
+      if (e == cudaSuccess && v_new)
+        e = cudaMemcpy2DAsync(ws + off_v, kvrow, static_cast<const unsigned char*>(v_new) + t * kvrow,
+                              tokens * kvrow, kvrow, batch, cudaMemcpyDeviceToDevice, st);
+      if (e != cudaSuccess) return cuda_fail(e, "multi-token decode staging");
+      rc = decode_impl(ws + off_q, k_new ? ws + off_k : nullptr, v_new ? ws + off_v : nullptr, k_cache,
+                       (flags & GEMMA_F_KEQV) ? nullptr : v_cache, cache_cap, lens_t, max_seq_len, batch, 0,
+                       n_q_heads, n_kv_heads, head_dim, rope_frac, rope_theta, scale, ws + off_o, ws + off_dec,
+                       dec_bytes, flags, stream, L);
+      if (rc) return rc;
+      e = cudaMemcpy2DAsync(static_cast<unsigned char*>(out) + t * qrow, tokens * qrow, ws + off_o, qrow, qrow,
+                            batch, cudaMemcpyDeviceToDevice, st);
+      if (e != cudaSuccess) return cuda_fail(e, "multi-token decode output copy");
+    }
+    return succeed();
+  }
   if (!verify_fast(tokens, window, n_q_heads, n_kv_heads, head_dim, flags)) {
     // the new tokens as a chunk after seq_lens - tokens cached tokens
     const size_t need = verify_route_ws(batch, tokens, n_q_heads, n_kv_heads, head_dim, window, cache_cap, flags);

@@ -241,12 +241,14 @@ int gemma_attn_decode(const void* q, const void* k_new, const void* v_new,
 /* decode: global layers with (n_q_heads / n_kv_heads) * tokens <= 128,   */
 /* unshared local layers with that product <= 64 and tokens <= window     */
 /* (the ring is read as it was, plus the new rows; it is written after).  */
-/* Other layers (int8, shared local, larger products) run as a chunked    */
-/* prefill of the tokens after seq_lens - tokens cached ones; a shared    */
-/* local layer needs GEMMA_F_SOURCE_WINDOW, with its source layer's call  */
-/* passing it too (see that flag). Cache effects: the rotated new keys    */
-/* and the values are written at their positions' slots, unless the layer */
-/* is shared.                                                             */
+/* An int8 global layer takes the tokens one at a time through single-   */
+/* token decode (its workspace does not grow with the cached length).     */
+/* Other layers (int8 local, shared local, larger products) run as a      */
+/* chunked prefill of the tokens after seq_lens - tokens cached ones; a   */
+/* shared local layer needs GEMMA_F_SOURCE_WINDOW, with its source        */
+/* layer's call passing it too (see that flag). Cache effects: the        */
+/* rotated new keys and the values are written at their positions' slots, */
+/* unless the layer is shared.                                            */
 /* ---------------------------------------------------------------------- */
 size_t gemma_attn_decode_multi_workspace_size(int batch, int tokens, int n_q_heads,
                                               int n_kv_heads, int head_dim, int window,

@@ -246,8 +246,13 @@ def test_decode_multi_workspace_sizes():
     assert routed >= 256 + native.gemma_attn_prefill_workspace_size_cached(1, 40, 32, 16, 256, 1024, 1024, 0)
     shared = native.gemma_attn_decode_multi_workspace_size(1, 4, 32, 16, 256, 1024, 4096, 1024, native.GEMMA_F_SHARED)
     assert shared >= 256 + native.gemma_attn_prefill_workspace_size_cached(1, 4, 32, 16, 256, 1024, 1024, 0)
+    # int8 global layers decode the tokens one at a time: the decode workspace plus one token's rows,
+    # whatever the cached length (a chunked prefill would need the whole prefix in bf16)
     q8 = native.gemma_attn_decode_multi_workspace_size(2, 4, 32, 4, 512, 0, 4096, 4096, native.GEMMA_F_KV_INT8)
-    assert q8 >= native.gemma_attn_prefill_workspace_size_cached(2, 4, 32, 4, 512, 0, 4096, native.GEMMA_F_KV_INT8)
+    assert q8 >= native.gemma_attn_decode_workspace_size(2, 32, 4, 512, 0, 4096) + 2 * (32 + 4) * 512 * 2 * 2
+    big = native.gemma_attn_decode_multi_workspace_size(64, 4, 32, 4, 512, 0, 131072, 131072, native.GEMMA_F_KV_INT8)
+    assert big < 1 << 30 < native.gemma_attn_prefill_workspace_size_cached(64, 4, 32, 4, 512, 0, 131072,
+                                                                             native.GEMMA_F_KV_INT8)
     assert native.gemma_attn_decode_multi_workspace_size(0, 4, 32, 4, 512, 0, 4096, 4096, 0) == 0
     assert native.gemma_attn_decode_multi_workspace_size(2, 0, 32, 4, 512, 0, 4096, 4096, 0) == 0
 

@@ -154,29 +154,70 @@ def test_multi_routed_layers(oracle, case):
     run_multi_case(oracle, frac=case.pop("frac", 1.0), theta=case.pop("theta", 1e4), **case)
 
 
-def test_multi_int8_global_matches_prefill_route(oracle):
-    """An int8 global layer goes through the chunked prefill: the result is
-    bit-identical to gemma_attn_prefill after seq_lens - tokens cached tokens
-    on a copy of the same cache."""
+@pytest.mark.parametrize("keqv", [False, True])
+def test_multi_int8_global_equals_consecutive_decodes(oracle, keqv):
+    """An int8 global layer takes the tokens one at a time through
+    single-token decode: bit-identical to T gemma_attn_decode calls at
+    lengths seq_lens - T + 1 .. seq_lens on a copy of the cache (which the
+    int8 decode tests hold to the oracle), with the same codes written."""
     dev = torch.device("cuda")
     B, T, Hq, Hkv, D, lens = 2, 4, 32, 4, 512, [1500, 300]
     cap = 1600
-    g = synth.generator(331, "cuda")
-    kc = synth.fill_int8_cache_(native.Int8KVCache(B, Hkv, cap, D, dev), g)
-    vc = synth.fill_int8_cache_(native.Int8KVCache(B, Hkv, cap, D, dev), g)
-    kc2, vc2 = native.Int8KVCache(B, Hkv, cap, D, dev), native.Int8KVCache(B, Hkv, cap, D, dev)
+    g = synth.generator(331 + keqv, "cuda")
+
+    def fresh():
+        return synth.fill_int8_cache_(native.Int8KVCache(B, Hkv, cap, D, dev), g)
+
+    kc = fresh()
+    vc = kc if keqv else fresh()
+    kc2 = native.Int8KVCache(B, Hkv, cap, D, dev)
+    kc2.buf.copy_(kc.buf)
+    vc2 = kc2
+    if not keqv:
+        vc2 = native.Int8KVCache(B, Hkv, cap, D, dev)
+        vc2.buf.copy_(vc.buf)
+    q = synth.randn_bf16((B, T, Hq, D), g, "cuda")
+    kn = synth.randn_bf16((B, T, Hkv, D), g, "cuda")
+    vn = None if keqv else synth.randn_bf16((B, T, Hkv, D), g, "cuda")
+    flags = native.GEMMA_F_KEQV if keqv else 0
+    kw = dict(window=0, rope_frac=0.25, rope_theta=1e6, scale=1.0 / math.sqrt(D), flags=flags)
+    o1 = torch.empty((B, T, Hq, D), dtype=torch.bfloat16, device=dev)
+    native.gemma_attn_decode_multi(q, kn, vn, kc, None if keqv else vc, max_seq_len=max(lens), out=o1,
+                                   seq_lens=torch.tensor(lens, dtype=torch.int32, device=dev), **kw)
+    o2 = torch.empty_like(o1)
+    for t in range(T):
+        ot = torch.empty((B, Hq, D), dtype=torch.bfloat16, device=dev)
+        native.gemma_attn_decode(q[:, t].contiguous(), kn[:, t].contiguous(),
+                                 None if keqv else vn[:, t].contiguous(), kc2, None if keqv else vc2,
+                                 seq_lens=torch.tensor([L - T + t + 1 for L in lens], dtype=torch.int32, device=dev),
+                                 max_seq_len=max(lens), out=ot, **kw)
+        o2[:, t] = ot
+    assert native.gemma_attn_sync_status() == 0, native.gemma_last_error()
+    assert torch.equal(o1.view(torch.int16), o2.view(torch.int16))
+    assert torch.equal(kc.buf, kc2.buf) and torch.equal(vc.buf, vc2.buf)
+
+
+def test_multi_int8_local_matches_prefill_route(oracle):
+    """An int8 local layer goes through the chunked prefill: bit-identical
+    to gemma_attn_prefill after seq_lens - T cached tokens."""
+    dev = torch.device("cuda")
+    B, T, Hq, Hkv, D, W, lens = 2, 4, 32, 16, 256, 1024, [1500, 300]
+    g = synth.generator(333, "cuda")
+    kc = synth.fill_int8_cache_(native.Int8KVCache(B, Hkv, W, D, dev), g)
+    vc = synth.fill_int8_cache_(native.Int8KVCache(B, Hkv, W, D, dev), g)
+    kc2, vc2 = native.Int8KVCache(B, Hkv, W, D, dev), native.Int8KVCache(B, Hkv, W, D, dev)
     kc2.buf.copy_(kc.buf)
     vc2.buf.copy_(vc.buf)
     q = synth.randn_bf16((B, T, Hq, D), g, "cuda")
     kn = synth.randn_bf16((B, T, Hkv, D), g, "cuda")
     vn = synth.randn_bf16((B, T, Hkv, D), g, "cuda")
-    sl = torch.tensor(lens, dtype=torch.int32, device=dev)
-    before = torch.tensor([L - T for L in lens], dtype=torch.int32, device=dev)
-    kw = dict(rope_frac=0.25, rope_theta=1e6, scale=1.0 / math.sqrt(D))
+    kw = dict(window=W, rope_frac=1.0, rope_theta=1e4, scale=1.0 / math.sqrt(D))
     o1 = torch.empty((B, T, Hq, D), dtype=torch.bfloat16, device=dev)
     o2 = torch.empty_like(o1)
-    native.gemma_attn_decode_multi(q, kn, vn, kc, vc, seq_lens=sl, max_seq_len=max(lens), window=0, out=o1, **kw)
-    native.gemma_attn_prefill(q, kn, vn, kc2, vc2, window=0, out=o2, seq_lens_before=before, **kw)
+    native.gemma_attn_decode_multi(q, kn, vn, kc, vc, max_seq_len=max(lens), out=o1,
+                                   seq_lens=torch.tensor(lens, dtype=torch.int32, device=dev), **kw)
+    native.gemma_attn_prefill(q, kn, vn, kc2, vc2, out=o2,
+                              seq_lens_before=torch.tensor([L - T for L in lens], dtype=torch.int32, device=dev), **kw)
     assert native.gemma_attn_sync_status() == 0, native.gemma_last_error()
     assert torch.equal(o1.view(torch.int16), o2.view(torch.int16))
     assert torch.equal(kc.buf, kc2.buf) and torch.equal(vc.buf, vc2.buf)
