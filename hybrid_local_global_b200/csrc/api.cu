@@ -990,6 +990,9 @@ static int multi_impl(const void* q, const void* k_new, const void* v_new, void*
   va.n_splits = n_splits;
   va.part_o = reinterpret_cast<float*>(ws + off_o);
   va.part_lse = reinterpret_cast<float*>(ws + off_lse);
+  // a single split (a local ring that B x Hkv CTAs cover) writes the output itself
+  const bool direct = n_splits == 1 && verify_tc_rows(n_q_heads, n_kv_heads, tokens, head_dim) != 0;
+  va.out = direct ? static_cast<bf16*>(out) : nullptr;
   va.status = status;
   va.wait_ns = (unsigned long long)g_wait_ns.load();
   {
@@ -1007,6 +1010,7 @@ static int multi_impl(const void* q, const void* k_new, const void* v_new, void*
     p_app2.done();
     if (e != cudaSuccess) return cuda_fail(e, "decode append launch");
   }
+  if (direct) return succeed();
 
   DecodeAttnArgs da{};
   da.tokens = tokens;

@@ -195,6 +195,8 @@ struct VerifyAttnArgs {
   int chunk, n_splits;      // keys per split (a multiple of 128), splits planned
   float* part_o;            // [B][tokens][Hq][n_splits][D]
   float* part_lse;          // [B][tokens][Hq][n_splits] (log2 domain)
+  bf16* out;                // transposed kernel, one split: the output [B][tokens][Hq][D]
+                            // written directly (no partials); else null
   int* status;
   unsigned long long wait_ns;
 };

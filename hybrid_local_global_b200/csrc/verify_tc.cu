@@ -71,8 +71,14 @@ struct VCtl {
   int q_issued, q_consumed;
 };
 
-template <int D, int NQ>
+// CTAS: resident CTAs per SM. A local layer's CTA streams one ring (about 1
+// MB at the 31B shape), so its prologue and epilogue weigh; two per SM with
+// a 2-stage ring overlap them (measured on the 31B-shaped B64 block, k = 4:
+// 208 -> 191 us per local layer). Global CTAs keep one per SM and the
+// deepest ring.
+template <int D, int NQ, bool LOCAL = false>
 struct VCfg {
+  static constexpr int CTAS = (LOCAL && D == 256 && NQ == 32) ? 2 : 1;
   static constexpr int MT = D / 128;     // K stages per tile = O^T blocks = V stages per tile
   static constexpr int Q_CH = NQ * 128;  // 64 dims of the NQ query rows
   static constexpr int Q_B = (D / 64) * Q_CH;
@@ -80,7 +86,7 @@ struct VCfg {
   static constexpr int P_BUF = 2 * P_CH;
   static constexpr int RED_B = 6 * NQ * 4;  // red [4][NQ], running maxima [NQ], factors [NQ]
   static constexpr int FIXED = ALIGN_B + Q_B + 2 * P_BUF + RED_B + (int)sizeof(VCtl<8>);
-  static constexpr int NS_FIT = (SMEM_MAX - FIXED) / STAGE_B;
+  static constexpr int NS_FIT = ((CTAS == 1 ? SMEM_MAX : 228 * 1024 / CTAS - 1024) - FIXED) / STAGE_B;
   static constexpr int NSTAGE = NS_FIT > 8 ? 8 : NS_FIT;
   static constexpr int SMEM = ALIGN_B + NSTAGE * STAGE_B + Q_B + 2 * P_BUF + RED_B + (int)sizeof(VCtl<NSTAGE>);
   static constexpr uint32_t COL_O = 0;
@@ -90,11 +96,12 @@ struct VCfg {
   static constexpr uint32_t IDESC_ST = tc::idesc_bf16_f32(128, NQ, 0, 0);  // K (K-major) x Q (K-major)
   static constexpr uint32_t IDESC_OT = tc::idesc_bf16_f32(128, NQ, 1, 0);  // V^T (MN-major) x P^T (K-major)
   static_assert(COLS <= 512, "TMEM plan");
-  static_assert(NSTAGE >= 3 && SMEM <= SMEM_MAX, "shared memory plan");
+  static_assert(NSTAGE >= (CTAS == 1 ? 3 : 2) && SMEM <= SMEM_MAX, "shared memory plan");
 };
 
 struct VArgs {
   int Hq, Hkv, tokens, chunk, n_splits;
+  bf16* out;  // one split: O / l straight into [B][tokens][Hq][D] (no partials, no combine); else null
   int window;  // LOCAL: ring slots
   int64_t key_cap;
   const int32_t* page_table;  // global layers on a paged pool (see VerifyAttnArgs); else null
@@ -154,11 +161,11 @@ __device__ __forceinline__ float reduce_columns(float (&x)[32], int lane) {
 // split also a tail tile of the new tokens' keys and values (tm_kt / tm_vt,
 // [B][tokens][Hkv][D]). Every split writes a partial.
 template <int D, int NQ, bool LOCAL>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(192, VCfg<D, NQ, LOCAL>::CTAS)
     k_verify_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_kt,
                 const __grid_constant__ CUtensorMap tm_vt, const VArgs a) {
-  using C = VCfg<D, NQ>;
+  using C = VCfg<D, NQ, LOCAL>;
   constexpr int NSTAGE = C::NSTAGE;
   constexpr int MT = C::MT;
   extern __shared__ unsigned char sm_raw[];
@@ -185,7 +192,14 @@ __global__ void __launch_bounds__(192, 1)
   const int64_t pos0 = n_keys - a.tokens;
   const int64_t k_begin = (int64_t)split * a.chunk;
   const int64_t k_stop = LOCAL ? (int64_t)a.window : n_keys;
-  if (pos0 < 0 || (!LOCAL && n_keys > a.key_cap) || k_begin >= k_stop) return;  // checked by the append kernel
+  if (pos0 < 0 || (!LOCAL && n_keys > a.key_cap) || k_begin >= k_stop) {  // checked by the append kernel
+    if (a.out && pos0 < 0)  // no combine will zero these rows
+      for (int i = threadIdx.x; i < nvalid * D; i += blockDim.x) {
+        const int n = i / D;
+        a.out[(((int64_t)b * a.tokens + n / G) * a.Hq + g * G + n % G) * D + i % D] = __float2bfloat16_rn(0.f);
+      }
+    return;
+  }
   const int64_t k_end = k_begin + a.chunk < k_stop ? k_begin + a.chunk : k_stop;
   const int n_ring = (int)((k_end - k_begin + BN - 1) / BN);
   const int n_tiles = n_ring + ((LOCAL && split == a.n_splits - 1) ? 1 : 0);  // LOCAL: + the tail tile
@@ -528,7 +542,7 @@ __global__ void __launch_bounds__(192, 1)
       if (kl < NQ) {
         const float L = (red[kl] + red[NQ + kl]) + (red[2 * NQ + kl] + red[3 * NQ + kl]);
         f_s[kl] = L > 0.f ? 1.f / L : 0.f;
-        if (kl < nvalid) {
+        if (kl < nvalid && !a.out) {
           const int64_t pr = ((row0 + kl / G) * a.Hq + g * G + kl % G) * a.n_splits + split;
           a.part_lse[pr] = L > 0.f ? m_s[kl] + __log2f(L) : -INFINITY;
         }
@@ -546,8 +560,11 @@ __global__ void __launch_bounds__(192, 1)
           for (int e = 0; e < 32; ++e) {
             const int n = c * 32 + e;
             if (n < nvalid) {
-              const int64_t pr = ((row0 + n / G) * a.Hq + g * G + n % G) * a.n_splits + split;
-              a.part_o[pr * D + m * 128 + kl] = __uint_as_float(o[e]) * f_s[n];
+              const int64_t hr = (row0 + n / G) * a.Hq + g * G + n % G;  // output row
+              if (a.out)
+                a.out[hr * D + m * 128 + kl] = __float2bfloat16_rn(__uint_as_float(o[e]) * f_s[n]);
+              else
+                a.part_o[(hr * a.n_splits + split) * D + m * 128 + kl] = __uint_as_float(o[e]) * f_s[n];
             }
           }
         }
@@ -574,7 +591,7 @@ __global__ void __launch_bounds__(192, 1)
 
 template <int D, int NQ, bool LOCAL>
 cudaError_t launch_as(const CUtensorMap (&m)[5], const VArgs& v, int B, cudaStream_t st) {
-  using C = VCfg<D, NQ>;
+  using C = VCfg<D, NQ, LOCAL>;
   cudaError_t e =
       cudaFuncSetAttribute(k_verify_tc<D, NQ, LOCAL>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
@@ -635,6 +652,7 @@ cudaError_t launch_verify_attn_tc(const VerifyAttnArgs& a, int B, int D, cudaStr
     maps[4] = mv;
   }
   VArgs v{};
+  v.out = a.out;
   v.window = a.window;
   v.page_table = a.page_table;
   v.page_size = a.page_size;
