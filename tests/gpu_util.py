@@ -8,7 +8,7 @@ import torch
 
 from hybrid_local_global_b200 import synth
 
-# Spec tolerance for bf16 outputs against the fp64 oracle.
+# Parity tolerance for bf16 outputs against the fp64 oracle.
 MAX_ABS = 2e-2
 MEAN_ABS = 2e-3
 
@@ -120,7 +120,7 @@ def rounding_bound(model: np.ndarray, v_absmax: float) -> float:
 
 def assert_close_to_model(gpu, model, exact, v_absmax, what=""):
     """GPU output against the exact attention of its rounded operands within
-    the rounding bound above (mean-abs within the benchmark spec's 2e-3), and
+    the rounding bound above (mean-abs within the parity tolerance 2e-3), and
     against the exact oracle within the model's own error plus that bound
     (the triangle inequality)."""
     tol = rounding_bound(model, v_absmax)

@@ -225,7 +225,7 @@ def test_multi_int8_local_matches_prefill_route(oracle):
 
 def test_multi_equals_consecutive_decodes(oracle):
     """T tokens in one call against T single-token decode calls on a copy of
-    the cache: the same rows within the benchmark spec's tolerance (the two paths
+    the cache: the same rows within the parity tolerance (the two paths
     round the query scaling differently), and the same cache bytes."""
     dev = torch.device("cuda")
     B, T, Hq, Hkv, D, lens = 3, 4, 32, 4, 512, [2000, 37, 4100]

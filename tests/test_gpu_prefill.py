@@ -202,7 +202,7 @@ def test_prefill_peaky(oracle, monkeypatch, kernel, D, W, Hkv, frac, theta):
     rounded the same way, with RoPE off) within the bound its own bf16
     roundings of P and of the output allow, and to the exact oracle within
     that model's error plus the same bound (the triangle inequality): no
-    fixed multiple of the benchmark spec's tolerance."""
+    fixed multiple of the parity tolerance."""
     monkeypatch.setenv("GEMMA_PREFILL_KERNEL", kernel)
     B, S, Hq, seed = 1, 640, 8, 7
     out = run_prefill_case(oracle, B=B, S=S, Hq=Hq, Hkv=Hkv, D=D, W=W, frac=frac, theta=theta, seed=seed,
@@ -216,7 +216,7 @@ def test_prefill_peaky(oracle, monkeypatch, kernel, D, W, Hkv, frac, theta):
 
 def assert_matches_rounded_model(oracle, out, q, k, v, W, frac, theta, what):
     """GPU output against the exact attention of the operands rounded as the
-    prefill kernels round them (spec tolerance), and against the exact
+    prefill kernels round them (parity tolerance), and against the exact
     oracle within that model's error plus the tolerance."""
     B, S, Hq, D = q.shape
     scale = 1.0 / math.sqrt(D)
