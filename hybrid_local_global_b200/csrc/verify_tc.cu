@@ -1,9 +1,10 @@
-// verify_tc.cu -- multi-token decode on a global layer with the tensor
-// cores: `tokens` new tokens per sequence (a drafter's proposals that the
-// target model checks in one pass, "Gemma 4: End-to-End Architecture
-// Walkthrough", Phase 4; "Gemma 4: Architecture, Training and Local
-// Deployment", 3.4), each attending to every cached key and to the earlier
-// new tokens ("Gemma 4: End-to-End Architecture Walkthrough", 3a/3b).
+// verify_tc.cu -- multi-token decode with the tensor cores: `tokens` new
+// tokens per sequence (a drafter's proposals that the target model checks
+// in one pass, "Gemma 4: End-to-End Architecture Walkthrough", Phase 4;
+// "Gemma 4: Architecture, Training and Local Deployment", 3.4), each
+// attending to the cached keys it sees and to the earlier new tokens: all
+// of them on a global layer, the window before its own position on a local
+// one ("Gemma 4: End-to-End Architecture Walkthrough", 3a/3b).
 //
 // Decode-shaped: few query rows (G q heads x tokens <= 64 per KV head)
 // against many keys, so the product is taken transposed. Per tile of 128
@@ -30,7 +31,11 @@
 //               and the partial sums are rescaled. Each thread keeps partial
 //               column sums of its keys; they are reduced once at the end.
 // Output: per query row, the split's normalised O and log2-sum-exp in the
-// same layout as single-token decode, merged by launch_decode_combine.
+// same layout as single-token decode, merged by launch_decode_combine; with
+// a single split the normalised O goes straight to the bf16 output.
+// Local layers (LOCAL) read their ring as it was before the new tokens plus
+// a tail tile of the new rows (see k_verify_tc); global layers may sit in a
+// paged pool (a tile's page from the page table).
 //
 // Every wait is bounded (%globaltimer deadline): a timeout raises the
 // CTA's abort flag and records GEMMA_ERR_DEVICE_TIMEOUT; copies in flight

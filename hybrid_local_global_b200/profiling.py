@@ -44,12 +44,22 @@ KERNEL_SOURCES = {
 }
 
 
+def _code_only(text: str) -> str:
+    """Source text without comments and blank lines (string literals in
+    these sources hold no comment markers), so that a record outlives an
+    edit of comments only."""
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", "", text)
+    return "\n".join(line.rstrip() for line in text.splitlines() if line.strip())
+
+
 def kernel_digest(kernel: str) -> str:
-    """First 16 hex digits of sha256 over the kernel's source files, in order."""
+    """First 16 hex digits of sha256 over the code (comments and blank lines
+    removed) of the kernel's source files, in order."""
     h = hashlib.sha256()
     for f in KERNEL_SOURCES[kernel]:
-        with open(os.path.join(CSRC, f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(CSRC, f), encoding="utf-8") as fh:
+            h.update(_code_only(fh.read()).encode())
     return h.hexdigest()[:16]
 
 
