@@ -995,6 +995,7 @@ static int multi_impl(const void* q, const void* k_new, const void* v_new, void*
   va.out = direct ? static_cast<bf16*>(out) : nullptr;
   va.status = status;
   va.wait_ns = (unsigned long long)g_wait_ns.load();
+  va.drop_first_copy = verify_tc_rows(n_q_heads, n_kv_heads, tokens, head_dim) ? g_drop_next.exchange(0) : 0;
   {
     ProfScope p_split(GEMMA_KERNEL_DECODE_SPLIT, st);
     e = launch_verify_attn_tc(va, batch, head_dim, st);

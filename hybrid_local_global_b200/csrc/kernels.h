@@ -199,6 +199,7 @@ struct VerifyAttnArgs {
                             // written directly (no partials); else null
   int* status;
   unsigned long long wait_ns;
+  int drop_first_copy;      // test hook (transposed kernel): skip the first K copy of unit 0
 };
 cudaError_t launch_verify_attn_tc(const VerifyAttnArgs& a, int B, int D, cudaStream_t st);
 cudaError_t launch_verify_attn_rows(const VerifyAttnArgs& a, int B, int D, cudaStream_t st);

@@ -116,6 +116,7 @@ struct VArgs {
   float* part_lse;
   int* status;
   unsigned long long wait_ns;
+  int drop_first_copy;  // test hook: the first K stage of unit (0, 0, 0) is never issued
 };
 
 __device__ __forceinline__ bool wait_all(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
@@ -295,6 +296,7 @@ __global__ void __launch_bounds__(192, VCfg<D, NQ, LOCAL>::CTAS)
               ok = false;
               break;
             }
+            if (a.drop_first_copy && item == 0 && split == 0 && g == 0 && b == 0) continue;
             const uint32_t dst = sStage + s * STAGE_B;
             const uint32_t bar = smem_u32(&ctl->full[s]);
             mbar_arrive_expect_tx(&ctl->full[s], STAGE_B);
@@ -674,6 +676,7 @@ cudaError_t launch_verify_attn_tc(const VerifyAttnArgs& a, int B, int D, cudaStr
   v.part_lse = a.part_lse;
   v.status = a.status;
   v.wait_ns = a.wait_ns;
+  v.drop_first_copy = a.drop_first_copy;
   if (D == 256) return NQ == 32 ? launch_nq<256, 32>(maps, v, B, st) : launch_nq<256, 64>(maps, v, B, st);
   return NQ == 32 ? launch_nq<512, 32>(maps, v, B, st) : launch_nq<512, 64>(maps, v, B, st);
 }

@@ -407,7 +407,8 @@ const char* gemma_last_error(void);
 int gemma_attn_set_wait_limit(long long max_ns);
 
 /* Test hook for the same path: when `enable` is nonzero, the next
- * gemma_attn_decode launch does not issue the first key/value copy of its
+ * gemma_attn_decode launch (or gemma_attn_decode_multi launch of the
+ * tensor-core kernel) does not issue the first key/value copy of its
  * first work unit, so that unit's consumers wait on a barrier nothing will
  * complete; their bounded wait runs out, the unit exits without output and
  * gemma_attn_sync_status reports GEMMA_ERR_DEVICE_TIMEOUT. Nothing faults or

@@ -20,7 +20,9 @@ pytestmark = pytest.mark.gpu
 
 
 def run_multi_case(oracle, *, lens, T, Hq, Hkv, D, W, frac, theta, seed, shared=False, keqv=False,
-                   cap_extra=16):
+                   cap_extra=16, expect_status=False):
+    """expect_status: the call is expected to report GEMMA_ERR_DEVICE_TIMEOUT
+    (a test hook dropped a copy); only that is checked."""
     dev = torch.device("cuda")
     B = len(lens)
     g = synth.generator(seed)
@@ -64,6 +66,9 @@ def run_multi_case(oracle, *, lens, T, Hq, Hkv, D, W, frac, theta, seed, shared=
                                    None if (shared or keqv) else vn.to(dev), kcd, None if keqv else vcd,
                                    seq_lens=sl, max_seq_len=max_len, window=W, rope_frac=frac,
                                    rope_theta=theta, scale=scale, out=out, flags=flags)
+    if expect_status:
+        assert native.gemma_attn_sync_status() == native.GEMMA_ERR_DEVICE_TIMEOUT
+        return out
     assert native.gemma_attn_sync_status() == 0, native.gemma_last_error()
     before = [L - T for L in lens]
     ref, _ = oracle.attention(to_bits(q), to_bits(k_log), None if keqv else to_bits(v_log), q_pos0=before,
@@ -372,3 +377,20 @@ def test_multi_paged_equals_contiguous(T):
             assert torch.equal(kp1[pg].view(torch.int16), kc1[b, :, p * ps:(p + 1) * ps].view(torch.int16))
             assert torch.equal(vp1[pg].view(torch.int16), vc1[b, :, p * ps:(p + 1) * ps].view(torch.int16))
     assert (kp1[~owned] == SENTINEL).all() and (vp1[~owned] == SENTINEL).all()
+
+
+@pytest.mark.parametrize("W", [0, 64], ids=["global", "local"])
+def test_multi_bounded_wait_times_out_and_context_survives(oracle, W):
+    """The tensor-core kernel's first copy is not issued (test hook): the
+    MMA warp's bounded wait gives up, the softmax warps leave together, the
+    status says GEMMA_ERR_DEVICE_TIMEOUT, and the next call on the same
+    context is correct."""
+    native.gemma_attn_set_wait_limit(20_000_000)  # 20 ms
+    try:
+        native.gemma_attn_debug_drop_next_copy(True)
+        run_multi_case(oracle, lens=[700, 300], T=4, Hq=8, Hkv=1 if W == 0 else 4, D=512 if W == 0 else 256, W=W,
+                       frac=0.25 if W == 0 else 1.0, theta=1e6 if W == 0 else 1e4, seed=371, expect_status=True)
+    finally:
+        native.gemma_attn_set_wait_limit(0)
+    run_multi_case(oracle, lens=[700, 300], T=4, Hq=8, Hkv=1 if W == 0 else 4, D=512 if W == 0 else 256, W=W,
+                   frac=0.25 if W == 0 else 1.0, theta=1e6 if W == 0 else 1e4, seed=372)
