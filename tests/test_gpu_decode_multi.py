@@ -394,3 +394,61 @@ def test_multi_bounded_wait_times_out_and_context_survives(oracle, W):
         native.gemma_attn_set_wait_limit(0)
     run_multi_case(oracle, lens=[700, 300], T=4, Hq=8, Hkv=1 if W == 0 else 4, D=512 if W == 0 else 256, W=W,
                    frac=0.25 if W == 0 else 1.0, theta=1e6 if W == 0 else 1e4, seed=372)
+
+
+def test_multi_31b_b64_k4_sampled(oracle):
+    """The benchmarked multi-token block at full size (B64, KV lengths
+    U[4096,131072], 4 new tokens, 5 local + 1 global layer), as bench.py
+    runs it: sampled sequences (the shortest, the longest and two seeded
+    others; rows are independent) of every layer against the oracle over the
+    cache as it was plus the new tokens."""
+    from hybrid_local_global_b200.workloads import WORKLOADS
+    w = WORKLOADS["31b_verify_b64_k4"]
+    T = w.tokens
+    dev = torch.device("cuda")
+    st = AttentionStack(w, dev)
+    lens_cpu = synth.decode_lengths(w.batch, w.len_lo, w.len_hi, seed=w.seed)
+    lens = lens_cpu.to(dev)
+    max_len = int(lens_cpu.max())
+    g = synth.generator(w.seed, "cuda")
+    for l in range(st.n_layers):
+        synth.fill_randn_bf16_(st.k_cache[l], g)
+        synth.fill_randn_bf16_(st.v_cache[l], g)
+    ws = torch.empty(st.decode_multi_workspace_bytes(T, max_len), dtype=torch.uint8, device=dev)
+    rng = np.random.default_rng(w.seed)
+    pick = set(rng.choice(w.batch, size=2, replace=False).tolist())
+    pick |= {int(lens_cpu.argmin()), int(lens_cpu.argmax())}
+    for l in range(st.n_layers):
+        t = st.layer_type(l)
+        D, Hkv, W = t.head_dim, t.n_kv_heads, t.window
+        q = synth.randn_bf16((w.batch, T, w.n_q_heads, D), g, "cuda")
+        kn = synth.randn_bf16((w.batch, T, Hkv, D), g, "cuda")
+        vn = synth.randn_bf16((w.batch, T, Hkv, D), g, "cuda")
+        snaps = {}
+        for b in pick:
+            n = int(lens_cpu[b]) - T  # cached positions before the new tokens
+            if W:
+                first = max(0, n - W)
+                slots = torch.tensor([p % W for p in range(first, n)], dtype=torch.long, device=dev)
+                snaps[b] = (first, st.k_cache[l][b].index_select(1, slots).cpu(),
+                            st.v_cache[l][b].index_select(1, slots).cpu())
+            else:
+                snaps[b] = (0, st.k_cache[l][b, :, :n].cpu(), st.v_cache[l][b, :, :n].cpu())
+        out = torch.empty_like(q)
+        st.decode_multi_layer(l, q, kn, vn, out, seq_lens=lens, max_seq_len=max_len, workspace=ws)
+        assert native.gemma_attn_sync_status() == 0, native.gemma_last_error()
+        for b in sorted(pick):
+            L = int(lens_cpu[b])
+            first, kc_b, vc_b = snaps[b]
+            k_log = torch.zeros((1, L, Hkv, D), dtype=torch.bfloat16)
+            v_log = torch.zeros_like(k_log)
+            k_log[0, first:L - T] = kc_b.transpose(0, 1)
+            v_log[0, first:L - T] = vc_b.transpose(0, 1)
+            k_log[0, L - T:] = kn[b].cpu()
+            v_log[0, L - T:] = vn[b].cpu()
+            ref, _ = oracle.attention(to_bits(q[b:b + 1].cpu()), to_bits(k_log), to_bits(v_log), q_pos0=L - T,
+                                      n_keys=L, rot_from=L - T, window=W, rope_frac=t.rope_frac,
+                                      theta=t.rope_theta, scale=t.scale)
+            got = out[b:b + 1].float().cpu().double().numpy().transpose(0, 2, 1, 3).reshape(-1, D)
+            assert_close(got, ref, what="31b_verify_b64_k4 layer %d b=%d L=%d" % (l, b, L))
+        del snaps
