@@ -408,3 +408,25 @@ def test_k_equals_v_worked_example_and_cached_keys(oracle):
     c, _ = oracle.attention(q, k, None, rot_from=T, rope_frac=1.0, **kw)
     d, _ = oracle.attention(q, k, k, rot_from=T, rope_frac=1.0, **kw)
     np.testing.assert_array_equal(c, d)
+
+
+@pytest.mark.parametrize("window", [0, 6])
+def test_new_token_chunk_equals_one_token_steps(oracle, window):
+    """Multi-token decode (the target's pass over a drafter's proposals): T
+    new tokens after L - T cached ones, each seeing the cache and the earlier
+    new tokens (window-limited on a local layer), give row for row what T
+    single-token steps at lengths L - T + 1 .. L give."""
+    B, T, L, Hq, Hkv, D = 1, 4, 19, 4, 2, 16
+    q = rand_bits((B, T, Hq, D), 71)
+    k = rand_bits((B, L, Hkv, D), 72)
+    v = rand_bits((B, L, Hkv, D), 73)
+    kw = dict(rot_from=L - T, window=window, rope_frac=0.25, theta=1e6, scale=0.3)
+    chunk, lse = oracle.attention(q, k, v, q_pos0=L - T, n_keys=L, **kw)
+    chunk = chunk.reshape(B, Hq, T, D)
+    lse = lse.reshape(B, Hq, T)
+    for t in range(T):
+        n = L - T + t + 1
+        one, lse1 = oracle.attention(np.ascontiguousarray(q[:, t:t + 1]), np.ascontiguousarray(k[:, :n]),
+                                     np.ascontiguousarray(v[:, :n]), q_pos0=n - 1, n_keys=n, **kw)
+        np.testing.assert_allclose(chunk[:, :, t].reshape(-1, D), one, rtol=0, atol=1e-13)
+        np.testing.assert_allclose(lse[:, :, t].reshape(-1), lse1, rtol=0, atol=1e-13)
