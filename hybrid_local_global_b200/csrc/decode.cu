@@ -63,7 +63,7 @@ struct DecCfg {
   static constexpr int GROUPB = RPC * D * 2 + 16;  // RPC consecutive K (or V) rows + 16 B pad
   static constexpr int GPR = KB / RPC;             // row groups per 16-row region
   static constexpr int SLOT_B = 2 * GPR * GROUPB;  // K region then V region (two K regions under K = V)
-  static constexpr int NSLOT = (D == 256) ? 6 : 3;
+  static constexpr int NSLOT = 3;  // head_dim 256: with four CTAs per SM (see the launch bounds)
   static_assert(NSLOT % NCW == 0, "each ring slot needs a single consumer warp");
   static constexpr int RING_B = NSLOT * SLOT_B;
   static constexpr int Q_B = 8 * ROWB;
@@ -95,8 +95,12 @@ __device__ __forceinline__ int key_of(int n) {
 
 // PAGED: the cache is a pool named by a.page_table (see cache_row); the
 // contiguous instance keeps the plain row arithmetic of one (b, g) range.
+// Head_dim 256 (local layers) runs four CTAs per SM with a 3-slot ring: the
+// short ring splits are latency-bound, and the extra resident warps pay
+// (measured on the 31B-shaped B64 block: its five local layers ~10 % faster
+// than two CTAs with a 6-slot ring). Head_dim 512 keeps two.
 template <int D, int RPC, bool PAGED>
-__global__ void __launch_bounds__(32 * (NCW + 1), 2) k_decode_split(DecodeAttnArgs a) {
+__global__ void __launch_bounds__(32 * (NCW + 1), D == 256 ? 4 : 2) k_decode_split(DecodeAttnArgs a) {
   using C = DecCfg<D, RPC>;
   extern __shared__ __align__(128) unsigned char sm[];
   unsigned char* ring = sm;
