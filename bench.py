@@ -62,6 +62,9 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 HEADLINE = "31b_block_s32768"
 EXTRA_PREFILL = "local_s1024,e2b_block_s8192,global_chunk_256k"
 EXTRA_DECODE = "global_decode_256k"
+# nominal per-GPU figures, for the second fraction each roofline object reports
+NOMINAL_BF16_TFLOPS = 2250.0   # dense bf16 (the 2:4-sparse figure halved)
+NOMINAL_HBM_GBS = 7700.0       # HBM3e, HGX B200
 
 
 def load_peaks():
@@ -278,6 +281,7 @@ def bench_prefill(args, w, dev, world, peaks, e2e=False, cpu=False):
     burst = peaks[0]["bf16_tflops"]
     roof = {"bound": "tensor", "kernel": "prefill attention", "achieved": round(achieved, 2),
             "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4), "peak_source": peak_source,
+            "frac_of_nominal": round(achieved / NOMINAL_BF16_TFLOPS, 4),
             "frac_of_burst": round(achieved / burst, 4), "traffic": None,
             "per_launch": "algorithmic FLOPs of all attention launches / their summed device time "
                           "(%d launches, %d per step; CUDA events around each launch, in a second timed "
@@ -580,6 +584,7 @@ def bench_decode(args, w, dev, world, peaks, cpu=False):
     peak = peaks[0]["hbm_gbs"]
     roof = {"bound": "hbm", "kernel": "split-K decode attention", "achieved": round(achieved, 1),
             "peak": peak, "unit": "GB/s", "frac": round(achieved / peak, 4),
+            "frac_of_nominal": round(achieved / NOMINAL_HBM_GBS, 4),
             "peak_source": "%s HBM copy (MEASURED_PEAKS.json)" % peaks[1], "traffic": None,
             "per_launch": "visible K (and V unless K = V) bytes of all split launches / their summed device time "
                           "(%d launches, %d per step; CUDA events around each launch, in a second timed pass "
@@ -730,6 +735,7 @@ def bench_verify(args, w, dev, world, peaks, cpu=False):
     peak = peaks[0]["hbm_gbs"]
     roof = {"bound": "hbm", "kernel": "multi-token decode attention (transposed tensor-core kernel)",
             "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s", "frac": round(achieved / peak, 4),
+            "frac_of_nominal": round(achieved / NOMINAL_HBM_GBS, 4),
             "peak_source": "%s HBM copy (MEASURED_PEAKS.json)" % peaks[1], "traffic": None,
             "per_launch": "K (and V unless K = V) bytes of all attention launches / their summed device time "
                           "(%d launches, %d per step; CUDA events around each launch, in a second timed pass "
