@@ -856,8 +856,9 @@ static int multi_impl(const void* q, const void* k_new, const void* v_new, void*
                       const CacheLayout& L) {
   int rc = check_heads(n_q_heads, n_kv_heads, head_dim, window, rope_frac, rope_theta, scale);
   if (rc) return rc;
-  if (batch <= 0 || tokens <= 0 || max_seq_len <= 0)
-    return fail(GEMMA_ERR_INVALID_ARG, "batch %d, tokens %d, max_seq_len %d", batch, tokens, max_seq_len);
+  if (batch <= 0 || tokens <= 0 || max_seq_len <= 0 || tokens > max_seq_len)
+    return fail(GEMMA_ERR_INVALID_ARG, "batch %d, tokens %d, max_seq_len %d (tokens <= max_seq_len)", batch, tokens,
+                max_seq_len);
   if (!seq_lens) return fail(GEMMA_ERR_INVALID_ARG, "null seq_lens");
   if (window == 0 && cache_cap < max_seq_len)
     return fail(GEMMA_ERR_CAPACITY, "global layer: cache_cap %d < max_seq_len %d", cache_cap, max_seq_len);

@@ -207,6 +207,7 @@ def _multi_raw(**over):
 @pytest.mark.parametrize("over,code", [
     (dict(), E.GEMMA_ERR_CAPACITY),                                   # the tensor-core path: accepted
     (dict(T=0), E.GEMMA_ERR_INVALID_ARG),
+    (dict(T=5000, wsb=1 << 30), E.GEMMA_ERR_INVALID_ARG),             # more new tokens than any length allows
     (dict(lens=None), E.GEMMA_ERR_INVALID_ARG),
     (dict(maxlen=0), E.GEMMA_ERR_INVALID_ARG),
     (dict(cap=1000), E.GEMMA_ERR_CAPACITY),                           # global cache < max length
