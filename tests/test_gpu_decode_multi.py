@@ -333,18 +333,19 @@ def test_multi_stack_31b_block(oracle):
 SENTINEL = -7.5  # bf16-exact fill of pool rows no sequence owns
 
 
-@pytest.mark.parametrize("T", [4, 8, 16], ids=["rows32", "rows64", "rows128"])
-def test_multi_paged_equals_contiguous(T):
+@pytest.mark.parametrize("T,keqv", [(4, False), (8, False), (16, False), (4, True)],
+                         ids=["rows32", "rows64", "rows128", "keqv"])
+def test_multi_paged_equals_contiguous(T, keqv):
     """A paged global cache (random page order, spare pages) gives the
     contiguous path's outputs bit for bit, holds the same rows at the same
     positions, and leaves pages no sequence owns untouched."""
     dev = torch.device("cuda")
     B, Hq, Hkv, D, ps, lens = 3, 32, 4, 512, 256, [2000, 37, 4100]
-    g = synth.generator(360 + T)
+    g = synth.generator(360 + T + keqv)
     pps = (max(lens) + ps - 1) // ps + 1
     n_pages, cap = B * pps + 3, pps * ps
     kc = synth.randn_bf16((B, Hkv, cap, D), g)
-    vc = synth.randn_bf16((B, Hkv, cap, D), g)
+    vc = kc if keqv else synth.randn_bf16((B, Hkv, cap, D), g)
     table = torch.tensor(np.random.default_rng(T).permutation(n_pages)[:B * pps].reshape(B, pps), dtype=torch.int32)
 
     def to_pool(c):
@@ -354,17 +355,20 @@ def test_multi_paged_equals_contiguous(T):
                 pool[int(table[b, p])] = c[b, :, p * ps:(p + 1) * ps]
         return pool
 
-    kp, vp = to_pool(kc).to(dev), to_pool(vc).to(dev)
-    kcd, vcd = kc.to(dev), vc.to(dev)
+    kp = to_pool(kc).to(dev)
+    vp = kp if keqv else to_pool(vc).to(dev)
+    kcd = kc.to(dev)
+    vcd = kcd if keqv else vc.to(dev)
     q = synth.randn_bf16((B, T, Hq, D), g).to(dev)
     kn = synth.randn_bf16((B, T, Hkv, D), g).to(dev)
-    vn = synth.randn_bf16((B, T, Hkv, D), g).to(dev)
+    vn = None if keqv else synth.randn_bf16((B, T, Hkv, D), g).to(dev)
     sl = torch.tensor(lens, dtype=torch.int32, device=dev)
-    kw = dict(seq_lens=sl, max_seq_len=max(lens), rope_frac=0.25, rope_theta=1e6, scale=1.0 / math.sqrt(D))
+    kw = dict(seq_lens=sl, max_seq_len=max(lens), rope_frac=0.25, rope_theta=1e6, scale=1.0 / math.sqrt(D),
+              flags=native.GEMMA_F_KEQV if keqv else 0)
     o1 = torch.empty((B, T, Hq, D), dtype=torch.bfloat16, device=dev)
     o2 = torch.empty_like(o1)
-    native.gemma_attn_decode_multi(q, kn, vn, kcd, vcd, window=0, out=o1, **kw)
-    native.gemma_attn_decode_multi_paged(q, kn, vn, kp, vp, table.to(dev), out=o2, **kw)
+    native.gemma_attn_decode_multi(q, kn, vn, kcd, None if keqv else vcd, window=0, out=o1, **kw)
+    native.gemma_attn_decode_multi_paged(q, kn, vn, kp, None if keqv else vp, table.to(dev), out=o2, **kw)
     assert native.gemma_attn_sync_status() == 0, native.gemma_last_error()
     assert torch.equal(o1.view(torch.int16), o2.view(torch.int16))
     kp1, vp1 = kp.cpu(), vp.cpu()
