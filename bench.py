@@ -32,7 +32,8 @@ the library records events around every launch.
 
 `cpu_baseline` objects time the fp64 CPU oracle on the host cores over a
 bounded, seeded sample of rows (prefill) or sequences (decode) of the same
-workload and inputs. --impl reference times the oracle alone, on the
+workload and inputs, and report in `parity` how far the GPU's outputs of the
+last timed step sit from the oracle's on that sample. --impl reference times the oracle alone, on the
 headline workload, each step a bounded sample of its rows.
 """
 from __future__ import annotations
@@ -390,18 +391,44 @@ def sample_rows(w, n, seed):
                      rng.integers(0, w.seq, n)], axis=1).astype(np.int32)
 
 
+class Parity:
+    """Largest and mean |GPU - oracle| over the outputs a CPU baseline
+    computed anyway, against the parity tolerance of the tests (max 2e-2,
+    mean 2e-3 for bf16 outputs)."""
+
+    def __init__(self):
+        self.mx, self.sum, self.n, self.rows = 0.0, 0.0, 0, 0
+
+    def add(self, gpu, ref):
+        gpu, ref = np.asarray(gpu, dtype=np.float64), np.asarray(ref, dtype=np.float64)
+        err = np.abs(gpu - ref)
+        if not np.isfinite(gpu).all():
+            err = np.full_like(err, np.inf)
+        self.mx = max(self.mx, float(err.max()) if err.size else 0.0)
+        self.sum += float(err.sum())
+        self.n += err.size
+        self.rows += err.size // ref.shape[-1] if err.size else 0
+
+    def summary(self, what):
+        mean = self.sum / max(self.n, 1)
+        return {"max_abs": float("%.4g" % self.mx), "mean_abs": float("%.4g" % mean), "rows": self.rows,
+                "within_tolerance": bool(self.mx <= 2e-2 and mean <= 2e-3), "compared": what}
+
+
 def oracle_prefill_rows(w, t, q, k, v, rows):
     """Times the oracle on `rows` of one layer (q [B,S,Hq,D], k/v [B,T,Hkv,D]
     bf16 bits in position order, the first w.prior keys already rotated);
-    returns (seconds, algorithmic FLOPs of those rows)."""
+    returns (seconds, algorithmic FLOPs of those rows, the rows' outputs
+    [n, D])."""
     import oracle
     t0 = time.perf_counter()
-    oracle.attention(q, k, v, q_pos0=w.prior, n_keys=w.prior + w.seq, rot_from=w.prior,
-                     window=t.window, rope_frac=t.rope_frac, theta=t.rope_theta, scale=t.scale, rows=rows)
+    out, _ = oracle.attention(q, k, v, q_pos0=w.prior, n_keys=w.prior + w.seq, rot_from=w.prior,
+                              window=t.window, rope_frac=t.rope_frac, theta=t.rope_theta, scale=t.scale,
+                              rows=rows)
     secs = time.perf_counter() - t0
     pos = w.prior + rows[:, 2].astype(np.int64)
     vis = np.minimum(pos + 1, t.window) if t.window else pos + 1
-    return secs, int(4 * t.head_dim * vis.sum())
+    return secs, int(4 * t.head_dim * vis.sum()), out
 
 
 def layer_bits_for_oracle(w, st, l, q, k, v):
@@ -421,16 +448,21 @@ def prefill_cpu_baseline(w, is_global, layers, st, flops_budget):
     import oracle
     n_rows = rows_for_budget(w, is_global, flops_budget)
     secs, flops = 0.0, 0
+    par = Parity()
     for l, g in enumerate(is_global):
         t = w.global_ if g else w.local
-        q, k, v, _ = layers[l]
+        q, k, v, out = layers[l]
         qb, kb, vb = layer_bits_for_oracle(w, st, l, q, k, v)
-        s, f = oracle_prefill_rows(w, t, qb, kb, vb, sample_rows(w, n_rows[l], seed=77 + l))
+        rows = sample_rows(w, n_rows[l], seed=77 + l)
+        s, f, ref = oracle_prefill_rows(w, t, qb, kb, vb, rows)
         secs += s
         flops += f
+        idx = torch.as_tensor(rows.astype(np.int64), device=out.device)
+        par.add(out[idx[:, 0], idx[:, 2], idx[:, 1]].double().cpu().numpy(), ref)
     n_all = w.batch * w.n_q_heads * w.seq
     return {"value": round(flops / secs / 1e12, 6), "unit": "TFLOP/s", "cores": oracle.default_threads(),
             "kind": "oracle", "seconds": round(secs, 2),
+            "parity": par.summary("the sampled rows, against the GPU output of the last timed step"),
             "sample": ("every row of every layer" if all(n >= n_all for n in n_rows) else
                        "%s seeded random rows (b, h, i) of the layers [%s] of the same workload and inputs "
                        "(rows are independent, so the rate is the workload's)"
@@ -485,10 +517,11 @@ def decode_cpu_baseline(w, st, layers, lens_cpu, n_random=2):
     seqs = sorted(pick)
     threads = oracle.default_threads()
     secs, nbytes = 0.0, 0
+    par = Parity()
     with cf.ThreadPoolExecutor(max_workers=threads) as ex:
         for l in range(st.n_layers):
             t = st.layer_type(l)
-            q = layers[l][0]
+            q, out = layers[l][0], layers[l][3]
             kc, vc = st.k_cache[l], st.v_cache[l]
             keqv = st.keqv(l)
             G = w.n_q_heads // t.n_kv_heads
@@ -520,13 +553,15 @@ def decode_cpu_baseline(w, st, layers, lens_cpu, n_random=2):
                 t0 = time.perf_counter()
                 futs = [ex.submit(oracle.attend_rows, qrot[h:h + 1], kf[h // G], vf[h // G], 0, n, t.scale)
                         for h in range(w.n_q_heads)]
-                for f in futs:
-                    f.result()
+                ref = np.concatenate([f.result()[0] for f in futs])
                 secs += time.perf_counter() - t0 + deq
+                par.add(out[b].double().cpu().numpy(), ref)
                 del kf, vf
             nbytes += visible_kv_bytes(st, l, lens_cpu, seqs=seqs)
     return {"value": round(nbytes / secs / 1e9, 3), "unit": "GB/s", "cores": threads, "kind": "oracle",
             "seconds": round(secs, 2),
+            "parity": par.summary("every q head of the sampled sequences, against the GPU output of the last "
+                                  "timed step"),
             "sample": "sequences %s (%s) of every layer, all q heads; bytes = their visible K+V cache bytes"
                       % (seqs, "the only one" if len(lens) == 1 else
                          "shortest, longest and %d seeded others" % (len(seqs) - 2))}
@@ -656,10 +691,11 @@ def verify_cpu_baseline(w, st, layers, lens_cpu, n_random=1):
     seqs = sorted(pick)
     threads = oracle.default_threads()
     secs, nbytes = 0.0, 0
+    par = Parity()
     with cf.ThreadPoolExecutor(max_workers=threads) as ex:
         for l in range(st.n_layers):
             t = st.layer_type(l)
-            q = layers[l][0]
+            q, out = layers[l][0], layers[l][3]
             kc, vc = st.k_cache[l], st.v_cache[l]
             keqv = st.keqv(l)
             G = w.n_q_heads // t.n_kv_heads
@@ -676,16 +712,24 @@ def verify_cpu_baseline(w, st, layers, lens_cpu, n_random=1):
                                          for h in range(w.n_q_heads)]) for tok in range(T)])  # [T, Hq, D]
                 lo = np.array([max(0, L - T + tok - t.window + 1 - first) if t.window else 0 for tok in range(T)])
                 hi = np.array([L - T + tok + 1 - first for tok in range(T)])
+                order = [(hk, tok) for hk in range(t.n_kv_heads) for tok in range(T)]
                 futs = [ex.submit(oracle.attend_rows, qr[tok, hk * G:(hk + 1) * G], kf[hk], vf[hk], lo[tok],
                                   hi[tok] - lo[tok], t.scale)
-                        for hk in range(t.n_kv_heads) for tok in range(T)]
-                for f in futs:
-                    f.result()
+                        for hk, tok in order]
+                refs = [f.result()[0] for f in futs]
                 secs += time.perf_counter() - t0
+                gpu_b = out[b].double().cpu().numpy()  # [T, Hq, D]
+                for (hk, tok), ref in zip(order, refs):
+                    # on a local ring an earlier token's oldest keys are overwritten by the step's own tokens
+                    if t.window == 0 or tok == T - 1:
+                        par.add(gpu_b[tok, hk * G:(hk + 1) * G], ref)
                 del kf, vf
             nbytes += verify_kv_bytes(st, l, lens_cpu, T, seqs=seqs)
     return {"value": round(nbytes / secs / 1e9, 3), "unit": "GB/s", "cores": threads, "kind": "oracle",
             "seconds": round(secs, 2),
+            "parity": par.summary("the sampled sequences' outputs whose keys all stay cached after the step "
+                                  "(every token on global layers, the last on local rings), against the GPU "
+                                  "output of the last timed step"),
             "sample": "sequences %s (shortest, longest and %d seeded other) of every layer, all q heads and "
                       "all %d new tokens; bytes = their K+V bytes as counted for the GPU"
                       % (seqs, len(seqs) - 2, T)}
@@ -811,7 +855,7 @@ def run_reference(args, world, rank):
         for i in range(args.warmup):
             oracle_prefill_rows(w, t, qb, kb, vb, sample_rows(w, n, seed=100 * l + i))
         for i in range(args.steps):
-            s, f = oracle_prefill_rows(w, t, qb, kb, vb, sample_rows(w, n, seed=100000 + 100 * l + i))
+            s, f, _ = oracle_prefill_rows(w, t, qb, kb, vb, sample_rows(w, n, seed=100000 + 100 * l + i))
             secs[i] += s
             flops[i] += f
         del qb, kb, vb
