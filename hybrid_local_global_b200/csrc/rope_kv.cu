@@ -118,7 +118,8 @@ __device__ __forceinline__ uint4 ld16_stream(const bf16* p, uint64_t pol) {
 }
 
 constexpr int ROPE_HB = 8;     // head vectors loaded before the first store
-constexpr int ROPE_RPT = 2;    // positions per thread
+constexpr int ROPE_RPT = 2;    // positions per thread, unless that leaves fewer than
+constexpr int ROPE_MIN_CTAS = 512;  // this many CTAs (about 3.5 per SM): then one
 
 // Prefill: rotate the chunk's Q into q_rot (times q_scale), rotate K and write
 // it (global: cache slot pos; local: the k_rot workspace the attention kernel
@@ -129,7 +130,9 @@ constexpr int ROPE_RPT = 2;    // positions per thread
 // fills the cache from k_rot and the caller's V.
 //
 // threadIdx.x owns 8 elements of the head vector, threadIdx.y one position
-// (of ROPE_RPT per thread): the angles of a position are formed once and
+// (of one or ROPE_RPT per thread, as the grid was sized: a CTA covers
+// ceil(S / (gridDim.x * blockDim.y)) rows of blockDim.y positions, so every
+// position has exactly one thread): the angles of a position are formed once and
 // serve all Hq + 2 Hkv head vectors, which are loaded ROPE_HB at a time so
 // several 16-byte loads are in flight per thread.
 // WIN: chunked local prefill, where the chunk's rotated K and its V go to
@@ -147,9 +150,10 @@ __global__ void __launch_bounds__(256, 2) k_prefill_rope(PrefillRopeArgs a) {
   const uint64_t pol = policy_evict_first();
   double inv_freq[4];
   chunk_inv_freq(e0, D, a.n_rot, a.log2_theta, inv_freq);
+  const int rpt = (a.S + gridDim.x * blockDim.y - 1) / (gridDim.x * blockDim.y);
 #pragma unroll 1
-  for (int rep = 0; rep < ROPE_RPT; ++rep) {
-    const int s = (blockIdx.x * ROPE_RPT + rep) * blockDim.y + threadIdx.y;
+  for (int rep = 0; rep < rpt; ++rep) {
+    const int s = (blockIdx.x * rpt + rep) * blockDim.y + threadIdx.y;
     if (s >= a.S) break;
     const int64_t pos = pos0 + s;
     const PairTrig t = chunk_trig(pos, e0, a.n_rot, inv_freq);
@@ -470,7 +474,8 @@ cudaError_t launch_quantize_rows(const QuantRowsArgs& a, int B, int D, cudaStrea
 cudaError_t launch_prefill_rope(const PrefillRopeArgs& a, int B, int D, cudaStream_t st) {
   const int tx = D / 8;
   dim3 block(tx, 256 / tx);
-  const int per_cta = block.y * ROPE_RPT;
+  int per_cta = block.y * ROPE_RPT;
+  if ((int64_t)((a.S + per_cta - 1) / per_cta) * B < ROPE_MIN_CTAS) per_cta = block.y;
   dim3 grid((a.S + per_cta - 1) / per_cta, B);
   const bool win = a.win_rows > 0 && a.v_win;
   if (D == 256) {
