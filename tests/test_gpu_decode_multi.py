@@ -3,7 +3,7 @@ the target model checks a drafter's proposals in speculative decoding)
 against the fp64 oracle, through the C ABI: the tensor-core path of global
 bf16 layers (q heads x tokens packed in one tile, split over the cached
 keys, combined), and the chunked-prefill route of local and int8 layers;
-cache slots written, KV sharing, K = V and the device range check."""
+cache slots written, KV sharing, K = V and the device range check on every route."""
 import math
 
 import numpy as np
@@ -280,6 +280,40 @@ def test_multi_range_check_reports(oracle):
     assert torch.count_nonzero(out[1].float()) == 0
     assert torch.isfinite(out[0].float()).all()
     assert native.gemma_attn_sync_status() == 0  # reading the status clears it
+
+
+@pytest.mark.parametrize("route", ["int8_global", "chunked_prefill"])
+def test_multi_range_check_other_routes(route):
+    """seq_lens below the token count on the two routes that do not run the
+    tensor-core multi-token kernel: the int8 global layer's per-token
+    decodes and the chunked prefill (q heads per KV head x tokens above
+    128). The device check reports GEMMA_ERR_DEVICE_RANGE, and the valid
+    sequence's output is bit-identical to a call where every length is
+    valid."""
+    dev = torch.device("cuda")
+    B, Hq, Hkv, D, cap = 2, 32, 4, 512, 512
+    T = 4 if route == "int8_global" else 17
+    g = synth.generator(353, "cuda")
+    if route == "int8_global":
+        kc = synth.fill_int8_cache_(native.Int8KVCache(B, Hkv, cap, D, dev), g)
+        vc = synth.fill_int8_cache_(native.Int8KVCache(B, Hkv, cap, D, dev), g)
+    else:
+        kc = synth.randn_bf16((B, Hkv, cap, D), g, "cuda")
+        vc = synth.randn_bf16((B, Hkv, cap, D), g, "cuda")
+    q = synth.randn_bf16((B, T, Hq, D), g, "cuda")
+    kn = synth.randn_bf16((B, T, Hkv, D), g, "cuda")
+    vn = synth.randn_bf16((B, T, Hkv, D), g, "cuda")
+    kw = dict(max_seq_len=300, window=0, rope_frac=0.25, rope_theta=1e6, scale=1.0 / math.sqrt(D))
+    bad = torch.full((B, T, Hq, D), float("nan"), dtype=torch.bfloat16, device=dev)
+    native.gemma_attn_decode_multi(q, kn, vn, kc, vc, out=bad,
+                                   seq_lens=torch.tensor([300, T - 1], dtype=torch.int32, device=dev), **kw)
+    assert native.gemma_attn_sync_status() == native.GEMMA_ERR_DEVICE_RANGE
+    good = torch.empty_like(bad)
+    native.gemma_attn_decode_multi(q, kn, vn, kc, vc, out=good,
+                                   seq_lens=torch.tensor([300, 300], dtype=torch.int32, device=dev), **kw)
+    assert native.gemma_attn_sync_status() == 0, native.gemma_last_error()
+    assert torch.isfinite(good.float()).all()
+    assert torch.equal(bad[0].view(torch.int16), good[0].view(torch.int16))
 
 
 def test_multi_stack_31b_block(oracle):
