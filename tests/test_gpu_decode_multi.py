@@ -1,9 +1,12 @@
 """GPU parity of multi-token decode (several new tokens per sequence, as when
 the target model checks a drafter's proposals in speculative decoding)
-against the fp64 oracle, through the C ABI: the tensor-core path of global
-bf16 layers (q heads x tokens packed in one tile, split over the cached
-keys, combined), and the chunked-prefill route of local and int8 layers;
-cache slots written, KV sharing, K = V and the device range check on every route."""
+against the fp64 oracle, through the C ABI. Covered: the tensor-core path of
+bf16 layers (global: q heads x tokens packed in one tile, split over the
+cached keys, combined; unshared local: the ring as it was plus the new rows),
+the per-token decode route of int8 global layers, and the chunked-prefill
+route of the rest (int8 local, shared local, more than 128 rows per KV head);
+cache slots written, KV sharing, K = V, paged caches, bounded-wait timeouts
+and the device range check on every route."""
 import math
 
 import numpy as np
