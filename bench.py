@@ -662,14 +662,16 @@ def bench_decode(args, w, dev, world, peaks, cpu=False):
 
 # --------------------------------------------------------------------------- multi-token decode (ours)
 def verify_kv_bytes(st, l, lens_cpu, T, seqs=None):
-    """K (and V unless K = V) bytes one multi-token decode of layer l reads:
-    a global layer every position of the sequence, a local layer the ring's
-    written slots before the T new tokens plus the T new rows."""
+    """Algorithmic K (and V unless K = V) bytes of one multi-token decode of
+    layer l: the keys at least one of the T new tokens sees, once per KV
+    head. A global layer: every position of the sequence; a local layer:
+    the last window + T - 1 positions (the oldest slot of a full ring is
+    older than every new token's window)."""
     t = st.layer_type(l)
     L = lens_cpu.to(torch.int64)
     if seqs is not None:
         L = L[list(seqs)]
-    keys = (torch.clamp(L - T, max=t.window) + T) if t.window else L
+    keys = torch.clamp(L, max=t.window + T - 1) if t.window else L
     return int(keys.sum()) * t.n_kv_heads * t.head_dim * 2 * (1 if st.keqv(l) else 2)
 
 
