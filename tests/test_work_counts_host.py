@@ -167,3 +167,25 @@ def test_multi_token_kv_bytes_short_sequences():
             assert len(seen) == keys_some_token_sees(L, T, t.window)
             keys += len(seen)
         assert bench.verify_kv_bytes(st, l, lens, T) == keys * t.n_kv_heads * 4 * t.head_dim
+
+
+@pytest.mark.parametrize("name", ["31b_decode_b64", "31b_decode_b16_12l_shared", "global_decode_256k_keqv"])
+def test_decode_step_bytes(name):
+    """A decode step's bytes: each layer's visible K/V rows, its queries read
+    and outputs written (bf16), and, on a layer that owns its cache, the new
+    token's K (and V unless K = V) row written; a shared layer writes none."""
+    w = WORKLOADS[name]
+    st = _Stack(w)
+    lens = lengths_of(w)
+    want = 0
+    for l in range(w.n_layers):
+        t = st.layer_type(l)
+        kv = 1 if st.keqv(l) else 2
+        keys = sum(oracle.visible_range(int(L) - 1, t.window, int(L))[2] for L in lens)
+        want += keys * t.n_kv_heads * 2 * t.head_dim * kv
+        want += w.batch * w.n_q_heads * t.head_dim * 2 * 2
+        if oracle.share_source(w.n_layers, w.ratio, w.n_shared, l) in (l, -1):
+            want += w.batch * t.n_kv_heads * t.head_dim * 2 * kv
+    assert bench.decode_bytes(w, st, lens) == want
+    if name == "31b_decode_b16_12l_shared":
+        assert [st.is_shared(l) for l in range(w.n_layers)] == [False] * 10 + [True, True]
