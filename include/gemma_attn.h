@@ -235,10 +235,11 @@ int gemma_attn_decode(const void* q, const void* k_new, const void* v_new,
 /* workspace: gemma_attn_decode_multi_workspace_size(...) bytes, 256-byte  */
 /*        aligned; scratch.                                                */
 /*                                                                        */
-/* bf16 layers on a contiguous cache run one tensor-core kernel per split */
-/* of the cached keys whose tile holds every q head of a KV head for all  */
-/* the tokens, so the cache is streamed once per step as in single-token  */
-/* decode: global layers with (n_q_heads / n_kv_heads) * tokens <= 128,   */
+/* bf16 layers (global ones contiguous or paged) run one tensor-core      */
+/* kernel per split of the cached keys whose tile holds every q head of a */
+/* KV head for all the tokens, so the cache is streamed once per step as  */
+/* in single-token decode: global layers with (n_q_heads / n_kv_heads) *  */
+/* tokens <= 128,                                                         */
 /* unshared local layers with that product <= 64 and tokens <= window     */
 /* (the ring is read as it was, plus the new rows; it is written after).  */
 /* An int8 global layer takes the tokens one at a time through single-   */
