@@ -200,6 +200,19 @@ def current_records(kernel):
             if r.get("kernel") == kernel and r.get("digest") == digest]
 
 
+def no_traffic_note(kernel, what="no ncu capture of the current kernel sources"):
+    """Why traffic is null: no capture at all, or captures of an earlier
+    version of the kernel (their digest differs from the built sources')."""
+    from hybrid_local_global_b200.profiling import kernel_digest, traffic_records
+    digest = kernel_digest(kernel)
+    old = sorted({r.get("file", "?") for r in traffic_records(os.path.join(ROOT, "profiles"))
+                  if r.get("kernel") == kernel and r.get("digest") != digest})
+    if not old:
+        return what
+    return "%s: %s holds a capture of an earlier version of %s (the sources have changed since), " \
+           "so its DRAM bytes are not reported for this one" % (what, ", ".join(old), kernel)
+
+
 def recorded_traffic(kernel, workload=None):
     """current_records of one workload (or of any, the last per layer type),
     keyed by layer type."""
@@ -309,7 +322,9 @@ def bench_prefill(args, w, dev, world, peaks, e2e=False, cpu=False):
         roof["traffic_note"] = ("DRAM read+write bytes per attention launch, mean over the step's layers, from "
                                 "ncu captures: %s" % "; ".join(sorted({per_kind[k][1] for k in kinds})))
     else:
-        roof["traffic_note"] = "no ncu capture of the current kernel sources for this layer shape"
+        roof["traffic_note"] = "; ".join(sorted({no_traffic_note(
+            "k_prefill_pair" if (w.global_ if g else w.local).head_dim == 512 else "k_prefill_tc",
+            "no ncu capture of the current kernel sources for this layer shape") for g in st.is_global}))
     launches = sum(v["launches"] for v in kern.values())
     res = {"metric": "prefill attention TFLOP/s", "value": round(value, 3), "unit": "TFLOP/s",
            "workload": w.name, "description": w.description,
@@ -639,7 +654,7 @@ def bench_decode(args, w, dev, world, peaks, cpu=False):
                                     "%s %.4f: %s in %s" % (k, ratio[k], rec[k]["workload"], rec[k]["file"])
                                     for k in sorted(rec)))
     else:
-        roof["traffic_note"] = "no ncu capture of the current kernel sources"
+        roof["traffic_note"] = no_traffic_note("k_decode_split_q8" if w.kv_int8 else "k_decode_split")
     res = {"metric": "decode KV GB/s", "value": round(value, 1), "unit": "GB/s",
            "workload": w.name, "description": w.description, "ms_per_step": round(dev_ms / args.steps, 4),
            "bytes_per_step": nbytes, "kv_bytes_per_step": kv_bytes,
@@ -798,7 +813,7 @@ def bench_verify(args, w, dev, world, peaks, cpu=False):
                                 % ", ".join("%s %.4f: %s in %s" % (k, ratio[k], rec[k]["workload"], rec[k]["file"])
                                             for k in sorted(rec)))
     else:
-        roof["traffic_note"] = "no ncu capture of the current kernel sources"
+        roof["traffic_note"] = no_traffic_note("k_verify_tc")
     res = {"metric": "multi-token decode KV GB/s", "value": round(value, 1), "unit": "GB/s",
            "workload": w.name, "description": w.description, "tokens": T,
            "ms_per_step": round(dev_ms / args.steps, 4),

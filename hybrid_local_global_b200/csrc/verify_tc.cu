@@ -66,7 +66,7 @@ struct VCtl {
   uint64_t full[NSTAGE];
   uint64_t empty[NSTAGE];
   uint64_t s_full[2];
-  uint64_t p_ready;
+  uint64_t p_ready[2];  // P^T of tile i in buffer i % 2: phase i/2 of p_ready[i % 2]
   uint64_t o_done[2];  // PV_i completes phase i/2 of o_done[i % 2]
   uint64_t drain;
   uint32_t tmem_base;
@@ -223,7 +223,8 @@ __global__ void __launch_bounds__(192, VCfg<D, NQ, LOCAL>::CTAS)
     }
     mbar_init(&ctl->s_full[0], 1);
     mbar_init(&ctl->s_full[1], 1);
-    mbar_init(&ctl->p_ready, 128);
+    mbar_init(&ctl->p_ready[0], 128);
+    mbar_init(&ctl->p_ready[1], 128);
     mbar_init(&ctl->o_done[0], 1);
     mbar_init(&ctl->o_done[1], 1);
     mbar_init(&ctl->drain, 1);
@@ -346,7 +347,10 @@ __global__ void __launch_bounds__(192, VCfg<D, NQ, LOCAL>::CTAS)
         if (lane == 0) tc::commit(smem_u32(&ctl->s_full[j & 1]));
       }
       if (j >= 1) {
-        if (!wait_all(&ctl->p_ready, (j - 1) & 1, abort_flag, deadline, a.status, 33, j)) {
+        // one barrier per P buffer: the softmax writes P^T of tile j + 1
+        // into this buffer only after PV_{j-1}, issued below, so it arrives
+        // at most one phase ahead of this wait
+        if (!wait_all(&ctl->p_ready[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag, deadline, a.status, 33, j)) {
           ok = false;
           break;
         }
@@ -526,7 +530,7 @@ __global__ void __launch_bounds__(192, VCfg<D, NQ, LOCAL>::CTAS)
       }
       fence_proxy_async_smem();
       tc::fence_before_sync();
-      mbar_arrive(&ctl->p_ready);
+      mbar_arrive(&ctl->p_ready[j & 1]);
     }
     {
       const bool fin = ok && !bad &&
