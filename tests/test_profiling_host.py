@@ -26,3 +26,43 @@ def test_traffic_records_match_current_sources():
         assert r["kernel"] in profiling.KERNEL_SOURCES
         assert int(r["bytes"]) > 0
         assert len(r["digest"]) == 16
+
+
+def test_parity_summary_of_the_cpu_baselines():
+    """bench.py's parity figures: the largest and the mean absolute error over
+    every element compared, rows counted by the reference's last dimension,
+    judged against the tests' tolerance (max 2e-2, mean 2e-3); a non-finite
+    GPU value fails it."""
+    import numpy as np
+    import bench
+    p = bench.Parity()
+    ref = np.zeros((3, 4))
+    p.add(ref + 0.01, ref)
+    p.add(np.full(4, 0.001), np.zeros(4))
+    s = p.summary("x")
+    assert s["rows"] == 4 and abs(s["max_abs"] - 0.01) < 1e-12
+    assert abs(s["mean_abs"] - (12 * 0.01 + 4 * 0.001) / 16) < 1e-9
+    assert s["within_tolerance"] is False  # mean 7.8e-3 > 2e-3
+    q = bench.Parity()
+    q.add(np.full((2, 8), 0.015), np.zeros((2, 8)))
+    q.add(np.zeros((30, 8)), np.zeros((30, 8)))
+    assert q.summary("x")["within_tolerance"] is True
+    r = bench.Parity()
+    r.add(np.array([[np.nan, 0.0]]), np.zeros((1, 2)))
+    assert r.summary("x")["within_tolerance"] is False
+
+
+def test_stale_traffic_record_is_named():
+    """A capture whose digest no longer matches the built sources is not used,
+    and the note says which file holds it."""
+    import bench
+    from hybrid_local_global_b200.profiling import kernel_digest, traffic_records
+    recs = traffic_records(os.path.join(ROOT, "profiles"))
+    for kernel in sorted({r["kernel"] for r in recs}):
+        stale = [r for r in recs if r["kernel"] == kernel and r.get("digest") != kernel_digest(kernel)]
+        note = bench.no_traffic_note(kernel)
+        if stale:
+            assert all(r["file"] in note for r in stale)
+            assert all(r.get("digest") != kernel_digest(kernel) for r in stale)
+        else:
+            assert note == "no ncu capture of the current kernel sources"

@@ -8,18 +8,13 @@ on a global layer: "Gemma 4: End-to-End Architecture Walkthrough", 3a) and
 to closed forms at the benchmarked sizes."""
 from __future__ import annotations
 
-import os
-import sys
-
 import pytest
 import torch
 
+import bench
 import oracle
 from hybrid_local_global_b200 import synth
 from hybrid_local_global_b200.workloads import WORKLOADS, prefill_flops, visible_pairs_prefill
-
-sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
-import bench  # noqa: E402
 
 
 def brute_pairs(seq, prior, window):
