@@ -1,0 +1,322 @@
+"""Race check, on the CPU, of the attention kernels' barrier protocols.
+
+Each tensor-core kernel runs four roles: a TMA producer, an MMA issuer, the
+softmax warps (modelled as one agent per CTA: they pass the same barriers
+together) and, asynchronously, the tensor pipe and the copy engine. This test
+models them step by step as the kernels order them, with mbarriers that
+behave as the hardware's do: a phase completes when its arrivals (and, for a
+copy, its bytes) are in, and a wait on a parity returns as soon as the
+barrier's current phase has the other parity. A wait is correct only if it
+returns exactly when the phase it means has completed; the model flags any
+wait that returns early or misses its phase (parity aliasing), any access to
+shared memory or TMEM that an in-flight copy or MMA could still touch, and
+deadlock. The tensor pipe completes one thread's MMAs in issue order, and a
+commit arrives once every earlier MMA has completed. A random scheduler
+interleaves the roles over many seeds.
+
+Kernels modelled:
+- k_verify_tc (multi-token decode): P^T in two shared-memory buffers, one
+  P-ready barrier per buffer. With a single barrier for both, the checker
+  finds schedules where the softmax arrives for tile j before the issuer
+  has waited for tile j - 1.
+- k_prefill_tc: P written over S in TMEM, one P-ready barrier; the softmax
+  consumes PV_{j-1} before it arrives for tile j.
+- k_prefill_pair: two CTAs; both producers fill their halves of a stage,
+  which complete on the leader's barrier (armed by the leader for both
+  halves' bytes); the leader issues cta_group::2 MMAs that read both CTAs'
+  shared memory and write both TMEMs; commits arrive on both CTAs'
+  barriers; both CTAs' softmax warps arrive on the leader's P-ready barrier.
+"""
+from __future__ import annotations
+
+import random
+
+import pytest
+
+
+class Bar:
+    def __init__(self, name, count):
+        self.name, self.count, self.pending, self.phase = name, count, count, 0
+
+    def arrive(self):
+        self.pending -= 1
+        if self.pending == 0:
+            self.phase += 1
+            self.pending = self.count
+
+
+KERNELS = {
+    # CTAs, P in shared memory (else over S in TMEM), one P-ready barrier per
+    # P buffer, the softmax consumes PV_{j-1} before it arrives for tile j
+    "verify": dict(n_cta=1, smem_p=True, per_buffer=True, pv_before_arrive=False),
+    "verify_single_p_ready": dict(n_cta=1, smem_p=True, per_buffer=False, pv_before_arrive=False),
+    "prefill": dict(n_cta=1, smem_p=False, per_buffer=False, pv_before_arrive=True),
+    "pair": dict(n_cta=2, smem_p=False, per_buffer=False, pv_before_arrive=True),
+}
+
+
+class Model:
+    """One CTA (or CTA pair) of a kernel over n_tiles key tiles, with KS
+    stages of K and VS stages of V per tile through an NSTAGE ring;
+    rescale decisions drawn at random."""
+
+    def __init__(self, kernel, n_tiles, KS, VS, NSTAGE, rng, skip=()):
+        cfg = KERNELS[kernel]
+        self.C = cfg["n_cta"]
+        self.smem_p, self.per_buffer = cfg["smem_p"], cfg["per_buffer"]
+        self.pv_before_arrive = cfg["pv_before_arrive"]
+        self.n, self.KS, self.VS, self.NS, self.rng = n_tiles, KS, VS, NSTAGE, rng
+        self.skip = set(skip)  # waits left out, to show the checker catches their absence
+        C, B = self.C, Bar
+        arms = 1 + C if C > 1 else 1  # pair: the leader's arm and both halves' bytes
+        self.q_full = B("q_full", arms)
+        self.full = [B("full%d" % s, arms) for s in range(NSTAGE)]  # the leader's
+        self.empty = [[B("empty%d/cta%d" % (s, c), 1) for s in range(NSTAGE)] for c in range(C)]
+        self.s_full = [[B("s_full%d/cta%d" % (i, c), 1) for i in range(2)] for c in range(C)]
+        self.o_done = [[B("o_done%d/cta%d" % (i, c), 1) for i in range(2)] for c in range(C)]
+        self.p_ready = [B("p_ready%d" % i, C) for i in range(2 if self.per_buffer else 1)]
+        self.violations = []
+        self.tc_queue = []      # ("mma", tag, reads, writes) or ("commit", [bars], done-tag), issue order
+        self.tma_inflight = []  # (resource written, bar)
+        self.s_read = [set() for _ in range(C)]
+        self.s_done, self.pv_done, self.pv_parts = set(), set(), {}
+        self.p_written = [set() for _ in range(C)]
+
+    # ---------------------------------------------------------------- helpers
+    def check_wait(self, bar, k, role=None):
+        """Hardware answer of a parity wait for phase k, checked against the
+        truth (phase k complete)."""
+        if role in self.skip:
+            return True
+        ret = (bar.phase & 1) != (k & 1)
+        if ret != (bar.phase > k):
+            self.violations.append("%s: wait for phase %d at phase %d returns %s" % (bar.name, k, bar.phase, ret))
+        return ret
+
+    def inflight(self, pred):
+        return any(op[0] == "mma" and pred(op) for op in self.tc_queue)
+
+    def reads(self, res):
+        return self.inflight(lambda op: res in op[2])
+
+    def writes(self, res):
+        return self.inflight(lambda op: res in op[3])
+
+    def hazard(self, what):
+        self.violations.append(what)
+
+    def p_res(self, c, t):
+        return ("P", c, t & 1) if self.smem_p else ("S", c, t & 1)
+
+    # ---------------------------------------------------------------- roles
+    def producer(self, c):
+        leader = c == 0
+        if leader and self.C > 1:
+            self.q_full.arrive()  # arm for both halves
+        self.tma_inflight.append((("Q", c), self.q_full))
+        item = 0
+        for j in range(self.n + 1):
+            for kind in (0, 1):
+                if (kind == 0 and j == self.n) or (kind == 1 and j == 0):
+                    continue
+                for _ in range(self.KS if kind == 0 else self.VS):
+                    s = item % self.NS
+                    if item >= self.NS:
+                        while not self.check_wait(self.empty[c][s], item // self.NS - 1, "empty"):
+                            yield
+                    if self.reads(("stage", c, s)):
+                        self.hazard("copy into stage %d of CTA %d while an MMA reads it" % (s, c))
+                    if leader and self.C > 1:
+                        self.full[s].arrive()  # arm
+                    self.tma_inflight.append((("stage", c, s), self.full[s]))
+                    item += 1
+                    yield
+
+    def issuer(self):
+        C = range(self.C)
+        while not self.check_wait(self.q_full, 0, "q_full"):
+            yield
+        item = 0
+        for j in range(self.n + 1):
+            if j < self.n:
+                for c in C:
+                    if j >= 2 and (j - 2) not in self.s_read[c]:
+                        self.hazard("S_%d issued over S_%d before CTA %d read it" % (j, j - 2, c))
+                for _ in range(self.KS):
+                    s = item % self.NS
+                    while not self.check_wait(self.full[s], item // self.NS, "full"):
+                        yield
+                    self.tc_queue.append(("mma", ("S", j), {("stage", c, s) for c in C} | {("Q", c) for c in C},
+                                          {("S", c, j & 1) for c in C}))
+                    self.tc_queue.append(("commit", [self.empty[c][s] for c in C], None))
+                    item += 1
+                    yield
+                self.tc_queue.append(("commit", [self.s_full[c][j & 1] for c in C], ("S", j)))
+                yield  # nothing orders the issuer's next wait after this commit
+            if j >= 1:
+                t = j - 1
+                bar, k = (self.p_ready[t & 1], t >> 1) if self.per_buffer else (self.p_ready[0], t)
+                while not self.check_wait(bar, k, "p_ready"):
+                    yield
+                for c in C:
+                    if t not in self.p_written[c]:
+                        self.hazard("PV_%d issued before CTA %d wrote P_%d" % (t, c, t))
+                for _ in range(self.VS):
+                    s = item % self.NS
+                    while not self.check_wait(self.full[s], item // self.NS, "full"):
+                        yield
+                    self.tc_queue.append(("mma", ("PV", t),
+                                          {("stage", c, s) for c in C} | {self.p_res(c, t) for c in C},
+                                          {("O", c) for c in C}))
+                    self.tc_queue.append(("commit", [self.empty[c][s] for c in C], None))
+                    item += 1
+                    yield
+                self.tc_queue.append(("commit", [self.o_done[c][t & 1] for c in C], ("PV", t)))
+
+    def softmax(self, c):
+        pv_seen = 0
+
+        def wait_pv(t, role):
+            while not self.check_wait(self.o_done[c][t & 1], t >> 1, role):
+                yield
+
+        for j in range(self.n):
+            while not self.check_wait(self.s_full[c][j & 1], j >> 1, "s_full"):
+                yield
+            if j not in self.s_done or self.writes(("S", c, j & 1)):
+                self.hazard("CTA %d read S_%d with its MMA not complete" % (c, j))
+            self.s_read[c].add(j)
+            yield
+            if j >= 1 and self.rng.random() < 0.4:  # a row or column maximum moved: rescale O
+                if pv_seen < j:
+                    yield from wait_pv(j - 1, "rescale")
+                    pv_seen = j
+                if self.writes(("O", c)) or self.reads(("O", c)):
+                    self.hazard("CTA %d rescaled O with a PV product in flight (tile %d)" % (c, j))
+                yield
+            if self.smem_p and j >= 2 and pv_seen < j - 1:  # the shared-memory P buffer is free
+                yield from wait_pv(j - 2, "p_buffer")
+                pv_seen = j - 1
+            res = self.p_res(c, j)
+            if self.reads(res) or self.writes(res):
+                self.hazard("CTA %d wrote P_%d over a buffer an MMA still uses" % (c, j))
+            self.p_written[c].add(j)
+            if self.pv_before_arrive and j >= 1 and pv_seen < j:
+                yield from wait_pv(j - 1, "pv_before_arrive")
+                pv_seen = j
+            (self.p_ready[j & 1] if self.per_buffer else self.p_ready[0]).arrive()
+            yield
+        yield from wait_pv(self.n - 1, "epilogue")
+        if self.writes(("O", c)):
+            self.hazard("CTA %d read O in the epilogue with a PV product in flight" % c)
+
+    def tensor_pipe_step(self):
+        op = self.tc_queue.pop(0)
+        if op[0] == "mma":
+            if op[1][0] == "PV":
+                self.pv_parts[op[1][1]] = self.pv_parts.get(op[1][1], 0) + 1
+            return
+        done = op[2]
+        if done and done[0] == "S":
+            self.s_done.add(done[1])
+        elif done and self.pv_parts.get(done[1]) == self.VS:
+            self.pv_done.add(done[1])
+        for bar in op[1]:
+            bar.arrive()
+
+    def copy_engine_step(self):
+        _, bar = self.tma_inflight.pop(self.rng.randrange(len(self.tma_inflight)))
+        bar.arrive()
+
+    def run(self, max_steps=200000):
+        agents = {"issuer": self.issuer()}
+        for c in range(self.C):
+            agents["producer%d" % c] = self.producer(c)
+            agents["softmax%d" % c] = self.softmax(c)
+        done = set()
+        for _ in range(max_steps):
+            choices = [a for a in agents if a not in done]
+            if self.tc_queue:
+                choices.append("tc")
+            if self.tma_inflight:
+                choices.append("tma")
+            if not choices:
+                return
+            pick = self.rng.choice(choices)
+            if pick == "tc":
+                self.tensor_pipe_step()
+            elif pick == "tma":
+                self.copy_engine_step()
+            else:
+                try:
+                    next(agents[pick])
+                except StopIteration:
+                    done.add(pick)
+        # the roles only spin on waits, so running out of steps is a deadlock
+        self.violations.append("deadlock: %s still running" % sorted(set(agents) - done))
+
+
+# (n_tiles, K stages per tile, V stages per tile, ring stages) as the kernels
+# are configured -- multi-token: D / 128 of each; prefill head_dim 256: 2 K
+# and 2 V stages of a 5-stage ring; pair head_dim 512: 2 K stages and 1 V
+# stage of a 3-stage ring -- and shorter rings, to stress their reuse
+SHAPES = {
+    "verify": [(1, 1, 1, 2), (2, 2, 2, 3), (3, 2, 2, 5), (6, 4, 4, 5), (8, 1, 1, 3), (7, 4, 4, 4)],
+    "prefill": [(1, 2, 2, 5), (3, 2, 2, 5), (6, 2, 2, 5), (9, 2, 2, 4), (5, 4, 2, 3)],
+    "pair": [(1, 2, 1, 3), (4, 2, 1, 3), (7, 2, 1, 3), (6, 1, 1, 2), (5, 2, 1, 4)],
+}
+
+
+@pytest.mark.parametrize("kernel,shape", [(k, s) for k, ss in SHAPES.items() for s in ss])
+def test_kernel_protocol_has_no_race(kernel, shape):
+    for seed in range(250):
+        m = Model(kernel, *shape, rng=random.Random(seed))
+        m.run()
+        assert not m.violations, "%s %s seed %d: %s" % (kernel, shape, seed, m.violations[:3])
+
+
+def test_single_p_ready_barrier_with_two_smem_buffers_can_alias():
+    """The checker is not vacuous: with one barrier for both shared-memory P
+    buffers (and no wait for PV_{j-1} before arriving) some schedule lets
+    the softmax complete tile j's phase before the issuer waits for tile
+    j - 1, and that wait then misses its phase."""
+    found = []
+    for seed in range(3000):
+        m = Model("verify_single_p_ready", 6, 1, 1, 3, rng=random.Random(seed))
+        m.run()
+        found += [v for v in m.violations if v.startswith("p_ready")]
+        if found:
+            break
+    assert found, "no aliasing schedule found"
+    assert "returns False" in found[0]
+
+
+@pytest.mark.parametrize("kernel,wait", [
+    ("verify", "empty"), ("verify", "full"), ("verify", "s_full"), ("verify", "p_ready"),
+    ("verify", "rescale"), ("verify", "epilogue"),
+    ("prefill", "empty"), ("prefill", "s_full"), ("prefill", "p_ready"), ("prefill", "rescale"),
+    ("prefill", "pv_before_arrive"), ("prefill", "epilogue"),
+    ("pair", "empty"), ("pair", "full"), ("pair", "s_full"), ("pair", "p_ready"), ("pair", "rescale"),
+    ("pair", "pv_before_arrive"), ("pair", "epilogue")])
+def test_each_wait_is_needed(kernel, wait):
+    """Leaving out any one of these waits lets some schedule touch a buffer an
+    in-flight copy or MMA still uses, alias a parity wait or deadlock: the
+    checks have teeth."""
+    shape = {"verify": (6, 2, 2, 3), "prefill": (6, 2, 2, 3), "pair": (6, 2, 1, 3)}[kernel]
+    for seed in range(600):
+        m = Model(kernel, *shape, rng=random.Random(seed), skip={wait})
+        m.run()
+        if m.violations:
+            return
+    pytest.fail("no schedule exposed the missing %s wait in %s" % (wait, kernel))
+
+
+def test_multi_token_p_buffer_wait_is_implied_by_in_order_completion():
+    """The multi-token kernel's explicit wait for PV_{j-2} before it reuses a
+    shared-memory P buffer never matters: one thread's MMAs complete in
+    order, so the S_j commit that starts tile j already follows PV_{j-2};
+    dropping the wait leaves every schedule clean."""
+    for seed in range(300):
+        m = Model("verify", 6, 2, 2, 3, rng=random.Random(seed), skip={"p_buffer"})
+        m.run()
+        assert not m.violations, m.violations[:3]
