@@ -26,6 +26,10 @@ Kernels modelled:
   halves' bytes); the leader issues cta_group::2 MMAs that read both CTAs'
   shared memory and write both TMEMs; commits arrive on both CTAs'
   barriers; both CTAs' softmax warps arrive on the leader's P-ready barrier.
+- k_decode_split / k_decode_split_q8: a copy warp fills a ring of slots that
+  three consumer warps take in turn; the ring size must be a multiple of the
+  consumer count (which the kernels assert), else a parity wait can return
+  for a slot's previous fill.
 """
 from __future__ import annotations
 
@@ -320,3 +324,96 @@ def test_multi_token_p_buffer_wait_is_implied_by_in_order_completion():
         m = Model("verify", 6, 2, 2, 3, rng=random.Random(seed), skip={"p_buffer"})
         m.run()
         assert not m.violations, m.violations[:3]
+
+
+class DecodeRing:
+    """The split-K decode kernels' ring (k_decode_split, k_decode_split_q8):
+    one producer warp copies sub-block t into slot t % NSLOT after the slot's
+    empty barrier says sub-block t - NSLOT was consumed; consumer warp w
+    takes sub-blocks w, w + NCW, ...: it waits on the slot's full barrier,
+    reads the slot and arrives on its empty barrier."""
+
+    def __init__(self, n_sub, NSLOT, NCW, rng):
+        self.n, self.NS, self.NCW, self.rng = n_sub, NSLOT, NCW, rng
+        self.full = [Bar("full%d" % s, 1) for s in range(NSLOT)]
+        self.empty = [Bar("empty%d" % s, 1) for s in range(NSLOT)]
+        self.content = [None] * NSLOT   # sub-block whose rows a slot holds
+        self.reading = [None] * NSLOT   # sub-block a consumer is reading from a slot
+        self.inflight = []              # (slot, sub-block)
+        self.violations = []
+
+    def check_wait(self, bar, k):
+        ret = (bar.phase & 1) != (k & 1)
+        if ret != (bar.phase > k):
+            self.violations.append("%s: wait for phase %d at phase %d returns %s" % (bar.name, k, bar.phase, ret))
+        return ret
+
+    def producer(self):
+        for t in range(self.n):
+            s = t % self.NS
+            if t >= self.NS:
+                while not self.check_wait(self.empty[s], t // self.NS - 1):
+                    yield
+            if self.reading[s] is not None:
+                self.violations.append("copy of %d into slot %d while %d is read" % (t, s, self.reading[s]))
+            self.inflight.append((s, t))
+            yield
+
+    def consumer(self, w):
+        for t in range(w, self.n, self.NCW):
+            s = t % self.NS
+            while not self.check_wait(self.full[s], t // self.NS):
+                yield
+            if self.content[s] != t or any(x == s for x, _ in self.inflight):
+                self.violations.append("sub-block %d read from slot %d holding %s" % (t, s, self.content[s]))
+            self.reading[s] = t
+            yield
+            self.reading[s] = None
+            self.empty[s].arrive()
+            yield
+
+    def run(self, max_steps=100000):
+        agents = {"producer": self.producer()}
+        for w in range(self.NCW):
+            agents["consumer%d" % w] = self.consumer(w)
+        done = set()
+        for _ in range(max_steps):
+            choices = [a for a in agents if a not in done] + (["copy"] if self.inflight else [])
+            if not choices:
+                return
+            pick = self.rng.choice(choices)
+            if pick == "copy":
+                s, t = self.inflight.pop(self.rng.randrange(len(self.inflight)))
+                self.content[s] = t
+                self.full[s].arrive()
+            else:
+                try:
+                    next(agents[pick])
+                except StopIteration:
+                    done.add(pick)
+        self.violations.append("deadlock: %s still running" % sorted(set(agents) - done))
+
+
+@pytest.mark.parametrize("NSLOT,NCW", [(3, 3), (6, 3)])
+def test_decode_ring_as_built_has_no_race(NSLOT, NCW):
+    """The ring sizes the decode kernels use (3 slots at bf16, 6 at int8, with
+    three consumer warps) under random schedules."""
+    for seed in range(300):
+        for n_sub in (1, 2, 5, 13, 40):
+            m = DecodeRing(n_sub, NSLOT, NCW, random.Random(seed))
+            m.run()
+            assert not m.violations, "n_sub %d seed %d: %s" % (n_sub, seed, m.violations[:3])
+
+
+def test_decode_ring_needs_one_consumer_per_slot():
+    """Why the kernels assert NSLOT % NCW == 0: with 4 slots and 3 consumer
+    warps a slot's successive fills go to different warps, and a warp's
+    parity wait can return for the fill before its own."""
+    found = []
+    for seed in range(2000):
+        m = DecodeRing(40, 4, 3, random.Random(seed))
+        m.run()
+        found += m.violations
+        if found:
+            break
+    assert found, "no violating schedule found"
