@@ -363,3 +363,92 @@ def test_binding_rejects_mixed_cache_kinds():
     for k, v in ((i8, bf), (bf, i8)):
         with pytest.raises(TypeError):
             native._kv_kind(k, v)
+
+
+# --------------------------------------------------------------------------- binding vs header
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _header_prototypes():
+    """{name: (return type, [parameter types])} of every function the C
+    header declares, types with names and comments stripped."""
+    import re
+    text = open(os.path.join(ROOT, "include", "gemma_attn.h")).read()
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    text = re.sub(r"#[^\n]*", " ", text)
+    protos = {}
+    for m in re.finditer(r"([A-Za-z_][\w\s\*]*?)\b(gemma_\w+)\s*\(([^;{}]*?)\)\s*;", text):
+        ret, name, params = m.group(1), m.group(2), m.group(3)
+        ret = " ".join(ret.replace("*", " * ").split())
+        types = []
+        for p in params.split(","):
+            p = " ".join(p.replace("*", " * ").split())
+            if not p or p == "void":
+                continue
+            words = p.split(" ")
+            if words[-1] != "*":
+                words = words[:-1]  # drop the parameter name
+            types.append(" ".join(w for w in words if w != "const"))
+        protos[name] = (ret.replace("const ", ""), types)
+    return protos
+
+
+def _ctype_of(c):
+    """ctypes class of a C type from the header; "pointer" for any data
+    pointer (void*, int32_t*, float*, double*, a struct pointer)."""
+    import ctypes
+    table = {"int": ctypes.c_int, "unsigned": ctypes.c_uint, "float": ctypes.c_float,
+             "size_t": ctypes.c_size_t, "long long": ctypes.c_longlong, "char *": ctypes.c_char_p,
+             "gemma_status": ctypes.c_int}
+    if c in table:
+        return table[c]
+    if c.endswith("*"):
+        return "pointer"
+    raise AssertionError("no ctypes mapping for %r" % c)
+
+
+def test_binding_signatures_match_the_header():
+    """Every function native.py binds has the header's arity and argument
+    types (a pointer for every pointer: void*, int32_t*, float*, double*,
+    a struct pointer), and its return type."""
+    import ctypes
+    protos = _header_prototypes()
+    bound = {f.__name__: f for f in vars(native).values() if isinstance(f, ctypes._CFuncPtr)}
+    assert len(bound) >= 20
+    for name, f in sorted(bound.items()):
+        assert name in protos, "%s is bound but not declared in the header" % name
+        ret, params = protos[name]
+        assert len(f.argtypes) == len(params), "%s: %d ctypes args, header has %d" % (
+            name, len(f.argtypes), len(params))
+        for i, (a, c) in enumerate(zip(f.argtypes, params)):
+            want = _ctype_of(c)
+            if want == "pointer":
+                assert a is ctypes.c_void_p or issubclass(a, ctypes._Pointer), "%s arg %d (%s): %r" % (name, i, c, a)
+            else:
+                assert a is want, "%s arg %d (%s): %r" % (name, i, c, a)
+        assert f.restype is _ctype_of(ret), "%s returns %r, header %r" % (name, f.restype, ret)
+
+
+def test_every_declared_function_is_bound_and_exported():
+    protos = _header_prototypes()
+    import ctypes
+    bound = {f.__name__ for f in vars(native).values() if isinstance(f, ctypes._CFuncPtr)}
+    assert set(protos) == bound, (sorted(set(protos) - bound), sorted(bound - set(protos)))
+
+
+def test_kv_desc_struct_matches_the_header():
+    import ctypes
+    import re
+    text = open(os.path.join(ROOT, "include", "gemma_attn.h")).read()
+    body = re.search(r"typedef struct gemma_kv_desc \{(.*?)\} gemma_kv_desc;", text, re.S).group(1)
+    body = re.sub(r"/\*.*?\*/", " ", body, flags=re.S)
+    fields = []
+    for decl in body.split(";"):
+        words = decl.replace("*", " * ").split()
+        if words:
+            fields.append((words[-1], " ".join(words[:-1])))
+    got = native.gemma_kv_desc._fields_
+    assert [n for n, _ in fields] == [n for n, _ in got]
+    for (n, c), (_, t) in zip(fields, got):
+        want = _ctype_of(c)
+        assert (t is ctypes.c_void_p) if want == "pointer" else (t is want), (n, c, t)
