@@ -30,6 +30,10 @@ Kernels modelled:
   three consumer warps take in turn; the ring size must be a multiple of the
   consumer count (which the kernels assert), else a parity wait can return
   for a slot's previous fill.
+- k_verify_tc's failure paths, one agent per warp: bounded waits give up at
+  random points; every warp still reaches the end, the four softmax warps
+  together (their decisions that lead to a named barrier are votes), TMEM is
+  released only after the MMAs drain, and no copy is in flight at exit.
 """
 from __future__ import annotations
 
@@ -417,3 +421,285 @@ def test_decode_ring_needs_one_consumer_per_slot():
         if found:
             break
     assert found, "no violating schedule found"
+
+
+# --------------------------------------------------------------------------- abort paths
+class NamedBar:
+    """A CTA barrier (bar.red.or / bar.sync on one id, or __syncthreads): a
+    generation completes when all `count` warps have arrived; a bar.red.or
+    returns the OR of their predicates. Every warp must make the same kind of
+    call in the same generation."""
+
+    def __init__(self, name, count, violations):
+        self.name, self.count, self.violations = name, count, violations
+        self.gen, self.arrived, self.result = 0, [], {}
+
+    def arrive(self, warp, kind, pred=False):
+        self.arrived.append((warp, kind, bool(pred)))
+        if len(self.arrived) == self.count:
+            kinds = {k for _, k, _ in self.arrived}
+            if len(kinds) > 1:
+                self.violations.append("%s: warps met at different calls %s" % (self.name, sorted(kinds)))
+            self.result[self.gen] = any(p for _, _, p in self.arrived)
+            self.gen += 1
+            self.arrived = []
+
+
+class VerifyAbortModel:
+    """k_verify_tc's roles with their failure paths, one agent per warp:
+    warp 0 the producer, warp 1 the MMA issuer, warps 2..5 the softmax. Any
+    bounded wait may give up (its deadline passes): it raises the CTA's abort
+    flag and returns false; later bounded waits see the flag and return false
+    too. The softmax warps take every decision that leads to a named barrier
+    by a vote, so they stay together; at the end all six warps meet at
+    __syncthreads, then the producer waits (bounded, flag ignored) for its
+    copies still in flight, and TMEM is released."""
+
+    def __init__(self, n_tiles, MT, NSTAGE, rng, p_fail, mutate=None):
+        self.n, self.MT, self.NS, self.rng, self.p_fail = n_tiles, MT, NSTAGE, rng, p_fail
+        self.mutate = mutate  # a planted protocol mistake, to show the checks catch it
+        self.violations = []
+        B = Bar
+        self.q_full = B("q_full", 1)
+        self.full = [B("full%d" % s, 1) for s in range(NSTAGE)]
+        self.empty = [B("empty%d" % s, 1) for s in range(NSTAGE)]
+        self.s_full = [B("s_full%d" % i, 1) for i in range(2)]
+        self.o_done = [B("o_done%d" % i, 1) for i in range(2)]
+        self.p_ready = [B("p_ready%d" % i, 4) for i in range(2)]  # 128 threads: 4 warp arrivals
+        self.drain = B("drain", 1)
+        self.bar1 = NamedBar("bar1", 4, self.violations)        # the softmax warps' barrier
+        self.block = NamedBar("syncthreads", 6, self.violations)
+        self.abort = False
+        self.tc_queue, self.tma_inflight = [], []
+        self.issued, self.consumed = [0] * NSTAGE, [0] * NSTAGE
+        self.q_issued = self.q_consumed = False
+        self.expire = set()         # agents whose blocked bounded wait the scheduler times out
+        self.blocked = {}           # agent -> (kind "bounded" | "barrier", can it move now?)
+        self.softmax_ok = {}
+
+    # -------------------------------------------------------------- primitives
+    def bwait(self, agent, bar, k, honour_abort=True):
+        """mbar_wait_bounded_at: True when phase k completed; False once the
+        deadline passes (abort raised) or, when honour_abort, the flag is up."""
+        if honour_abort and self.p_fail and self.rng.random() < self.p_fail:
+            # this wait's deadline passes early (as for a copy that never lands);
+            # the teardown waits are for copies that were issued and do land
+            self.abort = True
+            return False
+        while True:
+            if agent in self.expire:
+                self.expire.discard(agent)
+                self.abort = True
+                self.blocked.pop(agent, None)
+                return False
+            if honour_abort and self.abort:
+                self.blocked.pop(agent, None)
+                return False
+            if (bar.phase & 1) != (k & 1):
+                if bar.phase <= k:
+                    self.violations.append("%s: wait for phase %d at phase %d returns early" % (bar.name, k, bar.phase))
+                self.blocked.pop(agent, None)
+                return True
+            self.blocked[agent] = ("bounded", lambda: (bar.phase & 1) != (k & 1) or (honour_abort and self.abort))
+            yield
+
+    def meet(self, agent, nb, kind, pred=False):
+        gen = nb.gen
+        nb.arrive(agent, kind, pred)
+        while nb.gen == gen:
+            self.blocked[agent] = ("barrier", lambda: nb.gen != gen)
+            yield
+        self.blocked.pop(agent, None)
+        return nb.result[gen]
+
+    # -------------------------------------------------------------- roles
+    def producer(self):
+        a = "w0"
+        self.tma_inflight.append(("Q", self.q_full))
+        self.q_issued = True
+        item, ok = 0, True
+        for j in range(self.n + 1):
+            for kind in (0, 1):
+                if not ok or (kind == 0 and j == self.n) or (kind == 1 and j == 0):
+                    continue
+                for _ in range(self.MT):
+                    s = item % self.NS
+                    if item >= self.NS:
+                        ok = yield from self.bwait(a, self.empty[s], item // self.NS - 1)
+                        if not ok:
+                            break
+                    self.issued[s] += 1
+                    self.tma_inflight.append((s, self.full[s]))
+                    item += 1
+                    yield
+        yield from self.meet(a, self.block, "syncthreads")
+        if self.abort and self.mutate != "no_teardown_wait":  # copies in flight must land first
+            if self.q_issued and not self.q_consumed:
+                yield from self.bwait(a, self.q_full, 0, honour_abort=False)
+            for s in range(self.NS):
+                if self.issued[s] > self.consumed[s]:
+                    yield from self.bwait(a, self.full[s], self.issued[s] - 1, honour_abort=False)
+        if self.tma_inflight:
+            self.violations.append("CTA exits with copies in flight: %s" % [x[0] for x in self.tma_inflight])
+
+    def issuer(self):
+        a = "w1"
+        ok = yield from self.bwait(a, self.q_full, 0)
+        if ok:
+            self.q_consumed = True
+        item = 0
+        for j in range(self.n + 1):
+            if not ok:
+                break
+            if j < self.n:
+                for _ in range(self.MT):
+                    s = item % self.NS
+                    ok = yield from self.bwait(a, self.full[s], item // self.NS)
+                    if not ok:
+                        break
+                    self.consumed[s] += 1
+                    self.tc_queue.append(("mma", [self.empty[s]]))
+                    item += 1
+                    yield
+                if not ok:
+                    break
+                self.tc_queue.append(("commit", [self.s_full[j & 1]]))
+                yield
+            if j >= 1:
+                t = j - 1
+                ok = yield from self.bwait(a, self.p_ready[t & 1], t >> 1)
+                if not ok:
+                    break
+                for _ in range(self.MT):
+                    s = item % self.NS
+                    ok = yield from self.bwait(a, self.full[s], item // self.NS)
+                    if not ok:
+                        break
+                    self.consumed[s] += 1
+                    self.tc_queue.append(("mma", [self.empty[s]]))
+                    item += 1
+                    yield
+                if not ok:
+                    break
+                self.tc_queue.append(("commit", [self.o_done[t & 1]]))
+        # no MMA may be in flight when TMEM is released
+        if self.mutate != "no_drain":
+            self.tc_queue.append(("commit", [self.drain]))
+            yield from self.bwait(a, self.drain, 0, honour_abort=False)
+        yield from self.meet(a, self.block, "syncthreads")
+        if any(op[0] == "mma" for op in self.tc_queue):
+            self.violations.append("TMEM released with an MMA in flight")
+
+    def softmax(self, w):
+        a = "w%d" % (w + 2)
+        ok, bad, pv_seen = True, False, 0
+        for j in range(self.n):
+            if not bad:
+                got = yield from self.bwait(a, self.s_full[j & 1], j >> 1)
+                bad = not got
+            if self.mutate == "break_alone" and bad:
+                ok = False
+                break
+            if (yield from self.meet(a, self.bar1, "red.or", bad)):
+                ok = False
+                break
+            if (yield from self.meet(a, self.bar1, "red.or", self.rng.random() < 0.3)):  # some logit grew
+                yield from self.meet(a, self.bar1, "sync")
+                moved = yield from self.meet(a, self.bar1, "red.or", self.rng.random() < 0.5)
+                if moved and j >= 1 and pv_seen < j:
+                    got = yield from self.bwait(a, self.o_done[(j - 1) & 1], (j - 1) >> 1)
+                    if got:
+                        pv_seen = j
+                    else:
+                        bad = True
+            if not bad and j >= 2 and pv_seen < j - 1:
+                got = yield from self.bwait(a, self.o_done[j & 1], (j - 2) >> 1)
+                if got:
+                    pv_seen = j - 1
+                else:
+                    bad = True
+            if bad:
+                continue  # no arrival: the issuer's bounded wait sees the abort
+            self.p_ready[j & 1].arrive()
+            yield
+        fin = ok and not bad
+        if fin:
+            t = self.n - 1
+            fin = yield from self.bwait(a, self.o_done[t & 1], t >> 1)
+        ok = not (yield from self.meet(a, self.bar1, "red.or", not fin))
+        if ok:
+            yield from self.meet(a, self.bar1, "sync")
+            yield from self.meet(a, self.bar1, "sync")
+        self.softmax_ok[w] = ok
+        yield from self.meet(a, self.block, "syncthreads")
+
+    # -------------------------------------------------------------- scheduler
+    def run(self, max_steps=200000):
+        agents = {"w0": self.producer(), "w1": self.issuer()}
+        for w in range(4):
+            agents["w%d" % (w + 2)] = self.softmax(w)
+        done = set()
+        for _ in range(max_steps):
+            live = [x for x in agents if x not in done]
+            engines = (["tc"] if self.tc_queue else []) + (["tma"] if self.tma_inflight else [])
+            if not live and not engines:
+                break
+            runnable = [x for x in live if x not in self.blocked or self.blocked[x][1]()]
+            progress = runnable + engines
+            if not progress:
+                stuck = [x for x in live if self.blocked[x][0] == "bounded"]
+                if not stuck:
+                    self.violations.append("deadlock at named barriers: %s" % sorted(live))
+                    return
+                self.expire.add(self.rng.choice(stuck))  # its deadline passes
+                progress = stuck
+            elif self.rng.random() < 0.2:
+                progress = progress + [x for x in live if x not in runnable]  # polls that find nothing
+            pick = self.rng.choice(progress)
+            if pick == "tc":
+                op = self.tc_queue.pop(0)
+                for bar in op[1]:
+                    bar.arrive()
+            elif pick == "tma":
+                _, bar = self.tma_inflight.pop(self.rng.randrange(len(self.tma_inflight)))
+                bar.arrive()
+            else:
+                try:
+                    next(agents[pick])
+                except StopIteration:
+                    done.add(pick)
+        else:
+            self.violations.append("did not finish: %s" % sorted(set(agents) - done))
+            return
+        if len(set(self.softmax_ok.values())) > 1:
+            self.violations.append("softmax warps disagree on success: %s" % self.softmax_ok)
+        if not self.abort and not all(self.softmax_ok.values()):
+            self.violations.append("a run without timeouts failed")
+
+
+@pytest.mark.parametrize("p_fail", [0.0, 0.002, 0.02, 0.2])
+def test_multi_token_abort_paths_terminate_together(p_fail):
+    """With bounded waits giving up at random points (and, when nothing can
+    move, the deadline of a blocked wait passing), every warp of a
+    multi-token CTA reaches the end: the softmax warps agree on the outcome,
+    no named barrier is left half-met, TMEM is released only after the MMAs
+    drain, and no copy is still in flight when the CTA exits. Without
+    timeouts every run succeeds."""
+    for seed in range(200):
+        for shape in ((1, 1, 2), (4, 2, 3), (7, 4, 5)):
+            m = VerifyAbortModel(*shape, rng=random.Random(seed), p_fail=p_fail)
+            m.run()
+            assert not m.violations, "p_fail %g seed %d shape %s: %s" % (p_fail, seed, shape, m.violations[:3])
+
+
+@pytest.mark.parametrize("mutate", ["break_alone", "no_teardown_wait", "no_drain"])
+def test_multi_token_abort_checks_have_teeth(mutate):
+    """A softmax warp that leaves on its own failure instead of voting, a
+    producer that does not wait for its copies in flight, an issuer that
+    does not drain its MMAs: each is caught under random failures."""
+    for seed in range(400):
+        m = VerifyAbortModel(6, 2, 3, rng=random.Random(seed), p_fail=0.05, mutate=mutate)
+        m.run()
+        if m.violations:
+            return
+    pytest.fail("planted mistake %s not caught" % mutate)
