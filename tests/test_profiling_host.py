@@ -66,3 +66,56 @@ def test_stale_traffic_record_is_named():
             assert all(r.get("digest") != kernel_digest(kernel) for r in stale)
         else:
             assert note == "no ncu capture of the current kernel sources"
+
+
+def test_clock_rejection_rule():
+    """Hardware and thermal slowdowns disqualify a timed region, and so does
+    a clock well below its maximum with no reason; the power cap alone does
+    not."""
+    import bench
+    ok = {"sm_mhz": 1965, "sm_max_mhz": 1965, "reasons": []}
+    assert not bench.clock_rejected(ok)
+    assert not bench.clock_rejected({"sm_mhz": 1635, "sm_max_mhz": 1965, "reasons": ["sw_power_cap"]})
+    assert not bench.clock_rejected({"sm_mhz": 1200, "sm_max_mhz": 1965, "reasons": ["sw_power_cap"]})
+    for r in ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown"):
+        assert bench.clock_rejected({"sm_mhz": 1965, "sm_max_mhz": 1965, "reasons": [r, "sw_power_cap"]})
+    assert bench.clock_rejected({"sm_mhz": 1100, "sm_max_mhz": 1965, "reasons": []})
+    assert bench.clock_rejected({"sm_mhz": 1100, "sm_max_mhz": 1965, "reasons": ["applications_clocks"]})
+    assert not bench.clock_rejected({"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "note": "no samples"})
+
+
+def test_rejected_clock_record_is_measured_again_once(monkeypatch):
+    """timed_passes repeats the measurement once when any rank's clock record
+    is disqualified, keeps the second, and records the first; the repeat is
+    decided from the value reduced over the ranks."""
+    import bench
+
+    class Clk:
+        def __init__(self, summ):
+            self.summ = summ
+
+        def summary(self):
+            out = dict(self.summ)
+            if getattr(self, "rejected_first", None) is not None:
+                out["rejected_first_attempt"] = self.rejected_first
+            return out
+
+    bad = {"sm_mhz": 1965, "sm_max_mhz": 1965, "reasons": ["hw_slowdown"]}
+    good = {"sm_mhz": 1965, "sm_max_mhz": 1965, "reasons": []}
+    for records, other_rank_bad, want_calls in (([good], 0.0, 1), ([bad, good], 0.0, 2),
+                                                ([good, good], 1.0, 2), ([bad, bad], 0.0, 2)):
+        calls = []
+
+        def once(*a, **k):
+            calls.append(1)
+            return (10.0 * len(calls), 1.0, {}, Clk(records[len(calls) - 1]))
+
+        monkeypatch.setattr(bench, "timed_passes_once", once)
+        monkeypatch.setattr(bench, "max_over_ranks", lambda x, world: max(x, other_rank_bad))
+        ms, _, _, clk = bench.timed_passes(None, None, None, 2, None)
+        assert len(calls) == want_calls
+        assert ms == 10.0 * want_calls
+        if want_calls == 2:
+            assert "rejected_first_attempt" in clk.summary()
+        else:
+            assert "rejected_first_attempt" not in clk.summary()
