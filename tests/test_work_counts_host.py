@@ -184,3 +184,25 @@ def test_decode_step_bytes(name):
     assert bench.decode_bytes(w, st, lens) == want
     if name == "31b_decode_b16_12l_shared":
         assert [st.is_shared(l) for l in range(w.n_layers)] == [False] * 10 + [True, True]
+
+
+def test_prefill_attention_bytes_match_the_capture_records():
+    """The algorithmic bytes a prefill traffic record is scaled by: queries
+    read and outputs written once, the chunk's K and V read once (plus the
+    visible cached prefix on a chunk after cached tokens), bf16. They equal
+    the units each committed capture record states for its workload."""
+    import os
+    from hybrid_local_global_b200.profiling import traffic_records
+    from hybrid_local_global_b200.workloads import prefill_attn_bytes
+    recs = [r for r in traffic_records(os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
+                                                    "profiles"))
+            if r["kernel"] in ("k_prefill_tc", "k_prefill_pair") and "units" in r]
+    assert recs
+    for r in recs:
+        w = WORKLOADS[r["workload"]]
+        t = w.global_ if r["layer"] == "global" else w.local
+        assert prefill_attn_bytes(w, t) == int(r["units"]), r
+    w = WORKLOADS["31b_local_s8192"]
+    q = 8192 * 32 * 256 * 2
+    kv = 8192 * 16 * 256 * 2
+    assert prefill_attn_bytes(w, w.local) == 2 * q + 2 * kv == 402_653_184
