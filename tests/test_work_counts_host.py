@@ -206,3 +206,27 @@ def test_prefill_attention_bytes_match_the_capture_records():
     q = 8192 * 32 * 256 * 2
     kv = 8192 * 16 * 256 * 2
     assert prefill_attn_bytes(w, w.local) == 2 * q + 2 * kv == 402_653_184
+
+
+def test_decode_bytes_match_the_capture_records():
+    """Each committed decode and multi-token capture record's algorithmic
+    units equal what bench.py's counters give for its workload and layer."""
+    import os
+    from hybrid_local_global_b200.profiling import traffic_records
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    seen = 0
+    for r in traffic_records(os.path.join(root, "profiles")):
+        if r["kernel"] not in ("k_decode_split", "k_decode_split_q8", "k_verify_tc") or "units" not in r:
+            continue
+        w = WORKLOADS[r["workload"]]
+        st = _Stack(w)
+        lens = lengths_of(w)
+        layers = [l for l in range(w.n_layers) if (st.layer_type(l).window == 0) == (r["layer"] == "global")]
+        l = layers[0]
+        if r["kernel"] == "k_verify_tc":
+            got = bench.verify_kv_bytes(st, l, lens, w.tokens)
+        else:
+            got = bench.visible_kv_bytes(st, l, lens)
+        assert got == int(r["units"]), (r, got)
+        seen += 1
+    assert seen >= 5
